@@ -1,0 +1,447 @@
+"""Pins for the fp64 oracle: each check ties it to something other than itself
+(hand-worked exact values, closed forms, exact rational arithmetic, brute force,
+a correctly rounded exp), chosen so that a dropped term, a wrong sign or index or
+a transposed operand in the oracle fails at least one of them. CPU only.
+"""
+import itertools
+import json
+import math
+import os
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import dpa_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------- helpers (exact arithmetic)
+
+def rne_to_format(v: Fraction, mant_bits: int, emin: int) -> Fraction:
+    """Round a rational to the nearest value of a binary format with `mant_bits` stored
+    significand bits and minimum normal exponent `emin` (ties to even), no overflow."""
+    if v == 0:
+        return Fraction(0)
+    sign = -1 if v < 0 else 1
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, emin)
+    ulp = Fraction(2) ** (e - mant_bits)
+    n = a / ulp
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * ulp
+
+
+def f64_ulp(x: float) -> float:
+    return math.ulp(x)
+
+
+# ----------------------------------------------------------------- fp16 rounding
+
+def test_fp16_round_matches_exact_rounding_on_ties_and_near_ties():
+    vals = [1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 1.0 + 2.0 ** -11 + 2.0 ** -40,
+            1.0 + 2.0 ** -11 - 2.0 ** -40, 2.0 ** -24 * 1.5, 2.0 ** -24 * 2.5,
+            0.1, 1.0 / 3.0, 1.875 / 15.0, 0.11666666666666667, 6.1e-5, 65504.0, -0.3 / 15]
+    got = O.fp16_round(np.array(vals))
+    for v, g in zip(vals, got):
+        want = rne_to_format(Fraction(v), 10, -14)
+        assert Fraction(float(g)) == want, (v, g, float(want))
+
+
+# ----------------------------------------------------------------- uniform quantiser + F&C
+
+def test_hand_worked_group_exact():
+    fx = json.load(open(os.path.join(GOLDEN, "fc_worked_group.json")))
+    B, G = fx["B"], fx["G"]
+    w = np.array(fx["w"], dtype=np.float32)[None, :]
+    q, s, z = O.quantize_uniform(w, B, G)
+    assert float(s[0, 0]) == fx["s"] and float(z[0, 0]) == fx["z"]
+    assert q[0].tolist() == fx["q"]
+    for k in range(1, B + 1):
+        wh = O.dequant_uniform(q, s, z, B, k, G)[0]
+        assert wh.tolist() == fx["w_hat"][str(k)], k
+
+
+def test_quantizer_clamps_and_scale_from_exact_rounding():
+    # all-positive group: z would be negative and clamps to 0; the top code clamps to 15
+    w = np.array([[0.25, 0.5, 0.75, 1.0, 1.25, 1.5, 1.75, 2.0]], dtype=np.float32)
+    q, s, z = O.quantize_uniform(w, 4, 8)
+    s_exact = rne_to_format((Fraction(2.0) - Fraction(0.25)) / 15, 10, -14)
+    assert Fraction(float(s[0, 0])) == s_exact
+    assert z[0, 0] == 0.0
+    sf = float(s_exact)
+    want = [min(15, max(0, int(round(float(v) / sf)))) for v in w[0]]
+    assert q[0].tolist() == want and q[0, -1] == 15
+
+
+def test_quantizer_error_bound_random():
+    rng = np.random.default_rng(7)
+    w = (rng.standard_normal((16, 256)) * 0.02).astype(np.float32)
+    B, G = 4, 64
+    q, s, z = O.quantize_uniform(w, B, G)
+    assert q.min() >= 0 and q.max() <= 15
+    wh = O.dequant_uniform(q, s, z, B, B, G)
+    err = np.abs(w.astype(np.float64) - wh)
+    # inside [lo, hi] the rounding error is at most s/2 plus the clamp of one rounding
+    # of z (z rounding moves the grid by at most s/2)
+    assert np.all(err <= np.repeat(s, G, axis=1) * 1.0 + 1e-12)
+
+
+def _fc_pin_holds(fc, B):
+    codes = np.arange(2 ** B)
+    for k in range(1, B + 1):
+        qh = fc(codes, B, k)
+        d = B - k
+        if k == B and not np.array_equal(qh, codes.astype(np.float64)):
+            return False
+        if Fraction(sum(Fraction(float(c)) - Fraction(float(h)) for c, h in zip(codes, qh))) != 0:
+            return False
+        if np.max(np.abs(codes - qh)) != (2 ** d - 1) / 2:
+            return False
+        # 2*q_hat = top k bits, then a 0, then (B-k) ones
+        twice = (2 * qh).astype(np.int64)
+        want = ((codes >> d) << (d + 1)) | ((1 << d) - 1)
+        if not np.array_equal(twice, want):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("B", [2, 3, 4, 5])
+def test_floor_and_compensation_closed_forms(B):
+    assert _fc_pin_holds(O.fc_code, B)
+
+
+def test_planted_floor_without_compensation_fails_the_pin():
+    def plain_floor(q, B, k):       # the ablation the MatMoE review reports at 0% accuracy
+        d = B - k
+        return (np.asarray(q) >> d).astype(np.float64) * 2 ** d
+    assert not _fc_pin_holds(plain_floor, 4)
+    codes = np.arange(16)
+    for k in range(1, 4):
+        assert np.mean(codes - plain_floor(codes, 4, k)) == (2 ** (4 - k) - 1) / 2
+
+
+def test_bitplane_round_trip_and_prefix():
+    rng = np.random.default_rng(1)
+    q = rng.integers(0, 16, size=(5, 64))
+    pl = O.bitplanes(q, 4)
+    assert pl.shape == (4, 5, 64)
+    assert np.array_equal(pl[0], q >> 3) and np.array_equal(pl[3], q & 1)
+    for k in range(1, 5):
+        assert np.array_equal(O.codes_from_planes(pl, k, 4), (q >> (4 - k)) << (4 - k))
+        # F&C from the prefix alone equals F&C from the full code
+        fc_prefix = O.codes_from_planes(pl, k, 4).astype(np.float64) + (2 ** (4 - k) - 1) / 2
+        assert np.array_equal(fc_prefix, O.fc_code(q, 4, k))
+
+
+# ----------------------------------------------------------------- residual table
+
+def test_residual_table_exact_small():
+    rng = np.random.default_rng(3)
+    H, I, G, B = 16, 8, 8, 4
+    g = (rng.standard_normal((I, H)) * 0.02).astype(np.float32)
+    u = (rng.standard_normal((I, H)) * 0.02).astype(np.float32)
+    d = (rng.standard_normal((H, I)) * 0.02).astype(np.float32)
+    enc = O.encode_expert(g, u, d, 0, B, G)
+    for k in range(1, B + 1):
+        exact = Fraction(0)
+        for m, q, s, z in zip((g, u, d), enc["q"], enc["s"], enc["z"]):
+            R, C = m.shape
+            for i in range(R):
+                for j in range(C):
+                    qq = int(q[i, j])
+                    dd = B - k
+                    qh = Fraction((qq >> dd) << dd) + Fraction(2 ** dd - 1, 2)
+                    wh = Fraction(float(s[i, j // G])) * (qh - Fraction(float(z[i, j // G])))
+                    diff = Fraction(float(m[i, j])) - wh
+                    exact += diff * diff
+        assert abs(Fraction(enc["r"][k - 1]) - exact) <= exact * Fraction(1, 10 ** 12), k
+
+
+def test_residual_table_four_per_plane_uniform():
+    rng = np.random.default_rng(5)
+    H, I, G, B = 256, 128, 64, 4
+    mats = [(rng.standard_normal(sh) * 0.02).astype(np.float32) for sh in ((I, H), (I, H), (H, I))]
+    r = O.encode_expert(*mats, 0, B, G)["r"]
+    assert np.all(np.diff(r) < 0)
+    # dropping one more uniform bit multiplies the mean squared error by ~4 (closed form
+    # (4^d/4 - 1/4 + 1/12)/(4^(d-1)/4 - 1/4 + 1/12) -> 4); clamping makes it approximate
+    for k in range(1, B):
+        assert 3.3 < r[k - 1] / r[k] < 4.7, (k, r)
+
+
+def test_bcq_closed_forms():
+    G = 8
+    c = 0.0234375   # exactly representable in fp16
+    pattern = np.array([1, -1, -1, 1, 1, 1, -1, 1], dtype=np.float64)
+    w = (c * pattern).astype(np.float32)[None, :]
+    signs, alpha = O.encode_bcq_matrix(w, 3, G)
+    assert alpha[0, 0, 0] == c and alpha[1, 0, 0] == 0.0 and alpha[2, 0, 0] == 0.0
+    assert np.array_equal(signs[0, 0], pattern > 0)
+    assert np.all(signs[1, 0])        # residual is exactly 0 -> sign(0) = +1
+    # random: alpha_0 = fp16(mean |w|) computed exactly; residual non-increasing in k
+    rng = np.random.default_rng(9)
+    w = (rng.standard_normal((4, 32)) * 0.02).astype(np.float32)
+    signs, alpha = O.encode_bcq_matrix(w, 3, 16)
+    for r_ in range(4):
+        for gi in range(2):
+            seg = w[r_, gi * 16:(gi + 1) * 16]
+            m = sum(Fraction(abs(float(v))) for v in seg) / 16
+            assert Fraction(alpha[0, r_, gi]) == rne_to_format(m, 10, -14)
+            # least squares optimum for the chosen signs is the unrounded mean |R|
+    prev = np.inf
+    for k in range(1, 4):
+        e = np.sum((w.astype(np.float64) - O.dequant_bcq(signs, alpha, k, 16)) ** 2)
+        assert e <= prev
+        prev = e
+
+
+# ----------------------------------------------------------------- exp
+
+def _cr_exp(x: float) -> float:
+    getcontext().prec = 60
+    v = Decimal(x).exp()
+    return float(Fraction(v))   # float(Fraction) rounds correctly
+
+
+def test_dexp_within_one_ulp_of_correctly_rounded():
+    rng = np.random.default_rng(11)
+    xs = list(-rng.random(1500) * 50.0) + list(-rng.random(300) * 700.0) + \
+        [0.0, -1e-300, -2.0 ** -60, -0.5 * math.log(2), -math.log(2), -1.0, -707.9, -708.0, -30.0]
+    for x in xs:
+        got = O.dexp(x)
+        want = _cr_exp(x)
+        assert abs(got - want) <= f64_ulp(want), (x, got, want)
+    assert O.dexp(0.0) == 1.0
+    assert O.dexp(-709.0) == 0.0
+    s = sorted(xs)
+    vals = [O.dexp(x) for x in s]
+    assert all(a <= b for a, b in zip(vals, vals[1:]))
+
+
+def test_exp_constants_from_ln2():
+    getcontext().prec = 60
+    ln2 = Fraction(Decimal(2).ln())
+    assert Fraction(O.LN2_HI) <= ln2 < Fraction(O.LN2_HI) + Fraction(1, 2 ** 42)
+    assert (Fraction(O.LN2_HI) * 2 ** 42).denominator == 1
+    assert abs(Fraction(O.LN2_HI) + Fraction(O.LN2_LO) - ln2) < Fraction(1, 2 ** 100)
+    assert O.INV_LN2 == float(1 / ln2)
+    assert all(Fraction(c) == rne_to_format(Fraction(1, math.factorial(i)), 52, -1022)
+               for i, c in enumerate(O.EXP_TAYLOR))
+
+
+# ----------------------------------------------------------------- router
+
+def _bf16_bits(vals):
+    from dynamic_any_precision_b200.workloads import f32_to_bf16_bits
+    return f32_to_bf16_bits(np.asarray(vals, dtype=np.float32))
+
+
+def test_router_logit_is_exact_dot_rounded_once():
+    rng = np.random.default_rng(13)
+    T, E, H = 3, 5, 64
+    # wide exponent range (incl. values near bf16's subnormal end) so that a naive
+    # left-to-right fp64 sum would round differently
+    x = rng.standard_normal((T, H)) * np.exp2(rng.integers(-60, 30, size=(T, H)))
+    w = rng.standard_normal((E, H)) * np.exp2(rng.integers(-60, 30, size=(E, H)))
+    xb, wb = _bf16_bits(x), _bf16_bits(w)
+    logits = O.router_logits(xb, wb)
+    xf, wf = O.bf16_bits_to_f64(xb), O.bf16_bits_to_f64(wb)
+    for t in range(T):
+        for e in range(E):
+            exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[t], wf[e]))
+            assert Fraction(logits[t, e]) == rne_to_format(exact, 52, -1022)
+
+
+def test_topk_brute_force_ties_and_permutation():
+    row = np.array([0.5, 1.0, 1.0, -2.0, 0.75, 1.0])
+    assert O.topk_select(row, 3) == [1, 2, 5]
+    assert O.topk_select(row, 4) == [1, 2, 5, 4]
+    rng = np.random.default_rng(17)
+    T, E, H, K = 4, 16, 32, 4
+    xb = _bf16_bits(rng.standard_normal((T, H)))
+    wb = _bf16_bits(rng.standard_normal((E, H)) * 0.02)
+    idx, g, lg = O.route(xb, wb, K, 1)
+    for t in range(T):
+        brute = sorted(range(E), key=lambda e: -lg[t, e])[:K]
+        assert idx[t].tolist() == brute
+    perm = rng.permutation(E)
+    idx2, g2, _ = O.route(xb, wb[perm], K, 1)
+    assert np.array_equal(perm[idx2], idx) and np.array_equal(g2, g)
+
+
+def test_gate_identities():
+    rng = np.random.default_rng(19)
+    T, E, H, K = 3, 12, 32, 4
+    xb = _bf16_bits(rng.standard_normal((T, H)))
+    wb = _bf16_bits(rng.standard_normal((E, H)) * 0.3)
+    for norm in (0, 1):
+        idx, g, lg = O.route(xb, wb, K, norm)
+        for t in range(T):
+            sel = idx[t]
+            full = np.exp(lg[t] - lg[t].max())
+            den = full[sel].sum() if norm else full.sum()
+            np.testing.assert_allclose(g[t], full[sel] / den, rtol=1e-13)
+            if norm:
+                assert abs(g[t].sum() - 1.0) < 1e-15 * K
+            assert np.all(np.diff(g[t]) <= 0)
+
+
+# ----------------------------------------------------------------- allocation
+
+def _tiny_alloc_case(seed, T=4, K=2, E=8, B=4):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    g = rng.dirichlet(np.ones(K), size=T)
+    g = -np.sort(-g, axis=1)
+    base = rng.random(E) * 10 + 1
+    r = np.stack([base * 4.0 ** (B - k) * (1 + 0.3 * rng.random(E)) for k in range(1, B + 1)], axis=1)
+    return idx, g, r
+
+
+@pytest.mark.parametrize("seed,target", [(0, 3.0), (1, 2.5), (2, 2.125), (3, 3.75), (4, 3.0)])
+def test_allocation_matches_brute_force_optimum(seed, target):
+    kmin, kmax = 2, 4
+    idx, g, r = _tiny_alloc_case(seed)
+    k, lam = O.allocate(idx, g, r, kmin, kmax, target)
+    P = idx.size
+    e, gg = idx.reshape(-1), g.reshape(-1)
+    n_hi = int(k.sum())
+    assert n_hi <= target * P
+    def obj(kv):
+        return sum(Fraction(float(gg[p])) * Fraction(float(r[e[p], kv[p] - 1])) for p in range(P))
+    best, best_set = None, []
+    for kv in itertools.product(range(kmin, kmax + 1), repeat=P):
+        if sum(kv) > n_hi:
+            continue
+        o = obj(kv)
+        if best is None or o < best:
+            best, best_set = o, [kv]
+        elif o == best:
+            best_set.append(kv)
+    assert tuple(k.reshape(-1).tolist()) in best_set
+    # generic case: within one plane-step of the budget
+    assert n_hi > target * P - 1
+
+
+def test_allocation_endpoints_and_monotone_trace():
+    idx, g, r = _tiny_alloc_case(5, T=6, K=3)
+    k, _ = O.allocate(idx, g, r, 2, 4, 2.0)
+    assert np.all(k == 2)
+    k, _ = O.allocate(idx, g, r, 2, 4, 4.0)
+    assert np.all(k == 4)
+    trace = []
+    O.allocate(idx, g, r, 2, 4, 3.0, trace=trace)
+    assert len(trace) == 64
+    srt = sorted(trace)
+    assert all(a[1] >= b[1] for a, b in zip(srt, srt[1:]))   # N(lambda) non-increasing
+    with pytest.raises(ValueError):
+        O.allocate(idx, g, r, 2, 4, 4.5)
+
+
+def test_allocation_prefers_high_gate_pairs():
+    # two pairs on the same expert, one with a larger gate: at a budget that allows one
+    # extra plane, the larger gate gets it
+    idx = np.array([[0, 1], [0, 1]], dtype=np.int32)
+    g = np.array([[0.9, 0.1], [0.6, 0.4]])
+    r = np.array([[64.0, 16.0, 4.0, 1.0], [64.0, 16.0, 4.0, 1.0]])
+    k, lam = O.allocate(idx, g, r, 2, 4, 2.25)
+    assert k.tolist() == [[3, 2], [2, 2]]
+
+
+# ----------------------------------------------------------------- FFN and combine
+
+def test_expert_ffn_hand_worked():
+    x = np.array([1.0, 2.0])
+    wg = np.array([[0.5, 0.25]])
+    wu = np.array([[1.0, -1.0]])
+    wd = np.array([[2.0], [-4.0]])
+    o = O.expert_ffn(x, wg, wu, wd)
+    s1 = 1.0 / (1.0 + math.exp(-1.0))          # silu(1) = 1 * sigmoid(1); a = 1, u = -1
+    np.testing.assert_allclose(o, [-2.0 * s1, 4.0 * s1], rtol=1e-15)
+    # swapping gate and up gives a = -1, u = 1 -> a different value (catches a swap)
+    o2 = O.expert_ffn(x, wu, wg, wd)
+    assert not np.allclose(o, o2)
+
+
+def _mini_layer(seed, fmt=0, K=2, norm=1, B=4, kmin=2, kmax=4):
+    from dynamic_any_precision_b200.workloads import LayerShape
+    shape = LayerShape("mini", 32, 16, 4, K, 0, fmt, B, kmin, kmax, 16, norm, 3, (3.0,), seed)
+    rng = np.random.default_rng(seed)
+    experts = {}
+    for e in range(4):
+        mats = [(rng.standard_normal(sh) * 0.2).astype(np.float32) for sh in ((16, 32), (16, 32), (32, 16))]
+        experts[e] = O.encode_expert(*mats, fmt, B, 16)
+    xb = _bf16_bits(rng.standard_normal((3, 32)))
+    wb = _bf16_bits(rng.standard_normal((4, 32)))
+    return shape, experts, xb, wb
+
+
+def test_moe_combine_is_gate_weighted_sum_and_top1_identity():
+    shape, experts, xb, wb = _mini_layer(21)
+    y, aux = O.moe_forward(xb, wb, experts, shape, 3.0)
+    x = O.bf16_bits_to_f64(xb)
+    for t in range(3):
+        acc = np.zeros(32)
+        for j in range(2):
+            e, k = int(aux["idx"][t, j]), int(aux["k"][t, j])
+            wg, wu, wd = O.dequant_expert(experts[e], 0, 4, k, 16)
+            acc += aux["gates"][t, j] * O.expert_ffn(x[t], wg, wu, wd)
+        np.testing.assert_allclose(y[t], acc, rtol=1e-14, atol=1e-15)
+    shape1, experts1, xb1, wb1 = _mini_layer(22, K=1)
+    y1, aux1 = O.moe_forward(xb1, wb1, experts1, shape1, 3.0)
+    assert np.all(aux1["gates"] == 1.0)
+    for t in range(3):
+        e, k = int(aux1["idx"][t, 0]), int(aux1["k"][t, 0])
+        wg, wu, wd = O.dequant_expert(experts1[e], 0, 4, k, 16)
+        np.testing.assert_array_equal(y1[t], O.expert_ffn(O.bf16_bits_to_f64(xb1)[t], wg, wu, wd))
+
+
+def test_prefix_property_low_bits_ignored():
+    shape, experts, xb, wb = _mini_layer(23)
+    y, aux = O.moe_forward(xb, wb, experts, shape, 2.0)     # every pair reads k = 2 planes
+    assert np.all(aux["k"] == 2)
+    rng = np.random.default_rng(0)
+    poisoned = {}
+    for e, enc in experts.items():
+        enc2 = dict(enc)
+        enc2["q"] = [((q >> 2) << 2) | rng.integers(0, 4, size=q.shape).astype(np.uint8) for q in enc["q"]]
+        poisoned[e] = enc2
+    y2, _ = O.moe_forward(xb, wb, poisoned, shape, 2.0, r_table=np.stack([experts[e]["r"] for e in range(4)]))
+    np.testing.assert_array_equal(y, y2)
+
+
+def test_bcq_moe_runs_and_shared_expert_adds():
+    shape, experts, xb, wb = _mini_layer(24, fmt=1, B=3, kmin=1, kmax=3, norm=0)
+    y, aux = O.moe_forward(xb, wb, experts, shape, 2.0)
+    assert np.all(np.isfinite(y))
+    rng = np.random.default_rng(1)
+    sh = (_bf16_bits(rng.standard_normal((1, 16, 32)) * 0.1), _bf16_bits(rng.standard_normal((1, 16, 32)) * 0.1),
+          _bf16_bits(rng.standard_normal((1, 32, 16)) * 0.1))
+    y2, _ = O.moe_forward(xb, wb, experts, shape, 2.0, shared=sh)
+    x = O.bf16_bits_to_f64(xb)
+    for t in range(3):
+        extra = O.expert_ffn(x[t], O.bf16_bits_to_f64(sh[0][0]), O.bf16_bits_to_f64(sh[1][0]),
+                             O.bf16_bits_to_f64(sh[2][0]))
+        np.testing.assert_allclose(y2[t] - y[t], extra, rtol=1e-12, atol=1e-14)
+
+
+# ----------------------------------------------------------------- stack glue
+
+def test_rmsnorm_closed_form_and_bf16_rounding():
+    v = np.full((2, 8), 3.0)
+    np.testing.assert_allclose(O.rmsnorm(v), 3.0 / math.sqrt(9.0 + 1e-6), rtol=1e-15)
+    assert np.all(O.rmsnorm(np.zeros((1, 4))) == 0.0)
+    vals = [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -8 + 2.0 ** -30, -2.5, 1e-3, 123.456]
+    bits = O.f64_to_bf16_bits(np.array(vals))
+    for v_, b in zip(vals, bits):
+        got = Fraction(float(np.array([int(b) << 16], dtype=np.uint32).view(np.float32)[0]))
+        assert got == rne_to_format(Fraction(v_), 7, -126), v_
