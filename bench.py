@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark: MoE-layer decode tokens/s at a target bits-per-weight, and the HBM bandwidth of
+the planes the variable-plane expert GEMV reads, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dpa|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over one batch of synthetic tokens: route (exact-dot
+softmax top-k), plane allocation (64-step Lagrangian bisection), grouping by (expert, k), the
+gate/up GEMV with SwiGLU, the down GEMV and the gate-weighted combine - one dpa_moe_forward.
+Inputs are resident in HBM when the timed region starts. The layer is encoded once and copied
+`--copies` times in device memory; step i uses copy i % copies and its own tokens, so no weight
+byte is re-read within copies-1 steps and the L2 cache (126 MB) cannot serve the planes.
+The K timed steps are one CUDA graph; per-stage CUDA events inside it give the kernel times.
+
+N > 1 GPUs run independent replicas (no collective on the data path; the path shards by
+token batch), one process per GPU under torchrun; the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only), each step a
+bounded sample of the same workload (see cpu_baseline in the output).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_any_precision_b200 import workloads as W  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--impl", choices=("dpa", "reference"), default="dpa")
+    ap.add_argument("--workload", default=W.QWEN3_B1.name)
+    ap.add_argument("--target", type=float, default=None)
+    ap.add_argument("--copies", type=int, default=16)
+    ap.add_argument("--e2e-steps", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=24)
+    return ap.parse_args(argv)
+
+
+def peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML (read-only) in a thread."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.001):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                try:
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def build_layer(shape, seed=None):
+    """Encode one layer on the host (product encoder)."""
+    from dynamic_any_precision_b200 import dpa
+    desc = dpa.make_desc(shape)
+    g, u, d = W.all_expert_weights(shape, seed)
+    planes, meta, r = dpa.encode(desc, g, u, d)
+    del g, u, d
+    wr = W.router_weights(shape, seed)
+    sh = W.shared_weights_bf16(shape, seed) if shape.n_shared else None
+    return desc, planes, meta, r, wr, sh
+
+
+def algorithmic_bytes(shape, idx, k):
+    """Bytes the gate/up and down GEMVs must read for one step: for every active expert its first
+    kmax_e planes of each matrix plus its scale data (kmax_e = max k over its pairs)."""
+    H, I, G, B = shape.hidden, shape.inter, shape.group, shape.bits
+    plane = H * I // 8
+    kmax = {}
+    for e, kk in zip(idx.reshape(-1).tolist(), k.reshape(-1).tolist()):
+        kmax[e] = max(kmax.get(e, 0), kk)
+    gu = dn = 0
+    for e, km in kmax.items():
+        if shape.fmt == W.FMT_UNIFORM:
+            gu += 2 * km * plane + 2 * I * (H // G) * 4
+            dn += km * plane + H * (I // G) * 4
+        else:
+            gu += 2 * km * plane + 2 * km * I * (H // G) * 2
+            dn += km * plane + km * H * (I // G) * 2
+    return gu, dn, len(kmax)
+
+
+def run_dpa(args, shape, target, rank, world, dist):
+    import torch
+    from dynamic_any_precision_b200 import dpa
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    desc, planes, meta, r, wr, sh = build_layer(shape)
+    T, K = shape.tokens, shape.top_k
+    L = max(1, args.copies)
+    base = dpa.DeviceLayer.from_host(desc, planes, meta, r, wr, sh, device=dev)
+    layers = [base]
+    for _ in range(L - 1):
+        layers.append(dpa.DeviceLayer(desc, base.planes.clone(), base.meta.clone(), base.rtable.clone(),
+                                      base.w_router.clone(), base.shared))
+    n_total = args.warmup + args.steps
+    # distinct tokens per step (and per rank)
+    xs = np.stack([W.tokens(shape, T, step=1000 * rank + i) for i in range(n_total)])
+    x_dev = torch.from_numpy(xs.view(np.int16)).to(dev)
+    y_dev = torch.empty((n_total, T, shape.hidden), dtype=torch.int16, device=dev)
+    tg = torch.tensor([target], dtype=torch.float64, device=dev)
+    ws = dpa.new_workspace(desc, T, device=dev)
+    idx_all = torch.empty((args.steps, T, K), dtype=torch.int32, device=dev)
+    gate_all = torch.empty((args.steps, T, K), dtype=torch.float64, device=dev)
+    k_all = torch.empty((args.steps, T, K), dtype=torch.uint8, device=dev)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+
+    def step(i, timed_j=None):
+        aux = None
+        if timed_j is not None:
+            aux = {"topk_idx": idx_all[timed_j], "topk_gate": gate_all[timed_j], "k": k_all[timed_j],
+                   "events": events[timed_j]}
+        dpa.moe_forward(layers[i % L], x_dev[i], tg, ws, y=y_dev[i], aux=aux)
+
+    # eager run of every distinct layer copy once (loads the module, sets kernel attributes)
+    for i in range(min(L, n_total)):
+        step(i)
+    torch.cuda.synchronize()
+    assert dpa.device_status(ws) == 0
+
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g_warm, stream=s):
+            for i in range(args.warmup):
+                step(i)
+        with torch.cuda.graph(g_timed, stream=s):
+            for j in range(args.steps):
+                step(args.warmup + j, timed_j=j)
+    torch.cuda.synchronize()
+    g_warm.replay()
+    torch.cuda.synchronize()
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record()
+        g_timed.replay()
+        t1.record()
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    st = dpa.device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {dpa.STATUS_NAMES.get(st, st)}")
+    if dist is not None:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+
+    # per-stage kernel times inside the timed region
+    names = ["route", "allocate", "shared", "gateup", "down", "combine"]
+    stage_ms = {n: 0.0 for n in names}
+    for j in range(args.steps):
+        ev = events[j]
+        for q, n in enumerate(names):
+            stage_ms[n] += ev[q].elapsed_time(ev[q + 1])
+    idx_h, k_h = idx_all.cpu().numpy(), k_all.cpu().numpy()
+    gu_bytes = dn_bytes = 0
+    n_active = 0
+    for j in range(args.steps):
+        a, b, c = algorithmic_bytes(shape, idx_h[j], k_h[j])
+        gu_bytes += a
+        dn_bytes += b
+        n_active += c
+    mean_bpw = float(k_h.astype(np.float64).mean())
+
+    # e2e through the public API with host buffers (pinned), copies inside the timed region
+    e2e = None
+    if args.e2e_steps > 0:
+        n_e = min(args.e2e_steps, n_total)
+        x_host = torch.from_numpy(xs[:n_e].view(np.int16)).pin_memory()
+        y_host = torch.empty((n_e, T, shape.hidden), dtype=torch.int16).pin_memory()
+        x_buf = torch.empty((T, shape.hidden), dtype=torch.int16, device=dev)
+        y_buf = torch.empty((T, shape.hidden), dtype=torch.int16, device=dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(n_e):
+            x_buf.copy_(x_host[i], non_blocking=True)
+            dpa.moe_forward(layers[i % L], x_buf, tg, ws, y=y_buf)
+            y_host[i].copy_(y_buf, non_blocking=True)
+            torch.cuda.current_stream().synchronize()   # the host reads this step's result
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if dist is not None:
+            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * T * n_e / (e_ms * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(x_buf.numel() * 2), "d2h_bytes_per_step": int(y_buf.numel() * 2),
+               "steps": n_e}
+
+    launches_per_step = 5 + (2 if shape.n_shared else 0)
+    return {"ms": ms, "stage_ms": stage_ms, "gu_bytes": gu_bytes, "dn_bytes": dn_bytes, "n_active": n_active,
+            "mean_bpw": mean_bpw, "clocks": clk.summary(), "e2e": e2e, "launches": launches_per_step * args.steps}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(shape, target, n_tokens, seed_base=0):
+    """Times the fp64 oracle (as it stands) on `n_tokens` single-token steps of the workload.
+    Each step routes and allocates the token in full; of its top_k expert FFNs one (round
+    robin over the slots) is run and its time counted top_k times. Encoding the routed
+    experts is offline work (as in the product) and is not timed."""
+    from threadpoolctl import threadpool_limits
+    from oracle import dpa_oracle as O
+    wr = W.router_weights(shape)
+    xs = [W.tokens(shape, shape.tokens, step=seed_base + i) for i in range(n_tokens)]
+    with threadpool_limits(1):
+        routes = [O.route(x, wr, shape.top_k, shape.norm_topk) for x in xs]
+        need = sorted({int(routes[i][0][0, i % shape.top_k]) for i in range(n_tokens)}
+                      | {int(e) for rt in routes for e in np.unique(rt[0])})
+        experts = {}
+        for e in need:
+            g, u, d = W.expert_weights(shape, e)
+            experts[e] = O.encode_expert(g, u, d, shape.fmt, shape.bits, shape.group)
+        r = np.full((shape.n_experts, shape.bits), np.nan)
+        for e, enc in experts.items():
+            r[e] = enc["r"]
+        total = 0.0
+        for i, x in enumerate(xs):
+            t0 = time.perf_counter()
+            idx, g, _ = O.route(x, wr, shape.top_k, shape.norm_topk)
+            k, lam = O.allocate(idx, g, r, shape.kmin, shape.kmax, target)
+            t1 = time.perf_counter()
+            j = i % shape.top_k
+            xf = O.bf16_bits_to_f64(x)[0]
+            e, kk = int(idx[0, j]), int(k[0, j])
+            wg, wu, wd = O.dequant_expert(experts[e], shape.fmt, shape.bits, kk, shape.group)
+            O.expert_ffn(xf, wg, wu, wd)
+            t2 = time.perf_counter()
+            total += (t1 - t0) + shape.top_k * (t2 - t1)
+    return {"value": shape.tokens * n_tokens / total, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_tokens} single-token steps: route + allocate in full, 1 of {shape.top_k} expert "
+                      f"FFNs per step timed and counted x{shape.top_k}; fp64 numpy, 1 thread",
+            "seconds": total}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main(argv=None):
+    args = parse_args(argv)
+    shape = W.shape_by_name(args.workload)
+    target = args.target if args.target is not None else shape.targets[0]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    metric = "MoE-layer decode tokens/s at target bpw; HBM GB/s of planes read vs peak"
+    config = {"workload": shape.name, "hidden": shape.hidden, "inter": shape.inter, "experts": shape.n_experts,
+              "top_k": shape.top_k, "tokens_per_step": shape.tokens, "target_bpw": target,
+              "format": "uniform" if shape.fmt == W.FMT_UNIFORM else "bcq", "bits": shape.bits,
+              "kmin": shape.kmin, "kmax": shape.kmax, "group": shape.group, "parallelism": f"replicas{args.gpus}",
+              "l2": f"inputs larger than L2: {args.copies} device copies of the layer rotated per step"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        steps = args.steps
+        smp = oracle_sample(shape, target, args.warmup + steps)
+        line = {"impl": "reference", "metric": metric, "value": smp["value"], "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * shape.tokens / smp["value"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": smp["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    import torch
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+
+    res = run_dpa(args, shape, target, rank, world, dist)
+    hbm, peak_kind = peaks()
+    secs = res["ms"] * 1e-3
+    tokens = world * shape.tokens * args.steps
+    stage = res["stage_ms"]
+    dominant = max(("gateup", "down"), key=lambda n: stage[n])
+    dom_bytes = res["gu_bytes"] if dominant == "gateup" else res["dn_bytes"]
+    dom_s = stage[dominant] * 1e-3
+    achieved = dom_bytes / dom_s / 1e9 if dom_s > 0 else 0.0
+    all_bytes = res["gu_bytes"] + res["dn_bytes"]
+    line = {
+        "metric": metric,
+        "value": tokens / secs,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": res["ms"] / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u8s8-i32/f32 (decision path f64)",
+        "data": "synthetic",
+        "config": config,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "peak_source": peak_kind},
+        "planes_gbs_whole_step": all_bytes / secs / 1e9 / world,
+        "planes_frac_whole_step": all_bytes / secs / 1e9 / world / hbm,
+        "bytes_per_step": all_bytes / args.steps,
+        "active_experts_per_step": res["n_active"] / args.steps,
+        "mean_planes_per_pair": res["mean_bpw"],
+        "stages_us_per_step": {k: 1e3 * v / args.steps for k, v in stage.items()},
+        "clocks": res["clocks"],
+        "e2e": res["e2e"],
+        "gpu_launches": res["launches"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = oracle_sample(shape, target, args.cpu_sample_tokens, seed_base=50000)
+        line["cpu_baseline"] = {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+// Gate-weighted combine of the routed experts' outputs, plus the dense always-on experts.
+//
+// y[t] = bf16( sum over the token's slots, in slot order, of g * o_pair  (+ shared[t]) ).
+// A per-token gather (no atomics), so the sum order is fixed and the result deterministic.
+// Shared experts (DeepSeekMoE-style, always on) run densely in bf16 with fp32 accumulation;
+// they are neither allocated nor counted in the plane budget.
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dpa {
+namespace {
+
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+    const int t = blockIdx.y;
+    const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
+    if (n >= a.H) return;
+    float4 acc = a.shared_out ? *reinterpret_cast<const float4*>(a.shared_out + static_cast<size_t>(t) * a.H + n)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < a.K; ++s) {
+        const int p = t * a.K + s;
+        const int pos = a.pair_pos[p];
+        const float g = static_cast<float>(a.gate[p]);
+        const float4 o = *reinterpret_cast<const float4*>(a.out_pair + static_cast<size_t>(pos) * a.H + n);
+        r.x = fmaf(g, o.x, r.x);
+        r.y = fmaf(g, o.y, r.y);
+        r.z = fmaf(g, o.z, r.z);
+        r.w = fmaf(g, o.w, r.w);
+        if (a.pair_out_user) *reinterpret_cast<float4*>(a.pair_out_user + static_cast<size_t>(p) * a.H + n) = o;
+    }
+    acc.x += r.x;
+    acc.y += r.y;
+    acc.z += r.z;
+    acc.w += r.w;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 packed;
+    packed.x = *reinterpret_cast<uint32_t*>(&lo);
+    packed.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.y + static_cast<size_t>(t) * a.H + n) = packed;
+}
+
+// ---- dense shared experts: warp per (row, expert), all tokens in chunks of 8 ----
+constexpr int kTokChunk = 8;
+
+__device__ __forceinline__ void bf16x8_to_f32(uint4 v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__global__ void __launch_bounds__(256) shared_gateup_kernel(SharedArgs a) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int row = warp % a.I, s = warp / a.I;
+    if (s >= a.S) return;
+    const uint16_t* gr = a.wg + (static_cast<size_t>(s) * a.I + row) * a.H;
+    const uint16_t* ur = a.wu + (static_cast<size_t>(s) * a.I + row) * a.H;
+    for (int t0 = 0; t0 < a.T; t0 += kTokChunk) {
+        float ag[kTokChunk], au[kTokChunk];
+#pragma unroll
+        for (int i = 0; i < kTokChunk; ++i) ag[i] = au[i] = 0.f;
+        for (int j = lane * 8; j < a.H; j += 256) {
+            float g8[8], u8[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(gr + j), g8);
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(ur + j), u8);
+#pragma unroll
+            for (int i = 0; i < kTokChunk; ++i) {
+                if (t0 + i < a.T) {
+                    float x8[8];
+                    bf16x8_to_f32(*reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + i) * a.H + j), x8);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        ag[i] = fmaf(g8[q], x8[q], ag[i]);
+                        au[i] = fmaf(u8[q], x8[q], au[i]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kTokChunk; ++i) {
+            float g = ag[i], u = au[i];
+            for (int o = 16; o > 0; o >>= 1) {
+                g += __shfl_xor_sync(0xffffffffu, g, o);
+                u += __shfl_xor_sync(0xffffffffu, u, o);
+            }
+            if (lane == 0 && t0 + i < a.T)
+                a.h[(static_cast<size_t>(t0 + i) * a.S + s) * a.I + row] = g / (1.f + expf(-g)) * u;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) shared_down_kernel(SharedArgs a) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int n = warp;
+    if (n >= a.H) return;
+    for (int t0 = 0; t0 < a.T; t0 += kTokChunk) {
+        float acc[kTokChunk];
+#pragma unroll
+        for (int i = 0; i < kTokChunk; ++i) acc[i] = 0.f;
+        for (int s = 0; s < a.S; ++s) {
+            const uint16_t* dr = a.wd + (static_cast<size_t>(s) * a.H + n) * a.I;
+            for (int j = lane * 8; j < a.I; j += 256) {
+                float d8[8];
+                bf16x8_to_f32(*reinterpret_cast<const uint4*>(dr + j), d8);
+#pragma unroll
+                for (int i = 0; i < kTokChunk; ++i) {
+                    if (t0 + i < a.T) {
+                        const float* hr = a.h + (static_cast<size_t>(t0 + i) * a.S + s) * a.I + j;
+                        const float4 h0 = *reinterpret_cast<const float4*>(hr);
+                        const float4 h1 = *reinterpret_cast<const float4*>(hr + 4);
+                        acc[i] = fmaf(d8[0], h0.x, acc[i]);
+                        acc[i] = fmaf(d8[1], h0.y, acc[i]);
+                        acc[i] = fmaf(d8[2], h0.z, acc[i]);
+                        acc[i] = fmaf(d8[3], h0.w, acc[i]);
+                        acc[i] = fmaf(d8[4], h1.x, acc[i]);
+                        acc[i] = fmaf(d8[5], h1.y, acc[i]);
+                        acc[i] = fmaf(d8[6], h1.z, acc[i]);
+                        acc[i] = fmaf(d8[7], h1.w, acc[i]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kTokChunk; ++i) {
+            float v = acc[i];
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0 && t0 + i < a.T) a.out[static_cast<size_t>(t0 + i) * a.H + n] = v;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
+    const int per_block = 256 * 4;
+    dim3 grid((a.H + per_block - 1) / per_block, a.T);
+    combine_kernel<<<grid, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_shared(const SharedArgs& a, cudaStream_t stream) {
+    if (a.S == 0 || a.T == 0) return cudaSuccess;
+    const int warps1 = a.S * a.I;
+    shared_gateup_kernel<<<(warps1 + 7) / 8, 256, 0, stream>>>(a);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    shared_down_kernel<<<(a.H + 7) / 8, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace dpa

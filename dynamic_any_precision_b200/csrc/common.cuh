@@ -1,0 +1,154 @@
+// Device helpers shared by the sm_100a kernels: workspace header, error flag, bounded
+// mbarrier waits, bulk global->shared copies, MMA wrappers.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "dpa.h"
+
+namespace dpa {
+
+// ---- workspace header (first 256 bytes of every workspace) ----
+struct WsHeader {
+    uint32_t error;       // first device error code (0 = none)
+    uint32_t error_info;  // kernel-specific detail (which wait, which index)
+    uint32_t n_active;    // routed experts with at least one pair in the last forward
+    uint32_t pad[61];
+};
+static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
+
+__device__ __forceinline__ void set_error(WsHeader* h, uint32_t code, uint32_t info) {
+    if (atomicCAS(&h->error, 0u, code) == 0u) h->error_info = info;
+}
+
+// ---- bounded waits ----
+// Every spin in these kernels gives up after kWaitNs nanoseconds (device clock), records
+// DPA_ERR_DEVICE_TIMEOUT and returns, so a lost completion can never hang the GPU.
+constexpr uint64_t kWaitNs = 200ull * 1000ull * 1000ull;   // 200 ms
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` with a time limit. Returns false on timeout (after
+// recording the error). The caller must not read the buffers the barrier guards then.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, WsHeader* hdr,
+                                                  uint32_t where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer() - t0 > kWaitNs) {
+            set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
+            return false;
+        }
+    }
+    return true;
+}
+
+// CTA-uniform wait for a bulk-copy phase: thread 0 waits with a time limit (and on a
+// timeout gives the copies a second bounded chance to land, so none is left writing into
+// shared memory of a CTA that exits); the verdict is broadcast through `flag` so that every
+// thread returns or continues together. Then each thread observes the completed phase
+// itself (immediate), which orders the copied data before its reads.
+__device__ __forceinline__ bool cta_wait_copies(uint64_t* bar, uint32_t parity, WsHeader* hdr, uint32_t where,
+                                                int* flag) {
+    if (threadIdx.x == 0) {
+        bool ok = mbar_wait_bounded(bar, parity, hdr, where);
+        if (!ok) mbar_wait_bounded(bar, parity, hdr, where + 1);
+        *flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    const bool ok = *flag != 0;
+    if (ok) (void)mbar_try_wait(bar, parity);
+    return ok;
+}
+
+// Order this thread's (and, after a barrier, the CTA's) generic-proxy shared-memory accesses
+// before later async-proxy (bulk copy) writes to the same buffers.
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Untiled bulk copy global -> shared, completing `bytes` of transaction count on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ---- u8 x s8 MMA, m16n8k32, int32 accumulate ----
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---- fixed-point digits of a group of activations ----
+// A group of values v_j is represented exactly (or to 22 fractional bits of its largest
+// magnitude) as v_j = X_j * 2^(E - 22) with |X_j| <= 2^22, E = exponent with max|v| < 2^E.
+// X_j is split into balanced base-256 digits d0 + 256*d1 + 65536*d2, each an int8, which are
+// the s8 operand of the MMA.
+__device__ __forceinline__ int group_exponent(float maxabs) {
+    if (!(maxabs > 0.f)) return 0;
+    int e;
+    frexpf(maxabs, &e);
+    return e;
+}
+
+__device__ __forceinline__ int to_fixed(float v, int E) {
+    return __float2int_rn(ldexpf(v, 22 - E));
+}
+
+__device__ __forceinline__ void split_digits(int X, int8_t& d0, int8_t& d1, int8_t& d2) {
+    const int a0 = ((X + 128) & 255) - 128;
+    const int X1 = (X - a0) >> 8;
+    const int a1 = ((X1 + 128) & 255) - 128;
+    const int a2 = (X1 - a1) >> 8;
+    d0 = static_cast<int8_t>(a0);
+    d1 = static_cast<int8_t>(a1);
+    d2 = static_cast<int8_t>(a2);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+}  // namespace dpa

@@ -1,0 +1,373 @@
+// C ABI of the library (include/dpa.h): validation, sizes, workspace layout, launches.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "dpa.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kMaxDynSmem = 200 * 1024;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dpa_status check_desc(const dpa_layer_desc* d) {
+    if (!d) return DPA_ERR_INVALID_ARG;
+    if (d->hidden <= 0 || d->inter <= 0 || d->n_experts <= 0 || d->top_k <= 0 || d->group <= 0)
+        return DPA_ERR_INVALID_ARG;
+    if (d->format != DPA_FMT_UNIFORM && d->format != DPA_FMT_BCQ) return DPA_ERR_INVALID_ARG;
+    if (d->bits < 1 || d->kmin < 1 || d->kmin > d->kmax || d->kmax > d->bits) return DPA_ERR_INVALID_ARG;
+    if (d->norm_topk != 0 && d->norm_topk != 1) return DPA_ERR_INVALID_ARG;
+    if (d->n_shared < 0 || d->top_k > d->n_experts) return DPA_ERR_INVALID_ARG;
+    if (d->bits > 4 || d->n_experts > 1024 || d->top_k > 32 || d->n_shared > 8) return DPA_ERR_UNSUPPORTED;
+    if (d->hidden % 64 || d->inter % 64 || d->group % 64) return DPA_ERR_UNSUPPORTED;
+    if (d->hidden % d->group || d->inter % d->group) return DPA_ERR_UNSUPPORTED;
+    if (d->hidden > 16384 || d->inter > 16384) return DPA_ERR_UNSUPPORTED;
+    // the per-CTA staging of one work item must fit in shared memory
+    dpa::GemvArgs ga{};
+    ga.H = d->hidden;
+    ga.I = d->inter;
+    ga.B = d->bits;
+    ga.G = d->group;
+    ga.fmt = d->format;
+    if (dpa::gateup_smem_bytes(ga) > kMaxDynSmem || dpa::down_smem_bytes(ga) > kMaxDynSmem) return DPA_ERR_UNSUPPORTED;
+    return DPA_OK;
+}
+
+// ---- workspace layout ----
+struct WsLayout {
+    size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, sorted, pairpos, seg, kmaxe, active, xdig, xexp,
+        xsum, h, out_pair, sh_h, sh_out, total;
+};
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+WsLayout ws_layout(const dpa_layer_desc* d, int T) {
+    WsLayout L;
+    const size_t P = static_cast<size_t>(T) * d->top_k;
+    const int nk = d->kmax - d->kmin + 1;
+    const size_t E = d->n_experts, H = d->hidden, I = d->inter;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = align256(off + bytes);
+        return o;
+    };
+    L.hdr = take(sizeof(dpa::WsHeader));
+    L.counters = take(sizeof(unsigned) * T);
+    L.logits = take(8 * static_cast<size_t>(T) * E);
+    L.idx = take(4 * P);
+    L.gate = take(8 * P);
+    L.k = take(P);
+    L.lambda = take(8);
+    L.cbuf = take(8 * P * nk);
+    L.sorted = take(4 * P);
+    L.pairpos = take(4 * P);
+    L.seg = take(4 * (E * nk + 1));
+    L.kmaxe = take(4 * E);
+    L.active = take(4 * E);
+    L.xdig = take(3 * static_cast<size_t>(T) * H);
+    L.xexp = take(4 * static_cast<size_t>(T) * (H / d->group));
+    L.xsum = take(4 * static_cast<size_t>(T) * (H / d->group));
+    L.h = take(4 * P * I);
+    L.out_pair = take(4 * P * H);
+    L.sh_h = take(4 * static_cast<size_t>(T) * d->n_shared * I);
+    L.sh_out = take(4 * static_cast<size_t>(T) * H);
+    L.total = off;
+    return L;
+}
+
+int num_sms_current() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int n = 148;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (dev < 64) cache[dev] = n;
+    return n;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dpa_version(void) { return 100; }
+
+const char* dpa_status_string(dpa_status s) {
+    switch (s) {
+        case DPA_OK: return "ok";
+        case DPA_ERR_INVALID_ARG: return "invalid argument";
+        case DPA_ERR_UNSUPPORTED: return "unsupported shape";
+        case DPA_ERR_WORKSPACE: return "workspace too small";
+        case DPA_ERR_CUDA: return "CUDA error";
+        case DPA_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case DPA_ERR_DEVICE_INVALID_INPUT: return "invalid device input";
+    }
+    return "unknown status";
+}
+
+dpa_status dpa_encoded_sizes(const dpa_layer_desc* d, dpa_sizes* out) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (!out) return DPA_ERR_INVALID_ARG;
+    const uint64_t H = d->hidden, I = d->inter, B = d->bits, G = d->group;
+    const uint64_t mat_planes = B * H * I / 8;     // one matrix, all planes
+    std::memset(out, 0, sizeof(*out));
+    out->planes_matrix_offset[0] = 0;
+    out->planes_matrix_offset[1] = mat_planes;
+    out->planes_matrix_offset[2] = 2 * mat_planes;
+    out->planes_per_expert = 3 * mat_planes;
+    uint64_t mg, md;   // meta bytes of gate (= up) and down
+    if (d->format == DPA_FMT_UNIFORM) {
+        mg = I * (H / G) * 4;
+        md = H * (I / G) * 4;
+    } else {
+        mg = B * I * (H / G) * 2;
+        md = B * H * (I / G) * 2;
+    }
+    out->meta_matrix_offset[0] = 0;
+    out->meta_matrix_offset[1] = mg;
+    out->meta_matrix_offset[2] = 2 * mg;
+    out->meta_per_expert = 2 * mg + md;
+    out->planes_bytes = out->planes_per_expert * d->n_experts;
+    out->meta_bytes = out->meta_per_expert * d->n_experts;
+    out->rtable_bytes = static_cast<uint64_t>(d->n_experts) * B * 8;
+    return DPA_OK;
+}
+
+size_t dpa_forward_workspace_size(const dpa_layer_desc* d, int max_tokens) {
+    if (check_desc(d) != DPA_OK || max_tokens <= 0) return 0;
+    return ws_layout(d, max_tokens).total;
+}
+
+dpa_status dpa_route(const dpa_layer_desc* d, const void* x, int n_tokens, const void* w_router,
+                     int32_t* topk_idx, double* topk_gate, double* logits, void* ws, size_t ws_bytes,
+                     void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (n_tokens <= 0 || n_tokens > 65535 || !x || !w_router || !topk_idx || !topk_gate || !ws)
+        return DPA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(ws) || !aligned16(topk_idx) || !aligned16(topk_gate) ||
+        (logits && !aligned16(logits)))
+        return DPA_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(d, n_tokens);
+    if (ws_bytes < L.total) return DPA_ERR_WORKSPACE;
+    dpa::RouteArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.wr = static_cast<const uint16_t*>(w_router);
+    a.T = n_tokens;
+    a.E = d->n_experts;
+    a.H = d->hidden;
+    a.K = d->top_k;
+    a.G = d->group;
+    a.norm_topk = d->norm_topk;
+    a.logits_user = logits;
+    a.logits_ws = at<double>(ws, L.logits);
+    a.idx = topk_idx;
+    a.gate = topk_gate;
+    a.counters = at<unsigned>(ws, L.counters);
+    a.xdig = nullptr;
+    a.hdr = at<dpa::WsHeader>(ws, L.hdr);
+    return dpa::launch_route(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
+}
+
+static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, const int32_t* idx,
+                                const double* gate, int T, const double* target, uint8_t* k_out,
+                                double* lambda_out, void* ws, const WsLayout& L, bool permute, cudaStream_t s) {
+    dpa::AllocArgs a{};
+    a.rtable = rtable;
+    a.idx = idx;
+    a.gate = gate;
+    a.target = target;
+    a.T = T;
+    a.K = d->top_k;
+    a.E = d->n_experts;
+    a.B = d->bits;
+    a.kmin = d->kmin;
+    a.kmax = d->kmax;
+    a.k_out = k_out;
+    a.lambda_out = lambda_out;
+    a.cbuf = at<double>(ws, L.cbuf);
+    a.do_permute = permute ? 1 : 0;
+    a.sorted_pair = at<int32_t>(ws, L.sorted);
+    a.pair_pos = at<int32_t>(ws, L.pairpos);
+    a.seg_start = at<int32_t>(ws, L.seg);
+    a.exp_kmax = at<int32_t>(ws, L.kmaxe);
+    a.active = at<int32_t>(ws, L.active);
+    a.k_copy = nullptr;
+    a.hdr = at<dpa::WsHeader>(ws, L.hdr);
+    return dpa::launch_allocate(a, s) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
+}
+
+dpa_status dpa_allocate(const dpa_layer_desc* d, const double* rtable, const int32_t* topk_idx,
+                        const double* topk_gate, int n_tokens, const double* target_bpw, uint8_t* k_out,
+                        double* lambda_out, void* ws, size_t ws_bytes, void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (n_tokens <= 0 || n_tokens > 65535 || !rtable || !topk_idx || !topk_gate || !target_bpw || !k_out || !ws)
+        return DPA_ERR_INVALID_ARG;
+    if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(rtable) & 7) || (reinterpret_cast<uintptr_t>(topk_gate) & 7) ||
+        (reinterpret_cast<uintptr_t>(target_bpw) & 7) || (reinterpret_cast<uintptr_t>(topk_idx) & 3))
+        return DPA_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(d, n_tokens);
+    if (ws_bytes < L.total) return DPA_ERR_WORKSPACE;
+    return allocate_impl(d, rtable, topk_idx, topk_gate, n_tokens, target_bpw, k_out, lambda_out, ws, L, false,
+                         static_cast<cudaStream_t>(stream));
+}
+
+dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, const void* x, int n_tokens,
+                           const double* target_bpw, void* y, dpa_aux* aux, void* ws, size_t ws_bytes,
+                           void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (!w || !x || !y || !ws || !target_bpw || n_tokens <= 0 || n_tokens > 65535) return DPA_ERR_INVALID_ARG;
+    if (!w->planes || !w->meta || !w->rtable || !w->w_router) return DPA_ERR_INVALID_ARG;
+    if (d->n_shared > 0 && (!w->shared_gate || !w->shared_up || !w->shared_down)) return DPA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws) || !aligned16(w->planes) || !aligned16(w->meta) ||
+        !aligned16(w->w_router) || (reinterpret_cast<uintptr_t>(w->rtable) & 7) ||
+        (reinterpret_cast<uintptr_t>(target_bpw) & 7))
+        return DPA_ERR_INVALID_ARG;
+    if (d->n_shared > 0 && (!aligned16(w->shared_gate) || !aligned16(w->shared_up) || !aligned16(w->shared_down)))
+        return DPA_ERR_INVALID_ARG;
+    if (aux && aux->pair_out && !aligned16(aux->pair_out)) return DPA_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(d, n_tokens);
+    if (ws_bytes < L.total) return DPA_ERR_WORKSPACE;
+    dpa_sizes sz;
+    dpa_encoded_sizes(d, &sz);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int T = n_tokens, K = d->top_k;
+
+    int32_t* idx = (aux && aux->topk_idx) ? aux->topk_idx : at<int32_t>(ws, L.idx);
+    double* gate = (aux && aux->topk_gate) ? aux->topk_gate : at<double>(ws, L.gate);
+    uint8_t* kk = (aux && aux->k) ? aux->k : at<uint8_t>(ws, L.k);
+    double* lam = (aux && aux->lambda) ? aux->lambda : at<double>(ws, L.lambda);
+    dpa::WsHeader* hdr = at<dpa::WsHeader>(ws, L.hdr);
+
+    auto mark = [&](int i) {
+        if (aux && aux->events[i]) cudaEventRecord(static_cast<cudaEvent_t>(aux->events[i]), s);
+    };
+    mark(0);
+    // 1. route (+ fixed-point digits of x)
+    dpa::RouteArgs ra{};
+    ra.x = static_cast<const uint16_t*>(x);
+    ra.wr = static_cast<const uint16_t*>(w->w_router);
+    ra.T = T;
+    ra.E = d->n_experts;
+    ra.H = d->hidden;
+    ra.K = K;
+    ra.G = d->group;
+    ra.norm_topk = d->norm_topk;
+    ra.logits_user = nullptr;
+    ra.logits_ws = at<double>(ws, L.logits);
+    ra.idx = idx;
+    ra.gate = gate;
+    ra.counters = at<unsigned>(ws, L.counters);
+    ra.xdig = at<int8_t>(ws, L.xdig);
+    ra.xexp = at<int32_t>(ws, L.xexp);
+    ra.xsum = at<int32_t>(ws, L.xsum);
+    ra.hdr = hdr;
+    if (dpa::launch_route(ra, s) != cudaSuccess) return DPA_ERR_CUDA;
+    mark(1);
+
+    // 2. allocate + group pairs by (expert, k)
+    dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s);
+    if (st2 != DPA_OK) return st2;
+    mark(2);
+
+    // 3. dense shared experts
+    if (d->n_shared > 0) {
+        dpa::SharedArgs sa{};
+        sa.x = static_cast<const uint16_t*>(x);
+        sa.wg = static_cast<const uint16_t*>(w->shared_gate);
+        sa.wu = static_cast<const uint16_t*>(w->shared_up);
+        sa.wd = static_cast<const uint16_t*>(w->shared_down);
+        sa.h = at<float>(ws, L.sh_h);
+        sa.out = at<float>(ws, L.sh_out);
+        sa.T = T;
+        sa.S = d->n_shared;
+        sa.H = d->hidden;
+        sa.I = d->inter;
+        if (dpa::launch_shared(sa, s) != cudaSuccess) return DPA_ERR_CUDA;
+    }
+    mark(3);
+
+    // 4. variable-plane expert FFN
+    dpa::GemvArgs ga{};
+    ga.planes = static_cast<const uint8_t*>(w->planes);
+    ga.meta = static_cast<const uint8_t*>(w->meta);
+    ga.planes_per_expert = sz.planes_per_expert;
+    ga.meta_per_expert = sz.meta_per_expert;
+    for (int m = 0; m < 3; ++m) {
+        ga.planes_mat_off[m] = sz.planes_matrix_offset[m];
+        ga.meta_mat_off[m] = sz.meta_matrix_offset[m];
+    }
+    ga.E = d->n_experts;
+    ga.H = d->hidden;
+    ga.I = d->inter;
+    ga.K = K;
+    ga.B = d->bits;
+    ga.G = d->group;
+    ga.kmin = d->kmin;
+    ga.kmax = d->kmax;
+    ga.fmt = d->format;
+    ga.sorted_pair = at<int32_t>(ws, L.sorted);
+    ga.seg_start = at<int32_t>(ws, L.seg);
+    ga.exp_kmax = at<int32_t>(ws, L.kmaxe);
+    ga.active = at<int32_t>(ws, L.active);
+    ga.xdig = at<int8_t>(ws, L.xdig);
+    ga.xexp = at<int32_t>(ws, L.xexp);
+    ga.xsum = at<int32_t>(ws, L.xsum);
+    ga.h = at<float>(ws, L.h);
+    ga.out_pair = at<float>(ws, L.out_pair);
+    ga.hdr = hdr;
+    const int P = T * K;
+    ga.max_items = P < d->n_experts ? P : d->n_experts;
+    const int sms = num_sms_current();
+    if (dpa::launch_gateup(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
+    mark(4);
+    if (dpa::launch_down(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
+    mark(5);
+
+    // 5. combine
+    dpa::CombineArgs ca{};
+    ca.out_pair = at<float>(ws, L.out_pair);
+    ca.pair_pos = at<int32_t>(ws, L.pairpos);
+    ca.gate = gate;
+    ca.shared_out = d->n_shared > 0 ? at<float>(ws, L.sh_out) : nullptr;
+    ca.pair_out_user = aux ? aux->pair_out : nullptr;
+    ca.y = static_cast<uint16_t*>(y);
+    ca.T = T;
+    ca.K = K;
+    ca.H = d->hidden;
+    ca.hdr = hdr;
+    if (dpa::launch_combine(ca, s) != cudaSuccess) return DPA_ERR_CUDA;
+    mark(6);
+    return DPA_OK;
+}
+
+dpa_status dpa_device_status(void* ws, void* stream) {
+    if (!ws) return DPA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DPA_ERR_CUDA;
+    uint32_t v[2] = {0, 0};
+    if (cudaMemcpy(v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DPA_ERR_CUDA;
+    if (v[0] != 0) {
+        const uint32_t zero[2] = {0, 0};
+        if (cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return DPA_ERR_CUDA;
+    }
+    return static_cast<dpa_status>(v[0]);
+}
+
+}  // extern "C"

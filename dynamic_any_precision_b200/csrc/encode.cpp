@@ -1,0 +1,307 @@
+// Offline encoder of routed expert weights into prefix-decodable bitplanes (host C++).
+//
+// DPA-MoE: A Runtime Precision Control Framework for MoE Inference, Abstract: expert FFN
+// weights become prefix-decodable chunks under one shared scale ("SharedScale AnyBCQ"), and
+// per-expert reconstruction residuals are profiled offline.
+// MatMoE (review, "Core Contribution"): bitplane storage; one set of quantisation parameters
+// serves the low-bit prefix and the full precision.
+// DuoRate, Abstract: one stored tier of a prefix-readable weight stream plus a baked
+// distortion tensor.
+//
+// Build with -ffp-contract=off and without fast-math: every fp64 operation below is one IEEE
+// round-to-nearest operation, so the codes, scales and residual sums are reproducible.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "dpa.h"
+#include "layout.h"
+
+namespace {
+
+// ---- fp16 <-> fp64 (round to nearest, ties to even, gradual underflow) ----
+uint16_t f64_to_f16_bits(double v) {
+    uint64_t b;
+    std::memcpy(&b, &v, 8);
+    const uint16_t sign = static_cast<uint16_t>((b >> 48) & 0x8000u);
+    const int exp = static_cast<int>((b >> 52) & 0x7FF);
+    uint64_t man = b & ((1ull << 52) - 1);
+    if (exp == 0x7FF) return sign | 0x7C00u | (man ? 0x200u : 0u);
+    if (exp == 0 && man == 0) return sign;
+    // value = 1.man * 2^(exp-1023) (fp64 subnormals are far below fp16's range -> 0)
+    int e = exp - 1023;
+    if (exp == 0) return sign;
+    uint64_t sig = man | (1ull << 52);          // 53-bit significand
+    int shift;                                   // bits of sig to drop
+    uint16_t hexp;
+    if (e >= -14) {                              // normal fp16 candidate
+        shift = 52 - 10;
+        hexp = static_cast<uint16_t>(e + 15);
+    } else {                                     // subnormal fp16: unit 2^-24
+        shift = 52 - 10 + (-14 - e);
+        hexp = 0;
+        if (shift > 63) return sign;
+    }
+    uint64_t keep = sig >> shift;
+    uint64_t rem = sig & ((1ull << shift) - 1);
+    uint64_t half = 1ull << (shift - 1);
+    if (rem > half || (rem == half && (keep & 1))) keep += 1;
+    uint32_t out;
+    if (hexp == 0) {
+        out = static_cast<uint32_t>(keep);       // may carry into the smallest normal: fine
+    } else {
+        if (keep >> 11) { keep >>= 1; hexp += 1; }
+        if (hexp >= 31) return sign | 0x7C00u;   // overflow -> inf
+        out = (static_cast<uint32_t>(hexp) << 10) | static_cast<uint32_t>(keep & 0x3FF);
+    }
+    return sign | static_cast<uint16_t>(out);
+}
+
+double f16_bits_to_f64(uint16_t h) {
+    const int sign = (h >> 15) & 1;
+    const int exp = (h >> 10) & 0x1F;
+    const int man = h & 0x3FF;
+    double v;
+    if (exp == 0) v = std::ldexp(static_cast<double>(man), -24);
+    else if (exp == 31) v = man ? NAN : INFINITY;
+    else v = std::ldexp(static_cast<double>(man | 0x400), exp - 25);
+    return sign ? -v : v;
+}
+
+struct Mat {
+    const float* w;   // [R][C]
+    int R, C;
+};
+
+// Place the code bits of weight (row, col) of one matrix into its planes.
+inline void set_code(uint32_t* mat_planes, uint64_t plane_words, int R, int C, int row, int col,
+                     unsigned code, int B) {
+    const dpa_layout::BitPos bp = dpa_layout::bit_position(C, row, col);
+    for (int p = 0; p < B; ++p) {
+        if ((code >> (B - 1 - p)) & 1u)
+            mat_planes[static_cast<uint64_t>(p) * plane_words + bp.word] |= (1u << bp.bit);
+    }
+    (void)R;
+}
+
+struct EncodeJob {
+    const dpa_layer_desc* d;
+    dpa_sizes sz;
+    const float* wg; const float* wu; const float* wd;
+    uint8_t* planes; uint8_t* meta; double* rtable;
+    int e_begin;
+};
+
+// Uniform asymmetric codes of one matrix; accumulates (w - w_k)^2 into acc[k-1].
+bool encode_uniform_matrix(const Mat& m, int B, int G, uint32_t* mat_planes, uint16_t* mat_meta,
+                           double* acc) {
+    const double qmax = static_cast<double>((1 << B) - 1);
+    const int ng = m.C / G;
+    const uint64_t plane_words = static_cast<uint64_t>(m.R) * m.C / 32;
+    std::vector<double> s_row(ng), z_row(ng);
+    std::vector<unsigned> q_row(m.C);
+    for (int r = 0; r < m.R; ++r) {
+        const float* wr = m.w + static_cast<uint64_t>(r) * m.C;
+        for (int g = 0; g < ng; ++g) {
+            double lo = wr[g * G], hi = wr[g * G];
+            for (int j = 1; j < G; ++j) {
+                const double v = wr[g * G + j];
+                lo = v < lo ? v : lo;
+                hi = v > hi ? v : hi;
+            }
+            const double range = hi - lo;
+            const double s_raw = range / qmax;
+            uint16_t sb = f64_to_f16_bits(s_raw);
+            double s = f16_bits_to_f64(sb);
+            if (s == 0.0) { sb = 0x3C00u; s = 1.0; }
+            if (!std::isfinite(s)) return false;
+            double z = std::nearbyint(-lo / s);
+            z = z < 0.0 ? 0.0 : (z > qmax ? qmax : z);
+            s_row[g] = s;
+            z_row[g] = z;
+            mat_meta[(static_cast<uint64_t>(r) * ng + g) * 2 + 0] = sb;
+            mat_meta[(static_cast<uint64_t>(r) * ng + g) * 2 + 1] = f64_to_f16_bits(z);
+            for (int j = 0; j < G; ++j) {
+                const double v = wr[g * G + j];
+                double q = std::nearbyint(v / s) + z;
+                q = q < 0.0 ? 0.0 : (q > qmax ? qmax : q);
+                q_row[g * G + j] = static_cast<unsigned>(q);
+            }
+        }
+        for (int c = 0; c < m.C; ++c) {
+            set_code(mat_planes, plane_words, m.R, m.C, r, c, q_row[c], B);
+            const double w = wr[c];
+            const double s = s_row[c / G], z = z_row[c / G];
+            for (int k = 1; k <= B; ++k) {
+                const int dsh = B - k;
+                const double qk = static_cast<double>(q_row[c] >> dsh);
+                const double pw = static_cast<double>(1u << dsh);
+                const double qhat = qk * pw + (pw - 1.0) / 2.0;
+                const double what = s * (qhat - z);
+                const double diff = w - what;
+                acc[k - 1] = acc[k - 1] + diff * diff;
+            }
+        }
+    }
+    return true;
+}
+
+// Greedy binary-coded quantisation of one matrix; accumulates the residual per k.
+bool encode_bcq_matrix(const Mat& m, int B, int G, uint32_t* mat_planes, uint16_t* mat_meta,
+                       double* acc) {
+    const int ng = m.C / G;
+    const uint64_t plane_words = static_cast<uint64_t>(m.R) * m.C / 32;
+    const uint64_t meta_plane = static_cast<uint64_t>(m.R) * ng;
+    std::vector<double> res(G);
+    std::vector<double> alpha(static_cast<size_t>(B) * ng);
+    std::vector<unsigned> code(m.C);
+    for (int r = 0; r < m.R; ++r) {
+        const float* wr = m.w + static_cast<uint64_t>(r) * m.C;
+        for (int g = 0; g < ng; ++g) {
+            for (int j = 0; j < G; ++j) res[j] = wr[g * G + j];
+            for (int j = 0; j < G; ++j) code[g * G + j] = 0;
+            for (int i = 0; i < B; ++i) {
+                double total = 0.0;
+                for (int j = 0; j < G; ++j) total = total + std::fabs(res[j]);
+                const uint16_t ab = f64_to_f16_bits(total / static_cast<double>(G));
+                const double a = f16_bits_to_f64(ab);
+                if (!std::isfinite(a)) return false;
+                alpha[static_cast<size_t>(i) * ng + g] = a;
+                mat_meta[static_cast<uint64_t>(i) * meta_plane + static_cast<uint64_t>(r) * ng + g] = ab;
+                for (int j = 0; j < G; ++j) {
+                    const bool pos = res[j] >= 0.0;
+                    if (pos) code[g * G + j] |= 1u << (B - 1 - i);
+                    res[j] = res[j] - a * (pos ? 1.0 : -1.0);
+                }
+            }
+        }
+        for (int c = 0; c < m.C; ++c) {
+            set_code(mat_planes, plane_words, m.R, m.C, r, c, code[c], B);
+            const double w = wr[c];
+            for (int k = 1; k <= B; ++k) {
+                double what = 0.0;
+                for (int i = 0; i < k; ++i) {
+                    const bool pos = (code[c] >> (B - 1 - i)) & 1u;
+                    what = what + alpha[static_cast<size_t>(i) * ng + c / G] * (pos ? 1.0 : -1.0);
+                }
+                const double diff = w - what;
+                acc[k - 1] = acc[k - 1] + diff * diff;
+            }
+        }
+    }
+    return true;
+}
+
+bool encode_one_expert(const EncodeJob& job, int local_e) {
+    const dpa_layer_desc& d = *job.d;
+    const int e = job.e_begin + local_e;
+    const int H = d.hidden, I = d.inter, B = d.bits, G = d.group;
+    const uint64_t gate_off = static_cast<uint64_t>(local_e) * I * H;
+    const Mat mats[3] = {{job.wg + gate_off, I, H}, {job.wu + gate_off, I, H},
+                         {job.wd + static_cast<uint64_t>(local_e) * H * I, H, I}};
+    double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    uint8_t* ep = job.planes + static_cast<uint64_t>(e) * job.sz.planes_per_expert;
+    uint8_t* em = job.meta + static_cast<uint64_t>(e) * job.sz.meta_per_expert;
+    std::memset(ep, 0, job.sz.planes_per_expert);
+    for (int m = 0; m < 3; ++m) {
+        uint32_t* mp = reinterpret_cast<uint32_t*>(ep + job.sz.planes_matrix_offset[m]);
+        uint16_t* mm = reinterpret_cast<uint16_t*>(em + job.sz.meta_matrix_offset[m]);
+        const bool ok = d.format == DPA_FMT_UNIFORM ? encode_uniform_matrix(mats[m], B, G, mp, mm, acc)
+                                                    : encode_bcq_matrix(mats[m], B, G, mp, mm, acc);
+        if (!ok) return false;
+    }
+    for (int k = 0; k < B; ++k) job.rtable[static_cast<uint64_t>(e) * B + k] = acc[k];
+    return true;
+}
+
+}  // namespace
+
+extern "C" dpa_status dpa_encode(const dpa_layer_desc* desc, int e_begin, int n_e, const float* w_gate,
+                                 const float* w_up, const float* w_down, void* planes, void* meta,
+                                 double* rtable, int n_threads) {
+    dpa_sizes sz;
+    dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!w_gate || !w_up || !w_down || !planes || !meta || !rtable) return DPA_ERR_INVALID_ARG;
+    if (e_begin < 0 || n_e < 0 || e_begin + n_e > desc->n_experts) return DPA_ERR_INVALID_ARG;
+    if (n_e == 0) return DPA_OK;
+    EncodeJob job{desc, sz, w_gate, w_up, w_down, static_cast<uint8_t*>(planes),
+                  static_cast<uint8_t*>(meta), rtable, e_begin};
+    unsigned hw = std::thread::hardware_concurrency();
+    int nt = n_threads > 0 ? n_threads : static_cast<int>(hw ? hw : 1);
+    nt = std::min(nt, n_e);
+    std::atomic<int> next{0};
+    std::atomic<bool> ok{true};
+    auto worker = [&]() {
+        for (;;) {
+            const int i = next.fetch_add(1);
+            if (i >= n_e) break;
+            if (!encode_one_expert(job, i)) ok.store(false);
+        }
+    };
+    if (nt <= 1) {
+        worker();
+    } else {
+        std::vector<std::thread> th;
+        th.reserve(nt);
+        for (int t = 0; t < nt; ++t) th.emplace_back(worker);
+        for (auto& t : th) t.join();
+    }
+    return ok.load() ? DPA_OK : DPA_ERR_INVALID_ARG;
+}
+
+extern "C" dpa_status dpa_export_codes(const dpa_layer_desc* desc, const void* planes, int expert,
+                                       int matrix, uint8_t* codes) {
+    dpa_sizes sz;
+    dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!planes || !codes || expert < 0 || expert >= desc->n_experts || matrix < 0 || matrix > 2)
+        return DPA_ERR_INVALID_ARG;
+    const int R = matrix == DPA_MAT_DOWN ? desc->hidden : desc->inter;
+    const int C = matrix == DPA_MAT_DOWN ? desc->inter : desc->hidden;
+    const int B = desc->bits;
+    const uint32_t* mp = reinterpret_cast<const uint32_t*>(
+        static_cast<const uint8_t*>(planes) + static_cast<uint64_t>(expert) * sz.planes_per_expert +
+        sz.planes_matrix_offset[matrix]);
+    const uint64_t plane_words = static_cast<uint64_t>(R) * C / 32;
+    for (int r = 0; r < R; ++r) {
+        for (int c = 0; c < C; ++c) {
+            const dpa_layout::BitPos bp = dpa_layout::bit_position(C, r, c);
+            unsigned code = 0;
+            for (int p = 0; p < B; ++p)
+                code |= ((mp[static_cast<uint64_t>(p) * plane_words + bp.word] >> bp.bit) & 1u) << (B - 1 - p);
+            codes[static_cast<uint64_t>(r) * C + c] = static_cast<uint8_t>(code);
+        }
+    }
+    return DPA_OK;
+}
+
+extern "C" dpa_status dpa_export_meta(const dpa_layer_desc* desc, const void* meta, int expert, int matrix,
+                                      float* s_or_alpha, float* zero) {
+    dpa_sizes sz;
+    dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!meta || !s_or_alpha || expert < 0 || expert >= desc->n_experts || matrix < 0 || matrix > 2)
+        return DPA_ERR_INVALID_ARG;
+    const int R = matrix == DPA_MAT_DOWN ? desc->hidden : desc->inter;
+    const int C = matrix == DPA_MAT_DOWN ? desc->inter : desc->hidden;
+    const int ng = C / desc->group;
+    const uint16_t* mm = reinterpret_cast<const uint16_t*>(
+        static_cast<const uint8_t*>(meta) + static_cast<uint64_t>(expert) * sz.meta_per_expert +
+        sz.meta_matrix_offset[matrix]);
+    if (desc->format == DPA_FMT_UNIFORM) {
+        if (!zero) return DPA_ERR_INVALID_ARG;
+        for (uint64_t i = 0; i < static_cast<uint64_t>(R) * ng; ++i) {
+            s_or_alpha[i] = static_cast<float>(f16_bits_to_f64(mm[2 * i]));
+            zero[i] = static_cast<float>(f16_bits_to_f64(mm[2 * i + 1]));
+        }
+    } else {
+        for (uint64_t i = 0; i < static_cast<uint64_t>(desc->bits) * R * ng; ++i)
+            s_or_alpha[i] = static_cast<float>(f16_bits_to_f64(mm[i]));
+    }
+    return DPA_OK;
+}

@@ -1,0 +1,93 @@
+// Launch interfaces of the device kernels (internal to the library).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace dpa {
+
+struct RouteArgs {
+    const uint16_t* x;        // [T][H] bf16
+    const uint16_t* wr;       // [E][H] bf16
+    int T, E, H, K, G, norm_topk;
+    double* logits_user;      // [T][E] or nullptr
+    double* logits_ws;        // [T][E] workspace copy
+    int32_t* idx;             // [T][K]
+    double* gate;             // [T][K]
+    unsigned* counters;       // [T] zero between calls
+    int8_t* xdig;             // [T][3][H] or nullptr (digits not needed)
+    int32_t* xexp;            // [T][H/G]
+    int32_t* xsum;            // [T][H/G]
+    WsHeader* hdr;
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
+
+struct AllocArgs {
+    const double* rtable;     // [E][B]
+    const int32_t* idx;       // [T][K]
+    const double* gate;       // [T][K]
+    const double* target;     // device scalar
+    int T, K, E, B, kmin, kmax;
+    uint8_t* k_out;           // [T][K]
+    double* lambda_out;       // scalar or nullptr
+    double* cbuf;             // [P][nk] workspace
+    // permutation outputs (do_permute)
+    int do_permute;
+    int32_t* sorted_pair;     // [P] pair ids grouped by (expert, k)
+    int32_t* pair_pos;        // [P] position of each pair in sorted_pair
+    int32_t* seg_start;       // [E*nk + 1]
+    int32_t* exp_kmax;        // [E] (0 if no pair)
+    int32_t* active;          // [E] experts with pairs, ascending
+    uint8_t* k_copy;          // [P] internal copy of k (forward path)
+    WsHeader* hdr;
+};
+cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream);
+
+struct GemvArgs {
+    const uint8_t* planes;    // encoded layer
+    const uint8_t* meta;
+    uint64_t planes_per_expert, meta_per_expert;
+    uint64_t planes_mat_off[3], meta_mat_off[3];
+    int E, H, I, K, B, G, kmin, kmax, fmt;
+    const int32_t* sorted_pair;
+    const int32_t* seg_start;
+    const int32_t* exp_kmax;
+    const int32_t* active;
+    const int8_t* xdig;       // [T][3][H]
+    const int32_t* xexp;      // [T][H/G]
+    const int32_t* xsum;      // [T][H/G]
+    float* h;                 // [P][I] by sorted position
+    float* out_pair;          // [P][H] by sorted position
+    WsHeader* hdr;
+    int max_items;            // upper bound of work items (host-known)
+};
+cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms);
+size_t gateup_smem_bytes(const GemvArgs& a);   // dynamic shared memory of one CTA
+size_t down_smem_bytes(const GemvArgs& a);
+cudaError_t launch_down(const GemvArgs& a, cudaStream_t stream, int num_sms);
+
+struct CombineArgs {
+    const float* out_pair;    // [P][H] by sorted position
+    const int32_t* pair_pos;  // [P]
+    const double* gate;       // [T][K]
+    const float* shared_out;  // [T][H] or nullptr
+    float* pair_out_user;     // [T][K][H] diagnostic copy or nullptr
+    uint16_t* y;              // [T][H] bf16
+    int T, K, H;
+    WsHeader* hdr;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+struct SharedArgs {
+    const uint16_t* x;        // [T][H] bf16
+    const uint16_t* wg;       // [S][I][H]
+    const uint16_t* wu;
+    const uint16_t* wd;       // [S][H][I]
+    float* h;                 // [T][S][I] workspace
+    float* out;               // [T][H]
+    int T, S, H, I;
+};
+cudaError_t launch_shared(const SharedArgs& a, cudaStream_t stream);
+
+}  // namespace dpa

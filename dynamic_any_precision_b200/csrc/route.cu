@@ -1,0 +1,342 @@
+// Router: softmax top-k gating (DPA-MoE abstract: each token is routed to a small set of
+// experts; the gate scores then drive the plane allocation).
+//
+// The routing decision has to be reproducible bit for bit by any IEEE implementation, so:
+//  * the logit is the exact dot product of the bf16 token and the bf16 router row, rounded
+//    once to fp64. Products of two bf16 values are exact in fp64. A warp sums them in fp64 in
+//    any order and proves the sum exact (every product is a multiple of 2^L, L = lowest set
+//    bit of any operand pair, and sum|p| < 2^(L+52), so no partial sum can round). If the
+//    proof fails (operands spread over more than ~50 binades), the warp redoes the dot
+//    product in a 544-bit fixed-point accumulator and rounds that once.
+//  * exp is one fixed fp64 procedure (Cody & Waite reduction with ln 2 in two parts, degree-13
+//    Taylor polynomial in Horner form, scaling by 2^n), every step an explicitly rounded
+//    fp64 operation (this file is also compiled with --fmad=false).
+// The last block to finish a token (atomic ticket) selects its top-k and computes the gates,
+// and block 0 of each token writes the token's fixed-point digits for the expert GEMV.
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dpa {
+namespace {
+
+constexpr int kRouteWarps = 8;
+
+// ---------------- fp64 exp (see header comment) ----------------
+__device__ __forceinline__ double dexp_fixed(double x) {
+    const double INV_LN2 = 0x1.71547652b82fep+0;
+    const double LN2_HI = 0x1.62e42fefa3800p-1;
+    const double LN2_LO = 0x1.ef35793c76730p-45;
+    // 1/i!, i = 0..13, each rounded to nearest fp64
+    const double C[14] = {0x1.0000000000000p+0, 0x1.0000000000000p+0, 0x1.0000000000000p-1,
+                          0x1.5555555555555p-3, 0x1.5555555555555p-5, 0x1.1111111111111p-7,
+                          0x1.6c16c16c16c17p-10, 0x1.a01a01a01a01ap-13, 0x1.a01a01a01a01ap-16,
+                          0x1.71de3a556c734p-19, 0x1.27e4fb7789f5cp-22, 0x1.ae64567f544e4p-26,
+                          0x1.1eed8eff8d898p-29, 0x1.6124613a86d09p-33};
+    if (x < -708.0) return 0.0;
+    const double nf = rint(__dmul_rn(x, INV_LN2));   // ties to even
+    const int n = static_cast<int>(nf);
+    const double r = __dsub_rn(__dsub_rn(x, __dmul_rn(nf, LN2_HI)), __dmul_rn(nf, LN2_LO));
+    double p = C[13];
+#pragma unroll
+    for (int i = 12; i >= 0; --i) p = __dadd_rn(__dmul_rn(p, r), C[i]);
+    // p * 2^n is exact here: n >= -1021 and p in [0.7, 1.42], so the result is normal.
+    const double two_n = __longlong_as_double(static_cast<long long>(n + 1023) << 52);
+    return __dmul_rn(p, two_n);
+}
+
+// ---------------- bf16 decomposition ----------------
+struct Bf16Parts {
+    int mant;   // integer significand (0..255), 0 for +-0
+    int exp;    // value = mant * 2^exp
+    int sign;
+    bool finite;
+};
+
+__device__ __forceinline__ Bf16Parts bf16_parts(uint32_t u) {
+    Bf16Parts p;
+    const int E = (u >> 7) & 0xFF;
+    const int M = u & 0x7F;
+    p.sign = (u >> 15) & 1;
+    p.finite = E != 0xFF;
+    p.mant = E ? (M | 0x80) : M;
+    p.exp = (E ? E : 1) - 134;
+    return p;
+}
+
+// exponent of the lowest set bit of a nonzero bf16 value
+__device__ __forceinline__ int bf16_lsb(uint32_t u) {
+    const Bf16Parts p = bf16_parts(u);
+    return p.exp + (__ffs(p.mant) - 1);
+}
+
+// 2^k as a double, k in [-1022, 1023]
+__device__ __forceinline__ double pow2(int k) {
+    return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
+}
+
+// ---------------- exact fixed-point dot product (slow path) ----------------
+// Products are m * 2^f with m < 2^16 and f in [-266, 240]; bit b = f + 266 in [0, 506].
+constexpr int kLimbs = 17;   // 544 bits of 32-bit limbs held in int64 to absorb carries
+
+__device__ double exact_dot_fixed(const uint16_t* xs, const uint16_t* w, int H, int lane) {
+    long long limb[kLimbs];
+#pragma unroll
+    for (int i = 0; i < kLimbs; ++i) limb[i] = 0;
+    for (int j = lane; j < H; j += 32) {
+        const Bf16Parts a = bf16_parts(xs[j]);
+        const Bf16Parts b = bf16_parts(w[j]);
+        if (a.mant == 0 || b.mant == 0) continue;
+        const int bit = a.exp + b.exp + 266;
+        const long long v = static_cast<long long>(a.mant * b.mant) << (bit & 31);
+        const int L = bit >> 5;
+        if (a.sign ^ b.sign) limb[L] -= v; else limb[L] += v;
+    }
+#pragma unroll
+    for (int i = 0; i < kLimbs; ++i) {
+        long long v = limb[i];
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        limb[i] = v;
+    }
+    // every lane now holds the same limbs; normalise to a two's-complement 544-bit integer
+    uint32_t d[kLimbs];
+    long long carry = 0;
+    for (int i = 0; i < kLimbs; ++i) {
+        const long long v = limb[i] + carry;
+        d[i] = static_cast<uint32_t>(v & 0xffffffffll);
+        carry = v >> 32;   // arithmetic shift: floor division
+    }
+    const bool neg = carry < 0;
+    if (neg) {   // magnitude = -(value): invert and add one
+        uint64_t c = 1;
+        for (int i = 0; i < kLimbs; ++i) {
+            const uint64_t s = static_cast<uint64_t>(~d[i]) + c;
+            d[i] = static_cast<uint32_t>(s);
+            c = s >> 32;
+        }
+    }
+    int top = -1;
+    for (int i = kLimbs - 1; i >= 0; --i)
+        if (d[i]) { top = 32 * i + 31 - __clz(d[i]); break; }
+    if (top < 0) return 0.0;
+    auto bit_at = [&](int pos) -> uint32_t { return (d[pos >> 5] >> (pos & 31)) & 1u; };
+    double mag;
+    if (top <= 52) {
+        uint64_t m = static_cast<uint64_t>(d[0]) | (static_cast<uint64_t>(d[1]) << 32);
+        mag = __dmul_rn(static_cast<double>(m), pow2(-266));   // m < 2^53: exact
+    } else {
+        const int lo = top - 52;            // lowest kept bit
+        uint64_t m = 0;
+        for (int pos = top; pos >= lo; --pos) m = (m << 1) | bit_at(pos);
+        const uint32_t rbit = bit_at(lo - 1);
+        bool sticky = false;
+        for (int pos = lo - 2; pos >= 0 && !sticky; --pos) sticky = bit_at(pos) != 0;
+        int e = lo;
+        if (rbit && (sticky || (m & 1))) {
+            m += 1;
+            if (m >> 53) { m >>= 1; e += 1; }
+        }
+        mag = __dmul_rn(static_cast<double>(m), pow2(e - 266));
+    }
+    return neg ? -mag : mag;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+    for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_min_i(int v) {
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_max_f(float v) {
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);   // [H]
+    __shared__ int s_lsb_part[kRouteWarps];
+    __shared__ int s_last;
+    const int t = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.H, E = a.E;
+    const uint16_t* xrow = a.x + static_cast<size_t>(t) * H;
+
+    // stage the token, find the lowest set bit over its nonzero entries
+    int lsb_x = 1 << 20;
+    bool bad = false;
+    for (int j = threadIdx.x; j < H; j += blockDim.x) {
+        const uint16_t u = xrow[j];
+        xs[j] = u;
+        if (u & 0x7FFF) lsb_x = min(lsb_x, bf16_lsb(u));
+        bad |= ((u >> 7) & 0xFF) == 0xFF;
+    }
+    lsb_x = warp_min_i(lsb_x);
+    if (lane == 0) s_lsb_part[warp] = lsb_x;
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 1);
+    lsb_x = s_lsb_part[0];
+#pragma unroll
+    for (int w = 1; w < kRouteWarps; ++w) lsb_x = min(lsb_x, s_lsb_part[w]);
+
+    // ---- one warp per expert logit ----
+    const int e = blockIdx.x * kRouteWarps + warp;
+    if (e < E) {
+        const uint16_t* wrow = a.wr + static_cast<size_t>(e) * H;
+        double acc = 0.0, absacc = 0.0;
+        int lsb_w = 1 << 20;
+        bool wbad = false;
+        for (int j0 = lane * 8; j0 < H; j0 += 256) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(wrow + j0);
+            const uint4 xv = *reinterpret_cast<const uint4*>(xs + j0);
+            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+            const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t wu = (ww[q] >> (16 * h)) & 0xFFFFu;
+                    const uint32_t xu = (xx[q] >> (16 * h)) & 0xFFFFu;
+                    const double p = __dmul_rn(static_cast<double>(__uint_as_float(xu << 16)),
+                                               static_cast<double>(__uint_as_float(wu << 16)));
+                    acc = __dadd_rn(acc, p);
+                    absacc = __dadd_rn(absacc, fabs(p));
+                    if (wu & 0x7FFF) lsb_w = min(lsb_w, bf16_lsb(wu));
+                    wbad |= ((wu >> 7) & 0xFF) == 0xFF;
+                }
+            }
+        }
+        acc = warp_sum_f64(acc);
+        absacc = warp_sum_f64(absacc);
+        lsb_w = warp_min_i(lsb_w);
+        wbad = __any_sync(0xffffffffu, wbad);
+        double logit = acc;
+        if (absacc != 0.0) {
+            int ea;
+            frexp(absacc, &ea);              // absacc < 2^ea
+            if (ea > lsb_x + lsb_w + 52)     // exactness not proven: exact fixed-point path
+                logit = exact_dot_fixed(xs, wrow, H, lane);
+        }
+        if (lane == 0) {
+            double* dst = a.logits_user ? a.logits_user : a.logits_ws;
+            dst[static_cast<size_t>(t) * E + e] = logit;
+            if (wbad) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 2);
+        }
+    }
+
+    // ---- block 0 of the token: fixed-point digits of x for the expert GEMV ----
+    if (a.xdig != nullptr && blockIdx.x == 0) {
+        const int G = a.G, ng = H / G;
+        for (int g = warp; g < ng; g += kRouteWarps) {
+            float mx = 0.f;
+            for (int j = lane; j < G; j += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_float(xs[g * G + j])));
+            mx = warp_max_f(mx);
+            const int Eg = group_exponent(mx);
+            int sum = 0;
+            for (int j = lane; j < G; j += 32) {
+                const int X = to_fixed(bf16_bits_to_float(xs[g * G + j]), Eg);
+                sum += X;
+                int8_t d0, d1, d2;
+                split_digits(X, d0, d1, d2);
+                const size_t base = static_cast<size_t>(t) * 3 * H + g * G + j;
+                a.xdig[base] = d0;
+                a.xdig[base + H] = d1;
+                a.xdig[base + 2 * H] = d2;
+            }
+            sum = warp_sum_i(sum);
+            if (lane == 0) {
+                a.xexp[t * ng + g] = Eg;
+                a.xsum[t * ng + g] = sum;
+            }
+        }
+    }
+
+    // ---- last block of this token: top-k and gates ----
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const unsigned prev = atomicAdd(&a.counters[t], 1u);
+        s_last = prev == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!s_last) return;
+    if (threadIdx.x == 0) a.counters[t] = 0;   // ready for the next call
+    __threadfence();
+    if (warp != 0) return;
+
+    const double* lrow = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
+    double* vals = reinterpret_cast<double*>(smem_raw);   // reuse: [E] logits (x no longer needed)
+    for (int i = lane; i < E; i += 32) vals[i] = __ldcg(lrow + i);
+    __syncwarp();
+    const int K = a.K;
+    int my_e = -1;
+    double my_l = 0.0;
+    for (int r = 0; r < K; ++r) {
+        double bv = 0.0;
+        int be = -1;
+        for (int i = lane; i < E; i += 32) {
+            const double v = vals[i];
+            if (v != v) continue;   // NaN (already flagged as invalid input)
+            if (be < 0 || v > bv) { bv = v; be = i; }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            const bool take = oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be));
+            if (take) { bv = ov; be = oe; }
+        }
+        if (lane == r) { my_e = be; my_l = bv; }
+        if (be >= 0 && lane == (be & 31)) vals[be] = __longlong_as_double(0x7ff8000000000000ll);  // remove
+        __syncwarp();
+    }
+    const double lmax = __shfl_sync(0xffffffffu, my_l, 0);
+    double num = 0.0;
+    if (lane < K) num = dexp_fixed(__dsub_rn(my_l, lmax));
+    double den = 0.0;
+    if (a.norm_topk) {
+        for (int j = 0; j < K; ++j) den = __dadd_rn(den, __shfl_sync(0xffffffffu, num, j));
+    } else {
+        // softmax over every expert, summed in ascending expert id
+        double* ex = vals;
+        for (int i = lane; i < E; i += 32) ex[i] = dexp_fixed(__dsub_rn(__ldcg(lrow + i), lmax));
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < E; ++i) den = __dadd_rn(den, ex[i]);
+        den = __shfl_sync(0xffffffffu, den, 0);
+    }
+    if (lane < K) {
+        a.idx[t * K + lane] = my_e;
+        a.gate[t * K + lane] = __ddiv_rn(num, den);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
+    const int chunks = (a.E + kRouteWarps - 1) / kRouteWarps;
+    size_t smem = static_cast<size_t>(a.H) * 2;
+    const size_t need_vals = static_cast<size_t>(a.E) * 8;
+    if (need_vals > smem) smem = need_vals;
+    smem = (smem + 15) & ~static_cast<size_t>(15);
+    if (smem > 48 * 1024) {
+        cudaError_t err = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+    }
+    dim3 grid(chunks, a.T);
+    route_kernel<<<grid, kRouteWarps * 32, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+int route_chunks(int E) { return (E + kRouteWarps - 1) / kRouteWarps; }
+
+}  // namespace dpa

@@ -1,0 +1,220 @@
+/*
+ * dpa.h - C ABI of the B200 (sm_100a) routed MoE expert FFN over prefix-decodable
+ * bitplane weights.
+ *
+ * The method (pages cited by title and section):
+ *  - DPA-MoE: A Runtime Precision Control Framework for MoE Inference, Abstract:
+ *    expert FFN weights stored as prefix-decodable chunks with one shared scale
+ *    ("SharedScale AnyBCQ"), per-expert reconstruction residuals profiled offline,
+ *    chunks allocated after routing from the live router gate scores, so one encoded
+ *    layer runs at many weight budgets.
+ *  - DuoRate: Two-Rate Per-Expert Precision Allocation for MoE Serving, Abstract:
+ *    prefix-readable weight stream, baked distortion tensor, Lagrangian
+ *    rate-distortion allocation solved by a bisection; prefill reads at the stored rate.
+ *  - MatMoE: Matryoshka Mixture-of-Experts with Dynamic Mixed-Precision Quantization,
+ *    Abstract and review section "Core Contribution": bitplane storage,
+ *    floor-and-compensation (keep the top k of B code bits and add (2^(B-k)-1)/2),
+ *    routing-score driven per-expert bit-widths under a target average bit-width.
+ *
+ * Conventions for every call:
+ *  - Return value: DPA_OK or an error code; on error nothing has been launched and no
+ *    output has been written.
+ *  - "device" pointers are CUDA global memory owned by the caller; "host" pointers are
+ *    ordinary CPU memory owned by the caller. The library never allocates, frees or
+ *    keeps pointers between calls. Device calls are asynchronous on the given stream,
+ *    never synchronise (except dpa_device_status) and copy nothing back to the host, so
+ *    a sequence of them can be captured in a CUDA graph.
+ *  - Every device buffer must be 16-byte aligned (bulk copies), else DPA_ERR_INVALID_ARG.
+ *  - Errors found on the device (an out-of-range routed expert id passed to
+ *    dpa_allocate, a bounded wait that ran out) set a flag in the workspace; read and
+ *    clear it with dpa_device_status.
+ *  - Matrices are row-major. Token activations and router weights are bf16 bit patterns.
+ */
+#ifndef DPA_H
+#define DPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dpa_status {
+    DPA_OK = 0,
+    DPA_ERR_INVALID_ARG = 1,         /* bad pointer, size, alignment or descriptor field   */
+    DPA_ERR_UNSUPPORTED = 2,         /* shape outside what the kernels handle (see below)  */
+    DPA_ERR_WORKSPACE = 3,           /* workspace smaller than dpa_forward_workspace_size  */
+    DPA_ERR_CUDA = 4,                /* a CUDA runtime call failed                          */
+    DPA_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device wait ran out (reported by status) */
+    DPA_ERR_DEVICE_INVALID_INPUT = 6 /* device data out of range (reported by status)      */
+} dpa_status;
+
+enum { DPA_FMT_UNIFORM = 0, DPA_FMT_BCQ = 1 };
+enum { DPA_MAT_GATE = 0, DPA_MAT_UP = 1, DPA_MAT_DOWN = 2 };
+
+/* One MoE layer. gate/up are [inter][hidden], down is [hidden][inter] per expert.
+ *  format    DPA_FMT_UNIFORM: asymmetric B-bit codes, per-group fp16 scale s and zero z
+ *                             shared by every k; the first k planes read with
+ *                             floor-and-compensation: w = s*((q>>(B-k))*2^(B-k)
+ *                             + (2^(B-k)-1)/2 - z).
+ *            DPA_FMT_BCQ:     w = sum_{i<k} alpha_i * b_i, b_i in {-1,+1}, per-group fp16
+ *                             alpha_i (binary-coded quantisation, greedy fit).
+ *  bits      B, the stored planes (1..8).   kmin..kmax: planes a routed pair may read.
+ *  group     G, inputs per scale group.     norm_topk: 1 = softmax over the top_k
+ *            selected logits, 0 = softmax over all experts (then the top_k values).
+ *  n_shared  always-on experts run densely in bf16 (not allocated, not in the budget).
+ * Supported by the kernels: hidden, inter multiples of 64 and of group; group a multiple
+ * of 64; n_experts <= 1024; top_k <= 32; n_shared <= 8. */
+typedef struct dpa_layer_desc {
+    int32_t hidden, inter, n_experts, top_k, n_shared;
+    int32_t format, bits, kmin, kmax, group, norm_topk;
+} dpa_layer_desc;
+
+/* Bytes of one encoded layer (all routed experts).
+ *  planes: bit planes. For expert e and matrix m (rows R, cols C), plane p (p = 0 is the
+ *          most significant code bit, or the first BCQ sign plane) occupies R*C/8 bytes;
+ *          the B planes of (e, m) are stored one after another, so the first k planes of a
+ *          matrix are one contiguous prefix of its bytes. Matrices follow in the order
+ *          gate, up, down; experts follow in order.
+ *          Inside a plane the bits are in the decode kernel's fragment order: 16-row tiles,
+ *          then 64-column blocks, then 32 lanes of one 32-bit word. Lane l = 4*g + c holds
+ *          rows {g, g+8} and, for rho in 0..3 and m in 0..7, bit 4*m + rho is the weight at
+ *            row    = tile*16 + g + 8*(rho & 1)
+ *            column = block*64 + 32*(m & 1) + 16*(rho >> 1) + 4*c + (m >> 1).
+ *          Use dpa_export_codes to read codes back in natural order.
+ *  meta:   DPA_FMT_UNIFORM: per (e, m, row, group) an fp16 pair {s, z}, row-major,
+ *          [E][3][R][C/G] with the three matrices in order.
+ *          DPA_FMT_BCQ: per (e, m, plane, row, group) one fp16 alpha, [E][3][B][R][C/G]
+ *          (the first k planes' alphas are a contiguous prefix per (e, m)).
+ *  rtable: fp64 [E][B]; rtable[e][k-1] = ||W_e - W_e^(k)||_F^2 summed over gate, up, down.
+ *  *_matrix_offset: byte offset of matrix m of expert e is
+ *          e*planes_per_expert + planes_matrix_offset[m] (likewise for meta). */
+typedef struct dpa_sizes {
+    uint64_t planes_bytes, meta_bytes, rtable_bytes;
+    uint64_t planes_per_expert, meta_per_expert;
+    uint64_t planes_matrix_offset[3], meta_matrix_offset[3];
+} dpa_sizes;
+
+/* Device weights of one layer for dpa_moe_forward. planes/meta/rtable as written by
+ * dpa_encode and copied to the device unchanged. w_router: bf16 [n_experts][hidden].
+ * shared_*: bf16 dense always-on experts, gate/up [n_shared][inter][hidden],
+ * down [n_shared][hidden][inter]; NULL when n_shared == 0. */
+typedef struct dpa_layer_weights {
+    const void* planes;
+    const void* meta;
+    const double* rtable;
+    const void* w_router;
+    const void* shared_gate;
+    const void* shared_up;
+    const void* shared_down;
+} dpa_layer_weights;
+
+/* Optional device outputs of dpa_moe_forward's decision path (any field may be NULL).
+ * topk_idx int32 [T][top_k]; topk_gate fp64 [T][top_k]; k uint8 [T][top_k] (planes read
+ * by each routed pair); lambda fp64 scalar (the final Lagrange multiplier);
+ * pair_out fp32 [T][top_k][hidden]: each routed pair's expert output before the gate
+ * weighting (diagnostic; costs T*top_k*hidden*4 bytes of writes).
+ * events: optional cudaEvent_t handles (any may be NULL) recorded on the stream at the
+ * stage boundaries of dpa_moe_forward: [0] before routing, [1] after routing, [2] after
+ * allocation and grouping, [3] after the shared experts, [4] after the gate/up GEMV,
+ * [5] after the down GEMV, [6] after the combine. Recording also works under stream
+ * capture, so per-stage device times can be read from a replayed CUDA graph. */
+typedef struct dpa_aux {
+    int32_t* topk_idx;
+    double* topk_gate;
+    uint8_t* k;
+    double* lambda;
+    float* pair_out;
+    void* events[7];
+} dpa_aux;
+
+/* Validate a descriptor and return the encoded sizes. Host only. */
+dpa_status dpa_encoded_sizes(const dpa_layer_desc* desc, dpa_sizes* out);
+
+/* Offline encoder (host, synchronous, multithreaded with n_threads >= 1 or 0 = all cores).
+ * Encodes routed experts [e_begin, e_begin + n_e) of the layer.
+ * w_gate, w_up: host fp32 [n_e][inter][hidden]; w_down: host fp32 [n_e][hidden][inter]
+ * (the experts to encode, contiguous). planes, meta, rtable: host buffers sized for the
+ * WHOLE layer (dpa_encoded_sizes); only the parts of experts e_begin.. are written.
+ * Uniform codes per group of G inputs (DPA-MoE "SharedScale"; MatMoE shared quantisation
+ * parameters): lo/hi = group min/max, s = fp16((hi-lo)/(2^B-1)) (1 if it rounds to 0),
+ * z = clamp(rint(-lo/s), 0, 2^B-1), q = clamp(rint(w/s)+z, 0, 2^B-1), rint ties to even,
+ * fp64 arithmetic. BCQ per group: for each plane i, b_i = sign(R) (sign(0) = +1),
+ * alpha_i = fp16(sum|R|/G) (sequential sum), R -= alpha_i*b_i. rtable[e][k-1] is a
+ * sequential fp64 sum of (w - w_k)^2 over gate, up, down in row-major order.
+ * Errors: DPA_ERR_INVALID_ARG for NULL pointers, a range outside [0, n_experts), or a
+ * group whose scale does not fit fp16. */
+dpa_status dpa_encode(const dpa_layer_desc* desc, int e_begin, int n_e,
+                      const float* w_gate, const float* w_up, const float* w_down,
+                      void* planes, void* meta, double* rtable, int n_threads);
+
+/* Read codes of one encoded matrix back in natural order (host). codes: uint8 [R][C];
+ * code = sum_p plane_p << (B-1-p) over all B planes. */
+dpa_status dpa_export_codes(const dpa_layer_desc* desc, const void* planes, int expert,
+                            int matrix, uint8_t* codes);
+
+/* Read one matrix's scale data back as fp32 (host). Uniform: s_or_alpha [R][C/G] = s,
+ * zero [R][C/G] = z. BCQ: s_or_alpha [B][R][C/G] = alpha, zero unused (may be NULL). */
+dpa_status dpa_export_meta(const dpa_layer_desc* desc, const void* meta, int expert,
+                           int matrix, float* s_or_alpha, float* zero);
+
+/* Router (device): logits l[t][e] = the exact dot product of bf16 x[t] and bf16
+ * w_router[e], rounded once to fp64; top_k experts by descending logit (ties to the lower
+ * id); gates as described at dpa_layer_desc.norm_topk, using a fixed fp64 exp (Cody-Waite
+ * reduction with ln 2 in two parts, degree-13 Taylor polynomial, results below 2^-1021
+ * flushed to 0). Decisions are bit-identical to any IEEE implementation of the same steps.
+ * x: device bf16 [n_tokens][hidden]; w_router: device bf16 [n_experts][hidden];
+ * topk_idx: device int32 [n_tokens][top_k]; topk_gate: device fp64 [n_tokens][top_k];
+ * logits: optional device fp64 [n_tokens][n_experts] (NULL to skip).
+ * ws: device workspace of dpa_forward_workspace_size(desc, n_tokens) bytes. */
+dpa_status dpa_route(const dpa_layer_desc* desc, const void* x, int n_tokens,
+                     const void* w_router, int32_t* topk_idx, double* topk_gate,
+                     double* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* Plane allocation (device). For the P = n_tokens*top_k routed pairs (token-major, slot
+ * order) with expert e and gate g, and a multiplier lambda, each pair reads
+ *     k(lambda) = argmin_{kmin<=k<=kmax} fl(fl(g*rtable[e][k-1]) + fl(lambda*k))
+ * planes (ties to the smaller k). lambda comes from exactly 64 fp64 bisection steps on
+ * [0, 2*max_p fl(g_p*rtable[e_p][kmin-1]) + 1]: mid = 0.5*(lo+hi); if sum_p k_p(mid) >
+ * target*P then lo = mid else hi = mid; the result is lambda = hi and k = k(hi), so the
+ * mean planes per pair never exceeds the target (DuoRate Lagrangian bisection; MatMoE
+ * binary search to a target average bit-width).
+ * target_bpw: device fp64 scalar in [kmin, kmax] (a device value so one captured graph
+ * serves every budget; out of range -> k and lambda untouched, device flag
+ * DPA_ERR_DEVICE_INVALID_INPUT). k_out: device uint8 [n_tokens][top_k];
+ * lambda_out: device fp64 scalar (may be NULL). */
+dpa_status dpa_allocate(const dpa_layer_desc* desc, const double* rtable,
+                        const int32_t* topk_idx, const double* topk_gate, int n_tokens,
+                        const double* target_bpw, uint8_t* k_out, double* lambda_out,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes that dpa_route, dpa_allocate and dpa_moe_forward need for up to
+ * max_tokens tokens. Returns 0 for an invalid descriptor. */
+size_t dpa_forward_workspace_size(const dpa_layer_desc* desc, int max_tokens);
+
+/* One MoE layer forward (device): route, allocate, group pairs by expert and plane
+ * count, run each routed pair's SwiGLU expert reading only its first k planes
+ *   a = W_gate^(k) x, u = W_up^(k) x, h = silu(a) * u, o = W_down^(k) h,
+ * and write y[t] = bf16( sum_{slots} g * o  (+ dense shared experts) ).
+ * x: device bf16 [n_tokens][hidden]; y: device bf16 [n_tokens][hidden];
+ * target_bpw: device fp64 scalar (see dpa_allocate); aux: optional (may be NULL).
+ * ws must hold dpa_forward_workspace_size(desc, n_tokens) bytes and is clobbered. */
+dpa_status dpa_moe_forward(const dpa_layer_desc* desc, const dpa_layer_weights* weights,
+                           const void* x, int n_tokens, const double* target_bpw, void* y,
+                           dpa_aux* aux, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the device error flag in ws, clear it, and return it
+ * (DPA_OK if no device error was recorded). */
+dpa_status dpa_device_status(void* ws, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* dpa_status_string(dpa_status s);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int dpa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DPA_H */

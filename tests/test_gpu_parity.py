@@ -1,0 +1,263 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on the same seeded inputs.
+Routing indices, gates, plane counts and lambda must be bit-identical; outputs within
+|y - y_ref| <= 2e-3 * (1 + |y_ref|)."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+from dynamic_any_precision_b200 import dpa, workloads as W  # noqa: E402
+from oracle import dpa_oracle as O  # noqa: E402
+from oracle_jobs import pair_outputs, reference_layer  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+
+
+def within_tol(got, ref, tol=TOL):
+    err = np.abs(got - ref)
+    bound = tol * (1.0 + np.abs(ref))
+    return bool(np.all(err <= bound)), float(np.max(err / bound))
+
+
+def bits_to_f64(y_t):
+    return O.bf16_bits_to_f64(y_t.cpu().numpy().view(np.uint16))
+
+
+class GpuLayer:
+    """A layer encoded by the product encoder and resident on the GPU."""
+    _cache = {}
+
+    @classmethod
+    def get(cls, shape):
+        if shape.name not in cls._cache:
+            cls._cache[shape.name] = cls(shape)
+        return cls._cache[shape.name]
+
+    def __init__(self, shape):
+        self.shape = shape
+        self.desc = dpa.make_desc(shape)
+        g, u, d = W.all_expert_weights(shape)
+        planes, meta, r = dpa.encode(self.desc, g, u, d)
+        del g, u, d
+        self.wr = W.router_weights(shape)
+        sh = W.shared_weights_bf16(shape) if shape.n_shared else None
+        self.layer = dpa.DeviceLayer.from_host(self.desc, planes, meta, r, self.wr, sh)
+        self.planes_host = planes
+
+    def forward(self, x_bits, target, ws=None, with_pairs=True):
+        T = x_bits.shape[0]
+        K = self.shape.top_k
+        x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+        tg = torch.tensor([target], dtype=torch.float64, device="cuda")
+        ws = dpa.new_workspace(self.desc, T) if ws is None else ws
+        aux = {"topk_idx": torch.empty((T, K), dtype=torch.int32, device="cuda"),
+               "topk_gate": torch.empty((T, K), dtype=torch.float64, device="cuda"),
+               "k": torch.empty((T, K), dtype=torch.uint8, device="cuda"),
+               "lambda": torch.empty(1, dtype=torch.float64, device="cuda")}
+        if with_pairs:
+            aux["pair_out"] = torch.empty((T, K, self.shape.hidden), dtype=torch.float32, device="cuda")
+        y = dpa.moe_forward(self.layer, x, tg, ws, aux=aux)
+        st = dpa.device_status(ws)
+        assert st == 0, dpa.STATUS_NAMES.get(st, st)
+        out = {k: v.cpu().numpy() for k, v in aux.items()}
+        return bits_to_f64(y), out, ws
+
+
+def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None):
+    gl = GpuLayer.get(shape)
+    y, aux, _ = gl.forward(x_bits, target)
+    y_ref, ref = reference_layer(shape, x_bits, target, token_subset=token_subset)
+    assert np.array_equal(aux["topk_idx"], ref["idx"])
+    assert np.array_equal(aux["topk_gate"], ref["gates"])       # bit-identical fp64
+    assert np.array_equal(aux["k"].astype(np.int64), ref["k"])
+    assert aux["lambda"][0] == ref["lambda"]
+    rows = np.arange(x_bits.shape[0]) if token_subset is None else np.asarray(token_subset)
+    ok, worst = within_tol(y[rows], y_ref[rows])
+    assert ok, f"output tolerance exceeded: worst err/bound = {worst}"
+    if sample_pairs is not None:
+        ref_o = pair_outputs(shape, x_bits, ref, sample_pairs)
+        for (t, j), o in ref_o.items():
+            ok, worst = within_tol(aux["pair_out"][t, j].astype(np.float64), o, 1e-3)
+            assert ok, (t, j, worst)
+    # the achieved average never exceeds the target
+    assert aux["k"].astype(np.int64).sum() <= target * aux["k"].size
+    return y, aux, ref
+
+
+# ----------------------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("shape,T", [(W.TINY, 4), (W.QWEN3_B1, 1), (W.QWEN3_B64, 64), (W.DEEPSEEK_B16, 16),
+                                     (W.QWEN3_B1, 37), (W.TINY, 3)])
+def test_route_bit_exact(shape, T):
+    d = dpa.make_desc(shape)
+    wr = W.router_weights(shape)
+    x_bits = W.tokens(shape, T, step=11)
+    ws = dpa.new_workspace(d, T)
+    logits = torch.empty((T, shape.n_experts), dtype=torch.float64, device="cuda")
+    idx, gate = dpa.route(d, torch.from_numpy(x_bits.view(np.int16)).cuda(),
+                          torch.from_numpy(wr.view(np.int16)).cuda(), ws, logits=logits)
+    assert dpa.device_status(ws) == 0
+    ridx, rg, rl = O.route(x_bits, wr, shape.top_k, shape.norm_topk)
+    assert np.array_equal(logits.cpu().numpy(), rl)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.array_equal(gate.cpu().numpy(), rg)
+
+
+def test_route_exact_path_for_wide_exponent_spread():
+    # operands spread over ~200 binades, and large terms that cancel exactly, so the logit is
+    # decided by tiny terms: the fp64 fast path cannot prove exactness and the kernel must
+    # take the fixed-point path
+    shape = W.with_sizes(W.TINY, name="tiny_spread")
+    d = dpa.make_desc(shape)
+    rng = np.random.default_rng(5)
+    T, H, E = 4, shape.hidden, shape.n_experts
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    x[:, 0] = 2.0 ** 100
+    x[:, 1] = -(2.0 ** 100)
+    x[:, 2:10] *= np.float32(2.0 ** -100)
+    w = (rng.standard_normal((E, H)) * 0.02).astype(np.float32)
+    w[:, 1] = w[:, 0]
+    w[:, 10:20] *= np.float32(2.0 ** -60)
+    xb, wb = W.f32_to_bf16_bits(x), W.f32_to_bf16_bits(w)
+    ws = dpa.new_workspace(d, T)
+    logits = torch.empty((T, E), dtype=torch.float64, device="cuda")
+    idx, gate = dpa.route(d, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(wb.view(np.int16)).cuda(),
+                          ws, logits=logits)
+    assert dpa.device_status(ws) == 0
+    ridx, rg, rl = O.route(xb, wb, shape.top_k, shape.norm_topk)
+    assert np.array_equal(logits.cpu().numpy(), rl)
+    assert np.array_equal(idx.cpu().numpy(), ridx) and np.array_equal(gate.cpu().numpy(), rg)
+
+
+# ----------------------------------------------------------------------------- allocation
+
+def _alloc_inputs(seed, T, K, E, B, ties=False):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    g = -np.sort(-rng.dirichlet(np.ones(K), size=T), axis=1)
+    if ties:
+        g[:] = g[0]
+        idx[:] = idx[0]
+    base = rng.random(E) * 10 + 1
+    r = np.stack([base * 4.0 ** (B - k) * (1 + 0.3 * rng.random(E)) for k in range(1, B + 1)], axis=1)
+    return idx, g, r
+
+
+@pytest.mark.parametrize("T,K,E,kmin,kmax,B,target,ties", [
+    (4, 2, 8, 2, 4, 4, 3.0, False), (1, 8, 128, 2, 4, 4, 2.5, False), (64, 8, 128, 2, 4, 4, 2.0, False),
+    (64, 8, 128, 2, 4, 4, 3.5, False), (64, 8, 128, 2, 4, 4, 4.0, False), (16, 6, 64, 1, 3, 3, 2.0, False),
+    (2048, 8, 128, 2, 4, 4, 3.0, False), (7, 3, 16, 1, 4, 4, 2.75, False), (32, 8, 128, 2, 4, 4, 3.0, True)])
+def test_allocate_bit_exact(T, K, E, kmin, kmax, B, target, ties):
+    shape = W.with_sizes(W.QWEN3_B1, n_experts=E, top_k=K, kmin=kmin, kmax=kmax, bits=B, name="alloc")
+    d = dpa.make_desc(shape)
+    idx, g, r = _alloc_inputs(T * 1000 + E, T, K, E, B, ties)
+    rk, rlam = O.allocate(idx, g, r, kmin, kmax, target)
+    ws = dpa.new_workspace(d, T)
+    k, lam = dpa.allocate(d, torch.from_numpy(r).cuda(), torch.from_numpy(idx).cuda(), torch.from_numpy(g).cuda(),
+                          torch.tensor([target], dtype=torch.float64, device="cuda"), ws)
+    assert dpa.device_status(ws) == 0
+    assert np.array_equal(k.cpu().numpy().astype(np.int64), rk)
+    assert lam.item() == rlam
+
+
+def test_allocate_invalid_target_sets_device_flag():
+    shape = W.TINY
+    d = dpa.make_desc(shape)
+    idx, g, r = _alloc_inputs(1, 4, 2, 8, 4)
+    ws = dpa.new_workspace(d, 4)
+    k0 = torch.full((4, 2), 7, dtype=torch.uint8, device="cuda")
+    for bad in (1.5, 4.5, float("nan")):
+        st = dpa.lib().dpa_allocate(dpa.ctypes.byref(d), torch.from_numpy(r).cuda().data_ptr(),
+                                    torch.from_numpy(idx).cuda().data_ptr(), torch.from_numpy(g).cuda().data_ptr(), 4,
+                                    torch.tensor([bad], dtype=torch.float64, device="cuda").data_ptr(), k0.data_ptr(),
+                                    None, ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        assert dpa.device_status(ws) == 6
+        assert torch.all(k0 == 7)          # outputs untouched
+    assert dpa.device_status(ws) == 0      # flag cleared
+
+
+# ----------------------------------------------------------------------------- full layer
+
+def test_forward_tiny():
+    x = W.tokens(W.TINY)
+    check_forward(W.TINY, x, 3.0, sample_pairs=[(t, j) for t in range(4) for j in range(2)])
+
+
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_forward_tiny_ragged_and_targets(T):
+    x = W.tokens(W.TINY, T, step=T)
+    for target in (2.0, 2.5, 4.0):
+        check_forward(W.TINY, x, target)
+
+
+def test_forward_qwen3_batch1():
+    x = W.tokens(W.QWEN3_B1)
+    check_forward(W.QWEN3_B1, x, 2.5, sample_pairs=[(0, j) for j in range(8)])
+
+
+@pytest.mark.parametrize("target", [2.0, 3.0, 4.0])
+def test_forward_qwen3_batch64_sampled(target):
+    x = W.tokens(W.QWEN3_B64)
+    check_forward(W.QWEN3_B64, x, target, token_subset=[0, 5, 31, 63],
+                  sample_pairs=[(5, 0), (31, 7), (63, 3)])
+
+
+def test_forward_deepseek_bcq_shared():
+    x = W.tokens(W.DEEPSEEK_B16)
+    check_forward(W.DEEPSEEK_B16, x, 2.0, token_subset=[0, 7, 15], sample_pairs=[(0, 0), (15, 5)])
+
+
+def test_prefix_property_poisoned_planes():
+    # at target = kmin every pair reads kmin planes: overwriting planes >= kmin of every
+    # expert in device memory must not change a single output bit
+    shape = W.TINY
+    gl = GpuLayer.get(shape)
+    x = W.tokens(shape, 4, step=3)
+    y0, aux0, _ = gl.forward(x, float(shape.kmin))
+    assert np.all(aux0["k"] == shape.kmin)
+    s = dpa.encoded_sizes(gl.desc)
+    saved = gl.layer.planes.clone()
+    try:
+        p = gl.layer.planes
+        for e in range(shape.n_experts):
+            for m in range(3):
+                R = shape.hidden if m == 2 else shape.inter
+                C = shape.inter if m == 2 else shape.hidden
+                pb = R * C // 8
+                start = e * s.planes_per_expert + s.planes_matrix_offset[m]
+                p[start + shape.kmin * pb: start + shape.bits * pb] = 0xA5
+        torch.cuda.synchronize()
+        y1, aux1, _ = gl.forward(x, float(shape.kmin))
+        assert np.array_equal(y0, y1)
+    finally:
+        gl.layer.planes.copy_(saved)
+
+
+def test_forward_deterministic_and_graph_capture():
+    shape = W.TINY
+    gl = GpuLayer.get(shape)
+    x_bits = W.tokens(shape, 4, step=9)
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda()
+    tg = torch.tensor([3.0], dtype=torch.float64, device="cuda")
+    ws = dpa.new_workspace(gl.desc, 4)
+    y_eager = dpa.moe_forward(gl.layer, x, tg, ws).clone()
+    y_again = dpa.moe_forward(gl.layer, x, tg, ws).clone()
+    assert torch.equal(y_eager, y_again)
+    y_buf = torch.empty_like(y_eager)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        dpa.moe_forward(gl.layer, x, tg, ws, y=y_buf, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        dpa.moe_forward(gl.layer, x, tg, ws, y=y_buf)
+    for target in (3.0, 2.0, 4.0):
+        tg.fill_(target)
+        graph.replay()
+        torch.cuda.synchronize()
+        y_ref = dpa.moe_forward(gl.layer, x, tg, ws).clone()
+        assert torch.equal(y_buf, y_ref)
+    assert dpa.device_status(ws) == 0
