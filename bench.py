@@ -10,7 +10,8 @@ gate/up GEMV with SwiGLU, the down GEMV and the gate-weighted combine - one dpa_
 Inputs are resident in HBM when the timed region starts. The layer is encoded once and copied
 `--copies` times in device memory; step i uses copy i % copies and its own tokens, so no weight
 byte is re-read within copies-1 steps and the L2 cache (126 MB) cannot serve the planes.
-The K timed steps are one CUDA graph; per-stage CUDA events inside it give the kernel times.
+The K timed steps are one CUDA graph without instrumentation; a second graph of the same K
+steps with CUDA events at the stage boundaries gives the per-kernel device times.
 
 N > 1 GPUs run independent replicas (no collective on the data path; the path shards by
 token batch), one process per GPU under torchrun; the time is the max over ranks.
@@ -43,7 +44,7 @@ FALLBACK_HBM_GBS = 6650.0
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2048)
+    ap.add_argument("--steps", type=int, default=1024)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", choices=("dpa", "reference"), default="dpa")
     ap.add_argument("--workload", default=W.QWEN3_B1.name)
@@ -172,7 +173,7 @@ def run_dpa(args, shape, target, rank, world, dist):
                                       base.w_router.clone(), base.shared))
     n_total = args.warmup + args.steps
     # distinct tokens per step (and per rank)
-    xs = np.stack([W.tokens(shape, T, step=1000 * rank + i) for i in range(n_total)])
+    xs = np.stack([W.tokens(shape, T, step=1_000_000 * rank + i) for i in range(n_total)])
     x_dev = torch.from_numpy(xs.view(np.int16)).to(dev)
     y_dev = torch.empty((n_total, T, shape.hidden), dtype=torch.int16, device=dev)
     tg = torch.tensor([target], dtype=torch.float64, device=dev)
@@ -181,6 +182,9 @@ def run_dpa(args, shape, target, rank, world, dist):
     gate_all = torch.empty((args.steps, T, K), dtype=torch.float64, device=dev)
     k_all = torch.empty((args.steps, T, K), dtype=torch.uint8, device=dev)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for row in events:          # torch creates events lazily: record once so the handles exist
+        for ev in row:
+            ev.record()
 
     def step(i, timed_j=None):
         aux = None
@@ -197,12 +201,17 @@ def run_dpa(args, shape, target, rank, world, dist):
 
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
-    g_warm, g_timed = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    g_warm, g_timed, g_stages = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     with torch.cuda.stream(s):
         with torch.cuda.graph(g_warm, stream=s):
             for i in range(args.warmup):
                 step(i)
+        # the timed region: K steps, no instrumentation inside
         with torch.cuda.graph(g_timed, stream=s):
+            for j in range(args.steps):
+                step(args.warmup + j)
+        # the same K steps again with stage events, for per-kernel device times
+        with torch.cuda.graph(g_stages, stream=s):
             for j in range(args.steps):
                 step(args.warmup + j, timed_j=j)
     torch.cuda.synchronize()
@@ -229,7 +238,10 @@ def run_dpa(args, shape, target, rank, world, dist):
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         ms = float(tt.item())
 
-    # per-stage kernel times inside the timed region
+    # per-stage kernel times: the same steps replayed once more with stage events
+    g_stages.replay()
+    torch.cuda.synchronize()
+    assert dpa.device_status(ws) == 0
     names = ["route", "allocate", "shared", "gateup", "down", "combine"]
     stage_ms = {n: 0.0 for n in names}
     for j in range(args.steps):
@@ -280,6 +292,21 @@ def run_dpa(args, shape, target, rank, world, dist):
 
 # ----------------------------------------------------------------------------- CPU oracle
 
+def _oracle_encode_job(shape, e):
+    from oracle import dpa_oracle as O
+    g, u, d = W.expert_weights(shape, e)
+    return e, O.encode_expert(g, u, d, shape.fmt, shape.bits, shape.group)
+
+
+def _encode_pool(shape, experts):
+    """Oracle encode of the given experts in a spawned process pool (setup work)."""
+    import multiprocessing as mp
+    from concurrent.futures import ProcessPoolExecutor
+    n = max(1, min(32, (os.cpu_count() or 2) - 1, len(experts)))
+    with ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn")) as ex:
+        return dict(ex.map(_oracle_encode_job, [shape] * len(experts), experts))
+
+
 def oracle_sample(shape, target, n_tokens, seed_base=0):
     """Times the fp64 oracle (as it stands) on `n_tokens` single-token steps of the workload.
     Each step routes and allocates the token in full; of its top_k expert FFNs one (round
@@ -289,14 +316,10 @@ def oracle_sample(shape, target, n_tokens, seed_base=0):
     from oracle import dpa_oracle as O
     wr = W.router_weights(shape)
     xs = [W.tokens(shape, shape.tokens, step=seed_base + i) for i in range(n_tokens)]
+    routes = [O.route(x, wr, shape.top_k, shape.norm_topk) for x in xs]
+    need = sorted({int(e) for rt in routes for e in np.unique(rt[0])})
+    experts = _encode_pool(shape, need)          # offline setup, not timed
     with threadpool_limits(1):
-        routes = [O.route(x, wr, shape.top_k, shape.norm_topk) for x in xs]
-        need = sorted({int(routes[i][0][0, i % shape.top_k]) for i in range(n_tokens)}
-                      | {int(e) for rt in routes for e in np.unique(rt[0])})
-        experts = {}
-        for e in need:
-            g, u, d = W.expert_weights(shape, e)
-            experts[e] = O.encode_expert(g, u, d, shape.fmt, shape.bits, shape.group)
         r = np.full((shape.n_experts, shape.bits), np.nan)
         for e, enc in experts.items():
             r[e] = enc["r"]

@@ -20,16 +20,32 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     float4 acc = a.shared_out ? *reinterpret_cast<const float4*>(a.shared_out + static_cast<size_t>(t) * a.H + n)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < a.K; ++s) {
-        const int p = t * a.K + s;
-        const int pos = a.pair_pos[p];
-        const float g = static_cast<float>(a.gate[p]);
-        const float4 o = *reinterpret_cast<const float4*>(a.out_pair + static_cast<size_t>(pos) * a.H + n);
-        r.x = fmaf(g, o.x, r.x);
-        r.y = fmaf(g, o.y, r.y);
-        r.z = fmaf(g, o.z, r.z);
-        r.w = fmaf(g, o.w, r.w);
-        if (a.pair_out_user) *reinterpret_cast<float4*>(a.pair_out_user + static_cast<size_t>(p) * a.H + n) = o;
+    // slots in chunks of 8: all loads of a chunk are issued before the in-order accumulation
+    for (int s0 = 0; s0 < a.K; s0 += 8) {
+        int pos[8];
+        float g[8];
+        float4 o[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (s0 + u < a.K) {
+                pos[u] = a.pair_pos[t * a.K + s0 + u];
+                g[u] = static_cast<float>(a.gate[t * a.K + s0 + u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (s0 + u < a.K) o[u] = *reinterpret_cast<const float4*>(a.out_pair + static_cast<size_t>(pos[u]) * a.H + n);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            if (s0 + u < a.K) {
+                r.x = fmaf(g[u], o[u].x, r.x);
+                r.y = fmaf(g[u], o[u].y, r.y);
+                r.z = fmaf(g[u], o[u].z, r.z);
+                r.w = fmaf(g[u], o[u].w, r.w);
+                if (a.pair_out_user)
+                    *reinterpret_cast<float4*>(a.pair_out_user + static_cast<size_t>(t * a.K + s0 + u) * a.H + n) = o[u];
+            }
+        }
     }
     acc.x += r.x;
     acc.y += r.y;

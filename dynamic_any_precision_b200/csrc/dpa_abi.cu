@@ -40,8 +40,8 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 
 // ---- workspace layout ----
 struct WsLayout {
-    size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, sorted, pairpos, seg, kmaxe, active, xdig, xexp,
-        xsum, h, out_pair, sh_h, sh_out, total;
+    size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
+        desc, tiles, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -65,11 +65,7 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.k = take(P);
     L.lambda = take(8);
     L.cbuf = take(8 * P * nk);
-    L.sorted = take(4 * P);
     L.pairpos = take(4 * P);
-    L.seg = take(4 * (E * nk + 1));
-    L.kmaxe = take(4 * E);
-    L.active = take(4 * E);
     L.xdig = take(3 * static_cast<size_t>(T) * H);
     L.xexp = take(4 * static_cast<size_t>(T) * (H / d->group));
     L.xsum = take(4 * static_cast<size_t>(T) * (H / d->group));
@@ -77,6 +73,8 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.out_pair = take(4 * P * H);
     L.sh_h = take(4 * static_cast<size_t>(T) * d->n_shared * I);
     L.sh_out = take(4 * static_cast<size_t>(T) * H);
+    L.desc = take(16 * E);
+    L.tiles = take(16 * (P + E * nk));
     L.total = off;
     return L;
 }
@@ -201,12 +199,9 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.lambda_out = lambda_out;
     a.cbuf = at<double>(ws, L.cbuf);
     a.do_permute = permute ? 1 : 0;
-    a.sorted_pair = at<int32_t>(ws, L.sorted);
     a.pair_pos = at<int32_t>(ws, L.pairpos);
-    a.seg_start = at<int32_t>(ws, L.seg);
-    a.exp_kmax = at<int32_t>(ws, L.kmaxe);
-    a.active = at<int32_t>(ws, L.active);
-    a.k_copy = nullptr;
+    a.exp_desc = at<int4>(ws, L.desc);
+    a.tiles = at<int4>(ws, L.tiles);
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
     return dpa::launch_allocate(a, s) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
 }
@@ -255,8 +250,15 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     double* lam = (aux && aux->lambda) ? aux->lambda : at<double>(ws, L.lambda);
     dpa::WsHeader* hdr = at<dpa::WsHeader>(ws, L.hdr);
 
+    // stage events: under stream capture they must be external event-record nodes so that the
+    // replayed graph records them
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (aux) cudaStreamIsCapturing(s, &cap);
     auto mark = [&](int i) {
-        if (aux && aux->events[i]) cudaEventRecord(static_cast<cudaEvent_t>(aux->events[i]), s);
+        if (!aux || !aux->events[i]) return;
+        cudaEvent_t ev = static_cast<cudaEvent_t>(aux->events[i]);
+        if (cap == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+        else cudaEventRecord(ev, s);
     };
     mark(0);
     // 1. route (+ fixed-point digits of x)
@@ -322,10 +324,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     ga.kmin = d->kmin;
     ga.kmax = d->kmax;
     ga.fmt = d->format;
-    ga.sorted_pair = at<int32_t>(ws, L.sorted);
-    ga.seg_start = at<int32_t>(ws, L.seg);
-    ga.exp_kmax = at<int32_t>(ws, L.kmaxe);
-    ga.active = at<int32_t>(ws, L.active);
+    ga.exp_desc = at<int4>(ws, L.desc);
+    ga.tiles = at<int4>(ws, L.tiles);
     ga.xdig = at<int8_t>(ws, L.xdig);
     ga.xexp = at<int32_t>(ws, L.xexp);
     ga.xsum = at<int32_t>(ws, L.xsum);
@@ -334,6 +334,7 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     ga.hdr = hdr;
     const int P = T * K;
     ga.max_items = P < d->n_experts ? P : d->n_experts;
+    ga.max_tokens_per_expert = T;
     const int sms = num_sms_current();
     if (dpa::launch_gateup(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(4);

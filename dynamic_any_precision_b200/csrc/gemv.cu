@@ -11,7 +11,8 @@
 // sum of x over the plane's +1 bits.
 //
 // Work items are (active expert, row tile). A CTA stages the item's first kmax_e planes and
-// scales into shared memory with bulk copies (one mbarrier, bounded wait), then each warp:
+// scales into shared memory with bulk copies (one mbarrier, bounded wait) and the
+// activations' fixed-point digits with vector loads, then each warp:
 //   - gathers bit rho of every nibble of the plane words into a register of eight 4-bit
 //     codes (the plane layout puts each lane's MMA fragment in one 32-bit word per plane);
 //   - masks the register into two u8 A operands (even nibbles, and odd nibbles times 16);
@@ -21,7 +22,7 @@
 //   - per scale group, combines the digits, applies 2^(E-22), the group scale and the
 //     compensation term in fp32.
 // Tokens of one expert are grouped by their plane count k; a tile of two tokens shares k, and
-// tiles are processed in ascending k so the codes are built incrementally.
+// tiles come in ascending k so the codes are built incrementally.
 #include <cstdint>
 
 #include "common.cuh"
@@ -30,40 +31,9 @@
 namespace dpa {
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int NT = 4;   // n8 column tiles (two tokens each) per pass
-
-struct TileInfo {
-    int k;
-    int posA, posB;   // sorted pair positions (posB = -1: empty second slot)
-};
-
-__device__ __forceinline__ int expert_tiles(const int32_t* seg, int e, int nk) {
-    int n = 0;
-    for (int kc = 0; kc < nk; ++kc) n += (seg[e * nk + kc + 1] - seg[e * nk + kc] + 1) >> 1;
-    return n;
-}
-
-__device__ __forceinline__ TileInfo tile_info(const int32_t* seg, int e, int nk, int kmin, int tile) {
-    int acc = 0;
-    for (int kc = 0; kc < nk; ++kc) {
-        const int s = seg[e * nk + kc];
-        const int n = seg[e * nk + kc + 1] - s;
-        const int nt = (n + 1) >> 1;
-        if (tile < acc + nt) {
-            const int i = tile - acc;
-            TileInfo ti;
-            ti.k = kmin + kc;
-            ti.posA = s + 2 * i;
-            ti.posB = (2 * i + 1 < n) ? s + 2 * i + 1 : -1;
-            return ti;
-        }
-        acc += nt;
-    }
-    TileInfo ti{0, -1, -1};
-    return ti;
-}
+constexpr int kDigPad = 16;   // bytes added to each digit row in shared memory (bank spread)
 
 // bits at nibble position rho of plane word w, moved to nibble bit t, masked
 template <int RHO, int T>
@@ -72,6 +42,42 @@ __device__ __forceinline__ uint32_t nib_bits(uint32_t w) {
     if constexpr (T >= RHO) v = w << (T - RHO);
     else v = w >> (RHO - T);
     return v & (0x11111111u << T);
+}
+
+// OR the bits of plane word w (code bit t) into the four nibble registers
+template <int T>
+__device__ __forceinline__ void add_plane(uint32_t (&R)[4], uint32_t w) {
+    R[0] |= nib_bits<0, T>(w);
+    R[1] |= nib_bits<1, T>(w);
+    R[2] |= nib_bits<2, T>(w);
+    R[3] |= nib_bits<3, T>(w);
+}
+
+// OR planes [FROM, TO) (plane p at pl[p * ps]) into the nibble registers; code bit = B-1-p
+template <int B, int FROM, int TO>
+__device__ __forceinline__ void add_range(uint32_t (&R)[4], const uint32_t* pl, int ps) {
+    if constexpr (FROM < TO && FROM < B) {
+        add_plane<B - 1 - FROM>(R, pl[FROM * ps]);
+        add_range<B, FROM + 1, TO>(R, pl, ps);
+    }
+}
+
+// planes [from, to) with a warp-uniform jump: only the planes a tile reads are loaded and merged
+template <int B>
+__device__ __forceinline__ void add_planes(uint32_t (&R)[4], const uint32_t* pl, int ps, int from, int to) {
+    switch (from * 5 + to) {
+        case 1: add_range<B, 0, 1>(R, pl, ps); break;
+        case 2: add_range<B, 0, 2>(R, pl, ps); break;
+        case 3: add_range<B, 0, 3>(R, pl, ps); break;
+        case 4: add_range<B, 0, 4>(R, pl, ps); break;
+        case 7: add_range<B, 1, 2>(R, pl, ps); break;
+        case 8: add_range<B, 1, 3>(R, pl, ps); break;
+        case 9: add_range<B, 1, 4>(R, pl, ps); break;
+        case 13: add_range<B, 2, 3>(R, pl, ps); break;
+        case 14: add_range<B, 2, 4>(R, pl, ps); break;
+        case 19: add_range<B, 3, 4>(R, pl, ps); break;
+        default: break;
+    }
 }
 
 // fp32 value of the digits a lane holds for one output row: columns 2tq, 2tq+1 of the C
@@ -84,32 +90,82 @@ __device__ __forceinline__ float digit_value(int lo0, int hi0, int lo1, int hi1,
 
 __device__ __forceinline__ float pow2f(int k) { return __int_as_float((k + 127) << 23); }
 
-struct SmemSched {
-    int nt;          // tiles in this pass
-    TileInfo ti[NT];
-    int tokA[NT], tokB[NT];
+__device__ __forceinline__ int tile_tok(const int4& t, int half) {
+    const int v = half ? (t.w >> 16) & 0xFFFF : t.w & 0xFFFF;
+    return v == 0xFFFF ? -1 : v;
+}
+
+__device__ __forceinline__ void load_b(const int8_t* row, int b, int tq, uint32_t& b0L, uint32_t& b1L,
+                                       uint32_t& b0H, uint32_t& b1H) {
+    const int8_t* src = row + 64 * b + 4 * tq;
+    b0L = *reinterpret_cast<const uint32_t*>(src);
+    b1L = *reinterpret_cast<const uint32_t*>(src + 16);
+    b0H = *reinterpret_cast<const uint32_t*>(src + 32);
+    b1H = *reinterpret_cast<const uint32_t*>(src + 48);
+}
+
+struct Layout {
+    // byte offsets inside dynamic shared memory
+    size_t planes, meta, dig, xe, xs, red, total;
+    int dig_stride;   // bytes per digit row
 };
+
+__host__ __device__ inline size_t align16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
+
+// gate/up: planes [2][B][nblk][32], meta, digits [2NT][3][H+pad], exps/sums [2NT][ng], red
+__host__ __device__ inline Layout gateup_layout(int H, int G, int B, int fmt, int NT) {
+    Layout L;
+    const int nblk = H / 64, ng = H / G;
+    L.planes = 0;
+    L.meta = align16(static_cast<size_t>(2) * B * nblk * 128);
+    const size_t meta_bytes = fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(2) * 16 * ng * 4
+                                                     : static_cast<size_t>(2) * B * 16 * ng * 2;
+    L.dig = align16(L.meta + meta_bytes);
+    L.dig_stride = H + kDigPad;
+    L.xe = align16(L.dig + static_cast<size_t>(2 * NT) * 3 * L.dig_stride);
+    L.xs = align16(L.xe + static_cast<size_t>(2 * NT) * ng * 4);
+    L.red = align16(L.xs + static_cast<size_t>(2 * NT) * ng * 4);
+    L.total = align16(L.red + static_cast<size_t>(kWarps) * NT * 2 * 2 * 16 * 4);
+    return L;
+}
+
+// down: planes [B][4][nblk][32], meta, digits [2NT][3][I+pad], exps/sums [2NT][ng]
+__host__ __device__ inline Layout down_layout(int I, int G, int B, int fmt, int NT) {
+    Layout L;
+    const int nblk = I / 64, ng = I / G;
+    L.planes = 0;
+    L.meta = align16(static_cast<size_t>(B) * 4 * nblk * 128);
+    const size_t meta_bytes = fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(64) * ng * 4
+                                                     : static_cast<size_t>(B) * 64 * ng * 2;
+    L.dig = align16(L.meta + meta_bytes);
+    L.dig_stride = I + kDigPad;
+    L.xe = align16(L.dig + static_cast<size_t>(2 * NT) * 3 * L.dig_stride);
+    L.xs = align16(L.xe + static_cast<size_t>(2 * NT) * ng * 4);
+    L.red = align16(L.xs + static_cast<size_t>(2 * NT) * ng * 4);
+    L.total = align16(L.red + static_cast<size_t>(2) * 4 * NT * 2 * 16 * 4);
+    return L;
+}
 
 // ---------------------------------------------------------------------------------------
 // gate + up projections, SwiGLU epilogue -> h[pos][I]
 // ---------------------------------------------------------------------------------------
-template <int FMT, int B>
+template <int FMT, int B, int NT>
 __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int H = a.H, I = a.I, G = a.G;
     const int nblk = H >> 6, ng = H / G, bpg = G >> 6;
-    const int nk = a.kmax - a.kmin + 1;
     const int tiles_per_expert = I >> 4;
-    // shared memory carve-up
-    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem);                       // [2][B][nblk][32]
-    const size_t planes_bytes = static_cast<size_t>(2) * B * nblk * 128;
-    unsigned char* s_meta = smem + planes_bytes;                                   // see below
-    const size_t meta_bytes = FMT == DPA_FMT_UNIFORM ? static_cast<size_t>(2) * 16 * ng * 4
-                                                     : static_cast<size_t>(2) * B * 16 * ng * 2;
-    float* s_red = reinterpret_cast<float*>(s_meta + ((meta_bytes + 15) & ~size_t(15)));   // [4][NT][2][2][16]
+    const Layout Ly = gateup_layout(H, G, B, FMT, NT);
+    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + Ly.planes);
+    unsigned char* s_meta = smem + Ly.meta;
+    int8_t* s_dig = reinterpret_cast<int8_t*>(smem + Ly.dig);
+    int* s_xe = reinterpret_cast<int*>(smem + Ly.xe);
+    int* s_xs = reinterpret_cast<int*>(smem + Ly.xs);
+    float* s_red = reinterpret_cast<float*>(smem + Ly.red);
     __shared__ uint64_t s_bar;
     __shared__ int s_flag;
-    __shared__ SmemSched s_sched;
+    __shared__ int4 s_tile[NT];
+    __shared__ int s_nt;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tq = lane & 3;
@@ -120,13 +176,14 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
     }
     __syncthreads();
     uint32_t phase = 0;
-    // this warp's scale groups
-    const int g0 = (warp * ng) / kWarps, g1 = ((warp + 1) * ng) / kWarps;
+    const int g0 = (warp * ng) / kWarps, g1 = ((warp + 1) * ng) / kWarps;   // this warp's groups
+    const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
+    const int dstride = Ly.dig_stride;
 
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int e = a.active[item / tiles_per_expert];
+        const int4 desc = a.exp_desc[item / tiles_per_expert];
+        const int e = desc.x, kmax_e = desc.y, ntiles = desc.z, toff = desc.w;
         const int rt = item % tiles_per_expert;
-        const int kmax_e = a.exp_kmax[e];
         if (threadIdx.x == 0) {
             fence_proxy_async();   // earlier generic reads of these buffers precede the copies
             const uint32_t pbytes = static_cast<uint32_t>(nblk) * 128;
@@ -150,39 +207,54 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                 }
             }
         }
-        const int ntiles = expert_tiles(a.seg_start, e, nk);
-        const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 100, &s_flag);
-        phase ^= 1;
-        if (!ok) return;
-
+        bool waited = false;
         for (int pass0 = 0; pass0 < ntiles; pass0 += NT) {
             if (threadIdx.x < NT) {
                 const int i = threadIdx.x;
-                if (pass0 + i < ntiles) {
-                    const TileInfo ti = tile_info(a.seg_start, e, nk, a.kmin, pass0 + i);
-                    s_sched.ti[i] = ti;
-                    s_sched.tokA[i] = a.sorted_pair[ti.posA] / a.K;
-                    s_sched.tokB[i] = ti.posB >= 0 ? a.sorted_pair[ti.posB] / a.K : -1;
-                }
-                if (i == 0) s_sched.nt = min(NT, ntiles - pass0);
+                s_tile[i] = pass0 + i < ntiles ? a.tiles[toff + pass0 + i] : make_int4(0, -1, -1, -1);
             }
+            if (threadIdx.x == 0) s_nt = min(NT, ntiles - pass0);
             __syncthreads();
-            const int nt = s_sched.nt;
+            const int nt = s_nt;
+            // stage the digits, exponents and sums of the pass's tokens
+            {
+                const int chunks = (3 * H) >> 4;
+                for (int i = threadIdx.x; i < 2 * NT * chunks; i += kThreads) {
+                    const int slot = i / chunks, c = i - slot * chunks;
+                    const int tok = tile_tok(s_tile[slot >> 1], slot & 1);
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (tok >= 0) v = *reinterpret_cast<const uint4*>(a.xdig + static_cast<size_t>(tok) * 3 * H + 16 * c);
+                    const int d_ = (16 * c) / H, col = 16 * c - d_ * H;
+                    *reinterpret_cast<uint4*>(s_dig + (slot * 3 + d_) * dstride + col) = v;
+                }
+                for (int i = threadIdx.x; i < 2 * NT * ng; i += kThreads) {
+                    const int slot = i / ng, g = i - slot * ng;
+                    const int tok = tile_tok(s_tile[slot >> 1], slot & 1);
+                    s_xe[i] = tok >= 0 ? a.xexp[tok * ng + g] : 0;
+                    s_xs[i] = tok >= 0 ? a.xsum[tok * ng + g] : 0;
+                }
+            }
+            if (!waited) {
+                waited = true;
+                const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 100, &s_flag);
+                phase ^= 1;
+                if (!ok) return;
+            } else {
+                __syncthreads();
+            }
+
             float acc[NT][2][2];
 #pragma unroll
             for (int i = 0; i < NT; ++i)
 #pragma unroll
                 for (int m = 0; m < 2; ++m) acc[i][m][0] = acc[i][m][1] = 0.f;
-            // B-operand source rows for this lane (column n = gid: token half, digit)
-            const int dig = gid & 3;
-            const int half = gid >> 2;
-            const int8_t* xrow[NT];
+            const int8_t* brow[NT];
 #pragma unroll
             for (int i = 0; i < NT; ++i) {
-                const int tok = half ? s_sched.tokB[i] : s_sched.tokA[i];
-                xrow[i] = (i < nt && dig < 3 && tok >= 0) ? a.xdig + (static_cast<size_t>(tok) * 3 + dig) * H : nullptr;
+                const int slot = 2 * i + half;
+                brow[i] = (i < nt && dig < 3 && tile_tok(s_tile[i], half) >= 0) ? s_dig + (slot * 3 + dig) * dstride
+                                                                                  : nullptr;
             }
-            const int my_tok_half = tq >> 1;   // C columns 2tq,2tq+1 belong to token A (tq<2) or B
             for (int g = g0; g < g1; ++g) {
                 if constexpr (FMT == DPA_FMT_UNIFORM) {
                     int C[NT][2][2][4];
@@ -196,40 +268,19 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                                 for (int r = 0; r < 4; ++r) C[i][m][h][r] = 0;
                     for (int jb = 0; jb < bpg; ++jb) {
                         const int b = g * bpg + jb;
-                        uint32_t w[2][B];
-#pragma unroll
-                        for (int m = 0; m < 2; ++m)
-#pragma unroll
-                            for (int p = 0; p < B; ++p)
-                                w[m][p] = p < kmax_e ? s_planes[(static_cast<size_t>(m * B + p) * nblk + b) * 32 + lane] : 0u;
+                        const uint32_t* pg = s_planes + static_cast<size_t>(b) * 32 + lane;   // gate, plane 0
+                        const uint32_t* pu = pg + static_cast<size_t>(B) * nblk * 32;         // up, plane 0
+                        const int ps = nblk * 32;                                             // plane stride
                         uint32_t R[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
                         int cur = 0;
                         uint32_t Alo[2][4], Ahi[2][4];
 #pragma unroll
                         for (int i = 0; i < NT; ++i) {
                             if (i < nt) {
-                                const int ki = s_sched.ti[i].k;
+                                const int ki = s_tile[i].x;
                                 if (ki > cur) {
-#pragma unroll
-                                    for (int p = 0; p < B; ++p) {
-                                        if (p >= cur && p < ki) {
-#pragma unroll
-                                            for (int m = 0; m < 2; ++m) {
-                                                const uint32_t wv = w[m][p];
-                                                // code bit t = B-1-p
-                                                switch (B - 1 - p) {
-                                                    case 0: R[m][0] |= nib_bits<0, 0>(wv); R[m][1] |= nib_bits<1, 0>(wv);
-                                                            R[m][2] |= nib_bits<2, 0>(wv); R[m][3] |= nib_bits<3, 0>(wv); break;
-                                                    case 1: R[m][0] |= nib_bits<0, 1>(wv); R[m][1] |= nib_bits<1, 1>(wv);
-                                                            R[m][2] |= nib_bits<2, 1>(wv); R[m][3] |= nib_bits<3, 1>(wv); break;
-                                                    case 2: R[m][0] |= nib_bits<0, 2>(wv); R[m][1] |= nib_bits<1, 2>(wv);
-                                                            R[m][2] |= nib_bits<2, 2>(wv); R[m][3] |= nib_bits<3, 2>(wv); break;
-                                                    default: R[m][0] |= nib_bits<0, 3>(wv); R[m][1] |= nib_bits<1, 3>(wv);
-                                                            R[m][2] |= nib_bits<2, 3>(wv); R[m][3] |= nib_bits<3, 3>(wv); break;
-                                                }
-                                            }
-                                        }
-                                    }
+                                    add_planes<B>(R[0], pg, ps, cur, ki);
+                                    add_planes<B>(R[1], pu, ps, cur, ki);
                                     cur = ki;
 #pragma unroll
                                     for (int m = 0; m < 2; ++m)
@@ -240,13 +291,7 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                                         }
                                 }
                                 uint32_t b0L = 0, b1L = 0, b0H = 0, b1H = 0;
-                                if (xrow[i]) {
-                                    const int8_t* src = xrow[i] + 64 * b + 4 * tq;
-                                    b0L = __ldg(reinterpret_cast<const uint32_t*>(src));
-                                    b1L = __ldg(reinterpret_cast<const uint32_t*>(src + 16));
-                                    b0H = __ldg(reinterpret_cast<const uint32_t*>(src + 32));
-                                    b1H = __ldg(reinterpret_cast<const uint32_t*>(src + 48));
-                                }
+                                if (brow[i]) load_b(brow[i], b, tq, b0L, b1L, b0H, b1H);
 #pragma unroll
                                 for (int m = 0; m < 2; ++m) {
                                     mma_u8s8(C[i][m][0], Alo[m][0], Alo[m][1], Alo[m][2], Alo[m][3], b0L, b1L);
@@ -255,16 +300,14 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                             }
                         }
                     }
-                    // epilogue for group g
                     const uint32_t* meta_u = reinterpret_cast<const uint32_t*>(s_meta);
 #pragma unroll
                     for (int i = 0; i < NT; ++i) {
                         if (i < nt) {
-                            const int tok = my_tok_half ? s_sched.tokB[i] : s_sched.tokA[i];
-                            const int ki = s_sched.ti[i].k;
+                            const int slot = 2 * i + my_half;
+                            const int ki = s_tile[i].x;
                             const float ck = 0.5f * static_cast<float>((1 << (B - ki)) - 1);
-                            int Eg = 0, SX = 0;
-                            if (tok >= 0) { Eg = __ldg(a.xexp + tok * ng + g); SX = __ldg(a.xsum + tok * ng + g); }
+                            const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
                             const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                             for (int m = 0; m < 2; ++m) {
@@ -302,25 +345,19 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                                 uint32_t Alo[2][4], Ahi[2][4];
 #pragma unroll
                                 for (int m = 0; m < 2; ++m) {
-                                    const uint32_t wv = s_planes[(static_cast<size_t>(m * B + p) * nblk + b) * 32 + lane];
-                                    const uint32_t r0 = nib_bits<0, 0>(wv), r1 = nib_bits<1, 0>(wv);
-                                    const uint32_t r2 = nib_bits<2, 0>(wv), r3 = nib_bits<3, 0>(wv);
-                                    Alo[m][0] = r0 & 0x0F0F0F0Fu; Ahi[m][0] = r0 & 0xF0F0F0F0u;
-                                    Alo[m][1] = r1 & 0x0F0F0F0Fu; Ahi[m][1] = r1 & 0xF0F0F0F0u;
-                                    Alo[m][2] = r2 & 0x0F0F0F0Fu; Ahi[m][2] = r2 & 0xF0F0F0F0u;
-                                    Alo[m][3] = r3 & 0x0F0F0F0Fu; Ahi[m][3] = r3 & 0xF0F0F0F0u;
+                                    uint32_t R[4] = {0u, 0u, 0u, 0u};
+                                    add_plane<0>(R, s_planes[(static_cast<size_t>(m * B + p) * nblk + b) * 32 + lane]);
+#pragma unroll
+                                    for (int r = 0; r < 4; ++r) {
+                                        Alo[m][r] = R[r] & 0x0F0F0F0Fu;
+                                        Ahi[m][r] = R[r] & 0xF0F0F0F0u;
+                                    }
                                 }
 #pragma unroll
                                 for (int i = 0; i < NT; ++i) {
-                                    if (i < nt && s_sched.ti[i].k > p) {
+                                    if (i < nt && s_tile[i].x > p) {
                                         uint32_t b0L = 0, b1L = 0, b0H = 0, b1H = 0;
-                                        if (xrow[i]) {
-                                            const int8_t* src = xrow[i] + 64 * b + 4 * tq;
-                                            b0L = __ldg(reinterpret_cast<const uint32_t*>(src));
-                                            b1L = __ldg(reinterpret_cast<const uint32_t*>(src + 16));
-                                            b0H = __ldg(reinterpret_cast<const uint32_t*>(src + 32));
-                                            b1H = __ldg(reinterpret_cast<const uint32_t*>(src + 48));
-                                        }
+                                        if (brow[i]) load_b(brow[i], b, tq, b0L, b1L, b0H, b1H);
 #pragma unroll
                                         for (int m = 0; m < 2; ++m) {
                                             mma_u8s8(C[i][m][0], Alo[m][0], Alo[m][1], Alo[m][2], Alo[m][3], b0L, b1L);
@@ -331,10 +368,9 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                             }
 #pragma unroll
                             for (int i = 0; i < NT; ++i) {
-                                if (i < nt && s_sched.ti[i].k > p) {
-                                    const int tok = my_tok_half ? s_sched.tokB[i] : s_sched.tokA[i];
-                                    int Eg = 0, SX = 0;
-                                    if (tok >= 0) { Eg = __ldg(a.xexp + tok * ng + g); SX = __ldg(a.xsum + tok * ng + g); }
+                                if (i < nt && s_tile[i].x > p) {
+                                    const int slot = 2 * i + my_half;
+                                    const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
                                     const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                                     for (int m = 0; m < 2; ++m) {
@@ -362,13 +398,13 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                     for (int m = 0; m < 2; ++m)
 #pragma unroll
                         for (int rr = 0; rr < 2; ++rr)
-                            s_red[((((warp * NT + i) * 2 + m) * 2 + my_tok_half) * 16) + gid + 8 * rr] = acc[i][m][rr];
+                            s_red[((((warp * NT + i) * 2 + m) * 2 + my_half) * 16) + gid + 8 * rr] = acc[i][m][rr];
             }
             __syncthreads();
-            {
-                const int i = threadIdx.x >> 5, tk = (threadIdx.x >> 4) & 1, row = threadIdx.x & 15;
+            for (int q = threadIdx.x; q < NT * 32; q += kThreads) {
+                const int i = q >> 5, tk = (q >> 4) & 1, row = q & 15;
                 if (i < nt) {
-                    const int pos = tk ? s_sched.ti[i].posB : s_sched.ti[i].posA;
+                    const int pos = tk ? s_tile[i].z : s_tile[i].y;
                     if (pos >= 0) {
                         float ag = 0.f, au = 0.f;
 #pragma unroll
@@ -376,12 +412,16 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                             ag += s_red[((((w * NT + i) * 2 + 0) * 2 + tk) * 16) + row];
                             au += s_red[((((w * NT + i) * 2 + 1) * 2 + tk) * 16) + row];
                         }
-                        const float hval = ag / (1.f + expf(-ag)) * au;
-                        a.h[static_cast<size_t>(pos) * I + rt * 16 + row] = hval;
+                        a.h[static_cast<size_t>(pos) * I + rt * 16 + row] = ag / (1.f + expf(-ag)) * au;
                     }
                 }
             }
             __syncthreads();
+        }
+        if (!waited) {   // no tiles (cannot happen for an active expert): keep the phase in step
+            const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 102, &s_flag);
+            phase ^= 1;
+            if (!ok) return;
         }
     }
 }
@@ -389,25 +429,23 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
 // ---------------------------------------------------------------------------------------
 // down projection: out_pair[pos][H] = W_down^(k) h[pos]
 // ---------------------------------------------------------------------------------------
-template <int FMT, int B>
+template <int FMT, int B, int NT>
 __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int H = a.H, I = a.I, G = a.G;
     const int nblk = I >> 6, ng = I / G, bpg = G >> 6;
-    const int nk = a.kmax - a.kmin + 1;
-    const int tiles_per_expert = H >> 6;   // 64-row items
-    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem);                   // [B][4][nblk][32]
-    const size_t planes_bytes = static_cast<size_t>(B) * 4 * nblk * 128;
-    unsigned char* s_meta = smem + planes_bytes;
-    const size_t meta_bytes = FMT == DPA_FMT_UNIFORM ? static_cast<size_t>(64) * ng * 4
-                                                     : static_cast<size_t>(B) * 64 * ng * 2;
-    int8_t* s_dig = reinterpret_cast<int8_t*>(s_meta + ((meta_bytes + 15) & ~size_t(15)));   // [2NT][3][I]
-    int* s_exp = reinterpret_cast<int*>(s_dig + static_cast<size_t>(2 * NT) * 3 * I);          // [2NT][ng]
-    int* s_sum = s_exp + 2 * NT * ng;
+    const int tiles_per_expert = H >> 6;   // 64-row items: 4 row tiles x 2 K halves = 8 warps
+    const Layout Ly = down_layout(I, G, B, FMT, NT);
+    uint32_t* s_planes = reinterpret_cast<uint32_t*>(smem + Ly.planes);
+    unsigned char* s_meta = smem + Ly.meta;
+    int8_t* s_dig = reinterpret_cast<int8_t*>(smem + Ly.dig);
+    int* s_xe = reinterpret_cast<int*>(smem + Ly.xe);
+    int* s_xs = reinterpret_cast<int*>(smem + Ly.xs);
+    float* s_red = reinterpret_cast<float*>(smem + Ly.red);   // [2 halves][4 tiles][NT][2][16]
     __shared__ uint64_t s_bar;
     __shared__ int s_flag;
-    __shared__ SmemSched s_sched;
-    __shared__ int s_pos[2 * NT];
+    __shared__ int4 s_tile[NT];
+    __shared__ int s_nt;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tq = lane & 3;
@@ -418,11 +456,13 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
     }
     __syncthreads();
     uint32_t phase = 0;
+    const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
+    const int dstride = Ly.dig_stride;
 
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int e = a.active[item / tiles_per_expert];
+        const int4 desc = a.exp_desc[item / tiles_per_expert];
+        const int e = desc.x, kmax_e = desc.y, ntiles = desc.z, toff = desc.w;
         const int rt = item % tiles_per_expert;
-        const int kmax_e = a.exp_kmax[e];
         if (threadIdx.x == 0) {
             fence_proxy_async();
             const uint32_t pbytes = 4u * nblk * 128;
@@ -443,29 +483,20 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                     bulk_g2s(s_meta + p * mbytes, mb + p * mplane + static_cast<uint64_t>(rt) * mbytes, mbytes, &s_bar);
             }
         }
-        const int ntiles = expert_tiles(a.seg_start, e, nk);
-        bool copied = false;
-
+        bool waited = false;
         for (int pass0 = 0; pass0 < ntiles; pass0 += NT) {
             if (threadIdx.x < NT) {
                 const int i = threadIdx.x;
-                if (pass0 + i < ntiles) {
-                    const TileInfo ti = tile_info(a.seg_start, e, nk, a.kmin, pass0 + i);
-                    s_sched.ti[i] = ti;
-                    s_pos[2 * i] = ti.posA;
-                    s_pos[2 * i + 1] = ti.posB;
-                } else {
-                    s_pos[2 * i] = -1;
-                    s_pos[2 * i + 1] = -1;
-                }
-                if (i == 0) s_sched.nt = min(NT, ntiles - pass0);
+                s_tile[i] = pass0 + i < ntiles ? a.tiles[toff + pass0 + i] : make_int4(0, -1, -1, -1);
             }
+            if (threadIdx.x == 0) s_nt = min(NT, ntiles - pass0);
             __syncthreads();
-            const int nt = s_sched.nt;
+            const int nt = s_nt;
             // fixed-point digits of the pass's h rows: one warp per (slot, group)
             for (int task = warp; task < 2 * NT * ng; task += kWarps) {
-                const int slot = task / ng, g = task % ng;
-                const int pos = s_pos[slot];
+                const int slot = task / ng, g = task - slot * ng;
+                const int4 t = s_tile[slot >> 1];
+                const int pos = (slot & 1) ? t.z : t.y;
                 if (pos < 0) continue;
                 const float* hrow = a.h + static_cast<size_t>(pos) * I + g * G;
                 float mx = 0.f;
@@ -478,35 +509,38 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                     sum += X;
                     int8_t d0, d1, d2;
                     split_digits(X, d0, d1, d2);
-                    int8_t* dst = s_dig + static_cast<size_t>(slot) * 3 * I + g * G + j;
+                    int8_t* dst = s_dig + (slot * 3) * dstride + g * G + j;
                     dst[0] = d0;
-                    dst[I] = d1;
-                    dst[2 * I] = d2;
+                    dst[dstride] = d1;
+                    dst[2 * dstride] = d2;
                 }
                 for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                if (lane == 0) { s_exp[slot * ng + g] = Eg; s_sum[slot * ng + g] = sum; }
+                if (lane == 0) { s_xe[slot * ng + g] = Eg; s_xs[slot * ng + g] = sum; }
             }
-            if (!copied) {
+            if (!waited) {
+                waited = true;
                 const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 200, &s_flag);
                 phase ^= 1;
-                copied = true;
                 if (!ok) return;
+            } else {
+                __syncthreads();
             }
-            __syncthreads();
 
             float acc[NT][2];
 #pragma unroll
             for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = 0.f;
-            const int dig = gid & 3, half = gid >> 2;
-            const int8_t* xrow[NT];
+            const int8_t* brow[NT];
 #pragma unroll
             for (int i = 0; i < NT; ++i) {
                 const int slot = 2 * i + half;
-                xrow[i] = (i < nt && dig < 3 && s_pos[slot] >= 0) ? s_dig + (static_cast<size_t>(slot) * 3 + dig) * I : nullptr;
+                const int4 t = s_tile[i];
+                const int pos = half ? t.z : t.y;
+                brow[i] = (i < nt && dig < 3 && pos >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
             }
-            const int my_half = tq >> 1;
-            const uint32_t* wplanes = s_planes + static_cast<size_t>(warp) * nblk * 32;   // tile `warp` of 4
-            for (int g = 0; g < ng; ++g) {
+            const int rtile = warp & 3, khalf = warp >> 2;   // row tile of 4, half of the groups
+            const uint32_t* wplanes = s_planes + static_cast<size_t>(rtile) * nblk * 32;
+            const int gbeg = (khalf * ng) / 2, gend = ((khalf + 1) * ng) / 2;
+            for (int g = gbeg; g < gend; ++g) {
                 if constexpr (FMT == DPA_FMT_UNIFORM) {
                     int C[NT][2][4];
 #pragma unroll
@@ -517,34 +551,17 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                             for (int r = 0; r < 4; ++r) C[i][h][r] = 0;
                     for (int jb = 0; jb < bpg; ++jb) {
                         const int b = g * bpg + jb;
-                        uint32_t w[B];
-#pragma unroll
-                        for (int p = 0; p < B; ++p)
-                            w[p] = p < kmax_e ? wplanes[(static_cast<size_t>(p) * 4 * nblk + b) * 32 + lane] : 0u;
+                        const uint32_t* pw = wplanes + static_cast<size_t>(b) * 32 + lane;   // plane 0
+                        const int ps = 4 * nblk * 32;                                        // plane stride
                         uint32_t R[4] = {0u, 0u, 0u, 0u};
                         int cur = 0;
                         uint32_t Alo[4], Ahi[4];
 #pragma unroll
                         for (int i = 0; i < NT; ++i) {
                             if (i < nt) {
-                                const int ki = s_sched.ti[i].k;
+                                const int ki = s_tile[i].x;
                                 if (ki > cur) {
-#pragma unroll
-                                    for (int p = 0; p < B; ++p) {
-                                        if (p >= cur && p < ki) {
-                                            const uint32_t wv = w[p];
-                                            switch (B - 1 - p) {
-                                                case 0: R[0] |= nib_bits<0, 0>(wv); R[1] |= nib_bits<1, 0>(wv);
-                                                        R[2] |= nib_bits<2, 0>(wv); R[3] |= nib_bits<3, 0>(wv); break;
-                                                case 1: R[0] |= nib_bits<0, 1>(wv); R[1] |= nib_bits<1, 1>(wv);
-                                                        R[2] |= nib_bits<2, 1>(wv); R[3] |= nib_bits<3, 1>(wv); break;
-                                                case 2: R[0] |= nib_bits<0, 2>(wv); R[1] |= nib_bits<1, 2>(wv);
-                                                        R[2] |= nib_bits<2, 2>(wv); R[3] |= nib_bits<3, 2>(wv); break;
-                                                default: R[0] |= nib_bits<0, 3>(wv); R[1] |= nib_bits<1, 3>(wv);
-                                                        R[2] |= nib_bits<2, 3>(wv); R[3] |= nib_bits<3, 3>(wv); break;
-                                            }
-                                        }
-                                    }
+                                    add_planes<B>(R, pw, ps, cur, ki);
                                     cur = ki;
 #pragma unroll
                                     for (int r = 0; r < 4; ++r) {
@@ -553,13 +570,7 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                                     }
                                 }
                                 uint32_t b0L = 0, b1L = 0, b0H = 0, b1H = 0;
-                                if (xrow[i]) {
-                                    const int8_t* src = xrow[i] + 64 * b + 4 * tq;
-                                    b0L = *reinterpret_cast<const uint32_t*>(src);
-                                    b1L = *reinterpret_cast<const uint32_t*>(src + 16);
-                                    b0H = *reinterpret_cast<const uint32_t*>(src + 32);
-                                    b1H = *reinterpret_cast<const uint32_t*>(src + 48);
-                                }
+                                if (brow[i]) load_b(brow[i], b, tq, b0L, b1L, b0H, b1H);
                                 mma_u8s8(C[i][0], Alo[0], Alo[1], Alo[2], Alo[3], b0L, b1L);
                                 mma_u8s8(C[i][1], Ahi[0], Ahi[1], Ahi[2], Ahi[3], b0H, b1H);
                             }
@@ -570,15 +581,15 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                     for (int i = 0; i < NT; ++i) {
                         if (i < nt) {
                             const int slot = 2 * i + my_half;
-                            const int ki = s_sched.ti[i].k;
+                            const int ki = s_tile[i].x;
                             const float ck = 0.5f * static_cast<float>((1 << (B - ki)) - 1);
-                            const int Eg = s_exp[slot * ng + g], SX = s_sum[slot * ng + g];
+                            const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
                             const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                             for (int rr = 0; rr < 2; ++rr) {
                                 float v = digit_value(C[i][0][2 * rr], C[i][1][2 * rr], C[i][0][2 * rr + 1], C[i][1][2 * rr + 1], tq);
                                 v += __shfl_xor_sync(0xffffffffu, v, 1);
-                                const int row = warp * 16 + gid + 8 * rr;
+                                const int row = rtile * 16 + gid + 8 * rr;
                                 const uint32_t sz = meta_u[row * ng + g];
                                 const float s = __half2float(__ushort_as_half(static_cast<unsigned short>(sz & 0xFFFF)));
                                 const float z = __half2float(__ushort_as_half(static_cast<unsigned short>(sz >> 16)));
@@ -600,22 +611,19 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                                     for (int r = 0; r < 4; ++r) C[i][h][r] = 0;
                             for (int jb = 0; jb < bpg; ++jb) {
                                 const int b = g * bpg + jb;
-                                const uint32_t wv = wplanes[(static_cast<size_t>(p) * 4 * nblk + b) * 32 + lane];
-                                const uint32_t r0 = nib_bits<0, 0>(wv), r1 = nib_bits<1, 0>(wv);
-                                const uint32_t r2 = nib_bits<2, 0>(wv), r3 = nib_bits<3, 0>(wv);
-                                const uint32_t Alo[4] = {r0 & 0x0F0F0F0Fu, r1 & 0x0F0F0F0Fu, r2 & 0x0F0F0F0Fu, r3 & 0x0F0F0F0Fu};
-                                const uint32_t Ahi[4] = {r0 & 0xF0F0F0F0u, r1 & 0xF0F0F0F0u, r2 & 0xF0F0F0F0u, r3 & 0xF0F0F0F0u};
+                                uint32_t R[4] = {0u, 0u, 0u, 0u};
+                                add_plane<0>(R, wplanes[(static_cast<size_t>(p) * 4 * nblk + b) * 32 + lane]);
+                                uint32_t Alo[4], Ahi[4];
+#pragma unroll
+                                for (int r = 0; r < 4; ++r) {
+                                    Alo[r] = R[r] & 0x0F0F0F0Fu;
+                                    Ahi[r] = R[r] & 0xF0F0F0F0u;
+                                }
 #pragma unroll
                                 for (int i = 0; i < NT; ++i) {
-                                    if (i < nt && s_sched.ti[i].k > p) {
+                                    if (i < nt && s_tile[i].x > p) {
                                         uint32_t b0L = 0, b1L = 0, b0H = 0, b1H = 0;
-                                        if (xrow[i]) {
-                                            const int8_t* src = xrow[i] + 64 * b + 4 * tq;
-                                            b0L = *reinterpret_cast<const uint32_t*>(src);
-                                            b1L = *reinterpret_cast<const uint32_t*>(src + 16);
-                                            b0H = *reinterpret_cast<const uint32_t*>(src + 32);
-                                            b1H = *reinterpret_cast<const uint32_t*>(src + 48);
-                                        }
+                                        if (brow[i]) load_b(brow[i], b, tq, b0L, b1L, b0H, b1H);
                                         mma_u8s8(C[i][0], Alo[0], Alo[1], Alo[2], Alo[3], b0L, b1L);
                                         mma_u8s8(C[i][1], Ahi[0], Ahi[1], Ahi[2], Ahi[3], b0H, b1H);
                                     }
@@ -623,16 +631,16 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                             }
 #pragma unroll
                             for (int i = 0; i < NT; ++i) {
-                                if (i < nt && s_sched.ti[i].k > p) {
+                                if (i < nt && s_tile[i].x > p) {
                                     const int slot = 2 * i + my_half;
-                                    const int Eg = s_exp[slot * ng + g], SX = s_sum[slot * ng + g];
+                                    const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
                                     const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                                     for (int rr = 0; rr < 2; ++rr) {
                                         float v = digit_value(C[i][0][2 * rr], C[i][1][2 * rr], C[i][0][2 * rr + 1],
                                                               C[i][1][2 * rr + 1], tq);
                                         v += __shfl_xor_sync(0xffffffffu, v, 1);
-                                        const int row = warp * 16 + gid + 8 * rr;
+                                        const int row = rtile * 16 + gid + 8 * rr;
                                         const float al = __half2float(meta_h[(p * 64 + row) * ng + g]);
                                         acc[i][rr] = fmaf(al * sc2, fmaf(2.f, v, -static_cast<float>(SX)), acc[i][rr]);
                                     }
@@ -642,89 +650,92 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                     }
                 }
             }
-            // write outputs: lanes tq = 0 (token A) and tq = 2 (token B)
+            // the two K halves meet in shared memory (fixed order), then one store per output
             if ((tq & 1) == 0) {
 #pragma unroll
-                for (int i = 0; i < NT; ++i) {
-                    if (i < nt) {
-                        const int pos = s_pos[2 * i + my_half];
-                        if (pos >= 0) {
+                for (int i = 0; i < NT; ++i)
 #pragma unroll
-                            for (int rr = 0; rr < 2; ++rr)
-                                a.out_pair[static_cast<size_t>(pos) * H + rt * 64 + warp * 16 + gid + 8 * rr] = acc[i][rr];
-                        }
+                    for (int rr = 0; rr < 2; ++rr)
+                        s_red[(((khalf * 4 + rtile) * NT + i) * 2 + my_half) * 16 + gid + 8 * rr] = acc[i][rr];
+            }
+            __syncthreads();
+            for (int q = threadIdx.x; q < 4 * NT * 32; q += kThreads) {
+                const int row = q & 15, tk = (q >> 4) & 1, i = (q >> 5) % NT, tl = q / (32 * NT);
+                if (i < nt) {
+                    const int pos = tk ? s_tile[i].z : s_tile[i].y;
+                    if (pos >= 0) {
+                        const float v = s_red[(((0 * 4 + tl) * NT + i) * 2 + tk) * 16 + row] +
+                                        s_red[(((1 * 4 + tl) * NT + i) * 2 + tk) * 16 + row];
+                        a.out_pair[static_cast<size_t>(pos) * H + rt * 64 + tl * 16 + row] = v;
                     }
                 }
             }
             __syncthreads();
         }
-        if (!copied) {   // expert without tiles cannot happen (active), but keep the phase right
+        if (!waited) {
             const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 202, &s_flag);
             phase ^= 1;
             if (!ok) return;
         }
-        __syncthreads();
     }
 }
 
-template <int FMT>
+template <int FMT, int NT>
 void* pick_gateup(int B) {
     switch (B) {
-        case 1: return reinterpret_cast<void*>(gateup_kernel<FMT, 1>);
-        case 2: return reinterpret_cast<void*>(gateup_kernel<FMT, 2>);
-        case 3: return reinterpret_cast<void*>(gateup_kernel<FMT, 3>);
-        default: return reinterpret_cast<void*>(gateup_kernel<FMT, 4>);
+        case 1: return reinterpret_cast<void*>(gateup_kernel<FMT, 1, NT>);
+        case 2: return reinterpret_cast<void*>(gateup_kernel<FMT, 2, NT>);
+        case 3: return reinterpret_cast<void*>(gateup_kernel<FMT, 3, NT>);
+        default: return reinterpret_cast<void*>(gateup_kernel<FMT, 4, NT>);
     }
 }
-template <int FMT>
+template <int FMT, int NT>
 void* pick_down(int B) {
     switch (B) {
-        case 1: return reinterpret_cast<void*>(down_kernel<FMT, 1>);
-        case 2: return reinterpret_cast<void*>(down_kernel<FMT, 2>);
-        case 3: return reinterpret_cast<void*>(down_kernel<FMT, 3>);
-        default: return reinterpret_cast<void*>(down_kernel<FMT, 4>);
+        case 1: return reinterpret_cast<void*>(down_kernel<FMT, 1, NT>);
+        case 2: return reinterpret_cast<void*>(down_kernel<FMT, 2, NT>);
+        case 3: return reinterpret_cast<void*>(down_kernel<FMT, 3, NT>);
+        default: return reinterpret_cast<void*>(down_kernel<FMT, 4, NT>);
     }
 }
 
-}  // namespace
+int pick_nt(const GemvArgs& a) { return a.max_tokens_per_expert <= 2 ? 1 : 4; }
 
-size_t gateup_smem_bytes(const GemvArgs& a) {
-    const int nblk = a.H >> 6, ng = a.H / a.G;
-    size_t planes = static_cast<size_t>(2) * a.B * nblk * 128;
-    size_t meta = a.fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(2) * 16 * ng * 4 : static_cast<size_t>(2) * a.B * 16 * ng * 2;
-    meta = (meta + 15) & ~size_t(15);
-    return planes + meta + static_cast<size_t>(kWarps) * NT * 2 * 2 * 16 * 4;
-}
-
-size_t down_smem_bytes(const GemvArgs& a) {
-    const int nblk = a.I >> 6, ng = a.I / a.G;
-    size_t planes = static_cast<size_t>(a.B) * 4 * nblk * 128;
-    size_t meta = a.fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(64) * ng * 4 : static_cast<size_t>(a.B) * 64 * ng * 2;
-    meta = (meta + 15) & ~size_t(15);
-    return planes + meta + static_cast<size_t>(2 * NT) * 3 * a.I + static_cast<size_t>(2 * NT) * ng * 8;
-}
-
-static cudaError_t launch_generic(void* fn, size_t smem, int grid, const GemvArgs& a, cudaStream_t stream) {
-    if (grid <= 0) return cudaSuccess;
+cudaError_t launch_generic(void* fn, size_t smem, int items, int num_sms, const GemvArgs& a, cudaStream_t stream) {
+    if (items <= 0) return cudaSuccess;
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    const int grid = items < num_sms * per_sm ? items : num_sms * per_sm;
     GemvArgs copy = a;
     void* args[] = {&copy};
     return cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, smem, stream);
 }
 
+}  // namespace
+
+size_t gateup_smem_bytes(const GemvArgs& a) { return gateup_layout(a.H, a.G, a.B, a.fmt, 4).total; }
+size_t down_smem_bytes(const GemvArgs& a) { return down_layout(a.I, a.G, a.B, a.fmt, 4).total; }
+
 cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms) {
-    void* fn = a.fmt == DPA_FMT_UNIFORM ? pick_gateup<DPA_FMT_UNIFORM>(a.B) : pick_gateup<DPA_FMT_BCQ>(a.B);
-    const int items = a.max_items * (a.I >> 4);
-    const int grid = items < num_sms * 4 ? items : num_sms * 4;
-    return launch_generic(fn, gateup_smem_bytes(a), grid, a, stream);
+    const int nt = pick_nt(a);
+    void* fn;
+    if (a.fmt == DPA_FMT_UNIFORM) fn = nt == 1 ? pick_gateup<DPA_FMT_UNIFORM, 1>(a.B) : pick_gateup<DPA_FMT_UNIFORM, 4>(a.B);
+    else fn = nt == 1 ? pick_gateup<DPA_FMT_BCQ, 1>(a.B) : pick_gateup<DPA_FMT_BCQ, 4>(a.B);
+    return launch_generic(fn, gateup_layout(a.H, a.G, a.B, a.fmt, nt).total, a.max_items * (a.I >> 4), num_sms, a,
+                          stream);
 }
 
 cudaError_t launch_down(const GemvArgs& a, cudaStream_t stream, int num_sms) {
-    void* fn = a.fmt == DPA_FMT_UNIFORM ? pick_down<DPA_FMT_UNIFORM>(a.B) : pick_down<DPA_FMT_BCQ>(a.B);
-    const int items = a.max_items * (a.H >> 6);
-    const int grid = items < num_sms * 4 ? items : num_sms * 4;
-    return launch_generic(fn, down_smem_bytes(a), grid, a, stream);
+    const int nt = pick_nt(a);
+    void* fn;
+    if (a.fmt == DPA_FMT_UNIFORM) fn = nt == 1 ? pick_down<DPA_FMT_UNIFORM, 1>(a.B) : pick_down<DPA_FMT_UNIFORM, 4>(a.B);
+    else fn = nt == 1 ? pick_down<DPA_FMT_BCQ, 1>(a.B) : pick_down<DPA_FMT_BCQ, 4>(a.B);
+    return launch_generic(fn, down_layout(a.I, a.G, a.B, a.fmt, nt).total, a.max_items * (a.H >> 6), num_sms, a,
+                          stream);
 }
 
 }  // namespace dpa

@@ -20,6 +20,7 @@ struct RouteArgs {
     int32_t* xexp;            // [T][H/G]
     int32_t* xsum;            // [T][H/G]
     WsHeader* hdr;
+    int wpe;                  // warps per expert (set by the launcher)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
 
@@ -32,17 +33,16 @@ struct AllocArgs {
     uint8_t* k_out;           // [T][K]
     double* lambda_out;       // scalar or nullptr
     double* cbuf;             // [P][nk] workspace
-    // permutation outputs (do_permute)
+    // grouping outputs (do_permute)
     int do_permute;
-    int32_t* sorted_pair;     // [P] pair ids grouped by (expert, k)
-    int32_t* pair_pos;        // [P] position of each pair in sorted_pair
-    int32_t* seg_start;       // [E*nk + 1]
-    int32_t* exp_kmax;        // [E] (0 if no pair)
-    int32_t* active;          // [E] experts with pairs, ascending
-    uint8_t* k_copy;          // [P] internal copy of k (forward path)
+    int32_t* pair_pos;        // [P] position of each pair in the (expert, k)-grouped order
+    int4* exp_desc;           // [E] per active expert: {expert, kmax, n_tiles, first tile}
+    int4* tiles;              // [P + E*nk] two-token tiles: {k, posA, posB, tokA | tokB << 16}
     WsHeader* hdr;
 };
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream);
+size_t allocate_smem_bytes(int P, int E, int nk);
+int allocate_threads(int P);
 
 struct GemvArgs {
     const uint8_t* planes;    // encoded layer
@@ -50,17 +50,16 @@ struct GemvArgs {
     uint64_t planes_per_expert, meta_per_expert;
     uint64_t planes_mat_off[3], meta_mat_off[3];
     int E, H, I, K, B, G, kmin, kmax, fmt;
-    const int32_t* sorted_pair;
-    const int32_t* seg_start;
-    const int32_t* exp_kmax;
-    const int32_t* active;
+    const int4* exp_desc;     // per active expert {expert, kmax, n_tiles, first tile}
+    const int4* tiles;        // {k, posA, posB, tokA | tokB << 16}
     const int8_t* xdig;       // [T][3][H]
     const int32_t* xexp;      // [T][H/G]
     const int32_t* xsum;      // [T][H/G]
     float* h;                 // [P][I] by sorted position
     float* out_pair;          // [P][H] by sorted position
     WsHeader* hdr;
-    int max_items;            // upper bound of work items (host-known)
+    int max_items;            // upper bound of active experts (host-known)
+    int max_tokens_per_expert;  // host-known bound (selects the tile count per pass)
 };
 cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms);
 size_t gateup_smem_bytes(const GemvArgs& a);   // dynamic shared memory of one CTA

@@ -22,6 +22,7 @@ namespace dpa {
 namespace {
 
 constexpr int kRouteWarps = 8;
+constexpr int16_t kNoBit = 0x3FFF;   // lowest-set-bit marker of a zero element
 
 // ---------------- fp64 exp (see header comment) ----------------
 __device__ __forceinline__ double dexp_fixed(double x) {
@@ -164,67 +165,100 @@ __device__ __forceinline__ int warp_sum_i(int v) {
 
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);   // [H]
-    __shared__ int s_lsb_part[kRouteWarps];
+    const int H = a.H, E = a.E, H8 = H >> 3;
+    // token in lane-major order: element j lives at (j & 7) * H8 + (j >> 3), so the 8
+    // consecutive elements a lane multiplies sit in 8 conflict-free rows
+    double* xd = reinterpret_cast<double*>(smem_raw);                 // [H]
+    int16_t* xl = reinterpret_cast<int16_t*>(xd + H);                 // [H] lowest set bit (kNoBit: zero)
+    uint16_t* xs = reinterpret_cast<uint16_t*>(xl + H);               // [H] bf16 bits (natural order)
     __shared__ int s_last;
+    __shared__ int s_sel[32];
+    __shared__ double s_num[32];
+    __shared__ double s_den;
+    __shared__ double s_acc[kRouteWarps], s_abs[kRouteWarps];
+    __shared__ int s_lmin[kRouteWarps], s_bad[kRouteWarps];
     const int t = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int H = a.H, E = a.E;
+    const int wpe = a.wpe;                    // warps per expert (1, 2, 4 or 8)
+    const int part = warp % wpe;
     const uint16_t* xrow = a.x + static_cast<size_t>(t) * H;
 
-    // stage the token, find the lowest set bit over its nonzero entries
-    int lsb_x = 1 << 20;
     bool bad = false;
     for (int j = threadIdx.x; j < H; j += blockDim.x) {
         const uint16_t u = xrow[j];
+        const int q = (j & 7) * H8 + (j >> 3);
+        xd[q] = static_cast<double>(bf16_bits_to_float(u));
+        xl[q] = (u & 0x7FFF) ? static_cast<int16_t>(bf16_lsb(u)) : kNoBit;
         xs[j] = u;
-        if (u & 0x7FFF) lsb_x = min(lsb_x, bf16_lsb(u));
         bad |= ((u >> 7) & 0xFF) == 0xFF;
     }
-    lsb_x = warp_min_i(lsb_x);
-    if (lane == 0) s_lsb_part[warp] = lsb_x;
     if (__syncthreads_or(bad) && threadIdx.x == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 1);
-    lsb_x = s_lsb_part[0];
-#pragma unroll
-    for (int w = 1; w < kRouteWarps; ++w) lsb_x = min(lsb_x, s_lsb_part[w]);
 
-    // ---- one warp per expert logit ----
-    const int e = blockIdx.x * kRouteWarps + warp;
-    if (e < E) {
-        const uint16_t* wrow = a.wr + static_cast<size_t>(e) * H;
-        double acc = 0.0, absacc = 0.0;
-        int lsb_w = 1 << 20;
+    // ---- wpe warps per expert logit: partial sums of products, lowest bits, magnitudes ----
+    const int e = blockIdx.x * (kRouteWarps / wpe) + warp / wpe;
+    {
+        double acc0 = 0.0, acc1 = 0.0, abs0 = 0.0, abs1 = 0.0;
+        int lmin = 1 << 20;
         bool wbad = false;
-        for (int j0 = lane * 8; j0 < H; j0 += 256) {
-            const uint4 wv = *reinterpret_cast<const uint4*>(wrow + j0);
-            const uint4 xv = *reinterpret_cast<const uint4*>(xs + j0);
-            const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-            const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+        if (e < E) {
+            const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H);
+            const int stride = 32 * wpe;                  // uint4 columns per round
+            const int nq = (H8 + stride - 1) / stride;
+            for (int q0 = 0; q0 < nq; q0 += 8) {
+                uint4 wv[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+                for (int u = 0; u < 8; ++u) {
+                    const int col = (q0 + u) * stride + part * 32 + lane;
+                    if (q0 + u < nq && col < H8) wv[u] = wrow[col];
+                }
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t wu = (ww[q] >> (16 * h)) & 0xFFFFu;
-                    const uint32_t xu = (xx[q] >> (16 * h)) & 0xFFFFu;
-                    const double p = __dmul_rn(static_cast<double>(__uint_as_float(xu << 16)),
-                                               static_cast<double>(__uint_as_float(wu << 16)));
-                    acc = __dadd_rn(acc, p);
-                    absacc = __dadd_rn(absacc, fabs(p));
-                    if (wu & 0x7FFF) lsb_w = min(lsb_w, bf16_lsb(wu));
-                    wbad |= ((wu >> 7) & 0xFF) == 0xFF;
+                for (int u = 0; u < 8; ++u) {
+                    const int col = (q0 + u) * stride + part * 32 + lane;   // 8-element group index
+                    if (q0 + u < nq && col < H8) {
+                        const uint32_t ww[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            const uint32_t wu = (ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                            const double xv = xd[h * H8 + col];
+                            const double p = __dmul_rn(xv, static_cast<double>(__uint_as_float(wu << 16)));
+                            if (h & 1) { acc1 = __dadd_rn(acc1, p); abs1 = __dadd_rn(abs1, fabs(p)); }
+                            else { acc0 = __dadd_rn(acc0, p); abs0 = __dadd_rn(abs0, fabs(p)); }
+                            if (wu & 0x7FFF) lmin = min(lmin, static_cast<int>(xl[h * H8 + col]) + bf16_lsb(wu));
+                            wbad |= ((wu >> 7) & 0xFF) == 0xFF;
+                        }
+                    }
                 }
             }
         }
-        acc = warp_sum_f64(acc);
-        absacc = warp_sum_f64(absacc);
-        lsb_w = warp_min_i(lsb_w);
+        const double acc = warp_sum_f64(__dadd_rn(acc0, acc1));
+        const double absacc = warp_sum_f64(__dadd_rn(abs0, abs1));
+        lmin = warp_min_i(lmin);
         wbad = __any_sync(0xffffffffu, wbad);
+        if (lane == 0) {
+            s_acc[warp] = acc;
+            s_abs[warp] = absacc;
+            s_lmin[warp] = lmin;
+            s_bad[warp] = wbad ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    if (part == 0 && e < E) {
+        // combine the expert's partial sums (exact whenever the bound below holds)
+        double acc = s_acc[warp], absacc = s_abs[warp];
+        int lmin = s_lmin[warp], wbad = s_bad[warp];
+        for (int w = 1; w < wpe; ++w) {
+            acc = __dadd_rn(acc, s_acc[warp + w]);
+            absacc = __dadd_rn(absacc, s_abs[warp + w]);
+            lmin = min(lmin, s_lmin[warp + w]);
+            wbad |= s_bad[warp + w];
+        }
         double logit = acc;
         if (absacc != 0.0) {
             int ea;
-            frexp(absacc, &ea);              // absacc < 2^ea
-            if (ea > lsb_x + lsb_w + 52)     // exactness not proven: exact fixed-point path
-                logit = exact_dot_fixed(xs, wrow, H, lane);
+            frexp(absacc, &ea);   // absacc < 2^ea
+            // every product is a multiple of 2^lmin and sum |p| < 2^(lmin+53): no partial sum
+            // in any order can round, so acc is the exact dot product. Otherwise recompute.
+            if (ea > lmin + 52) logit = exact_dot_fixed(xs, a.wr + static_cast<size_t>(e) * H, H, lane);
         }
         if (lane == 0) {
             double* dst = a.logits_user ? a.logits_user : a.logits_ws;
@@ -271,60 +305,69 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     if (!s_last) return;
     if (threadIdx.x == 0) a.counters[t] = 0;   // ready for the next call
     __threadfence();
-    if (warp != 0) return;
 
     const double* lrow = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
-    double* vals = reinterpret_cast<double*>(smem_raw);   // reuse: [E] logits (x no longer needed)
-    for (int i = lane; i < E; i += 32) vals[i] = __ldcg(lrow + i);
-    __syncwarp();
+    double* vals = reinterpret_cast<double*>(smem_raw);   // reuse: [E] logits (token no longer needed)
+    for (int i = threadIdx.x; i < E; i += blockDim.x) vals[i] = __ldcg(lrow + i);
+    __syncthreads();
     const int K = a.K;
-    int my_e = -1;
-    double my_l = 0.0;
-    for (int r = 0; r < K; ++r) {
-        double bv = 0.0;
-        int be = -1;
-        for (int i = lane; i < E; i += 32) {
-            const double v = vals[i];
-            if (v != v) continue;   // NaN (already flagged as invalid input)
-            if (be < 0 || v > bv) { bv = v; be = i; }
+    // rank of each expert = number of experts before it (descending logit, ties to the lower
+    // id; NaN ranks last). Q threads share a candidate, each counting over 1/Q of the experts.
+    int Q = 1;
+    while (Q < 32 && Q * 2 * E <= static_cast<int>(blockDim.x)) Q *= 2;
+    const int chunk = (E + Q - 1) / Q;
+    for (int base = 0; base < E * Q; base += blockDim.x) {
+        const int idx = base + threadIdx.x;
+        const int c = idx / Q, q = idx % Q;
+        int rank = 0;
+        if (c < E) {
+            const double v = vals[c];
+            if (v == v) {
+                const int j1 = min(E, (q + 1) * chunk);
+                for (int j = q * chunk; j < j1; ++j) {
+                    const double u = vals[j];
+                    rank += (u > v || (u == v && j < c)) ? 1 : 0;
+                }
+            } else {
+                rank = q == 0 ? E : 0;
+            }
         }
-        for (int o = 16; o > 0; o >>= 1) {
-            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-            const bool take = oe >= 0 && (be < 0 || ov > bv || (ov == bv && oe < be));
-            if (take) { bv = ov; be = oe; }
-        }
-        if (lane == r) { my_e = be; my_l = bv; }
-        if (be >= 0 && lane == (be & 31)) vals[be] = __longlong_as_double(0x7ff8000000000000ll);  // remove
-        __syncwarp();
+        for (int o = 1; o < Q; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+        if (c < E && q == 0 && rank < K) s_sel[rank] = c;
     }
-    const double lmax = __shfl_sync(0xffffffffu, my_l, 0);
-    double num = 0.0;
-    if (lane < K) num = dexp_fixed(__dsub_rn(my_l, lmax));
-    double den = 0.0;
-    if (a.norm_topk) {
-        for (int j = 0; j < K; ++j) den = __dadd_rn(den, __shfl_sync(0xffffffffu, num, j));
-    } else {
-        // softmax over every expert, summed in ascending expert id
-        double* ex = vals;
-        for (int i = lane; i < E; i += 32) ex[i] = dexp_fixed(__dsub_rn(__ldcg(lrow + i), lmax));
-        __syncwarp();
-        if (lane == 0)
+    __syncthreads();
+    const double lmax = vals[s_sel[0]];
+    if (threadIdx.x < K) s_num[threadIdx.x] = dexp_fixed(__dsub_rn(vals[s_sel[threadIdx.x]], lmax));
+    double* ex = vals + E;   // [E] exp values (norm over all experts)
+    if (!a.norm_topk)
+        for (int i = threadIdx.x; i < E; i += blockDim.x) ex[i] = dexp_fixed(__dsub_rn(vals[i], lmax));
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double den = 0.0;
+        if (a.norm_topk) {
+            for (int j = 0; j < K; ++j) den = __dadd_rn(den, s_num[j]);
+        } else {
             for (int i = 0; i < E; ++i) den = __dadd_rn(den, ex[i]);
-        den = __shfl_sync(0xffffffffu, den, 0);
+        }
+        s_den = den;
     }
-    if (lane < K) {
-        a.idx[t * K + lane] = my_e;
-        a.gate[t * K + lane] = __ddiv_rn(num, den);
+    __syncthreads();
+    if (threadIdx.x < K) {
+        a.idx[t * K + threadIdx.x] = s_sel[threadIdx.x];
+        a.gate[t * K + threadIdx.x] = __ddiv_rn(s_num[threadIdx.x], s_den);
     }
 }
 
 }  // namespace
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
-    const int chunks = (a.E + kRouteWarps - 1) / kRouteWarps;
-    size_t smem = static_cast<size_t>(a.H) * 2;
-    const size_t need_vals = static_cast<size_t>(a.E) * 8;
+    // few tokens: split each expert's dot product over 4 warps to shorten the serial chain
+    RouteArgs b = a;
+    b.wpe = a.T <= 16 ? 4 : 1;
+    const int epb = kRouteWarps / b.wpe;
+    const int chunks = (a.E + epb - 1) / epb;
+    size_t smem = static_cast<size_t>(a.H) * 12;              // fp64 token, lowest bits, bf16 copy
+    const size_t need_vals = static_cast<size_t>(a.E) * 16;   // logits and exps
     if (need_vals > smem) smem = need_vals;
     smem = (smem + 15) & ~static_cast<size_t>(15);
     if (smem > 48 * 1024) {
@@ -333,10 +376,9 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
         if (err != cudaSuccess) return err;
     }
     dim3 grid(chunks, a.T);
-    route_kernel<<<grid, kRouteWarps * 32, smem, stream>>>(a);
+    route_kernel<<<grid, kRouteWarps * 32, smem, stream>>>(b);
     return cudaGetLastError();
 }
 
-int route_chunks(int E) { return (E + kRouteWarps - 1) / kRouteWarps; }
 
 }  // namespace dpa

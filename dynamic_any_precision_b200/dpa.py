@@ -249,6 +249,8 @@ def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] =
                     _dptr(aux.get("lambda")), _dptr(aux.get("pair_out")))
         for i, ev in enumerate(aux.get("events") or ()):
             if ev is not None:
+                if not ev.cuda_event:
+                    raise ValueError("record a torch.cuda.Event once before passing it (lazy creation)")
                 aux_s.events[i] = ev.cuda_event
     _check(lib().dpa_moe_forward(ctypes.byref(layer.desc), ctypes.byref(layer.weights), _dptr(x), T, _dptr(target),
                                  _dptr(y), ctypes.byref(aux_s) if aux_s is not None else None, _dptr(ws), ws.numel(),
