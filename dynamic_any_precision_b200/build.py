@@ -32,6 +32,7 @@ CU_SOURCES = {
     "gemv.cu": [],
     "combine.cu": [],
     "dpa_abi.cu": [],
+    "route_noalloc.cu": [],
 }
 CPP_SOURCES = {"encode.cpp": ["-O2", "-ffp-contract=off", "-fno-fast-math"]}
 

@@ -189,6 +189,22 @@ dpa_status dpa_allocate(const dpa_layer_desc* desc, const double* rtable,
                         const double* target_bpw, uint8_t* k_out, double* lambda_out,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of dpa_route, for callers that cannot allocate device memory:
+ * for example a plugin whose host engine owns every byte of device memory, or a loop that
+ * must not call the allocator. It has no counterpart in the pages; it exists for those callers.
+ * Same inputs, outputs and decisions as dpa_route, but no workspace: its scratch (per-token
+ * counters and a logits buffer) lives in a fixed array of about 0.5 MB inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ * Limits: n_tokens <= 1024 and n_tokens * n_experts <= 65536, else DPA_ERR_UNSUPPORTED
+ * (nothing launched). The first call on a device looks up the array's device address, so
+ * make it before any stream capture. Every call shares the array: calls whose executions
+ * overlap on the GPU (other streams, other threads) race and must be serialised by the
+ * caller. Device-side input checks (NaN/Inf tokens) are not reported by this variant.
+ * logits may be NULL. stream: cudaStream_t. */
+dpa_status dpa_route_noalloc(const dpa_layer_desc* desc, const void* x, int n_tokens,
+                             const void* w_router, int32_t* topk_idx, double* topk_gate,
+                             double* logits, void* stream);
+
 /* Workspace bytes that dpa_route, dpa_allocate and dpa_moe_forward need for up to
  * max_tokens tokens. Returns 0 for an invalid descriptor. */
 size_t dpa_forward_workspace_size(const dpa_layer_desc* desc, int max_tokens);
