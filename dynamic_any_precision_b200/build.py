@@ -33,6 +33,7 @@ CU_SOURCES = {
     "combine.cu": [],
     "dpa_abi.cu": [],
     "route_noalloc.cu": [],
+    "stack_glue.cu": [],
 }
 CPP_SOURCES = {"encode.cpp": ["-O2", "-ffp-contract=off", "-fno-fast-math"]}
 

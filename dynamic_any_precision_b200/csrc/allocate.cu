@@ -45,6 +45,22 @@ __device__ __forceinline__ int choose_k(const double* c, int nk, int kmin, doubl
 
 __device__ __forceinline__ double midpoint(double lo, double hi) { return __dmul_rn(0.5, __dadd_rn(lo, hi)); }
 
+// the same decision with the pair's costs in registers (nk <= 4 because B <= 4)
+__device__ __forceinline__ int choose_k_reg(const double (&c)[4], int nk, int kmin, double lam) {
+    double best = __dadd_rn(c[0], __dmul_rn(lam, static_cast<double>(kmin)));
+    int kb = kmin;
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+        if (i < nk) {
+            const double cost = __dadd_rn(c[i], __dmul_rn(lam, static_cast<double>(kmin + i)));
+            if (cost < best) { best = cost; kb = kmin + i; }
+        }
+    }
+    return kb;
+}
+
+constexpr int kRegPairs = 4;   // pairs per lane held in registers by the small-batch bisection
+
 // inclusive block scan of one int per thread
 __device__ __forceinline__ int block_incl_scan(int v, int* s_tmp) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -95,9 +111,15 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_tmp[32];
     __shared__ double s_max[32];
-    __shared__ int s_ok;
-    __shared__ double s_lohi[2];
     __shared__ unsigned char s_pred[2][kAllocThreads];
+    // speculative replay of the bisection (small batches)
+    __shared__ double s_bp[kSmallP * 3];
+    __shared__ int s_bj[kSmallP * 3];
+    __shared__ int s_order[kSmallP * 3];
+    __shared__ int s_nbp;
+    __shared__ double s_mid[64], s_lo[65], s_hi[65];
+    __shared__ unsigned char s_spred[64];
+    __shared__ unsigned s_mis[4];
     const int P = a.T * a.K;
     const int nk = a.kmax - a.kmin + 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -105,36 +127,39 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     double* c_base = Ls.costs_in_smem ? reinterpret_cast<double*>(smem + Ls.costs) : a.cbuf;
     uint8_t* s_k = smem + Ls.kk;
 
-    if (tid == 0) {
-        const double tg = *a.target;
-        s_ok = (tg >= static_cast<double>(a.kmin) && tg <= static_cast<double>(a.kmax)) ? 1 : 0;
-        if (!s_ok) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 10);
-    }
-    __syncthreads();
-    int bad = 0;
+    pdl_wait();   // the routed pairs come from the previous kernel
+    // the budget, the pairs' experts and gates are loaded together (one round trip)
+    const double target = *a.target;
+    int bad = (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1;
+    if (bad && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 10);
+    int bad_e = 0;
     for (int p = tid; p < P; p += blockDim.x) {
         const int e = a.idx[p];
-        bad |= (e < 0 || e >= a.E) ? 1 : 0;
+        bad_e |= (e < 0 || e >= a.E) ? 1 : 0;
     }
-    if (__syncthreads_or(bad)) {
-        if (tid == 0) { set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 11); s_ok = 0; }
-    }
-    __syncthreads();
-    if (!s_ok) {
+    const int any_bad_e = __syncthreads_or(bad_e);
+    if (any_bad_e && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 11);
+    if (bad || any_bad_e) {
         if (a.do_permute && tid == 0) a.hdr->n_active = 0;
         return;
     }
-    const double target = *a.target;
 
-    // costs c[p][i] = fl(g_p * r_{e_p}(kmin + i))
+    // costs c[p][i] = fl(g_p * r_{e_p}(kmin + i)); the rtable loads of a pair are issued together
     double mx = 0.0;
     for (int p = tid; p < P; p += blockDim.x) {
         const int e = a.idx[p];
         const double g = a.gate[p];
-        for (int i = 0; i < nk; ++i) {
-            const double c = __dmul_rn(g, a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)]);
-            c_base[static_cast<size_t>(p) * nk + i] = c;
-            if (i == 0) mx = fmax(mx, c);
+        double r[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i < nk) r[i] = a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i < nk) {
+                const double c = __dmul_rn(g, r[i]);
+                c_base[static_cast<size_t>(p) * nk + i] = c;
+                if (i == 0) mx = fmax(mx, c);
+            }
         }
     }
     for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -148,40 +173,146 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     double hi = __dadd_rn(__dmul_rn(2.0, mx), 1.0);
 
     if (P <= kSmallP) {
-        // one warp: lane n-1 evaluates node n of a depth-5 tree of midpoints, predicates come
-        // back as a ballot and every lane walks the tree in registers (no block barriers)
-        if (warp == 0) {
-            for (int it = 0; it < 64;) {
-                const int D = min(5, 64 - it);
-                const int node = lane + 1;
-                int pred = 0;
-                if (node < (1 << D)) {
-                    const int depth = 31 - __clz(node);
-                    double l = lo, h = hi;
-                    for (int lev = depth - 1; lev >= 0; --lev) {
-                        const double m = midpoint(l, h);
-                        if ((node >> lev) & 1) l = m; else h = m;
-                    }
-                    const double mid = midpoint(l, h);
-                    int n = 0;
-                    for (int p = 0; p < P; ++p) n += choose_k(c_base + p * nk, nk, a.kmin, mid);
-                    pred = static_cast<double>(n) > budget ? 1 : 0;
-                }
-                const unsigned mask = __ballot_sync(0xffffffffu, pred);   // bit (node-1)
-                int nd = 1;
-                for (int lev = 0; lev < D; ++lev) {
-                    const int pr = (mask >> (nd - 1)) & 1;
-                    const double m = midpoint(lo, hi);
-                    if (pr) lo = m; else hi = m;
-                    nd = 2 * nd + pr;
-                }
-                it += D;
+        // 4 warps, 4 lanes per node: 32 node slots hold the 31 midpoints of the next 5 steps.
+        // Each lane counts planes for every 4th pair; the 4-lane sums give N(mid); each warp's
+        // 8 predicates travel through shared memory as one byte, and every thread walks the
+        // tree in registers.
+        const int slot = tid >> 2, gl = tid & 3;   // node slot 0..31, lane in node
+        const double* s_costs = reinterpret_cast<const double*>(smem + Ls.costs);   // P*nk <= kSmemCostDoubles
+        // this lane's pairs (gl, gl+4, ...) and their costs, kept in registers across all rounds
+        const bool in_regs = P <= 4 * kRegPairs;
+        double creg[kRegPairs][4];
+#pragma unroll
+        for (int j = 0; j < kRegPairs; ++j)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int p = gl + 4 * j;
+                creg[j][i] = (in_regs && p < P && i < nk) ? s_costs[p * nk + i] : 0.0;
             }
-            if (lane == 0) { s_lohi[0] = lo; s_lohi[1] = hi; }
+        // ---- speculation. In real arithmetic each pair's choice falls at the breakpoints of the
+        // lower convex hull of its points (k, c_k); summing the falls gives the lambda below which
+        // N(lambda) > budget. One thread replays the 64 steps with that threshold, recording each
+        // midpoint; then every recorded step's predicate is evaluated exactly, in parallel. The
+        // replay is kept up to the first step whose exact predicate disagrees; from there the exact
+        // tree bisection below takes over. Either way the steps taken are the exact ones.
+        if (tid == 0) s_nbp = 0;
+        __syncthreads();
+        if (tid < P) {
+            const double* c = s_costs + tid * nk;
+            int cur = 0;   // choice as lambda -> 0+: the smallest cost, ties to the smaller k
+            for (int i = 1; i < nk; ++i) if (c[i] < c[cur]) cur = i;
+            while (cur > 0) {
+                int jn = -1;
+                double tn = 0.0;
+                for (int j = 0; j < cur; ++j) {   // the next smaller k to take over as lambda grows
+                    const double t = (c[j] - c[cur]) / static_cast<double>(cur - j);
+                    if (jn < 0 || t < tn) { jn = j; tn = t; }
+                }
+                const int slotb = atomicAdd(&s_nbp, 1);
+                s_bp[slotb] = tn;
+                s_bj[slotb] = cur - jn;
+                cur = jn;
+            }
         }
         __syncthreads();
-        lo = s_lohi[0];
-        hi = s_lohi[1];
+        const int nbp = s_nbp;
+        for (int i = tid; i < nbp; i += blockDim.x) {   // descending order of the breakpoints
+            const double v = s_bp[i];
+            int r = 0;
+            for (int j = 0; j < nbp; ++j) r += (s_bp[j] > v || (s_bp[j] == v && j < i)) ? 1 : 0;
+            s_order[r] = i;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            double lam_c = 0.0;    // N(lambda) > budget exactly for lambda < lam_c (real arithmetic)
+            int cum = P * a.kmin;
+            for (int m = 0; m < nbp; ++m) {
+                cum += s_bj[s_order[m]];
+                if (static_cast<double>(cum) > budget) { lam_c = s_bp[s_order[m]]; break; }
+            }
+            double l = lo, h = hi;
+            for (int i = 0; i < 64; ++i) {
+                s_lo[i] = l;
+                s_hi[i] = h;
+                const double m = midpoint(l, h);
+                const int pr = m < lam_c ? 1 : 0;
+                s_mid[i] = m;
+                s_spred[i] = static_cast<unsigned char>(pr);
+                if (pr) l = m; else h = m;
+            }
+            s_lo[64] = l;
+            s_hi[64] = h;
+        }
+        __syncthreads();
+        {   // exact check of the 64 recorded steps: two threads per step
+            const int node = tid >> 1, gl2 = tid & 1;
+            int n = 0;
+            const double m = s_mid[node];
+            for (int p = gl2; p < P; p += 2) n += choose_k(s_costs + p * nk, nk, a.kmin, m);
+            n += __shfl_xor_sync(0xffffffffu, n, 1);
+            const int pr = static_cast<double>(n) > budget ? 1 : 0;
+            const unsigned bad_mask = __ballot_sync(0xffffffffu, gl2 == 0 && pr != s_spred[node]);
+            if (lane == 0) s_mis[warp] = bad_mask;   // bit 2j of warp w: step 16w + j
+        }
+        __syncthreads();
+        int it0 = 64;
+        for (int w = 0; w < 4 && it0 == 64; ++w)
+            if (s_mis[w]) it0 = 16 * w + (__ffs(static_cast<int>(s_mis[w])) - 1) / 2;
+        lo = s_lo[it0];
+        hi = s_hi[it0];
+
+        int round = 0;
+        for (int it = it0; it < 64; ++round) {
+            const int D = min(5, 64 - it);
+            const int node = slot + 1;
+            const bool active = node < (1 << D);
+            int n = 0;
+            if (active) {
+                const int depth = 31 - __clz(node);
+                double l = lo, h = hi;
+                for (int lev = depth - 1; lev >= 0; --lev) {
+                    const double m = midpoint(l, h);
+                    if ((node >> lev) & 1) l = m; else h = m;
+                }
+                const double mid = midpoint(l, h);
+                if (in_regs) {
+#pragma unroll
+                    for (int j = 0; j < kRegPairs; ++j)
+                        if (gl + 4 * j < P) n += choose_k_reg(creg[j], nk, a.kmin, mid);
+                } else {
+                    int n0 = 0, n1 = 0;
+                    int p = gl;
+                    for (; p + 4 < P; p += 8) {   // two independent pairs per iteration
+                        n0 += choose_k(s_costs + p * nk, nk, a.kmin, mid);
+                        n1 += choose_k(s_costs + (p + 4) * nk, nk, a.kmin, mid);
+                    }
+                    if (p < P) n0 += choose_k(s_costs + p * nk, nk, a.kmin, mid);
+                    n = n0 + n1;
+                }
+            }
+            n += __shfl_xor_sync(0xffffffffu, n, 1);
+            n += __shfl_xor_sync(0xffffffffu, n, 2);
+            const int pred = (active && static_cast<double>(n) > budget) ? 1 : 0;
+            const unsigned bal = __ballot_sync(0xffffffffu, pred && gl == 0);   // bits 4*i: node 8*warp+i+1
+            if (lane == 0) {
+                unsigned b = 0;
+                for (int i = 0; i < 8; ++i) b |= ((bal >> (4 * i)) & 1u) << i;
+                s_pred[round & 1][warp] = static_cast<unsigned char>(b);
+            }
+            __syncthreads();
+            const unsigned mask = static_cast<unsigned>(s_pred[round & 1][0]) |
+                                  (static_cast<unsigned>(s_pred[round & 1][1]) << 8) |
+                                  (static_cast<unsigned>(s_pred[round & 1][2]) << 16) |
+                                  (static_cast<unsigned>(s_pred[round & 1][3]) << 24);   // bit node-1
+            int nd = 1;
+            for (int lev = 0; lev < D; ++lev) {
+                const int pr = (mask >> (nd - 1)) & 1;
+                const double m = midpoint(lo, hi);
+                if (pr) lo = m; else hi = m;
+                nd = 2 * nd + pr;
+            }
+            it += D;
+        }
     } else {
         // whole block: a group of gs threads per node, trees of depth D per round
         int gs_log = 0;
@@ -282,7 +413,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         const int rank = rank_base + rank_incl - flag;
         const int tile_off = tile_base + tiles_incl - ntiles;
         if (flag) {
-            a.exp_desc[rank] = make_int4(e, km, ntiles, tile_off);
+            a.exp_desc[2 * rank] = make_int4(e, km, ntiles, tile_off);
             int t = tile_off;
             for (int i = 0; i < nk; ++i) {
                 const int s0 = s_seg[e * nk + i];
@@ -291,7 +422,9 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                     const int posA = s0 + j, posB = j + 1 < n ? s0 + j + 1 : -1;
                     const int tokA = s_sorted[posA] / a.K;
                     const int tokB = posB >= 0 ? s_sorted[posB] / a.K : -1;
-                    a.tiles[t++] = make_int4(a.kmin + i, posA, posB, (tokA & 0xFFFF) | ((tokB & 0xFFFF) << 16));
+                    const int4 tile = make_int4(a.kmin + i, posA, posB, (tokA & 0xFFFF) | ((tokB & 0xFFFF) << 16));
+                    if (t == tile_off) a.exp_desc[2 * rank + 1] = tile;   // first tile rides with the descriptor
+                    a.tiles[t++] = tile;
                 }
             }
         }
@@ -309,7 +442,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
 
 size_t allocate_smem_bytes(int P, int E, int nk) { return alloc_smem_layout(P, E, nk).total; }
 
-int allocate_threads(int P) { return P <= kSmallP ? 128 : kAllocThreads; }
+int allocate_threads(int P) { return P <= kSmallP ? 128 : kAllocThreads; }   // small: 4 warps x 8 nodes
 
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream) {
     const int nk = a.kmax - a.kmin + 1;
@@ -320,8 +453,10 @@ cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream) {
                                                static_cast<int>(smem));
         if (err != cudaSuccess) return err;
     }
-    allocate_kernel<<<1, allocate_threads(P), smem, stream>>>(a);
-    return cudaGetLastError();
+    AllocArgs b = a;
+    void* args[] = {&b};
+    return launch_pdl_raw(reinterpret_cast<const void*>(allocate_kernel), dim3(1), dim3(allocate_threads(P)), smem,
+                          stream, args);
 }
 
 }  // namespace dpa

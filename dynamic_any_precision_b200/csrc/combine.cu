@@ -14,6 +14,7 @@ namespace dpa {
 namespace {
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+    pdl_wait();
     const int t = blockIdx.y;
     const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
     if (n >= a.H) return;
@@ -72,6 +73,7 @@ __device__ __forceinline__ void bf16x8_to_f32(uint4 v, float (&f)[8]) {
 }
 
 __global__ void __launch_bounds__(256) shared_gateup_kernel(SharedArgs a) {
+    pdl_wait();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int row = warp % a.I, s = warp / a.I;
     if (s >= a.S) return;
@@ -112,6 +114,7 @@ __global__ void __launch_bounds__(256) shared_gateup_kernel(SharedArgs a) {
 }
 
 __global__ void __launch_bounds__(256) shared_down_kernel(SharedArgs a) {
+    pdl_wait();
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
     const int n = warp;
     if (n >= a.H) return;
@@ -156,18 +159,21 @@ __global__ void __launch_bounds__(256) shared_down_kernel(SharedArgs a) {
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
     const int per_block = 256 * 4;
     dim3 grid((a.H + per_block - 1) / per_block, a.T);
-    combine_kernel<<<grid, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    CombineArgs b = a;
+    void* args[] = {&b};
+    return launch_pdl_raw(reinterpret_cast<const void*>(combine_kernel), grid, dim3(256), 0, stream, args);
 }
 
 cudaError_t launch_shared(const SharedArgs& a, cudaStream_t stream) {
     if (a.S == 0 || a.T == 0) return cudaSuccess;
     const int warps1 = a.S * a.I;
-    shared_gateup_kernel<<<(warps1 + 7) / 8, 256, 0, stream>>>(a);
-    cudaError_t err = cudaGetLastError();
+    SharedArgs b = a;
+    void* args[] = {&b};
+    cudaError_t err = launch_pdl_raw(reinterpret_cast<const void*>(shared_gateup_kernel), dim3((warps1 + 7) / 8),
+                                     dim3(256), 0, stream, args);
     if (err != cudaSuccess) return err;
-    shared_down_kernel<<<(a.H + 7) / 8, 256, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl_raw(reinterpret_cast<const void*>(shared_down_kernel), dim3((a.H + 7) / 8), dim3(256), 0,
+                          stream, args);
 }
 
 }  // namespace dpa

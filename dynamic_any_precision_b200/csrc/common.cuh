@@ -111,6 +111,32 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// ---- programmatic dependent launch ----
+// Kernels of a forward are launched with programmatic stream serialisation and issue no explicit
+// trigger, so a successor is released when its predecessor's CTAs have all exited; the launch
+// and prologue work before wait (descriptor and weight prefetch) then overlap the predecessor's
+// tail. wait blocks until the predecessor has completed and its memory is visible; every kernel
+// calls it before its first read of a predecessor's output and before its first global write.
+// Outside such a launch it is a no-op. (Triggering at kernel entry was measured slower: the
+// early-resident successor CTAs take SM slots from the predecessor.)
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch with programmatic stream serialisation (see above).
+inline cudaError_t launch_pdl_raw(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                  void** args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
 // ---- u8 x s8 MMA, m16n8k32, int32 accumulate ----
 __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {

@@ -24,7 +24,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
     if (d->norm_topk != 0 && d->norm_topk != 1) return DPA_ERR_INVALID_ARG;
     if (d->n_shared < 0 || d->top_k > d->n_experts) return DPA_ERR_INVALID_ARG;
     if (d->bits > 4 || d->n_experts > 1024 || d->top_k > 32 || d->n_shared > 8) return DPA_ERR_UNSUPPORTED;
-    if (d->hidden % 64 || d->inter % 64 || d->group % 64) return DPA_ERR_UNSUPPORTED;
+    if (d->hidden % 64 || d->inter % 64 || d->group % 64 || d->group > 512) return DPA_ERR_UNSUPPORTED;
     if (d->hidden % d->group || d->inter % d->group) return DPA_ERR_UNSUPPORTED;
     if (d->hidden > 16384 || d->inter > 16384) return DPA_ERR_UNSUPPORTED;
     // the per-CTA staging of one work item must fit in shared memory
@@ -73,7 +73,7 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.out_pair = take(4 * P * H);
     L.sh_h = take(4 * static_cast<size_t>(T) * d->n_shared * I);
     L.sh_out = take(4 * static_cast<size_t>(T) * H);
-    L.desc = take(16 * E);
+    L.desc = take(32 * E);
     L.tiles = take(16 * (P + E * nk));
     L.total = off;
     return L;
@@ -356,6 +356,15 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     if (dpa::launch_combine(ca, s) != cudaSuccess) return DPA_ERR_CUDA;
     mark(6);
     return DPA_OK;
+}
+
+dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidden, void* x, void* stream) {
+    if (!h || !x || n_tokens <= 0 || n_tokens > 2147483647 || hidden <= 0 || hidden % 4) return DPA_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(x) || (y && !aligned16(y))) return DPA_ERR_INVALID_ARG;
+    return dpa::launch_residual_rmsnorm(static_cast<const uint16_t*>(y), h, static_cast<uint16_t*>(x), n_tokens, hidden,
+                                        1e-6f, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DPA_OK
+               : DPA_ERR_CUDA;
 }
 
 dpa_status dpa_device_status(void* ws, void* stream) {

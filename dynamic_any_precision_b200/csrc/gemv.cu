@@ -169,19 +169,27 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tq = lane & 3;
-    const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     if (threadIdx.x == 0) {
         mbar_init(&s_bar, 1);
         fence_barrier_init();
     }
+    pdl_wait();   // work lists and activations come from the previous kernels
+    const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     __syncthreads();
     uint32_t phase = 0;
     const int g0 = (warp * ng) / kWarps, g1 = ((warp + 1) * ng) / kWarps;   // this warp's groups
     const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
     const int dstride = Ly.dig_stride;
 
+    // the first item's descriptor is loaded together with the active count (the index is in
+    // bounds for every launched CTA; its contents are used only if the item exists)
+    int4 desc = a.exp_desc[2 * (blockIdx.x / tiles_per_expert)];
+    int4 tile0 = a.exp_desc[2 * (blockIdx.x / tiles_per_expert) + 1];
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int4 desc = a.exp_desc[item / tiles_per_expert];
+        if (item != blockIdx.x) {
+            desc = a.exp_desc[2 * (item / tiles_per_expert)];
+            tile0 = a.exp_desc[2 * (item / tiles_per_expert) + 1];
+        }
         const int e = desc.x, kmax_e = desc.y, ntiles = desc.z, toff = desc.w;
         const int rt = item % tiles_per_expert;
         if (threadIdx.x == 0) {
@@ -209,23 +217,40 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
         }
         bool waited = false;
         for (int pass0 = 0; pass0 < ntiles; pass0 += NT) {
-            if (threadIdx.x < NT) {
+            if (NT == 1) {
+                if (threadIdx.x == 0) s_tile[0] = pass0 == 0 ? tile0 : a.tiles[toff + pass0];
+            } else if (threadIdx.x < NT) {
                 const int i = threadIdx.x;
                 s_tile[i] = pass0 + i < ntiles ? a.tiles[toff + pass0 + i] : make_int4(0, -1, -1, -1);
             }
             if (threadIdx.x == 0) s_nt = min(NT, ntiles - pass0);
             __syncthreads();
             const int nt = s_nt;
-            // stage the digits, exponents and sums of the pass's tokens
+            // stage the digits, exponents and sums of the pass's tokens (loads issued first)
             {
                 const int chunks = (3 * H) >> 4;
-                for (int i = threadIdx.x; i < 2 * NT * chunks; i += kThreads) {
-                    const int slot = i / chunks, c = i - slot * chunks;
-                    const int tok = tile_tok(s_tile[slot >> 1], slot & 1);
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (tok >= 0) v = *reinterpret_cast<const uint4*>(a.xdig + static_cast<size_t>(tok) * 3 * H + 16 * c);
-                    const int d_ = (16 * c) / H, col = 16 * c - d_ * H;
-                    *reinterpret_cast<uint4*>(s_dig + (slot * 3 + d_) * dstride + col) = v;
+                for (int i0 = threadIdx.x; i0 < 2 * NT * chunks; i0 += 4 * kThreads) {
+                    uint4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * kThreads;
+                        v[u] = make_uint4(0u, 0u, 0u, 0u);
+                        if (i < 2 * NT * chunks) {
+                            const int slot = i / chunks, c = i - slot * chunks;
+                            const int tok = tile_tok(s_tile[slot >> 1], slot & 1);
+                            if (tok >= 0)
+                                v[u] = *reinterpret_cast<const uint4*>(a.xdig + static_cast<size_t>(tok) * 3 * H + 16 * c);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * kThreads;
+                        if (i < 2 * NT * chunks) {
+                            const int slot = i / chunks, c = i - slot * chunks;
+                            const int d_ = (16 * c) / H, col = 16 * c - d_ * H;
+                            *reinterpret_cast<uint4*>(s_dig + (slot * 3 + d_) * dstride + col) = v[u];
+                        }
+                    }
                 }
                 for (int i = threadIdx.x; i < 2 * NT * ng; i += kThreads) {
                     const int slot = i / ng, g = i - slot * ng;
@@ -449,18 +474,24 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tq = lane & 3;
-    const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     if (threadIdx.x == 0) {
         mbar_init(&s_bar, 1);
         fence_barrier_init();
     }
+    pdl_wait();   // work lists and activations come from the previous kernels
+    const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     __syncthreads();
     uint32_t phase = 0;
     const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
     const int dstride = Ly.dig_stride;
 
+    int4 desc = a.exp_desc[2 * (blockIdx.x / tiles_per_expert)];
+    int4 tile0 = a.exp_desc[2 * (blockIdx.x / tiles_per_expert) + 1];
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int4 desc = a.exp_desc[item / tiles_per_expert];
+        if (item != blockIdx.x) {
+            desc = a.exp_desc[2 * (item / tiles_per_expert)];
+            tile0 = a.exp_desc[2 * (item / tiles_per_expert) + 1];
+        }
         const int e = desc.x, kmax_e = desc.y, ntiles = desc.z, toff = desc.w;
         const int rt = item % tiles_per_expert;
         if (threadIdx.x == 0) {
@@ -485,34 +516,57 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
         }
         bool waited = false;
         for (int pass0 = 0; pass0 < ntiles; pass0 += NT) {
-            if (threadIdx.x < NT) {
+            if (NT == 1) {
+                if (threadIdx.x == 0) s_tile[0] = pass0 == 0 ? tile0 : a.tiles[toff + pass0];
+            } else if (threadIdx.x < NT) {
                 const int i = threadIdx.x;
                 s_tile[i] = pass0 + i < ntiles ? a.tiles[toff + pass0 + i] : make_int4(0, -1, -1, -1);
             }
             if (threadIdx.x == 0) s_nt = min(NT, ntiles - pass0);
             __syncthreads();
             const int nt = s_nt;
-            // fixed-point digits of the pass's h rows: one warp per (slot, group)
+            // fixed-point digits of the pass's h rows: one warp per (slot, group); a lane holds
+            // 4 consecutive values per 128-column chunk, all loaded before use
             for (int task = warp; task < 2 * NT * ng; task += kWarps) {
                 const int slot = task / ng, g = task - slot * ng;
                 const int4 t = s_tile[slot >> 1];
                 const int pos = (slot & 1) ? t.z : t.y;
                 if (pos < 0) continue;
                 const float* hrow = a.h + static_cast<size_t>(pos) * I + g * G;
+                float4 hv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = 128 * u + 4 * lane;
+                    hv[u] = j < G ? *reinterpret_cast<const float4*>(hrow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
                 float mx = 0.f;
-                for (int j = lane; j < G; j += 32) mx = fmaxf(mx, fabsf(hrow[j]));
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[u].x), fabsf(hv[u].y)), fmaxf(fabsf(hv[u].z), fabsf(hv[u].w))));
                 for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 const int Eg = group_exponent(mx);
                 int sum = 0;
-                for (int j = lane; j < G; j += 32) {
-                    const int X = to_fixed(hrow[j], Eg);
-                    sum += X;
-                    int8_t d0, d1, d2;
-                    split_digits(X, d0, d1, d2);
-                    int8_t* dst = s_dig + (slot * 3) * dstride + g * G + j;
-                    dst[0] = d0;
-                    dst[dstride] = d1;
-                    dst[2 * dstride] = d2;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = 128 * u + 4 * lane;
+                    if (j < G) {
+                        const float vv[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+                        uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int X = to_fixed(vv[q], Eg);
+                            sum += X;
+                            int8_t d0, d1, d2;
+                            split_digits(X, d0, d1, d2);
+                            p0 |= static_cast<uint32_t>(static_cast<uint8_t>(d0)) << (8 * q);
+                            p1 |= static_cast<uint32_t>(static_cast<uint8_t>(d1)) << (8 * q);
+                            p2 |= static_cast<uint32_t>(static_cast<uint8_t>(d2)) << (8 * q);
+                        }
+                        int8_t* dst = s_dig + (slot * 3) * dstride + g * G + j;
+                        *reinterpret_cast<uint32_t*>(dst) = p0;
+                        *reinterpret_cast<uint32_t*>(dst + dstride) = p1;
+                        *reinterpret_cast<uint32_t*>(dst + 2 * dstride) = p2;
+                    }
                 }
                 for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
                 if (lane == 0) { s_xe[slot * ng + g] = Eg; s_xs[slot * ng + g] = sum; }
@@ -712,7 +766,7 @@ cudaError_t launch_generic(void* fn, size_t smem, int items, int num_sms, const 
     const int grid = items < num_sms * per_sm ? items : num_sms * per_sm;
     GemvArgs copy = a;
     void* args[] = {&copy};
-    return cudaLaunchKernel(fn, dim3(grid), dim3(kThreads), args, smem, stream);
+    return launch_pdl_raw(fn, dim3(grid), dim3(kThreads), smem, stream, args);
 }
 
 }  // namespace

@@ -36,7 +36,7 @@ struct AllocArgs {
     // grouping outputs (do_permute)
     int do_permute;
     int32_t* pair_pos;        // [P] position of each pair in the (expert, k)-grouped order
-    int4* exp_desc;           // [E] per active expert: {expert, kmax, n_tiles, first tile}
+    int4* exp_desc;           // [E][2] per active expert: {expert, kmax, n_tiles, first tile}, first tile
     int4* tiles;              // [P + E*nk] two-token tiles: {k, posA, posB, tokA | tokB << 16}
     WsHeader* hdr;
 };
@@ -50,7 +50,7 @@ struct GemvArgs {
     uint64_t planes_per_expert, meta_per_expert;
     uint64_t planes_mat_off[3], meta_mat_off[3];
     int E, H, I, K, B, G, kmin, kmax, fmt;
-    const int4* exp_desc;     // per active expert {expert, kmax, n_tiles, first tile}
+    const int4* exp_desc;     // per active expert [2]: {expert, kmax, n_tiles, first tile}, first tile
     const int4* tiles;        // {k, posA, posB, tokA | tokB << 16}
     const int8_t* xdig;       // [T][3][H]
     const int32_t* xexp;      // [T][H/G]
@@ -88,5 +88,8 @@ struct SharedArgs {
     int T, S, H, I;
 };
 cudaError_t launch_shared(const SharedArgs& a, cudaStream_t stream);
+
+cudaError_t launch_residual_rmsnorm(const uint16_t* y, float* h, uint16_t* x, int T, int H, float eps,
+                                    cudaStream_t stream);
 
 }  // namespace dpa

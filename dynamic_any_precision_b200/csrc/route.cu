@@ -22,6 +22,7 @@ namespace dpa {
 namespace {
 
 constexpr int kRouteWarps = 8;
+constexpr int kPrefetch = 8;   // router-row uint4 loads a lane issues at once
 constexpr int16_t kNoBit = 0x3FFF;   // lowest-set-bit marker of a zero element
 
 // ---------------- fp64 exp (see header comment) ----------------
@@ -183,37 +184,69 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     const int part = warp % wpe;
     const uint16_t* xrow = a.x + static_cast<size_t>(t) * H;
 
+    // this warp's router-row loads go out first, so they overlap the staging of the token
+    const int e = blockIdx.x * (kRouteWarps / wpe) + warp / wpe;
+    const int wstride = 32 * wpe;                       // uint4 columns per round
+    const int nq = (H8 + wstride - 1) / wstride;
+    uint4 wpre[kPrefetch];
+    if (e < E) {
+        const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H);
+#pragma unroll
+        for (int u = 0; u < kPrefetch; ++u) {
+            const int col = u * wstride + part * 32 + lane;
+            if (u < nq && col < H8) wpre[u] = wrow[col];
+        }
+    }
+
+    // the token and the workspace may come from the previous kernel: wait for it from here on
+    pdl_wait();
+
+    // stage the token: each thread loads up to 4 x 8 elements with all loads issued first
     bool bad = false;
-    for (int j = threadIdx.x; j < H; j += blockDim.x) {
-        const uint16_t u = xrow[j];
-        const int q = (j & 7) * H8 + (j >> 3);
-        xd[q] = static_cast<double>(bf16_bits_to_float(u));
-        xl[q] = (u & 0x7FFF) ? static_cast<int16_t>(bf16_lsb(u)) : kNoBit;
-        xs[j] = u;
-        bad |= ((u >> 7) & 0xFF) == 0xFF;
+    for (int c0 = threadIdx.x; c0 < H8; c0 += 4 * blockDim.x) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 + u * blockDim.x;
+            if (c < H8) v[u] = reinterpret_cast<const uint4*>(xrow)[c];
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 + u * blockDim.x;   // 8-element group index
+            if (c < H8) {
+                const uint32_t ww[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    const uint16_t xu = static_cast<uint16_t>((ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu);
+                    const int q = h * H8 + c;
+                    xd[q] = static_cast<double>(bf16_bits_to_float(xu));
+                    xl[q] = (xu & 0x7FFF) ? static_cast<int16_t>(bf16_lsb(xu)) : kNoBit;
+                    bad |= ((xu >> 7) & 0xFF) == 0xFF;
+                }
+                reinterpret_cast<uint4*>(xs)[c] = v[u];
+            }
+        }
     }
     if (__syncthreads_or(bad) && threadIdx.x == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 1);
 
     // ---- wpe warps per expert logit: partial sums of products, lowest bits, magnitudes ----
-    const int e = blockIdx.x * (kRouteWarps / wpe) + warp / wpe;
     {
         double acc0 = 0.0, acc1 = 0.0, abs0 = 0.0, abs1 = 0.0;
         int lmin = 1 << 20;
         bool wbad = false;
         if (e < E) {
             const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H);
-            const int stride = 32 * wpe;                  // uint4 columns per round
-            const int nq = (H8 + stride - 1) / stride;
-            for (int q0 = 0; q0 < nq; q0 += 8) {
-                uint4 wv[8];
+            for (int q0 = 0; q0 < nq; q0 += kPrefetch) {
+                uint4 wv[kPrefetch];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int col = (q0 + u) * stride + part * 32 + lane;
-                    if (q0 + u < nq && col < H8) wv[u] = wrow[col];
+                for (int u = 0; u < kPrefetch; ++u) {
+                    const int col = (q0 + u) * wstride + part * 32 + lane;
+                    if (q0 == 0) wv[u] = wpre[u];
+                    else if (q0 + u < nq && col < H8) wv[u] = wrow[col];
                 }
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int col = (q0 + u) * stride + part * 32 + lane;   // 8-element group index
+                for (int u = 0; u < kPrefetch; ++u) {
+                    const int col = (q0 + u) * wstride + part * 32 + lane;   // 8-element group index
                     if (q0 + u < nq && col < H8) {
                         const uint32_t ww[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
 #pragma unroll
@@ -267,10 +300,10 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
         }
     }
 
-    // ---- block 0 of the token: fixed-point digits of x for the expert GEMV ----
-    if (a.xdig != nullptr && blockIdx.x == 0) {
+    // ---- fixed-point digits of x for the expert GEMV: the token's blocks share the groups ----
+    if (a.xdig != nullptr) {
         const int G = a.G, ng = H / G;
-        for (int g = warp; g < ng; g += kRouteWarps) {
+        for (int g = blockIdx.x + warp * gridDim.x; g < ng; g += gridDim.x * kRouteWarps) {
             float mx = 0.f;
             for (int j = lane; j < G; j += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_float(xs[g * G + j])));
             mx = warp_max_f(mx);
@@ -304,11 +337,16 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     __syncthreads();
     if (!s_last) return;
     if (threadIdx.x == 0) a.counters[t] = 0;   // ready for the next call
-    __threadfence();
 
+    // the other blocks fenced their logits before taking a ticket; read them from L2
     const double* lrow = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
-    double* vals = reinterpret_cast<double*>(smem_raw);   // reuse: [E] logits (token no longer needed)
-    for (int i = threadIdx.x; i < E; i += blockDim.x) vals[i] = __ldcg(lrow + i);
+    double* vals = reinterpret_cast<double*>(smem_raw);             // [E] logits (token no longer needed)
+    float* fk = reinterpret_cast<float*>(vals + E);                 // [E] fp32 roundings of the logits
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        const double v = __ldcg(lrow + i);
+        vals[i] = v;
+        fk[i] = v == v ? __double2float_rn(v) : -INFINITY;   // NaN is never larger
+    }
     __syncthreads();
     const int K = a.K;
     // rank of each expert = number of experts before it (descending logit, ties to the lower
@@ -323,11 +361,38 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
         if (c < E) {
             const double v = vals[c];
             if (v == v) {
-                const int j1 = min(E, (q + 1) * chunk);
-                for (int j = q * chunk; j < j1; ++j) {
-                    const double u = vals[j];
-                    rank += (u > v || (u == v && j < c)) ? 1 : 0;
+                // fp32 rounding is monotone: fk[j] > fk[c] implies vals[j] > vals[c]; only equal fp32
+                // values need the exact fp64 comparison (with ties to the lower expert id)
+                const float fv = fk[c];
+                const int j0 = q * chunk, j1 = min(E, (q + 1) * chunk);
+                int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+                int j = j0;
+                for (; j + 4 <= j1; j += 4) {   // four independent comparisons per iteration
+                    const float u0 = fk[j], u1 = fk[j + 1], u2 = fk[j + 2], u3 = fk[j + 3];
+                    r0 += u0 > fv ? 1 : 0;
+                    r1 += u1 > fv ? 1 : 0;
+                    r2 += u2 > fv ? 1 : 0;
+                    r3 += u3 > fv ? 1 : 0;
+                    if (u0 == fv || u1 == fv || u2 == fv || u3 == fv) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int jj = j + u;
+                            if (fk[jj] == fv && jj != c) {
+                                const double w = vals[jj];
+                                r0 += (w > v || (w == v && jj < c)) ? 1 : 0;
+                            }
+                        }
+                    }
                 }
+                for (; j < j1; ++j) {
+                    const float u = fk[j];
+                    r0 += u > fv ? 1 : 0;
+                    if (u == fv && j != c) {
+                        const double w = vals[j];
+                        r0 += (w > v || (w == v && j < c)) ? 1 : 0;
+                    }
+                }
+                rank = (r0 + r1) + (r2 + r3);
             } else {
                 rank = q == 0 ? E : 0;
             }
@@ -338,7 +403,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     __syncthreads();
     const double lmax = vals[s_sel[0]];
     if (threadIdx.x < K) s_num[threadIdx.x] = dexp_fixed(__dsub_rn(vals[s_sel[threadIdx.x]], lmax));
-    double* ex = vals + E;   // [E] exp values (norm over all experts)
+    double* ex = vals + 2 * E;   // [E] exp values (norm over all experts), after the fp32 keys
     if (!a.norm_topk)
         for (int i = threadIdx.x; i < E; i += blockDim.x) ex[i] = dexp_fixed(__dsub_rn(vals[i], lmax));
     __syncthreads();
@@ -367,7 +432,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
     const int epb = kRouteWarps / b.wpe;
     const int chunks = (a.E + epb - 1) / epb;
     size_t smem = static_cast<size_t>(a.H) * 12;              // fp64 token, lowest bits, bf16 copy
-    const size_t need_vals = static_cast<size_t>(a.E) * 16;   // logits and exps
+    const size_t need_vals = static_cast<size_t>(a.E) * 24;   // logits, keys and exps
     if (need_vals > smem) smem = need_vals;
     smem = (smem + 15) & ~static_cast<size_t>(15);
     if (smem > 48 * 1024) {
@@ -376,8 +441,8 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
         if (err != cudaSuccess) return err;
     }
     dim3 grid(chunks, a.T);
-    route_kernel<<<grid, kRouteWarps * 32, smem, stream>>>(b);
-    return cudaGetLastError();
+    void* args[] = {&b};
+    return launch_pdl_raw(reinterpret_cast<const void*>(route_kernel), grid, dim3(kRouteWarps * 32), smem, stream, args);
 }
 
 

@@ -13,7 +13,8 @@ from typing import Optional, Tuple
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libdpa_b200.so")
+# the in-tree build; DPA_LIB may name another build of the same library (e.g. a debug build)
+LIB_PATH = os.environ.get("DPA_LIB") or os.path.join(_PKG, "lib", "libdpa_b200.so")
 
 DPA_OK = 0
 STATUS_NAMES = {0: "DPA_OK", 1: "DPA_ERR_INVALID_ARG", 2: "DPA_ERR_UNSUPPORTED", 3: "DPA_ERR_WORKSPACE",
@@ -55,7 +56,7 @@ class Aux(ctypes.Structure):
 
 EXPORTED = ("dpa_encoded_sizes", "dpa_encode", "dpa_export_codes", "dpa_export_meta", "dpa_route",
             "dpa_allocate", "dpa_forward_workspace_size", "dpa_moe_forward", "dpa_device_status",
-            "dpa_status_string", "dpa_version")
+            "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm")
 
 _lib = None
 
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
     L.dpa_forward_workspace_size.restype = sz
     L.dpa_moe_forward.argtypes = [P(LayerDesc), P(LayerWeights), vp, i32, vp, vp, P(Aux), vp, sz, vp]
     L.dpa_device_status.argtypes = [vp, vp]
+    L.dpa_residual_rmsnorm.argtypes = [vp, vp, i32, i32, vp, vp]
     L.dpa_status_string.argtypes = [i32]
     L.dpa_status_string.restype = ctypes.c_char_p
     L.dpa_version.argtypes = []
@@ -256,6 +258,14 @@ def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] =
                                  _dptr(y), ctypes.byref(aux_s) if aux_s is not None else None, _dptr(ws), ws.numel(),
                                  _stream(stream)), "dpa_moe_forward")
     return y
+
+
+def residual_rmsnorm(h, x, y=None, stream=None):
+    """Stack glue: h += y (if given), x = bf16(RMSNorm(h)). h fp32 [T][H] (in place),
+    x and y bf16 bits [T][H] (int16 tensors)."""
+    T, H = h.shape
+    _check(lib().dpa_residual_rmsnorm(_dptr(y), _dptr(h), T, H, _dptr(x), _stream(stream)), "dpa_residual_rmsnorm")
+    return x
 
 
 def device_status(ws, stream=None) -> int:

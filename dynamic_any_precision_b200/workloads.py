@@ -96,14 +96,27 @@ def expert_weights(shape: LayerShape, e: int, seed: Optional[int] = None,
     return gate, up, down
 
 
-def all_expert_weights(shape: LayerShape, seed: Optional[int] = None):
-    """Stacked fp32 weights of every routed expert: gate [E][I][H], up [E][I][H], down [E][H][I]."""
+def all_expert_weights(shape: LayerShape, seed: Optional[int] = None, threads: int = 0):
+    """Stacked fp32 weights of every routed expert: gate [E][I][H], up [E][I][H], down [E][H][I].
+    Experts are drawn from their own keyed streams, so drawing them in parallel threads gives
+    the same values as drawing them one by one."""
+    from concurrent.futures import ThreadPoolExecutor
+    import os
     E, H, I = shape.n_experts, shape.hidden, shape.inter
     gate = np.empty((E, I, H), np.float32)
     up = np.empty((E, I, H), np.float32)
     down = np.empty((E, H, I), np.float32)
-    for e in range(E):
+
+    def fill(e):
         gate[e], up[e], down[e] = expert_weights(shape, e, seed)
+
+    n = threads or min(16, os.cpu_count() or 1)
+    if n <= 1 or E <= 2:
+        for e in range(E):
+            fill(e)
+    else:
+        with ThreadPoolExecutor(n) as ex:
+            list(ex.map(fill, range(E)))
     return gate, up, down
 
 

@@ -60,12 +60,13 @@ enum { DPA_MAT_GATE = 0, DPA_MAT_UP = 1, DPA_MAT_DOWN = 2 };
  *                             + (2^(B-k)-1)/2 - z).
  *            DPA_FMT_BCQ:     w = sum_{i<k} alpha_i * b_i, b_i in {-1,+1}, per-group fp16
  *                             alpha_i (binary-coded quantisation, greedy fit).
- *  bits      B, the stored planes (1..8).   kmin..kmax: planes a routed pair may read.
+ *  bits      B, the stored planes (1..4).   kmin..kmax: planes a routed pair may read.
  *  group     G, inputs per scale group.     norm_topk: 1 = softmax over the top_k
  *            selected logits, 0 = softmax over all experts (then the top_k values).
  *  n_shared  always-on experts run densely in bf16 (not allocated, not in the budget).
  * Supported by the kernels: hidden, inter multiples of 64 and of group; group a multiple
- * of 64; n_experts <= 1024; top_k <= 32; n_shared <= 8. */
+ * of 64 and at most 512; bits <= 4; n_experts <= 1024; top_k <= 32; n_shared <= 8; a work
+ * item's staging must fit in shared memory (else DPA_ERR_UNSUPPORTED). */
 typedef struct dpa_layer_desc {
     int32_t hidden, inter, n_experts, top_k, n_shared;
     int32_t format, bits, kmin, kmax, group, norm_topk;
@@ -219,6 +220,16 @@ size_t dpa_forward_workspace_size(const dpa_layer_desc* desc, int max_tokens);
 dpa_status dpa_moe_forward(const dpa_layer_desc* desc, const dpa_layer_weights* weights,
                            const void* x, int n_tokens, const double* target_bpw, void* y,
                            dpa_aux* aux, void* ws, size_t ws_bytes, void* stream);
+
+/* Glue between the layers of a stack of MoE layers (pre-norm residual):
+ *   h += y                     (skipped when y is NULL)
+ *   x  = bf16( h / sqrt(mean_j h_j^2 + 1e-6) )
+ * h: device fp32 [n_tokens][hidden], the residual stream (updated in place);
+ * y: device bf16 [n_tokens][hidden] (the previous layer's output) or NULL;
+ * x: device bf16 [n_tokens][hidden], the next layer's input. hidden must be a multiple of 4.
+ * The pages give no form for the glue; this is the plainest reading of a residual add and an
+ * RMSNorm (unit weight) between the layers. */
+dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidden, void* x, void* stream);
 
 /* Synchronise `stream`, read the device error flag in ws, clear it, and return it
  * (DPA_OK if no device error was recorded). */
