@@ -30,6 +30,7 @@ CU_SOURCES = {
     "route.cu": ["--fmad=false"],
     "allocate.cu": ["--fmad=false"],
     "gemv.cu": [],
+    "gemm_tc.cu": [],
     "combine.cu": [],
     "dpa_abi.cu": [],
     "route_noalloc.cu": [],

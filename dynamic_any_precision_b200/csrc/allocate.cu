@@ -392,26 +392,38 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         const int pos = atomicAdd(&s_counts[key], 1);
         s_sorted[pos] = p;
         a.pair_pos[p] = pos;
+        if (a.pos_tok) a.pos_tok[pos] = p / a.K;
     }
     __syncthreads();
     // per-expert descriptors and two-token tiles (tiles never straddle k classes); experts in
     // rounds of blockDim so that the active list stays in ascending expert order
-    int rank_base = 0, tile_base = 0;
+    int rank_base = 0, tile_base = 0, gt_base = 0;
     for (int e0 = 0; e0 < a.E; e0 += blockDim.x) {
         const int e = e0 + tid;
-        int km = 0, ntiles = 0;
+        int km = 0, ntiles = 0, ngt = 0;
         if (e < a.E) {
             for (int i = 0; i < nk; ++i) {
                 const int n = s_seg[e * nk + i + 1] - s_seg[e * nk + i];
                 if (n > 0) km = a.kmin + i;
                 ntiles += (n + 1) >> 1;
+                ngt += (n + kGemmTileTokens - 1) / kGemmTileTokens;
             }
         }
         const int flag = km > 0 ? 1 : 0;
         const int rank_incl = block_incl_scan(flag, s_tmp);
         const int tiles_incl = block_incl_scan(ntiles, s_tmp);
+        const int gt_incl = a.gtiles ? block_incl_scan(ngt, s_tmp) : 0;
         const int rank = rank_base + rank_incl - flag;
         const int tile_off = tile_base + tiles_incl - ntiles;
+        if (a.gtiles && ngt > 0) {   // token tiles of the prefill GEMMs: one (expert, k) class each
+            int t = gt_base + gt_incl - ngt;
+            for (int i = 0; i < nk; ++i) {
+                const int s0 = s_seg[e * nk + i];
+                const int n = s_seg[e * nk + i + 1] - s0;
+                for (int j = 0; j < n; j += kGemmTileTokens)
+                    a.gtiles[t++] = make_int4(e, a.kmin + i, s0 + j, min(kGemmTileTokens, n - j));
+            }
+        }
         if (flag) {
             a.exp_desc[2 * rank] = make_int4(e, km, ntiles, tile_off);
             int t = tile_off;
@@ -429,13 +441,17 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             }
         }
         // totals of this round (the last thread's inclusive sums), broadcast
-        if (tid == blockDim.x - 1) { s_tmp[0] = rank_incl; s_tmp[1] = tiles_incl; }
+        if (tid == blockDim.x - 1) { s_tmp[0] = rank_incl; s_tmp[1] = tiles_incl; s_tmp[2] = gt_incl; }
         __syncthreads();
         rank_base += s_tmp[0];
         tile_base += s_tmp[1];
+        gt_base += s_tmp[2];
         __syncthreads();
     }
-    if (tid == 0) a.hdr->n_active = static_cast<uint32_t>(rank_base);
+    if (tid == 0) {
+        a.hdr->n_active = static_cast<uint32_t>(rank_base);
+        a.hdr->n_gtiles = static_cast<uint32_t>(gt_base);
+    }
 }
 
 }  // namespace

@@ -9,12 +9,16 @@
 
 namespace dpa {
 
+// Tokens per tile of the prefill tensor-core GEMMs (the MMA's N extent at most).
+constexpr int kGemmTileTokens = 128;
+
 // ---- workspace header (first 256 bytes of every workspace) ----
 struct WsHeader {
     uint32_t error;       // first device error code (0 = none)
     uint32_t error_info;  // kernel-specific detail (which wait, which index)
     uint32_t n_active;    // routed experts with at least one pair in the last forward
-    uint32_t pad[61];
+    uint32_t n_gtiles;    // token tiles of the prefill GEMMs in the last forward (0 on the decode path)
+    uint32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 
@@ -48,6 +52,10 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void mbarrier_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {

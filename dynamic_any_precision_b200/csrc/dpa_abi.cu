@@ -41,7 +41,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
-        desc, tiles, total;
+        desc, tiles, gtiles, postok, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -75,6 +75,8 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.sh_out = take(4 * static_cast<size_t>(T) * H);
     L.desc = take(32 * E);
     L.tiles = take(16 * (P + E * nk));
+    L.gtiles = take(16 * (P / dpa::kGemmTileTokens + E * nk + 1));
+    L.postok = take(4 * P);
     L.total = off;
     return L;
 }
@@ -98,6 +100,42 @@ T* at(void* ws, size_t off) {
 }
 
 }  // namespace
+
+// Stage events of dpa_moe_forward: under stream capture they must be external event-record
+// nodes so that the replayed graph records them.
+struct StageMarks {
+    const dpa_aux* aux;
+    cudaStream_t s;
+    cudaStreamCaptureStatus cap;
+    void operator()(int i) const {
+        if (!aux || !aux->events[i]) return;
+        cudaEvent_t ev = static_cast<cudaEvent_t>(aux->events[i]);
+        if (cap == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+        else cudaEventRecord(ev, s);
+    }
+};
+
+// 5. combine: y[t] = bf16(sum over slots in order of gate * expert output (+ shared experts))
+static dpa_status combine_stage(const dpa_layer_desc* d, const dpa_layer_weights* w, const double* gate, int T,
+                                const dpa_aux* aux, void* y, void* ws, const WsLayout& L, dpa::WsHeader* hdr,
+                                cudaStream_t s, const StageMarks& mark) {
+    (void)w;
+    const int K = d->top_k;
+    dpa::CombineArgs ca{};
+    ca.out_pair = at<float>(ws, L.out_pair);
+    ca.pair_pos = at<int32_t>(ws, L.pairpos);
+    ca.gate = gate;
+    ca.shared_out = d->n_shared > 0 ? at<float>(ws, L.sh_out) : nullptr;
+    ca.pair_out_user = aux ? aux->pair_out : nullptr;
+    ca.y = static_cast<uint16_t*>(y);
+    ca.T = T;
+    ca.K = K;
+    ca.H = d->hidden;
+    ca.hdr = hdr;
+    if (dpa::launch_combine(ca, s) != cudaSuccess) return DPA_ERR_CUDA;
+    mark(6);
+    return DPA_OK;
+}
 
 extern "C" {
 
@@ -183,7 +221,8 @@ dpa_status dpa_route(const dpa_layer_desc* d, const void* x, int n_tokens, const
 
 static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, const int32_t* idx,
                                 const double* gate, int T, const double* target, uint8_t* k_out,
-                                double* lambda_out, void* ws, const WsLayout& L, bool permute, cudaStream_t s) {
+                                double* lambda_out, void* ws, const WsLayout& L, bool permute, cudaStream_t s,
+                                bool gemm_tiles = false) {
     dpa::AllocArgs a{};
     a.rtable = rtable;
     a.idx = idx;
@@ -202,6 +241,8 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.pair_pos = at<int32_t>(ws, L.pairpos);
     a.exp_desc = at<int4>(ws, L.desc);
     a.tiles = at<int4>(ws, L.tiles);
+    a.gtiles = gemm_tiles ? at<int4>(ws, L.gtiles) : nullptr;
+    a.pos_tok = gemm_tiles ? at<int32_t>(ws, L.postok) : nullptr;
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
     return dpa::launch_allocate(a, s) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
 }
@@ -243,6 +284,13 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     dpa_encoded_sizes(d, &sz);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int T = n_tokens, K = d->top_k;
+    const int path = aux ? aux->expert_path : DPA_PATH_AUTO;
+    if (path < DPA_PATH_AUTO || path > DPA_PATH_TC) return DPA_ERR_INVALID_ARG;
+    const bool tc_shape = d->format == DPA_FMT_UNIFORM && d->hidden % 128 == 0 && d->inter % 64 == 0;
+    if (path == DPA_PATH_TC && !tc_shape) return DPA_ERR_UNSUPPORTED;
+    const bool use_tc = path == DPA_PATH_TC ||
+                        (path == DPA_PATH_AUTO && tc_shape &&
+                         static_cast<long long>(T) * K >= static_cast<long long>(DPA_TC_MIN_PAIRS_PER_EXPERT) * d->n_experts);
 
     int32_t* idx = (aux && aux->topk_idx) ? aux->topk_idx : at<int32_t>(ws, L.idx);
     double* gate = (aux && aux->topk_gate) ? aux->topk_gate : at<double>(ws, L.gate);
@@ -250,16 +298,9 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     double* lam = (aux && aux->lambda) ? aux->lambda : at<double>(ws, L.lambda);
     dpa::WsHeader* hdr = at<dpa::WsHeader>(ws, L.hdr);
 
-    // stage events: under stream capture they must be external event-record nodes so that the
-    // replayed graph records them
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (aux) cudaStreamIsCapturing(s, &cap);
-    auto mark = [&](int i) {
-        if (!aux || !aux->events[i]) return;
-        cudaEvent_t ev = static_cast<cudaEvent_t>(aux->events[i]);
-        if (cap == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
-        else cudaEventRecord(ev, s);
-    };
+    const StageMarks mark{aux, s, cap};
     mark(0);
     // 1. route (+ fixed-point digits of x)
     dpa::RouteArgs ra{};
@@ -284,7 +325,7 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     mark(1);
 
     // 2. allocate + group pairs by (expert, k)
-    dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s);
+    dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s, use_tc);
     if (st2 != DPA_OK) return st2;
     mark(2);
 
@@ -306,6 +347,33 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     mark(3);
 
     // 4. variable-plane expert FFN
+    const int sms = num_sms_current();
+    if (use_tc) {
+        dpa::GemmArgs ta{};
+        ta.planes = static_cast<const uint8_t*>(w->planes);
+        ta.meta = static_cast<const uint8_t*>(w->meta);
+        ta.planes_per_expert = sz.planes_per_expert;
+        ta.meta_per_expert = sz.meta_per_expert;
+        for (int m = 0; m < 3; ++m) {
+            ta.planes_mat_off[m] = sz.planes_matrix_offset[m];
+            ta.meta_mat_off[m] = sz.meta_matrix_offset[m];
+        }
+        ta.H = d->hidden;
+        ta.I = d->inter;
+        ta.B = d->bits;
+        ta.G = d->group;
+        ta.gtiles = at<int4>(ws, L.gtiles);
+        ta.pos_tok = at<int32_t>(ws, L.postok);
+        ta.x = static_cast<const uint16_t*>(x);
+        ta.hbuf = at<uint16_t>(ws, L.h);
+        ta.out_pair = at<float>(ws, L.out_pair);
+        ta.hdr = hdr;
+        if (dpa::launch_gemm_gateup(ta, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
+        mark(4);
+        if (dpa::launch_gemm_down(ta, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
+        mark(5);
+        return combine_stage(d, w, gate, T, aux, y, ws, L, hdr, s, mark);
+    }
     dpa::GemvArgs ga{};
     ga.planes = static_cast<const uint8_t*>(w->planes);
     ga.meta = static_cast<const uint8_t*>(w->meta);
@@ -335,27 +403,11 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     const int P = T * K;
     ga.max_items = P < d->n_experts ? P : d->n_experts;
     ga.max_tokens_per_expert = T;
-    const int sms = num_sms_current();
     if (dpa::launch_gateup(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(4);
     if (dpa::launch_down(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(5);
-
-    // 5. combine
-    dpa::CombineArgs ca{};
-    ca.out_pair = at<float>(ws, L.out_pair);
-    ca.pair_pos = at<int32_t>(ws, L.pairpos);
-    ca.gate = gate;
-    ca.shared_out = d->n_shared > 0 ? at<float>(ws, L.sh_out) : nullptr;
-    ca.pair_out_user = aux ? aux->pair_out : nullptr;
-    ca.y = static_cast<uint16_t*>(y);
-    ca.T = T;
-    ca.K = K;
-    ca.H = d->hidden;
-    ca.hdr = hdr;
-    if (dpa::launch_combine(ca, s) != cudaSuccess) return DPA_ERR_CUDA;
-    mark(6);
-    return DPA_OK;
+    return combine_stage(d, w, gate, T, aux, y, ws, L, hdr, s, mark);
 }
 
 dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidden, void* x, void* stream) {

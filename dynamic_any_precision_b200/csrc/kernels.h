@@ -38,11 +38,31 @@ struct AllocArgs {
     int32_t* pair_pos;        // [P] position of each pair in the (expert, k)-grouped order
     int4* exp_desc;           // [E][2] per active expert: {expert, kmax, n_tiles, first tile}, first tile
     int4* tiles;              // [P + E*nk] two-token tiles: {k, posA, posB, tokA | tokB << 16}
+    int4* gtiles;             // nullptr, or [P/kGemmTileTokens + E*nk] GEMM token tiles {e, k, pos0, n}
+    int32_t* pos_tok;         // nullptr, or [P] token of each grouped position
     WsHeader* hdr;
 };
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream);
 size_t allocate_smem_bytes(int P, int E, int nk);
 int allocate_threads(int P);
+
+// Prefill expert FFN on tcgen05: grouped GEMMs over the GEMM token tiles of the allocation.
+struct GemmArgs {
+    const uint8_t* planes;    // encoded layer (uniform format)
+    const uint8_t* meta;
+    uint64_t planes_per_expert, meta_per_expert;
+    uint64_t planes_mat_off[3], meta_mat_off[3];
+    int H, I, B, G;
+    const int4* gtiles;       // {e, k, pos0, n}, count in hdr->n_gtiles
+    const int32_t* pos_tok;   // [P] token of each grouped position
+    const uint16_t* x;        // [T][H] bf16 activations
+    uint16_t* hbuf;           // [P][I] fp16 SwiGLU outputs, grouped order
+    float* out_pair;          // [P][H] per-pair expert outputs, grouped order
+    WsHeader* hdr;
+};
+cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t stream, int sms);
+cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t stream, int sms);
+size_t gemm_tc_smem_bytes();
 
 struct GemvArgs {
     const uint8_t* planes;    // encoded layer

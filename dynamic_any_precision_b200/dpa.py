@@ -51,7 +51,9 @@ class LayerWeights(ctypes.Structure):
 class Aux(ctypes.Structure):
     _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_gate", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("lambda_", ctypes.c_void_p), ("pair_out", ctypes.c_void_p),
-                ("events", ctypes.c_void_p * 7)]
+                ("events", ctypes.c_void_p * 7), ("expert_path", ctypes.c_int32)]
+
+PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 
 
 EXPORTED = ("dpa_encoded_sizes", "dpa_encode", "dpa_export_codes", "dpa_export_meta", "dpa_route",
@@ -239,8 +241,9 @@ class DeviceLayer:
 def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] = None, stream=None):
     """One MoE layer. x: CUDA int16/bf16 bits [T][H]; target: CUDA fp64 scalar tensor.
     aux: optional dict of preallocated CUDA tensors with keys topk_idx, topk_gate, k, lambda,
-    pair_out, and/or "events": up to 7 torch.cuda.Event(enable_timing=True) recorded at the
-    stage boundaries. Returns y (int16 bf16 bits [T][H])."""
+    pair_out, "events": up to 7 torch.cuda.Event(enable_timing=True) recorded at the
+    stage boundaries, and "expert_path" (PATH_AUTO, PATH_GEMV or PATH_TC).
+    Returns y (int16 bf16 bits [T][H])."""
     import torch
     T = x.shape[0]
     if y is None:
@@ -254,6 +257,7 @@ def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] =
                 if not ev.cuda_event:
                     raise ValueError("record a torch.cuda.Event once before passing it (lazy creation)")
                 aux_s.events[i] = ev.cuda_event
+        aux_s.expert_path = int(aux.get("expert_path", PATH_AUTO))
     _check(lib().dpa_moe_forward(ctypes.byref(layer.desc), ctypes.byref(layer.weights), _dptr(x), T, _dptr(target),
                                  _dptr(y), ctypes.byref(aux_s) if aux_s is not None else None, _dptr(ws), ws.numel(),
                                  _stream(stream)), "dpa_moe_forward")

@@ -120,7 +120,20 @@ typedef struct dpa_layer_weights {
  * stage boundaries of dpa_moe_forward: [0] before routing, [1] after routing, [2] after
  * allocation and grouping, [3] after the shared experts, [4] after the gate/up GEMV,
  * [5] after the down GEMV, [6] after the combine. Recording also works under stream
- * capture, so per-stage device times can be read from a replayed CUDA graph. */
+ * capture, so per-stage device times can be read from a replayed CUDA graph. On the
+ * tensor-core path [4] and [5] follow the gate/up and down GEMMs.
+ * expert_path: which kernels run the routed experts' FFN (same results up to the
+ * rounding of fp32 accumulation and of the fp16 SwiGLU intermediate on the tensor-core path):
+ *   DPA_PATH_AUTO (0)  tensor-core GEMMs when the format is uniform, hidden % 128 == 0,
+ *                      inter % 64 == 0 and the batch routes at least DPA_TC_MIN_PAIRS_PER_EXPERT
+ *                      pairs per expert on average (T*top_k >= that * n_experts); else GEMV;
+ *   DPA_PATH_GEMV (1)  the batched GEMV kernels (any shape check_desc accepts);
+ *   DPA_PATH_TC (2)    the tcgen05 grouped GEMMs (DPA_ERR_UNSUPPORTED when the shape does
+ *                      not qualify as above, minus the pairs-per-expert condition). */
+#define DPA_PATH_AUTO 0
+#define DPA_PATH_GEMV 1
+#define DPA_PATH_TC 2
+#define DPA_TC_MIN_PAIRS_PER_EXPERT 16
 typedef struct dpa_aux {
     int32_t* topk_idx;
     double* topk_gate;
@@ -128,6 +141,7 @@ typedef struct dpa_aux {
     double* lambda;
     float* pair_out;
     void* events[7];
+    int32_t expert_path;
 } dpa_aux;
 
 /* Validate a descriptor and return the encoded sizes. Host only. */

@@ -45,7 +45,7 @@ class GpuLayer:
         self.layer = dpa.DeviceLayer.from_host(self.desc, planes, meta, r, self.wr, sh)
         self.planes_host = planes
 
-    def forward(self, x_bits, target, ws=None, with_pairs=True):
+    def forward(self, x_bits, target, ws=None, with_pairs=True, path=dpa.PATH_AUTO):
         T = x_bits.shape[0]
         K = self.shape.top_k
         x = torch.from_numpy(x_bits.view(np.int16)).cuda()
@@ -54,19 +54,20 @@ class GpuLayer:
         aux = {"topk_idx": torch.empty((T, K), dtype=torch.int32, device="cuda"),
                "topk_gate": torch.empty((T, K), dtype=torch.float64, device="cuda"),
                "k": torch.empty((T, K), dtype=torch.uint8, device="cuda"),
-               "lambda": torch.empty(1, dtype=torch.float64, device="cuda")}
+               "lambda": torch.empty(1, dtype=torch.float64, device="cuda"),
+               "expert_path": path}
         if with_pairs:
             aux["pair_out"] = torch.empty((T, K, self.shape.hidden), dtype=torch.float32, device="cuda")
         y = dpa.moe_forward(self.layer, x, tg, ws, aux=aux)
         st = dpa.device_status(ws)
         assert st == 0, dpa.STATUS_NAMES.get(st, st)
-        out = {k: v.cpu().numpy() for k, v in aux.items()}
+        out = {k: v.cpu().numpy() for k, v in aux.items() if k != "expert_path"}
         return bits_to_f64(y), out, ws
 
 
-def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None):
+def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None, path=dpa.PATH_AUTO, pair_tol=1e-3):
     gl = GpuLayer.get(shape)
-    y, aux, _ = gl.forward(x_bits, target)
+    y, aux, _ = gl.forward(x_bits, target, path=path)
     y_ref, ref = reference_layer(shape, x_bits, target, token_subset=token_subset)
     assert np.array_equal(aux["topk_idx"], ref["idx"])
     assert np.array_equal(aux["topk_gate"], ref["gates"])       # bit-identical fp64
@@ -78,7 +79,7 @@ def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None):
     if sample_pairs is not None:
         ref_o = pair_outputs(shape, x_bits, ref, sample_pairs)
         for (t, j), o in ref_o.items():
-            ok, worst = within_tol(aux["pair_out"][t, j].astype(np.float64), o, 1e-3)
+            ok, worst = within_tol(aux["pair_out"][t, j].astype(np.float64), o, pair_tol)
             assert ok, (t, j, worst)
     # the achieved average never exceeds the target
     assert aux["k"].astype(np.int64).sum() <= target * aux["k"].size
