@@ -32,6 +32,11 @@ namespace {
 constexpr int kAllocThreads = 1024;       // maximum block size
 constexpr int kSmemCostDoubles = 8192;    // costs kept in shared memory up to this many
 constexpr int kSmallP = 64;               // up to this many pairs one warp runs the bisection
+constexpr int kCoopThreads = 512;         // grid-wide bisection: threads per CTA
+constexpr int kCoopMaxPairsPerBlock = 6144;   // shared-memory costs: 6144 pairs x 32 B = 192 KB per CTA
+constexpr int kCoopDepth = 6;             // bisection steps per grid round (63 midpoints)
+constexpr int kCoopMinPairs = 2048;       // below this the single-CTA bisection is faster
+static_assert((64 + kCoopDepth - 1) / kCoopDepth <= kCoopRoundsMax, "round counters");
 
 __device__ __forceinline__ int choose_k(const double* c, int nk, int kmin, double lam) {
     double best = __dadd_rn(c[0], __dmul_rn(lam, static_cast<double>(kmin)));
@@ -140,10 +145,19 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     const int any_bad_e = __syncthreads_or(bad_e);
     if (any_bad_e && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 11);
     if (bad || any_bad_e) {
-        if (a.do_permute && tid == 0) a.hdr->n_active = 0;
+        if (a.do_permute && tid == 0) {   // nothing downstream may read a previous call's work lists
+            a.hdr->n_active = 0;
+            a.hdr->n_gtiles = 0;
+        }
         return;
     }
 
+    if (a.k_given) {   // plane counts (and lambda) already chosen by the grid-wide bisection
+        for (int p = tid; p < P; p += blockDim.x) s_k[p] = a.k_out[p];
+        __syncthreads();
+        goto grouping;
+    }
+    {
     // costs c[p][i] = fl(g_p * r_{e_p}(kmin + i)); the rtable loads of a pair are issued together
     double mx = 0.0;
     for (int p = tid; p < P; p += blockDim.x) {
@@ -361,6 +375,8 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         s_k[p] = static_cast<uint8_t>(k);
     }
     if (tid == 0 && a.lambda_out) *a.lambda_out = hi;
+    }
+grouping:
     if (!a.do_permute) return;
 
     // ---------------- grouping by (expert, k), all in shared memory ----------------
@@ -454,22 +470,198 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     }
 }
 
+// ---------------- grid-wide bisection for large batches ----------------
+// The same 64 exact steps, evaluated by every SM: each CTA keeps the costs of its share of the
+// pairs in shared memory; a round computes N(mid) for the 2^D - 1 midpoints the next D
+// steps can visit (integer sums, so the order of the additions does not matter), a bounded
+// grid barrier publishes the counts, and every thread walks the tree with the exact predicates.
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// All CTAs of the (cooperatively launched, hence co-resident) grid arrive; false on timeout.
+__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned target, WsHeader* hdr, int* s_flag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        bool ok = true;
+        if (ld_acquire_u32(ctr) < target) {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire_u32(ctr) < target) {
+                if (globaltimer() - t0 > kWaitNs) {
+                    set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, 0x240);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        *s_flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+__global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a, CoopSync* cs, int per_block) {
+    // this CTA's pairs [p0, p1) with their costs in shared memory; warp w evaluates the
+    // midpoints w+1, w+1+nw, ... over all of them (lanes stride the pairs)
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    double* s_c = reinterpret_cast<double*>(smem_raw);   // [per_block][4]
+    __shared__ double s_mid[64];
+    __shared__ double s_red[kCoopThreads / 32];
+    __shared__ int s_flag;
+    const int P = a.T * a.K;
+    const int nk = a.kmax - a.kmin + 1;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const unsigned G = gridDim.x;
+    const int p0 = blockIdx.x * per_block, p1 = min(P, p0 + per_block), np = max(0, p1 - p0);
+
+    const double target = *a.target;
+    if (!(target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax))) {
+        if (blockIdx.x == 0 && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 10);
+        return;   // every CTA reads the same target: the whole grid leaves here
+    }
+    double mx = 0.0;
+    int bad_e = 0;
+    for (int j = tid; j < np; j += blockDim.x) {
+        const int p = p0 + j;
+        const int e = a.idx[p];
+        double c[4] = {0.0, 0.0, 0.0, 0.0};
+        if (e < 0 || e >= a.E) {
+            bad_e = 1;
+        } else {
+            const double g = a.gate[p];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (i < nk) c[i] = __dmul_rn(g, a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)]);
+            mx = fmax(mx, c[0]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) s_c[4 * j + i] = c[i];
+    }
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_red[warp] = mx;
+    const int any_bad = __syncthreads_or(bad_e);
+    if (tid == 0) {
+        double m = s_red[0];
+        for (int w = 1; w < nw; ++w) m = fmax(m, s_red[w]);
+        // costs are >= 0, so their bit patterns order like their values
+        atomicMax(&cs->mx_bits, static_cast<unsigned long long>(__double_as_longlong(m)));
+        if (any_bad) atomicOr(&cs->bad, 1u);
+    }
+    unsigned phase = 1;
+    if (!grid_barrier(&cs->barrier, G * phase++, a.hdr, &s_flag)) return;
+    if (__ldcg(&cs->bad)) {
+        if (blockIdx.x == 0 && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 11);
+        return;
+    }
+    mx = __longlong_as_double(static_cast<long long>(__ldcg(&cs->mx_bits)));
+    const double budget = __dmul_rn(target, static_cast<double>(P));
+    double lo = 0.0;
+    double hi = __dadd_rn(__dmul_rn(2.0, mx), 1.0);
+
+    int round = 0;
+    for (int it = 0; it < 64; ++round) {
+        const int D = min(kCoopDepth, 64 - it);
+        const int n_nodes = (1 << D) - 1;
+        if (tid < n_nodes) {   // midpoint of heap node tid + 1: replay its path from the root
+            const int node = tid + 1;
+            const int depth = 31 - __clz(node);
+            double l = lo, h = hi;
+            for (int lev = depth - 1; lev >= 0; --lev) {
+                const double m = midpoint(l, h);
+                if ((node >> lev) & 1) l = m; else h = m;
+            }
+            s_mid[node] = midpoint(l, h);
+        }
+        __syncthreads();
+        for (int node = warp + 1; node <= n_nodes; node += nw) {
+            const double m = s_mid[node];
+            int n = 0;
+            for (int j = lane; j < np; j += 32) {
+                const double* c = s_c + 4 * j;
+                double best = __dadd_rn(c[0], __dmul_rn(m, static_cast<double>(a.kmin)));
+                int kb = a.kmin;
+                for (int i = 1; i < nk; ++i) {
+                    const double cost = __dadd_rn(c[i], __dmul_rn(m, static_cast<double>(a.kmin + i)));
+                    if (cost < best) { best = cost; kb = a.kmin + i; }
+                }
+                n += kb;
+            }
+            n = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n)));
+            if (lane == 0 && n) atomicAdd(&cs->counts[round][node][0], n);
+        }
+        if (!grid_barrier(&cs->barrier, G * phase++, a.hdr, &s_flag)) return;
+        int nd = 1;
+        for (int lev = 0; lev < D; ++lev) {
+            const int n = __ldcg(&cs->counts[round][nd][0]);
+            const int pr = static_cast<double>(n) > budget ? 1 : 0;
+            const double m = midpoint(lo, hi);
+            if (pr) lo = m; else hi = m;
+            nd = 2 * nd + pr;
+        }
+        it += D;
+    }
+    for (int j = tid; j < np; j += blockDim.x) {
+        const double* c = s_c + 4 * j;
+        double best = __dadd_rn(c[0], __dmul_rn(hi, static_cast<double>(a.kmin)));
+        int kb = a.kmin;
+        for (int i = 1; i < nk; ++i) {
+            const double cost = __dadd_rn(c[i], __dmul_rn(hi, static_cast<double>(a.kmin + i)));
+            if (cost < best) { best = cost; kb = a.kmin + i; }
+        }
+        a.k_out[p0 + j] = static_cast<uint8_t>(kb);
+    }
+    if (blockIdx.x == 0 && tid == 0 && a.lambda_out) *a.lambda_out = hi;
+}
+
 }  // namespace
 
 size_t allocate_smem_bytes(int P, int E, int nk) { return alloc_smem_layout(P, E, nk).total; }
 
 int allocate_threads(int P) { return P <= kSmallP ? 128 : kAllocThreads; }   // small: 4 warps x 8 nodes
 
-cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream) {
+cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* coop, int sms) {
     const int nk = a.kmax - a.kmin + 1;
     const int P = a.T * a.K;
+    AllocArgs b = a;
+    const int coop_blocks = sms > 0 ? (P / 64 < sms ? (P + 63) / 64 : sms) : 1;
+    int per_block = (P + coop_blocks - 1) / coop_blocks;
+    if (coop && P > kCoopMinPairs && per_block <= kCoopMaxPairsPerBlock) {
+        // grid-wide bisection: the pairs split over (at most) every SM, costs in shared memory
+        const int blocks = coop_blocks;
+        const size_t smem = static_cast<size_t>(per_block) * 32;
+        cudaError_t err = cudaMemsetAsync(coop, 0, sizeof(CoopSync), stream);
+        if (err != cudaSuccess) return err;
+        if (smem > 48 * 1024) {
+            err = cudaFuncSetAttribute(allocate_coop_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+            if (err != cudaSuccess) return err;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(blocks);
+        cfg.blockDim = dim3(kCoopThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        void* cargs[] = {&b, &coop, &per_block};
+        err = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(allocate_coop_kernel), cargs);
+        if (err != cudaSuccess) return err;
+        b.k_given = 1;
+    }
     const size_t smem = allocate_smem_bytes(P, a.E, nk);
     if (smem > 48 * 1024) {
         cudaError_t err = cudaFuncSetAttribute(allocate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
         if (err != cudaSuccess) return err;
     }
-    AllocArgs b = a;
     void* args[] = {&b};
     return launch_pdl_raw(reinterpret_cast<const void*>(allocate_kernel), dim3(1), dim3(allocate_threads(P)), smem,
                           stream, args);

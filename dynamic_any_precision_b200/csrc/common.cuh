@@ -70,13 +70,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended (not spinning, so issuing nothing) for up to
+// `ns` nanoseconds while the phase is incomplete.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of `bar` with a time limit. Returns false on timeout (after
 // recording the error). The caller must not read the buffers the barrier guards then.
+// While waiting, the thread sleeps in the barrier for up to 20 us per try instead of spinning.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, WsHeader* hdr,
                                                   uint32_t where) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_suspend(bar, parity, 20000u)) {
         if (globaltimer() - t0 > kWaitNs) {
             set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
             return false;

@@ -41,7 +41,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
-        desc, tiles, gtiles, postok, total;
+        desc, tiles, gtiles, postok, coop, rstats, xperm, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -77,6 +77,9 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.tiles = take(16 * (P + E * nk));
     L.gtiles = take(16 * (P / dpa::kGemmTileTokens + E * nk + 1));
     L.postok = take(4 * P);
+    L.coop = take(sizeof(dpa::CoopSync));
+    L.rstats = take((8 + 2 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 16);
+    L.xperm = take(2 * P * H);
     L.total = off;
     return L;
 }
@@ -135,6 +138,16 @@ static dpa_status combine_stage(const dpa_layer_desc* d, const dpa_layer_weights
     if (dpa::launch_combine(ca, s) != cudaSuccess) return DPA_ERR_CUDA;
     mark(6);
     return DPA_OK;
+}
+
+// Per-row exactness statistics of the large-batch router, carved from the workspace.
+static void set_route_stats(dpa::RouteArgs& r, void* ws, const WsLayout& L, int T, int E) {
+    unsigned char* base = at<unsigned char>(ws, L.rstats);
+    r.n2_x = reinterpret_cast<double*>(base);
+    r.n2_w = r.n2_x + T;
+    const size_t lsb_off = (8 * (static_cast<size_t>(T) + E) + 15) & ~static_cast<size_t>(15);
+    r.lsb_x = reinterpret_cast<int16_t*>(base + lsb_off);   // 16-byte aligned rows of H/64 entries
+    r.lsb_w = r.lsb_x + static_cast<size_t>(T) * (r.H / 64);
 }
 
 extern "C" {
@@ -216,7 +229,9 @@ dpa_status dpa_route(const dpa_layer_desc* d, const void* x, int n_tokens, const
     a.counters = at<unsigned>(ws, L.counters);
     a.xdig = nullptr;
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
-    return dpa::launch_route(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
+    set_route_stats(a, ws, L, n_tokens, d->n_experts);
+    return dpa::launch_route(a, static_cast<cudaStream_t>(stream), num_sms_current()) == cudaSuccess ? DPA_OK
+                                                                                                 : DPA_ERR_CUDA;
 }
 
 static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, const int32_t* idx,
@@ -244,7 +259,8 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.gtiles = gemm_tiles ? at<int4>(ws, L.gtiles) : nullptr;
     a.pos_tok = gemm_tiles ? at<int32_t>(ws, L.postok) : nullptr;
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
-    return dpa::launch_allocate(a, s) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
+    return dpa::launch_allocate(a, s, at<dpa::CoopSync>(ws, L.coop), num_sms_current()) == cudaSuccess ? DPA_OK
+                                                                                                  : DPA_ERR_CUDA;
 }
 
 dpa_status dpa_allocate(const dpa_layer_desc* d, const double* rtable, const int32_t* topk_idx,
@@ -286,7 +302,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     const int T = n_tokens, K = d->top_k;
     const int path = aux ? aux->expert_path : DPA_PATH_AUTO;
     if (path < DPA_PATH_AUTO || path > DPA_PATH_TC) return DPA_ERR_INVALID_ARG;
-    const bool tc_shape = d->format == DPA_FMT_UNIFORM && d->hidden % 128 == 0 && d->inter % 64 == 0;
+    const bool tc_shape = d->format == DPA_FMT_UNIFORM && d->hidden % 256 == 0 && d->inter % 256 == 0 &&
+                          (d->group & (d->group - 1)) == 0;   // scale groups of 64 * 2^n inputs
     if (path == DPA_PATH_TC && !tc_shape) return DPA_ERR_UNSUPPORTED;
     const bool use_tc = path == DPA_PATH_TC ||
                         (path == DPA_PATH_AUTO && tc_shape &&
@@ -317,11 +334,12 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     ra.idx = idx;
     ra.gate = gate;
     ra.counters = at<unsigned>(ws, L.counters);
-    ra.xdig = at<int8_t>(ws, L.xdig);
+    ra.xdig = use_tc ? nullptr : at<int8_t>(ws, L.xdig);   // the tensor-core path reads x directly
     ra.xexp = at<int32_t>(ws, L.xexp);
     ra.xsum = at<int32_t>(ws, L.xsum);
     ra.hdr = hdr;
-    if (dpa::launch_route(ra, s) != cudaSuccess) return DPA_ERR_CUDA;
+    set_route_stats(ra, ws, L, T, d->n_experts);
+    if (dpa::launch_route(ra, s, num_sms_current()) != cudaSuccess) return DPA_ERR_CUDA;
     mark(1);
 
     // 2. allocate + group pairs by (expert, k)
@@ -362,12 +380,17 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
         ta.I = d->inter;
         ta.B = d->bits;
         ta.G = d->group;
+        ta.T = T;
+        ta.P = T * K;
         ta.gtiles = at<int4>(ws, L.gtiles);
         ta.pos_tok = at<int32_t>(ws, L.postok);
         ta.x = static_cast<const uint16_t*>(x);
+        ta.xperm = at<uint16_t>(ws, L.xperm);
+        ta.E = d->n_experts;
         ta.hbuf = at<uint16_t>(ws, L.h);
         ta.out_pair = at<float>(ws, L.out_pair);
         ta.hdr = hdr;
+        if (dpa::launch_permute_rows(ta, s) != cudaSuccess) return DPA_ERR_CUDA;
         if (dpa::launch_gemm_gateup(ta, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
         mark(4);
         if (dpa::launch_gemm_down(ta, s, sms) != cudaSuccess) return DPA_ERR_CUDA;

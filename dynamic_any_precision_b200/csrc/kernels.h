@@ -21,8 +21,13 @@ struct RouteArgs {
     int32_t* xsum;            // [T][H/G]
     WsHeader* hdr;
     int wpe;                  // warps per expert (set by the launcher)
+    // large-batch path (nullptr: always the per-logit kernel): per-row exactness statistics
+    int16_t* lsb_x;           // [T][H/64] lowest set bit over each 64-input block's nonzero elements
+    double* n2_x;             // [T] sum of squares
+    int16_t* lsb_w;           // [E][H/64]
+    double* n2_w;             // [E]
 };
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream);
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms = 148);
 
 struct AllocArgs {
     const double* rtable;     // [E][B]
@@ -38,11 +43,21 @@ struct AllocArgs {
     int32_t* pair_pos;        // [P] position of each pair in the (expert, k)-grouped order
     int4* exp_desc;           // [E][2] per active expert: {expert, kmax, n_tiles, first tile}, first tile
     int4* tiles;              // [P + E*nk] two-token tiles: {k, posA, posB, tokA | tokB << 16}
+    int k_given;              // 1: k_out already holds the plane counts (grid-wide bisection ran)
     int4* gtiles;             // nullptr, or [P/kGemmTileTokens + E*nk] GEMM token tiles {e, k, pos0, n}
     int32_t* pos_tok;         // nullptr, or [P] token of each grouped position
     WsHeader* hdr;
 };
-cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream);
+// Counters of the grid-wide bisection (zeroed by the launcher before every call).
+constexpr int kCoopRoundsMax = 16;
+struct CoopSync {
+    unsigned barrier;
+    unsigned bad;
+    unsigned long long mx_bits;
+    int counts[kCoopRoundsMax][64][32];   // one 128-byte line per node: CTAs' atomics do not queue on one line
+};
+// coop: workspace counters for the grid-wide bisection of large batches (nullptr: single CTA).
+cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* coop = nullptr, int sms = 0);
 size_t allocate_smem_bytes(int P, int E, int nk);
 int allocate_threads(int P);
 
@@ -53,13 +68,17 @@ struct GemmArgs {
     uint64_t planes_per_expert, meta_per_expert;
     uint64_t planes_mat_off[3], meta_mat_off[3];
     int H, I, B, G;
+    int T, P;                 // tokens, routed pairs (rows of x and of hbuf)
     const int4* gtiles;       // {e, k, pos0, n}, count in hdr->n_gtiles
     const int32_t* pos_tok;   // [P] token of each grouped position
     const uint16_t* x;        // [T][H] bf16 activations
+    uint16_t* xperm;          // [P][H] bf16 activations in grouped pair order (written by the permute)
+    int E;
     uint16_t* hbuf;           // [P][I] fp16 SwiGLU outputs, grouped order
     float* out_pair;          // [P][H] per-pair expert outputs, grouped order
     WsHeader* hdr;
 };
+cudaError_t launch_permute_rows(const GemmArgs& a, cudaStream_t stream);
 cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t stream, int sms);
 cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t stream, int sms);
 size_t gemm_tc_smem_bytes();

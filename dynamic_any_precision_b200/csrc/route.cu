@@ -24,6 +24,8 @@ namespace {
 constexpr int kRouteWarps = 8;
 constexpr int kPrefetch = 8;   // router-row uint4 loads a lane issues at once
 constexpr int16_t kNoBit = 0x3FFF;   // lowest-set-bit marker of a zero element
+constexpr int kRouteTiledMinTokens = 128;   // from here on the logits run as a tiled GEMM
+constexpr int kMaxLsbBlocks = 256;          // H <= 16384 on the tiled path
 
 // ---------------- fp64 exp (see header comment) ----------------
 __device__ __forceinline__ double dexp_fixed(double x) {
@@ -164,6 +166,151 @@ __device__ __forceinline__ int warp_sum_i(int v) {
     return v;
 }
 
+// Exact dot product of one (token, router row) pair by a warp: fp64 sum with the per-product
+// lowest-bit proof (every product a multiple of 2^lmin, sum |p| < 2^(lmin+53)), else the
+// fixed-point accumulator. Both operands are bf16 rows in global or shared memory.
+__device__ double exact_dot_warp(const uint16_t* x, const uint16_t* w, int H, int lane) {
+    double acc = 0.0, absacc = 0.0;
+    int lmin = 1 << 20;
+    for (int j = lane; j < H; j += 32) {
+        const uint32_t xu = x[j], wu = w[j];
+        const double p = __dmul_rn(static_cast<double>(__uint_as_float(xu << 16)),
+                                   static_cast<double>(__uint_as_float(wu << 16)));
+        acc = __dadd_rn(acc, p);
+        absacc = __dadd_rn(absacc, fabs(p));
+        if ((xu & 0x7FFF) && (wu & 0x7FFF)) lmin = min(lmin, bf16_lsb(xu) + bf16_lsb(wu));
+    }
+    acc = warp_sum_f64(acc);
+    absacc = warp_sum_f64(absacc);
+    lmin = warp_min_i(lmin);
+    if (absacc == 0.0) return acc;
+    int ea;
+    frexp(absacc, &ea);   // absacc < 2^ea
+    if (ea <= lmin + 52) return acc;
+    return exact_dot_fixed(x, w, H, lane);
+}
+
+// Fixed-point digits of token t for the expert GEMV: groups g = g0, g0 + gstep, ... handled by
+// this warp; xs is the token's bf16 row (shared or global memory).
+__device__ void token_digits(const RouteArgs& a, int t, const uint16_t* xs, int g0, int gstep) {
+    const int H = a.H, G = a.G, ng = H / G, lane = threadIdx.x & 31;
+    for (int g = g0; g < ng; g += gstep) {
+        float mx = 0.f;
+        for (int j = lane; j < G; j += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_float(xs[g * G + j])));
+        mx = warp_max_f(mx);
+        const int Eg = group_exponent(mx);
+        int sum = 0;
+        for (int j = lane; j < G; j += 32) {
+            const int X = to_fixed(bf16_bits_to_float(xs[g * G + j]), Eg);
+            sum += X;
+            int8_t d0, d1, d2;
+            split_digits(X, d0, d1, d2);
+            const size_t base = static_cast<size_t>(t) * 3 * H + g * G + j;
+            a.xdig[base] = d0;
+            a.xdig[base + H] = d1;
+            a.xdig[base + 2 * H] = d2;
+        }
+        sum = warp_sum_i(sum);
+        if (lane == 0) {
+            a.xexp[t * ng + g] = Eg;
+            a.xsum[t * ng + g] = sum;
+        }
+    }
+}
+
+// Top-k by exact fp64 logit (descending, ties to the lower expert id, NaN last) and the gates
+// (fixed fp64 exp; softmax over the top-k or over all experts). Whole block; smem_raw holds at
+// least 24 * E bytes.
+__device__ void select_topk_gates(const RouteArgs& a, int t, unsigned char* smem_raw) {
+    __shared__ int s_sel[32];
+    __shared__ double s_num[32];
+    __shared__ double s_den;
+    const int E = a.E;
+    // the logits were written by other blocks or kernels (fenced / completed); read them from L2
+    const double* lrow = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
+    double* vals = reinterpret_cast<double*>(smem_raw);             // [E] logits (token no longer needed)
+    float* fk = reinterpret_cast<float*>(vals + E);                 // [E] fp32 roundings of the logits
+    for (int i = threadIdx.x; i < E; i += blockDim.x) {
+        const double v = __ldcg(lrow + i);
+        vals[i] = v;
+        fk[i] = v == v ? __double2float_rn(v) : -INFINITY;   // NaN is never larger
+    }
+    __syncthreads();
+    const int K = a.K;
+    // rank of each expert = number of experts before it (descending logit, ties to the lower
+    // id; NaN ranks last). Q threads share a candidate, each counting over 1/Q of the experts.
+    int Q = 1;
+    while (Q < 32 && Q * 2 * E <= static_cast<int>(blockDim.x)) Q *= 2;
+    const int chunk = (E + Q - 1) / Q;
+    for (int base = 0; base < E * Q; base += blockDim.x) {
+        const int idx = base + threadIdx.x;
+        const int c = idx / Q, q = idx % Q;
+        int rank = 0;
+        if (c < E) {
+            const double v = vals[c];
+            if (v == v) {
+                // fp32 rounding is monotone: fk[j] > fk[c] implies vals[j] > vals[c]; only equal fp32
+                // values need the exact fp64 comparison (with ties to the lower expert id)
+                const float fv = fk[c];
+                const int j0 = q * chunk, j1 = min(E, (q + 1) * chunk);
+                int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+                int j = j0;
+                for (; j + 4 <= j1; j += 4) {   // four independent comparisons per iteration
+                    const float u0 = fk[j], u1 = fk[j + 1], u2 = fk[j + 2], u3 = fk[j + 3];
+                    r0 += u0 > fv ? 1 : 0;
+                    r1 += u1 > fv ? 1 : 0;
+                    r2 += u2 > fv ? 1 : 0;
+                    r3 += u3 > fv ? 1 : 0;
+                    if (u0 == fv || u1 == fv || u2 == fv || u3 == fv) {
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int jj = j + u;
+                            if (fk[jj] == fv && jj != c) {
+                                const double w = vals[jj];
+                                r0 += (w > v || (w == v && jj < c)) ? 1 : 0;
+                            }
+                        }
+                    }
+                }
+                for (; j < j1; ++j) {
+                    const float u = fk[j];
+                    r0 += u > fv ? 1 : 0;
+                    if (u == fv && j != c) {
+                        const double w = vals[j];
+                        r0 += (w > v || (w == v && j < c)) ? 1 : 0;
+                    }
+                }
+                rank = (r0 + r1) + (r2 + r3);
+            } else {
+                rank = q == 0 ? E : 0;
+            }
+        }
+        for (int o = 1; o < Q; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+        if (c < E && q == 0 && rank < K) s_sel[rank] = c;
+    }
+    __syncthreads();
+    const double lmax = vals[s_sel[0]];
+    if (threadIdx.x < K) s_num[threadIdx.x] = dexp_fixed(__dsub_rn(vals[s_sel[threadIdx.x]], lmax));
+    double* ex = vals + 2 * E;   // [E] exp values (norm over all experts), after the fp32 keys
+    if (!a.norm_topk)
+        for (int i = threadIdx.x; i < E; i += blockDim.x) ex[i] = dexp_fixed(__dsub_rn(vals[i], lmax));
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double den = 0.0;
+        if (a.norm_topk) {
+            for (int j = 0; j < K; ++j) den = __dadd_rn(den, s_num[j]);
+        } else {
+            for (int i = 0; i < E; ++i) den = __dadd_rn(den, ex[i]);
+        }
+        s_den = den;
+    }
+    __syncthreads();
+    if (threadIdx.x < K) {
+        a.idx[t * K + threadIdx.x] = s_sel[threadIdx.x];
+        a.gate[t * K + threadIdx.x] = __ddiv_rn(s_num[threadIdx.x], s_den);
+    }
+}
+
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int H = a.H, E = a.E, H8 = H >> 3;
@@ -173,9 +320,6 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     int16_t* xl = reinterpret_cast<int16_t*>(xd + H);                 // [H] lowest set bit (kNoBit: zero)
     uint16_t* xs = reinterpret_cast<uint16_t*>(xl + H);               // [H] bf16 bits (natural order)
     __shared__ int s_last;
-    __shared__ int s_sel[32];
-    __shared__ double s_num[32];
-    __shared__ double s_den;
     __shared__ double s_acc[kRouteWarps], s_abs[kRouteWarps];
     __shared__ int s_lmin[kRouteWarps], s_bad[kRouteWarps];
     const int t = blockIdx.y;
@@ -301,31 +445,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     }
 
     // ---- fixed-point digits of x for the expert GEMV: the token's blocks share the groups ----
-    if (a.xdig != nullptr) {
-        const int G = a.G, ng = H / G;
-        for (int g = blockIdx.x + warp * gridDim.x; g < ng; g += gridDim.x * kRouteWarps) {
-            float mx = 0.f;
-            for (int j = lane; j < G; j += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_float(xs[g * G + j])));
-            mx = warp_max_f(mx);
-            const int Eg = group_exponent(mx);
-            int sum = 0;
-            for (int j = lane; j < G; j += 32) {
-                const int X = to_fixed(bf16_bits_to_float(xs[g * G + j]), Eg);
-                sum += X;
-                int8_t d0, d1, d2;
-                split_digits(X, d0, d1, d2);
-                const size_t base = static_cast<size_t>(t) * 3 * H + g * G + j;
-                a.xdig[base] = d0;
-                a.xdig[base + H] = d1;
-                a.xdig[base + 2 * H] = d2;
-            }
-            sum = warp_sum_i(sum);
-            if (lane == 0) {
-                a.xexp[t * ng + g] = Eg;
-                a.xsum[t * ng + g] = sum;
-            }
-        }
-    }
+    if (a.xdig != nullptr) token_digits(a, t, xs, blockIdx.x + warp * gridDim.x, gridDim.x * kRouteWarps);
 
     // ---- last block of this token: top-k and gates ----
     __syncthreads();
@@ -338,94 +458,255 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     if (!s_last) return;
     if (threadIdx.x == 0) a.counters[t] = 0;   // ready for the next call
 
-    // the other blocks fenced their logits before taking a ticket; read them from L2
-    const double* lrow = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
-    double* vals = reinterpret_cast<double*>(smem_raw);             // [E] logits (token no longer needed)
-    float* fk = reinterpret_cast<float*>(vals + E);                 // [E] fp32 roundings of the logits
-    for (int i = threadIdx.x; i < E; i += blockDim.x) {
-        const double v = __ldcg(lrow + i);
-        vals[i] = v;
-        fk[i] = v == v ? __double2float_rn(v) : -INFINITY;   // NaN is never larger
-    }
-    __syncthreads();
-    const int K = a.K;
-    // rank of each expert = number of experts before it (descending logit, ties to the lower
-    // id; NaN ranks last). Q threads share a candidate, each counting over 1/Q of the experts.
-    int Q = 1;
-    while (Q < 32 && Q * 2 * E <= static_cast<int>(blockDim.x)) Q *= 2;
-    const int chunk = (E + Q - 1) / Q;
-    for (int base = 0; base < E * Q; base += blockDim.x) {
-        const int idx = base + threadIdx.x;
-        const int c = idx / Q, q = idx % Q;
-        int rank = 0;
-        if (c < E) {
-            const double v = vals[c];
-            if (v == v) {
-                // fp32 rounding is monotone: fk[j] > fk[c] implies vals[j] > vals[c]; only equal fp32
-                // values need the exact fp64 comparison (with ties to the lower expert id)
-                const float fv = fk[c];
-                const int j0 = q * chunk, j1 = min(E, (q + 1) * chunk);
-                int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
-                int j = j0;
-                for (; j + 4 <= j1; j += 4) {   // four independent comparisons per iteration
-                    const float u0 = fk[j], u1 = fk[j + 1], u2 = fk[j + 2], u3 = fk[j + 3];
-                    r0 += u0 > fv ? 1 : 0;
-                    r1 += u1 > fv ? 1 : 0;
-                    r2 += u2 > fv ? 1 : 0;
-                    r3 += u3 > fv ? 1 : 0;
-                    if (u0 == fv || u1 == fv || u2 == fv || u3 == fv) {
+    select_topk_gates(a, t, smem_raw);
+}
+
+
+// ---------------- large batches: logits as a tiled fp64 GEMM ----------------
+// Exactness without per-product bookkeeping. Split the H inputs into blocks b of 64. Every
+// product x_j * w_j of block b is a multiple of 2^(Lx_b + Lw_b) (lowest set bit over the block's
+// nonzero elements of the token / the router row), so every product is a multiple of 2^L with
+// L = min_b (Lx_b + Lw_b); by Cauchy-Schwarz, sum_j |x_j w_j| <= |x| |w|. If
+// |x|^2 |w|^2 < 2^(2 (L + 53)), every partial sum in any order is a multiple of 2^L below
+// 2^(L+53): exact in fp64. Then the logit may be accumulated in any blocking and summed across
+// CTAs with fp64 atomics. Logits whose bound fails are recomputed with the fixed-point dot
+// product by the selection kernel, so the result is always the exact dot product rounded once,
+// as in the per-logit kernel.
+
+constexpr int kNoLsb = 0x3FFF;      // block (or row) without a nonzero element
+constexpr int kLsbBlock = 64;       // inputs per lowest-bit block
+
+// One CTA per row (tokens 0..T-1, then router rows): per-block lowest set bit, sum of squares,
+// NaN/Inf flag.
+__global__ void __launch_bounds__(128) route_stats_kernel(RouteArgs a) {
+    __shared__ double s_n[4];
+    __shared__ int s_b[4];
+    pdl_wait();
+    const int r = blockIdx.x, H = a.H, nb = H / kLsbBlock;
+    const bool is_tok = r < a.T;
+    const uint16_t* row = is_tok ? a.x + static_cast<size_t>(r) * H : a.wr + static_cast<size_t>(r - a.T) * H;
+    int16_t* lrow = is_tok ? a.lsb_x + static_cast<size_t>(r) * nb : a.lsb_w + static_cast<size_t>(r - a.T) * nb;
+    int bad = 0;
+    double n2 = 0.0;
+    // thread c covers elements 8c .. 8c+7; 8 consecutive lanes make one block of 64
+    for (int c0 = 0; c0 < H / 8; c0 += blockDim.x) {
+        const int c = c0 + threadIdx.x;
+        int l = kNoLsb;
+        if (c < H / 8) {
+            const uint4 v = reinterpret_cast<const uint4*>(row)[c];
+            const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int jj = j + u;
-                            if (fk[jj] == fv && jj != c) {
-                                const double w = vals[jj];
-                                r0 += (w > v || (w == v && jj < c)) ? 1 : 0;
-                            }
-                        }
-                    }
-                }
-                for (; j < j1; ++j) {
-                    const float u = fk[j];
-                    r0 += u > fv ? 1 : 0;
-                    if (u == fv && j != c) {
-                        const double w = vals[j];
-                        r0 += (w > v || (w == v && j < c)) ? 1 : 0;
-                    }
-                }
-                rank = (r0 + r1) + (r2 + r3);
-            } else {
-                rank = q == 0 ? E : 0;
+            for (int h = 0; h < 8; ++h) {
+                const uint32_t u = (ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                if (u & 0x7FFF) l = min(l, bf16_lsb(u));
+                bad |= ((u >> 7) & 0xFF) == 0xFF;
+                const double d = static_cast<double>(__uint_as_float(u << 16));
+                n2 = __dadd_rn(n2, __dmul_rn(d, d));
             }
         }
-        for (int o = 1; o < Q; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
-        if (c < E && q == 0 && rank < K) s_sel[rank] = c;
+        for (int o = 1; o < 8; o <<= 1) l = min(l, __shfl_xor_sync(0xffffffffu, l, o));
+        if (c < H / 8 && (c & 7) == 0) lrow[c >> 3] = static_cast<int16_t>(l);
     }
-    __syncthreads();
-    const double lmax = vals[s_sel[0]];
-    if (threadIdx.x < K) s_num[threadIdx.x] = dexp_fixed(__dsub_rn(vals[s_sel[threadIdx.x]], lmax));
-    double* ex = vals + 2 * E;   // [E] exp values (norm over all experts), after the fp32 keys
-    if (!a.norm_topk)
-        for (int i = threadIdx.x; i < E; i += blockDim.x) ex[i] = dexp_fixed(__dsub_rn(vals[i], lmax));
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    n2 = warp_sum_f64(n2);
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) { s_n[warp] = n2; s_b[warp] = bad; }
     __syncthreads();
     if (threadIdx.x == 0) {
-        double den = 0.0;
-        if (a.norm_topk) {
-            for (int j = 0; j < K; ++j) den = __dadd_rn(den, s_num[j]);
-        } else {
-            for (int i = 0; i < E; ++i) den = __dadd_rn(den, ex[i]);
+        for (int w = 1; w < 4; ++w) { n2 = __dadd_rn(n2, s_n[w]); bad |= s_b[w]; }
+        if (is_tok) a.n2_x[r] = n2;
+        else a.n2_w[r - a.T] = n2;
+        if (bad) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, is_tok ? 1 : 2);
+    }
+}
+
+constexpr int kGT = 64, kGE = 128, kGK = 32;   // CTA tile: tokens x experts, k per stage
+constexpr int kGThreads = 256;                  // 8 warps of 16 tokens x 64 experts
+
+__device__ __forceinline__ double bf16_to_f64(uint32_t u) { return static_cast<double>(__uint_as_float(u << 16)); }
+
+// grid (ceil(T/64), ceil(E/128), k slices). Shared: x [2][kGK][kGT], w [2][kGK][kGE] in fp64.
+__global__ void __launch_bounds__(kGThreads) route_gemm_kernel(RouteArgs a, int kslice) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    double* sx = reinterpret_cast<double*>(smem_raw);          // [2][kGK][kGT]
+    double* sw = sx + 2 * kGK * kGT;                            // [2][kGK][kGE]
+    const int H = a.H, T = a.T, E = a.E;
+    const int t0 = blockIdx.x * kGT, e0 = blockIdx.y * kGE;
+    const int k0 = blockIdx.z * kslice, k1 = min(H, k0 + kslice);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wt = warp & 3, we = warp >> 2, tg = lane & 3, eg = lane >> 2;
+    const int tb = 16 * wt + 4 * tg, eb = 64 * we + 8 * eg;   // this thread's 4 tokens, 8 experts
+    pdl_wait();
+
+    // staging: x tile 64 x 32 (one uint4 per thread), w tile 128 x 32 (two per thread)
+    const int xt = tid & 63, xk = (tid >> 6) * 8;
+    const int wi = tid & 127, wk = (tid >> 7) * 8;
+    uint4 rx, rw0, rw1;
+    auto load = [&](int kc) {
+        rx = make_uint4(0, 0, 0, 0);
+        rw0 = rx;
+        rw1 = rx;
+        if (t0 + xt < T) rx = *reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + xt) * H + kc + xk);
+        if (e0 + wi < E) {
+            const uint16_t* wrow = a.wr + static_cast<size_t>(e0 + wi) * H + kc;
+            rw0 = *reinterpret_cast<const uint4*>(wrow + wk);
+            rw1 = *reinterpret_cast<const uint4*>(wrow + wk + 16);
         }
-        s_den = den;
+    };
+    auto store = [&](int buf) {
+        double* bx = sx + buf * kGK * kGT;
+        double* bw = sw + buf * kGK * kGE;
+        const uint32_t xv[4] = {rx.x, rx.y, rx.z, rx.w};
+        const uint32_t w0[4] = {rw0.x, rw0.y, rw0.z, rw0.w};
+        const uint32_t w1[4] = {rw1.x, rw1.y, rw1.z, rw1.w};
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            const int sh = 16 * (h & 1);
+            bx[(xk + h) * kGT + xt] = bf16_to_f64((xv[h >> 1] >> sh) & 0xFFFFu);
+            bw[(wk + h) * kGE + wi] = bf16_to_f64((w0[h >> 1] >> sh) & 0xFFFFu);
+            bw[(wk + 16 + h) * kGE + wi] = bf16_to_f64((w1[h >> 1] >> sh) & 0xFFFFu);
+        }
+    };
+
+    double acc[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+
+    int buf = 0;
+    load(k0);
+    store(0);
+    __syncthreads();
+    for (int kc = k0; kc < k1; kc += kGK) {
+        const bool more = kc + kGK < k1;
+        if (more) load(kc + kGK);
+        const double* bx = sx + buf * kGK * kGT;
+        const double* bw = sw + buf * kGK * kGE;
+#pragma unroll 4
+        for (int k = 0; k < kGK; ++k) {
+            const double2 x01 = *reinterpret_cast<const double2*>(bx + k * kGT + tb);
+            const double2 x23 = *reinterpret_cast<const double2*>(bx + k * kGT + tb + 2);
+            const double2 w01 = *reinterpret_cast<const double2*>(bw + k * kGE + eb);
+            const double2 w23 = *reinterpret_cast<const double2*>(bw + k * kGE + eb + 2);
+            const double2 w45 = *reinterpret_cast<const double2*>(bw + k * kGE + eb + 4);
+            const double2 w67 = *reinterpret_cast<const double2*>(bw + k * kGE + eb + 6);
+            const double xv[4] = {x01.x, x01.y, x23.x, x23.y};
+            const double wv[8] = {w01.x, w01.y, w23.x, w23.y, w45.x, w45.y, w67.x, w67.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = __fma_rn(xv[i], wv[j], acc[i][j]);
+        }
+        if (more) store(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+    }
+    double* dst = a.logits_user ? a.logits_user : a.logits_ws;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + tb + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = e0 + eb + j;
+            if (e < E) atomicAdd(dst + static_cast<size_t>(t) * E + e, acc[i][j]);
+        }
+    }
+}
+
+// One CTA (4 warps) per token: check each logit's exactness bound, recompute the failures with
+// the fixed-point dot product, then top-k and gates (and the GEMV digits when requested).
+__global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ int s_fail[256];
+    __shared__ int s_nfail;
+    __shared__ int16_t s_lx[kMaxLsbBlocks];
+    pdl_wait();
+    const int t = blockIdx.x, E = a.E, H = a.H, nb = H / kLsbBlock;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double* dst = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
+    if (threadIdx.x == 0) s_nfail = 0;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) s_lx[b] = a.lsb_x[static_cast<size_t>(t) * nb + b];
+    __syncthreads();
+    const double nx = a.n2_x[t];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        const int16_t* lw = a.lsb_w + static_cast<size_t>(e) * nb;
+        int L = 2 * kNoLsb;
+        for (int b0 = 0; b0 < nb; b0 += 8) {   // nb is a multiple of 8 (H % 512 == 0 on this path)
+            const uint4 v = *reinterpret_cast<const uint4*>(lw + b0);
+            const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const int lv = static_cast<int16_t>((ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu);
+                L = min(L, static_cast<int>(s_lx[b0 + h]) + lv);
+            }
+        }
+        bool ok = true;
+        if (L < kNoLsb) {   // some block has nonzero products (else the logit is exactly 0)
+            const int L2 = 2 * (L + 53);
+            // margin 2^-20 covers the rounding of the two fp64 sums of squares
+            const double lhs = __dmul_rn(__dmul_rn(nx, a.n2_w[e]), 1.0 + 0x1p-20);
+            ok = L2 >= 1024 || (L2 > -1022 && lhs < pow2(L2));
+        }
+        if (!ok) {
+            const int slot = atomicAdd(&s_nfail, 1);
+            if (slot < 256) s_fail[slot] = e;
+        }
     }
     __syncthreads();
-    if (threadIdx.x < K) {
-        a.idx[t * K + threadIdx.x] = s_sel[threadIdx.x];
-        a.gate[t * K + threadIdx.x] = __ddiv_rn(s_num[threadIdx.x], s_den);
+    const int nfail = s_nfail;
+    const uint16_t* xrow = a.x + static_cast<size_t>(t) * H;
+    if (nfail > 0) {
+        // more failures than the list holds: recompute every logit of the token
+        const int n = nfail <= 256 ? nfail : E;
+        for (int i = warp; i < n; i += 4) {
+            const int e = nfail <= 256 ? s_fail[i] : i;
+            const double v = exact_dot_warp(xrow, a.wr + static_cast<size_t>(e) * H, H, lane);
+            if (lane == 0) dst[e] = v;
+        }
+        __syncthreads();
     }
+    select_topk_gates(a, t, smem_raw);
+    if (a.xdig != nullptr) token_digits(a, t, xrow, warp, 4);
 }
 
 }  // namespace
 
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream) {
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms) {
+    if (a.T >= kRouteTiledMinTokens && a.H % kGK == 0 && a.H % (8 * kLsbBlock) == 0 &&
+        a.H / kLsbBlock <= kMaxLsbBlocks && a.lsb_x != nullptr) {
+        // large batch: stats, tiled fp64 GEMM with split-K atomics, per-token selection
+        double* dst = a.logits_user ? a.logits_user : a.logits_ws;
+        cudaError_t err = cudaMemsetAsync(dst, 0, sizeof(double) * static_cast<size_t>(a.T) * a.E, stream);
+        if (err != cudaSuccess) return err;
+        RouteArgs b = a;
+        void* args[] = {&b};
+        err = launch_pdl_raw(reinterpret_cast<const void*>(route_stats_kernel), dim3(a.T + a.E), dim3(128), 0,
+                             stream, args);
+        if (err != cudaSuccess) return err;
+        const int gx = (a.T + kGT - 1) / kGT, gy = (a.E + kGE - 1) / kGE;
+        const int nchunks = a.H / kGK;
+        int ks = 1;   // k slices: enough CTAs for every SM, each slice a whole number of chunks
+        while (gx * gy * ks < sms && ks * 2 <= nchunks && nchunks % (ks * 2) == 0) ks *= 2;
+        int kslice = (nchunks / ks) * kGK;
+        const size_t smem = sizeof(double) * 2 * kGK * (kGT + kGE);
+        err = cudaFuncSetAttribute(route_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        void* gargs[] = {&b, &kslice};
+        err = launch_pdl_raw(reinterpret_cast<const void*>(route_gemm_kernel), dim3(gx, gy, ks), dim3(kGThreads), smem,
+                             stream, gargs);
+        if (err != cudaSuccess) return err;
+        size_t ssm = (static_cast<size_t>(a.E) * 24 + 15) & ~static_cast<size_t>(15);
+        if (ssm > 48 * 1024) {
+            err = cudaFuncSetAttribute(route_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(ssm));
+            if (err != cudaSuccess) return err;
+        }
+        return launch_pdl_raw(reinterpret_cast<const void*>(route_select_kernel), dim3(a.T), dim3(128), ssm, stream,
+                              args);
+    }
     // few tokens: split each expert's dot product over 4 warps to shorten the serial chain
     RouteArgs b = a;
     b.wpe = a.T <= 16 ? 4 : 1;

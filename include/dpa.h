@@ -124,8 +124,9 @@ typedef struct dpa_layer_weights {
  * tensor-core path [4] and [5] follow the gate/up and down GEMMs.
  * expert_path: which kernels run the routed experts' FFN (same results up to the
  * rounding of fp32 accumulation and of the fp16 SwiGLU intermediate on the tensor-core path):
- *   DPA_PATH_AUTO (0)  tensor-core GEMMs when the format is uniform, hidden % 128 == 0,
- *                      inter % 64 == 0 and the batch routes at least DPA_TC_MIN_PAIRS_PER_EXPERT
+ *   DPA_PATH_AUTO (0)  tensor-core GEMMs when the format is uniform, hidden % 256 == 0,
+ *                      inter % 256 == 0, the group is a power of two and the batch routes at
+ *                      least DPA_TC_MIN_PAIRS_PER_EXPERT
  *                      pairs per expert on average (T*top_k >= that * n_experts); else GEMV;
  *   DPA_PATH_GEMV (1)  the batched GEMV kernels (any shape check_desc accepts);
  *   DPA_PATH_TC (2)    the tcgen05 grouped GEMMs (DPA_ERR_UNSUPPORTED when the shape does

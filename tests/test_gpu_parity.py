@@ -89,7 +89,9 @@ def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None, p
 # ----------------------------------------------------------------------------- routing
 
 @pytest.mark.parametrize("shape,T", [(W.TINY, 4), (W.QWEN3_B1, 1), (W.QWEN3_B64, 64), (W.DEEPSEEK_B16, 16),
-                                     (W.QWEN3_B1, 37), (W.TINY, 3)])
+                                     (W.QWEN3_B1, 37), (W.TINY, 3),
+                                     # from 128 tokens on: tiled fp64 GEMM (ragged token tiles)
+                                     (W.TINY, 200), (W.DEEPSEEK_B16, 130), (W.QWEN3_B64, 300)])
 def test_route_bit_exact(shape, T):
     d = dpa.make_desc(shape)
     wr = W.router_weights(shape)
@@ -105,14 +107,15 @@ def test_route_bit_exact(shape, T):
     assert np.array_equal(gate.cpu().numpy(), rg)
 
 
-def test_route_exact_path_for_wide_exponent_spread():
+@pytest.mark.parametrize("T", [4, 150])
+def test_route_exact_path_for_wide_exponent_spread(T):
     # operands spread over ~200 binades, and large terms that cancel exactly, so the logit is
     # decided by tiny terms: the fp64 fast path cannot prove exactness and the kernel must
-    # take the fixed-point path
+    # take the fixed-point path (per-logit kernel at 4 tokens, tiled kernel's fallback at 150)
     shape = W.with_sizes(W.TINY, name="tiny_spread")
     d = dpa.make_desc(shape)
     rng = np.random.default_rng(5)
-    T, H, E = 4, shape.hidden, shape.n_experts
+    H, E = shape.hidden, shape.n_experts
     x = rng.standard_normal((T, H)).astype(np.float32)
     x[:, 0] = 2.0 ** 100
     x[:, 1] = -(2.0 ** 100)
