@@ -39,6 +39,7 @@ from dynamic_any_precision_b200 import workloads as W  # noqa: E402
 
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1400.0   # sustained bf16 under the power cap, an earlier measurement on this machine
 
 
 def parse_args(argv=None):
@@ -63,6 +64,15 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def _peaks():
+    """All measured peaks as a dict (empty when the file is absent)."""
+    try:
+        with open(PEAKS_PATH) as f:
+            return json.load(f)
+    except Exception:
+        return {}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -285,8 +295,12 @@ def run_dpa(args, shape, target, rank, world, dist):
                "h2d_bytes_per_step": int(x_buf.numel() * 2), "d2h_bytes_per_step": int(y_buf.numel() * 2),
                "steps": n_e}
 
-    launches_per_step = 5 + (2 if shape.n_shared else 0)
-    return {"ms": ms, "stage_ms": stage_ms, "gu_bytes": gu_bytes, "dn_bytes": dn_bytes, "n_active": n_active,
+    P = T * K
+    tc = (shape.fmt == dpa.FMT_UNIFORM and shape.hidden % 256 == 0 and shape.inter % 256 == 0 and
+          P >= 16 * shape.n_experts)
+    launches_per_step = ((3 if T >= 128 else 1) + (2 if P > 2048 else 1) + (3 if tc else 2) + 1 +
+                         (2 if shape.n_shared else 0))
+    return {"tc": tc, "ms": ms, "stage_ms": stage_ms, "gu_bytes": gu_bytes, "dn_bytes": dn_bytes, "n_active": n_active,
             "mean_bpw": mean_bpw, "clocks": clk.summary(), "e2e": e2e, "launches": launches_per_step * args.steps}
 
 
@@ -478,6 +492,17 @@ def main(argv=None):
                 "prefill_tokens_per_s": world * W.STACK_PREFILL_TOKENS / (res["prefill_ms"] * 1e-3),
                 "prefill_ms": res["prefill_ms"], "clocks": res["clocks"], "gpu_launches": res["launches"],
                 "host_build_s": res["build_s"]}
+        # whole-prefill tensor throughput: 2 flop per multiply-add of the three expert matrices over
+        # every routed pair and layer (routing, allocation and glue counted in the time, not the flops)
+        flops = 2.0 * W.STACK_PREFILL_TOKENS * shape.top_k * 3 * shape.hidden * shape.inter * res["n_layers"]
+        pk = _peaks()
+        peak = pk.get("bf16_tflops_sustained") if pk else None
+        achieved = flops / (res["prefill_ms"] * 1e-3) / 1e12
+        line["prefill_roofline"] = {"bound": "tensor", "achieved": achieved,
+                                    "peak": peak if peak else FALLBACK_BF16_TFLOPS, "unit": "TFLOP/s",
+                                    "frac": achieved / (peak if peak else FALLBACK_BF16_TFLOPS),
+                                    "scope": "whole prefill step (route, allocate, permute, GEMMs, combine, glue)",
+                                    "peak_source": "measured sustained bf16" if peak else "fallback"}
         if rank == 0:
             print(json.dumps(line), flush=True)
         if dist is not None:
@@ -511,6 +536,7 @@ def main(argv=None):
         "config": config,
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None, "peak_source": peak_kind},
+        "dtype_note": "tensor-core path: bf16 x bf16 (gate/up), fp16 x fp16 (down), fp32 accumulate" if res["tc"] else None,
         "planes_gbs_whole_step": all_bytes / secs / 1e9 / world,
         "planes_frac_whole_step": all_bytes / secs / 1e9 / world / hbm,
         "bytes_per_step": all_bytes / args.steps,
@@ -521,6 +547,21 @@ def main(argv=None):
         "e2e": res["e2e"],
         "gpu_launches": res["launches"],
     }
+    if res["tc"]:
+        # prefill-sized batches run the expert FFN as tcgen05 GEMMs: tensor-bound. The gate/up stage
+        # (row permutation + GEMM) is timed against the sustained bf16 peak (it runs inside a step).
+        pk = _peaks()
+        tpeak = pk.get("bf16_tflops_sustained") or FALLBACK_BF16_TFLOPS
+        flops = 2.0 * shape.tokens * shape.top_k * 2 * shape.hidden * shape.inter * args.steps
+        gu_s = stage["gateup"] * 1e-3
+        ach = flops / gu_s / 1e12 if gu_s > 0 else 0.0
+        line["roofline"] = {"bound": "tensor", "kernel": "gateup", "achieved": ach, "peak": tpeak,
+                            "unit": "TFLOP/s", "frac": ach / tpeak, "traffic": None,
+                            "peak_source": "measured sustained bf16" if pk.get("bf16_tflops_sustained") else "fallback"}
+        line["dtype"] = "bf16/fp16 tensor-core operands, f32 accumulate (decision path f64)"
+        line.pop("dtype_note", None)
+    else:
+        line.pop("dtype_note", None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         smp = oracle_sample(shape, target, args.cpu_sample_tokens, seed_base=50000)
         line["cpu_baseline"] = {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample")}

@@ -60,8 +60,11 @@ QWEN3_STACK = LayerShape("qwen3_30b_a3b_moe_stack48", 2048, 768, 128, 8, 0, FMT_
                          128, 1, 32, (2.0, 3.0, 4.0), 4, layers=48)
 STACK_PREFILL_TOKENS = 2048
 STACK_DECODE_STEPS = 256
+# one layer of the stack's prefill on its own (read at the stored rate: all pairs k = kmax)
+QWEN3_PREFILL = LayerShape("qwen3_30b_a3b_moe_prefill_t2048", 2048, 768, 128, 8, 0, FMT_UNIFORM, 4, 2, 4,
+                           128, 1, STACK_PREFILL_TOKENS, (4.0, 3.0), 5)
 
-ALL_SHAPES = (TINY, QWEN3_B1, QWEN3_B64, DEEPSEEK_B16, QWEN3_STACK)
+ALL_SHAPES = (TINY, QWEN3_B1, QWEN3_B64, DEEPSEEK_B16, QWEN3_STACK, QWEN3_PREFILL)
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
