@@ -41,7 +41,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
-        desc, tiles, gtiles, postok, coop, rstats, xperm, total;
+        desc, tiles, gtiles, postok, coop, rstats, xperm, hdig, hexp, hsum, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -80,6 +80,9 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.coop = take(sizeof(dpa::CoopSync));
     L.rstats = take((8 + 2 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 16);
     L.xperm = take(2 * P * H);
+    L.hdig = take(3 * P * I);
+    L.hexp = take(4 * P * (I / d->group));
+    L.hsum = take(4 * P * (I / d->group));
     L.total = off;
     return L;
 }
@@ -422,6 +425,10 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     ga.xsum = at<int32_t>(ws, L.xsum);
     ga.h = at<float>(ws, L.h);
     ga.out_pair = at<float>(ws, L.out_pair);
+    ga.hdig = at<int8_t>(ws, L.hdig);
+    ga.hexp = at<int32_t>(ws, L.hexp);
+    ga.hsum = at<int32_t>(ws, L.hsum);
+    ga.P = T * K;
     ga.hdr = hdr;
     const int P = T * K;
     ga.max_items = P < d->n_experts ? P : d->n_experts;

@@ -122,9 +122,11 @@ __host__ __device__ inline Layout gateup_layout(int H, int G, int B, int fmt, in
                                                      : static_cast<size_t>(2) * B * 16 * ng * 2;
     L.dig = align16(L.meta + meta_bytes);
     L.dig_stride = H + kDigPad;
-    L.xe = align16(L.dig + static_cast<size_t>(2 * NT) * 3 * L.dig_stride);
-    L.xs = align16(L.xe + static_cast<size_t>(2 * NT) * ng * 4);
-    L.red = align16(L.xs + static_cast<size_t>(2 * NT) * ng * 4);
+    // multi-token kernels read the digits from global memory (no staged copy)
+    const size_t sl = NT == 1 ? static_cast<size_t>(2 * NT) : 0;
+    L.xe = align16(L.dig + sl * 3 * L.dig_stride);
+    L.xs = align16(L.xe + sl * ng * 4);
+    L.red = align16(L.xs + sl * ng * 4);
     L.total = align16(L.red + static_cast<size_t>(kWarps) * NT * 2 * 2 * 16 * 4);
     return L;
 }
@@ -139,9 +141,10 @@ __host__ __device__ inline Layout down_layout(int I, int G, int B, int fmt, int 
                                                      : static_cast<size_t>(B) * 64 * ng * 2;
     L.dig = align16(L.meta + meta_bytes);
     L.dig_stride = I + kDigPad;
-    L.xe = align16(L.dig + static_cast<size_t>(2 * NT) * 3 * L.dig_stride);
-    L.xs = align16(L.xe + static_cast<size_t>(2 * NT) * ng * 4);
-    L.red = align16(L.xs + static_cast<size_t>(2 * NT) * ng * 4);
+    const size_t sl = NT == 1 ? static_cast<size_t>(2 * NT) : 0;
+    L.xe = align16(L.dig + sl * 3 * L.dig_stride);
+    L.xs = align16(L.xe + sl * ng * 4);
+    L.red = align16(L.xs + sl * ng * 4);
     L.total = align16(L.red + static_cast<size_t>(2) * 4 * NT * 2 * 16 * 4);
     return L;
 }
@@ -226,8 +229,9 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
             if (threadIdx.x == 0) s_nt = min(NT, ntiles - pass0);
             __syncthreads();
             const int nt = s_nt;
-            // stage the digits, exponents and sums of the pass's tokens (loads issued first)
-            {
+            // stage the digits, exponents and sums of the pass's tokens (loads issued first);
+            // multi-token kernels read them from global memory instead (L1/L2 resident)
+            if constexpr (NT == 1) {
                 const int chunks = (3 * H) >> 4;
                 for (int i0 = threadIdx.x; i0 < 2 * NT * chunks; i0 += 4 * kThreads) {
                     uint4 v[4];
@@ -277,8 +281,12 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
 #pragma unroll
             for (int i = 0; i < NT; ++i) {
                 const int slot = 2 * i + half;
-                brow[i] = (i < nt && dig < 3 && tile_tok(s_tile[i], half) >= 0) ? s_dig + (slot * 3 + dig) * dstride
-                                                                                  : nullptr;
+                const int tk_ = tile_tok(s_tile[i], half);
+                if constexpr (NT == 1)
+                    brow[i] = (i < nt && dig < 3 && tk_ >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
+                else
+                    brow[i] = (i < nt && dig < 3 && tk_ >= 0) ? a.xdig + static_cast<size_t>(tk_) * 3 * H + dig * H
+                                                              : nullptr;
             }
             for (int g = g0; g < g1; ++g) {
                 if constexpr (FMT == DPA_FMT_UNIFORM) {
@@ -332,7 +340,15 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                             const int slot = 2 * i + my_half;
                             const int ki = s_tile[i].x;
                             const float ck = 0.5f * static_cast<float>((1 << (B - ki)) - 1);
-                            const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
+                            int Eg, SX;
+                            if constexpr (NT == 1) {
+                                Eg = s_xe[slot * ng + g];
+                                SX = s_xs[slot * ng + g];
+                            } else {
+                                const int tk_ = tile_tok(s_tile[i], my_half);
+                                Eg = tk_ >= 0 ? __ldg(a.xexp + tk_ * ng + g) : 0;
+                                SX = tk_ >= 0 ? __ldg(a.xsum + tk_ * ng + g) : 0;
+                            }
                             const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                             for (int m = 0; m < 2; ++m) {
@@ -395,7 +411,15 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                             for (int i = 0; i < NT; ++i) {
                                 if (i < nt && s_tile[i].x > p) {
                                     const int slot = 2 * i + my_half;
-                                    const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
+                                    int Eg, SX;
+                            if constexpr (NT == 1) {
+                                Eg = s_xe[slot * ng + g];
+                                SX = s_xs[slot * ng + g];
+                            } else {
+                                const int tk_ = tile_tok(s_tile[i], my_half);
+                                Eg = tk_ >= 0 ? __ldg(a.xexp + tk_ * ng + g) : 0;
+                                SX = tk_ >= 0 ? __ldg(a.xsum + tk_ * ng + g) : 0;
+                            }
                                     const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                                     for (int m = 0; m < 2; ++m) {
@@ -527,7 +551,8 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
             const int nt = s_nt;
             // fixed-point digits of the pass's h rows: one warp per (slot, group); a lane holds
             // 4 consecutive values per 128-column chunk, all loaded before use
-            for (int task = warp; task < 2 * NT * ng; task += kWarps) {
+            // (multi-token kernels read the digits written by hdigits_kernel)
+            for (int task = warp; NT == 1 && task < 2 * NT * ng; task += kWarps) {
                 const int slot = task / ng, g = task - slot * ng;
                 const int4 t = s_tile[slot >> 1];
                 const int pos = (slot & 1) ? t.z : t.y;
@@ -589,7 +614,11 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                 const int slot = 2 * i + half;
                 const int4 t = s_tile[i];
                 const int pos = half ? t.z : t.y;
-                brow[i] = (i < nt && dig < 3 && pos >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
+                if constexpr (NT == 1)
+                    brow[i] = (i < nt && dig < 3 && pos >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
+                else
+                    brow[i] = (i < nt && dig < 3 && pos >= 0) ? a.hdig + static_cast<size_t>(pos) * 3 * I + dig * I
+                                                              : nullptr;
             }
             const int rtile = warp & 3, khalf = warp >> 2;   // row tile of 4, half of the groups
             const uint32_t* wplanes = s_planes + static_cast<size_t>(rtile) * nblk * 32;
@@ -637,7 +666,15 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                             const int slot = 2 * i + my_half;
                             const int ki = s_tile[i].x;
                             const float ck = 0.5f * static_cast<float>((1 << (B - ki)) - 1);
-                            const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
+                            int Eg, SX;
+                            if constexpr (NT == 1) {
+                                Eg = s_xe[slot * ng + g];
+                                SX = s_xs[slot * ng + g];
+                            } else {
+                                const int pos_ = my_half ? s_tile[i].z : s_tile[i].y;
+                                Eg = pos_ >= 0 ? __ldg(a.hexp + pos_ * ng + g) : 0;
+                                SX = pos_ >= 0 ? __ldg(a.hsum + pos_ * ng + g) : 0;
+                            }
                             const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                             for (int rr = 0; rr < 2; ++rr) {
@@ -687,7 +724,15 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                             for (int i = 0; i < NT; ++i) {
                                 if (i < nt && s_tile[i].x > p) {
                                     const int slot = 2 * i + my_half;
-                                    const int Eg = s_xe[slot * ng + g], SX = s_xs[slot * ng + g];
+                                    int Eg, SX;
+                            if constexpr (NT == 1) {
+                                Eg = s_xe[slot * ng + g];
+                                SX = s_xs[slot * ng + g];
+                            } else {
+                                const int pos_ = my_half ? s_tile[i].z : s_tile[i].y;
+                                Eg = pos_ >= 0 ? __ldg(a.hexp + pos_ * ng + g) : 0;
+                                SX = pos_ >= 0 ? __ldg(a.hsum + pos_ * ng + g) : 0;
+                            }
                                     const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                                     for (int rr = 0; rr < 2; ++rr) {
@@ -734,6 +779,57 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
     }
 }
 
+// Fixed-point digits of every pair's SwiGLU row h[pos] (for the multi-token down kernel):
+// one warp per (position, group), the same arithmetic as the staged per-CTA digits.
+__global__ void __launch_bounds__(256) hdigits_kernel(GemvArgs a) {
+    pdl_wait();
+    const int I = a.I, G = a.G, ng = I / G;
+    const int task = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (task >= a.P * ng) return;
+    const int pos = task / ng, g = task - pos * ng;
+    const float* hrow = a.h + static_cast<size_t>(pos) * I + g * G;
+    float4 hv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int j = 128 * u + 4 * lane;
+        hv[u] = j < G ? *reinterpret_cast<const float4*>(hrow + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mx = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(hv[u].x), fabsf(hv[u].y)), fmaxf(fabsf(hv[u].z), fabsf(hv[u].w))));
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const int Eg = group_exponent(mx);
+    int sum = 0;
+    int8_t* drow = a.hdig + static_cast<size_t>(pos) * 3 * I + g * G;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int j = 128 * u + 4 * lane;
+        if (j < G) {
+            const float vv[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+            uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int X = to_fixed(vv[q], Eg);
+                sum += X;
+                int8_t d0, d1, d2;
+                split_digits(X, d0, d1, d2);
+                p0 |= static_cast<uint32_t>(static_cast<uint8_t>(d0)) << (8 * q);
+                p1 |= static_cast<uint32_t>(static_cast<uint8_t>(d1)) << (8 * q);
+                p2 |= static_cast<uint32_t>(static_cast<uint8_t>(d2)) << (8 * q);
+            }
+            *reinterpret_cast<uint32_t*>(drow + j) = p0;
+            *reinterpret_cast<uint32_t*>(drow + I + j) = p1;
+            *reinterpret_cast<uint32_t*>(drow + 2 * I + j) = p2;
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+        a.hexp[pos * ng + g] = Eg;
+        a.hsum[pos * ng + g] = sum;
+    }
+}
+
 template <int FMT, int NT>
 void* pick_gateup(int B) {
     switch (B) {
@@ -771,8 +867,14 @@ cudaError_t launch_generic(void* fn, size_t smem, int items, int num_sms, const 
 
 }  // namespace
 
-size_t gateup_smem_bytes(const GemvArgs& a) { return gateup_layout(a.H, a.G, a.B, a.fmt, 4).total; }
-size_t down_smem_bytes(const GemvArgs& a) { return down_layout(a.I, a.G, a.B, a.fmt, 4).total; }
+size_t gateup_smem_bytes(const GemvArgs& a) {
+    const size_t s1 = gateup_layout(a.H, a.G, a.B, a.fmt, 1).total, s4 = gateup_layout(a.H, a.G, a.B, a.fmt, 4).total;
+    return s1 > s4 ? s1 : s4;
+}
+size_t down_smem_bytes(const GemvArgs& a) {
+    const size_t s1 = down_layout(a.I, a.G, a.B, a.fmt, 1).total, s4 = down_layout(a.I, a.G, a.B, a.fmt, 4).total;
+    return s1 > s4 ? s1 : s4;
+}
 
 cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms) {
     const int nt = pick_nt(a);
@@ -785,6 +887,14 @@ cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms) {
 
 cudaError_t launch_down(const GemvArgs& a, cudaStream_t stream, int num_sms) {
     const int nt = pick_nt(a);
+    if (nt > 1) {   // digits of every h row once, for the multi-token down kernel
+        const int tasks = a.P * (a.I / a.G);
+        GemvArgs copy = a;
+        void* args[] = {&copy};
+        cudaError_t err = launch_pdl_raw(reinterpret_cast<const void*>(hdigits_kernel), dim3((tasks + 7) / 8), dim3(256),
+                                         0, stream, args);
+        if (err != cudaSuccess) return err;
+    }
     void* fn;
     if (a.fmt == DPA_FMT_UNIFORM) fn = nt == 1 ? pick_down<DPA_FMT_UNIFORM, 1>(a.B) : pick_down<DPA_FMT_UNIFORM, 4>(a.B);
     else fn = nt == 1 ? pick_down<DPA_FMT_BCQ, 1>(a.B) : pick_down<DPA_FMT_BCQ, 4>(a.B);

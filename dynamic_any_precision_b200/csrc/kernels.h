@@ -96,6 +96,10 @@ struct GemvArgs {
     const int32_t* xsum;      // [T][H/G]
     float* h;                 // [P][I] by sorted position
     float* out_pair;          // [P][H] by sorted position
+    int8_t* hdig;             // [P][3][I] digits of h (multi-token down kernel)
+    int32_t* hexp;            // [P][I/G]
+    int32_t* hsum;            // [P][I/G]
+    int P;                    // routed pairs
     WsHeader* hdr;
     int max_items;            // upper bound of active experts (host-known)
     int max_tokens_per_expert;  // host-known bound (selects the tile count per pass)
