@@ -32,6 +32,7 @@ namespace {
 constexpr int kAllocThreads = 1024;       // maximum block size
 constexpr int kSmemCostDoubles = 8192;    // costs kept in shared memory up to this many
 constexpr int kSmallP = 64;               // up to this many pairs one warp runs the bisection
+constexpr int kSpecMaxP = 2048;           // up to this many pairs the whole block speculates and verifies
 constexpr int kCoopThreads = 512;         // grid-wide bisection: threads per CTA
 constexpr int kCoopMaxPairsPerBlock = 6144;   // shared-memory costs: 6144 pairs x 32 B = 192 KB per CTA
 constexpr int kCoopDepth = 6;             // bisection steps per grid round (63 midpoints)
@@ -91,7 +92,7 @@ __device__ __forceinline__ int block_incl_scan(int v, int* s_tmp) {
 
 // Shared-memory carve-up: [costs (if they fit)] [counts E*nk] [seg E*nk+1] [sorted P] [k P]
 struct AllocSmem {
-    size_t costs, counts, seg, sorted, kk, total;
+    size_t costs, counts, seg, sorted, kk, bp, bj, total;
     bool costs_in_smem;
 };
 
@@ -108,6 +109,13 @@ __host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk) {
     off += static_cast<size_t>(P) * 4;
     L.kk = off;
     off += static_cast<size_t>(P);
+    // breakpoints of the speculative bisection (mid-size batches): P*(nk-1) doubles and ints
+    const size_t nbp = (P > kSmallP && P <= kSpecMaxP && L.costs_in_smem) ? static_cast<size_t>(P) * (nk - 1) : 0;
+    off = (off + 7) & ~static_cast<size_t>(7);
+    L.bp = off;
+    off += nbp * 8;
+    L.bj = off;
+    off += nbp * 4;
     L.total = (off + 15) & ~static_cast<size_t>(15);
     return L;
 }
@@ -328,6 +336,147 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             it += D;
         }
     } else {
+        int it_start = 0;
+        if (P <= kSpecMaxP && Ls.costs_in_smem) {
+            // ---- speculation for mid-size batches (the same idea as above, at block scale).
+            // Breakpoints of every pair's lower convex hull, at fixed slots p*(nk-1)+i (unused: -1).
+            const double* s_costs = reinterpret_cast<const double*>(smem + Ls.costs);
+            double* s_bpv = reinterpret_cast<double*>(smem + Ls.bp);
+            int* s_bjv = reinterpret_cast<int*>(smem + Ls.bj);
+            const int nslot = nk - 1;
+            for (int p = tid; p < P; p += blockDim.x) {
+                const double* c = s_costs + p * nk;
+                int cur = 0;
+                for (int i = 1; i < nk; ++i) if (c[i] < c[cur]) cur = i;
+                int slotb = 0;
+                while (cur > 0) {
+                    int jn = -1;
+                    double tn = 0.0;
+                    for (int j = 0; j < cur; ++j) {
+                        const double t = (c[j] - c[cur]) / static_cast<double>(cur - j);
+                        if (jn < 0 || t < tn) { jn = j; tn = t; }
+                    }
+                    s_bpv[p * nslot + slotb] = tn;
+                    s_bjv[p * nslot + slotb] = cur - jn;
+                    ++slotb;
+                    cur = jn;
+                }
+                for (; slotb < nslot; ++slotb) {
+                    s_bpv[p * nslot + slotb] = -1.0;
+                    s_bjv[p * nslot + slotb] = 0;
+                }
+            }
+            // lam_c = the largest breakpoint v with W(>= v) > budget - P*kmin (W: summed jumps):
+            // weighted radix select, 8 bits per pass, on the (non-negative) fp64 bit patterns
+            __shared__ int s_hist[256];
+            __shared__ unsigned long long s_prefix;
+            __shared__ double s_rem;
+            __shared__ int s_found;
+            const int nall = P * nslot;
+            if (tid == 0) {
+                s_prefix = 0ull;
+                s_rem = __dsub_rn(budget, static_cast<double>(P * a.kmin));
+                s_found = 1;
+            }
+            for (int pass = 0; pass < 8; ++pass) {
+                const int shift = 56 - 8 * pass;
+                for (int b = tid; b < 256; b += blockDim.x) s_hist[b] = 0;
+                __syncthreads();
+                const unsigned long long pre = s_prefix;
+                const unsigned long long hmask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+                if (s_found) {
+                    // the leading digits repeat across most keys: aggregate equal buckets per warp
+                    // before the shared-memory atomic
+                    for (int q0 = warp * 32; q0 < nall; q0 += blockDim.x) {
+                        const int q = q0 + lane;
+                        int bucket = -1, wgt = 0;
+                        if (q < nall) {
+                            const double v = s_bpv[q];
+                            if (v >= 0.0) {
+                                const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(v));
+                                if ((key & hmask) == pre) {
+                                    bucket = static_cast<int>((key >> shift) & 255u);
+                                    wgt = s_bjv[q];
+                                }
+                            }
+                        }
+                        const unsigned grp = __match_any_sync(0xffffffffu, bucket);
+                        const int tot = static_cast<int>(__reduce_add_sync(grp, static_cast<unsigned>(wgt)));
+                        if (bucket >= 0 && lane == __ffs(static_cast<int>(grp)) - 1) atomicAdd(&s_hist[bucket], tot);
+                    }
+                }
+                __syncthreads();
+                if (warp == 0 && s_found) {
+                    // lane l holds buckets 255-8l .. 248-8l; the first bucket from the top whose
+                    // cumulative weight exceeds the remainder is picked
+                    const double rem = s_rem;
+                    int part = 0;
+                    for (int u = 0; u < 8; ++u) part += s_hist[255 - 8 * lane - u];
+                    int incl = part;
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += t;
+                    }
+                    const int excl = incl - part;
+                    const bool crosses = static_cast<double>(incl) > rem && !(static_cast<double>(excl) > rem);
+                    const unsigned who = __ballot_sync(0xffffffffu, crosses);
+                    if (who == 0u) {
+                        if (lane == 0) s_found = 0;   // the jumps never exceed the budget: lam_c = 0
+                    } else if (lane == __ffs(static_cast<int>(who)) - 1) {
+                        int acc = excl, pick = -1;
+                        for (int u = 0; u < 8; ++u) {
+                            const int b = 255 - 8 * lane - u;
+                            const int h = s_hist[b];
+                            if (static_cast<double>(acc + h) > rem) { pick = b; break; }
+                            acc += h;
+                        }
+                        s_prefix = pre | (static_cast<unsigned long long>(pick) << shift);
+                        s_rem = __dsub_rn(rem, static_cast<double>(acc));
+                    }
+                }
+                __syncthreads();
+            }
+            if (tid == 0) {
+                const double lam_c = s_found ? __longlong_as_double(static_cast<long long>(s_prefix)) : 0.0;
+                double l = lo, h = hi;
+                for (int i = 0; i < 64; ++i) {   // replay with the real-arithmetic predicate
+                    s_lo[i] = l;
+                    s_hi[i] = h;
+                    const double m = midpoint(l, h);
+                    const int pr = m < lam_c ? 1 : 0;
+                    s_mid[i] = m;
+                    s_spred[i] = static_cast<unsigned char>(pr);
+                    if (pr) l = m; else h = m;
+                }
+                s_lo[64] = l;
+                s_hi[64] = h;
+            }
+            __syncthreads();
+            // exact check of the 64 recorded steps: warp w checks steps 2w and 2w+1 (32 warps)
+            for (int st0 = 2 * warp; st0 < 64; st0 += 2 * nw) {
+                const double m0 = s_mid[st0], m1 = s_mid[st0 + 1];
+                int n0 = 0, n1 = 0;
+                for (int p = lane; p < P; p += 32) {
+                    const double* c = s_costs + p * nk;
+                    n0 += choose_k(c, nk, a.kmin, m0);
+                    n1 += choose_k(c, nk, a.kmin, m1);
+                }
+                n0 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n0)));
+                n1 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n1)));
+                if (lane == 0) {
+                    s_pred[0][st0] = (static_cast<double>(n0) > budget ? 1 : 0) != s_spred[st0] ? 1 : 0;
+                    s_pred[0][st0 + 1] = (static_cast<double>(n1) > budget ? 1 : 0) != s_spred[st0 + 1] ? 1 : 0;
+                }
+            }
+            __syncthreads();
+            int it0 = 64;
+            for (int i = 0; i < 64; ++i)
+                if (s_pred[0][i]) { it0 = i; break; }
+            lo = s_lo[it0];
+            hi = s_hi[it0];
+            it_start = it0;
+            __syncthreads();   // s_pred is reused by the tree below
+        }
         // whole block: a group of gs threads per node, trees of depth D per round
         int gs_log = 0;
         while ((1 << gs_log) < 32 && (P >> (gs_log + 3)) > 0) ++gs_log;   // ~8 pairs per thread
@@ -338,7 +487,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         const int node_slot = tid >> gs_log;
         const int glane = tid & (gs - 1);
         int round = 0;
-        for (int it = 0; it < 64; ++round) {
+        for (int it = it_start; it < 64; ++round) {
             const int D = min(dmax, 64 - it);
             const int n_nodes = (1 << D) - 1;
             const int node = node_slot + 1;   // heap index

@@ -151,7 +151,11 @@ def _alloc_inputs(seed, T, K, E, B, ties=False):
 @pytest.mark.parametrize("T,K,E,kmin,kmax,B,target,ties", [
     (4, 2, 8, 2, 4, 4, 3.0, False), (1, 8, 128, 2, 4, 4, 2.5, False), (64, 8, 128, 2, 4, 4, 2.0, False),
     (64, 8, 128, 2, 4, 4, 3.5, False), (64, 8, 128, 2, 4, 4, 4.0, False), (16, 6, 64, 1, 3, 3, 2.0, False),
-    (2048, 8, 128, 2, 4, 4, 3.0, False), (7, 3, 16, 1, 4, 4, 2.75, False), (32, 8, 128, 2, 4, 4, 3.0, True)])
+    (2048, 8, 128, 2, 4, 4, 3.0, False), (7, 3, 16, 1, 4, 4, 2.75, False), (32, 8, 128, 2, 4, 4, 3.0, True),
+    # mid-size batches (block-scale speculation and verification): edge of the range, four
+    # plane counts, ties
+    (256, 8, 128, 2, 4, 4, 2.5, False), (100, 8, 128, 1, 4, 4, 1.7, False), (64, 8, 128, 2, 4, 4, 3.0, True),
+    (9, 8, 128, 2, 4, 4, 2.2, False)])
 def test_allocate_bit_exact(T, K, E, kmin, kmax, B, target, ties):
     shape = W.with_sizes(W.QWEN3_B1, n_experts=E, top_k=K, kmin=kmin, kmax=kmax, bits=B, name="alloc")
     d = dpa.make_desc(shape)
