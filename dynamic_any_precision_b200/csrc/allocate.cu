@@ -39,26 +39,42 @@ constexpr int kCoopDepth = 6;             // bisection steps per grid round (63 
 constexpr int kCoopMinPairs = 2048;       // below this the single-CTA bisection is faster
 static_assert((64 + kCoopDepth - 1) / kCoopDepth <= kCoopRoundsMax, "round counters");
 
-__device__ __forceinline__ int choose_k(const double* c, int nk, int kmin, double lam) {
-    double best = __dadd_rn(c[0], __dmul_rn(lam, static_cast<double>(kmin)));
+// The plane counts as fp64 constants, converted once per thread (an integer-to-fp64 conversion
+// inside the decision loops costs more than the decision itself), and the candidate loop
+// unrolled over the at most four counts (B <= 4).
+struct KVals {
+    double v[4];
+};
+__device__ __forceinline__ KVals make_kvals(int kmin) {
+    KVals k;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) k.v[i] = static_cast<double>(kmin + i);
+    return k;
+}
+
+__device__ __forceinline__ int choose_k(const double* c, int nk, int kmin, const KVals& kv, double lam) {
+    double best = __dadd_rn(c[0], __dmul_rn(lam, kv.v[0]));
     int kb = kmin;
-    for (int i = 1; i < nk; ++i) {
-        const double cost = __dadd_rn(c[i], __dmul_rn(lam, static_cast<double>(kmin + i)));
-        if (cost < best) { best = cost; kb = kmin + i; }
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+        if (i < nk) {
+            const double cost = __dadd_rn(c[i], __dmul_rn(lam, kv.v[i]));
+            if (cost < best) { best = cost; kb = kmin + i; }
+        }
     }
     return kb;
 }
 
 __device__ __forceinline__ double midpoint(double lo, double hi) { return __dmul_rn(0.5, __dadd_rn(lo, hi)); }
 
-// the same decision with the pair's costs in registers (nk <= 4 because B <= 4)
-__device__ __forceinline__ int choose_k_reg(const double (&c)[4], int nk, int kmin, double lam) {
-    double best = __dadd_rn(c[0], __dmul_rn(lam, static_cast<double>(kmin)));
+// the same decision with the pair's costs in registers
+__device__ __forceinline__ int choose_k_reg(const double (&c)[4], int nk, int kmin, const KVals& kv, double lam) {
+    double best = __dadd_rn(c[0], __dmul_rn(lam, kv.v[0]));
     int kb = kmin;
 #pragma unroll
     for (int i = 1; i < 4; ++i) {
         if (i < nk) {
-            const double cost = __dadd_rn(c[i], __dmul_rn(lam, static_cast<double>(kmin + i)));
+            const double cost = __dadd_rn(c[i], __dmul_rn(lam, kv.v[i]));
             if (cost < best) { best = cost; kb = kmin + i; }
         }
     }
@@ -135,6 +151,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     __shared__ unsigned s_mis[4];
     const int P = a.T * a.K;
     const int nk = a.kmax - a.kmin + 1;
+    const KVals kv = make_kvals(a.kmin);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const AllocSmem Ls = alloc_smem_layout(P, a.E, nk);
     double* c_base = Ls.costs_in_smem ? reinterpret_cast<double*>(smem + Ls.costs) : a.cbuf;
@@ -270,7 +287,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             const int node = tid >> 1, gl2 = tid & 1;
             int n = 0;
             const double m = s_mid[node];
-            for (int p = gl2; p < P; p += 2) n += choose_k(s_costs + p * nk, nk, a.kmin, m);
+            for (int p = gl2; p < P; p += 2) n += choose_k(s_costs + p * nk, nk, a.kmin, kv, m);
             n += __shfl_xor_sync(0xffffffffu, n, 1);
             const int pr = static_cast<double>(n) > budget ? 1 : 0;
             const unsigned bad_mask = __ballot_sync(0xffffffffu, gl2 == 0 && pr != s_spred[node]);
@@ -300,15 +317,15 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                 if (in_regs) {
 #pragma unroll
                     for (int j = 0; j < kRegPairs; ++j)
-                        if (gl + 4 * j < P) n += choose_k_reg(creg[j], nk, a.kmin, mid);
+                        if (gl + 4 * j < P) n += choose_k_reg(creg[j], nk, a.kmin, kv, mid);
                 } else {
                     int n0 = 0, n1 = 0;
                     int p = gl;
                     for (; p + 4 < P; p += 8) {   // two independent pairs per iteration
-                        n0 += choose_k(s_costs + p * nk, nk, a.kmin, mid);
-                        n1 += choose_k(s_costs + (p + 4) * nk, nk, a.kmin, mid);
+                        n0 += choose_k(s_costs + p * nk, nk, a.kmin, kv, mid);
+                        n1 += choose_k(s_costs + (p + 4) * nk, nk, a.kmin, kv, mid);
                     }
-                    if (p < P) n0 += choose_k(s_costs + p * nk, nk, a.kmin, mid);
+                    if (p < P) n0 += choose_k(s_costs + p * nk, nk, a.kmin, kv, mid);
                     n = n0 + n1;
                 }
             }
@@ -458,8 +475,8 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                 int n0 = 0, n1 = 0;
                 for (int p = lane; p < P; p += 32) {
                     const double* c = s_costs + p * nk;
-                    n0 += choose_k(c, nk, a.kmin, m0);
-                    n1 += choose_k(c, nk, a.kmin, m1);
+                    n0 += choose_k(c, nk, a.kmin, kv, m0);
+                    n1 += choose_k(c, nk, a.kmin, kv, m1);
                 }
                 n0 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n0)));
                 n1 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n1)));
@@ -501,7 +518,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                     if ((node >> lev) & 1) l = m; else h = m;
                 }
                 const double mid = midpoint(l, h);
-                for (int p = glane; p < P; p += gs) local += choose_k(c_base + static_cast<size_t>(p) * nk, nk, a.kmin, mid);
+                for (int p = glane; p < P; p += gs) local += choose_k(c_base + static_cast<size_t>(p) * nk, nk, a.kmin, kv, mid);
             }
             // every lane of the warp takes part in the group reduction (inactive lanes add 0)
             for (int o = gs >> 1; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
@@ -519,7 +536,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     }
     // final plane counts
     for (int p = tid; p < P; p += blockDim.x) {
-        const int k = choose_k(c_base + static_cast<size_t>(p) * nk, nk, a.kmin, hi);
+        const int k = choose_k(c_base + static_cast<size_t>(p) * nk, nk, a.kmin, kv, hi);
         a.k_out[p] = static_cast<uint8_t>(k);
         s_k[p] = static_cast<uint8_t>(k);
     }
@@ -664,6 +681,7 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
     __shared__ int s_flag;
     const int P = a.T * a.K;
     const int nk = a.kmax - a.kmin + 1;
+    const KVals kv = make_kvals(a.kmin);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     const unsigned G = gridDim.x;
     const int p0 = blockIdx.x * per_block, p1 = min(P, p0 + per_block), np = max(0, p1 - p0);
@@ -731,14 +749,7 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
             const double m = s_mid[node];
             int n = 0;
             for (int j = lane; j < np; j += 32) {
-                const double* c = s_c + 4 * j;
-                double best = __dadd_rn(c[0], __dmul_rn(m, static_cast<double>(a.kmin)));
-                int kb = a.kmin;
-                for (int i = 1; i < nk; ++i) {
-                    const double cost = __dadd_rn(c[i], __dmul_rn(m, static_cast<double>(a.kmin + i)));
-                    if (cost < best) { best = cost; kb = a.kmin + i; }
-                }
-                n += kb;
+                n += choose_k(s_c + 4 * j, nk, a.kmin, kv, m);
             }
             n = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n)));
             if (lane == 0 && n) atomicAdd(&cs->counts[round][node][0], n);
@@ -755,14 +766,7 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
         it += D;
     }
     for (int j = tid; j < np; j += blockDim.x) {
-        const double* c = s_c + 4 * j;
-        double best = __dadd_rn(c[0], __dmul_rn(hi, static_cast<double>(a.kmin)));
-        int kb = a.kmin;
-        for (int i = 1; i < nk; ++i) {
-            const double cost = __dadd_rn(c[i], __dmul_rn(hi, static_cast<double>(a.kmin + i)));
-            if (cost < best) { best = cost; kb = a.kmin + i; }
-        }
-        a.k_out[p0 + j] = static_cast<uint8_t>(kb);
+        a.k_out[p0 + j] = static_cast<uint8_t>(choose_k(s_c + 4 * j, nk, a.kmin, kv, hi));
     }
     if (blockIdx.x == 0 && tid == 0 && a.lambda_out) *a.lambda_out = hi;
 }

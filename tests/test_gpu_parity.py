@@ -155,7 +155,12 @@ def _alloc_inputs(seed, T, K, E, B, ties=False):
     # mid-size batches (block-scale speculation and verification): edge of the range, four
     # plane counts, ties
     (256, 8, 128, 2, 4, 4, 2.5, False), (100, 8, 128, 1, 4, 4, 1.7, False), (64, 8, 128, 2, 4, 4, 3.0, True),
-    (9, 8, 128, 2, 4, 4, 2.2, False)])
+    (9, 8, 128, 2, 4, 4, 2.2, False),
+    # up to 32 pairs (one warp): a single pair, the 32-pair edge, budgets at kmin and kmax,
+    # duplicated pairs, three-plane BCQ-like ranges; 33 pairs falls back to the block kernel
+    (1, 1, 8, 1, 4, 4, 1.0, False), (1, 1, 8, 1, 4, 4, 2.6, False), (4, 8, 128, 2, 4, 4, 2.0, False),
+    (4, 8, 128, 2, 4, 4, 4.0, False), (4, 8, 128, 2, 4, 4, 3.3, False), (4, 8, 128, 2, 4, 4, 2.5, True),
+    (5, 6, 64, 1, 3, 3, 2.0, False), (2, 8, 128, 2, 4, 4, 3.1, False), (11, 3, 16, 1, 4, 4, 2.4, False)])
 def test_allocate_bit_exact(T, K, E, kmin, kmax, B, target, ties):
     shape = W.with_sizes(W.QWEN3_B1, n_experts=E, top_k=K, kmin=kmin, kmax=kmax, bits=B, name="alloc")
     d = dpa.make_desc(shape)
