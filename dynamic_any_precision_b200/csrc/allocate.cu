@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     uint8_t* s_k = smem + Ls.kk;
 
     pdl_wait();   // the routed pairs come from the previous kernel
+    pdl_trigger();   // the successor may become resident now (it waits for this kernel)
     // the budget, the pairs' experts and gates are loaded together (one round trip)
     const double target = *a.target;
     int bad = (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1;

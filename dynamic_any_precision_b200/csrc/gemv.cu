@@ -176,13 +176,30 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
         mbar_init(&s_bar, 1);
         fence_barrier_init();
     }
+    const int dstride = Ly.dig_stride;
+    // A single token (P == K) sits in the first half of every tile. Its digits were written by
+    // the router two launches back, which completed before the previous launch passed its own
+    // dependency wait, so they are staged before this kernel's wait (L2 reads).
+    const bool single = NT == 1 && a.P == a.K;
+    if (single) {
+        const int chunks = (3 * H) >> 4;
+        for (int c = threadIdx.x; c < 2 * chunks; c += kThreads) {
+            const int slot = c / chunks, cc = c - slot * chunks;
+            const uint4 v = slot == 0 ? __ldcg(reinterpret_cast<const uint4*>(a.xdig) + cc) : make_uint4(0u, 0u, 0u, 0u);
+            const int d_ = (16 * cc) / H, col = 16 * cc - d_ * H;
+            *reinterpret_cast<uint4*>(s_dig + (slot * 3 + d_) * dstride + col) = v;
+        }
+        for (int i = threadIdx.x; i < 2 * ng; i += kThreads) {
+            s_xe[i] = i < ng ? __ldcg(a.xexp + i) : 0;
+            s_xs[i] = i < ng ? __ldcg(a.xsum + i) : 0;
+        }
+    }
     pdl_wait();   // work lists and activations come from the previous kernels
     const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     __syncthreads();
     uint32_t phase = 0;
     const int g0 = (warp * ng) / kWarps, g1 = ((warp + 1) * ng) / kWarps;   // this warp's groups
     const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
-    const int dstride = Ly.dig_stride;
 
     // the first item's descriptor is loaded together with the active count (the index is in
     // bounds for every launched CTA; its contents are used only if the item exists)
@@ -231,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
             const int nt = s_nt;
             // stage the digits, exponents and sums of the pass's tokens (loads issued first);
             // multi-token kernels read them from global memory instead (L1/L2 resident)
-            if constexpr (NT == 1) {
+            if (NT == 1 && !single) {
                 const int chunks = (3 * H) >> 4;
                 for (int i0 = threadIdx.x; i0 < 2 * NT * chunks; i0 += 4 * kThreads) {
                     uint4 v[4];
