@@ -82,6 +82,9 @@ __device__ __forceinline__ int choose_k_reg(const double (&c)[4], int nk, int km
 }
 
 constexpr int kRegPairs = 4;   // pairs per lane held in registers by the small-batch bisection
+// 1/d for the plane-count gap d = 1..3 of a hull breakpoint (B <= 4); the breakpoints only
+// steer the speculation, so a rounded 1/3 is fine
+__device__ __forceinline__ double inv_gap(int d) { return d == 1 ? 1.0 : (d == 2 ? 0.5 : 1.0 / 3.0); }
 
 // inclusive block scan of one int per thread
 __device__ __forceinline__ int block_incl_scan(int v, int* s_tmp) {
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     __shared__ int s_nbp;
     __shared__ double s_mid[64], s_lo[65], s_hi[65];
     __shared__ unsigned char s_spred[64];
-    __shared__ unsigned s_mis[4];
+    __shared__ unsigned s_mis[8];
     const int P = a.T * a.K;
     const int nk = a.kmax - a.kmin + 1;
     const KVals kv = make_kvals(a.kmin);
@@ -209,11 +212,12 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     for (int w = 1; w < nw; ++w) mx = fmax(mx, s_max[w]);
 
     const double budget = __dmul_rn(target, static_cast<double>(P));
+    const int nb = static_cast<int>(floor(budget));   // an integer count n exceeds budget iff n > nb
     double lo = 0.0;
     double hi = __dadd_rn(__dmul_rn(2.0, mx), 1.0);
 
     if (P <= kSmallP) {
-        // 4 warps, 4 lanes per node: 32 node slots hold the 31 midpoints of the next 5 steps.
+        // 8 warps, 4 lanes per node: 64 node slots hold the 63 midpoints of the next 6 steps.
         // Each lane counts planes for every 4th pair; the 4-lane sums give N(mid); each warp's
         // 8 predicates travel through shared memory as one byte, and every thread walks the
         // tree in registers.
@@ -245,7 +249,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                 int jn = -1;
                 double tn = 0.0;
                 for (int j = 0; j < cur; ++j) {   // the next smaller k to take over as lambda grows
-                    const double t = (c[j] - c[cur]) / static_cast<double>(cur - j);
+                    const double t = __dmul_rn(__dsub_rn(c[j], c[cur]), inv_gap(cur - j));
                     if (jn < 0 || t < tn) { jn = j; tn = t; }
                 }
                 const int slotb = atomicAdd(&s_nbp, 1);
@@ -268,7 +272,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             int cum = P * a.kmin;
             for (int m = 0; m < nbp; ++m) {
                 cum += s_bj[s_order[m]];
-                if (static_cast<double>(cum) > budget) { lam_c = s_bp[s_order[m]]; break; }
+                if (cum > nb) { lam_c = s_bp[s_order[m]]; break; }
             }
             double l = lo, h = hi;
             for (int i = 0; i < 64; ++i) {
@@ -284,26 +288,27 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             s_hi[64] = h;
         }
         __syncthreads();
-        {   // exact check of the 64 recorded steps: two threads per step
-            const int node = tid >> 1, gl2 = tid & 1;
+        {   // exact check of the 64 recorded steps: four threads per step
+            const int node = tid >> 2, gl4 = tid & 3;
             int n = 0;
             const double m = s_mid[node];
-            for (int p = gl2; p < P; p += 2) n += choose_k(s_costs + p * nk, nk, a.kmin, kv, m);
+            for (int p = gl4; p < P; p += 4) n += choose_k(s_costs + p * nk, nk, a.kmin, kv, m);
             n += __shfl_xor_sync(0xffffffffu, n, 1);
-            const int pr = static_cast<double>(n) > budget ? 1 : 0;
-            const unsigned bad_mask = __ballot_sync(0xffffffffu, gl2 == 0 && pr != s_spred[node]);
-            if (lane == 0) s_mis[warp] = bad_mask;   // bit 2j of warp w: step 16w + j
+            n += __shfl_xor_sync(0xffffffffu, n, 2);
+            const int pr = n > nb ? 1 : 0;
+            const unsigned bad_mask = __ballot_sync(0xffffffffu, gl4 == 0 && pr != s_spred[node]);
+            if (lane == 0) s_mis[warp] = bad_mask;   // bit 4j of warp w: step 8w + j
         }
         __syncthreads();
         int it0 = 64;
-        for (int w = 0; w < 4 && it0 == 64; ++w)
-            if (s_mis[w]) it0 = 16 * w + (__ffs(static_cast<int>(s_mis[w])) - 1) / 2;
+        for (int w = 0; w < 8 && it0 == 64; ++w)
+            if (s_mis[w]) it0 = 8 * w + (__ffs(static_cast<int>(s_mis[w])) - 1) / 4;
         lo = s_lo[it0];
         hi = s_hi[it0];
 
         int round = 0;
         for (int it = it0; it < 64; ++round) {
-            const int D = min(5, 64 - it);
+            const int D = min(6, 64 - it);
             const int node = slot + 1;
             const bool active = node < (1 << D);
             int n = 0;
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             }
             n += __shfl_xor_sync(0xffffffffu, n, 1);
             n += __shfl_xor_sync(0xffffffffu, n, 2);
-            const int pred = (active && static_cast<double>(n) > budget) ? 1 : 0;
+            const int pred = (active && n > nb) ? 1 : 0;
             const unsigned bal = __ballot_sync(0xffffffffu, pred && gl == 0);   // bits 4*i: node 8*warp+i+1
             if (lane == 0) {
                 unsigned b = 0;
@@ -340,13 +345,12 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                 s_pred[round & 1][warp] = static_cast<unsigned char>(b);
             }
             __syncthreads();
-            const unsigned mask = static_cast<unsigned>(s_pred[round & 1][0]) |
-                                  (static_cast<unsigned>(s_pred[round & 1][1]) << 8) |
-                                  (static_cast<unsigned>(s_pred[round & 1][2]) << 16) |
-                                  (static_cast<unsigned>(s_pred[round & 1][3]) << 24);   // bit node-1
+            unsigned long long mask = 0ull;   // bit node-1
+#pragma unroll
+            for (int w = 0; w < 8; ++w) mask |= static_cast<unsigned long long>(s_pred[round & 1][w]) << (8 * w);
             int nd = 1;
             for (int lev = 0; lev < D; ++lev) {
-                const int pr = (mask >> (nd - 1)) & 1;
+                const int pr = static_cast<int>((mask >> (nd - 1)) & 1ull);
                 const double m = midpoint(lo, hi);
                 if (pr) lo = m; else hi = m;
                 nd = 2 * nd + pr;
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                     int jn = -1;
                     double tn = 0.0;
                     for (int j = 0; j < cur; ++j) {
-                        const double t = (c[j] - c[cur]) / static_cast<double>(cur - j);
+                        const double t = __dmul_rn(__dsub_rn(c[j], c[cur]), inv_gap(cur - j));
                         if (jn < 0 || t < tn) { jn = j; tn = t; }
                     }
                     s_bpv[p * nslot + slotb] = tn;
@@ -482,8 +486,8 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                 n0 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n0)));
                 n1 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n1)));
                 if (lane == 0) {
-                    s_pred[0][st0] = (static_cast<double>(n0) > budget ? 1 : 0) != s_spred[st0] ? 1 : 0;
-                    s_pred[0][st0 + 1] = (static_cast<double>(n1) > budget ? 1 : 0) != s_spred[st0 + 1] ? 1 : 0;
+                    s_pred[0][st0] = (n0 > nb ? 1 : 0) != s_spred[st0] ? 1 : 0;
+                    s_pred[0][st0 + 1] = (n1 > nb ? 1 : 0) != s_spred[st0 + 1] ? 1 : 0;
                 }
             }
             __syncthreads();
@@ -523,7 +527,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             }
             // every lane of the warp takes part in the group reduction (inactive lanes add 0)
             for (int o = gs >> 1; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-            if (active && glane == 0) s_pred[round & 1][node] = static_cast<double>(local) > budget ? 1 : 0;
+            if (active && glane == 0) s_pred[round & 1][node] = local > nb ? 1 : 0;
             __syncthreads();
             int node_w = 1;
             for (int lev = 0; lev < D; ++lev) {
@@ -728,6 +732,7 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
     }
     mx = __longlong_as_double(static_cast<long long>(__ldcg(&cs->mx_bits)));
     const double budget = __dmul_rn(target, static_cast<double>(P));
+    const int nb = static_cast<int>(floor(budget));   // an integer count n exceeds budget iff n > nb
     double lo = 0.0;
     double hi = __dadd_rn(__dmul_rn(2.0, mx), 1.0);
 
@@ -759,7 +764,7 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
         int nd = 1;
         for (int lev = 0; lev < D; ++lev) {
             const int n = __ldcg(&cs->counts[round][nd][0]);
-            const int pr = static_cast<double>(n) > budget ? 1 : 0;
+            const int pr = n > nb ? 1 : 0;
             const double m = midpoint(lo, hi);
             if (pr) lo = m; else hi = m;
             nd = 2 * nd + pr;
@@ -776,7 +781,7 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
 
 size_t allocate_smem_bytes(int P, int E, int nk) { return alloc_smem_layout(P, E, nk).total; }
 
-int allocate_threads(int P) { return P <= kSmallP ? 128 : kAllocThreads; }   // small: 4 warps x 8 nodes
+int allocate_threads(int P) { return P <= kSmallP ? 256 : kAllocThreads; }   // small: 8 warps x 8 nodes
 
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* coop, int sms) {
     const int nk = a.kmax - a.kmin + 1;
