@@ -22,7 +22,8 @@ namespace dpa {
 namespace {
 
 constexpr int kRouteWarps = 8;
-constexpr int kPrefetch = 8;   // router-row uint4 loads a lane issues at once
+// Router-row uint4 loads a lane issues at once (PF, a template parameter of the per-logit kernel):
+// the number a lane needs in total when that is at most 8, so that no unrolled slot idles.
 constexpr int16_t kNoBit = 0x3FFF;   // lowest-set-bit marker of a zero element
 constexpr int kRouteTiledMinTokens = 128;   // from here on the logits run as a tiled GEMM
 constexpr int kMaxLsbBlocks = 256;          // H <= 16384 on the tiled path
@@ -311,6 +312,7 @@ __device__ void select_topk_gates(const RouteArgs& a, int t, unsigned char* smem
     }
 }
 
+template <int PF>
 __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const int H = a.H, E = a.E, H8 = H >> 3;
@@ -332,11 +334,11 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
     const int e = blockIdx.x * (kRouteWarps / wpe) + warp / wpe;
     const int wstride = 32 * wpe;                       // uint4 columns per round
     const int nq = (H8 + wstride - 1) / wstride;
-    uint4 wpre[kPrefetch];
+    uint4 wpre[PF];
     if (e < E) {
         const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H);
 #pragma unroll
-        for (int u = 0; u < kPrefetch; ++u) {
+        for (int u = 0; u < PF; ++u) {
             const int col = u * wstride + part * 32 + lane;
             if (u < nq && col < H8) wpre[u] = wrow[col];
         }
@@ -380,16 +382,16 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
         bool wbad = false;
         if (e < E) {
             const uint4* wrow = reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e) * H);
-            for (int q0 = 0; q0 < nq; q0 += kPrefetch) {
-                uint4 wv[kPrefetch];
+            for (int q0 = 0; q0 < nq; q0 += PF) {
+                uint4 wv[PF];
 #pragma unroll
-                for (int u = 0; u < kPrefetch; ++u) {
+                for (int u = 0; u < PF; ++u) {
                     const int col = (q0 + u) * wstride + part * 32 + lane;
                     if (q0 == 0) wv[u] = wpre[u];
                     else if (q0 + u < nq && col < H8) wv[u] = wrow[col];
                 }
 #pragma unroll
-                for (int u = 0; u < kPrefetch; ++u) {
+                for (int u = 0; u < PF; ++u) {
                     const int col = (q0 + u) * wstride + part * 32 + lane;   // 8-element group index
                     if (q0 + u < nq && col < H8) {
                         const uint32_t ww[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
@@ -716,14 +718,17 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms) {
     const size_t need_vals = static_cast<size_t>(a.E) * 24;   // logits, keys and exps
     if (need_vals > smem) smem = need_vals;
     smem = (smem + 15) & ~static_cast<size_t>(15);
+    const int nq = (a.H / 8 + 32 * b.wpe - 1) / (32 * b.wpe);   // uint4 router loads per lane
+    const void* fn = nq <= 2 ? reinterpret_cast<const void*>(route_kernel<2>)
+                             : (nq <= 4 ? reinterpret_cast<const void*>(route_kernel<4>)
+                                        : reinterpret_cast<const void*>(route_kernel<8>));
     if (smem > 48 * 1024) {
-        cudaError_t err = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
+        cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (err != cudaSuccess) return err;
     }
     dim3 grid(chunks, a.T);
     void* args[] = {&b};
-    return launch_pdl_raw(reinterpret_cast<const void*>(route_kernel), grid, dim3(kRouteWarps * 32), smem, stream, args);
+    return launch_pdl_raw(fn, grid, dim3(kRouteWarps * 32), smem, stream, args);
 }
 
 
