@@ -104,6 +104,37 @@ __device__ __forceinline__ void load_b(const int8_t* row, int b, int tq, uint32_
     b1H = *reinterpret_cast<const uint32_t*>(src + 48);
 }
 
+
+// Bulk copies (no multicast) of one pass's activation digits into the padded shared slots:
+// lane s of warp 0 (s < 2 NT) copies the three W-byte digit rows of its slot's source row
+// src (a token, or a pair position) and, when copy_es, its ng exponents and sums. Empty slots
+// get zero exponents and sums. One arrive with the total byte count completes the barrier.
+template <int NT>
+__device__ __forceinline__ void issue_digit_copies(int src, const int8_t* dig, const int32_t* ex, const int32_t* sm, int W,
+                                                   int ng, bool copy_es, int8_t* s_dig, int dstride, int* s_xe, int* s_xs,
+                                                   uint64_t* bar) {
+    const int lane = threadIdx.x & 31;
+    const unsigned valid = __ballot_sync(0xffffffffu, lane < 2 * NT && src >= 0);
+    if (lane == 0) {
+        const uint32_t per = 3u * static_cast<uint32_t>(W) + (copy_es ? 8u * static_cast<uint32_t>(ng) : 0u);
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(__popc(valid)) * per);
+    }
+    __syncwarp();
+    if (lane < 2 * NT) {
+        if (src >= 0) {
+            fence_proxy_async();   // the CTA's earlier generic reads of the slot precede the copies
+            const int8_t* row = dig + static_cast<size_t>(src) * 3 * W;
+            for (int d = 0; d < 3; ++d) bulk_g2s(s_dig + (lane * 3 + d) * dstride, row + d * W, static_cast<uint32_t>(W), bar);
+            if (copy_es) {
+                bulk_g2s(s_xe + lane * ng, ex + static_cast<size_t>(src) * ng, static_cast<uint32_t>(ng) * 4u, bar);
+                bulk_g2s(s_xs + lane * ng, sm + static_cast<size_t>(src) * ng, static_cast<uint32_t>(ng) * 4u, bar);
+            }
+        } else if (copy_es) {
+            for (int g = 0; g < ng; ++g) { s_xe[lane * ng + g] = 0; s_xs[lane * ng + g] = 0; }
+        }
+    }
+}
+
 struct Layout {
     // byte offsets inside dynamic shared memory
     size_t planes, meta, dig, xe, xs, red, total;
@@ -122,8 +153,7 @@ __host__ __device__ inline Layout gateup_layout(int H, int G, int B, int fmt, in
                                                      : static_cast<size_t>(2) * B * 16 * ng * 2;
     L.dig = align16(L.meta + meta_bytes);
     L.dig_stride = H + kDigPad;
-    // multi-token kernels read the digits from global memory (no staged copy)
-    const size_t sl = NT == 1 ? static_cast<size_t>(2 * NT) : 0;
+    const size_t sl = static_cast<size_t>(2 * NT);   // token slots of one pass
     L.xe = align16(L.dig + sl * 3 * L.dig_stride);
     L.xs = align16(L.xe + sl * ng * 4);
     L.red = align16(L.xs + sl * ng * 4);
@@ -141,7 +171,7 @@ __host__ __device__ inline Layout down_layout(int I, int G, int B, int fmt, int 
                                                      : static_cast<size_t>(B) * 64 * ng * 2;
     L.dig = align16(L.meta + meta_bytes);
     L.dig_stride = I + kDigPad;
-    const size_t sl = NT == 1 ? static_cast<size_t>(2 * NT) : 0;
+    const size_t sl = static_cast<size_t>(2 * NT);   // pair slots of one pass
     L.xe = align16(L.dig + sl * 3 * L.dig_stride);
     L.xs = align16(L.xe + sl * ng * 4);
     L.red = align16(L.xs + sl * ng * 4);
@@ -153,7 +183,7 @@ __host__ __device__ inline Layout down_layout(int I, int G, int B, int fmt, int 
 // gate + up projections, SwiGLU epilogue -> h[pos][I]
 // ---------------------------------------------------------------------------------------
 template <int FMT, int B, int NT>
-__global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kThreads, NT > 1 ? 2 : 0) gateup_kernel(GemvArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int H = a.H, I = a.I, G = a.G;
     const int nblk = H >> 6, ng = H / G, bpg = G >> 6;
@@ -165,7 +195,7 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
     int* s_xe = reinterpret_cast<int*>(smem + Ly.xe);
     int* s_xs = reinterpret_cast<int*>(smem + Ly.xs);
     float* s_red = reinterpret_cast<float*>(smem + Ly.red);
-    __shared__ uint64_t s_bar;
+    __shared__ uint64_t s_bar, s_bard;   // planes and scales; the pass's digits
     __shared__ int s_flag;
     __shared__ int4 s_tile[NT];
     __shared__ int s_nt;
@@ -174,6 +204,7 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
     const int gid = lane >> 2, tq = lane & 3;
     if (threadIdx.x == 0) {
         mbar_init(&s_bar, 1);
+        mbar_init(&s_bard, 1);
         fence_barrier_init();
     }
     const int dstride = Ly.dig_stride;
@@ -197,7 +228,8 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
     pdl_wait();   // work lists and activations come from the previous kernels
     const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     __syncthreads();
-    uint32_t phase = 0;
+    uint32_t phase = 0, phase_d = 0;
+    const bool copy_es = (ng & 3) == 0;   // exponent and sum rows are whole 16-byte units
     const int g0 = (warp * ng) / kWarps, g1 = ((warp + 1) * ng) / kWarps;   // this warp's groups
     const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
 
@@ -246,8 +278,8 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
             if (threadIdx.x == 0) s_nt = min(NT, ntiles - pass0);
             __syncthreads();
             const int nt = s_nt;
-            // stage the digits, exponents and sums of the pass's tokens (loads issued first);
-            // multi-token kernels read them from global memory instead (L1/L2 resident)
+            // stage the digits, exponents and sums of the pass's tokens: loads issued first
+            // (one- and two-token passes), or bulk copies (multi-token passes)
             if (NT == 1 && !single) {
                 const int chunks = (3 * H) >> 4;
                 for (int i0 = threadIdx.x; i0 < 2 * NT * chunks; i0 += 4 * kThreads) {
@@ -280,6 +312,22 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                     s_xs[i] = tok >= 0 ? a.xsum[tok * ng + g] : 0;
                 }
             }
+            if constexpr (NT > 1) {
+                if (warp == 0)
+                    issue_digit_copies<NT>(lane < 2 * NT ? tile_tok(s_tile[lane >> 1], lane & 1) : -1, a.xdig, a.xexp,
+                                           a.xsum, H, ng, copy_es, s_dig, dstride, s_xe, s_xs, &s_bard);
+                if (!copy_es) {
+                    for (int i = threadIdx.x; i < 2 * NT * ng; i += kThreads) {
+                        const int slot = i / ng, g = i - slot * ng;
+                        const int tok = tile_tok(s_tile[slot >> 1], slot & 1);
+                        s_xe[i] = tok >= 0 ? a.xexp[tok * ng + g] : 0;
+                        s_xs[i] = tok >= 0 ? a.xsum[tok * ng + g] : 0;
+                    }
+                }
+                const bool okd = cta_wait_copies(&s_bard, phase_d, a.hdr, 104, &s_flag);
+                phase_d ^= 1;
+                if (!okd) return;
+            }
             if (!waited) {
                 waited = true;
                 const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 100, &s_flag);
@@ -299,11 +347,7 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
             for (int i = 0; i < NT; ++i) {
                 const int slot = 2 * i + half;
                 const int tk_ = tile_tok(s_tile[i], half);
-                if constexpr (NT == 1)
-                    brow[i] = (i < nt && dig < 3 && tk_ >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
-                else
-                    brow[i] = (i < nt && dig < 3 && tk_ >= 0) ? a.xdig + static_cast<size_t>(tk_) * 3 * H + dig * H
-                                                              : nullptr;
+                brow[i] = (i < nt && dig < 3 && tk_ >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
             }
             for (int g = g0; g < g1; ++g) {
                 if constexpr (FMT == DPA_FMT_UNIFORM) {
@@ -358,14 +402,8 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                             const int ki = s_tile[i].x;
                             const float ck = 0.5f * static_cast<float>((1 << (B - ki)) - 1);
                             int Eg, SX;
-                            if constexpr (NT == 1) {
-                                Eg = s_xe[slot * ng + g];
-                                SX = s_xs[slot * ng + g];
-                            } else {
-                                const int tk_ = tile_tok(s_tile[i], my_half);
-                                Eg = tk_ >= 0 ? __ldg(a.xexp + tk_ * ng + g) : 0;
-                                SX = tk_ >= 0 ? __ldg(a.xsum + tk_ * ng + g) : 0;
-                            }
+                            Eg = s_xe[slot * ng + g];
+                            SX = s_xs[slot * ng + g];
                             const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                             for (int m = 0; m < 2; ++m) {
@@ -429,14 +467,8 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
                                 if (i < nt && s_tile[i].x > p) {
                                     const int slot = 2 * i + my_half;
                                     int Eg, SX;
-                            if constexpr (NT == 1) {
-                                Eg = s_xe[slot * ng + g];
-                                SX = s_xs[slot * ng + g];
-                            } else {
-                                const int tk_ = tile_tok(s_tile[i], my_half);
-                                Eg = tk_ >= 0 ? __ldg(a.xexp + tk_ * ng + g) : 0;
-                                SX = tk_ >= 0 ? __ldg(a.xsum + tk_ * ng + g) : 0;
-                            }
+                            Eg = s_xe[slot * ng + g];
+                            SX = s_xs[slot * ng + g];
                                     const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                                     for (int m = 0; m < 2; ++m) {
@@ -496,7 +528,7 @@ __global__ void __launch_bounds__(kThreads) gateup_kernel(GemvArgs a) {
 // down projection: out_pair[pos][H] = W_down^(k) h[pos]
 // ---------------------------------------------------------------------------------------
 template <int FMT, int B, int NT>
-__global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
+__global__ void __launch_bounds__(kThreads, NT > 1 ? 2 : 0) down_kernel(GemvArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int H = a.H, I = a.I, G = a.G;
     const int nblk = I >> 6, ng = I / G, bpg = G >> 6;
@@ -508,7 +540,7 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
     int* s_xe = reinterpret_cast<int*>(smem + Ly.xe);
     int* s_xs = reinterpret_cast<int*>(smem + Ly.xs);
     float* s_red = reinterpret_cast<float*>(smem + Ly.red);   // [2 halves][4 tiles][NT][2][16]
-    __shared__ uint64_t s_bar;
+    __shared__ uint64_t s_bar, s_bard;   // planes and scales; the pass's h digits (multi-token)
     __shared__ int s_flag;
     __shared__ int4 s_tile[NT];
     __shared__ int s_nt;
@@ -517,12 +549,13 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
     const int gid = lane >> 2, tq = lane & 3;
     if (threadIdx.x == 0) {
         mbar_init(&s_bar, 1);
+        mbar_init(&s_bard, 1);
         fence_barrier_init();
     }
     pdl_wait();   // work lists and activations come from the previous kernels
     const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     __syncthreads();
-    uint32_t phase = 0;
+    uint32_t phase = 0, phase_d = 0;
     const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
     const int dstride = Ly.dig_stride;
 
@@ -568,7 +601,6 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
             const int nt = s_nt;
             // fixed-point digits of the pass's h rows: one warp per (slot, group); a lane holds
             // 4 consecutive values per 128-column chunk, all loaded before use
-            // (multi-token kernels read the digits written by hdigits_kernel)
             for (int task = warp; NT == 1 && task < 2 * NT * ng; task += kWarps) {
                 const int slot = task / ng, g = task - slot * ng;
                 const int4 t = s_tile[slot >> 1];
@@ -613,6 +645,24 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                 for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
                 if (lane == 0) { s_xe[slot * ng + g] = Eg; s_xs[slot * ng + g] = sum; }
             }
+            if constexpr (NT > 1) {   // digits of every h row were written by hdigits_kernel
+                if (warp == 0)
+                    issue_digit_copies<NT>(lane < 2 * NT ? ((lane & 1) ? s_tile[lane >> 1].z : s_tile[lane >> 1].y) : -1,
+                                           a.hdig, a.hexp, a.hsum, I, ng, (ng & 3) == 0, s_dig, dstride, s_xe, s_xs,
+                                           &s_bard);
+                if ((ng & 3) != 0) {
+                    for (int i = threadIdx.x; i < 2 * NT * ng; i += kThreads) {
+                        const int slot = i / ng, g = i - slot * ng;
+                        const int4 t = s_tile[slot >> 1];
+                        const int pos = (slot & 1) ? t.z : t.y;
+                        s_xe[i] = pos >= 0 ? a.hexp[pos * ng + g] : 0;
+                        s_xs[i] = pos >= 0 ? a.hsum[pos * ng + g] : 0;
+                    }
+                }
+                const bool okd = cta_wait_copies(&s_bard, phase_d, a.hdr, 204, &s_flag);
+                phase_d ^= 1;
+                if (!okd) return;
+            }
             if (!waited) {
                 waited = true;
                 const bool ok = cta_wait_copies(&s_bar, phase, a.hdr, 200, &s_flag);
@@ -631,11 +681,7 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                 const int slot = 2 * i + half;
                 const int4 t = s_tile[i];
                 const int pos = half ? t.z : t.y;
-                if constexpr (NT == 1)
-                    brow[i] = (i < nt && dig < 3 && pos >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
-                else
-                    brow[i] = (i < nt && dig < 3 && pos >= 0) ? a.hdig + static_cast<size_t>(pos) * 3 * I + dig * I
-                                                              : nullptr;
+                brow[i] = (i < nt && dig < 3 && pos >= 0) ? s_dig + (slot * 3 + dig) * dstride : nullptr;
             }
             const int rtile = warp & 3, khalf = warp >> 2;   // row tile of 4, half of the groups
             const uint32_t* wplanes = s_planes + static_cast<size_t>(rtile) * nblk * 32;
@@ -684,14 +730,8 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                             const int ki = s_tile[i].x;
                             const float ck = 0.5f * static_cast<float>((1 << (B - ki)) - 1);
                             int Eg, SX;
-                            if constexpr (NT == 1) {
-                                Eg = s_xe[slot * ng + g];
-                                SX = s_xs[slot * ng + g];
-                            } else {
-                                const int pos_ = my_half ? s_tile[i].z : s_tile[i].y;
-                                Eg = pos_ >= 0 ? __ldg(a.hexp + pos_ * ng + g) : 0;
-                                SX = pos_ >= 0 ? __ldg(a.hsum + pos_ * ng + g) : 0;
-                            }
+                            Eg = s_xe[slot * ng + g];
+                            SX = s_xs[slot * ng + g];
                             const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                             for (int rr = 0; rr < 2; ++rr) {
@@ -742,14 +782,8 @@ __global__ void __launch_bounds__(kThreads) down_kernel(GemvArgs a) {
                                 if (i < nt && s_tile[i].x > p) {
                                     const int slot = 2 * i + my_half;
                                     int Eg, SX;
-                            if constexpr (NT == 1) {
-                                Eg = s_xe[slot * ng + g];
-                                SX = s_xs[slot * ng + g];
-                            } else {
-                                const int pos_ = my_half ? s_tile[i].z : s_tile[i].y;
-                                Eg = pos_ >= 0 ? __ldg(a.hexp + pos_ * ng + g) : 0;
-                                SX = pos_ >= 0 ? __ldg(a.hsum + pos_ * ng + g) : 0;
-                            }
+                            Eg = s_xe[slot * ng + g];
+                            SX = s_xs[slot * ng + g];
                                     const float sc2 = pow2f(Eg - 22);
 #pragma unroll
                                     for (int rr = 0; rr < 2; ++rr) {
