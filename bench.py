@@ -149,6 +149,16 @@ def build_layer(shape, seed=None):
     return desc, planes, meta, r, wr, sh
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant
+# kernel, from one ncu capture of the current kernel code; the command and the figures are in
+# profiles/ (gateup_down_qwen3_moe_decode_b1.md, gemm_tc_qwen3_moe_prefill_t2048.md). Workloads
+# without such a capture report null.
+NCU_TRAFFIC_BYTES = {
+    ("qwen3_30b_a3b_moe_decode_b1", 2.5): 8_704_512,            # gateup_kernel<0,4,1>
+    ("qwen3_30b_a3b_moe_prefill_t2048", 4.0): 302_900_000,      # gemm_tc_kernel<0,4> (gate/up)
+}
+
+
 def algorithmic_bytes(shape, idx, k):
     """Bytes the gate/up and down GEMVs must read for one step: for every active expert its first
     kmax_e planes of each matrix plus its scale data (kmax_e = max k over its pairs)."""
@@ -535,7 +545,8 @@ def main(argv=None):
         "data": "synthetic",
         "config": config,
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "peak_source": peak_kind},
+                     "frac": achieved / hbm, "traffic": NCU_TRAFFIC_BYTES.get((shape.name, target)),
+                     "traffic_unit": "bytes per launch", "peak_source": peak_kind},
         "dtype_note": "tensor-core path: bf16 x bf16 (gate/up), fp16 x fp16 (down), fp32 accumulate" if res["tc"] else None,
         "planes_gbs_whole_step": all_bytes / secs / 1e9 / world,
         "planes_frac_whole_step": all_bytes / secs / 1e9 / world / hbm,
@@ -556,7 +567,8 @@ def main(argv=None):
         gu_s = stage["gateup"] * 1e-3
         ach = flops / gu_s / 1e12 if gu_s > 0 else 0.0
         line["roofline"] = {"bound": "tensor", "kernel": "gateup", "achieved": ach, "peak": tpeak,
-                            "unit": "TFLOP/s", "frac": ach / tpeak, "traffic": None,
+                            "unit": "TFLOP/s", "frac": ach / tpeak,
+                            "traffic": NCU_TRAFFIC_BYTES.get((shape.name, target)), "traffic_unit": "bytes per launch",
                             "peak_source": "measured sustained bf16" if pk.get("bf16_tflops_sustained") else "fallback"}
         line["dtype"] = "bf16/fp16 tensor-core operands, f32 accumulate (decision path f64)"
         line.pop("dtype_note", None)
