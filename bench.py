@@ -150,9 +150,8 @@ def build_layer(shape, seed=None):
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant
-# kernel, from one ncu capture of the current kernel code; the command and the figures are in
-# profiles/ (gateup_down_qwen3_moe_decode_b1.md, gemm_tc_qwen3_moe_prefill_t2048.md). Workloads
-# without such a capture report null.
+# kernel, from one ncu capture of the current kernel code (the capture commands and figures are
+# kept with the profile summaries). Workloads without such a capture report null.
 NCU_TRAFFIC_BYTES = {
     ("qwen3_30b_a3b_moe_decode_b1", 2.5): 8_704_512,            # gateup_kernel<0,4,1>
     ("qwen3_30b_a3b_moe_prefill_t2048", 4.0): 302_900_000,      # gemm_tc_kernel<0,4> (gate/up)
