@@ -14,14 +14,15 @@ namespace dpa {
 namespace {
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
-    pdl_wait();
     const int t = blockIdx.y;
     const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 4;
-    if (n >= a.H) return;
-    float4 acc = a.shared_out ? *reinterpret_cast<const float4*>(a.shared_out + static_cast<size_t>(t) * a.H + n)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n >= a.H) return;   // nothing to read or write
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-    // slots in chunks of 8: all loads of a chunk are issued before the in-order accumulation
+    // slots in chunks of 8: all loads of a chunk are issued before the in-order accumulation.
+    // The pair positions (allocation) and gates (router) were final before the expert kernels
+    // that precede this launch passed their own waits, so the first chunk's are read (from L2)
+    // before this kernel's dependency wait; the per-pair outputs only after it.
+    bool waited = false;
     for (int s0 = 0; s0 < a.K; s0 += 8) {
         int pos[8];
         float g[8];
@@ -29,9 +30,13 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
             if (s0 + u < a.K) {
-                pos[u] = a.pair_pos[t * a.K + s0 + u];
-                g[u] = static_cast<float>(a.gate[t * a.K + s0 + u]);
+                pos[u] = __ldcg(a.pair_pos + t * a.K + s0 + u);
+                g[u] = static_cast<float>(__ldcg(a.gate + t * a.K + s0 + u));
             }
+        }
+        if (!waited) {
+            pdl_wait();
+            waited = true;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u)
@@ -48,6 +53,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
             }
         }
     }
+    if (!waited) pdl_wait();
+    float4 acc = a.shared_out ? *reinterpret_cast<const float4*>(a.shared_out + static_cast<size_t>(t) * a.H + n)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     acc.x += r.x;
     acc.y += r.y;
     acc.z += r.z;

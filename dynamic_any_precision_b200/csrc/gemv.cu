@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kThreads, NT > 1 ? 2 : 0) gateup_kernel(GemvAr
         }
     }
     pdl_wait();   // work lists and activations come from the previous kernels
+    pdl_trigger();   // the down kernel may become resident and fetch its first planes
     const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
     __syncthreads();
     uint32_t phase = 0, phase_d = 0;
@@ -552,42 +553,48 @@ __global__ void __launch_bounds__(kThreads, NT > 1 ? 2 : 0) down_kernel(GemvArgs
         mbar_init(&s_bard, 1);
         fence_barrier_init();
     }
-    pdl_wait();   // work lists and activations come from the previous kernels
-    const int n_items = static_cast<int>(a.hdr->n_active) * tiles_per_expert;
+    // The work lists come from the allocation, which completed before the gate/up kernel (this
+    // kernel's predecessor) passed its own dependency wait, and the planes are static: the first
+    // item's descriptor is read (from L2) and its plane copies issued before this kernel's wait.
+    const int n_items = static_cast<int>(__ldcg(&a.hdr->n_active)) * tiles_per_expert;
+    int4 desc = __ldcg(a.exp_desc + 2 * (blockIdx.x / tiles_per_expert));
+    int4 tile0 = __ldcg(a.exp_desc + 2 * (blockIdx.x / tiles_per_expert) + 1);
+    auto issue_planes = [&](const int4& d, int rt) {   // thread 0: the item's planes and scales
+        const int e = d.x, kmax_e = d.y;
+        fence_proxy_async();
+        const uint32_t pbytes = 4u * nblk * 128;
+        const uint32_t mbytes = FMT == DPA_FMT_UNIFORM ? 64u * ng * 4 : 64u * ng * 2;
+        const uint32_t total = kmax_e * pbytes + (FMT == DPA_FMT_UNIFORM ? mbytes : kmax_e * mbytes);
+        mbar_arrive_expect_tx(&s_bar, total);
+        const uint64_t plane_stride = static_cast<uint64_t>(H) * I / 8;
+        const uint8_t* base = a.planes + e * a.planes_per_expert + a.planes_mat_off[2];
+        for (int p = 0; p < kmax_e; ++p)
+            bulk_g2s(s_planes + static_cast<size_t>(p) * 4 * nblk * 32,
+                     base + p * plane_stride + static_cast<uint64_t>(rt) * pbytes, pbytes, &s_bar);
+        const uint8_t* mb = a.meta + e * a.meta_per_expert + a.meta_mat_off[2];
+        if (FMT == DPA_FMT_UNIFORM) {
+            bulk_g2s(s_meta, mb + static_cast<uint64_t>(rt) * mbytes, mbytes, &s_bar);
+        } else {
+            const uint64_t mplane = static_cast<uint64_t>(H) * ng * 2;
+            for (int p = 0; p < kmax_e; ++p)
+                bulk_g2s(s_meta + p * mbytes, mb + p * mplane + static_cast<uint64_t>(rt) * mbytes, mbytes, &s_bar);
+        }
+    };
+    if (threadIdx.x == 0 && static_cast<int>(blockIdx.x) < n_items) issue_planes(desc, blockIdx.x % tiles_per_expert);
+    pdl_wait();   // h and its digits come from the previous kernel
     __syncthreads();
     uint32_t phase = 0, phase_d = 0;
     const int dig = gid & 3, half = gid >> 2, my_half = tq >> 1;
     const int dstride = Ly.dig_stride;
 
-    int4 desc = a.exp_desc[2 * (blockIdx.x / tiles_per_expert)];
-    int4 tile0 = a.exp_desc[2 * (blockIdx.x / tiles_per_expert) + 1];
     for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
         if (item != blockIdx.x) {
             desc = a.exp_desc[2 * (item / tiles_per_expert)];
             tile0 = a.exp_desc[2 * (item / tiles_per_expert) + 1];
         }
-        const int e = desc.x, kmax_e = desc.y, ntiles = desc.z, toff = desc.w;
+        const int kmax_e = desc.y, ntiles = desc.z, toff = desc.w;
         const int rt = item % tiles_per_expert;
-        if (threadIdx.x == 0) {
-            fence_proxy_async();
-            const uint32_t pbytes = 4u * nblk * 128;
-            const uint32_t mbytes = FMT == DPA_FMT_UNIFORM ? 64u * ng * 4 : 64u * ng * 2;
-            const uint32_t total = kmax_e * pbytes + (FMT == DPA_FMT_UNIFORM ? mbytes : kmax_e * mbytes);
-            mbar_arrive_expect_tx(&s_bar, total);
-            const uint64_t plane_stride = static_cast<uint64_t>(H) * I / 8;
-            const uint8_t* base = a.planes + e * a.planes_per_expert + a.planes_mat_off[2];
-            for (int p = 0; p < kmax_e; ++p)
-                bulk_g2s(s_planes + static_cast<size_t>(p) * 4 * nblk * 32,
-                         base + p * plane_stride + static_cast<uint64_t>(rt) * pbytes, pbytes, &s_bar);
-            const uint8_t* mb = a.meta + e * a.meta_per_expert + a.meta_mat_off[2];
-            if (FMT == DPA_FMT_UNIFORM) {
-                bulk_g2s(s_meta, mb + static_cast<uint64_t>(rt) * mbytes, mbytes, &s_bar);
-            } else {
-                const uint64_t mplane = static_cast<uint64_t>(H) * ng * 2;
-                for (int p = 0; p < kmax_e; ++p)
-                    bulk_g2s(s_meta + p * mbytes, mb + p * mplane + static_cast<uint64_t>(rt) * mbytes, mbytes, &s_bar);
-            }
-        }
+        if (threadIdx.x == 0 && item != static_cast<int>(blockIdx.x)) issue_planes(desc, rt);
         bool waited = false;
         for (int pass0 = 0; pass0 < ntiles; pass0 += NT) {
             if (NT == 1) {
