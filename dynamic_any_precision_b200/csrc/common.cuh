@@ -140,10 +140,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 // work before wait (descriptor and weight prefetch) then overlap the predecessor. wait blocks
 // until the predecessor has completed and its memory is visible; every kernel calls it before
 // its first read of a predecessor's output and before its first global write. Outside such a
-// launch both are no-ops. Only the single-CTA allocation triggers early (after its own wait):
-// the expert kernel's CTAs then sit resident and waiting while the bisection runs. (Triggering
-// in every kernel was measured slower at batch 1, 42.9 vs 41.1 us per step: early-resident
-// successor CTAs take SM slots from a wide predecessor.)
+// launch both are no-ops. The single-CTA allocation and the gate/up kernel trigger early
+// (after their own waits): the next kernel's CTAs then become resident and read what is
+// already final (work lists, static weights) while the predecessor runs. (Triggering in every
+// kernel was measured slower at batch 1, 42.9 vs 41.1 us per step: early-resident successor
+// CTAs take SM slots from a wide predecessor.)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
