@@ -158,6 +158,22 @@ NCU_TRAFFIC_BYTES = {
 }
 
 
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of per-rank device times (ms) over all ranks (every rank gets it);
+    the values unchanged when there is one process."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    tt = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return [float(v) for v in tt.tolist()]
+
+
+def replica_token_seed(rank: int, step: int) -> int:
+    """Seed of the synthetic tokens of one step on one rank: distinct per rank and step."""
+    return 1_000_000 * rank + step
+
+
 def algorithmic_bytes(shape, idx, k):
     """Bytes the gate/up and down GEMVs must read for one step: for every active expert its first
     kmax_e planes of each matrix plus its scale data (kmax_e = max k over its pairs)."""
@@ -192,7 +208,7 @@ def run_dpa(args, shape, target, rank, world, dist):
                                       base.w_router.clone(), base.shared))
     n_total = args.warmup + args.steps
     # distinct tokens per step (and per rank)
-    xs = np.stack([W.tokens(shape, T, step=1_000_000 * rank + i) for i in range(n_total)])
+    xs = np.stack([W.tokens(shape, T, step=replica_token_seed(rank, i)) for i in range(n_total)])
     x_dev = torch.from_numpy(xs.view(np.int16)).to(dev)
     y_dev = torch.empty((n_total, T, shape.hidden), dtype=torch.int16, device=dev)
     tg = torch.tensor([target], dtype=torch.float64, device=dev)
@@ -252,10 +268,7 @@ def run_dpa(args, shape, target, rank, world, dist):
     st = dpa.device_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {dpa.STATUS_NAMES.get(st, st)}")
-    if dist is not None:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(dist, [ms], dev)[0]
 
     # per-stage kernel times: the same steps replayed once more with stage events
     g_stages.replay()
@@ -296,10 +309,7 @@ def run_dpa(args, shape, target, rank, world, dist):
         e1.record()
         torch.cuda.synchronize()
         e_ms = e0.elapsed_time(e1)
-        if dist is not None:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(dist, [e_ms], dev)[0]
         e2e = {"value": world * T * n_e / (e_ms * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(x_buf.numel() * 2), "d2h_bytes_per_step": int(y_buf.numel() * 2),
                "steps": n_e}
@@ -383,10 +393,7 @@ def run_stack(args, shape, rank, world, dist):
         dist.barrier()
     ms = t0.elapsed_time(t1)
     assert dpa.device_status(bufs["ws"]) == 0
-    if dist is not None:
-        tt = torch.tensor([ms, prefill_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, prefill_ms = float(tt[0].item()), float(tt[1].item())
+    ms, prefill_ms = max_over_ranks(dist, [ms, prefill_ms], dev)
     del graphs
     n_layers = stack.n_layers
     return {"ms": ms, "prefill_ms": prefill_ms, "clocks": clk.summary(), "n_layers": n_layers,
