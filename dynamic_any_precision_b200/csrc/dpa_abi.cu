@@ -11,8 +11,6 @@
 
 namespace {
 
-constexpr size_t kMaxDynSmem = 200 * 1024;
-
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 dpa_status check_desc(const dpa_layer_desc* d) {
@@ -34,7 +32,8 @@ dpa_status check_desc(const dpa_layer_desc* d) {
     ga.B = d->bits;
     ga.G = d->group;
     ga.fmt = d->format;
-    if (dpa::gateup_smem_bytes(ga) > kMaxDynSmem || dpa::down_smem_bytes(ga) > kMaxDynSmem) return DPA_ERR_UNSUPPORTED;
+    if (dpa::gateup_smem_bytes(ga) > dpa::kGemvMaxSmem || dpa::down_smem_bytes(ga) > dpa::kGemvMaxSmem)
+        return DPA_ERR_UNSUPPORTED;
     return DPA_OK;
 }
 

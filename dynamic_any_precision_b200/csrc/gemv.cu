@@ -907,7 +907,14 @@ void* pick_down(int B) {
     }
 }
 
-int pick_nt(const GemvArgs& a) { return a.max_tokens_per_expert <= 2 ? 1 : 4; }
+// tiles per pass: 4 when experts may hold more than two tokens and the multi-token staging of
+// both kernels fits in shared memory, else 1
+int pick_nt(const GemvArgs& a) {
+    if (a.max_tokens_per_expert <= 2) return 1;
+    const bool fits = gateup_layout(a.H, a.G, a.B, a.fmt, 4).total <= kGemvMaxSmem &&
+                      down_layout(a.I, a.G, a.B, a.fmt, 4).total <= kGemvMaxSmem;
+    return fits ? 4 : 1;
+}
 
 cudaError_t launch_generic(void* fn, size_t smem, int items, int num_sms, const GemvArgs& a, cudaStream_t stream) {
     if (items <= 0) return cudaSuccess;
@@ -925,14 +932,8 @@ cudaError_t launch_generic(void* fn, size_t smem, int items, int num_sms, const 
 
 }  // namespace
 
-size_t gateup_smem_bytes(const GemvArgs& a) {
-    const size_t s1 = gateup_layout(a.H, a.G, a.B, a.fmt, 1).total, s4 = gateup_layout(a.H, a.G, a.B, a.fmt, 4).total;
-    return s1 > s4 ? s1 : s4;
-}
-size_t down_smem_bytes(const GemvArgs& a) {
-    const size_t s1 = down_layout(a.I, a.G, a.B, a.fmt, 1).total, s4 = down_layout(a.I, a.G, a.B, a.fmt, 4).total;
-    return s1 > s4 ? s1 : s4;
-}
+size_t gateup_smem_bytes(const GemvArgs& a) { return gateup_layout(a.H, a.G, a.B, a.fmt, 1).total; }
+size_t down_smem_bytes(const GemvArgs& a) { return down_layout(a.I, a.G, a.B, a.fmt, 1).total; }
 
 cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms) {
     const int nt = pick_nt(a);

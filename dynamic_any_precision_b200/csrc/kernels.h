@@ -105,8 +105,12 @@ struct GemvArgs {
     int max_tokens_per_expert;  // host-known bound (selects the tile count per pass)
 };
 cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms);
-size_t gateup_smem_bytes(const GemvArgs& a);   // dynamic shared memory of one CTA
-size_t down_smem_bytes(const GemvArgs& a);
+// Dynamic shared memory a GEMV work item may stage. The single-pass (one- and two-token)
+// kernels must fit for a layer to be accepted; the multi-token kernels run only where they fit
+// too, the single-pass ones (one tile per pass) elsewhere.
+constexpr size_t kGemvMaxSmem = 200 * 1024;
+size_t gateup_smem_bytes(const GemvArgs& a);   // one CTA of the single-pass gate/up kernel
+size_t down_smem_bytes(const GemvArgs& a);     // one CTA of the single-pass down kernel
 cudaError_t launch_down(const GemvArgs& a, cudaStream_t stream, int num_sms);
 
 struct CombineArgs {
