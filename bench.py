@@ -153,7 +153,6 @@ def build_layer(shape, seed=None):
 # kernel, from one ncu capture of the current kernel code (the capture commands and figures are
 # kept with the profile summaries). Workloads without such a capture report null.
 NCU_TRAFFIC_BYTES = {
-    ("qwen3_30b_a3b_moe_decode_b1", 2.5): 8_704_512,            # gateup_kernel<0,4,1>
     ("qwen3_30b_a3b_moe_prefill_t2048", 4.0): 302_900_000,      # gemm_tc_kernel<0,4> (gate/up)
 }
 
