@@ -1,9 +1,9 @@
 // Post-routing plane allocation and token->expert grouping.
 //
-// DPA-MoE, Abstract: chunks are allocated at inference time from the live router gate
-// scores. DuoRate, Abstract: a Lagrangian rate-distortion allocation solved by a bisection.
-// MatMoE, review "Core Contribution": a binary search sets the precision split so that the
-// average bit-width meets a target.
+// DPA-MoE, Abstract: how many chunks a routed pair reads is decided after routing, from the
+// gate scores of the current call. DuoRate, Abstract: per-expert rates trade rate against
+// distortion through a Lagrange multiplier, found by bisection. MatMoE, review "Core
+// Contribution": a binary search picks the mix of precisions that meets a mean bit-width.
 //
 // For a multiplier lambda each routed pair p (expert e, gate g) reads
 //     k_p(lambda) = argmin_{kmin<=k<=kmax} fl(fl(g * r_e(k)) + fl(lambda * k))

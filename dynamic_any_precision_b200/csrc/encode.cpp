@@ -1,12 +1,13 @@
 // Offline encoder of routed expert weights into prefix-decodable bitplanes (host C++).
 //
-// DPA-MoE: A Runtime Precision Control Framework for MoE Inference, Abstract: expert FFN
-// weights become prefix-decodable chunks under one shared scale ("SharedScale AnyBCQ"), and
-// per-expert reconstruction residuals are profiled offline.
-// MatMoE (review, "Core Contribution"): bitplane storage; one set of quantisation parameters
-// serves the low-bit prefix and the full precision.
-// DuoRate, Abstract: one stored tier of a prefix-readable weight stream plus a baked
-// distortion tensor.
+// DPA-MoE: A Runtime Precision Control Framework for MoE Inference, Abstract: each expert's
+// FFN weights are encoded so that every leading run of chunks decodes on its own, all runs
+// sharing one scale (the page names the format SharedScale AnyBCQ), and each expert's
+// reconstruction error is measured ahead of time.
+// MatMoE (review, "Core Contribution"): weights are kept as bitplanes, and the low-bit prefix
+// and the full code use the same quantisation parameters.
+// DuoRate, Abstract: a single stored copy whose prefix can be read at any rate, plus a
+// precomputed table of distortions.
 //
 // Build with -ffp-contract=off and without fast-math: every fp64 operation below is one IEEE
 // round-to-nearest operation, so the codes, scales and residual sums are reproducible.

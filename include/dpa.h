@@ -4,13 +4,14 @@
  *
  * The method (pages cited by title and section):
  *  - DPA-MoE: A Runtime Precision Control Framework for MoE Inference, Abstract:
- *    expert FFN weights stored as prefix-decodable chunks with one shared scale
- *    ("SharedScale AnyBCQ"), per-expert reconstruction residuals profiled offline,
- *    chunks allocated after routing from the live router gate scores, so one encoded
- *    layer runs at many weight budgets.
+ *    expert weights in chunks that decode by prefix under one shared scale (the page's
+ *    SharedScale AnyBCQ); each expert's reconstruction error measured ahead of time; the
+ *    chunk count of each routed pair chosen after routing from the current gate scores,
+ *    so one encoded layer serves many weight budgets.
  *  - DuoRate: Two-Rate Per-Expert Precision Allocation for MoE Serving, Abstract:
- *    prefix-readable weight stream, baked distortion tensor, Lagrangian
- *    rate-distortion allocation solved by a bisection; prefill reads at the stored rate.
+ *    one stored copy read by prefix, a precomputed distortion table, per-expert rates
+ *    from a Lagrangian rate/distortion trade-off found by bisection; prefill reads every
+ *    stored plane.
  *  - MatMoE: Matryoshka Mixture-of-Experts with Dynamic Mixed-Precision Quantization,
  *    Abstract and review section "Core Contribution": bitplane storage,
  *    floor-and-compensation (keep the top k of B code bits and add (2^(B-k)-1)/2),

@@ -66,8 +66,8 @@ def bf16_bits_to_f64(bits) -> np.ndarray:
 
 # ---------------------------------------------------------------------------
 # Uniform asymmetric group quantisation with one scale/zero shared by every k
-# [DPA] "SharedScale"; [MAT] Core Contribution: shared quantization parameters
-# for the 2-bit prefix and the higher precision.
+# [DPA] (one scale shared by every prefix); [MAT] Core Contribution: the low-bit prefix and
+# the full code use the same quantisation parameters.
 # Reading: plain round-to-nearest (the trained-parameter variant needs data).
 # ---------------------------------------------------------------------------
 
