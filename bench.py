@@ -48,13 +48,25 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=1024)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", choices=("dpa", "reference"), default="dpa")
-    ap.add_argument("--workload", default=W.QWEN3_B1.name)
+    ap.add_argument("--workload", default=W.QWEN3_B64.name)
     ap.add_argument("--target", type=float, default=None)
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="time only the headline budget (the batch-64 workload sweeps all its budgets)")
     ap.add_argument("--copies", type=int, default=16)
     ap.add_argument("--e2e-steps", type=int, default=256)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-sample-tokens", type=int, default=24)
+    ap.add_argument("--cpu-sample-pairs", type=int, default=24,
+                    help="expert FFN pairs the CPU-baseline sample times (round robin over the steps)")
     return ap.parse_args(argv)
+
+
+# The headline budget of each workload: the batch-64 layer is quoted at 3.0 bpw, the middle of
+# its sweep; the others at their first (or only) budget.
+HEADLINE_TARGET = {W.QWEN3_B64.name: 3.0}
+
+
+def headline_target(shape):
+    return HEADLINE_TARGET.get(shape.name, shape.targets[0])
 
 
 def peaks():
@@ -192,7 +204,9 @@ def algorithmic_bytes(shape, idx, k):
     return gu, dn, len(kmax)
 
 
-def run_dpa(args, shape, target, rank, world, dist):
+def run_dpa(args, shape, targets, rank, world, dist):
+    """Times K graph-replayed steps at each budget in `targets` (the budget is a device scalar, so
+    one captured graph serves them all). Returns one result dict per budget."""
     import torch
     from dynamic_any_precision_b200 import dpa
 
@@ -210,7 +224,7 @@ def run_dpa(args, shape, target, rank, world, dist):
     xs = np.stack([W.tokens(shape, T, step=replica_token_seed(rank, i)) for i in range(n_total)])
     x_dev = torch.from_numpy(xs.view(np.int16)).to(dev)
     y_dev = torch.empty((n_total, T, shape.hidden), dtype=torch.int16, device=dev)
-    tg = torch.tensor([target], dtype=torch.float64, device=dev)
+    tg = torch.tensor([targets[0]], dtype=torch.float64, device=dev)
     ws = dpa.new_workspace(desc, T, device=dev)
     idx_all = torch.empty((args.steps, T, K), dtype=torch.int32, device=dev)
     gate_all = torch.empty((args.steps, T, K), dtype=torch.float64, device=dev)
@@ -249,47 +263,59 @@ def run_dpa(args, shape, target, rank, world, dist):
             for j in range(args.steps):
                 step(args.warmup + j, timed_j=j)
     torch.cuda.synchronize()
-    g_warm.replay()
-    torch.cuda.synchronize()
 
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t0.record()
-        g_timed.replay()
-        t1.record()
-        torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    ms = t0.elapsed_time(t1)
-    st = dpa.device_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {dpa.STATUS_NAMES.get(st, st)}")
-    ms = max_over_ranks(dist, [ms], dev)[0]
-
-    # per-stage kernel times: the same steps replayed once more with stage events
-    g_stages.replay()
-    torch.cuda.synchronize()
-    assert dpa.device_status(ws) == 0
     names = ["route", "allocate", "shared", "gateup", "down", "combine"]
-    stage_ms = {n: 0.0 for n in names}
-    for j in range(args.steps):
-        ev = events[j]
-        for q, n in enumerate(names):
-            stage_ms[n] += ev[q].elapsed_time(ev[q + 1])
-    idx_h, k_h = idx_all.cpu().numpy(), k_all.cpu().numpy()
-    gu_bytes = dn_bytes = 0
-    n_active = 0
-    for j in range(args.steps):
-        a, b, c = algorithmic_bytes(shape, idx_h[j], k_h[j])
-        gu_bytes += a
-        dn_bytes += b
-        n_active += c
-    mean_bpw = float(k_h.astype(np.float64).mean())
+    results = []
+    for target in targets:
+        tg.fill_(target)
+        # untimed: the warm-up steps, then one whole replay of the timed graph itself (its upload
+        # and first launch stay outside the measurement)
+        g_warm.replay()
+        g_timed.replay()
+        torch.cuda.synchronize()
+        assert dpa.device_status(ws) == 0
 
-    # e2e through the public API with host buffers (pinned), copies inside the timed region
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            t0.record()
+            g_timed.replay()
+            t1.record()
+            torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        ms = t0.elapsed_time(t1)
+        st = dpa.device_status(ws)
+        if st != 0:
+            raise RuntimeError(f"device status {dpa.STATUS_NAMES.get(st, st)}")
+        ms = max_over_ranks(dist, [ms], dev)[0]
+
+        # per-stage kernel times: the same steps replayed once more with stage events
+        g_stages.replay()
+        torch.cuda.synchronize()
+        assert dpa.device_status(ws) == 0
+        stage_ms = {n: 0.0 for n in names}
+        for j in range(args.steps):
+            ev = events[j]
+            for q, n in enumerate(names):
+                stage_ms[n] += ev[q].elapsed_time(ev[q + 1])
+        idx_h, k_h = idx_all.cpu().numpy(), k_all.cpu().numpy()
+        gu_bytes = dn_bytes = 0
+        n_active = 0
+        for j in range(args.steps):
+            a, b, c = algorithmic_bytes(shape, idx_h[j], k_h[j])
+            gu_bytes += a
+            dn_bytes += b
+            n_active += c
+        mean_bpw = float(k_h.astype(np.float64).mean())
+        results.append({"target": target, "ms": ms, "stage_ms": stage_ms, "gu_bytes": gu_bytes, "dn_bytes": dn_bytes,
+                        "n_active": n_active, "mean_bpw": mean_bpw, "clocks": clk.summary()})
+
+    # e2e through the public API with host buffers (pinned), copies inside the timed region, at the
+    # first (headline) budget
+    tg.fill_(targets[0])
     e2e = None
     if args.e2e_steps > 0:
         n_e = min(args.e2e_steps, n_total)
@@ -317,9 +343,10 @@ def run_dpa(args, shape, target, rank, world, dist):
     tc = (shape.fmt == dpa.FMT_UNIFORM and shape.hidden % 256 == 0 and shape.inter % 256 == 0 and
           P >= 16 * shape.n_experts)
     launches_per_step = ((3 if T >= 128 else 1) + (2 if P > 2048 else 1) + (3 if tc else 2) + 1 +
-                         (2 if shape.n_shared else 0))
-    return {"tc": tc, "ms": ms, "stage_ms": stage_ms, "gu_bytes": gu_bytes, "dn_bytes": dn_bytes, "n_active": n_active,
-            "mean_bpw": mean_bpw, "clocks": clk.summary(), "e2e": e2e, "launches": launches_per_step * args.steps}
+                         (2 if shape.n_shared else 0) + (1 if (not tc and T > 2) else 0))
+    for res in results:
+        res.update({"tc": tc, "e2e": e2e, "launches": launches_per_step * args.steps})
+    return results
 
 
 def run_stack(args, shape, rank, world, dist):
@@ -416,39 +443,64 @@ def _encode_pool(shape, experts):
         return dict(ex.map(_oracle_encode_job, [shape] * len(experts), experts))
 
 
-def oracle_sample(shape, target, n_tokens, seed_base=0):
-    """Times the fp64 oracle (as it stands) on `n_tokens` single-token steps of the workload.
-    Each step routes and allocates the token in full; of its top_k expert FFNs one (round
-    robin over the slots) is run and its time counted top_k times. Encoding the routed
-    experts is offline work (as in the product) and is not timed."""
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(shape, target, n_steps, n_pairs, seed_base=0):
+    """Times the fp64 oracle (as it stands, one thread) on a bounded sample of the workload.
+    Each sampled step routes and allocates its whole batch; `n_pairs` expert FFNs (dequantise at
+    the pair's k, SwiGLU, down) are timed round robin over the steps' routed pairs, and their mean
+    time counts once per routed pair of a step. Encoding the routed experts (offline work in the
+    method too) runs beforehand in a spawned process pool and is not timed."""
     from threadpoolctl import threadpool_limits
     from oracle import dpa_oracle as O
+    T, K = shape.tokens, shape.top_k
     wr = W.router_weights(shape)
-    xs = [W.tokens(shape, shape.tokens, step=seed_base + i) for i in range(n_tokens)]
-    routes = [O.route(x, wr, shape.top_k, shape.norm_topk) for x in xs]
+    xs = [W.tokens(shape, T, step=seed_base + i) for i in range(n_steps)]
+    routes = [O.route(x, wr, K, shape.norm_topk) for x in xs]
     need = sorted({int(e) for rt in routes for e in np.unique(rt[0])})
     experts = _encode_pool(shape, need)          # offline setup, not timed
+    ffn_s = []
+    ra_s = []
     with threadpool_limits(1):
         r = np.full((shape.n_experts, shape.bits), np.nan)
         for e, enc in experts.items():
             r[e] = enc["r"]
-        total = 0.0
+        per_step = max(1, -(-n_pairs // n_steps))
         for i, x in enumerate(xs):
             t0 = time.perf_counter()
-            idx, g, _ = O.route(x, wr, shape.top_k, shape.norm_topk)
+            idx, g, _ = O.route(x, wr, K, shape.norm_topk)
             k, lam = O.allocate(idx, g, r, shape.kmin, shape.kmax, target)
-            t1 = time.perf_counter()
-            j = i % shape.top_k
-            xf = O.bf16_bits_to_f64(x)[0]
-            e, kk = int(idx[0, j]), int(k[0, j])
-            wg, wu, wd = O.dequant_expert(experts[e], shape.fmt, shape.bits, kk, shape.group)
-            O.expert_ffn(xf, wg, wu, wd)
-            t2 = time.perf_counter()
-            total += (t1 - t0) + shape.top_k * (t2 - t1)
-    return {"value": shape.tokens * n_tokens / total, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n_tokens} single-token steps: route + allocate in full, 1 of {shape.top_k} expert "
-                      f"FFNs per step timed and counted x{shape.top_k}; fp64 numpy, 1 thread",
-            "seconds": total}
+            ra_s.append(time.perf_counter() - t0)
+            xf = O.bf16_bits_to_f64(x)
+            for q in range(per_step):
+                p = (i * per_step + q) % (T * K)
+                t, j = divmod(p, K)
+                t1 = time.perf_counter()
+                e, kk = int(idx[t, j]), int(k[t, j])
+                wg, wu, wd = O.dequant_expert(experts[e], shape.fmt, shape.bits, kk, shape.group)
+                O.expert_ffn(xf[t], wg, wu, wd)
+                ffn_s.append(time.perf_counter() - t1)
+    step_s = statistics.mean(ra_s) + T * K * statistics.mean(ffn_s)
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except AttributeError:
+        affinity = os.cpu_count()
+    return {"value": T / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_steps} steps of {T} token(s): route + allocate of the whole batch timed per step; "
+                      f"{len(ffn_s)} of the steps' {T * K}-pair expert FFNs timed, their mean counted once per "
+                      f"routed pair; fp64 numpy, 1 thread",
+            "affinity_cores": affinity, "cpu_model": _cpu_model(), "ms_per_step": 1e3 * step_s,
+            "seconds": sum(ra_s) + sum(ffn_s)}
 
 
 # ----------------------------------------------------------------------------- main
@@ -456,7 +508,7 @@ def oracle_sample(shape, target, n_tokens, seed_base=0):
 def main(argv=None):
     args = parse_args(argv)
     shape = W.shape_by_name(args.workload)
-    target = args.target if args.target is not None else shape.targets[0]
+    target = args.target if args.target is not None else headline_target(shape)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -471,12 +523,15 @@ def main(argv=None):
         if rank != 0:
             return 0
         steps = args.steps
-        smp = oracle_sample(shape, target, args.warmup + steps)
+        # a bounded sample: at most 8 steps and 4 expert FFNs per step, whatever K and W are
+        n_steps = max(1, min(8, args.warmup + steps))
+        smp = oracle_sample(shape, target, n_steps, 4 * n_steps)
         line = {"impl": "reference", "metric": metric, "value": smp["value"], "unit": "tokens/s", "n_gpus": args.gpus,
-                "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * shape.tokens / smp["value"],
+                "steps": steps, "warmup": args.warmup, "ms_per_step": smp["ms_per_step"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": config,
-                "cpu_baseline": {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "cpu_baseline": {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample", "affinity_cores",
+                                                     "cpu_model")},
                 "e2e": {"value": smp["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return 0
@@ -525,16 +580,36 @@ def main(argv=None):
             dist.destroy_process_group()
         return 0
 
-    res = run_dpa(args, shape, target, rank, world, dist)
+    targets = [target]
+    if args.target is None and not args.no_sweep and len(shape.targets) > 1:
+        targets += [t for t in shape.targets if t != target]
+    results = run_dpa(args, shape, targets, rank, world, dist)
     hbm, peak_kind = peaks()
-    secs = res["ms"] * 1e-3
     tokens = world * shape.tokens * args.steps
+
+    def summarise(res):
+        stage = res["stage_ms"]
+        dominant = max(("gateup", "down"), key=lambda n: stage[n])
+        dom_bytes = res["gu_bytes"] if dominant == "gateup" else res["dn_bytes"]
+        dom_s = stage[dominant] * 1e-3
+        achieved = dom_bytes / dom_s / 1e9 if dom_s > 0 else 0.0
+        all_bytes = res["gu_bytes"] + res["dn_bytes"]
+        secs = res["ms"] * 1e-3
+        gu_s, dn_s = stage["gateup"] * 1e-3, stage["down"] * 1e-3
+        return dominant, achieved, all_bytes, secs, {
+            "target_bpw": res["target"], "value": tokens / secs, "ms_per_step": res["ms"] / args.steps,
+            "mean_planes_per_pair": res["mean_bpw"], "bytes_per_step": all_bytes / args.steps,
+            "active_experts_per_step": res["n_active"] / args.steps,
+            "gateup_gbs": res["gu_bytes"] / gu_s / 1e9 if gu_s > 0 else None,
+            "gateup_frac": res["gu_bytes"] / gu_s / 1e9 / hbm if gu_s > 0 else None,
+            "down_gbs": res["dn_bytes"] / dn_s / 1e9 if dn_s > 0 else None,
+            "down_frac": res["dn_bytes"] / dn_s / 1e9 / hbm if dn_s > 0 else None,
+            "planes_frac_whole_step": all_bytes / secs / 1e9 / world / hbm,
+            "clocks": res["clocks"]}
+
+    res = results[0]
+    dominant, achieved, all_bytes, secs, head = summarise(res)
     stage = res["stage_ms"]
-    dominant = max(("gateup", "down"), key=lambda n: stage[n])
-    dom_bytes = res["gu_bytes"] if dominant == "gateup" else res["dn_bytes"]
-    dom_s = stage[dominant] * 1e-3
-    achieved = dom_bytes / dom_s / 1e9 if dom_s > 0 else 0.0
-    all_bytes = res["gu_bytes"] + res["dn_bytes"]
     line = {
         "metric": metric,
         "value": tokens / secs,
@@ -552,7 +627,6 @@ def main(argv=None):
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": NCU_TRAFFIC_BYTES.get((shape.name, target)),
                      "traffic_unit": "bytes per launch", "peak_source": peak_kind},
-        "dtype_note": "tensor-core path: bf16 x bf16 (gate/up), fp16 x fp16 (down), fp32 accumulate" if res["tc"] else None,
         "planes_gbs_whole_step": all_bytes / secs / 1e9 / world,
         "planes_frac_whole_step": all_bytes / secs / 1e9 / world / hbm,
         "bytes_per_step": all_bytes / args.steps,
@@ -563,6 +637,8 @@ def main(argv=None):
         "e2e": res["e2e"],
         "gpu_launches": res["launches"],
     }
+    if len(results) > 1:
+        line["sweep"] = [summarise(r_)[4] for r_ in results]
     if res["tc"]:
         # prefill-sized batches run the expert FFN as tcgen05 GEMMs: tensor-bound. The gate/up stage
         # (row permutation + GEMM) is timed against the sustained bf16 peak (it runs inside a step).
@@ -576,12 +652,10 @@ def main(argv=None):
                             "traffic": NCU_TRAFFIC_BYTES.get((shape.name, target)), "traffic_unit": "bytes per launch",
                             "peak_source": "measured sustained bf16" if pk.get("bf16_tflops_sustained") else "fallback"}
         line["dtype"] = "bf16/fp16 tensor-core operands, f32 accumulate (decision path f64)"
-        line.pop("dtype_note", None)
-    else:
-        line.pop("dtype_note", None)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = oracle_sample(shape, target, args.cpu_sample_tokens, seed_base=50000)
-        line["cpu_baseline"] = {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        smp = oracle_sample(shape, target, 4, args.cpu_sample_pairs, seed_base=50000)
+        line["cpu_baseline"] = {k: smp[k] for k in ("value", "unit", "cores", "kind", "sample", "affinity_cores",
+                                                    "cpu_model")}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

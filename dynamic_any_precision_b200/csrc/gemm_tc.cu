@@ -19,16 +19,17 @@
 // same 64 up rows, interleaved by 16 inside each 32-lane quadrant, so that SwiGLU pairs lane t
 // with lane t ^ 16 of the same warp.
 //
-// Roles (448 threads, one CTA per SM, persistent over the work items (token tile, row block)):
+// Roles (576 threads, one CTA per SM, persistent over the work items (token tile, row block)):
 //   warps 0-3   drain: tcgen05.ld each finished group's accumulator and the running sum,
-//               run += s[n, g] * acc, tcgen05.st the running sum (TMEM columns 256..383);
+//               run += s[n, g] * acc, tcgen05.st the running sum (TMEM columns 384..511);
 //               epilogue per item (SwiGLU -> fp16 h, or fp32 per-pair outputs)
-//   warps 4-11  decoders: plane words of a stage -> swizzled K-major A tile; fence; arrive
-//   warp 12     loader: TMA tensor loads, no multicast. Plane words: per (plane, matrix) one box
+//   warps 4-15  decoders, three groups of four warps; group q fills A slot q (K stages
+//               c = q mod 3): plane words of a stage -> swizzled K-major A tile; fence; arrive
+//   warp 16     loader: TMA tensor loads, no multicast. Plane words: per (plane, matrix) one box
 //               of 4 (gate/up) or 8 (down) row tiles x 4 stages of columns (a "plane stage"
 //               holds 4 K stages). Activations: one 2D box of 128 rows x 64 columns per K stage
 //               from the pair-ordered rows (x gathered by permute_rows_kernel, or h)
-//   warp 13     TMEM allocation and the single MMA-issuing thread
+//   warp 17     TMEM allocation and the single MMA-issuing thread
 // Every wait is bounded (globaltimer); on a timeout the kernel records DPA_ERR_DEVICE_TIMEOUT,
 // every role leaves its loop, in-flight copies and MMAs are awaited, and TMEM is released.
 #include <cuda.h>

@@ -176,7 +176,11 @@ dpa_status dpa_export_codes(const dpa_layer_desc* desc, const void* planes, int 
 dpa_status dpa_export_meta(const dpa_layer_desc* desc, const void* meta, int expert,
                            int matrix, float* s_or_alpha, float* zero);
 
-/* Router (device): logits l[t][e] = the exact dot product of bf16 x[t] and bf16
+/* Router (device). Defined by: DPA-MoE: A Runtime Precision Control Framework for MoE
+ * Inference, Abstract (each token is sent to a small set of experts by the router, and
+ * the live gate scores then drive the allocation); the softmax/top-k gating form is the
+ * plainest reading, the pages print no formula for it.
+ * Logits l[t][e] = the exact dot product of bf16 x[t] and bf16
  * w_router[e], rounded once to fp64; top_k experts by descending logit (ties to the lower
  * id); gates as described at dpa_layer_desc.norm_topk, using a fixed fp64 exp (Cody-Waite
  * reduction with ln 2 in two parts, degree-13 Taylor polynomial, results below 2^-1021
@@ -226,7 +230,14 @@ dpa_status dpa_route_noalloc(const dpa_layer_desc* desc, const void* x, int n_to
  * max_tokens tokens. Returns 0 for an invalid descriptor. */
 size_t dpa_forward_workspace_size(const dpa_layer_desc* desc, int max_tokens);
 
-/* One MoE layer forward (device): route, allocate, group pairs by expert and plane
+/* One MoE layer forward (device). Defined by: DPA-MoE: A Runtime Precision Control
+ * Framework for MoE Inference, Abstract (post-routing allocation of prefix-decodable
+ * chunks from live gate scores, one encoded layer at many budgets); MatMoE: Matryoshka
+ * Mixture-of-Experts with Dynamic Mixed-Precision Quantization, review section "Core
+ * Contribution" (bitplane storage read by prefix, floor-and-compensation); DuoRate:
+ * Two-Rate Per-Expert Precision Allocation for MoE Serving, Abstract (the Lagrangian
+ * bisection; a decode step pays only for the planes of the experts it selects).
+ * Steps: route, allocate, group pairs by expert and plane
  * count, run each routed pair's SwiGLU expert reading only its first k planes
  *   a = W_gate^(k) x, u = W_up^(k) x, h = silu(a) * u, o = W_down^(k) h,
  * and write y[t] = bf16( sum_{slots} g * o  (+ dense shared experts) ).

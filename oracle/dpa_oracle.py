@@ -27,15 +27,19 @@ Parity status of each function (what pins it; see tests/test_oracle_pins.py):
                       bit-pattern identity); planted no-compensation control fails
   encode (r table)    pinned: exact rational sum on small inputs; monotone in k;
                       ~4x per plane for uniform codes (closed-form approximation)
-  encode_bcq_matrix   pinned: optimal alpha for fixed signs; equal-magnitude closed form;
-                      residual non-increasing
+  encode_bcq_matrix   pinned: hand-worked group with exact signs, alphas, w_hat(k) and
+  / dequant_bcq       residuals (tests/golden/bcq_worked_group.json); exact-rational greedy fit
+                      and residual table on random experts; equal-magnitude closed form;
+                      planted sign and plane-index mistakes fail the pin
   dexp                pinned: within 1 ulp of a correctly rounded exp (decimal module)
   route               pinned: logit = exact rational dot product rounded once; brute-force
                       top-k; expert permutation equivariance; softmax identities
   allocate            pinned: brute-force constrained optimum (Everett) on tiny inputs,
                       budget criterion, endpoint targets, monotone N along the bisection
   expert_ffn / moe    pinned: hand-worked tiny layer; top-1 identity; linearity of the
-                      gate-weighted combine; prefix property (low bits ignored)
+                      gate-weighted combine; prefix property (low bits ignored); at
+                      target = kmax = B the layer equals a torch fp32 computation (topk,
+                      softmax, textbook dequantisation, matmul, silu) on the dense weights
   rmsnorm / stack     pinned: closed form on constant vectors; composition check
 """
 from __future__ import annotations
@@ -349,22 +353,6 @@ def allocate(idx: np.ndarray, gates: np.ndarray, r: np.ndarray, kmin: int, kmax:
             hi = mid
     k = choose_k(c, hi, kmin, kmax)
     return k.reshape(idx.shape), hi
-
-
-# ---------------------------------------------------------------------------
-# Token -> expert permutation: pairs grouped by expert, then by k, then token order.
-# (Pure bookkeeping; only the grouping is checked, any order inside a group is valid.)
-# ---------------------------------------------------------------------------
-
-
-def permute(idx: np.ndarray, k: np.ndarray, n_experts: int):
-    e = idx.reshape(-1)
-    kk = k.reshape(-1)
-    order = sorted(range(e.size), key=lambda p: (int(e[p]), int(kk[p]), p))
-    kmax_e = np.zeros(n_experts, dtype=np.int64)
-    for p in range(e.size):
-        kmax_e[e[p]] = max(kmax_e[e[p]], kk[p])
-    return np.asarray(order, dtype=np.int64), kmax_e
 
 
 # ---------------------------------------------------------------------------

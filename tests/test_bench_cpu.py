@@ -79,5 +79,14 @@ def test_reference_arm_prints_one_contract_line():
     assert line["unit"] == "tokens/s" and line["higher_is_better"] is True and line["value"] > 0
     assert line["config"]["workload"] == W.TINY.name
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] == 1 and line["cpu_baseline"]["affinity_cores"] >= 1
+    assert isinstance(line["cpu_baseline"]["cpu_model"], str)
     assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def test_headline_budget_of_each_workload():
+    # the batch-64 layer is quoted at the middle of its budget sweep, the others at their budget
+    assert bench.headline_target(W.QWEN3_B64) == 3.0
+    assert bench.headline_target(W.QWEN3_B1) == 2.5
+    assert bench.parse_args([]).workload == W.QWEN3_B64.name

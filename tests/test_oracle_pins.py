@@ -204,6 +204,114 @@ def test_bcq_closed_forms():
         prev = e
 
 
+def _golden_bcq():
+    fx = json.load(open(os.path.join(GOLDEN, "bcq_worked_group.json")))
+    u = fx["unit"]
+    w = np.array(fx["w_units"], dtype=np.float64) * u
+    return fx, u, w
+
+
+def _bcq_pin_holds(encode, dequant):
+    """The hand-worked group: exact signs, alphas, w_hat(k) and squared residuals."""
+    fx, u, w = _golden_bcq()
+    B, G = fx["B"], fx["G"]
+    signs, alpha = encode(w.astype(np.float32)[None, :], B, G)
+    if not np.array_equal(signs[:, 0, :].astype(int), np.array(fx["signs"])):
+        return False
+    if [float(a) for a in alpha[:, 0, 0]] != [a * u for a in fx["alpha_units"]]:
+        return False
+    for k in range(1, B + 1):
+        wh = dequant(signs, alpha, k, G)[0]
+        if wh.tolist() != [v * u for v in fx["w_hat_units"][str(k)]]:
+            return False
+        if float(np.sum((w - wh) ** 2)) != fx["r_units2"][str(k)] * u * u:
+            return False
+    return True
+
+
+def test_bcq_hand_worked_group_exact():
+    assert _bcq_pin_holds(O.encode_bcq_matrix, O.dequant_bcq)
+
+
+def test_planted_bcq_mistakes_fail_the_pin():
+    def sign_swap_after_first(signs, alpha, k, G):      # b = -1 for a set bit on planes >= 1
+        B, R, C = signs.shape
+        out = np.zeros((R, C))
+        for i in range(k):
+            b = np.where(signs[i], 1.0, -1.0) * (1.0 if i == 0 else -1.0)
+            out = out + np.repeat(alpha[i], G, axis=1) * b
+        return out
+
+    def alpha_of_previous_plane(signs, alpha, k, G):    # plane i scaled by alpha_{i-1}
+        B, R, C = signs.shape
+        out = np.zeros((R, C))
+        for i in range(k):
+            out = out + np.repeat(alpha[max(i - 1, 0)], G, axis=1) * np.where(signs[i], 1.0, -1.0)
+        return out
+
+    def one_plane_short(signs, alpha, k, G):            # dropped last term
+        return O.dequant_bcq(signs, alpha, k - 1, G) if k > 1 else np.zeros(signs.shape[1:])
+
+    def refit_sign_of_zero_negative(w, B, G):           # sign(0) = -1 instead of +1
+        R, C = w.shape
+        res = np.asarray(w, np.float64).reshape(R, C // G, G).copy()
+        signs = np.empty((B, R, C // G, G), dtype=bool)
+        alpha = np.empty((B, R, C // G))
+        for i in range(B):
+            pos = res > 0.0
+            a = O.fp16_round(np.abs(res).sum(-1) / G)
+            res = res - a[..., None] * np.where(pos, 1.0, -1.0)
+            signs[i], alpha[i] = pos, a
+        return signs.reshape(B, R, C), alpha
+
+    for bad in (sign_swap_after_first, alpha_of_previous_plane, one_plane_short):
+        assert not _bcq_pin_holds(O.encode_bcq_matrix, bad), bad.__name__
+    # the sign(0) reading shows on a group whose residual reaches exactly 0
+    c = 0.0234375
+    w = (c * np.array([1, -1, -1, 1, 1, 1, -1, 1], dtype=np.float64)).astype(np.float32)[None, :]
+    s_good, _ = O.encode_bcq_matrix(w, 3, 8)
+    s_bad, _ = refit_sign_of_zero_negative(w, 3, 8)
+    assert np.all(s_good[1]) and not np.array_equal(s_good, s_bad)
+
+
+def _exact_greedy_bcq(row_group, B):
+    """Greedy binary-coded fit of one group in exact rational arithmetic: signs (True = +1),
+    alphas (fp16-rounded exact means) and the exact squared residual after each plane."""
+    R = [Fraction(float(v)) for v in row_group]
+    G = len(R)
+    signs, alphas, res2 = [], [], []
+    for _ in range(B):
+        b = [r >= 0 for r in R]
+        a = rne_to_format(sum(abs(r) for r in R) / G, 10, -14)
+        R = [r - a if bb else r + a for r, bb in zip(R, b)]
+        signs.append(b)
+        alphas.append(a)
+        res2.append(sum(r * r for r in R))
+    return signs, alphas, res2
+
+
+def test_bcq_fit_and_residual_table_exact_random():
+    # values on a 2^-24 grid below 0.1 in magnitude: the exact greedy fit and the oracle's fp64
+    # fit take the same steps, and every residual and sum of squares is exact in fp64
+    rng = np.random.default_rng(31)
+    H, I, G, B = 16, 8, 8, 3
+    mats = [np.clip(np.round(rng.standard_normal(sh) * 0.02 * 2.0 ** 24) / 2.0 ** 24, -0.09, 0.09).astype(np.float32)
+            for sh in ((I, H), (I, H), (H, I))]
+    enc = O.encode_expert(*mats, 1, B, G)
+    total = [Fraction(0)] * B
+    for m, sg, al in zip(mats, enc["signs"], enc["alpha"]):
+        Rr, C = m.shape
+        for i in range(Rr):
+            for gi in range(C // G):
+                signs, alphas, res2 = _exact_greedy_bcq(m[i, gi * G:(gi + 1) * G], B)
+                for p in range(B):
+                    assert Fraction(float(al[p, i, gi])) == alphas[p]
+                    assert sg[p, i, gi * G:(gi + 1) * G].tolist() == signs[p]
+                    total[p] += res2[p]
+    for k in range(1, B + 1):
+        assert Fraction(float(enc["r"][k - 1])) == total[k - 1], k
+
+
 # ----------------------------------------------------------------- exp
 
 def _cr_exp(x: float) -> float:
@@ -432,6 +540,62 @@ def test_bcq_moe_runs_and_shared_expert_adds():
         extra = O.expert_ffn(x[t], O.bf16_bits_to_f64(sh[0][0]), O.bf16_bits_to_f64(sh[1][0]),
                              O.bf16_bits_to_f64(sh[2][0]))
         np.testing.assert_allclose(y2[t] - y[t], extra, rtol=1e-12, atol=1e-14)
+
+
+def _torch_layer_at_full_rate(shape, experts, xb, wb):
+    """The layer at k = B with library routines only (torch, CPU): fp64 logits, torch.topk,
+    torch.softmax, the textbook dequantisation s*(q - z) or sum_i alpha_i*b_i of the stored
+    codes, and fp32 matmuls with torch's silu."""
+    import torch
+    x64 = torch.from_numpy(O.bf16_bits_to_f64(xb))
+    w64 = torch.from_numpy(O.bf16_bits_to_f64(wb))
+    logits = x64 @ w64.T
+    top, idx = torch.topk(logits, shape.top_k, dim=1)
+    if shape.norm_topk:
+        gates = torch.softmax(top, dim=1)
+    else:
+        gates = torch.gather(torch.softmax(logits, dim=1), 1, idx)
+    G = shape.group
+
+    def dense(enc, m):
+        if shape.fmt == 0:
+            q = torch.from_numpy(enc["q"][m].astype(np.float32))
+            s = torch.from_numpy(enc["s"][m].astype(np.float32)).repeat_interleave(G, dim=1)
+            z = torch.from_numpy(enc["z"][m].astype(np.float32)).repeat_interleave(G, dim=1)
+            return s * (q - z)
+        sg = torch.from_numpy(enc["signs"][m])
+        al = torch.from_numpy(enc["alpha"][m].astype(np.float32)).repeat_interleave(G, dim=2)
+        return (al * (sg.float() * 2.0 - 1.0)).sum(dim=0)
+
+    x32 = x64.float()
+    y = torch.zeros((xb.shape[0], shape.hidden), dtype=torch.float32)
+    for t in range(xb.shape[0]):
+        for j in range(shape.top_k):
+            enc = experts[int(idx[t, j])]
+            wg, wu, wd = dense(enc, 0), dense(enc, 1), dense(enc, 2)
+            h = torch.nn.functional.silu(wg @ x32[t]) * (wu @ x32[t])
+            y[t] += float(gates[t, j]) * (wd @ h)
+    return y.numpy().astype(np.float64), idx.numpy(), gates.numpy()
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_layer_at_full_rate_matches_torch_library_routines(fmt):
+    from dynamic_any_precision_b200.workloads import LayerShape
+    B, kmin = (4, 2) if fmt == 0 else (3, 1)
+    shape = LayerShape("lib_check", 64, 32, 6, 2, 0, fmt, B, kmin, B, 16, 1 - fmt, 5, (float(B),), 41)
+    rng = np.random.default_rng(41 + fmt)
+    experts = {}
+    for e in range(shape.n_experts):
+        mats = [(rng.standard_normal(sh) * 0.1).astype(np.float32) for sh in ((32, 64), (32, 64), (64, 32))]
+        experts[e] = O.encode_expert(*mats, fmt, B, 16)
+    xb = _bf16_bits(rng.standard_normal((5, 64)))
+    wb = _bf16_bits(rng.standard_normal((6, 64)) * 0.3)
+    y, aux = O.moe_forward(xb, wb, experts, shape, float(B))
+    assert np.all(aux["k"] == B)
+    y_t, idx_t, g_t = _torch_layer_at_full_rate(shape, experts, xb, wb)
+    assert np.array_equal(aux["idx"], idx_t)
+    np.testing.assert_allclose(aux["gates"], g_t, rtol=1e-12, atol=0)
+    np.testing.assert_allclose(y, y_t, rtol=2e-5, atol=2e-6)
 
 
 # ----------------------------------------------------------------- stack glue
