@@ -163,9 +163,13 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     pdl_wait();   // the routed pairs come from the previous kernel
     pdl_trigger();   // the successor may become resident now (it waits for this kernel)
     // the budget, the pairs' experts and gates are loaded together (one round trip)
-    const double target = *a.target;
-    int bad = (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1;
-    if (bad && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 10);
+    const double target = a.policy == DPA_ALLOC_THRESHOLD ? 0.0 : *a.target;   // unused by the threshold
+    const double tau = a.policy == DPA_ALLOC_THRESHOLD ? *a.threshold : 0.0;
+    // the budget policies need a target in [kmin, kmax]; the threshold policy a finite threshold
+    int bad = a.policy == DPA_ALLOC_THRESHOLD
+                  ? ((tau >= -1.0e300 && tau <= 1.0e300) ? 0 : 1)
+                  : ((target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1);
+    if (bad && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, a.policy == DPA_ALLOC_THRESHOLD ? 12 : 10);
     int bad_e = 0;
     for (int p = tid; p < P; p += blockDim.x) {
         const int e = a.idx[p];
@@ -183,6 +187,30 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
 
     if (a.k_given) {   // plane counts (and lambda) already chosen by the grid-wide bisection
         for (int p = tid; p < P; p += blockDim.x) s_k[p] = a.k_out[p];
+        __syncthreads();
+        goto grouping;
+    }
+    if (a.policy == DPA_ALLOC_UNIFORM) {
+        // equal shares of floor(target * P) planes; the first (budget mod P) pairs one more
+        const int nb = static_cast<int>(floor(__dmul_rn(target, static_cast<double>(P))));
+        const int base = nb / P, rem = nb - base * P;
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int k = base + (p < rem ? 1 : 0);
+            a.k_out[p] = static_cast<uint8_t>(k);
+            s_k[p] = static_cast<uint8_t>(k);
+        }
+        if (tid == 0 && a.lambda_out) *a.lambda_out = 0.0;
+        __syncthreads();
+        goto grouping;
+    }
+    if (a.policy == DPA_ALLOC_THRESHOLD) {
+        // high precision above the calibrated score threshold, low precision otherwise
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int k = a.gate[p] > tau ? a.kmax : a.kmin;
+            a.k_out[p] = static_cast<uint8_t>(k);
+            s_k[p] = static_cast<uint8_t>(k);
+        }
+        if (tid == 0 && a.lambda_out) *a.lambda_out = tau;
         __syncthreads();
         goto grouping;
     }
@@ -777,7 +805,50 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
     if (blockIdx.x == 0 && tid == 0 && a.lambda_out) *a.lambda_out = hi;
 }
 
+// ---------------- threshold calibration (score-threshold policy) ----------------
+// MatMoE, review "Core Contribution": a binary search over a calibration distribution of routing
+// scores sets the threshold above which an expert runs at high precision, so that the average
+// bit-width meets the target. 64 fp64 bisection steps on [0, 1]: with c(mid) = #{s > mid},
+// the plane count kmin*n + (kmax-kmin)*c(mid) above floor(target*n) moves lo up, else hi down;
+// the threshold is hi. One CTA; the counts are exact integer sums.
+constexpr int kCalibThreads = 1024;
+
+__global__ void __launch_bounds__(kCalibThreads) calibrate_kernel(CalibArgs a) {
+    __shared__ int s_cnt[kCalibThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    pdl_wait();
+    const double target = *a.target;
+    if (!(target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax))) {
+        if (tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 13);
+        return;
+    }
+    const long long nb = static_cast<long long>(floor(__dmul_rn(target, static_cast<double>(a.n))));
+    const long long base = static_cast<long long>(a.kmin) * a.n;
+    const int dk = a.kmax - a.kmin;
+    double lo = 0.0, hi = 1.0;
+    for (int it = 0; it < 64; ++it) {
+        const double mid = __dmul_rn(0.5, __dadd_rn(lo, hi));
+        int c = 0;
+        for (int i = tid; i < a.n; i += blockDim.x) c += a.scores[i] > mid ? 1 : 0;
+        c = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+        if (lane == 0) s_cnt[warp] = c;
+        __syncthreads();
+        long long tot = 0;
+        for (int w = 0; w < nw; ++w) tot += s_cnt[w];
+        __syncthreads();
+        if (base + static_cast<long long>(dk) * tot > nb) lo = mid; else hi = mid;
+    }
+    if (tid == 0) *a.threshold_out = hi;
+}
+
 }  // namespace
+
+cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t stream) {
+    CalibArgs b = a;
+    void* args[] = {&b};
+    return launch_pdl_raw(reinterpret_cast<const void*>(calibrate_kernel), dim3(1), dim3(kCalibThreads), 0, stream,
+                          args);
+}
 
 size_t allocate_smem_bytes(int P, int E, int nk) { return alloc_smem_layout(P, E, nk).total; }
 
@@ -789,7 +860,7 @@ cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* c
     AllocArgs b = a;
     const int coop_blocks = sms > 0 ? (P / 64 < sms ? (P + 63) / 64 : sms) : 1;
     int per_block = (P + coop_blocks - 1) / coop_blocks;
-    if (coop && P > kCoopMinPairs && per_block <= kCoopMaxPairsPerBlock) {
+    if (coop && a.policy == DPA_ALLOC_LAGRANGE && P > kCoopMinPairs && per_block <= kCoopMaxPairsPerBlock) {
         // grid-wide bisection: the pairs split over (at most) every SM, costs in shared memory
         const int blocks = coop_blocks;
         const size_t smem = static_cast<size_t>(per_block) * 32;

@@ -239,8 +239,11 @@ dpa_status dpa_route(const dpa_layer_desc* d, const void* x, int n_tokens, const
 static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, const int32_t* idx,
                                 const double* gate, int T, const double* target, uint8_t* k_out,
                                 double* lambda_out, void* ws, const WsLayout& L, bool permute, cudaStream_t s,
-                                bool gemm_tiles = false) {
+                                bool gemm_tiles = false, int policy = DPA_ALLOC_LAGRANGE,
+                                const double* threshold = nullptr) {
     dpa::AllocArgs a{};
+    a.policy = policy;
+    a.threshold = threshold;
     a.rtable = rtable;
     a.idx = idx;
     a.gate = gate;
@@ -265,20 +268,61 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
                                                                                                   : DPA_ERR_CUDA;
 }
 
-dpa_status dpa_allocate(const dpa_layer_desc* d, const double* rtable, const int32_t* topk_idx,
-                        const double* topk_gate, int n_tokens, const double* target_bpw, uint8_t* k_out,
-                        double* lambda_out, void* ws, size_t ws_bytes, void* stream) {
+static bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+// The policy and its scalar inputs: the budget policies read the target, the threshold policy
+// the threshold.
+static bool policy_inputs_ok(int policy, const double* target, const double* threshold) {
+    if (policy == DPA_ALLOC_LAGRANGE || policy == DPA_ALLOC_UNIFORM) return target && aligned8(target);
+    if (policy == DPA_ALLOC_THRESHOLD) return threshold && aligned8(threshold) && (!target || aligned8(target));
+    return false;
+}
+
+dpa_status dpa_allocate_ex(const dpa_layer_desc* d, int policy, const double* rtable, const int32_t* topk_idx,
+                           const double* topk_gate, int n_tokens, const double* target_bpw, const double* threshold,
+                           uint8_t* k_out, double* lambda_out, void* ws, size_t ws_bytes, void* stream) {
     const dpa_status st = check_desc(d);
     if (st != DPA_OK) return st;
-    if (n_tokens <= 0 || n_tokens > 65535 || !rtable || !topk_idx || !topk_gate || !target_bpw || !k_out || !ws)
-        return DPA_ERR_INVALID_ARG;
-    if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(rtable) & 7) || (reinterpret_cast<uintptr_t>(topk_gate) & 7) ||
-        (reinterpret_cast<uintptr_t>(target_bpw) & 7) || (reinterpret_cast<uintptr_t>(topk_idx) & 3))
+    if (n_tokens <= 0 || n_tokens > 65535 || !topk_idx || !topk_gate || !k_out || !ws) return DPA_ERR_INVALID_ARG;
+    if (!policy_inputs_ok(policy, target_bpw, threshold)) return DPA_ERR_INVALID_ARG;
+    if (policy == DPA_ALLOC_LAGRANGE && !rtable) return DPA_ERR_INVALID_ARG;
+    if (!aligned16(ws) || (rtable && !aligned8(rtable)) || !aligned8(topk_gate) ||
+        (reinterpret_cast<uintptr_t>(topk_idx) & 3) || (lambda_out && !aligned8(lambda_out)))
         return DPA_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(d, n_tokens);
     if (ws_bytes < L.total) return DPA_ERR_WORKSPACE;
-    return allocate_impl(d, rtable, topk_idx, topk_gate, n_tokens, target_bpw, k_out, lambda_out, ws, L, false,
-                         static_cast<cudaStream_t>(stream));
+    // the threshold policy reads no target: the threshold pointer stands in for it
+    const double* tg = target_bpw ? target_bpw : threshold;
+    return allocate_impl(d, rtable, topk_idx, topk_gate, n_tokens, tg, k_out, lambda_out, ws, L, false,
+                         static_cast<cudaStream_t>(stream), false, policy, threshold);
+}
+
+dpa_status dpa_allocate(const dpa_layer_desc* d, const double* rtable, const int32_t* topk_idx,
+                        const double* topk_gate, int n_tokens, const double* target_bpw, uint8_t* k_out,
+                        double* lambda_out, void* ws, size_t ws_bytes, void* stream) {
+    return dpa_allocate_ex(d, DPA_ALLOC_LAGRANGE, rtable, topk_idx, topk_gate, n_tokens, target_bpw, nullptr, k_out,
+                           lambda_out, ws, ws_bytes, stream);
+}
+
+dpa_status dpa_calibrate_threshold(const dpa_layer_desc* d, const double* scores, int n_scores,
+                                   const double* target_bpw, double* threshold_out, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (!scores || n_scores <= 0 || n_scores > (1 << 26) || !target_bpw || !threshold_out || !ws)
+        return DPA_ERR_INVALID_ARG;
+    if (!aligned8(scores) || !aligned8(target_bpw) || !aligned8(threshold_out) || !aligned16(ws))
+        return DPA_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(d, 1).total) return DPA_ERR_WORKSPACE;
+    dpa::CalibArgs a{};
+    a.scores = scores;
+    a.n = n_scores;
+    a.kmin = d->kmin;
+    a.kmax = d->kmax;
+    a.target = target_bpw;
+    a.threshold_out = threshold_out;
+    a.hdr = at<dpa::WsHeader>(ws, 0);
+    return dpa::launch_calibrate(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
 }
 
 dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, const void* x, int n_tokens,
@@ -304,6 +348,9 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     const int T = n_tokens, K = d->top_k;
     const int path = aux ? aux->expert_path : DPA_PATH_AUTO;
     if (path < DPA_PATH_AUTO || path > DPA_PATH_TC) return DPA_ERR_INVALID_ARG;
+    const int policy = aux ? aux->alloc_policy : DPA_ALLOC_LAGRANGE;
+    const double* threshold = aux ? aux->threshold : nullptr;
+    if (!policy_inputs_ok(policy, target_bpw, threshold)) return DPA_ERR_INVALID_ARG;
     const bool tc_shape = d->format == DPA_FMT_UNIFORM && d->hidden % 256 == 0 && d->inter % 256 == 0 &&
                           (d->group & (d->group - 1)) == 0;   // scale groups of 64 * 2^n inputs
     if (path == DPA_PATH_TC && !tc_shape) return DPA_ERR_UNSUPPORTED;
@@ -345,7 +392,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     mark(1);
 
     // 2. allocate + group pairs by (expert, k)
-    dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s, use_tc);
+    dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s, use_tc, policy,
+                                   threshold);
     if (st2 != DPA_OK) return st2;
     mark(2);
 

@@ -47,6 +47,8 @@ struct AllocArgs {
     int4* gtiles;             // nullptr, or [P/kGemmTileTokens + E*nk] GEMM token tiles {e, k, pos0, n}
     int32_t* pos_tok;         // nullptr, or [P] token of each grouped position
     WsHeader* hdr;
+    int policy;               // DPA_ALLOC_LAGRANGE, DPA_ALLOC_UNIFORM or DPA_ALLOC_THRESHOLD
+    const double* threshold;  // device scalar (DPA_ALLOC_THRESHOLD)
 };
 // Counters of the grid-wide bisection (zeroed by the launcher before every call).
 constexpr int kCoopRoundsMax = 16;
@@ -60,6 +62,16 @@ struct CoopSync {
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* coop = nullptr, int sms = 0);
 size_t allocate_smem_bytes(int P, int E, int nk);
 int allocate_threads(int P);
+
+// Threshold calibration of the score-threshold policy: 64 bisection steps over n scores.
+struct CalibArgs {
+    const double* scores;     // [n]
+    int n, kmin, kmax;
+    const double* target;     // device scalar
+    double* threshold_out;    // device scalar
+    WsHeader* hdr;
+};
+cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t stream);
 
 // Prefill expert FFN on tcgen05: grouped GEMMs over the GEMM token tiles of the allocation.
 struct GemmArgs {

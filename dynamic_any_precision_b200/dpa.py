@@ -51,14 +51,16 @@ class LayerWeights(ctypes.Structure):
 class Aux(ctypes.Structure):
     _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_gate", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("lambda_", ctypes.c_void_p), ("pair_out", ctypes.c_void_p),
-                ("events", ctypes.c_void_p * 7), ("expert_path", ctypes.c_int32)]
+                ("events", ctypes.c_void_p * 7), ("expert_path", ctypes.c_int32),
+                ("alloc_policy", ctypes.c_int32), ("threshold", ctypes.c_void_p)]
 
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD = 0, 1, 2
 
 
 EXPORTED = ("dpa_encoded_sizes", "dpa_encode", "dpa_export_codes", "dpa_export_meta", "dpa_route",
-            "dpa_allocate", "dpa_forward_workspace_size", "dpa_moe_forward", "dpa_device_status",
-            "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm")
+            "dpa_allocate", "dpa_allocate_ex", "dpa_calibrate_threshold", "dpa_forward_workspace_size",
+            "dpa_moe_forward", "dpa_device_status", "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm")
 
 _lib = None
 
@@ -80,6 +82,8 @@ def lib() -> ctypes.CDLL:
     L.dpa_export_meta.argtypes = [P(LayerDesc), vp, i32, i32, vp, vp]
     L.dpa_route.argtypes = [P(LayerDesc), vp, i32, vp, vp, vp, vp, vp, sz, vp]
     L.dpa_allocate.argtypes = [P(LayerDesc), vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
+    L.dpa_allocate_ex.argtypes = [P(LayerDesc), i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.dpa_calibrate_threshold.argtypes = [P(LayerDesc), vp, i32, vp, vp, vp, sz, vp]
     L.dpa_forward_workspace_size.argtypes = [P(LayerDesc), i32]
     L.dpa_forward_workspace_size.restype = sz
     L.dpa_moe_forward.argtypes = [P(LayerDesc), P(LayerWeights), vp, i32, vp, vp, P(Aux), vp, sz, vp]
@@ -203,15 +207,32 @@ def route(desc: LayerDesc, x, w_router, ws, logits=None, stream=None):
     return idx, gate
 
 
-def allocate(desc: LayerDesc, rtable, idx, gate, target, ws, stream=None):
-    """target: CUDA fp64 scalar tensor. Returns (k uint8 [T][K], lambda fp64 [1])."""
+def allocate(desc: LayerDesc, rtable, idx, gate, target, ws, stream=None, policy: int = ALLOC_LAGRANGE,
+             threshold=None):
+    """target: CUDA fp64 scalar tensor (None for the threshold policy); threshold: CUDA fp64
+    scalar tensor (threshold policy). Returns (k uint8 [T][K], lambda fp64 [1])."""
     import torch
     T = idx.shape[0]
     k = torch.empty((T, desc.top_k), dtype=torch.uint8, device=idx.device)
     lam = torch.empty(1, dtype=torch.float64, device=idx.device)
-    _check(lib().dpa_allocate(ctypes.byref(desc), _dptr(rtable), _dptr(idx), _dptr(gate), T, _dptr(target), _dptr(k),
-                              _dptr(lam), _dptr(ws), ws.numel(), _stream(stream)), "dpa_allocate")
+    if policy == ALLOC_LAGRANGE:
+        _check(lib().dpa_allocate(ctypes.byref(desc), _dptr(rtable), _dptr(idx), _dptr(gate), T, _dptr(target),
+                                  _dptr(k), _dptr(lam), _dptr(ws), ws.numel(), _stream(stream)), "dpa_allocate")
+    else:
+        _check(lib().dpa_allocate_ex(ctypes.byref(desc), policy, _dptr(rtable), _dptr(idx), _dptr(gate), T,
+                                     _dptr(target), _dptr(threshold), _dptr(k), _dptr(lam), _dptr(ws), ws.numel(),
+                                     _stream(stream)), "dpa_allocate_ex")
     return k, lam
+
+
+def calibrate_threshold(desc: LayerDesc, scores, target, ws, stream=None):
+    """scores: CUDA fp64 tensor (any shape) of calibration routing scores; target: CUDA fp64
+    scalar tensor. Returns the threshold as a CUDA fp64 [1] tensor."""
+    import torch
+    tau = torch.empty(1, dtype=torch.float64, device=scores.device)
+    _check(lib().dpa_calibrate_threshold(ctypes.byref(desc), _dptr(scores), scores.numel(), _dptr(target), _dptr(tau),
+                                         _dptr(ws), ws.numel(), _stream(stream)), "dpa_calibrate_threshold")
+    return tau
 
 
 class DeviceLayer:
@@ -242,7 +263,8 @@ def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] =
     """One MoE layer. x: CUDA int16/bf16 bits [T][H]; target: CUDA fp64 scalar tensor.
     aux: optional dict of preallocated CUDA tensors with keys topk_idx, topk_gate, k, lambda,
     pair_out, "events": up to 7 torch.cuda.Event(enable_timing=True) recorded at the
-    stage boundaries, and "expert_path" (PATH_AUTO, PATH_GEMV or PATH_TC).
+    stage boundaries, "expert_path" (PATH_AUTO, PATH_GEMV or PATH_TC), "alloc_policy"
+    (ALLOC_LAGRANGE, ALLOC_UNIFORM or ALLOC_THRESHOLD) and "threshold" (CUDA fp64 scalar).
     Returns y (int16 bf16 bits [T][H])."""
     import torch
     T = x.shape[0]
@@ -258,6 +280,8 @@ def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] =
                     raise ValueError("record a torch.cuda.Event once before passing it (lazy creation)")
                 aux_s.events[i] = ev.cuda_event
         aux_s.expert_path = int(aux.get("expert_path", PATH_AUTO))
+        aux_s.alloc_policy = int(aux.get("alloc_policy", ALLOC_LAGRANGE))
+        aux_s.threshold = _dptr(aux.get("threshold"))
     _check(lib().dpa_moe_forward(ctypes.byref(layer.desc), ctypes.byref(layer.weights), _dptr(x), T, _dptr(target),
                                  _dptr(y), ctypes.byref(aux_s) if aux_s is not None else None, _dptr(ws), ws.numel(),
                                  _stream(stream)), "dpa_moe_forward")

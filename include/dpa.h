@@ -136,6 +136,9 @@ typedef struct dpa_layer_weights {
 #define DPA_PATH_GEMV 1
 #define DPA_PATH_TC 2
 #define DPA_TC_MIN_PAIRS_PER_EXPERT 16
+/* alloc_policy: how the routed pairs' plane counts are chosen (see dpa_allocate_ex); threshold:
+ * device fp64 scalar read by DPA_ALLOC_THRESHOLD (NULL otherwise). With alloc_policy = 0 the
+ * Lagrangian allocation of dpa_allocate runs. */
 typedef struct dpa_aux {
     int32_t* topk_idx;
     double* topk_gate;
@@ -144,6 +147,8 @@ typedef struct dpa_aux {
     float* pair_out;
     void* events[7];
     int32_t expert_path;
+    int32_t alloc_policy;
+    const double* threshold;
 } dpa_aux;
 
 /* Validate a descriptor and return the encoded sizes. Host only. */
@@ -210,6 +215,47 @@ dpa_status dpa_allocate(const dpa_layer_desc* desc, const double* rtable,
                         const double* target_bpw, uint8_t* k_out, double* lambda_out,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation policies (dpa_allocate_ex, dpa_aux.alloc_policy):
+ *  DPA_ALLOC_LAGRANGE (0)  the gate-driven Lagrangian allocation of dpa_allocate (DPA-MoE,
+ *                          Abstract; DuoRate, Abstract). lambda_out = the final multiplier.
+ *  DPA_ALLOC_UNIFORM (1)   the control DPA-MoE, Abstract, compares with: uniform chunk
+ *                          allocation at a matched budget. The budget floor(target*P) planes
+ *                          is shared equally: every pair reads floor(budget/P) planes and the
+ *                          first (budget mod P) pairs in token-major slot order one more; the
+ *                          gates are ignored. lambda_out = 0.
+ *  DPA_ALLOC_THRESHOLD (2) MatMoE, review "Core Contribution": a pair whose routing score (its
+ *                          gate) is above a threshold reads kmax planes, every other pair kmin.
+ *                          The threshold comes from dpa_calibrate_threshold ahead of time; no
+ *                          budget is enforced on the live batch. target_bpw is not read (may be
+ *                          NULL). lambda_out = the threshold. */
+#define DPA_ALLOC_LAGRANGE 0
+#define DPA_ALLOC_UNIFORM 1
+#define DPA_ALLOC_THRESHOLD 2
+
+/* dpa_allocate with a choice of policy (device). Arguments as dpa_allocate, plus
+ * policy (above) and threshold: device fp64 scalar, read by DPA_ALLOC_THRESHOLD only (a NaN or
+ * infinite threshold sets the device flag DPA_ERR_DEVICE_INVALID_INPUT and leaves k untouched).
+ * Errors: DPA_ERR_INVALID_ARG for an unknown policy or a missing threshold. */
+dpa_status dpa_allocate_ex(const dpa_layer_desc* desc, int policy, const double* rtable,
+                           const int32_t* topk_idx, const double* topk_gate, int n_tokens,
+                           const double* target_bpw, const double* threshold, uint8_t* k_out,
+                           double* lambda_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Threshold of DPA_ALLOC_THRESHOLD from a calibration set of routing scores (device).
+ * Defined by: MatMoE, review "Core Contribution" (a binary search over a calibration score
+ * distribution sets the threshold so that the average bit-width meets the target).
+ * scores: device fp64 [n_scores], the gates of a calibration batch's routed pairs (for
+ * example dpa_route's topk_gate on calibration tokens). 64 fp64 bisection steps on [0, 1]:
+ *   mid = 0.5*(lo+hi); planes = kmin*n + (kmax-kmin)*#{s > mid};
+ *   if planes > target*n then lo = mid else hi = mid;
+ * threshold_out (device fp64 scalar) = hi, so the calibration set's average plane count is at
+ * most the target. target_bpw: device fp64 scalar in [kmin, kmax] (else the device flag
+ * DPA_ERR_DEVICE_INVALID_INPUT, threshold untouched). ws: at least
+ * dpa_forward_workspace_size(desc, 1) bytes (its error flag is used). */
+dpa_status dpa_calibrate_threshold(const dpa_layer_desc* desc, const double* scores, int n_scores,
+                                   const double* target_bpw, double* threshold_out, void* ws,
+                                   size_t ws_bytes, void* stream);
+
 /* Allocation-free variant of dpa_route, for callers that cannot allocate device memory:
  * for example a plugin whose host engine owns every byte of device memory, or a loop that
  * must not call the allocator. It has no counterpart in the pages; it exists for those callers.
@@ -217,8 +263,11 @@ dpa_status dpa_allocate(const dpa_layer_desc* desc, const double* rtable,
  * counters and a logits buffer) lives in a fixed array of about 0.5 MB inside the library,
  * which every GPU that loads the library holds until the process exits.
  * Limits: n_tokens <= 1024 and n_tokens * n_experts <= 65536, else DPA_ERR_UNSUPPORTED
- * (nothing launched). The first call on a device looks up the array's device address, so
- * make it before any stream capture. Every call shares the array: calls whose executions
+ * (nothing launched). Every batch runs the router's per-logit kernel (dpa_route switches to
+ * its tiled kernels from 128 tokens; the decisions are the same). The first call on a device
+ * looks up the array's device address, so make it before any stream capture; the address is
+ * kept for the life of the process, so resetting the device (cudaDeviceReset) after that first
+ * call is not supported. Every call shares the array: calls whose executions
  * overlap on the GPU (other streams, other threads) race and must be serialised by the
  * caller. Device-side input checks (NaN/Inf tokens) are not reported by this variant.
  * logits may be NULL. stream: cudaStream_t. */

@@ -36,6 +36,10 @@ Parity status of each function (what pins it; see tests/test_oracle_pins.py):
                       top-k; expert permutation equivariance; softmax identities
   allocate            pinned: brute-force constrained optimum (Everett) on tiny inputs,
                       budget criterion, endpoint targets, monotone N along the bisection
+  allocate_uniform    pinned: closed form (sum = floor(target*P), spread <= 1, integer targets)
+  calibrate_threshold pinned: brute force over the cut points of the score distribution;
+  / allocate_threshold endpoints; two plane counts and equal residuals reduce the Lagrangian
+                      allocation of a batch to the threshold calibrated on that batch
   expert_ffn / moe    pinned: hand-worked tiny layer; top-1 identity; linearity of the
                       gate-weighted combine; prefix property (low bits ignored); at
                       target = kmax = B the layer equals a torch fp32 computation (topk,
@@ -356,6 +360,65 @@ def allocate(idx: np.ndarray, gates: np.ndarray, r: np.ndarray, kmin: int, kmax:
 
 
 # ---------------------------------------------------------------------------
+# Allocation policies other than the Lagrangian (the controls and the prior design the pages
+# compare with).
+# [DPA] Abstract: DPA-MoE is compared with "uniform chunk allocation at matched budgets".
+#   Reading: every routed pair gets an equal share of the same plane budget floor(target * P)
+#   (the Lagrangian's budget rule): k = floor(N / P) planes, and the first N mod P pairs in
+#   token-major slot order one plane more. It ignores the gates.
+# [MAT] Core Contribution: at run time an expert whose routing score is above a threshold runs
+#   at high precision and the others at low precision; the threshold comes from a binary search
+#   over a calibration distribution of routing scores so that the average bit-width meets the
+#   target. Readings: the routing score is the pair's gate g; high = kmax, low = kmin planes; the
+#   calibration distribution is the gates of a calibration batch's routed pairs; the search is
+#   64 fp64 bisection steps on [0, 1] (gates lie in [0, 1]) with the count of scores strictly
+#   above the midpoint:
+#       mid = 0.5 * (lo + hi); if kmin * n + (kmax - kmin) * #{s > mid} > target * n: lo = mid
+#       else hi = mid,
+#   and the threshold is hi, so the calibration average never exceeds the target. At run time
+#   k = kmax if g > threshold else kmin, with no budget enforced on the live batch (the threshold
+#   is fixed ahead of time).
+# ---------------------------------------------------------------------------
+
+
+def allocate_uniform(P: int, kmin: int, kmax: int, target: float) -> np.ndarray:
+    """Equal shares of the budget floor(target * P) planes over the P pairs (token-major order)."""
+    if not (kmin <= target <= kmax):
+        raise ValueError("target outside [kmin, kmax]")
+    n = int(math.floor(float(target) * float(P)))
+    base, rem = divmod(n, P)
+    return np.array([base + (1 if p < rem else 0) for p in range(P)], dtype=np.int64)
+
+
+def calibrate_threshold(scores: np.ndarray, kmin: int, kmax: int, target: float, iters: int = 64,
+                        trace: Optional[list] = None) -> float:
+    """Threshold on the routing score so that the calibration scores' average plane count
+    (kmax above the threshold, kmin otherwise) does not exceed the target."""
+    if not (kmin <= target <= kmax):
+        raise ValueError("target outside [kmin, kmax]")
+    s = np.asarray(scores, dtype=np.float64).reshape(-1)
+    n = s.size
+    budget = float(target) * float(n)
+    lo, hi = 0.0, 1.0
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        planes = kmin * n + (kmax - kmin) * int(np.count_nonzero(s > mid))
+        if trace is not None:
+            trace.append((mid, planes))
+        if float(planes) > budget:
+            lo = mid
+        else:
+            hi = mid
+    return hi
+
+
+def allocate_threshold(gates: np.ndarray, threshold: float, kmin: int, kmax: int) -> np.ndarray:
+    """k = kmax where the pair's gate is above the threshold, else kmin."""
+    g = np.asarray(gates, dtype=np.float64)
+    return np.where(g > float(threshold), kmax, kmin).astype(np.int64)
+
+
+# ---------------------------------------------------------------------------
 # Expert FFN (SwiGLU) and gate-weighted combine.
 #   a = W_gate^(k) x, u = W_up^(k) x, h = silu(a) * u, o = W_down^(k) h,
 #   y_t = sum_{slots j} g_{t,j} o_{t,j}  (+ sum of shared experts, dense, gate 1).
@@ -376,38 +439,70 @@ def expert_ffn(x: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) ->
     return wd @ h
 
 
+def combine_token(gates_row: Sequence[float], outs: Sequence[np.ndarray],
+                  shared_outs: Sequence[np.ndarray] = ()) -> np.ndarray:
+    """y_t = sum over slots j, in slot order, of g_{t,j} * o_{t,j}, then + each shared expert's
+    output (gate weight 1), accumulated in fp64 from zero."""
+    acc = np.zeros(np.asarray(outs[0] if len(outs) else shared_outs[0]).shape)
+    for g, o in zip(gates_row, outs):
+        acc = acc + float(g) * o
+    for o in shared_outs:
+        acc = acc + o
+    return acc
+
+
+def shared_outputs(x_row: np.ndarray, shared) -> List[np.ndarray]:
+    """Outputs of the always-on experts (dense bf16 weights) for one token."""
+    if shared is None:
+        return []
+    sg, su, sd = shared
+    return [expert_ffn(x_row, bf16_bits_to_f64(sg[s]), bf16_bits_to_f64(su[s]), bf16_bits_to_f64(sd[s]))
+            for s in range(sg.shape[0])]
+
+
+ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD = 0, 1, 2
+
+
+def allocate_policy(policy: int, idx: np.ndarray, gates: np.ndarray, r_table: Optional[np.ndarray], kmin: int,
+                    kmax: int, target: float, threshold: Optional[float] = None):
+    """Plane counts [T][K] and the policy's multiplier (lambda; the threshold; 0 for uniform)."""
+    if policy == ALLOC_LAGRANGE:
+        return allocate(idx, gates, r_table, kmin, kmax, target)
+    if policy == ALLOC_UNIFORM:
+        return allocate_uniform(idx.size, kmin, kmax, target).reshape(idx.shape), 0.0
+    if policy == ALLOC_THRESHOLD:
+        return allocate_threshold(gates, threshold, kmin, kmax).reshape(idx.shape), float(threshold)
+    raise ValueError("unknown allocation policy")
+
+
 def moe_forward(x_bits: np.ndarray, wr_bits: np.ndarray, experts: Dict[int, Dict], shape,
                 target: float, shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]] = None,
                 r_table: Optional[np.ndarray] = None, logits: Optional[np.ndarray] = None,
-                token_subset: Optional[Sequence[int]] = None):
+                token_subset: Optional[Sequence[int]] = None, policy: int = ALLOC_LAGRANGE,
+                threshold: Optional[float] = None):
     """One MoE layer. `experts` maps expert id -> encode_expert() output (only the experts that
     are routed to are needed); `r_table` is [E][B] (all experts' residuals; defaults to the
     encoded ones, which then must cover every expert). Returns y fp64 [T][H] (rows outside
     token_subset are NaN) and the decision-path results."""
     fmt, B, G = shape.fmt, shape.bits, shape.group
     idx, g, logits = route(x_bits, wr_bits, shape.top_k, shape.norm_topk, logits)
-    if r_table is None:
+    if r_table is None and policy == ALLOC_LAGRANGE:
         r_table = np.stack([experts[e]["r"] for e in range(shape.n_experts)])
-    k, lam = allocate(idx, g, r_table, shape.kmin, shape.kmax, target)
+    k, lam = allocate_policy(policy, idx, g, r_table, shape.kmin, shape.kmax, target, threshold)
     x = bf16_bits_to_f64(x_bits)
     T = x.shape[0]
     toks = range(T) if token_subset is None else token_subset
     y = np.full((T, shape.hidden), np.nan)
     dense_cache: Dict[Tuple[int, int], List[np.ndarray]] = {}
     for t in toks:
-        acc = np.zeros(shape.hidden)
+        outs = []
         for j in range(shape.top_k):
             e, kk = int(idx[t, j]), int(k[t, j])
             if (e, kk) not in dense_cache:
                 dense_cache[(e, kk)] = dequant_expert(experts[e], fmt, B, kk, G)
             wg, wu, wd = dense_cache[(e, kk)]
-            acc = acc + g[t, j] * expert_ffn(x[t], wg, wu, wd)
-        if shared is not None:
-            sg, su, sd = shared
-            for s in range(sg.shape[0]):
-                acc = acc + expert_ffn(x[t], bf16_bits_to_f64(sg[s]), bf16_bits_to_f64(su[s]),
-                                       bf16_bits_to_f64(sd[s]))
-        y[t] = acc
+            outs.append(expert_ffn(x[t], wg, wu, wd))
+        y[t] = combine_token(g[t], outs, shared_outputs(x[t], shared))
     return y, {"idx": idx, "gates": g, "logits": logits, "k": k, "lambda": lam}
 
 

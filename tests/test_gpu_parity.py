@@ -8,7 +8,7 @@ torch = pytest.importorskip("torch")
 
 from dynamic_any_precision_b200 import dpa, workloads as W  # noqa: E402
 from oracle import dpa_oracle as O  # noqa: E402
-from oracle_jobs import pair_outputs, reference_layer  # noqa: E402
+from oracle_jobs import pair_outputs, reference_layer, reference_layer_parallel  # noqa: E402
 
 pytestmark = pytest.mark.gpu
 TOL = 2e-3
@@ -210,7 +210,7 @@ def test_forward_qwen3_batch1():
     check_forward(W.QWEN3_B1, x, 2.5, sample_pairs=[(0, j) for j in range(8)])
 
 
-@pytest.mark.parametrize("target", [2.0, 3.0, 4.0])
+@pytest.mark.parametrize("target", [2.0, 2.5, 3.0, 3.5, 4.0])
 def test_forward_qwen3_batch64_sampled(target):
     x = W.tokens(W.QWEN3_B64)
     check_forward(W.QWEN3_B64, x, target, token_subset=[0, 5, 31, 63],
@@ -246,6 +246,89 @@ def test_prefix_property_poisoned_planes():
         assert np.array_equal(y0, y1)
     finally:
         gl.layer.planes.copy_(saved)
+
+
+def _poison_unread(gl, idx, k, seed_byte=0xA5):
+    """Overwrite, in device memory, every byte the forward must not read: planes >= kmax_e of
+    each routed expert e (kmax_e = the largest k among its pairs; for binary-coded layers also
+    those planes' alphas, with NaN), and all planes and scale data of experts nobody routed to
+    (scales and zeros as NaN). Returns the saved copies."""
+    shape = gl.shape
+    s = dpa.encoded_sizes(gl.desc)
+    saved = (gl.layer.planes.clone(), gl.layer.meta.clone())
+    kmax_e = {}
+    for e, kk in zip(idx.reshape(-1).tolist(), k.reshape(-1).tolist()):
+        kmax_e[e] = max(kmax_e.get(e, 0), int(kk))
+    p, mt = gl.layer.planes, gl.layer.meta
+    H, I, G, B = shape.hidden, shape.inter, shape.group, shape.bits
+    for e in range(shape.n_experts):
+        km = kmax_e.get(e, 0)
+        for m in range(3):
+            R, C = (H, I) if m == 2 else (I, H)
+            pb = R * C // 8
+            start = e * s.planes_per_expert + s.planes_matrix_offset[m]
+            p[start + km * pb: start + B * pb] = seed_byte
+            mstart = e * s.meta_per_expert + s.meta_matrix_offset[m]
+            if shape.fmt == W.FMT_BCQ:
+                ab = R * (C // G) * 2          # one plane's alphas
+                mt[mstart + km * ab: mstart + B * ab] = 0xFF
+            elif km == 0:
+                mt[mstart: mstart + R * (C // G) * 4] = 0xFF
+    torch.cuda.synchronize()
+    return saved
+
+
+@pytest.mark.parametrize("shape,T,target", [(W.QWEN3_B64, 4, 2.5), (W.QWEN3_B64, 9, 3.0), (W.QWEN3_B1, 1, 2.5),
+                                            (W.DEEPSEEK_B16, 16, 2.0)])
+def test_prefix_property_mixed_k_poisoned(shape, T, target):
+    # mixed plane counts: each routed expert reads only its first kmax_e planes (and, binary-coded,
+    # their alphas); poisoning everything beyond, and every unrouted expert, changes no output bit
+    gl = GpuLayer.get(shape)
+    x = W.tokens(shape, T, step=41)
+    y0, aux0, _ = gl.forward(x, target)
+    assert len(np.unique(aux0["k"])) > 1
+    saved = _poison_unread(gl, aux0["topk_idx"], aux0["k"])
+    try:
+        y1, aux1, _ = gl.forward(x, target)
+        assert np.array_equal(aux1["k"], aux0["k"])
+        assert np.array_equal(y0, y1)
+        assert np.array_equal(aux0["pair_out"], aux1["pair_out"])
+    finally:
+        gl.layer.planes.copy_(saved[0])
+        gl.layer.meta.copy_(saved[1])
+        torch.cuda.synchronize()
+
+
+def test_forward_activation_groups_spanning_many_binades():
+    # the expert kernels hold each scale group of activations as 22-bit fixed point under the
+    # group's largest exponent; groups spanning ~40 binades (values 2^-30 .. 2^9) lose only
+    # digits far below the tolerance
+    shape = W.TINY
+    rng = np.random.default_rng(77)
+    T, H = 6, shape.hidden
+    mag = np.exp2(rng.integers(-30, 10, size=(T, H)).astype(np.float64))
+    x = (mag * np.sign(rng.standard_normal((T, H))) * (1 + rng.random((T, H)))).astype(np.float32)
+    xb = W.f32_to_bf16_bits(x)
+    for target in (2.0, 3.0, 4.0):
+        check_forward(shape, xb, target, sample_pairs=[(0, 0), (T - 1, 1)])
+
+
+@pytest.mark.parametrize("fmt", [W.FMT_UNIFORM, W.FMT_BCQ])
+def test_forward_wide_hidden_several_tiles_per_expert(fmt):
+    # hidden 8192: the multi-token staging does not fit, so experts with many tokens run one
+    # two-token tile per pass, several passes per work item (8 experts, top-2, 16 tokens)
+    if fmt == W.FMT_UNIFORM:
+        shape = W.with_sizes(W.TINY, name="wide_h8192_uniform", hidden=8192, inter=512, group=128, tokens=16,
+                             seed=61)
+        target = 3.0
+    else:
+        shape = W.with_sizes(W.TINY, name="wide_h8192_bcq", hidden=8192, inter=512, group=128, tokens=16, fmt=W.FMT_BCQ,
+                             bits=3, kmin=1, kmax=3, norm_topk=0, seed=62)
+        target = 2.0
+    x = W.tokens(shape, 16, step=5)
+    y, aux, ref = check_forward(shape, x, target, sample_pairs=[(0, 0), (15, 1), (7, 0)])
+    counts = np.bincount(aux["topk_idx"].reshape(-1), minlength=shape.n_experts)
+    assert counts.max() >= 3
 
 
 def test_forward_deterministic_and_graph_capture():

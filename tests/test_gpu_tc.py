@@ -11,6 +11,7 @@ import pytest
 torch = pytest.importorskip("torch")
 
 from dynamic_any_precision_b200 import dpa, workloads as W  # noqa: E402
+from oracle_jobs import reference_layer_parallel  # noqa: E402
 from test_gpu_parity import GpuLayer, check_forward, within_tol  # noqa: E402
 
 pytestmark = pytest.mark.gpu
@@ -32,6 +33,31 @@ def test_tc_qwen3_prefill_sampled(target):
     x = W.tokens(W.QWEN3_B64, 256, step=7)
     check_forward(W.QWEN3_B64, x, target, token_subset=[0, 17, 128, 255], path=dpa.PATH_TC,
                   sample_pairs=[(0, 0), (17, 3), (255, 7)])
+
+
+@pytest.mark.parametrize("target", [4.0, 3.0])
+def test_tc_full_prefill_against_oracle(target):
+    # 2048 tokens (16,384 pairs, ~128 per expert: full 128-token tiles): the oracle routes and
+    # allocates every token (lambda couples the whole batch) and runs the expert FFNs of a strided
+    # 64-token subset; decisions bit-identical, outputs and per-pair outputs within 2e-3
+    gl = GpuLayer.get(W.QWEN3_B64)
+    T = 2048
+    x = W.tokens(W.QWEN3_B64, T, step=11)
+    ws = dpa.new_workspace(gl.desc, T)
+    y, aux, _ = gl.forward(x, target, ws=ws, with_pairs=True, path=dpa.PATH_TC)
+    subset = list(range(5, T, 32))
+    y_ref, ref = reference_layer_parallel(W.QWEN3_B64, x, target, subset)
+    assert np.array_equal(aux["topk_idx"], ref["idx"])
+    assert np.array_equal(aux["topk_gate"], ref["gates"])
+    assert np.array_equal(aux["k"].astype(np.int64), ref["k"])
+    assert aux["lambda"][0] == ref["lambda"]
+    if target < 4.0:
+        assert len(np.unique(aux["k"])) > 1
+    ok, worst = within_tol(y[subset], y_ref[subset])
+    assert ok, f"output tolerance exceeded: worst err/bound = {worst}"
+    for (t, j), o in ref["pair_out"].items():
+        ok, worst = within_tol(aux["pair_out"][t, j].astype(np.float64), o)
+        assert ok, (t, j, worst)
 
 
 def test_tc_agrees_with_gemv_at_full_prefill_size():

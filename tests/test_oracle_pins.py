@@ -465,6 +465,75 @@ def test_allocation_prefers_high_gate_pairs():
     assert k.tolist() == [[3, 2], [2, 2]]
 
 
+# ----------------------------------------------------------------- allocation policies
+
+@pytest.mark.parametrize("P,target", [(8, 3.0), (8, 2.5), (7, 2.2), (512, 3.1), (96, 2.0), (1, 3.999)])
+def test_uniform_allocation_closed_form(P, target):
+    kmin, kmax = 2, 4
+    k = O.allocate_uniform(P, kmin, kmax, target)
+    total = int(Fraction(target) * P)                      # floor of the exact budget
+    assert int(k.sum()) == total and k.max() - k.min() <= 1
+    assert np.all((k >= kmin) & (k <= kmax))
+    assert np.all(np.diff(k) <= 0)                        # the extra planes go to the first pairs
+    if float(target).is_integer():
+        assert np.all(k == int(target))
+
+
+def _brute_force_threshold_count(scores, kmin, kmax, target):
+    """Largest high set of the form {s > v} (v = 0 or a score) whose average fits the target."""
+    n = len(scores)
+    best = 0
+    for v in [0.0] + list(scores):
+        m = sum(1 for s in scores if s > v)
+        if Fraction(kmin * n + (kmax - kmin) * m) <= Fraction(target) * n:
+            best = max(best, m)
+    return best
+
+
+@pytest.mark.parametrize("seed,target,kmin,kmax", [(0, 3.0, 2, 4), (1, 2.5, 2, 4), (2, 1.7, 1, 3), (3, 3.9, 2, 4),
+                                                   (4, 2.0, 2, 4), (5, 4.0, 2, 4), (6, 2.2, 2, 3)])
+def test_threshold_calibration_matches_brute_force(seed, target, kmin, kmax):
+    rng = np.random.default_rng(seed)
+    scores = rng.dirichlet(np.ones(8), size=6).reshape(-1)       # 48 gate-like scores in (0, 1)
+    scores[5] = scores[7]                                        # a tie
+    tau = O.calibrate_threshold(scores, kmin, kmax, target)
+    k = O.allocate_threshold(scores, tau, kmin, kmax)
+    assert Fraction(int(k.sum())) <= Fraction(target) * scores.size
+    assert int(np.count_nonzero(k == kmax)) == _brute_force_threshold_count(scores.tolist(), kmin, kmax, target)
+    if target == kmin:
+        assert np.all(k == kmin)
+    if target == kmax:
+        assert np.all(k == kmax)
+    trace = []
+    O.calibrate_threshold(scores, kmin, kmax, target, trace=trace)
+    srt = sorted(trace)
+    assert len(trace) == 64 and all(a[1] >= b[1] for a, b in zip(srt, srt[1:]))
+
+
+def test_two_plane_lagrangian_with_equal_residuals_is_a_score_threshold():
+    # with two plane counts and the same residuals for every expert, pair p reads kmax exactly
+    # when g_p (r(kmin) - r(kmax)) > lambda: a threshold on the gate. The Lagrangian allocation of
+    # a batch then equals the threshold policy calibrated on that batch's own gates.
+    rng = np.random.default_rng(12)
+    T, K, E = 16, 4, 16
+    idx = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    g = -np.sort(-rng.dirichlet(np.ones(K), size=T), axis=1)
+    r = np.tile(np.array([64.0, 16.0, 4.0, 1.0]), (E, 1))
+    for target in (2.25, 2.5, 2.8):
+        k_lag, _ = O.allocate(idx, g, r, 2, 3, target)
+        tau = O.calibrate_threshold(g, 2, 3, target)
+        assert np.array_equal(O.allocate_threshold(g, tau, 2, 3), k_lag), target
+
+
+def test_moe_forward_policies_use_their_plane_counts():
+    shape, experts, xb, wb = _mini_layer(25)
+    y_u, aux_u = O.moe_forward(xb, wb, experts, shape, 2.5, policy=O.ALLOC_UNIFORM)
+    assert aux_u["k"].reshape(-1).tolist() == O.allocate_uniform(6, 2, 4, 2.5).tolist()
+    y_t, aux_t = O.moe_forward(xb, wb, experts, shape, 3.0, policy=O.ALLOC_THRESHOLD, threshold=0.5)
+    assert np.array_equal(aux_t["k"], np.where(aux_t["gates"] > 0.5, 4, 2))
+    assert aux_t["lambda"] == 0.5
+
+
 # ----------------------------------------------------------------- FFN and combine
 
 def test_expert_ffn_hand_worked():

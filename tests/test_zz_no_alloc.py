@@ -45,6 +45,36 @@ def test_route_noalloc_matches_route_on_two_calls_in_a_row(shape, T):
         assert torch.equal(logits, ref_logits)
 
 
+@pytest.mark.parametrize("T", [128, 512])
+def test_route_noalloc_large_batches_against_oracle(T):
+    # from 128 tokens on dpa_route switches to its tiled kernels while this entry point keeps the
+    # per-logit kernel; 512 tokens x 128 experts fills its logits scratch exactly. Decisions must
+    # equal the oracle's bit for bit, and dpa_route's, on two calls in a row.
+    from oracle_jobs import route_parallel
+    shape = W.QWEN3_B64
+    fn = _noalloc_fn()
+    desc = dpa.make_desc(shape)
+    wr = torch.from_numpy(W.router_weights(shape).view(np.int16)).cuda()
+    ws = dpa.new_workspace(desc, T)
+    for step in (31, 32):
+        xb = W.tokens(shape, T, step=step)
+        x = torch.from_numpy(xb.view(np.int16)).cuda()
+        idx = torch.empty((T, shape.top_k), dtype=torch.int32, device="cuda")
+        gate = torch.empty((T, shape.top_k), dtype=torch.float64, device="cuda")
+        logits = torch.empty((T, shape.n_experts), dtype=torch.float64, device="cuda")
+        st = fn(ctypes.byref(desc), x.data_ptr(), T, wr.data_ptr(), idx.data_ptr(), gate.data_ptr(),
+                logits.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        ridx, rg, rl = route_parallel(shape, xb)
+        assert np.array_equal(logits.cpu().numpy(), rl)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        assert np.array_equal(gate.cpu().numpy(), rg)
+        ref_idx, ref_gate = dpa.route(desc, x, wr, ws)
+        assert dpa.device_status(ws) == 0
+        assert torch.equal(idx, ref_idx) and torch.equal(gate, ref_gate)
+
+
 def test_route_noalloc_rejects_sizes_beyond_its_scratch():
     fn = _noalloc_fn()
     desc = dpa.make_desc(W.QWEN3_B1)
