@@ -342,8 +342,9 @@ def run_dpa(args, shape, targets, rank, world, dist):
     P = T * K
     tc = (shape.fmt == dpa.FMT_UNIFORM and shape.hidden % 256 == 0 and shape.inter % 256 == 0 and
           P >= 16 * shape.n_experts)
-    launches_per_step = ((3 if T >= 128 else 1) + (2 if P > 2048 else 1) + (3 if tc else 2) + 1 +
-                         (2 if shape.n_shared else 0) + (1 if (not tc and T > 2) else 0))
+    # route (1, or 3 from 128 tokens), allocate (1, or 2 above 2048 pairs), the expert FFN (3: gate/up,
+    # h digits, down; or 3 on the tensor-core path: row permute, two GEMMs), combine, shared experts (2)
+    launches_per_step = ((3 if T >= 128 else 1) + (2 if P > 2048 else 1) + 3 + 1 + (2 if shape.n_shared else 0))
     for res in results:
         res.update({"tc": tc, "e2e": e2e, "launches": launches_per_step * args.steps})
     return results

@@ -29,12 +29,14 @@ NVCC_COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-
 CU_SOURCES = {
     "route.cu": ["--fmad=false"],
     "allocate.cu": ["--fmad=false"],
-    "gemv.cu": [],
+    "gemv2.cu": [],
     "gemm_tc.cu": [],
     "combine.cu": [],
     "dpa_abi.cu": [],
     "route_noalloc.cu": [],
     "stack_glue.cu": [],
+    "probe.cu": [],
+    "rates.cu": ["--fmad=false"],
 }
 CPP_SOURCES = {"encode.cpp": ["-O2", "-ffp-contract=off", "-fno-fast-math"]}
 

@@ -163,12 +163,14 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     pdl_wait();   // the routed pairs come from the previous kernel
     pdl_trigger();   // the successor may become resident now (it waits for this kernel)
     // the budget, the pairs' experts and gates are loaded together (one round trip)
-    const double target = a.policy == DPA_ALLOC_THRESHOLD ? 0.0 : *a.target;   // unused by the threshold
+    const bool budget_policy = a.policy == DPA_ALLOC_LAGRANGE || a.policy == DPA_ALLOC_UNIFORM;
+    const double target = budget_policy ? *a.target : 0.0;   // the other policies read no budget
     const double tau = a.policy == DPA_ALLOC_THRESHOLD ? *a.threshold : 0.0;
     // the budget policies need a target in [kmin, kmax]; the threshold policy a finite threshold
     int bad = a.policy == DPA_ALLOC_THRESHOLD
                   ? ((tau >= -1.0e300 && tau <= 1.0e300) ? 0 : 1)
-                  : ((target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1);
+                  : (!budget_policy || (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)))
+                        ? 0 : 1;
     if (bad && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, a.policy == DPA_ALLOC_THRESHOLD ? 12 : 10);
     int bad_e = 0;
     for (int p = tid; p < P; p += blockDim.x) {
@@ -181,6 +183,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         if (a.do_permute && tid == 0) {   // nothing downstream may read a previous call's work lists
             a.hdr->n_active = 0;
             a.hdr->n_gtiles = 0;
+            a.hdr->n_vgroups = 0;
         }
         return;
     }
@@ -196,6 +199,29 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         const int base = nb / P, rem = nb - base * P;
         for (int p = tid; p < P; p += blockDim.x) {
             const int k = base + (p < rem ? 1 : 0);
+            a.k_out[p] = static_cast<uint8_t>(k);
+            s_k[p] = static_cast<uint8_t>(k);
+        }
+        if (tid == 0 && a.lambda_out) *a.lambda_out = 0.0;
+        __syncthreads();
+        goto grouping;
+    }
+    if (a.policy == DPA_ALLOC_EXPERT_TABLE) {
+        // every pair reads its expert's rate (solved ahead of time from a workload profile)
+        int bad_k = 0;
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int k = a.expert_k[a.idx[p]];
+            bad_k |= (k < a.kmin || k > a.kmax) ? 1 : 0;
+        }
+        if (__syncthreads_or(bad_k)) {
+            if (tid == 0) {
+                set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 14);
+                if (a.do_permute) { a.hdr->n_active = 0; a.hdr->n_gtiles = 0; a.hdr->n_vgroups = 0; }
+            }
+            return;
+        }
+        for (int p = tid; p < P; p += blockDim.x) {
+            const int k = a.expert_k[a.idx[p]];
             a.k_out[p] = static_cast<uint8_t>(k);
             s_k[p] = static_cast<uint8_t>(k);
         }
@@ -612,24 +638,46 @@ grouping:
     __syncthreads();
     // per-expert descriptors and two-token tiles (tiles never straddle k classes); experts in
     // rounds of blockDim so that the active list stays in ascending expert order
-    int rank_base = 0, tile_base = 0, gt_base = 0;
+    int rank_base = 0, tile_base = 0, gt_base = 0, vt_base = 0, vg_base = 0;
+    const int vtpg = a.vtiles_per_group > 0 ? a.vtiles_per_group : 1;
     for (int e0 = 0; e0 < a.E; e0 += blockDim.x) {
         const int e = e0 + tid;
-        int km = 0, ntiles = 0, ngt = 0;
+        int km = 0, ntiles = 0, ngt = 0, nvt = 0;
         if (e < a.E) {
             for (int i = 0; i < nk; ++i) {
                 const int n = s_seg[e * nk + i + 1] - s_seg[e * nk + i];
                 if (n > 0) km = a.kmin + i;
                 ntiles += (n + 1) >> 1;
                 ngt += (n + kGemmTileTokens - 1) / kGemmTileTokens;
+                nvt += (n + 3) >> 2;
             }
         }
+        const int nvg = (nvt + vtpg - 1) / vtpg;
         const int flag = km > 0 ? 1 : 0;
         const int rank_incl = block_incl_scan(flag, s_tmp);
         const int tiles_incl = block_incl_scan(ntiles, s_tmp);
         const int gt_incl = a.gtiles ? block_incl_scan(ngt, s_tmp) : 0;
+        const int vt_incl = a.vgroups ? block_incl_scan(nvt, s_tmp) : 0;
+        const int vg_incl = a.vgroups ? block_incl_scan(nvg, s_tmp) : 0;
         const int rank = rank_base + rank_incl - flag;
         const int tile_off = tile_base + tiles_incl - ntiles;
+        if (a.vgroups && nvt > 0) {   // 4-pair tiles of one (expert, k) class, in groups of vtpg tiles
+            int t = vt_base + vt_incl - nvt, gi = vg_base + vg_incl - nvg, in_group = 0, g_first = t, g_km = 0;
+            for (int i = 0; i < nk; ++i) {
+                const int s0 = s_seg[e * nk + i];
+                const int n = s_seg[e * nk + i + 1] - s0;
+                for (int j = 0; j < n; j += 4) {
+                    a.vtiles[t++] = make_int4(a.kmin + i, s0 + j, min(4, n - j), 0);
+                    g_km = a.kmin + i;
+                    if (++in_group == vtpg) {
+                        a.vgroups[gi++] = make_int4(e, g_km, in_group, g_first);
+                        in_group = 0;
+                        g_first = t;
+                    }
+                }
+            }
+            if (in_group > 0) a.vgroups[gi++] = make_int4(e, g_km, in_group, g_first);
+        }
         if (a.gtiles && ngt > 0) {   // token tiles of the prefill GEMMs: one (expert, k) class each
             int t = gt_base + gt_incl - ngt;
             for (int i = 0; i < nk; ++i) {
@@ -656,16 +704,25 @@ grouping:
             }
         }
         // totals of this round (the last thread's inclusive sums), broadcast
-        if (tid == blockDim.x - 1) { s_tmp[0] = rank_incl; s_tmp[1] = tiles_incl; s_tmp[2] = gt_incl; }
+        if (tid == blockDim.x - 1) {
+            s_tmp[0] = rank_incl;
+            s_tmp[1] = tiles_incl;
+            s_tmp[2] = gt_incl;
+            s_tmp[3] = vt_incl;
+            s_tmp[4] = vg_incl;
+        }
         __syncthreads();
         rank_base += s_tmp[0];
         tile_base += s_tmp[1];
         gt_base += s_tmp[2];
+        vt_base += s_tmp[3];
+        vg_base += s_tmp[4];
         __syncthreads();
     }
     if (tid == 0) {
         a.hdr->n_active = static_cast<uint32_t>(rank_base);
         a.hdr->n_gtiles = static_cast<uint32_t>(gt_base);
+        a.hdr->n_vgroups = static_cast<uint32_t>(vg_base);
     }
 }
 
@@ -674,35 +731,6 @@ grouping:
 // pairs in shared memory; a round computes N(mid) for the 2^D - 1 midpoints the next D
 // steps can visit (integer sums, so the order of the additions does not matter), a bounded
 // grid barrier publishes the counts, and every thread walks the tree with the exact predicates.
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// All CTAs of the (cooperatively launched, hence co-resident) grid arrive; false on timeout.
-__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned target, WsHeader* hdr, int* s_flag) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1u);
-        bool ok = true;
-        if (ld_acquire_u32(ctr) < target) {
-            const uint64_t t0 = globaltimer();
-            while (ld_acquire_u32(ctr) < target) {
-                if (globaltimer() - t0 > kWaitNs) {
-                    set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, 0x240);
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        *s_flag = ok ? 1 : 0;
-    }
-    __syncthreads();
-    return *s_flag != 0;
-}
 
 __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a, CoopSync* cs, int per_block) {
     // this CTA's pairs [p0, p1) with their costs in shared memory; warp w evaluates the

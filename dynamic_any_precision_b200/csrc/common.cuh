@@ -18,7 +18,8 @@ struct WsHeader {
     uint32_t error_info;  // kernel-specific detail (which wait, which index)
     uint32_t n_active;    // routed experts with at least one pair in the last forward
     uint32_t n_gtiles;    // token tiles of the prefill GEMMs in the last forward (0 on the decode path)
-    uint32_t pad[60];
+    uint32_t n_vgroups;   // token groups of the pipelined expert GEMV in the last forward
+    uint32_t pad[59];
 };
 static_assert(sizeof(WsHeader) == 256, "header is one 256-byte block");
 
@@ -88,16 +89,65 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t pa
 // recording the error). The caller must not read the buffers the barrier guards then.
 // While waiting, the thread sleeps in the barrier for up to 20 us per try instead of spinning.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, WsHeader* hdr,
-                                                  uint32_t where) {
+                                                  uint32_t where, uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (!mbar_try_wait_suspend(bar, parity, 20000u)) {
-        if (globaltimer() - t0 > kWaitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
             return false;
         }
     }
     return true;
+}
+
+// The same wait for kernels whose roles end together: it also gives up as soon as another thread
+// of the CTA has set `abort` (after a timeout of its own), and a timeout sets `abort`.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                    WsHeader* hdr, uint32_t where, uint64_t limit_ns = kWaitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait_suspend(bar, parity, 10000u)) {
+        if (*abort) return false;
+        if (globaltimer() - t0 > limit_ns) {
+            set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid barrier of a cooperatively launched (hence co-resident) grid: every CTA adds one to *ctr
+// and waits until it reaches `target`; false (and DPA_ERR_DEVICE_TIMEOUT recorded) when the
+// limit runs out first. The verdict is shared with the CTA through *s_flag.
+__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned target, WsHeader* hdr, int* s_flag,
+                                             uint32_t where = 0x240, uint64_t limit_ns = kWaitNs) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        bool ok = true;
+        if (ld_acquire_u32(ctr) < target) {
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire_u32(ctr) < target) {
+                if (globaltimer() - t0 > limit_ns) {
+                    set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        *s_flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *s_flag != 0;
 }
 
 // CTA-uniform wait for a bulk-copy phase: thread 0 waits with a time limit (and on a

@@ -25,14 +25,9 @@ dpa_status check_desc(const dpa_layer_desc* d) {
     if (d->hidden % 64 || d->inter % 64 || d->group % 64 || d->group > 512) return DPA_ERR_UNSUPPORTED;
     if (d->hidden % d->group || d->inter % d->group) return DPA_ERR_UNSUPPORTED;
     if (d->hidden > 16384 || d->inter > 16384) return DPA_ERR_UNSUPPORTED;
-    // the per-CTA staging of one work item must fit in shared memory
-    dpa::GemvArgs ga{};
-    ga.H = d->hidden;
-    ga.I = d->inter;
-    ga.B = d->bits;
-    ga.G = d->group;
-    ga.fmt = d->format;
-    if (dpa::gateup_smem_bytes(ga) > dpa::kGemvMaxSmem || dpa::down_smem_bytes(ga) > dpa::kGemvMaxSmem)
+    // the staging of the expert GEMV's small-batch variant must fit in shared memory
+    if (dpa::vp_smem_bytes(d->hidden, d->group, d->format, d->bits, 2, false) > dpa::kVpMaxSmem ||
+        dpa::vp_smem_bytes(d->inter, d->group, d->format, d->bits, 1, false) > dpa::kVpMaxSmem)
         return DPA_ERR_UNSUPPORTED;
     return DPA_OK;
 }
@@ -40,7 +35,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
-        desc, tiles, gtiles, postok, coop, rstats, xperm, hdig, hexp, hsum, total;
+        desc, tiles, gtiles, postok, coop, rstats, xperm, hdig, hexp, hsum, vtiles, vgroups, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -65,9 +60,11 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.lambda = take(8);
     L.cbuf = take(8 * P * nk);
     L.pairpos = take(4 * P);
-    L.xdig = take(3 * static_cast<size_t>(T) * H);
-    L.xexp = take(4 * static_cast<size_t>(T) * (H / d->group));
-    L.xsum = take(4 * static_cast<size_t>(T) * (H / d->group));
+    const size_t ngp_h = ((H / d->group) + 3) & ~static_cast<size_t>(3);
+    const size_t ngp_i = ((I / d->group) + 3) & ~static_cast<size_t>(3);
+    L.xdig = take(2 * static_cast<size_t>(T) * H);
+    L.xexp = take(4 * static_cast<size_t>(T) * ngp_h);
+    L.xsum = take(4 * static_cast<size_t>(T) * ngp_h);
     L.h = take(4 * P * I);
     L.out_pair = take(4 * P * H);
     L.sh_h = take(4 * static_cast<size_t>(T) * d->n_shared * I);
@@ -79,9 +76,11 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.coop = take(sizeof(dpa::CoopSync));
     L.rstats = take((8 + 2 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 16);
     L.xperm = take(2 * P * H);
-    L.hdig = take(3 * P * I);
-    L.hexp = take(4 * P * (I / d->group));
-    L.hsum = take(4 * P * (I / d->group));
+    L.hdig = take(2 * P * I);
+    L.hexp = take(4 * P * ngp_i);
+    L.hsum = take(4 * P * ngp_i);
+    L.vtiles = take(16 * (P / 4 + E * nk + 1));
+    L.vgroups = take(16 * (P / 4 + E * nk + 1));
     L.total = off;
     return L;
 }
@@ -240,10 +239,12 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
                                 const double* gate, int T, const double* target, uint8_t* k_out,
                                 double* lambda_out, void* ws, const WsLayout& L, bool permute, cudaStream_t s,
                                 bool gemm_tiles = false, int policy = DPA_ALLOC_LAGRANGE,
-                                const double* threshold = nullptr) {
+                                const double* threshold = nullptr, int vtiles_per_group = 1,
+                                const uint8_t* expert_k = nullptr) {
     dpa::AllocArgs a{};
     a.policy = policy;
     a.threshold = threshold;
+    a.expert_k = expert_k;
     a.rtable = rtable;
     a.idx = idx;
     a.gate = gate;
@@ -262,7 +263,10 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.exp_desc = at<int4>(ws, L.desc);
     a.tiles = at<int4>(ws, L.tiles);
     a.gtiles = gemm_tiles ? at<int4>(ws, L.gtiles) : nullptr;
-    a.pos_tok = gemm_tiles ? at<int32_t>(ws, L.postok) : nullptr;
+    a.pos_tok = permute ? at<int32_t>(ws, L.postok) : nullptr;
+    a.vtiles = permute && !gemm_tiles ? at<int4>(ws, L.vtiles) : nullptr;
+    a.vgroups = permute && !gemm_tiles ? at<int4>(ws, L.vgroups) : nullptr;
+    a.vtiles_per_group = vtiles_per_group;
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
     return dpa::launch_allocate(a, s, at<dpa::CoopSync>(ws, L.coop), num_sms_current()) == cudaSuccess ? DPA_OK
                                                                                                   : DPA_ERR_CUDA;
@@ -272,36 +276,85 @@ static bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7
 
 // The policy and its scalar inputs: the budget policies read the target, the threshold policy
 // the threshold.
-static bool policy_inputs_ok(int policy, const double* target, const double* threshold) {
+static bool policy_inputs_ok(int policy, const double* target, const double* threshold, const uint8_t* expert_k) {
     if (policy == DPA_ALLOC_LAGRANGE || policy == DPA_ALLOC_UNIFORM) return target && aligned8(target);
     if (policy == DPA_ALLOC_THRESHOLD) return threshold && aligned8(threshold) && (!target || aligned8(target));
+    if (policy == DPA_ALLOC_EXPERT_TABLE) return expert_k != nullptr && (!target || aligned8(target));
     return false;
 }
 
 dpa_status dpa_allocate_ex(const dpa_layer_desc* d, int policy, const double* rtable, const int32_t* topk_idx,
                            const double* topk_gate, int n_tokens, const double* target_bpw, const double* threshold,
-                           uint8_t* k_out, double* lambda_out, void* ws, size_t ws_bytes, void* stream) {
+                           const uint8_t* expert_k, uint8_t* k_out, double* lambda_out, void* ws, size_t ws_bytes,
+                           void* stream) {
     const dpa_status st = check_desc(d);
     if (st != DPA_OK) return st;
     if (n_tokens <= 0 || n_tokens > 65535 || !topk_idx || !topk_gate || !k_out || !ws) return DPA_ERR_INVALID_ARG;
-    if (!policy_inputs_ok(policy, target_bpw, threshold)) return DPA_ERR_INVALID_ARG;
+    if (!policy_inputs_ok(policy, target_bpw, threshold, expert_k)) return DPA_ERR_INVALID_ARG;
     if (policy == DPA_ALLOC_LAGRANGE && !rtable) return DPA_ERR_INVALID_ARG;
     if (!aligned16(ws) || (rtable && !aligned8(rtable)) || !aligned8(topk_gate) ||
         (reinterpret_cast<uintptr_t>(topk_idx) & 3) || (lambda_out && !aligned8(lambda_out)))
         return DPA_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(d, n_tokens);
     if (ws_bytes < L.total) return DPA_ERR_WORKSPACE;
-    // the threshold policy reads no target: the threshold pointer stands in for it
-    const double* tg = target_bpw ? target_bpw : threshold;
-    return allocate_impl(d, rtable, topk_idx, topk_gate, n_tokens, tg, k_out, lambda_out, ws, L, false,
-                         static_cast<cudaStream_t>(stream), false, policy, threshold);
+    // the threshold and table policies read no target (the kernel never dereferences it then)
+    return allocate_impl(d, rtable, topk_idx, topk_gate, n_tokens, target_bpw, k_out, lambda_out, ws, L, false,
+                         static_cast<cudaStream_t>(stream), false, policy, threshold, 1, expert_k);
 }
 
 dpa_status dpa_allocate(const dpa_layer_desc* d, const double* rtable, const int32_t* topk_idx,
                         const double* topk_gate, int n_tokens, const double* target_bpw, uint8_t* k_out,
                         double* lambda_out, void* ws, size_t ws_bytes, void* stream) {
-    return dpa_allocate_ex(d, DPA_ALLOC_LAGRANGE, rtable, topk_idx, topk_gate, n_tokens, target_bpw, nullptr, k_out,
-                           lambda_out, ws, ws_bytes, stream);
+    return dpa_allocate_ex(d, DPA_ALLOC_LAGRANGE, rtable, topk_idx, topk_gate, n_tokens, target_bpw, nullptr, nullptr,
+                           k_out, lambda_out, ws, ws_bytes, stream);
+}
+
+dpa_status dpa_profile_prefill(const dpa_layer_desc* d, const void* x, int n_tokens, const int32_t* topk_idx,
+                               double* m, int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (!x || n_tokens <= 0 || n_tokens > 65535 || !topk_idx || !m || !counts || !ws) return DPA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) & 1) || (reinterpret_cast<uintptr_t>(topk_idx) & 3) || !aligned8(m) ||
+        (reinterpret_cast<uintptr_t>(counts) & 3) || !aligned16(ws))
+        return DPA_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(d, 1).total) return DPA_ERR_WORKSPACE;
+    dpa::ProfileArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.idx = topk_idx;
+    a.T = n_tokens;
+    a.H = d->hidden;
+    a.K = d->top_k;
+    a.E = d->n_experts;
+    a.m = m;
+    a.counts = counts;
+    a.hdr = at<dpa::WsHeader>(ws, 0);
+    return dpa::launch_profile(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
+}
+
+dpa_status dpa_solve_expert_rates(const dpa_layer_desc* d, const double* T, const double* m, const int32_t* counts,
+                                  const double* target_bpw, uint8_t* k_table, double* lambda_out, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (!T || !m || !counts || !target_bpw || !k_table || !ws) return DPA_ERR_INVALID_ARG;
+    if (!aligned8(T) || !aligned8(m) || (reinterpret_cast<uintptr_t>(counts) & 3) || !aligned8(target_bpw) ||
+        (lambda_out && !aligned8(lambda_out)) || !aligned16(ws))
+        return DPA_ERR_INVALID_ARG;
+    if (ws_bytes < ws_layout(d, 1).total) return DPA_ERR_WORKSPACE;
+    dpa::RatesArgs a{};
+    a.tdist = T;
+    a.m = m;
+    a.counts = counts;
+    a.target = target_bpw;
+    a.E = d->n_experts;
+    a.B = d->bits;
+    a.H = d->hidden;
+    a.kmin = d->kmin;
+    a.kmax = d->kmax;
+    a.k_table = k_table;
+    a.lambda_out = lambda_out;
+    a.hdr = at<dpa::WsHeader>(ws, 0);
+    return dpa::launch_solve_rates(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DPA_OK : DPA_ERR_CUDA;
 }
 
 dpa_status dpa_calibrate_threshold(const dpa_layer_desc* d, const double* scores, int n_scores,
@@ -350,7 +403,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     if (path < DPA_PATH_AUTO || path > DPA_PATH_TC) return DPA_ERR_INVALID_ARG;
     const int policy = aux ? aux->alloc_policy : DPA_ALLOC_LAGRANGE;
     const double* threshold = aux ? aux->threshold : nullptr;
-    if (!policy_inputs_ok(policy, target_bpw, threshold)) return DPA_ERR_INVALID_ARG;
+    const uint8_t* expert_k = aux ? aux->expert_k : nullptr;
+    if (!policy_inputs_ok(policy, target_bpw, threshold, expert_k)) return DPA_ERR_INVALID_ARG;
     const bool tc_shape = d->format == DPA_FMT_UNIFORM && d->hidden % 256 == 0 && d->inter % 256 == 0 &&
                           (d->group & (d->group - 1)) == 0;   // scale groups of 64 * 2^n inputs
     if (path == DPA_PATH_TC && !tc_shape) return DPA_ERR_UNSUPPORTED;
@@ -392,8 +446,13 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     mark(1);
 
     // 2. allocate + group pairs by (expert, k)
+    // the expert GEMV's variant: one token per expert (batch 1) runs the small-batch kernels;
+    // otherwise token groups of up to two 4-pair tiles, where their staging fits
+    const bool multi = T > 1 &&
+                       dpa::vp_smem_bytes(d->hidden, d->group, d->format, d->bits, 2, true) <= dpa::kVpMaxSmem &&
+                       dpa::vp_smem_bytes(d->inter, d->group, d->format, d->bits, 1, true) <= dpa::kVpMaxSmem;
     dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s, use_tc, policy,
-                                   threshold);
+                                   threshold, multi ? 2 : 1, expert_k);
     if (st2 != DPA_OK) return st2;
     mark(2);
 
@@ -447,42 +506,60 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
         mark(5);
         return combine_stage(d, w, gate, T, aux, y, ws, L, hdr, s, mark);
     }
-    dpa::GemvArgs ga{};
-    ga.planes = static_cast<const uint8_t*>(w->planes);
-    ga.meta = static_cast<const uint8_t*>(w->meta);
-    ga.planes_per_expert = sz.planes_per_expert;
-    ga.meta_per_expert = sz.meta_per_expert;
-    for (int m = 0; m < 3; ++m) {
-        ga.planes_mat_off[m] = sz.planes_matrix_offset[m];
-        ga.meta_mat_off[m] = sz.meta_matrix_offset[m];
-    }
-    ga.E = d->n_experts;
-    ga.H = d->hidden;
-    ga.I = d->inter;
-    ga.K = K;
-    ga.B = d->bits;
-    ga.G = d->group;
-    ga.kmin = d->kmin;
-    ga.kmax = d->kmax;
-    ga.fmt = d->format;
-    ga.exp_desc = at<int4>(ws, L.desc);
-    ga.tiles = at<int4>(ws, L.tiles);
-    ga.xdig = at<int8_t>(ws, L.xdig);
-    ga.xexp = at<int32_t>(ws, L.xexp);
-    ga.xsum = at<int32_t>(ws, L.xsum);
-    ga.h = at<float>(ws, L.h);
-    ga.out_pair = at<float>(ws, L.out_pair);
-    ga.hdig = at<int8_t>(ws, L.hdig);
-    ga.hexp = at<int32_t>(ws, L.hexp);
-    ga.hsum = at<int32_t>(ws, L.hsum);
-    ga.P = T * K;
-    ga.hdr = hdr;
     const int P = T * K;
-    ga.max_items = P < d->n_experts ? P : d->n_experts;
-    ga.max_tokens_per_expert = T;
-    if (dpa::launch_gateup(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
+    const int nk = d->kmax - d->kmin + 1;
+    dpa::VpArgs va{};
+    va.planes = static_cast<const uint8_t*>(w->planes);
+    va.meta = static_cast<const uint8_t*>(w->meta);
+    va.planes_per_expert = sz.planes_per_expert;
+    va.meta_per_expert = sz.meta_per_expert;
+    for (int m = 0; m < 3; ++m) {
+        va.planes_mat_off[m] = sz.planes_matrix_offset[m];
+        va.meta_mat_off[m] = sz.meta_matrix_offset[m];
+    }
+    va.fmt = d->format;
+    va.B = d->bits;
+    va.G = d->group;
+    va.multi = multi ? 1 : 0;
+    va.vgroups = at<int4>(ws, L.vgroups);
+    va.vtiles = at<int4>(ws, L.vtiles);
+    va.pos_tok = at<int32_t>(ws, L.postok);
+    va.hdr = hdr;
+    const int tiles_bound = P / 4 + d->n_experts * nk;
+    va.max_groups = P < tiles_bound ? P : tiles_bound;
+    // gate and up with SwiGLU: x digits by token -> h [P][I]
+    va.R = d->inter;
+    va.K = d->hidden;
+    va.mat0 = 0;
+    va.nmat = 2;
+    va.dig = at<int8_t>(ws, L.xdig);
+    va.dexp = at<int32_t>(ws, L.xexp);
+    va.dsum = at<int32_t>(ws, L.xsum);
+    va.dig_by_token = 1;
+    va.out = at<float>(ws, L.h);
+    if (dpa::launch_vp_gemv(va, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(4);
-    if (dpa::launch_down(ga, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
+    // digits of h, then down -> per-pair outputs [P][H]
+    dpa::DigitArgs da{};
+    da.x16 = nullptr;
+    da.x32 = at<float>(ws, L.h);
+    da.rows = P;
+    da.K = d->inter;
+    da.G = d->group;
+    da.dig = at<int8_t>(ws, L.hdig);
+    da.dexp = at<int32_t>(ws, L.hexp);
+    da.dsum = at<int32_t>(ws, L.hsum);
+    if (dpa::launch_digits(da, s) != cudaSuccess) return DPA_ERR_CUDA;
+    va.R = d->hidden;
+    va.K = d->inter;
+    va.mat0 = 2;
+    va.nmat = 1;
+    va.dig = at<int8_t>(ws, L.hdig);
+    va.dexp = at<int32_t>(ws, L.hexp);
+    va.dsum = at<int32_t>(ws, L.hsum);
+    va.dig_by_token = 0;
+    va.out = at<float>(ws, L.out_pair);
+    if (dpa::launch_vp_gemv(va, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(5);
     return combine_stage(d, w, gate, T, aux, y, ws, L, hdr, s, mark);
 }

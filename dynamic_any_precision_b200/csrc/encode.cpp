@@ -255,6 +255,92 @@ extern "C" dpa_status dpa_encode(const dpa_layer_desc* desc, int e_begin, int n_
     return ok.load() ? DPA_OK : DPA_ERR_INVALID_ARG;
 }
 
+namespace {
+
+// Per input channel j of expert e: T[k-1][j] = sum over the rows of gate, then of up, of
+// (w - w_k)^2 for the stored codes read at k planes (rows in order, one fp64 sum per channel).
+bool distortion_one_expert(const dpa_layer_desc& d, const dpa_sizes& sz, int e, const float* wg, const float* wu,
+                           const uint8_t* planes, const uint8_t* meta, double* T) {
+    const int H = d.hidden, I = d.inter, B = d.bits, G = d.group, ng = H / G;
+    const uint64_t plane_words = static_cast<uint64_t>(I) * H / 32;
+    std::vector<double> acc(static_cast<size_t>(B) * H, 0.0);
+    for (int m = 0; m < 2; ++m) {
+        const float* w = m == 0 ? wg : wu;
+        const uint32_t* mp = reinterpret_cast<const uint32_t*>(planes + static_cast<uint64_t>(e) * sz.planes_per_expert +
+                                                               sz.planes_matrix_offset[m]);
+        const uint16_t* mm = reinterpret_cast<const uint16_t*>(meta + static_cast<uint64_t>(e) * sz.meta_per_expert +
+                                                               sz.meta_matrix_offset[m]);
+        for (int r = 0; r < I; ++r) {
+            for (int c = 0; c < H; ++c) {
+                const dpa_layout::BitPos bp = dpa_layout::bit_position(H, r, c);
+                unsigned code = 0;
+                for (int p = 0; p < B; ++p)
+                    code |= ((mp[static_cast<uint64_t>(p) * plane_words + bp.word] >> bp.bit) & 1u) << (B - 1 - p);
+                const double wv = w[static_cast<uint64_t>(r) * H + c];
+                for (int k = 1; k <= B; ++k) {
+                    double what;
+                    if (d.format == DPA_FMT_UNIFORM) {
+                        const double s = f16_bits_to_f64(mm[(static_cast<uint64_t>(r) * ng + c / G) * 2]);
+                        const double z = f16_bits_to_f64(mm[(static_cast<uint64_t>(r) * ng + c / G) * 2 + 1]);
+                        const int dsh = B - k;
+                        const double qk = static_cast<double>(code >> dsh);
+                        const double pw = static_cast<double>(1u << dsh);
+                        what = s * ((qk * pw + (pw - 1.0) / 2.0) - z);
+                    } else {
+                        what = 0.0;
+                        for (int i = 0; i < k; ++i) {
+                            const double a = f16_bits_to_f64(
+                                mm[static_cast<uint64_t>(i) * I * ng + static_cast<uint64_t>(r) * ng + c / G]);
+                            what = what + a * (((code >> (B - 1 - i)) & 1u) ? 1.0 : -1.0);
+                        }
+                    }
+                    const double diff = wv - what;
+                    acc[static_cast<size_t>(k - 1) * H + c] = acc[static_cast<size_t>(k - 1) * H + c] + diff * diff;
+                }
+            }
+        }
+    }
+    for (size_t i = 0; i < acc.size(); ++i) T[i] = acc[i];
+    return true;
+}
+
+}  // namespace
+
+extern "C" dpa_status dpa_distortion_tensor(const dpa_layer_desc* desc, int e_begin, int n_e, const float* w_gate,
+                                            const float* w_up, const void* planes, const void* meta, double* T,
+                                            int n_threads) {
+    dpa_sizes sz;
+    dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!w_gate || !w_up || !planes || !meta || !T) return DPA_ERR_INVALID_ARG;
+    if (e_begin < 0 || n_e < 0 || e_begin + n_e > desc->n_experts) return DPA_ERR_INVALID_ARG;
+    if (n_e == 0) return DPA_OK;
+    const uint64_t per = static_cast<uint64_t>(desc->inter) * desc->hidden;
+    const uint64_t tper = static_cast<uint64_t>(desc->bits) * desc->hidden;
+    unsigned hw = std::thread::hardware_concurrency();
+    int nt = n_threads > 0 ? n_threads : static_cast<int>(hw ? hw : 1);
+    nt = std::min(nt, n_e);
+    std::atomic<int> next{0};
+    auto worker = [&]() {
+        for (;;) {
+            const int i = next.fetch_add(1);
+            if (i >= n_e) break;
+            const int e = e_begin + i;
+            distortion_one_expert(*desc, sz, e, w_gate + i * per, w_up + i * per, static_cast<const uint8_t*>(planes),
+                                  static_cast<const uint8_t*>(meta), T + static_cast<uint64_t>(e) * tper);
+        }
+    };
+    if (nt <= 1) {
+        worker();
+    } else {
+        std::vector<std::thread> th;
+        th.reserve(nt);
+        for (int t = 0; t < nt; ++t) th.emplace_back(worker);
+        for (auto& t : th) t.join();
+    }
+    return DPA_OK;
+}
+
 extern "C" dpa_status dpa_export_codes(const dpa_layer_desc* desc, const void* planes, int expert,
                                        int matrix, uint8_t* codes) {
     dpa_sizes sz;

@@ -16,9 +16,9 @@ struct RouteArgs {
     int32_t* idx;             // [T][K]
     double* gate;             // [T][K]
     unsigned* counters;       // [T] zero between calls
-    int8_t* xdig;             // [T][3][H] or nullptr (digits not needed)
-    int32_t* xexp;            // [T][H/G]
-    int32_t* xsum;            // [T][H/G]
+    int8_t* xdig;             // [T][2][H] activation digits for the expert GEMV, or nullptr
+    int32_t* xexp;            // [T][ngp] group exponents (ngp = H/G rounded up to 4)
+    int32_t* xsum;            // [T][ngp] group sums
     WsHeader* hdr;
     int wpe;                  // warps per expert (set by the launcher)
     // large-batch path (nullptr: always the per-logit kernel): per-row exactness statistics
@@ -49,6 +49,13 @@ struct AllocArgs {
     WsHeader* hdr;
     int policy;               // DPA_ALLOC_LAGRANGE, DPA_ALLOC_UNIFORM or DPA_ALLOC_THRESHOLD
     const double* threshold;  // device scalar (DPA_ALLOC_THRESHOLD)
+    // work list of the pipelined expert GEMV (nullptr: not written): tiles of up to 4 pairs of
+    // one (expert, k) class, {k, pos0, n, 0}, and token groups of up to vtiles_per_group tiles of
+    // one expert, {expert, kmax over the group, n tiles, first tile}; count in hdr->n_vgroups
+    int4* vtiles;             // [P/4 + E*nk]
+    int4* vgroups;            // [P/4 + E*nk]
+    int vtiles_per_group;
+    const uint8_t* expert_k;  // [E] plane count per expert (DPA_ALLOC_EXPERT_TABLE)
 };
 // Counters of the grid-wide bisection (zeroed by the launcher before every call).
 constexpr int kCoopRoundsMax = 16;
@@ -73,6 +80,29 @@ struct CalibArgs {
 };
 cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t stream);
 
+// Workload profile of a prefill and the per-expert read rates solved from it.
+struct ProfileArgs {
+    const uint16_t* x;        // [T][H] bf16 prefill activations
+    const int32_t* idx;       // [T][K] routed experts
+    int T, H, K, E;
+    double* m;                // [H] mean square per input channel
+    int32_t* counts;          // [E] routed pairs per expert
+    WsHeader* hdr;
+};
+cudaError_t launch_profile(const ProfileArgs& a, cudaStream_t stream);
+struct RatesArgs {
+    const double* tdist;      // [E][B][H] distortion tensor
+    const double* m;          // [H]
+    const int32_t* counts;    // [E]
+    const double* target;     // device scalar
+    int E, B, H, kmin, kmax;
+    uint8_t* k_table;         // [E]
+    double* lambda_out;       // scalar or nullptr
+    WsHeader* hdr;
+};
+cudaError_t launch_solve_rates(const RatesArgs& a, cudaStream_t stream);
+size_t rates_smem_bytes(int E, int nk);
+
 // Prefill expert FFN on tcgen05: grouped GEMMs over the GEMM token tiles of the allocation.
 struct GemmArgs {
     const uint8_t* planes;    // encoded layer (uniform format)
@@ -95,35 +125,47 @@ cudaError_t launch_gemm_gateup(const GemmArgs& a, cudaStream_t stream, int sms);
 cudaError_t launch_gemm_down(const GemmArgs& a, cudaStream_t stream, int sms);
 size_t gemm_tc_smem_bytes();
 
-struct GemvArgs {
+// Pipelined variable-plane expert GEMV (decode batches): one launch computes either gate and up
+// with the SwiGLU epilogue (nmat = 2: out = h [P][R], R = inter) or down (nmat = 1: out =
+// per-pair outputs [P][R], R = hidden) for every (token group, row block) item.
+struct VpArgs {
     const uint8_t* planes;    // encoded layer
     const uint8_t* meta;
     uint64_t planes_per_expert, meta_per_expert;
     uint64_t planes_mat_off[3], meta_mat_off[3];
-    int E, H, I, K, B, G, kmin, kmax, fmt;
-    const int4* exp_desc;     // per active expert [2]: {expert, kmax, n_tiles, first tile}, first tile
-    const int4* tiles;        // {k, posA, posB, tokA | tokB << 16}
-    const int8_t* xdig;       // [T][3][H]
-    const int32_t* xexp;      // [T][H/G]
-    const int32_t* xsum;      // [T][H/G]
-    float* h;                 // [P][I] by sorted position
-    float* out_pair;          // [P][H] by sorted position
-    int8_t* hdig;             // [P][3][I] digits of h (multi-token down kernel)
-    int32_t* hexp;            // [P][I/G]
-    int32_t* hsum;            // [P][I/G]
-    int P;                    // routed pairs
+    int fmt, B, G;
+    int R, K;                 // rows and columns of each matrix of this launch
+    int mat0, nmat;           // first matrix (0: gate, up; 2: down) and the matrix count
+    int multi;                // 1: 64-row items, groups of up to 4 tiles; 0: the small-batch variant
+    const int4* vgroups;      // {expert, kmax, n tiles, first tile}, count in hdr->n_vgroups
+    const int4* vtiles;       // {k, pos0, n, 0}
+    const int32_t* pos_tok;   // [P] token of each grouped position
+    const int8_t* dig;        // activation digit rows [rows][2][K] (permuted 64-column blocks)
+    const int32_t* dexp;      // [rows][ngp] group exponents
+    const int32_t* dsum;      // [rows][ngp] group sums of the fixed-point values
+    int dig_by_token;         // 1: the digit row of a pair is its token (x); 0: its position (h)
+    float* out;               // [P][R] by grouped position
     WsHeader* hdr;
-    int max_items;            // upper bound of active experts (host-known)
-    int max_tokens_per_expert;  // host-known bound (selects the tile count per pass)
+    int max_groups;           // host bound of the token groups
 };
-cudaError_t launch_gateup(const GemvArgs& a, cudaStream_t stream, int num_sms);
-// Dynamic shared memory a GEMV work item may stage. The single-pass (one- and two-token)
-// kernels must fit for a layer to be accepted; the multi-token kernels run only where they fit
-// too, the single-pass ones (one tile per pass) elsewhere.
-constexpr size_t kGemvMaxSmem = 200 * 1024;
-size_t gateup_smem_bytes(const GemvArgs& a);   // one CTA of the single-pass gate/up kernel
-size_t down_smem_bytes(const GemvArgs& a);     // one CTA of the single-pass down kernel
-cudaError_t launch_down(const GemvArgs& a, cudaStream_t stream, int num_sms);
+cudaError_t launch_vp_gemv(const VpArgs& a, cudaStream_t stream, int sms);
+// dynamic shared memory of one CTA of a variant (multi: 64-row items, small: the other)
+size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, bool multi);
+constexpr size_t kVpMaxSmem = 227 * 1024;
+
+// Fixed-point digits of activation rows (x as bf16, or h as fp32), per group of G columns:
+// X = rint(v * 2^(14 - E)) with |v| < 2^E, as digits d0 + 256 d1 in rows [rows][2][K] with each
+// 64-column block permuted for the B operand; exponents and sums [rows][ngp], ngp = K/G rounded
+// up to a multiple of 4.
+struct DigitArgs {
+    const uint16_t* x16;      // bf16 rows or nullptr
+    const float* x32;         // fp32 rows (when x16 is nullptr)
+    int rows, K, G;
+    int8_t* dig;
+    int32_t* dexp;
+    int32_t* dsum;
+};
+cudaError_t launch_digits(const DigitArgs& d, cudaStream_t stream);
 
 struct CombineArgs {
     const float* out_pair;    // [P][H] by sorted position

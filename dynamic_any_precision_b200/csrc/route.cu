@@ -192,9 +192,13 @@ __device__ double exact_dot_warp(const uint16_t* x, const uint16_t* w, int H, in
 }
 
 // Fixed-point digits of token t for the expert GEMV: groups g = g0, g0 + gstep, ... handled by
-// this warp; xs is the token's bf16 row (shared or global memory).
+// this warp; xs is the token's bf16 row (shared or global memory). Per group of G inputs,
+// X = rint(x * 2^(14 - E)) with |x| < 2^E, stored as digits d0 + 256 d1 in rows [T][2][H] whose
+// 64-column blocks are permuted (column c at byte 16*((c%16)/4) + 4*(c/16) + c%4) so that one
+// 16-byte load gives an MMA lane its B-operand words; exponents and sums [T][ngp], ngp = H/G
+// rounded up to a multiple of 4.
 __device__ void token_digits(const RouteArgs& a, int t, const uint16_t* xs, int g0, int gstep) {
-    const int H = a.H, G = a.G, ng = H / G, lane = threadIdx.x & 31;
+    const int H = a.H, G = a.G, ng = H / G, ngp = (ng + 3) & ~3, lane = threadIdx.x & 31;
     for (int g = g0; g < ng; g += gstep) {
         float mx = 0.f;
         for (int j = lane; j < G; j += 32) mx = fmaxf(mx, fabsf(bf16_bits_to_float(xs[g * G + j])));
@@ -202,19 +206,20 @@ __device__ void token_digits(const RouteArgs& a, int t, const uint16_t* xs, int 
         const int Eg = group_exponent(mx);
         int sum = 0;
         for (int j = lane; j < G; j += 32) {
-            const int X = to_fixed(bf16_bits_to_float(xs[g * G + j]), Eg);
+            const int c = g * G + j;
+            const int X = __float2int_rn(ldexpf(bf16_bits_to_float(xs[c]), 14 - Eg));
             sum += X;
-            int8_t d0, d1, d2;
-            split_digits(X, d0, d1, d2);
-            const size_t base = static_cast<size_t>(t) * 3 * H + g * G + j;
-            a.xdig[base] = d0;
-            a.xdig[base + H] = d1;
-            a.xdig[base + 2 * H] = d2;
+            const int lo = ((X + 128) & 255) - 128;
+            const int hi = (X - lo) >> 8;
+            const int cb = c & 63;
+            const size_t off = static_cast<size_t>(t) * 2 * H + (c & ~63) + 16 * ((cb & 15) >> 2) + 4 * (cb >> 4) + (cb & 3);
+            a.xdig[off] = static_cast<int8_t>(lo);
+            a.xdig[off + H] = static_cast<int8_t>(hi);
         }
         sum = warp_sum_i(sum);
         if (lane == 0) {
-            a.xexp[t * ng + g] = Eg;
-            a.xsum[t * ng + g] = sum;
+            a.xexp[t * ngp + g] = Eg;
+            a.xsum[t * ngp + g] = sum;
         }
     }
 }

@@ -52,15 +52,16 @@ class Aux(ctypes.Structure):
     _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_gate", ctypes.c_void_p), ("k", ctypes.c_void_p),
                 ("lambda_", ctypes.c_void_p), ("pair_out", ctypes.c_void_p),
                 ("events", ctypes.c_void_p * 7), ("expert_path", ctypes.c_int32),
-                ("alloc_policy", ctypes.c_int32), ("threshold", ctypes.c_void_p)]
+                ("alloc_policy", ctypes.c_int32), ("threshold", ctypes.c_void_p), ("expert_k", ctypes.c_void_p)]
 
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
-ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD = 0, 1, 2
+ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD, ALLOC_EXPERT_TABLE = 0, 1, 2, 3
 
 
 EXPORTED = ("dpa_encoded_sizes", "dpa_encode", "dpa_export_codes", "dpa_export_meta", "dpa_route",
             "dpa_allocate", "dpa_allocate_ex", "dpa_calibrate_threshold", "dpa_forward_workspace_size",
-            "dpa_moe_forward", "dpa_device_status", "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm")
+            "dpa_moe_forward", "dpa_device_status", "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm",
+            "dpa_debug_timeout_probe", "dpa_distortion_tensor", "dpa_profile_prefill", "dpa_solve_expert_rates")
 
 _lib = None
 
@@ -82,12 +83,16 @@ def lib() -> ctypes.CDLL:
     L.dpa_export_meta.argtypes = [P(LayerDesc), vp, i32, i32, vp, vp]
     L.dpa_route.argtypes = [P(LayerDesc), vp, i32, vp, vp, vp, vp, vp, sz, vp]
     L.dpa_allocate.argtypes = [P(LayerDesc), vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]
-    L.dpa_allocate_ex.argtypes = [P(LayerDesc), i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.dpa_allocate_ex.argtypes = [P(LayerDesc), i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.dpa_distortion_tensor.argtypes = [P(LayerDesc), i32, i32, vp, vp, vp, vp, vp, i32]
+    L.dpa_profile_prefill.argtypes = [P(LayerDesc), vp, i32, vp, vp, vp, vp, sz, vp]
+    L.dpa_solve_expert_rates.argtypes = [P(LayerDesc), vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.dpa_calibrate_threshold.argtypes = [P(LayerDesc), vp, i32, vp, vp, vp, sz, vp]
     L.dpa_forward_workspace_size.argtypes = [P(LayerDesc), i32]
     L.dpa_forward_workspace_size.restype = sz
     L.dpa_moe_forward.argtypes = [P(LayerDesc), P(LayerWeights), vp, i32, vp, vp, P(Aux), vp, sz, vp]
     L.dpa_device_status.argtypes = [vp, vp]
+    L.dpa_debug_timeout_probe.argtypes = [vp, sz, i32, ctypes.c_uint64, vp]
     L.dpa_residual_rmsnorm.argtypes = [vp, vp, i32, i32, vp, vp]
     L.dpa_status_string.argtypes = [i32]
     L.dpa_status_string.restype = ctypes.c_char_p
@@ -208,9 +213,10 @@ def route(desc: LayerDesc, x, w_router, ws, logits=None, stream=None):
 
 
 def allocate(desc: LayerDesc, rtable, idx, gate, target, ws, stream=None, policy: int = ALLOC_LAGRANGE,
-             threshold=None):
-    """target: CUDA fp64 scalar tensor (None for the threshold policy); threshold: CUDA fp64
-    scalar tensor (threshold policy). Returns (k uint8 [T][K], lambda fp64 [1])."""
+             threshold=None, expert_k=None):
+    """target: CUDA fp64 scalar tensor (None for the threshold and table policies); threshold:
+    CUDA fp64 scalar tensor (threshold policy); expert_k: CUDA uint8 [E] (table policy).
+    Returns (k uint8 [T][K], lambda fp64 [1])."""
     import torch
     T = idx.shape[0]
     k = torch.empty((T, desc.top_k), dtype=torch.uint8, device=idx.device)
@@ -220,9 +226,42 @@ def allocate(desc: LayerDesc, rtable, idx, gate, target, ws, stream=None, policy
                                   _dptr(k), _dptr(lam), _dptr(ws), ws.numel(), _stream(stream)), "dpa_allocate")
     else:
         _check(lib().dpa_allocate_ex(ctypes.byref(desc), policy, _dptr(rtable), _dptr(idx), _dptr(gate), T,
-                                     _dptr(target), _dptr(threshold), _dptr(k), _dptr(lam), _dptr(ws), ws.numel(),
-                                     _stream(stream)), "dpa_allocate_ex")
+                                     _dptr(target), _dptr(threshold), _dptr(expert_k), _dptr(k), _dptr(lam),
+                                     _dptr(ws), ws.numel(), _stream(stream)), "dpa_allocate_ex")
     return k, lam
+
+
+def distortion_tensor(desc: LayerDesc, w_gate: np.ndarray, w_up: np.ndarray, planes: np.ndarray, meta: np.ndarray,
+                      e_begin: int = 0, out: Optional[np.ndarray] = None, n_threads: int = 0) -> np.ndarray:
+    """Host distortion tensor [E][B][H] fp64 for experts [e_begin, e_begin + n) of the layer."""
+    T = np.zeros((desc.n_experts, desc.bits, desc.hidden), np.float64) if out is None else out
+    wg = np.ascontiguousarray(w_gate, np.float32)
+    wu = np.ascontiguousarray(w_up, np.float32)
+    n = wg.shape[0] if wg.ndim == 3 else 1
+    _check(lib().dpa_distortion_tensor(ctypes.byref(desc), e_begin, n, _ptr(wg), _ptr(wu), _ptr(planes), _ptr(meta),
+                                       _ptr(T), n_threads), "dpa_distortion_tensor")
+    return T
+
+
+def profile_prefill(desc: LayerDesc, x, idx, ws, stream=None):
+    """x: CUDA bf16 bits [T][H]; idx: CUDA int32 [T][K]. Returns (m fp64 [H], counts int32 [E])."""
+    import torch
+    m = torch.empty(desc.hidden, dtype=torch.float64, device=x.device)
+    counts = torch.empty(desc.n_experts, dtype=torch.int32, device=x.device)
+    _check(lib().dpa_profile_prefill(ctypes.byref(desc), _dptr(x), x.shape[0], _dptr(idx), _dptr(m), _dptr(counts),
+                                     _dptr(ws), ws.numel(), _stream(stream)), "dpa_profile_prefill")
+    return m, counts
+
+
+def solve_expert_rates(desc: LayerDesc, tdist, m, counts, target, ws, stream=None):
+    """tdist: CUDA fp64 [E][B][H]. Returns (k_table uint8 [E], lambda fp64 [1])."""
+    import torch
+    kt = torch.empty(desc.n_experts, dtype=torch.uint8, device=m.device)
+    lam = torch.empty(1, dtype=torch.float64, device=m.device)
+    _check(lib().dpa_solve_expert_rates(ctypes.byref(desc), _dptr(tdist), _dptr(m), _dptr(counts), _dptr(target),
+                                        _dptr(kt), _dptr(lam), _dptr(ws), ws.numel(), _stream(stream)),
+           "dpa_solve_expert_rates")
+    return kt, lam
 
 
 def calibrate_threshold(desc: LayerDesc, scores, target, ws, stream=None):
@@ -282,6 +321,7 @@ def moe_forward(layer: DeviceLayer, x, target, ws, y=None, aux: Optional[dict] =
         aux_s.expert_path = int(aux.get("expert_path", PATH_AUTO))
         aux_s.alloc_policy = int(aux.get("alloc_policy", ALLOC_LAGRANGE))
         aux_s.threshold = _dptr(aux.get("threshold"))
+        aux_s.expert_k = _dptr(aux.get("expert_k"))
     _check(lib().dpa_moe_forward(ctypes.byref(layer.desc), ctypes.byref(layer.weights), _dptr(x), T, _dptr(target),
                                  _dptr(y), ctypes.byref(aux_s) if aux_s is not None else None, _dptr(ws), ws.numel(),
                                  _stream(stream)), "dpa_moe_forward")

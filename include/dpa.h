@@ -137,8 +137,9 @@ typedef struct dpa_layer_weights {
 #define DPA_PATH_TC 2
 #define DPA_TC_MIN_PAIRS_PER_EXPERT 16
 /* alloc_policy: how the routed pairs' plane counts are chosen (see dpa_allocate_ex); threshold:
- * device fp64 scalar read by DPA_ALLOC_THRESHOLD (NULL otherwise). With alloc_policy = 0 the
- * Lagrangian allocation of dpa_allocate runs. */
+ * device fp64 scalar read by DPA_ALLOC_THRESHOLD (NULL otherwise); expert_k: device uint8 [E]
+ * read by DPA_ALLOC_EXPERT_TABLE (NULL otherwise). With alloc_policy = 0 the Lagrangian
+ * allocation of dpa_allocate runs. */
 typedef struct dpa_aux {
     int32_t* topk_idx;
     double* topk_gate;
@@ -149,6 +150,7 @@ typedef struct dpa_aux {
     int32_t expert_path;
     int32_t alloc_policy;
     const double* threshold;
+    const uint8_t* expert_k;
 } dpa_aux;
 
 /* Validate a descriptor and return the encoded sizes. Host only. */
@@ -227,19 +229,64 @@ dpa_status dpa_allocate(const dpa_layer_desc* desc, const double* rtable,
  *                          gate) is above a threshold reads kmax planes, every other pair kmin.
  *                          The threshold comes from dpa_calibrate_threshold ahead of time; no
  *                          budget is enforced on the live batch. target_bpw is not read (may be
- *                          NULL). lambda_out = the threshold. */
+ *                          NULL). lambda_out = the threshold.
+ *  DPA_ALLOC_EXPERT_TABLE (3) DuoRate, Abstract: every pair routed to expert e reads expert_k[e]
+ *                          planes, a per-workload table solved ahead of time by
+ *                          dpa_solve_expert_rates. target_bpw is not read (may be NULL).
+ *                          lambda_out = 0. */
 #define DPA_ALLOC_LAGRANGE 0
 #define DPA_ALLOC_UNIFORM 1
 #define DPA_ALLOC_THRESHOLD 2
+#define DPA_ALLOC_EXPERT_TABLE 3
 
 /* dpa_allocate with a choice of policy (device). Arguments as dpa_allocate, plus
- * policy (above) and threshold: device fp64 scalar, read by DPA_ALLOC_THRESHOLD only (a NaN or
- * infinite threshold sets the device flag DPA_ERR_DEVICE_INVALID_INPUT and leaves k untouched).
- * Errors: DPA_ERR_INVALID_ARG for an unknown policy or a missing threshold. */
+ * policy (above); threshold: device fp64 scalar, read by DPA_ALLOC_THRESHOLD only (a NaN or
+ * infinite threshold sets the device flag DPA_ERR_DEVICE_INVALID_INPUT and leaves k untouched);
+ * expert_k: device uint8 [n_experts], read by DPA_ALLOC_EXPERT_TABLE only (an entry outside
+ * [kmin, kmax] for a routed expert sets the same flag). rtable is read by DPA_ALLOC_LAGRANGE only.
+ * Errors: DPA_ERR_INVALID_ARG for an unknown policy or a missing input of the policy. */
 dpa_status dpa_allocate_ex(const dpa_layer_desc* desc, int policy, const double* rtable,
                            const int32_t* topk_idx, const double* topk_gate, int n_tokens,
-                           const double* target_bpw, const double* threshold, uint8_t* k_out,
-                           double* lambda_out, void* ws, size_t ws_bytes, void* stream);
+                           const double* target_bpw, const double* threshold, const uint8_t* expert_k,
+                           uint8_t* k_out, double* lambda_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Distortion tensor of the workload-profiled read rates (host, synchronous). Defined by:
+ * DuoRate, Abstract (a distortion tensor baked offline beside the stored weights). For routed
+ * experts [e_begin, e_begin + n_e): T[e][k-1][j] = sum over the rows of gate, then of up, of
+ * (w - w_k)^2 at input channel j, w_k the stored code read at k planes (one sequential fp64 sum
+ * per channel, rows in order). w_gate, w_up: host fp32 [n_e][inter][hidden] (the experts'
+ * original weights); planes, meta: the host output of dpa_encode for the whole layer;
+ * T: host fp64 [n_experts][bits][hidden] (only the given experts' parts are written).
+ * n_threads >= 1, or 0 for all cores. */
+dpa_status dpa_distortion_tensor(const dpa_layer_desc* desc, int e_begin, int n_e, const float* w_gate,
+                                 const float* w_up, const void* planes, const void* meta, double* T,
+                                 int n_threads);
+
+/* Workload profile of a prefill (device). Defined by: DuoRate, Abstract (the workload's own
+ * prefill is profiled, without labels). m[j] = (sum over tokens in order of x[t][j]^2) / T in
+ * fp64; counts[e] = pairs of topk_idx routed to e. x: device bf16 [n_tokens][hidden];
+ * topk_idx: device int32 [n_tokens][top_k] (dpa_route's output); m: device fp64 [hidden];
+ * counts: device int32 [n_experts] (overwritten). An out-of-range expert id sets the device
+ * flag DPA_ERR_DEVICE_INVALID_INPUT. ws: at least dpa_forward_workspace_size(desc, 1) bytes. */
+dpa_status dpa_profile_prefill(const dpa_layer_desc* desc, const void* x, int n_tokens,
+                               const int32_t* topk_idx, double* m, int32_t* counts, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Per-expert decode read rates from a workload profile (device). Defined by: DuoRate, Abstract
+ * (a Lagrangian rate/distortion allocation under the decode functional, one dot product per
+ * expert and a bisection; routing frequency cancels from each expert's decision).
+ * D_e(k) = <m, T[e][k-1]> summed as 32 chunks of hidden/32 channels (each sequential) combined
+ * by the pairwise tree p[i]+p[i+16], +[i+8], +[i+4], +[i+2], +[i+1];
+ * k_e(lambda) = argmin_{kmin<=k<=kmax} fl(D_e(k) + fl(lambda*k)), ties to the smaller k;
+ * 64 fp64 bisection steps on [0, 2 max_e D_e(kmin) + 1]: if sum_e counts[e]*k_e(mid) >
+ * target*sum_e counts[e] then lo = mid else hi = mid; k_table[e] = k_e(hi) for every expert.
+ * T: device fp64 [n_experts][bits][hidden]; m, counts as from dpa_profile_prefill;
+ * target_bpw: device fp64 scalar in [kmin, kmax] (else the device flag
+ * DPA_ERR_DEVICE_INVALID_INPUT, table untouched); k_table: device uint8 [n_experts];
+ * lambda_out: device fp64 scalar or NULL. ws: at least dpa_forward_workspace_size(desc, 1). */
+dpa_status dpa_solve_expert_rates(const dpa_layer_desc* desc, const double* T, const double* m,
+                                  const int32_t* counts, const double* target_bpw, uint8_t* k_table,
+                                  double* lambda_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Threshold of DPA_ALLOC_THRESHOLD from a calibration set of routing scores (device).
  * Defined by: MatMoE, review "Core Contribution" (a binary search over a calibration score
@@ -306,6 +353,18 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* desc, const dpa_layer_weights* 
  * The pages give no form for the glue; this is the plainest reading of a residual add and an
  * RMSNorm (unit weight) between the layers. */
 dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidden, void* x, void* stream);
+
+/* Test support for the device-side failure handling (the pages have no counterpart).
+ * Runs one of the library's bounded device waits against a barrier that nothing completes,
+ * with a limit of limit_ns (1e3 .. 2e9 ns) instead of the kernels' 200 ms:
+ *   kind 0  the mbarrier wait of the bulk-copy and tensor-core pipelines;
+ *   kind 1  the abortable wait of the expert GEMV (one warp times out, the others leave on the
+ *           CTA's abort flag);
+ *   kind 2  the grid barrier of the cooperative allocation, one of two CTAs held back.
+ * The kernel returns after the limit and records DPA_ERR_DEVICE_TIMEOUT in ws's device flag
+ * (read it with dpa_device_status); nothing else is written except, for kind 2, a counter at
+ * byte 256 of ws. ws: device, 16-byte aligned, at least 512 bytes. */
+dpa_status dpa_debug_timeout_probe(void* ws, size_t ws_bytes, int kind, uint64_t limit_ns, void* stream);
 
 /* Synchronise `stream`, read the device error flag in ws, clear it, and return it
  * (DPA_OK if no device error was recorded). */

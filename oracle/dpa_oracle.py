@@ -40,6 +40,12 @@ Parity status of each function (what pins it; see tests/test_oracle_pins.py):
   calibrate_threshold pinned: brute force over the cut points of the score distribution;
   / allocate_threshold endpoints; two plane counts and equal residuals reduce the Lagrangian
                       allocation of a batch to the threshold calibrated on that batch
+  distortion_tensor   pinned: channel sums equal the gate+up residual (exact rational, small)
+  prefill_profile     pinned: exact rational mean squares; counts by brute force
+  tree_dot            pinned: within a few ulps of the exact rational dot product; order check
+  solve_expert_rates  pinned: brute-force count-weighted optimum (Everett) on tiny inputs;
+                      frequency cancels (scaling counts leaves every k(lambda) unchanged);
+                      endpoint targets; monotone plane count along the bisection
   expert_ffn / moe    pinned: hand-worked tiny layer; top-1 identity; linearity of the
                       gate-weighted combine; prefix property (low bits ignored); at
                       target = kmax = B the layer equals a torch fp32 computation (topk,
@@ -419,6 +425,107 @@ def allocate_threshold(gates: np.ndarray, threshold: float, kmin: int, kmax: int
 
 
 # ---------------------------------------------------------------------------
+# Workload-profiled per-expert read rates ([DUO] Abstract: one uniform tier of a prefix-readable
+# stream is stored with a baked distortion tensor; online, the workload's own prefill is profiled
+# without labels and a Lagrangian rate-distortion allocation is solved under the decode
+# functional; routing frequency cancels from every per-expert decision; the solve is one dot
+# product per expert and a bisection; prefill reads at the stored rate, decode at the workload's).
+# Readings:
+#   distortion tensor  T[e][k-1][j] = sum over the rows i of the gate and up projections of
+#                      (W - W_hat^(k))[i][j]^2: the squared reconstruction error that input
+#                      channel j meets at k planes (the down projection's input is internal to
+#                      the expert and is not profiled);
+#   profile            m[j] = (sum over the prefill tokens, in token order, of x[t][j]^2) / T and
+#                      c[e] = the number of prefill pairs routed to expert e;
+#   distortion         D_e(k) = <m, T[e][k-1]>, summed as 32 chunks of H/32 consecutive channels
+#                      (each sequential from 0) combined by the pairwise tree
+#                      p[i] + p[i+16], then + [i+8], + [i+4], + [i+2], + [i+1];
+#   decode functional  expected planes read per selected expert: sum_e c_e k_e / sum_e c_e;
+#   decision           k_e(lambda) = argmin_k fl(D_e(k) + fl(lambda * k)), ties to the smaller k:
+#                      the objective sum_e c_e (D_e(k_e) + lambda k_e) separates per expert and
+#                      c_e > 0 drops out of each argmin;
+#   bisection          64 steps on [0, 2 max_e D_e(kmin) + 1]: if sum_e c_e k_e(mid) >
+#                      target * sum_e c_e then lo = mid else hi = mid; lambda = hi. Experts the
+#                      prefill never routed to get k_e(hi) too (they may be selected in decode).
+# In decode every pair routed to e then reads k_e planes (the expert-rate table).
+# ---------------------------------------------------------------------------
+
+
+def distortion_tensor(enc: Dict, fmt: int, B: int, G: int, gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """T [B][H]: per input channel, the squared error of gate and up at k = 1..B planes."""
+    H = gate.shape[1]
+    out = np.zeros((B, H), dtype=np.float64)
+    for k in range(1, B + 1):
+        wg, wu, _ = dequant_expert(enc, fmt, B, k, G)
+        dg = gate.astype(np.float64) - wg
+        du = up.astype(np.float64) - wu
+        for j in range(H):   # rows in order, gate then up, one sequential sum per channel
+            col = np.concatenate([dg[:, j], du[:, j]])
+            out[k - 1, j] = float(np.cumsum(col * col)[-1])
+    return out
+
+
+def prefill_profile(x_bits: np.ndarray, idx: np.ndarray, n_experts: int):
+    """m [H] (mean square of each input channel over the prefill tokens) and c [E] (pair counts)."""
+    x = bf16_bits_to_f64(x_bits)
+    T, H = x.shape
+    m = np.empty(H, dtype=np.float64)
+    for j in range(H):
+        acc = 0.0
+        for t in range(T):
+            acc = acc + x[t, j] * x[t, j]
+        m[j] = acc / float(T)
+    c = np.bincount(np.asarray(idx).reshape(-1), minlength=n_experts).astype(np.int64)
+    return m, c
+
+
+def tree_dot(m: np.ndarray, t: np.ndarray) -> float:
+    """<m, t> in the fixed order above: 32 sequential chunk sums, then the pairwise tree."""
+    H = m.size
+    step = H // 32
+    part = []
+    for c in range(32):
+        acc = 0.0
+        for j in range(c * step, (c + 1) * step):
+            acc = acc + float(m[j]) * float(t[j])
+        part.append(acc)
+    width = 16
+    while width >= 1:
+        part = [part[i] + part[i + width] for i in range(width)]
+        width //= 2
+    return part[0]
+
+
+def solve_expert_rates(Tdist: np.ndarray, m: np.ndarray, counts: np.ndarray, kmin: int, kmax: int,
+                       target: float, iters: int = 64):
+    """k_e for every expert (int [E]) and lambda. Tdist: [E][B][H]."""
+    if not (kmin <= target <= kmax):
+        raise ValueError("target outside [kmin, kmax]")
+    E = Tdist.shape[0]
+    D = np.array([[tree_dot(m, Tdist[e, k - 1]) for k in range(kmin, kmax + 1)] for e in range(E)])
+    ks = np.arange(kmin, kmax + 1, dtype=np.float64)
+
+    def decide(lam):
+        return (np.argmin(D + lam * ks[None, :], axis=1) + kmin).astype(np.int64)
+
+    budget = float(target) * float(int(np.sum(counts)))
+    lo, hi = 0.0, 2.0 * float(np.max(D[:, 0])) + 1.0
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        n = int(np.sum(np.asarray(counts, dtype=np.int64) * decide(mid)))
+        if float(n) > budget:
+            lo = mid
+        else:
+            hi = mid
+    return decide(hi), hi, D
+
+
+def allocate_expert_table(idx: np.ndarray, k_table: np.ndarray) -> np.ndarray:
+    """Every pair reads its expert's rate."""
+    return np.asarray(k_table, dtype=np.int64)[np.asarray(idx)]
+
+
+# ---------------------------------------------------------------------------
 # Expert FFN (SwiGLU) and gate-weighted combine.
 #   a = W_gate^(k) x, u = W_up^(k) x, h = silu(a) * u, o = W_down^(k) h,
 #   y_t = sum_{slots j} g_{t,j} o_{t,j}  (+ sum of shared experts, dense, gate 1).
@@ -460,12 +567,16 @@ def shared_outputs(x_row: np.ndarray, shared) -> List[np.ndarray]:
             for s in range(sg.shape[0])]
 
 
-ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD = 0, 1, 2
+ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD, ALLOC_EXPERT_TABLE = 0, 1, 2, 3
 
 
 def allocate_policy(policy: int, idx: np.ndarray, gates: np.ndarray, r_table: Optional[np.ndarray], kmin: int,
-                    kmax: int, target: float, threshold: Optional[float] = None):
-    """Plane counts [T][K] and the policy's multiplier (lambda; the threshold; 0 for uniform)."""
+                    kmax: int, target: float, threshold: Optional[float] = None,
+                    expert_k: Optional[np.ndarray] = None):
+    """Plane counts [T][K] and the policy's multiplier (lambda; the threshold; 0 for uniform and
+    for the expert-rate table)."""
+    if policy == ALLOC_EXPERT_TABLE:
+        return allocate_expert_table(idx, expert_k), 0.0
     if policy == ALLOC_LAGRANGE:
         return allocate(idx, gates, r_table, kmin, kmax, target)
     if policy == ALLOC_UNIFORM:
@@ -479,7 +590,7 @@ def moe_forward(x_bits: np.ndarray, wr_bits: np.ndarray, experts: Dict[int, Dict
                 target: float, shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]] = None,
                 r_table: Optional[np.ndarray] = None, logits: Optional[np.ndarray] = None,
                 token_subset: Optional[Sequence[int]] = None, policy: int = ALLOC_LAGRANGE,
-                threshold: Optional[float] = None):
+                threshold: Optional[float] = None, expert_k: Optional[np.ndarray] = None):
     """One MoE layer. `experts` maps expert id -> encode_expert() output (only the experts that
     are routed to are needed); `r_table` is [E][B] (all experts' residuals; defaults to the
     encoded ones, which then must cover every expert). Returns y fp64 [T][H] (rows outside
@@ -488,7 +599,7 @@ def moe_forward(x_bits: np.ndarray, wr_bits: np.ndarray, experts: Dict[int, Dict
     idx, g, logits = route(x_bits, wr_bits, shape.top_k, shape.norm_topk, logits)
     if r_table is None and policy == ALLOC_LAGRANGE:
         r_table = np.stack([experts[e]["r"] for e in range(shape.n_experts)])
-    k, lam = allocate_policy(policy, idx, g, r_table, shape.kmin, shape.kmax, target, threshold)
+    k, lam = allocate_policy(policy, idx, g, r_table, shape.kmin, shape.kmax, target, threshold, expert_k)
     x = bf16_bits_to_f64(x_bits)
     T = x.shape[0]
     toks = range(T) if token_subset is None else token_subset

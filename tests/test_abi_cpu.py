@@ -57,12 +57,12 @@ def test_descriptor_validation(field, value, code):
     assert dpa.lib().dpa_encoded_sizes(ctypes.byref(d), ctypes.byref(s)) == code
 
 
-@pytest.mark.parametrize("hidden,code", [(2048, 0), (4608, 0), (8192, 0), (9216, 2)])
-def test_hidden_size_limit_follows_the_single_pass_staging(hidden, code):
-    # a layer is accepted when one work item of the single-pass GEMV kernels fits in shared
-    # memory (4-bit planes, group 128: hidden up to 8192); wider multi-token staging is used
-    # only where it fits as well
-    d = dpa.make_desc(W.with_sizes(W.QWEN3_B64, hidden=hidden, name=f"h{hidden}"))
+@pytest.mark.parametrize("hidden,group,code", [(2048, 128, 0), (8192, 128, 0), (9216, 128, 0), (16384, 64, 0),
+                                              (16448, 64, 2)])
+def test_hidden_size_limit(hidden, group, code):
+    # the expert GEMV stages a chunk of columns at a time, so its shared memory grows only with the
+    # scale data of an item's rows: every hidden size up to the descriptor limit (16384) fits
+    d = dpa.make_desc(W.with_sizes(W.QWEN3_B64, hidden=hidden, group=group, name=f"h{hidden}"))
     s = dpa.Sizes()
     assert dpa.lib().dpa_encoded_sizes(ctypes.byref(d), ctypes.byref(s)) == code
 

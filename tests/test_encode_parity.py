@@ -71,3 +71,22 @@ def test_plane_prefix_is_contiguous():
         trunc = dpa.export_codes(d, cut, 0, 0)
         sh_ = sh.bits - k
         assert np.array_equal(full >> sh_, trunc >> sh_)
+
+
+@pytest.mark.parametrize("shape,experts", [(W.TINY, [0, 5]),
+                                           (W.with_sizes(W.DEEPSEEK_B16, hidden=256, inter=128, name="bcq_small"), [3])])
+def test_distortion_tensor_bit_identical(shape, experts):
+    # the baked distortion tensor of the workload-profiled read rates (host C++) against the oracle
+    d = dpa.make_desc(shape)
+    out = None
+    T = None
+    for e in experts:
+        g, u, dn = W.expert_weights(shape, e)
+        out = dpa.encode(d, g[None], u[None], dn[None], e_begin=e, out=out)
+    planes, meta, _ = out
+    for e in experts:
+        g, u, dn = W.expert_weights(shape, e)
+        T = dpa.distortion_tensor(d, g[None], u[None], planes, meta, e_begin=e, out=T)
+        enc = O.encode_expert(g, u, dn, shape.fmt, shape.bits, shape.group)
+        want = O.distortion_tensor(enc, shape.fmt, shape.bits, shape.group, g, u)
+        assert np.array_equal(T[e], want), e

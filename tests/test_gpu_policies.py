@@ -88,15 +88,15 @@ def test_invalid_policy_inputs():
     L = dpa.lib()
     args = (dpa.ctypes.byref(d),)
     # unknown policy, and a threshold policy without a threshold: rejected on the host
-    for pol, thr in ((3, None), (dpa.ALLOC_THRESHOLD, None)):
+    for pol, thr in ((4, None), (dpa.ALLOC_THRESHOLD, None), (dpa.ALLOC_EXPERT_TABLE, None)):
         st = L.dpa_allocate_ex(*args, pol, None, _dev(idx).data_ptr(), _dev(g).data_ptr(), 4,
-                               _scalar(3.0).data_ptr(), thr, k0.data_ptr(), None, ws.data_ptr(), ws.numel(),
+                               _scalar(3.0).data_ptr(), thr, None, k0.data_ptr(), None, ws.data_ptr(), ws.numel(),
                                torch.cuda.current_stream().cuda_stream)
         assert st == 1
     # a NaN threshold and an out-of-range calibration target: device flag, outputs untouched
     bad = _scalar(float("nan"))
     st = L.dpa_allocate_ex(*args, dpa.ALLOC_THRESHOLD, None, _dev(idx).data_ptr(), _dev(g).data_ptr(), 4, None,
-                           bad.data_ptr(), k0.data_ptr(), None, ws.data_ptr(), ws.numel(),
+                           bad.data_ptr(), None, k0.data_ptr(), None, ws.data_ptr(), ws.numel(),
                            torch.cuda.current_stream().cuda_stream)
     assert st == 0
     assert dpa.device_status(ws) == 6 and torch.all(k0 == 7)

@@ -534,6 +534,100 @@ def test_moe_forward_policies_use_their_plane_counts():
     assert aux_t["lambda"] == 0.5
 
 
+# ----------------------------------------------------------------- workload-profiled read rates
+
+def test_distortion_tensor_channels_sum_to_the_gate_up_residual():
+    rng = np.random.default_rng(51)
+    H, I, G, B = 64, 16, 16, 4
+    g = (rng.standard_normal((I, H)) * 0.02).astype(np.float32)
+    u = (rng.standard_normal((I, H)) * 0.02).astype(np.float32)
+    d = (rng.standard_normal((H, I)) * 0.02).astype(np.float32)
+    for fmt, bb in ((0, B), (1, 3)):
+        enc = O.encode_expert(g, u, d, fmt, bb, G)
+        T = O.distortion_tensor(enc, fmt, bb, G, g, u)
+        for k in range(1, bb + 1):
+            wg, wu, _ = O.dequant_expert(enc, fmt, bb, k, G)
+            exact = [sum((Fraction(float(gm[i, j])) - Fraction(float(wm[i, j]))) ** 2
+                         for gm, wm in ((g, wg), (u, wu)) for i in range(I)) for j in range(H)]
+            for j in range(H):
+                assert abs(Fraction(T[k - 1, j]) - exact[j]) <= exact[j] * Fraction(1, 10 ** 12)
+        # monotone in k for uniform codes (each extra plane halves the step)
+        if fmt == 0:
+            assert np.all(T[:-1].sum(axis=1) > T[1:].sum(axis=1))
+
+
+def test_prefill_profile_exact_and_counts():
+    rng = np.random.default_rng(52)
+    x = _bf16_bits(rng.standard_normal((5, 32)))
+    idx = np.array([[0, 3], [3, 1], [0, 3], [2, 0], [3, 1]])
+    m, c = O.prefill_profile(x, idx, 6)
+    xf = O.bf16_bits_to_f64(x)
+    for j in range(32):
+        exact = sum(Fraction(float(xf[t, j])) ** 2 for t in range(5)) / 5
+        assert abs(Fraction(m[j]) - exact) <= exact * Fraction(1, 10 ** 14)
+    assert c.tolist() == [3, 2, 1, 4, 0, 0]
+
+
+def test_tree_dot_order_and_accuracy():
+    rng = np.random.default_rng(53)
+    m = rng.random(64) * 3
+    t = rng.random(64) * 1e-3
+    v = O.tree_dot(m, t)
+    exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(m, t))
+    assert abs(Fraction(v) - exact) <= abs(exact) * Fraction(8, 2 ** 53)
+    # the chunk/tree order: a value in chunk 0 and its negative in chunk 16 cancel at the first
+    # tree level, so a 1 in chunk 1 survives (a left-to-right sum would lose it)
+    m2 = np.ones(64)
+    t2 = np.zeros(64)
+    t2[0], t2[32], t2[2] = 1e17, -1e17, 1.0
+    assert O.tree_dot(m2, t2) == 1.0
+    seq = 0.0
+    for v in t2:
+        seq = seq + v
+    assert seq == 0.0
+
+
+def _rates_case(seed, E=5, B=4, H=32):
+    rng = np.random.default_rng(seed)
+    base = rng.random((E, 1)) * 5 + 0.5
+    T = np.stack([base * 4.0 ** (B - k) * (1 + 0.2 * rng.random((E, H))) for k in range(1, B + 1)], axis=1)
+    m = rng.random(H) + 0.1
+    counts = rng.integers(0, 6, size=E)
+    counts[0] = max(counts[0], 1)
+    return T, m, counts
+
+
+@pytest.mark.parametrize("seed,target", [(0, 3.0), (1, 2.5), (2, 3.6), (3, 2.2), (4, 4.0), (5, 2.0)])
+def test_expert_rates_match_brute_force_and_frequency_cancels(seed, target):
+    kmin, kmax = 2, 4
+    T, m, counts = _rates_case(seed)
+    k, lam, D = O.solve_expert_rates(T, m, counts, kmin, kmax, target)
+    n_hi = int(np.sum(counts * k))
+    assert n_hi <= target * counts.sum()
+    if target in (kmin, kmax):
+        assert np.all(k[counts > 0] == target)
+    # the count-weighted objective is minimal among all tables that read at most as many planes
+    best, best_set = None, []
+    for kv in itertools.product(range(kmin, kmax + 1), repeat=len(k)):
+        if sum(c * kk for c, kk in zip(counts, kv)) > n_hi:
+            continue
+        o = sum(Fraction(int(c)) * Fraction(float(D[e, kk - kmin])) for e, (c, kk) in enumerate(zip(counts, kv)))
+        if best is None or o < best:
+            best, best_set = o, [kv]
+        elif o == best:
+            best_set.append(kv)
+    used = counts > 0
+    assert any(all(a == b for a, b, u in zip(k.tolist(), bs, used) if u) for bs in best_set)
+    # frequency cancels: scaling every count by 3 leaves the solution unchanged
+    k3, lam3, _ = O.solve_expert_rates(T, m, counts * 3, kmin, kmax, target)
+    assert np.array_equal(k3, k) and lam3 == lam
+
+
+def test_expert_rate_table_allocation():
+    idx = np.array([[0, 2], [1, 2]])
+    assert O.allocate_expert_table(idx, np.array([4, 2, 3])).tolist() == [[4, 3], [2, 3]]
+
+
 # ----------------------------------------------------------------- FFN and combine
 
 def test_expert_ffn_hand_worked():
