@@ -657,26 +657,37 @@ grouping:
         const int rank_incl = block_incl_scan(flag, s_tmp);
         const int tiles_incl = block_incl_scan(ntiles, s_tmp);
         const int gt_incl = a.gtiles ? block_incl_scan(ngt, s_tmp) : 0;
-        const int vt_incl = a.vgroups ? block_incl_scan(nvt, s_tmp) : 0;
-        const int vg_incl = a.vgroups ? block_incl_scan(nvg, s_tmp) : 0;
+        const int vt_incl = a.vrec ? block_incl_scan(nvt, s_tmp) : 0;
+        const int vg_incl = a.vrec ? block_incl_scan(nvg, s_tmp) : 0;
         const int rank = rank_base + rank_incl - flag;
         const int tile_off = tile_base + tiles_incl - ntiles;
-        if (a.vgroups && nvt > 0) {   // 4-pair tiles of one (expert, k) class, in groups of vtpg tiles
-            int t = vt_base + vt_incl - nvt, gi = vg_base + vg_incl - nvg, in_group = 0, g_first = t, g_km = 0;
+        if (a.vrec && nvt > 0) {   // 4-pair tiles of one (expert, k) class, in groups of vtpg tiles
+            int gi = vg_base + vg_incl - nvg, in_group = 0;
+            int32_t* rec = a.vrec + static_cast<size_t>(gi) * kVRecInts;
             for (int i = 0; i < nk; ++i) {
                 const int s0 = s_seg[e * nk + i];
                 const int n = s_seg[e * nk + i + 1] - s0;
                 for (int j = 0; j < n; j += 4) {
-                    a.vtiles[t++] = make_int4(a.kmin + i, s0 + j, min(4, n - j), 0);
-                    g_km = a.kmin + i;
-                    if (++in_group == vtpg) {
-                        a.vgroups[gi++] = make_int4(e, g_km, in_group, g_first);
+                    if (in_group == 0) {   // a new record: expert, and every slot unused
+                        rec[0] = e;
+                        for (int q = 3; q < kVRecInts; ++q) rec[q] = q >= 8 && q < 24 ? -1 : 0;
+                    }
+                    const int cnt = min(4, n - j);
+                    rec[1] = a.kmin + i;            // tiles ascend in k: the last is the group's kmax
+                    rec[4 + in_group] = a.kmin + i;
+                    rec[6 + in_group] = cnt;
+                    for (int q = 0; q < cnt; ++q) {
+                        const int pos = s0 + j + q;
+                        rec[8 + 4 * in_group + q] = pos;                    // output row
+                        rec[16 + 4 * in_group + q] = s_sorted[pos] / a.K;   // token
+                    }
+                    rec[2] = ++in_group;
+                    if (in_group == vtpg) {
                         in_group = 0;
-                        g_first = t;
+                        rec += kVRecInts;
                     }
                 }
             }
-            if (in_group > 0) a.vgroups[gi++] = make_int4(e, g_km, in_group, g_first);
         }
         if (a.gtiles && ngt > 0) {   // token tiles of the prefill GEMMs: one (expert, k) class each
             int t = gt_base + gt_incl - ngt;

@@ -26,8 +26,8 @@ dpa_status check_desc(const dpa_layer_desc* d) {
     if (d->hidden % d->group || d->inter % d->group) return DPA_ERR_UNSUPPORTED;
     if (d->hidden > 16384 || d->inter > 16384) return DPA_ERR_UNSUPPORTED;
     // the staging of the expert GEMV's small-batch variant must fit in shared memory
-    if (dpa::vp_smem_bytes(d->hidden, d->group, d->format, d->bits, 2, false) > dpa::kVpMaxSmem ||
-        dpa::vp_smem_bytes(d->inter, d->group, d->format, d->bits, 1, false) > dpa::kVpMaxSmem)
+    if (dpa::vp_smem_bytes(d->hidden, d->group, d->format, d->bits, 2, 1) > dpa::kVpMaxSmem ||
+        dpa::vp_smem_bytes(d->inter, d->group, d->format, d->bits, 1, 1) > dpa::kVpMaxSmem)
         return DPA_ERR_UNSUPPORTED;
     return DPA_OK;
 }
@@ -35,7 +35,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
-        desc, tiles, gtiles, postok, coop, rstats, xperm, hdig, hexp, hsum, vtiles, vgroups, total;
+        desc, tiles, gtiles, postok, coop, rstats, xperm, hdig, hexp, hsum, vrec, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -79,8 +79,7 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.hdig = take(2 * P * I);
     L.hexp = take(4 * P * ngp_i);
     L.hsum = take(4 * P * ngp_i);
-    L.vtiles = take(16 * (P / 4 + E * nk + 1));
-    L.vgroups = take(16 * (P / 4 + E * nk + 1));
+    L.vrec = take(4 * dpa::kVRecInts * (P / 4 + E * nk + 1));
     L.total = off;
     return L;
 }
@@ -263,9 +262,8 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.exp_desc = at<int4>(ws, L.desc);
     a.tiles = at<int4>(ws, L.tiles);
     a.gtiles = gemm_tiles ? at<int4>(ws, L.gtiles) : nullptr;
-    a.pos_tok = permute ? at<int32_t>(ws, L.postok) : nullptr;
-    a.vtiles = permute && !gemm_tiles ? at<int4>(ws, L.vtiles) : nullptr;
-    a.vgroups = permute && !gemm_tiles ? at<int4>(ws, L.vgroups) : nullptr;
+    a.pos_tok = gemm_tiles ? at<int32_t>(ws, L.postok) : nullptr;
+    a.vrec = permute && !gemm_tiles ? at<int32_t>(ws, L.vrec) : nullptr;
     a.vtiles_per_group = vtiles_per_group;
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
     return dpa::launch_allocate(a, s, at<dpa::CoopSync>(ws, L.coop), num_sms_current()) == cudaSuccess ? DPA_OK
@@ -448,11 +446,10 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     // 2. allocate + group pairs by (expert, k)
     // the expert GEMV's variant: one token per expert (batch 1) runs the small-batch kernels;
     // otherwise token groups of up to two 4-pair tiles, where their staging fits
-    const bool multi = T > 1 &&
-                       dpa::vp_smem_bytes(d->hidden, d->group, d->format, d->bits, 2, true) <= dpa::kVpMaxSmem &&
-                       dpa::vp_smem_bytes(d->inter, d->group, d->format, d->bits, 1, true) <= dpa::kVpMaxSmem;
+    // token groups of the expert GEMV: two 4-pair tiles where the group slots fit, else one
+    const int tpg = dpa::vp_tiles_per_group(d->hidden, d->inter, d->group, d->format, d->bits);
     dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s, use_tc, policy,
-                                   threshold, multi ? 2 : 1, expert_k);
+                                   threshold, tpg, expert_k);
     if (st2 != DPA_OK) return st2;
     mark(2);
 
@@ -520,10 +517,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     va.fmt = d->format;
     va.B = d->bits;
     va.G = d->group;
-    va.multi = multi ? 1 : 0;
-    va.vgroups = at<int4>(ws, L.vgroups);
-    va.vtiles = at<int4>(ws, L.vtiles);
-    va.pos_tok = at<int32_t>(ws, L.postok);
+    va.tiles_per_group = tpg;
+    va.vrec = at<int32_t>(ws, L.vrec);
     va.hdr = hdr;
     const int tiles_bound = P / 4 + d->n_experts * nk;
     va.max_groups = P < tiles_bound ? P : tiles_bound;
@@ -571,6 +566,55 @@ dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidde
                                         1e-6f, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? DPA_OK
                : DPA_ERR_CUDA;
+}
+
+dpa_status dpa_stream_prefixes(const dpa_layer_desc* d, const void* host_planes, const void* host_meta,
+                               const int32_t* experts, const uint8_t* kplanes, int n, void* dev_planes, void* dev_meta,
+                               uint64_t* bytes_out, void* stream) {
+    const dpa_status st = check_desc(d);
+    if (st != DPA_OK) return st;
+    if (!host_planes || !host_meta || !experts || !kplanes || n < 0 || !dev_planes || !dev_meta)
+        return DPA_ERR_INVALID_ARG;
+    dpa_sizes sz;
+    dpa_encoded_sizes(d, &sz);
+    for (int i = 0; i < n; ++i)
+        if (experts[i] < 0 || experts[i] >= d->n_experts || kplanes[i] < 1 || kplanes[i] > d->bits)
+            return DPA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint8_t* hp = static_cast<const uint8_t*>(host_planes);
+    const uint8_t* hm = static_cast<const uint8_t*>(host_meta);
+    uint8_t* dp = static_cast<uint8_t*>(dev_planes);
+    uint8_t* dm = static_cast<uint8_t*>(dev_meta);
+    const uint64_t H = d->hidden, I = d->inter, G = d->group, B = d->bits;
+    uint64_t total = 0;
+    for (int i = 0; i < n; ++i) {
+        const uint64_t e = static_cast<uint64_t>(experts[i]), k = kplanes[i];
+        for (int m = 0; m < 3; ++m) {
+            // the first k planes of a matrix are one contiguous prefix of its bytes
+            const uint64_t plane_bytes = H * I / 8;
+            const uint64_t off = e * sz.planes_per_expert + sz.planes_matrix_offset[m];
+            if (cudaMemcpyAsync(dp + off, hp + off, k * plane_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return DPA_ERR_CUDA;
+            total += k * plane_bytes;
+            if (d->format == DPA_FMT_BCQ) {   // the first k planes' alphas, a prefix per matrix too
+                const uint64_t R = m == 2 ? H : I, C = m == 2 ? I : H;
+                const uint64_t moff = e * sz.meta_per_expert + sz.meta_matrix_offset[m];
+                const uint64_t abytes = k * R * (C / G) * 2;
+                if (cudaMemcpyAsync(dm + moff, hm + moff, abytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                    return DPA_ERR_CUDA;
+                total += abytes;
+            }
+        }
+        if (d->format == DPA_FMT_UNIFORM) {   // scales and zeros serve every k: the expert's whole block
+            const uint64_t moff = e * sz.meta_per_expert;
+            if (cudaMemcpyAsync(dm + moff, hm + moff, sz.meta_per_expert, cudaMemcpyHostToDevice, s) != cudaSuccess)
+                return DPA_ERR_CUDA;
+            total += sz.meta_per_expert;
+        }
+    }
+    (void)B;
+    if (bytes_out) *bytes_out = total;
+    return DPA_OK;
 }
 
 dpa_status dpa_device_status(void* ws, void* stream) {

@@ -16,17 +16,18 @@
 // gathered into nibbles (one register of eight 4-bit codes per nibble position rho), split into
 // the low and high nibbles of each byte, and masked to the k planes a token tile reads.
 //
-// Work: items are (token group, row block). A token group is up to NTILE tiles of up to four
-// pairs of one expert, each tile of one plane count k (tiles ascending in k). One CTA per SM,
-// persistent over its items:
-//   - warp 16 (producer) streams each item's columns in chunks into a ring of stages with bulk
-//     copies (no multicast): for every matrix and plane p < kmax of the group and every row
-//     tile, the chunk's plane words; the chunk's digit rows of the group's tokens; with the
-//     item's first chunk also its scales and the tokens' group exponents and sums;
-//   - warps 0-15 (consumers) take row tile rt and column slice cs of every chunk; they wait for
-//     a stage's full barrier, compute, and release it through the stage's empty barrier;
-//   - at the end of an item the column slices of a row tile are summed in a fixed order and the
-//     epilogue (SwiGLU for gate/up, the per-pair output for down) is written.
+// Work. A token group (written by the allocation as one record) is up to NTILE tiles of up to
+// four pairs of one expert, each tile of one plane count k, tiles ascending in k. Items are
+// (token group, block of RB = 16 NRT rows); every CTA (one per SM, persistent) takes a contiguous
+// range of items, so consecutive items mostly share their group. Roles:
+//   - warp 8 (producer): per group, bulk copies (no multicast) of the tokens' digit rows, group
+//     exponents and sums into one of two group slots; per item and chunk of up to 2048 columns,
+//     bulk copies of the chunk's plane words (one copy per matrix, plane p < kmax and row tile:
+//     2 bytes per column) and, with the first chunk, the item's scale data into a ring stage;
+//   - warps 0-7 (consumers): row tile rt and column slice cs of every chunk; wait for the stage,
+//     compute, release it; after the item's last chunk the slices of a row tile are summed in a
+//     fixed order by one of them (rotating with the item) and the epilogue (SwiGLU for gate/up,
+//     the per-pair output for down) is written.
 // Every wait is bounded (globaltimer); on a timeout the kernel records DPA_ERR_DEVICE_TIMEOUT,
 // sets a CTA-wide abort flag that ends every other wait, and the producer waits for the copies
 // it issued before the CTA exits.
@@ -42,23 +43,24 @@ constexpr int kCW = 8;                        // consumer warps
 constexpr int kVThreads = (kCW + 1) * 32;     // + the producer warp
 constexpr int kMaxStages = 8;                 // ring depth: as many stages as shared memory holds
 constexpr int kMaxB = 4;
+constexpr int kMaxChunk = 2048;               // columns per chunk
 constexpr int kDigPad = 64;                   // bytes of padding per staged digit row (banks)
 
 template <int NRT>
 struct Geo {
     static constexpr int CS = kCW / NRT;      // column slices per chunk
-    static constexpr int CWS = 128;           // columns per slice (two 64-column blocks)
-    static constexpr int CK = CS * CWS;       // columns per chunk
     static constexpr int RB = 16 * NRT;       // rows per item
 };
 
 __host__ __device__ inline size_t al16(size_t v) { return (v + 15) & ~static_cast<size_t>(15); }
 __host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~static_cast<size_t>(127); }
 
-struct VLayout {                             // byte offsets in dynamic shared memory (< 227 KB)
-    uint32_t stage, st_dig, dig_stride;       // per stage: planes at 0, digits at st_dig
-    uint32_t slot, sl_exp, sl_sum, sl_tab;    // per item slot: meta at 0, then exps, sums, table
-    uint32_t red, red_per;                    // reduction buffer (NRT x (CS-1) warps)
+struct VLayout {                              // byte offsets in dynamic shared memory (< 227 KB)
+    uint32_t CK;                              // columns per chunk
+    uint32_t stage, st_meta;                  // per stage: planes at 0, then the item's scale data
+    uint32_t slot, sl_exp, sl_sum, sl_rec;    // per group slot: digits at 0, exps, sums, record
+    uint32_t dig_stride;                      // bytes per staged digit row (K + pad)
+    uint32_t slots, red, red_per;             // group slots' offset; reduction buffer
     uint32_t total;
     int nst;                                  // stages in the ring
     int ngp;                                  // exps/sums row stride (ints)
@@ -70,34 +72,37 @@ __host__ __device__ inline VLayout vlayout(int K, int G, int fmt, int B) {
     VLayout L;
     const size_t ng = K / G;
     L.ngp = static_cast<int>((ng + 3) & ~static_cast<size_t>(3));
-    const size_t dig_stride = Gm::CK + kDigPad;
-    const size_t planes = static_cast<size_t>(NMAT) * kMaxB * NRT * (Gm::CK / 64) * 128;
-    const size_t stage = al128(planes + static_cast<size_t>(4 * NTILE) * 2 * dig_stride);
+    const size_t CK = K < kMaxChunk ? K : kMaxChunk;
+    const size_t planes = static_cast<size_t>(NMAT) * kMaxB * NRT * (CK / 64) * 128;
     const size_t meta = fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(NMAT) * Gm::RB * ng * 4
                                                : static_cast<size_t>(NMAT) * B * Gm::RB * ng * 2;
-    const size_t sl_exp = al16(meta);
+    const size_t stage = al128(planes + al16(meta));
+    const size_t dig_stride = static_cast<size_t>(K) + kDigPad;
+    const size_t digs = static_cast<size_t>(4 * NTILE) * 2 * dig_stride;
+    const size_t sl_exp = al16(digs);
     const size_t sl_sum = sl_exp + static_cast<size_t>(4 * NTILE) * L.ngp * 4;
-    const size_t sl_tab = sl_sum + static_cast<size_t>(4 * NTILE) * L.ngp * 4;
-    // table: {e, kmax, ntiles, rb}, NTILE x {k, n, 0, 0}, 4*NTILE digit rows, 4*NTILE output rows
-    const size_t slot = al128(sl_tab + 16 + 16 * NTILE + 8 * 4 * NTILE);
+    const size_t sl_rec = sl_sum + static_cast<size_t>(4 * NTILE) * L.ngp * 4;
+    const size_t slot = al128(sl_rec + kVRecInts * 4);
     const size_t red_per = static_cast<size_t>(32) * NTILE * NMAT * 2 * 4;
-    const size_t fixed = 2 * slot + static_cast<size_t>(NRT) * (Gm::CS - 1) * red_per;
+    const size_t red = static_cast<size_t>(NRT) * Gm::CS * red_per;   // one partial per warp
+    const size_t fixed = 2 * slot + red;
     int nst = 2;   // at least double buffering; more while the ring fits beside the fixed parts
     while (nst < kMaxStages && fixed + (nst + 1) * stage <= kVpMaxSmem) ++nst;
-    const size_t red = nst * stage + 2 * slot;
-    size_t total = red + static_cast<size_t>(NRT) * (Gm::CS - 1) * red_per;
+    size_t total = nst * stage + fixed;
     if (total > 0xFFFFFFFFull) total = 0xFFFFFFFFull;   // rejected by the caller (too large)
-    L.nst = nst;
+    L.CK = static_cast<uint32_t>(CK);
     L.stage = static_cast<uint32_t>(stage);
-    L.st_dig = static_cast<uint32_t>(planes);
-    L.dig_stride = static_cast<uint32_t>(dig_stride);
+    L.st_meta = static_cast<uint32_t>(planes);
     L.slot = static_cast<uint32_t>(slot);
     L.sl_exp = static_cast<uint32_t>(sl_exp);
     L.sl_sum = static_cast<uint32_t>(sl_sum);
-    L.sl_tab = static_cast<uint32_t>(sl_tab);
-    L.red = static_cast<uint32_t>(red);
+    L.sl_rec = static_cast<uint32_t>(sl_rec);
+    L.dig_stride = static_cast<uint32_t>(dig_stride);
+    L.slots = static_cast<uint32_t>(nst * stage);
+    L.red = static_cast<uint32_t>(nst * stage + 2 * slot);
     L.red_per = static_cast<uint32_t>(red_per);
     L.total = static_cast<uint32_t>(total);
+    L.nst = nst;
     return L;
 }
 
@@ -142,26 +147,28 @@ __device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) 
 // ---- B operand: the lane's 16 digit bytes of one 64-column block (one 16-byte load) ----
 __device__ __forceinline__ uint4 lds128(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
 
-template <int NRT, int NTILE, int NMAT>
-struct Item {
-    int e, kmax, nt, rb;
+// the group of the current item, as the consumers read it from the group slot's record
+template <int NTILE>
+struct Group {
+    int kmax, nt;
     int tk[NTILE], tn[NTILE];
 };
 
 // ---------------------------------------------------------------------------------------
-// consumer: one column slice of one chunk, uniform codes
+// consumer: one column slice of one chunk, uniform codes. Blocks [b0, b1) of the chunk; the
+// group slot holds the tokens' digits for every column (col0 = the chunk's first column).
 // ---------------------------------------------------------------------------------------
 template <int B, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L, const unsigned char* st,
-                                              const unsigned char* sl, const Item<NRT, NTILE, NMAT>& it, int col0,
-                                              int rt, int cs, float (&acc)[NTILE][NMAT][2]) {
+                                              const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0,
+                                              int b1, int rt, float (&acc)[NTILE][NMAT][2]) {
     using Gm = Geo<NRT>;
     const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
-    const int G = a.G, K = a.K, ng = K / G;
+    const int G = a.G, K = a.K, ng = K / G, nbc = L.CK / 64;
     const uint32_t* planes = reinterpret_cast<const uint32_t*>(st);
-    const unsigned char* dig = st + L.st_dig;
-    const int* sexp = reinterpret_cast<const int*>(sl + L.sl_exp);
-    const int* ssum = reinterpret_cast<const int*>(sl + L.sl_sum);
+    const uint32_t* meta = reinterpret_cast<const uint32_t*>(st + L.st_meta);
+    const int* sexp = reinterpret_cast<const int*>(gs + L.sl_exp);
+    const int* ssum = reinterpret_cast<const int*>(gs + L.sl_sum);
     int C[NTILE][NMAT][4];
 #pragma unroll
     for (int t = 0; t < NTILE; ++t)
@@ -169,35 +176,33 @@ __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L,
         for (int m = 0; m < NMAT; ++m) C[t][m][0] = C[t][m][1] = C[t][m][2] = C[t][m][3] = 0;
     bool has_start = false;
 #pragma unroll 1
-    for (int blk = 0; blk < 2; ++blk) {
-        const int cb = cs * 2 + blk;                     // block inside the chunk
+    for (int cb = b0; cb < b1; ++cb) {
         const int colb = col0 + cb * 64;                 // global column of the block
-        if (colb >= K) break;
         if (colb % G == 0) has_start = true;
         // the B fragments of the tiles (shared by the matrices), then one matrix at a time
         uint4 bt[NTILE];
 #pragma unroll
         for (int t = 0; t < NTILE; ++t)
-            if (t < it.nt)
-                bt[t] = lds128(dig + static_cast<size_t>((4 * t + (gid >> 1)) * 2 + (gid & 1)) * L.dig_stride +
-                               cb * 64 + 16 * tq);
+            if (t < gr.nt)
+                bt[t] = lds128(gs + static_cast<size_t>((4 * t + (gid >> 1)) * 2 + (gid & 1)) * L.dig_stride + colb +
+                               16 * tq);
 #pragma unroll
         for (int m = 0; m < NMAT; ++m) {
             uint32_t w[kMaxB];
 #pragma unroll
             for (int p = 0; p < kMaxB; ++p)
-                w[p] = p < it.kmax ? planes[(((m * kMaxB + p) * NRT + rt) * (Gm::CK / 64) + cb) * 32 + lane] : 0u;
+                w[p] = p < gr.kmax ? planes[(((m * kMaxB + p) * NRT + rt) * nbc + cb) * 32 + lane] : 0u;
             uint32_t R[4], Rh[4];
-            assemble<B>(R, w, it.kmax);
+            assemble<B>(R, w, gr.kmax);
 #pragma unroll
             for (int r = 0; r < 4; ++r) Rh[r] = R[r] >> 4;
             int level = -1;
             uint32_t Alo[4], Ahi[4];
 #pragma unroll
             for (int t = 0; t < NTILE; ++t) {
-                if (t < it.nt) {
-                    if (it.tk[t] != level) {
-                        level = it.tk[t];
+                if (t < gr.nt) {
+                    if (gr.tk[t] != level) {
+                        level = gr.tk[t];
                         const uint32_t mk = level_mask(B, level);
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
@@ -210,11 +215,9 @@ __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L,
                 }
             }
         }
-        // a group portion ends at the slice end, at the end of the columns, or at a group boundary
-        const bool end = blk == 1 || colb + 64 >= K || (colb + 64) % G == 0;
-        if (end) {
+        // a group portion ends at the slice end or at a group boundary
+        if (cb + 1 == b1 || (colb + 64) % G == 0) {
             const int g = colb / G;
-            const uint32_t* meta = reinterpret_cast<const uint32_t*>(sl);
             float s[NMAT][2], z[NMAT][2];
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
@@ -226,11 +229,11 @@ __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L,
                 }
 #pragma unroll
             for (int t = 0; t < NTILE; ++t) {
-                if (t < it.nt) {
+                if (t < gr.nt) {
                     const int j = 4 * t + tq;
                     const float f = pow2i(sexp[j * L.ngp + g] - 14);
                     const float sx = has_start ? static_cast<float>(ssum[j * L.ngp + g]) : 0.f;
-                    const float ck = 0.5f * static_cast<float>((1 << (B - it.tk[t])) - 1);
+                    const float ck = 0.5f * static_cast<float>((1 << (B - gr.tk[t])) - 1);
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m)
 #pragma unroll
@@ -252,55 +255,54 @@ __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L,
 // ---------------------------------------------------------------------------------------
 template <int B, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_bcq(const VpArgs& a, const VLayout& L, const unsigned char* st,
-                                          const unsigned char* sl, const Item<NRT, NTILE, NMAT>& it, int col0, int rt,
-                                          int cs, float (&acc)[NTILE][NMAT][2]) {
+                                          const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0, int b1,
+                                          int rt, float (&acc)[NTILE][NMAT][2]) {
     using Gm = Geo<NRT>;
     const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
-    const int G = a.G, K = a.K, ng = K / G;
+    const int G = a.G, K = a.K, ng = K / G, nbc = L.CK / 64;
     const uint32_t* planes = reinterpret_cast<const uint32_t*>(st);
-    const unsigned char* dig = st + L.st_dig;
-    const int* sexp = reinterpret_cast<const int*>(sl + L.sl_exp);
-    const int* ssum = reinterpret_cast<const int*>(sl + L.sl_sum);
-    const __half* meta = reinterpret_cast<const __half*>(sl);
-    // the slice's blocks in group portions: [b0, b1) of blocks 0..1
-    int b0 = 0;
-    while (b0 < 2) {
-        const int colb0 = col0 + (cs * 2 + b0) * 64;
-        if (colb0 >= K) break;
-        int b1 = b0 + 1;
-        if (b1 < 2 && (colb0 + 64) % G != 0 && colb0 + 64 < K) b1 = 2;
+    const __half* meta = reinterpret_cast<const __half*>(st + L.st_meta);
+    const int* sexp = reinterpret_cast<const int*>(gs + L.sl_exp);
+    const int* ssum = reinterpret_cast<const int*>(gs + L.sl_sum);
+    // the slice's blocks in group portions [p0, p1)
+    int p0 = b0;
+    while (p0 < b1) {
+        const int colb0 = col0 + p0 * 64;
+        int p1 = p0 + 1;
+        while (p1 < b1 && (col0 + p1 * 64) % G != 0) ++p1;
         const int g = colb0 / G;
         const bool has_start = colb0 % G == 0;
 #pragma unroll
         for (int p = 0; p < B; ++p) {
-            if (p < it.kmax) {
+            if (p < gr.kmax) {
                 int C[NTILE][NMAT][4];
 #pragma unroll
                 for (int t = 0; t < NTILE; ++t)
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m) C[t][m][0] = C[t][m][1] = C[t][m][2] = C[t][m][3] = 0;
-                for (int blk = b0; blk < b1; ++blk) {
-                    const int cb = cs * 2 + blk;
-                    uint32_t lo[NMAT][4], hi[NMAT][4];
+#pragma unroll 1
+                for (int cb = p0; cb < p1; ++cb) {
+                    const int colb = col0 + cb * 64;
+                    uint4 bt[NTILE];
+#pragma unroll
+                    for (int t = 0; t < NTILE; ++t)
+                        if (t < gr.nt && gr.tk[t] > p)
+                            bt[t] = lds128(gs + static_cast<size_t>((4 * t + (gid >> 1)) * 2 + (gid & 1)) * L.dig_stride +
+                                           colb + 16 * tq);
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m) {
-                        const uint32_t w = planes[(((m * kMaxB + p) * NRT + rt) * (Gm::CK / 64) + cb) * 32 + lane];
+                        const uint32_t w = planes[(((m * kMaxB + p) * NRT + rt) * nbc + cb) * 32 + lane];
+                        uint32_t lo[4], hi[4];
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
-                            lo[m][r] = (w >> r) & 0x01010101u;
-                            hi[m][r] = (w >> (r + 4)) & 0x01010101u;
+                            lo[r] = (w >> r) & 0x01010101u;
+                            hi[r] = (w >> (r + 4)) & 0x01010101u;
                         }
-                    }
 #pragma unroll
-                    for (int t = 0; t < NTILE; ++t) {
-                        if (t < it.nt && it.tk[t] > p) {
-                            const uint4 b = lds128(dig +
-                                                   static_cast<size_t>((4 * t + (gid >> 1)) * 2 + (gid & 1)) * L.dig_stride +
-                                                   cb * 64 + 16 * tq);
-#pragma unroll
-                            for (int m = 0; m < NMAT; ++m) {
-                                mma_u8s8(C[t][m], lo[m][0], lo[m][1], lo[m][2], lo[m][3], b.x, b.y);
-                                mma_u8s8(C[t][m], hi[m][0], hi[m][1], hi[m][2], hi[m][3], b.z, b.w);
+                        for (int t = 0; t < NTILE; ++t) {
+                            if (t < gr.nt && gr.tk[t] > p) {
+                                mma_u8s8(C[t][m], lo[0], lo[1], lo[2], lo[3], bt[t].x, bt[t].y);
+                                mma_u8s8(C[t][m], hi[0], hi[1], hi[2], hi[3], bt[t].z, bt[t].w);
                             }
                         }
                     }
@@ -310,10 +312,10 @@ __device__ __forceinline__ void slice_bcq(const VpArgs& a, const VLayout& L, con
                 for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr)
-                        al[m][rr] = __half2float(meta[((m * it.kmax + p) * Gm::RB + rt * 16 + gid + 8 * rr) * ng + g]);
+                        al[m][rr] = __half2float(meta[((m * gr.kmax + p) * Gm::RB + rt * 16 + gid + 8 * rr) * ng + g]);
 #pragma unroll
                 for (int t = 0; t < NTILE; ++t) {
-                    if (t < it.nt && it.tk[t] > p) {
+                    if (t < gr.nt && gr.tk[t] > p) {
                         const int j = 4 * t + tq;
                         const float f = pow2i(sexp[j * L.ngp + g] - 14);
                         const float sx = has_start ? static_cast<float>(ssum[j * L.ngp + g]) : 0.f;
@@ -328,27 +330,27 @@ __device__ __forceinline__ void slice_bcq(const VpArgs& a, const VLayout& L, con
                 }
             }
         }
-        b0 = b1;
+        p0 = p1;
     }
 }
 
 template <int FMT, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_dispatch(const VpArgs& a, const VLayout& L, const unsigned char* st,
-                                               const unsigned char* sl, const Item<NRT, NTILE, NMAT>& it, int col0,
-                                               int rt, int cs, float (&acc)[NTILE][NMAT][2]) {
+                                               const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0,
+                                               int b1, int rt, float (&acc)[NTILE][NMAT][2]) {
     if constexpr (FMT == DPA_FMT_UNIFORM) {
         switch (a.B) {
-            case 1: slice_uniform<1, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
-            case 2: slice_uniform<2, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
-            case 3: slice_uniform<3, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
-            default: slice_uniform<4, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
+            case 1: slice_uniform<1, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+            case 2: slice_uniform<2, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+            case 3: slice_uniform<3, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+            default: slice_uniform<4, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
         }
     } else {
         switch (a.B) {
-            case 1: slice_bcq<1, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
-            case 2: slice_bcq<2, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
-            case 3: slice_bcq<3, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
-            default: slice_bcq<4, NRT, NTILE, NMAT>(a, L, st, sl, it, col0, rt, cs, acc); break;
+            case 1: slice_bcq<1, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+            case 2: slice_bcq<2, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+            case 3: slice_bcq<3, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+            default: slice_bcq<4, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
         }
     }
 }
@@ -360,7 +362,7 @@ template <int FMT, int NRT, int NTILE, int NMAT>
 __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
     using Gm = Geo<NRT>;
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ uint64_t s_full[kMaxStages], s_empty[kMaxStages], s_slot_empty[2];
+    __shared__ uint64_t s_full[kMaxStages], s_empty[kMaxStages], s_gfull[2], s_gempty[2];
     __shared__ uint64_t s_red_full[NRT], s_red_free[NRT];
     __shared__ int s_abort;
     const VLayout L = vlayout<NRT, NTILE, NMAT>(a.K, a.G, FMT, a.B);
@@ -370,7 +372,10 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], kCW);
         }
-        for (int b = 0; b < 2; ++b) mbar_init(&s_slot_empty[b], kCW);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_gfull[b], 1);
+            mbar_init(&s_gempty[b], kCW);
+        }
         for (int r = 0; r < NRT; ++r) {
             mbar_init(&s_red_full[r], Gm::CS - 1);
             mbar_init(&s_red_free[r], 1);
@@ -383,118 +388,97 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
     volatile int* abort = &s_abort;
     const int K = a.K, ng = K / a.G;
     const int n_rb = a.R / Gm::RB;
-    const int n_chunks = (K + Gm::CK - 1) / Gm::CK;
+    const int n_chunks = (K + static_cast<int>(L.CK) - 1) / static_cast<int>(L.CK);
     const int n_items = static_cast<int>(__ldcg(&a.hdr->n_vgroups)) * n_rb;
+    // this CTA's contiguous range of items
+    const int it0 = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
+    const int it1 = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
 
     if (warp == kCW) {
         // ================================ producer ================================
-        int q = 0;   // chunk counter over this CTA's items
-        int issued_upto = 0;
-        for (int n = 0, it = blockIdx.x; it < n_items && !*abort; ++n, it += gridDim.x) {
-            const int slot = n & 1;
-            unsigned char* sl = smem + L.nst * L.stage + slot * L.slot;
-            if (n >= 2 && !vwait(&s_slot_empty[slot], ((n - 2) >> 1) & 1, abort, a.hdr, 0x301)) break;
+        int q = 0, gcount = 0, cur_g = -1, kmax = 0, e = 0;
+        int issued_upto = 0, groups_issued = 0;
+        const uint32_t mrow = FMT == DPA_FMT_UNIFORM ? static_cast<uint32_t>(Gm::RB * ng * 4)
+                                                     : static_cast<uint32_t>(Gm::RB * ng * 2);
+        const uint64_t plane_bytes = static_cast<uint64_t>(a.R) * K / 8;
+        for (int it = it0; it < it1 && !*abort; ++it) {
             const int gi = it / n_rb, rb = it - gi * n_rb;
-            const int4 grp = __ldcg(a.vgroups + gi);   // {e, kmax, ntiles, first tile}
-            const int e = grp.x, kmax = grp.y, nt = grp.z;
-            int4 tile = make_int4(0, 0, 0, 0);
-            if (lane < nt) tile = __ldcg(a.vtiles + grp.w + lane);   // {k, pos0, n, 0}
-            // token slots j = 4t + jj: digit row and output row of each
-            const int tj = lane >> 2, jj = lane & 3;
-            const int t_k = __shfl_sync(0xffffffffu, tile.x, tj & (NTILE - 1));
-            const int t_pos0 = __shfl_sync(0xffffffffu, tile.y, tj & (NTILE - 1));
-            const int t_n = __shfl_sync(0xffffffffu, tile.z, tj & (NTILE - 1));
-            (void)t_k;
-            int drow = -1, opos = -1;
-            if (lane < 4 * NTILE && tj < nt && jj < t_n) {
-                opos = t_pos0 + jj;
-                drow = a.dig_by_token ? __ldcg(a.pos_tok + opos) : opos;
+            if (gi != cur_g) {
+                // ---- a new token group: its record, digit rows, exponents and sums -> group slot
+                const int slot = gcount & 1;
+                if (gcount >= 2 && !vwait(&s_gempty[slot], ((gcount - 2) >> 1) & 1, abort, a.hdr, 0x301)) break;
+                const int rv = __ldcg(a.vrec + static_cast<size_t>(gi) * kVRecInts + lane);
+                e = __shfl_sync(0xffffffffu, rv, 0);
+                kmax = __shfl_sync(0xffffffffu, rv, 1);
+                const int drow = __shfl_sync(0xffffffffu, rv, (a.dig_by_token ? 16 : 8) + (lane & 7));
+                const bool valid = lane < 4 * NTILE && drow >= 0;
+                unsigned char* gs = smem + L.slots + slot * L.slot;
+                reinterpret_cast<int*>(gs + L.sl_rec)[lane] = rv;
+                __syncwarp();
+                const uint32_t nvalid = static_cast<uint32_t>(__popc(__ballot_sync(0xffffffffu, valid)));
+                if (lane == 0) {
+                    fence_proxy_async();
+                    mbar_arrive_expect_tx(&s_gfull[slot], nvalid * (2u * K + 2u * L.ngp * 4u));
+                }
+                __syncwarp();
+                fence_proxy_async();
+                if (valid) {
+                    for (int d = 0; d < 2; ++d)
+                        bulk_g2s(gs + static_cast<size_t>(lane * 2 + d) * L.dig_stride,
+                                 a.dig + (static_cast<size_t>(drow) * 2 + d) * K, static_cast<uint32_t>(K), &s_gfull[slot]);
+                    bulk_g2s(gs + L.sl_exp + static_cast<size_t>(lane) * L.ngp * 4,
+                             a.dexp + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u, &s_gfull[slot]);
+                    bulk_g2s(gs + L.sl_sum + static_cast<size_t>(lane) * L.ngp * 4,
+                             a.dsum + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u, &s_gfull[slot]);
+                }
+                cur_g = gi;
+                ++gcount;
+                groups_issued = gcount;
             }
-            int* tab = reinterpret_cast<int*>(sl + L.sl_tab);
-            if (lane == 0) {
-                tab[0] = e;
-                tab[1] = kmax;
-                tab[2] = nt;
-                tab[3] = rb;
-            }
-            if (lane < NTILE) {
-                tab[4 + 4 * lane] = lane < nt ? tile.x : 0;
-                tab[4 + 4 * lane + 1] = lane < nt ? tile.z : 0;
-            }
-            if (lane < 4 * NTILE) {
-                tab[4 + 4 * NTILE + lane] = drow;
-                tab[4 + 8 * NTILE + lane] = opos;
-            }
-            __syncwarp();
-            const unsigned valid = __ballot_sync(0xffffffffu, drow >= 0);
             const uint8_t* pbase = a.planes + static_cast<uint64_t>(e) * a.planes_per_expert;
-            const uint64_t plane_bytes = static_cast<uint64_t>(a.R) * K / 8;
+            const uint8_t* mbase = a.meta + static_cast<uint64_t>(e) * a.meta_per_expert;
+            const int n_meta = FMT == DPA_FMT_UNIFORM ? NMAT : NMAT * kmax;
             for (int c = 0; c < n_chunks; ++c, ++q) {
                 const int s = q % L.nst;
                 const int round = q / L.nst;
                 if (round > 0 && !vwait(&s_empty[s], (round - 1) & 1, abort, a.hdr, 0x302)) goto producer_done;
                 unsigned char* st = smem + s * L.stage;
-                const int col0 = c * Gm::CK;
-                const int cols = min(Gm::CK, K - col0);
-                // bytes of this stage: planes, digits, and (first chunk) the slot's scales, exps, sums
-                uint32_t bytes = static_cast<uint32_t>(NMAT * kmax * NRT) * (cols / 64) * 128u +
-                                 static_cast<uint32_t>(__popc(valid)) * 2u * cols;
-                const uint32_t mrow = FMT == DPA_FMT_UNIFORM ? static_cast<uint32_t>(Gm::RB * ng * 4)
-                                                             : static_cast<uint32_t>(Gm::RB * ng * 2);
-                const int n_meta = FMT == DPA_FMT_UNIFORM ? NMAT : NMAT * kmax;
-                if (c == 0) bytes += n_meta * mrow + static_cast<uint32_t>(__popc(valid)) * 2u * L.ngp * 4u;
+                const int col0 = c * static_cast<int>(L.CK);
+                const int cols = min(static_cast<int>(L.CK), K - col0);
+                const int n_pc = NMAT * kmax * NRT;
+                const uint32_t bytes = static_cast<uint32_t>(n_pc) * (cols / 64) * 128u + n_meta * mrow;
                 if (lane == 0) {
                     fence_proxy_async();
                     mbar_arrive_expect_tx(&s_full[s], bytes);
                 }
                 __syncwarp();
                 fence_proxy_async();
-                // plane words: (m, p, rt) copies of cols/64 blocks
-                const int n_pc = NMAT * kmax * NRT;
+                // plane words: (m, p, rt) copies of the chunk's columns (2 bytes per column)
                 for (int i = lane; i < n_pc; i += 32) {
                     const int rt = i % NRT, mp = i / NRT, p = mp % kmax, m = mp / kmax;
                     const uint8_t* src = pbase + a.planes_mat_off[a.mat0 + m] + p * plane_bytes +
                                          static_cast<uint64_t>(rb * NRT + rt) * (K / 64) * 128 +
                                          static_cast<uint64_t>(col0 / 64) * 128;
-                    bulk_g2s(st + ((static_cast<size_t>(m * kMaxB + p) * NRT + rt) * (Gm::CK / 64)) * 128, src,
+                    bulk_g2s(st + ((static_cast<size_t>(m * kMaxB + p) * NRT + rt) * (L.CK / 64)) * 128, src,
                              static_cast<uint32_t>(cols / 64) * 128u, &s_full[s]);
                 }
-                // digit rows of the tokens (two per token slot)
-                if (lane < 4 * NTILE && drow >= 0) {
-                    for (int d = 0; d < 2; ++d)
-                        bulk_g2s(st + L.st_dig + static_cast<size_t>(lane * 2 + d) * L.dig_stride,
-                                 a.dig + (static_cast<size_t>(drow) * 2 + d) * K + col0, static_cast<uint32_t>(cols),
-                                 &s_full[s]);
-                }
-                if (c == 0) {
-                    const uint8_t* mbase = a.meta + static_cast<uint64_t>(e) * a.meta_per_expert;
-                    for (int i = lane; i < n_meta; i += 32) {
-                        if (FMT == DPA_FMT_UNIFORM) {
-                            bulk_g2s(sl + static_cast<size_t>(i) * mrow,
-                                     mbase + a.meta_mat_off[a.mat0 + i] + static_cast<uint64_t>(rb) * mrow, mrow,
-                                     &s_full[s]);
-                        } else {
-                            const int m = i / kmax, p = i % kmax;
-                            bulk_g2s(sl + static_cast<size_t>(i) * mrow,
-                                     mbase + a.meta_mat_off[a.mat0 + m] + static_cast<uint64_t>(p) * a.R * ng * 2 +
-                                         static_cast<uint64_t>(rb) * mrow,
-                                     mrow, &s_full[s]);
-                        }
+                // the item's scale data (every stage carries it, for the chunks that follow)
+                for (int i = lane; i < n_meta; i += 32) {
+                    const uint8_t* src;
+                    if (FMT == DPA_FMT_UNIFORM) {
+                        src = mbase + a.meta_mat_off[a.mat0 + i] + static_cast<uint64_t>(rb) * mrow;
+                    } else {
+                        const int m = i / kmax, p = i % kmax;
+                        src = mbase + a.meta_mat_off[a.mat0 + m] + static_cast<uint64_t>(p) * a.R * ng * 2 +
+                              static_cast<uint64_t>(rb) * mrow;
                     }
-                    if (lane < 4 * NTILE && drow >= 0) {
-                        bulk_g2s(sl + L.sl_exp + static_cast<size_t>(lane) * L.ngp * 4,
-                                 a.dexp + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u,
-                                 &s_full[s]);
-                        bulk_g2s(sl + L.sl_sum + static_cast<size_t>(lane) * L.ngp * 4,
-                                 a.dsum + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u,
-                                 &s_full[s]);
-                    }
+                    bulk_g2s(st + L.st_meta + static_cast<size_t>(i) * mrow, src, mrow, &s_full[s]);
                 }
                 issued_upto = q + 1;
             }
         }
     producer_done:
-        // before the CTA exits every copy it issued must have landed: wait for the last stages
+        // before the CTA exits every copy it issued must have landed: the last stages and groups
         for (int q2 = max(0, issued_upto - L.nst); q2 < issued_upto; ++q2) {
             const int s = q2 % L.nst;
             if (!mbar_try_wait(&s_full[s], (q2 / L.nst) & 1)) {
@@ -503,16 +487,45 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                     if (globaltimer() - t0 > kWaitNs) { set_error(a.hdr, DPA_ERR_DEVICE_TIMEOUT, 0x310); break; }
             }
         }
+        for (int g2 = max(0, groups_issued - 2); g2 < groups_issued; ++g2) {
+            const int slot = g2 & 1;
+            if (!mbar_try_wait(&s_gfull[slot], (g2 >> 1) & 1)) {
+                const uint64_t t0 = globaltimer();
+                while (!mbar_try_wait_suspend(&s_gfull[slot], (g2 >> 1) & 1, 10000u))
+                    if (globaltimer() - t0 > kWaitNs) { set_error(a.hdr, DPA_ERR_DEVICE_TIMEOUT, 0x311); break; }
+            }
+        }
         return;
     }
 
     // ================================ consumers ================================
     const int rt = warp / Gm::CS, cs = warp % Gm::CS;
-    int q = 0;
-    for (int n = 0, it = blockIdx.x; it < n_items; ++n, it += gridDim.x) {
-        const int slot = n & 1;
-        const unsigned char* sl = smem + L.nst * L.stage + slot * L.slot;
-        Item<NRT, NTILE, NMAT> item;
+    const int gid = lane >> 2, tq = lane & 3;
+    float* red = reinterpret_cast<float*>(smem + L.red);
+    int q = 0, gcount = 0, cur_g = -1, ni = 0;
+    const unsigned char* gs = nullptr;
+    Group<NTILE> gr;
+    for (int it = it0; it < it1; ++it, ++ni) {
+        const int gi = it / n_rb, rb = it - gi * n_rb;
+        if (gi != cur_g) {
+            if (cur_g >= 0) {   // the previous group's slot is no longer read
+                __syncwarp();
+                if (lane == 0) mbarrier_arrive(&s_gempty[(gcount - 1) & 1]);
+            }
+            const int slot = gcount & 1;
+            if (!vwait(&s_gfull[slot], (gcount >> 1) & 1, abort, a.hdr, 0x321)) return;
+            gs = smem + L.slots + slot * L.slot;
+            const int* rec = reinterpret_cast<const int*>(gs + L.sl_rec);
+            gr.kmax = rec[1];
+            gr.nt = rec[2];
+#pragma unroll
+            for (int t = 0; t < NTILE; ++t) {
+                gr.tk[t] = rec[4 + t];
+                gr.tn[t] = rec[6 + t];
+            }
+            cur_g = gi;
+            ++gcount;
+        }
         float acc[NTILE][NMAT][2];
 #pragma unroll
         for (int t = 0; t < NTILE; ++t)
@@ -521,29 +534,21 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
         for (int c = 0; c < n_chunks; ++c, ++q) {
             const int s = q % L.nst;
             if (!vwait(&s_full[s], (q / L.nst) & 1, abort, a.hdr, 0x320)) return;
-            if (c == 0) {
-                const int* tab = reinterpret_cast<const int*>(sl + L.sl_tab);
-                item.e = tab[0];
-                item.kmax = tab[1];
-                item.nt = tab[2];
-                item.rb = tab[3];
-#pragma unroll
-                for (int t = 0; t < NTILE; ++t) {
-                    item.tk[t] = tab[4 + 4 * t];
-                    item.tn[t] = tab[4 + 4 * t + 1];
-                }
-            }
-            slice_dispatch<FMT, NRT, NTILE, NMAT>(a, L, smem + s * L.stage, sl, item, c * Gm::CK, rt, cs, acc);
+            const int col0 = c * static_cast<int>(L.CK);
+            const int nbc = min(static_cast<int>(L.CK), K - col0) / 64;
+            const int b0 = (cs * nbc) / Gm::CS, b1 = ((cs + 1) * nbc) / Gm::CS;
+            slice_dispatch<FMT, NRT, NTILE, NMAT>(a, L, smem + s * L.stage, gs, gr, col0, b0, b1, rt, acc);
             __syncwarp();
             if (lane == 0) mbarrier_arrive(&s_empty[s]);
         }
-        // ---- the column slices of this row tile meet (fixed order), then the epilogue ----
-        // red_full completes once per item (the CS-1 slices arrive); red_free once per item (the
-        // summing warp has read them), so a slice writes item n's partials after item n-1's read
-        float* red = reinterpret_cast<float*>(smem + L.red);
-        if (cs > 0) {
-            if (n >= 1 && !vwait(&s_red_free[rt], (n - 1) & 1, abort, a.hdr, 0x330)) return;
-            float* dst = red + (static_cast<size_t>(rt) * (Gm::CS - 1) + (cs - 1)) * (L.red_per / 4);
+        // ---- the column slices of this row tile meet: one of them (rotating with the item)
+        // sums the partials in slice order and writes the epilogue ----
+        const int reducer = ni % Gm::CS;
+        float* part = red + static_cast<size_t>(rt * Gm::CS) * (L.red_per / 4);
+        if (cs != reducer) {
+            // the previous item's reducer must have read its partials before they are rewritten
+            if (ni >= 1 && !vwait(&s_red_free[rt], (ni - 1) & 1, abort, a.hdr, 0x330)) return;
+            float* dst = part + static_cast<size_t>(cs) * (L.red_per / 4);
 #pragma unroll
             for (int t = 0; t < NTILE; ++t)
 #pragma unroll
@@ -553,41 +558,46 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
             __syncwarp();
             if (lane == 0) mbarrier_arrive(&s_red_full[rt]);
         } else {
-            if (Gm::CS > 1 && !vwait(&s_red_full[rt], n & 1, abort, a.hdr, 0x331)) return;
-            for (int c2 = 1; c2 < Gm::CS; ++c2) {
-                const float* src = red + (static_cast<size_t>(rt) * (Gm::CS - 1) + (c2 - 1)) * (L.red_per / 4);
+            if (Gm::CS > 1 && !vwait(&s_red_full[rt], ni & 1, abort, a.hdr, 0x331)) return;
+            float sum[NTILE][NMAT][2];
+#pragma unroll
+            for (int t = 0; t < NTILE; ++t)
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) sum[t][m][rr] = 0.f;
+            for (int c2 = 0; c2 < Gm::CS; ++c2) {   // fixed order: slice 0, 1, ...
+                const float* src = part + static_cast<size_t>(c2) * (L.red_per / 4);
 #pragma unroll
                 for (int t = 0; t < NTILE; ++t)
 #pragma unroll
                     for (int m = 0; m < NMAT; ++m)
 #pragma unroll
-                        for (int rr = 0; rr < 2; ++rr) acc[t][m][rr] += src[((t * NMAT + m) * 2 + rr) * 32 + lane];
+                        for (int rr = 0; rr < 2; ++rr)
+                            sum[t][m][rr] += c2 == cs ? acc[t][m][rr] : src[((t * NMAT + m) * 2 + rr) * 32 + lane];
             }
             __syncwarp();
             if (Gm::CS > 1 && lane == 0) mbarrier_arrive(&s_red_free[rt]);
-            const int* tab = reinterpret_cast<const int*>(sl + L.sl_tab);
-            const int gid = lane >> 2, tq = lane & 3;
+            const int* rec = reinterpret_cast<const int*>(gs + L.sl_rec);
 #pragma unroll
             for (int t = 0; t < NTILE; ++t) {
-                if (t < item.nt && tq < item.tn[t]) {
-                    const int pos = tab[4 + 8 * NTILE + 4 * t + tq];
+                if (t < gr.nt && tq < gr.tn[t]) {
+                    const int pos = rec[8 + 4 * t + tq];
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
-                        const int row = item.rb * Gm::RB + rt * 16 + gid + 8 * rr;
+                        const int row = rb * Gm::RB + rt * 16 + gid + 8 * rr;
                         float v;
                         if constexpr (NMAT == 2) {
-                            const float ag = acc[t][0][rr], au = acc[t][1][rr];
+                            const float ag = sum[t][0][rr], au = sum[t][1][rr];
                             v = ag / (1.f + expf(-ag)) * au;
                         } else {
-                            v = acc[t][0][rr];
+                            v = sum[t][0][rr];
                         }
                         a.out[static_cast<size_t>(pos) * a.R + row] = v;
                     }
                 }
             }
         }
-        __syncwarp();
-        if (lane == 0) mbarrier_arrive(&s_slot_empty[slot]);
     }
 }
 
@@ -650,25 +660,34 @@ cudaError_t launch_variant(const VpArgs& a, cudaStream_t stream, int sms) {
 
 }  // namespace
 
-size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, bool multi) {
+// Variants: gate/up (two matrices) on 16-row items, down (one matrix) on 32-row items; token
+// groups of two tiles (8 tokens), or one tile (4 tokens) where the group slot would not fit.
+int vp_tiles_per_group(int K_gateup, int K_down, int G, int fmt, int B) {
+    const bool two = vlayout<1, 2, 2>(K_gateup, G, fmt, B).total <= kVpMaxSmem &&
+                     vlayout<2, 2, 1>(K_down, G, fmt, B).total <= kVpMaxSmem;
+    return two ? 2 : 1;
+}
+
+size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, int tiles_per_group) {
     if (nmat == 2)
-        return multi ? vlayout<4, 2, 2>(K, G, fmt, B).total : vlayout<1, 1, 2>(K, G, fmt, B).total;
-    return multi ? vlayout<4, 2, 1>(K, G, fmt, B).total : vlayout<4, 1, 1>(K, G, fmt, B).total;
+        return tiles_per_group == 2 ? vlayout<1, 2, 2>(K, G, fmt, B).total : vlayout<1, 1, 2>(K, G, fmt, B).total;
+    return tiles_per_group == 2 ? vlayout<2, 2, 1>(K, G, fmt, B).total : vlayout<2, 1, 1>(K, G, fmt, B).total;
 }
 
 cudaError_t launch_vp_gemv(const VpArgs& a, cudaStream_t stream, int sms) {
+    const bool two = a.tiles_per_group == 2;
     if (a.nmat == 2) {
         if (a.fmt == DPA_FMT_UNIFORM)
-            return a.multi ? launch_variant<DPA_FMT_UNIFORM, 4, 2, 2>(a, stream, sms)
-                           : launch_variant<DPA_FMT_UNIFORM, 1, 1, 2>(a, stream, sms);
-        return a.multi ? launch_variant<DPA_FMT_BCQ, 4, 2, 2>(a, stream, sms)
-                       : launch_variant<DPA_FMT_BCQ, 1, 1, 2>(a, stream, sms);
+            return two ? launch_variant<DPA_FMT_UNIFORM, 1, 2, 2>(a, stream, sms)
+                       : launch_variant<DPA_FMT_UNIFORM, 1, 1, 2>(a, stream, sms);
+        return two ? launch_variant<DPA_FMT_BCQ, 1, 2, 2>(a, stream, sms)
+                   : launch_variant<DPA_FMT_BCQ, 1, 1, 2>(a, stream, sms);
     }
     if (a.fmt == DPA_FMT_UNIFORM)
-        return a.multi ? launch_variant<DPA_FMT_UNIFORM, 4, 2, 1>(a, stream, sms)
-                       : launch_variant<DPA_FMT_UNIFORM, 4, 1, 1>(a, stream, sms);
-    return a.multi ? launch_variant<DPA_FMT_BCQ, 4, 2, 1>(a, stream, sms)
-                   : launch_variant<DPA_FMT_BCQ, 4, 1, 1>(a, stream, sms);
+        return two ? launch_variant<DPA_FMT_UNIFORM, 2, 2, 1>(a, stream, sms)
+                   : launch_variant<DPA_FMT_UNIFORM, 2, 1, 1>(a, stream, sms);
+    return two ? launch_variant<DPA_FMT_BCQ, 2, 2, 1>(a, stream, sms)
+               : launch_variant<DPA_FMT_BCQ, 2, 1, 1>(a, stream, sms);
 }
 
 cudaError_t launch_digits(const DigitArgs& d, cudaStream_t stream) {

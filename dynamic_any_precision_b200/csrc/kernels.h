@@ -29,6 +29,11 @@ struct RouteArgs {
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms = 148);
 
+// A token group of the expert GEMV: [0] expert, [1] kmax over the group, [2] tiles (<= 2),
+// [4 + t] plane count of tile t, [6 + t] pairs in tile t (<= 4), [8 + 4t + q] grouped position
+// (output row) of pair q of tile t, [16 + 4t + q] its token; unused slots hold -1.
+constexpr int kVRecInts = 32;
+
 struct AllocArgs {
     const double* rtable;     // [E][B]
     const int32_t* idx;       // [T][K]
@@ -49,11 +54,10 @@ struct AllocArgs {
     WsHeader* hdr;
     int policy;               // DPA_ALLOC_LAGRANGE, DPA_ALLOC_UNIFORM or DPA_ALLOC_THRESHOLD
     const double* threshold;  // device scalar (DPA_ALLOC_THRESHOLD)
-    // work list of the pipelined expert GEMV (nullptr: not written): tiles of up to 4 pairs of
-    // one (expert, k) class, {k, pos0, n, 0}, and token groups of up to vtiles_per_group tiles of
-    // one expert, {expert, kmax over the group, n tiles, first tile}; count in hdr->n_vgroups
-    int4* vtiles;             // [P/4 + E*nk]
-    int4* vgroups;            // [P/4 + E*nk]
+    // work list of the pipelined expert GEMV (nullptr: not written): token groups of up to
+    // vtiles_per_group (<= 2) tiles of up to 4 pairs of one (expert, k) class, as records of
+    // kVRecInts ints (see kVRec*); count in hdr->n_vgroups
+    int32_t* vrec;            // [P/4 + E*nk][kVRecInts]
     int vtiles_per_group;
     const uint8_t* expert_k;  // [E] plane count per expert (DPA_ALLOC_EXPERT_TABLE)
 };
@@ -136,10 +140,8 @@ struct VpArgs {
     int fmt, B, G;
     int R, K;                 // rows and columns of each matrix of this launch
     int mat0, nmat;           // first matrix (0: gate, up; 2: down) and the matrix count
-    int multi;                // 1: 64-row items, groups of up to 4 tiles; 0: the small-batch variant
-    const int4* vgroups;      // {expert, kmax, n tiles, first tile}, count in hdr->n_vgroups
-    const int4* vtiles;       // {k, pos0, n, 0}
-    const int32_t* pos_tok;   // [P] token of each grouped position
+    int tiles_per_group;      // 1 or 2 (the allocation's grouping)
+    const int32_t* vrec;      // token group records [n_vgroups][kVRecInts], count in hdr->n_vgroups
     const int8_t* dig;        // activation digit rows [rows][2][K] (permuted 64-column blocks)
     const int32_t* dexp;      // [rows][ngp] group exponents
     const int32_t* dsum;      // [rows][ngp] group sums of the fixed-point values
@@ -149,8 +151,10 @@ struct VpArgs {
     int max_groups;           // host bound of the token groups
 };
 cudaError_t launch_vp_gemv(const VpArgs& a, cudaStream_t stream, int sms);
-// dynamic shared memory of one CTA of a variant (multi: 64-row items, small: the other)
-size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, bool multi);
+// tiles per token group the layer's shapes allow (2 where the group slots fit, else 1)
+int vp_tiles_per_group(int K_gateup, int K_down, int G, int fmt, int B);
+// dynamic shared memory of one CTA of a variant
+size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, int tiles_per_group);
 constexpr size_t kVpMaxSmem = 227 * 1024;
 
 // Fixed-point digits of activation rows (x as bf16, or h as fp32), per group of G columns:

@@ -25,7 +25,10 @@ constexpr int kRouteWarps = 8;
 // Router-row uint4 loads a lane issues at once (PF, a template parameter of the per-logit kernel):
 // the number a lane needs in total when that is at most 8, so that no unrolled slot idles.
 constexpr int16_t kNoBit = 0x3FFF;   // lowest-set-bit marker of a zero element
-constexpr int kRouteTiledMinTokens = 128;   // from here on the logits run as a tiled GEMM
+#ifndef DPA_ROUTE_TILED_MIN_TOKENS
+#define DPA_ROUTE_TILED_MIN_TOKENS 128
+#endif
+constexpr int kRouteTiledMinTokens = DPA_ROUTE_TILED_MIN_TOKENS;   // from here on the logits run as a tiled GEMM
 constexpr int kMaxLsbBlocks = 256;          // H <= 16384 on the tiled path
 
 // ---------------- fp64 exp (see header comment) ----------------
@@ -244,7 +247,8 @@ __device__ void select_topk_gates(const RouteArgs& a, int t, unsigned char* smem
     __syncthreads();
     const int K = a.K;
     // rank of each expert = number of experts before it (descending logit, ties to the lower
-    // id; NaN ranks last). Q threads share a candidate, each counting over 1/Q of the experts.
+    // id; NaN ranks last, NaNs by id). Q threads share a candidate, each counting over 1/Q of
+    // the experts. The ranks are a permutation of 0..E-1, so s_sel[0..K) is always written.
     int Q = 1;
     while (Q < 32 && Q * 2 * E <= static_cast<int>(blockDim.x)) Q *= 2;
     const int chunk = (E + Q - 1) / Q;
@@ -288,7 +292,16 @@ __device__ void select_topk_gates(const RouteArgs& a, int t, unsigned char* smem
                 }
                 rank = (r0 + r1) + (r2 + r3);
             } else {
-                rank = q == 0 ? E : 0;
+                // a NaN logit (a non-finite token or router weight, flagged as invalid input)
+                // ranks after every number and after the NaNs of lower id, so that the ranks
+                // stay a permutation and every selected slot holds a valid expert id
+                const int j0 = q * chunk, j1 = min(E, (q + 1) * chunk);
+                int r = 0;
+                for (int j = j0; j < j1; ++j) {
+                    const double w = vals[j];
+                    r += (w == w || j < c) ? 1 : 0;
+                }
+                rank = r;
             }
         }
         for (int o = 1; o < Q; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);

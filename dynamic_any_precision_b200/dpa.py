@@ -61,7 +61,8 @@ ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD, ALLOC_EXPERT_TABLE = 0, 1, 2, 3
 EXPORTED = ("dpa_encoded_sizes", "dpa_encode", "dpa_export_codes", "dpa_export_meta", "dpa_route",
             "dpa_allocate", "dpa_allocate_ex", "dpa_calibrate_threshold", "dpa_forward_workspace_size",
             "dpa_moe_forward", "dpa_device_status", "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm",
-            "dpa_debug_timeout_probe", "dpa_distortion_tensor", "dpa_profile_prefill", "dpa_solve_expert_rates")
+            "dpa_debug_timeout_probe", "dpa_distortion_tensor", "dpa_profile_prefill", "dpa_solve_expert_rates",
+            "dpa_stream_prefixes")
 
 _lib = None
 
@@ -93,6 +94,7 @@ def lib() -> ctypes.CDLL:
     L.dpa_moe_forward.argtypes = [P(LayerDesc), P(LayerWeights), vp, i32, vp, vp, P(Aux), vp, sz, vp]
     L.dpa_device_status.argtypes = [vp, vp]
     L.dpa_debug_timeout_probe.argtypes = [vp, sz, i32, ctypes.c_uint64, vp]
+    L.dpa_stream_prefixes.argtypes = [P(LayerDesc), vp, vp, vp, vp, i32, vp, vp, P(ctypes.c_uint64), vp]
     L.dpa_residual_rmsnorm.argtypes = [vp, vp, i32, i32, vp, vp]
     L.dpa_status_string.argtypes = [i32]
     L.dpa_status_string.restype = ctypes.c_char_p
@@ -334,6 +336,19 @@ def residual_rmsnorm(h, x, y=None, stream=None):
     T, H = h.shape
     _check(lib().dpa_residual_rmsnorm(_dptr(y), _dptr(h), T, H, _dptr(x), _stream(stream)), "dpa_residual_rmsnorm")
     return x
+
+
+def stream_prefixes(desc: LayerDesc, host_planes, host_meta, experts, kplanes, dev_planes, dev_meta,
+                    stream=None) -> int:
+    """Copy the first kplanes[i] planes (and their scale data) of experts[i] from the host
+    layer (pinned torch uint8 tensors) to the device layer. Returns the bytes issued."""
+    ex = np.ascontiguousarray(experts, dtype=np.int32)
+    kp = np.ascontiguousarray(kplanes, dtype=np.uint8)
+    nbytes = ctypes.c_uint64(0)
+    _check(lib().dpa_stream_prefixes(ctypes.byref(desc), host_planes.data_ptr(), host_meta.data_ptr(), _ptr(ex),
+                                     _ptr(kp), int(ex.size), _dptr(dev_planes), _dptr(dev_meta), ctypes.byref(nbytes),
+                                     _stream(stream)), "dpa_stream_prefixes")
+    return int(nbytes.value)
 
 
 def device_status(ws, stream=None) -> int:

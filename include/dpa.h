@@ -354,6 +354,23 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* desc, const dpa_layer_weights* 
  * RMSNorm (unit weight) between the layers. */
 dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidden, void* x, void* stream);
 
+/* Prefix streaming of offloaded experts (host -> device). Defined by: MatMoE, review section on
+ * the SSD-offloading regime (nested bitplanes let an offloaded expert's low-precision prefix be
+ * fetched on its own); DuoRate, Abstract (a weight stream readable by prefix).
+ * For each listed expert experts[i] (host int32 [n]) copies the first kplanes[i] (host uint8 [n],
+ * 1..bits) planes of its gate, up and down matrices from host_planes to the same offsets of
+ * dev_planes - one contiguous prefix per matrix, one cudaMemcpyAsync each - and the scale data
+ * those planes need from host_meta to dev_meta (uniform: the expert's scales and zeros;
+ * binary-coded: the first kplanes[i] alpha planes of each matrix). host_* are encoded layers
+ * (dpa_encode's layout), ideally page-locked so that the copies are asynchronous; dev_* are
+ * device buffers of the same sizes. The bytes issued are written to *bytes_out (may be NULL).
+ * After the copies complete, a forward whose pairs read at most kplanes[i] planes of expert
+ * experts[i] reads only streamed bytes. Errors: DPA_ERR_INVALID_ARG for NULL pointers or an
+ * expert id or plane count out of range (nothing issued). */
+dpa_status dpa_stream_prefixes(const dpa_layer_desc* desc, const void* host_planes, const void* host_meta,
+                               const int32_t* experts, const uint8_t* kplanes, int n, void* dev_planes,
+                               void* dev_meta, uint64_t* bytes_out, void* stream);
+
 /* Test support for the device-side failure handling (the pages have no counterpart).
  * Runs one of the library's bounded device waits against a barrier that nothing completes,
  * with a limit of limit_ns (1e3 .. 2e9 ns) instead of the kernels' 200 ms:

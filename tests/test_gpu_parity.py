@@ -14,9 +14,21 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-3
 
 
-def within_tol(got, ref, tol=TOL):
+def half_ulp_bf16(v):
+    """Half the spacing of bf16 values at |v| (8 significant bits): the most that rounding an
+    exact result to the bf16 output format can move it."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.where(a > 0, np.ldexp(1.0, (e - 8).astype(int)), 0.0)
+
+
+def within_tol(got, ref, tol=TOL, bf16_out=False):
+    """|got - ref| <= tol * (1 + |ref|); for bf16 layer outputs the format's own rounding (half a
+    bf16 ulp of ref) comes on top: the fp32 result meets the tolerance, then it is rounded."""
     err = np.abs(got - ref)
     bound = tol * (1.0 + np.abs(ref))
+    if bf16_out:
+        bound = bound + half_ulp_bf16(ref)
     return bool(np.all(err <= bound)), float(np.max(err / bound))
 
 
@@ -74,7 +86,7 @@ def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None, p
     assert np.array_equal(aux["k"].astype(np.int64), ref["k"])
     assert aux["lambda"][0] == ref["lambda"]
     rows = np.arange(x_bits.shape[0]) if token_subset is None else np.asarray(token_subset)
-    ok, worst = within_tol(y[rows], y_ref[rows])
+    ok, worst = within_tol(y[rows], y_ref[rows], bf16_out=True)
     assert ok, f"output tolerance exceeded: worst err/bound = {worst}"
     if sample_pairs is not None:
         ref_o = pair_outputs(shape, x_bits, ref, sample_pairs)
@@ -300,13 +312,13 @@ def test_prefix_property_mixed_k_poisoned(shape, T, target):
 
 
 def test_forward_activation_groups_spanning_many_binades():
-    # the expert kernels hold each scale group of activations as 22-bit fixed point under the
-    # group's largest exponent; groups spanning ~40 binades (values 2^-30 .. 2^9) lose only
+    # the expert kernels hold each scale group of activations as 15-bit fixed point under the
+    # group's largest exponent; groups spanning ~40 binades (magnitudes 2^-38 .. 2) lose only
     # digits far below the tolerance
     shape = W.TINY
     rng = np.random.default_rng(77)
     T, H = 6, shape.hidden
-    mag = np.exp2(rng.integers(-30, 10, size=(T, H)).astype(np.float64))
+    mag = np.exp2(rng.integers(-38, 1, size=(T, H)).astype(np.float64))
     x = (mag * np.sign(rng.standard_normal((T, H))) * (1 + rng.random((T, H)))).astype(np.float32)
     xb = W.f32_to_bf16_bits(x)
     for target in (2.0, 3.0, 4.0):

@@ -53,7 +53,7 @@ def test_tc_full_prefill_against_oracle(target):
     assert aux["lambda"][0] == ref["lambda"]
     if target < 4.0:
         assert len(np.unique(aux["k"])) > 1
-    ok, worst = within_tol(y[subset], y_ref[subset])
+    ok, worst = within_tol(y[subset], y_ref[subset], bf16_out=True)
     assert ok, f"output tolerance exceeded: worst err/bound = {worst}"
     for (t, j), o in ref["pair_out"].items():
         ok, worst = within_tol(aux["pair_out"][t, j].astype(np.float64), o)
