@@ -363,7 +363,11 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
     using Gm = Geo<NRT>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ uint64_t s_full[kMaxStages], s_empty[kMaxStages], s_gfull[2], s_gempty[2];
-    __shared__ uint64_t s_red_full[NRT], s_red_free[NRT];
+    // the reduction's "partials written" barrier alternates with the item's parity: warps run up
+    // to a ring's depth apart, so when an item's reducer arrives one shared barrier could be in
+    // the previous item's phase, this one's, or the next one's, which a parity wait cannot tell
+    // apart; with two, each is at most one phase from the one awaited
+    __shared__ uint64_t s_red_full[NRT][2], s_red_free[NRT];
     __shared__ int s_abort;
     const VLayout L = vlayout<NRT, NTILE, NMAT>(a.K, a.G, FMT, a.B);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -377,7 +381,8 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
             mbar_init(&s_gempty[b], kCW);
         }
         for (int r = 0; r < NRT; ++r) {
-            mbar_init(&s_red_full[r], Gm::CS - 1);
+            mbar_init(&s_red_full[r][0], Gm::CS - 1);
+            mbar_init(&s_red_full[r][1], Gm::CS - 1);
             mbar_init(&s_red_free[r], 1);
         }
         s_abort = 0;
@@ -556,9 +561,9 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) dst[((t * NMAT + m) * 2 + rr) * 32 + lane] = acc[t][m][rr];
             __syncwarp();
-            if (lane == 0) mbarrier_arrive(&s_red_full[rt]);
+            if (lane == 0) mbarrier_arrive(&s_red_full[rt][ni & 1]);
         } else {
-            if (Gm::CS > 1 && !vwait(&s_red_full[rt], ni & 1, abort, a.hdr, 0x331)) return;
+            if (Gm::CS > 1 && !vwait(&s_red_full[rt][ni & 1], (ni >> 1) & 1, abort, a.hdr, 0x331)) return;
             float sum[NTILE][NMAT][2];
 #pragma unroll
             for (int t = 0; t < NTILE; ++t)

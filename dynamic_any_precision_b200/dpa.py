@@ -351,6 +351,15 @@ def stream_prefixes(desc: LayerDesc, host_planes, host_meta, experts, kplanes, d
     return int(nbytes.value)
 
 
+def device_error_detail(ws) -> Tuple[int, int]:
+    """(code, detail) of the device error flag in ws, without clearing it (synchronises). The
+    detail says which check or wait recorded it."""
+    import torch
+    torch.cuda.synchronize(ws.device)
+    v = ws[:8].cpu().numpy().view(np.uint32)
+    return int(v[0]), int(v[1])
+
+
 def device_status(ws, stream=None) -> int:
     """Synchronise, read and clear the device error flag; returns the status code."""
     return int(lib().dpa_device_status(_dptr(ws), _stream(stream)))

@@ -71,8 +71,9 @@ class GpuLayer:
         if with_pairs:
             aux["pair_out"] = torch.empty((T, K, self.shape.hidden), dtype=torch.float32, device="cuda")
         y = dpa.moe_forward(self.layer, x, tg, ws, aux=aux)
+        detail = dpa.device_error_detail(ws)
         st = dpa.device_status(ws)
-        assert st == 0, dpa.STATUS_NAMES.get(st, st)
+        assert st == 0, (dpa.STATUS_NAMES.get(st, st), hex(detail[1]))
         out = {k: v.cpu().numpy() for k, v in aux.items() if k != "expert_path"}
         return bits_to_f64(y), out, ws
 
