@@ -34,8 +34,8 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 
 // ---- workspace layout ----
 struct WsLayout {
-    size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xexp, xsum, h, out_pair, sh_h, sh_out,
-        desc, tiles, gtiles, postok, coop, rstats, xperm, hdig, hexp, hsum, vrec, total;
+    size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xscl, xfsx, h, out_pair, sh_h, sh_out,
+        desc, tiles, gtiles, postok, coop, rstats, rpart, xperm, hdig, hscl, hfsx, vrec, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -63,8 +63,8 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     const size_t ngp_h = ((H / d->group) + 3) & ~static_cast<size_t>(3);
     const size_t ngp_i = ((I / d->group) + 3) & ~static_cast<size_t>(3);
     L.xdig = take(2 * static_cast<size_t>(T) * H);
-    L.xexp = take(4 * static_cast<size_t>(T) * ngp_h);
-    L.xsum = take(4 * static_cast<size_t>(T) * ngp_h);
+    L.xscl = take(4 * static_cast<size_t>(T) * ngp_h);
+    L.xfsx = take(4 * static_cast<size_t>(T) * ngp_h);
     L.h = take(4 * P * I);
     L.out_pair = take(4 * P * H);
     L.sh_h = take(4 * static_cast<size_t>(T) * d->n_shared * I);
@@ -75,10 +75,11 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.postok = take(4 * P);
     L.coop = take(sizeof(dpa::CoopSync));
     L.rstats = take((8 + 2 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 16);
+    L.rpart = take(8 * dpa::route_partial_doubles(T, static_cast<int>(E), static_cast<int>(H)));
     L.xperm = take(2 * P * H);
     L.hdig = take(2 * P * I);
-    L.hexp = take(4 * P * ngp_i);
-    L.hsum = take(4 * P * ngp_i);
+    L.hscl = take(4 * P * ngp_i);
+    L.hfsx = take(4 * P * ngp_i);
     L.vrec = take(4 * dpa::kVRecInts * (P / 4 + E * nk + 1));
     L.total = off;
     return L;
@@ -148,6 +149,7 @@ static void set_route_stats(dpa::RouteArgs& r, void* ws, const WsLayout& L, int 
     const size_t lsb_off = (8 * (static_cast<size_t>(T) + E) + 15) & ~static_cast<size_t>(15);
     r.lsb_x = reinterpret_cast<int16_t*>(base + lsb_off);   // 16-byte aligned rows of H/64 entries
     r.lsb_w = r.lsb_x + static_cast<size_t>(T) * (r.H / 64);
+    r.part = at<double>(ws, L.rpart);
 }
 
 extern "C" {
@@ -436,8 +438,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     ra.gate = gate;
     ra.counters = at<unsigned>(ws, L.counters);
     ra.xdig = use_tc ? nullptr : at<int8_t>(ws, L.xdig);   // the tensor-core path reads x directly
-    ra.xexp = at<int32_t>(ws, L.xexp);
-    ra.xsum = at<int32_t>(ws, L.xsum);
+    ra.xscl = at<float>(ws, L.xscl);
+    ra.xfsx = at<float>(ws, L.xfsx);
     ra.hdr = hdr;
     set_route_stats(ra, ws, L, T, d->n_experts);
     if (dpa::launch_route(ra, s, num_sms_current()) != cudaSuccess) return DPA_ERR_CUDA;
@@ -528,8 +530,8 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     va.mat0 = 0;
     va.nmat = 2;
     va.dig = at<int8_t>(ws, L.xdig);
-    va.dexp = at<int32_t>(ws, L.xexp);
-    va.dsum = at<int32_t>(ws, L.xsum);
+    va.dscl = at<float>(ws, L.xscl);
+    va.dfsx = at<float>(ws, L.xfsx);
     va.dig_by_token = 1;
     va.out = at<float>(ws, L.h);
     if (dpa::launch_vp_gemv(va, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
@@ -542,16 +544,16 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     da.K = d->inter;
     da.G = d->group;
     da.dig = at<int8_t>(ws, L.hdig);
-    da.dexp = at<int32_t>(ws, L.hexp);
-    da.dsum = at<int32_t>(ws, L.hsum);
+    da.dscl = at<float>(ws, L.hscl);
+    da.dfsx = at<float>(ws, L.hfsx);
     if (dpa::launch_digits(da, s) != cudaSuccess) return DPA_ERR_CUDA;
     va.R = d->hidden;
     va.K = d->inter;
     va.mat0 = 2;
     va.nmat = 1;
     va.dig = at<int8_t>(ws, L.hdig);
-    va.dexp = at<int32_t>(ws, L.hexp);
-    va.dsum = at<int32_t>(ws, L.hsum);
+    va.dscl = at<float>(ws, L.hscl);
+    va.dfsx = at<float>(ws, L.hfsx);
     va.dig_by_token = 0;
     va.out = at<float>(ws, L.out_pair);
     if (dpa::launch_vp_gemv(va, s, sms) != cudaSuccess) return DPA_ERR_CUDA;

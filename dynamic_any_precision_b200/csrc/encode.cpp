@@ -80,13 +80,25 @@ struct Mat {
 
 // Place the code bits of weight (row, col) of one matrix into its planes.
 inline void set_code(uint32_t* mat_planes, uint64_t plane_words, int R, int C, int row, int col,
-                     unsigned code, int B) {
-    const dpa_layout::BitPos bp = dpa_layout::bit_position(C, row, col);
+                     unsigned code, int B, bool uniform) {
     for (int p = 0; p < B; ++p) {
-        if ((code >> (B - 1 - p)) & 1u)
+        if ((code >> (B - 1 - p)) & 1u) {
+            const dpa_layout::BitPos bp = dpa_layout::bit_position(C, row, col, p, B, uniform);
             mat_planes[static_cast<uint64_t>(p) * plane_words + bp.word] |= (1u << bp.bit);
+        }
     }
     (void)R;
+}
+
+// The code of weight (row, col) read back from its planes.
+inline unsigned get_code(const uint32_t* mat_planes, uint64_t plane_words, int C, int row, int col, int B,
+                         bool uniform) {
+    unsigned code = 0;
+    for (int p = 0; p < B; ++p) {
+        const dpa_layout::BitPos bp = dpa_layout::bit_position(C, row, col, p, B, uniform);
+        code |= ((mat_planes[static_cast<uint64_t>(p) * plane_words + bp.word] >> bp.bit) & 1u) << (B - 1 - p);
+    }
+    return code;
 }
 
 struct EncodeJob {
@@ -134,7 +146,7 @@ bool encode_uniform_matrix(const Mat& m, int B, int G, uint32_t* mat_planes, uin
             }
         }
         for (int c = 0; c < m.C; ++c) {
-            set_code(mat_planes, plane_words, m.R, m.C, r, c, q_row[c], B);
+            set_code(mat_planes, plane_words, m.R, m.C, r, c, q_row[c], B, true);
             const double w = wr[c];
             const double s = s_row[c / G], z = z_row[c / G];
             for (int k = 1; k <= B; ++k) {
@@ -181,7 +193,7 @@ bool encode_bcq_matrix(const Mat& m, int B, int G, uint32_t* mat_planes, uint16_
             }
         }
         for (int c = 0; c < m.C; ++c) {
-            set_code(mat_planes, plane_words, m.R, m.C, r, c, code[c], B);
+            set_code(mat_planes, plane_words, m.R, m.C, r, c, code[c], B, false);
             const double w = wr[c];
             for (int k = 1; k <= B; ++k) {
                 double what = 0.0;
@@ -272,10 +284,7 @@ bool distortion_one_expert(const dpa_layer_desc& d, const dpa_sizes& sz, int e, 
                                                                sz.meta_matrix_offset[m]);
         for (int r = 0; r < I; ++r) {
             for (int c = 0; c < H; ++c) {
-                const dpa_layout::BitPos bp = dpa_layout::bit_position(H, r, c);
-                unsigned code = 0;
-                for (int p = 0; p < B; ++p)
-                    code |= ((mp[static_cast<uint64_t>(p) * plane_words + bp.word] >> bp.bit) & 1u) << (B - 1 - p);
+                const unsigned code = get_code(mp, plane_words, H, r, c, B, d.format == DPA_FMT_UNIFORM);
                 const double wv = w[static_cast<uint64_t>(r) * H + c];
                 for (int k = 1; k <= B; ++k) {
                     double what;
@@ -357,11 +366,8 @@ extern "C" dpa_status dpa_export_codes(const dpa_layer_desc* desc, const void* p
     const uint64_t plane_words = static_cast<uint64_t>(R) * C / 32;
     for (int r = 0; r < R; ++r) {
         for (int c = 0; c < C; ++c) {
-            const dpa_layout::BitPos bp = dpa_layout::bit_position(C, r, c);
-            unsigned code = 0;
-            for (int p = 0; p < B; ++p)
-                code |= ((mp[static_cast<uint64_t>(p) * plane_words + bp.word] >> bp.bit) & 1u) << (B - 1 - p);
-            codes[static_cast<uint64_t>(r) * C + c] = static_cast<uint8_t>(code);
+            codes[static_cast<uint64_t>(r) * C + c] =
+                static_cast<uint8_t>(get_code(mp, plane_words, C, r, c, B, desc->format == DPA_FMT_UNIFORM));
         }
     }
     return DPA_OK;

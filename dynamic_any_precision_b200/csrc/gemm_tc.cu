@@ -323,14 +323,18 @@ __device__ __forceinline__ void decode_stage(const unsigned char* sp, unsigned c
     const int R0 = 16 * i + g8, R1 = R0 + 8;
 #pragma unroll
     for (int rho = 0; rho < 4; ++rho) {
-        // nibble m of N0 / N1 = code bits (plane 0 = MSB) at bit 4m + rho of lanes 2w / 2w+1
-        uint32_t N0 = 0u, N1 = 0u;
+        // nibble m of N0 / N1 = the code (plane 0 = MSB) at position rho of lanes 2w / 2w+1: in
+        // plane pl that bit sits at 4m + (B-1-pl) - rho (mod 32), so the planes merge under fixed
+        // masks and one rotation by rho puts every nibble in place (planes >= k read as zero)
+        uint32_t N0 = wx[0], N1 = wy[0];
 #pragma unroll
-        for (int pl = 0; pl < B; ++pl) {
-            const int t = B - 1 - pl;
-            N0 |= (t >= rho ? (wx[pl] << (t - rho)) : (wx[pl] >> (rho - t))) & (0x11111111u << t);
-            N1 |= (t >= rho ? (wy[pl] << (t - rho)) : (wy[pl] >> (rho - t))) & (0x11111111u << t);
+        for (int pl = 1; pl < B; ++pl) {
+            const uint32_t M = 0x11111111u << ((B - 1 - pl - rho) & 3);
+            N0 = (N0 & ~M) | (wx[pl] & M);
+            N1 = (N1 & ~M) | (wy[pl] & M);
         }
+        N0 = __funnelshift_l(N0, N0, rho);
+        N1 = __funnelshift_l(N1, N1, rho);
         const int R = (rho & 1) ? R1 : R0;
         const uint32_t Kr = (rho & 1) ? K1 : K0;
 #pragma unroll

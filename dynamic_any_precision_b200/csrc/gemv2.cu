@@ -43,7 +43,11 @@ constexpr int kCW = 8;                        // consumer warps
 constexpr int kVThreads = (kCW + 1) * 32;     // + the producer warp
 constexpr int kMaxStages = 8;                 // ring depth: as many stages as shared memory holds
 constexpr int kMaxB = 4;
-constexpr int kMaxChunk = 2048;               // columns per chunk
+constexpr int kMaxChunk = 1024;               // columns per chunk
+// Row tiles (16 rows each) per item: the larger where the ring and group slots fit in shared
+// memory, else the smaller (wide matrices, whose scale data and digit rows take more room).
+constexpr int kGuNRT = 2, kGuNRTSmall = 1;    // gate/up: 32 (16) rows, 4 (8) column slices
+constexpr int kDnNRT = 4, kDnNRTSmall = 2;    // down: 64 (32) rows, 2 (4) column slices
 constexpr int kDigPad = 64;                   // bytes of padding per staged digit row (banks)
 
 template <int NRT>
@@ -58,7 +62,7 @@ __host__ __device__ inline size_t al128(size_t v) { return (v + 127) & ~static_c
 struct VLayout {                              // byte offsets in dynamic shared memory (< 227 KB)
     uint32_t CK;                              // columns per chunk
     uint32_t stage, st_meta;                  // per stage: planes at 0, then the item's scale data
-    uint32_t slot, sl_exp, sl_sum, sl_rec;    // per group slot: digits at 0, exps, sums, record
+    uint32_t slot, sl_exp, sl_sum, sl_rec;    // per group slot: digits at 0, scales, scaled sums, record
     uint32_t dig_stride;                      // bytes per staged digit row (K + pad)
     uint32_t slots, red, red_per;             // group slots' offset; reduction buffer
     uint32_t total;
@@ -112,37 +116,44 @@ __device__ __forceinline__ bool vwait(uint64_t* bar, uint32_t parity, volatile i
     return mbar_wait_abortable(bar, parity, abort, hdr, where);
 }
 
-// ---- nibble assembly (as in the plane layout of dpa.h: bit 4m + rho of a lane's word) ----
-template <int RHO, int T>
-__device__ __forceinline__ uint32_t nibs(uint32_t w) {
-    uint32_t v;
-    if constexpr (T >= RHO) v = w << (T - RHO);
-    else v = w >> (RHO - T);
-    return v & (0x11111111u << T);
+// ---- uniform codes: plane merge (the plane layout of layout.h: in plane p, position rho of
+// nibble m sits at bit 4m + (B-1-p) - rho, mod 32) ----
+// The words of planes [0, KM) merged with fixed masks: bit (4m + T - RHO) mod 32 comes from the
+// plane whose code bit is T. Rotating the result left by RHO gives the register of 8 codes of
+// position RHO (nibble m = code m); positions of planes >= KM hold plane 0's bits, which the
+// level mask of a k <= KM read removes.
+template <int B, int KM, int RHO>
+__device__ __forceinline__ uint32_t merge_planes(const uint32_t (&w)[kMaxB]) {
+    uint32_t x = w[0];
+#pragma unroll
+    for (int p = 1; p < KM; ++p) {
+        const uint32_t M = 0x11111111u << ((B - 1 - p - RHO) & 3);
+        x = (x & ~M) | (w[p] & M);
+    }
+    return x;
 }
-template <int T>
-__device__ __forceinline__ void add_plane(uint32_t (&R)[4], uint32_t w) {
-    R[0] |= nibs<0, T>(w);
-    R[1] |= nibs<1, T>(w);
-    R[2] |= nibs<2, T>(w);
-    R[3] |= nibs<3, T>(w);
-}
-// planes [0, kmax) of one lane's words (plane p at w[p]); code bit of plane p = B-1-p
-template <int B>
-__device__ __forceinline__ void assemble(uint32_t (&R)[4], const uint32_t (&w)[kMaxB], int kmax) {
-    R[0] = R[1] = R[2] = R[3] = 0u;
-    if constexpr (B >= 1) add_plane<B - 1>(R, w[0]);
-    if constexpr (B >= 2) if (kmax > 1) add_plane<B - 2>(R, w[1]);
-    if constexpr (B >= 3) if (kmax > 2) add_plane<B - 3>(R, w[2]);
-    if constexpr (B >= 4) if (kmax > 3) add_plane<0>(R, w[3]);
+__device__ __forceinline__ uint32_t rotl(uint32_t x, int s) { return __funnelshift_l(x, x, s); }
+__device__ __forceinline__ uint32_t rotr(uint32_t x, int s) { return __funnelshift_r(x, x, s); }
+// Codes of position rho, unmasked: lo[rho] holds nibble 2b in the low half of byte b, hi[rho]
+// nibble 2b+1 (the A bytes of the block's first and second 32-column MMA).
+template <int B, int KM>
+__device__ __forceinline__ void decode_uniform(uint32_t (&lo)[4], uint32_t (&hi)[4], const uint32_t (&w)[kMaxB]) {
+    const uint32_t x0 = merge_planes<B, KM, 0>(w), x1 = merge_planes<B, KM, 1>(w);
+    const uint32_t x2 = merge_planes<B, KM, 2>(w), x3 = merge_planes<B, KM, 3>(w);
+    lo[0] = x0;
+    hi[0] = rotr(x0, 4);
+    lo[1] = rotl(x1, 1);
+    hi[1] = rotr(x1, 3);
+    lo[2] = rotl(x2, 2);
+    hi[2] = rotr(x2, 2);
+    lo[3] = rotl(x3, 3);
+    hi[3] = rotr(x3, 1);
 }
 // the codes of a k-plane read: the top k of B bits of every nibble, in the low nibble of a byte
-__device__ __forceinline__ uint32_t level_mask(int B, int k) {
+__host__ __device__ inline uint32_t level_mask(int B, int k) {
     const uint32_t nib = ((1u << k) - 1u) << (B - k);
     return 0x0F0F0F0Fu & (nib * 0x01010101u);
 }
-
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((e + 127) << 23); }
 
 // ---- B operand: the lane's 16 digit bytes of one 64-column block (one 16-byte load) ----
 __device__ __forceinline__ uint4 lds128(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
@@ -152,62 +163,75 @@ template <int NTILE>
 struct Group {
     int kmax, nt;
     int tk[NTILE], tn[NTILE];
+    uint32_t mk[NTILE];   // uniform codes: level mask of the tile's plane count
+    float ck[NTILE];      // uniform codes: compensation constant c_k = (2^(B-k) - 1) / 2
 };
 
+// Where a slice's blocks fall in the scale groups: the first block's group and its index in
+// the group (one division per slice; the block loop only counts).
+struct SlicePos {
+    int g, j;
+};
+__device__ __forceinline__ SlicePos slice_pos(int col0, int b0, int bpg) {
+    const int blk = col0 / 64 + b0;
+    SlicePos sp;
+    sp.g = blk / bpg;
+    sp.j = blk - sp.g * bpg;
+    return sp;
+}
+
 // ---------------------------------------------------------------------------------------
-// consumer: one column slice of one chunk, uniform codes. Blocks [b0, b1) of the chunk; the
-// group slot holds the tokens' digits for every column (col0 = the chunk's first column).
+// consumer: one column slice of one chunk, uniform codes, KM = the group's kmax planes and NT
+// token tiles (both compile-time here). Blocks [b0, b1) of the chunk; the group slot holds the
+// tokens' digits for every column (col0 = the chunk's first column). Per scale-group portion:
+// int32 MMA accumulation, then one fp32 epilogue
+//   acc += s * (f v + (c_k - z) f SX)   [the SX term once per group: in its first block's slice]
+// with f = 2^(E-14) and f SX read from the slot.
 // ---------------------------------------------------------------------------------------
-template <int B, int NRT, int NTILE, int NMAT>
+template <int B, int KM, int NT, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L, const unsigned char* st,
                                               const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0,
                                               int b1, int rt, float (&acc)[NTILE][NMAT][2]) {
     using Gm = Geo<NRT>;
     const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
-    const int G = a.G, K = a.K, ng = K / G, nbc = L.CK / 64;
-    const uint32_t* planes = reinterpret_cast<const uint32_t*>(st);
-    const uint32_t* meta = reinterpret_cast<const uint32_t*>(st + L.st_meta);
-    const int* sexp = reinterpret_cast<const int*>(gs + L.sl_exp);
-    const int* ssum = reinterpret_cast<const int*>(gs + L.sl_sum);
-    int C[NTILE][NMAT][4];
-#pragma unroll
-    for (int t = 0; t < NTILE; ++t)
-#pragma unroll
-        for (int m = 0; m < NMAT; ++m) C[t][m][0] = C[t][m][1] = C[t][m][2] = C[t][m][3] = 0;
-    bool has_start = false;
+    const int ng = a.K / a.G, bpg = a.G / 64, nbc = L.CK / 64;
+    const int pstride = NRT * nbc * 32;                                   // words per (matrix, plane) slab
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(st) + rt * nbc * 32 + lane;
+    const uint32_t* mrow = reinterpret_cast<const uint32_t*>(st + L.st_meta) + (rt * 16 + gid) * ng;
+    const float* fscl = reinterpret_cast<const float*>(gs + L.sl_exp) + tq * L.ngp;
+    const float* ffsx = reinterpret_cast<const float*>(gs + L.sl_sum) + tq * L.ngp;
+    const unsigned char* bsrc = gs + static_cast<size_t>((gid >> 1) * 2 + (gid & 1)) * L.dig_stride + 16 * tq + col0;
+    SlicePos sp = slice_pos(col0, b0, bpg);
+    int cb = b0;
 #pragma unroll 1
-    for (int cb = b0; cb < b1; ++cb) {
-        const int colb = col0 + cb * 64;                 // global column of the block
-        if (colb % G == 0) has_start = true;
-        // the B fragments of the tiles (shared by the matrices), then one matrix at a time
-        uint4 bt[NTILE];
+    while (cb < b1) {
+        const int n = min(bpg - sp.j, b1 - cb);   // blocks of this group portion
+        const bool has_start = sp.j == 0;
+        int C[NT][NMAT][4];
 #pragma unroll
-        for (int t = 0; t < NTILE; ++t)
-            if (t < gr.nt)
-                bt[t] = lds128(gs + static_cast<size_t>((4 * t + (gid >> 1)) * 2 + (gid & 1)) * L.dig_stride + colb +
-                               16 * tq);
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
-        for (int m = 0; m < NMAT; ++m) {
-            uint32_t w[kMaxB];
+            for (int m = 0; m < NMAT; ++m) C[t][m][0] = C[t][m][1] = C[t][m][2] = C[t][m][3] = 0;
+#pragma unroll 1
+        for (int i = 0; i < n; ++i, ++cb) {
+            uint4 bt[NT];
 #pragma unroll
-            for (int p = 0; p < kMaxB; ++p)
-                w[p] = p < gr.kmax ? planes[(((m * kMaxB + p) * NRT + rt) * nbc + cb) * 32 + lane] : 0u;
-            uint32_t R[4], Rh[4];
-            assemble<B>(R, w, gr.kmax);
+            for (int t = 0; t < NT; ++t) bt[t] = lds128(bsrc + static_cast<size_t>(8 * t) * L.dig_stride + cb * 64);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) Rh[r] = R[r] >> 4;
-            int level = -1;
-            uint32_t Alo[4], Ahi[4];
+            for (int m = 0; m < NMAT; ++m) {
+                uint32_t w[kMaxB];
 #pragma unroll
-            for (int t = 0; t < NTILE; ++t) {
-                if (t < gr.nt) {
-                    if (gr.tk[t] != level) {
-                        level = gr.tk[t];
-                        const uint32_t mk = level_mask(B, level);
+                for (int p = 0; p < kMaxB; ++p) w[p] = p < KM ? pw[(m * kMaxB + p) * pstride + cb * 32] : 0u;
+                uint32_t R[4], Rh[4];
+                decode_uniform<B, KM>(R, Rh, w);
+                uint32_t Alo[4], Ahi[4];
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    if (t == 0 || gr.mk[t] != gr.mk[t - 1]) {
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
-                            Alo[r] = R[r] & mk;
-                            Ahi[r] = Rh[r] & mk;
+                            Alo[r] = R[r] & gr.mk[t];
+                            Ahi[r] = Rh[r] & gr.mk[t];
                         }
                     }
                     mma_u8s8(C[t][m], Alo[0], Alo[1], Alo[2], Alo[3], bt[t].x, bt[t].y);
@@ -215,143 +239,156 @@ __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L,
                 }
             }
         }
-        // a group portion ends at the slice end or at a group boundary
-        if (cb + 1 == b1 || (colb + 64) % G == 0) {
-            const int g = colb / G;
-            float s[NMAT][2], z[NMAT][2];
+        // ---- epilogue of the portion of group g ----
+        const int g = sp.g;
+        float s[NMAT][2], z[NMAT][2];
+#pragma unroll
+        for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const uint32_t sz = mrow[(m * Gm::RB + 8 * rr) * ng + g];
+                s[m][rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(sz & 0xFFFFu)));
+                z[m][rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(sz >> 16)));
+            }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const float f = fscl[4 * t * L.ngp + g];
+            const float fsx = has_start ? ffsx[4 * t * L.ngp + g] : 0.f;
+            const float a0 = gr.ck[t] * fsx;
 #pragma unroll
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
-                    const uint32_t sz = meta[(m * Gm::RB + rt * 16 + gid + 8 * rr) * ng + g];
-                    s[m][rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(sz & 0xFFFFu)));
-                    z[m][rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(sz >> 16)));
+                    const float v = static_cast<float>(C[t][m][2 * rr] + 256 * C[t][m][2 * rr + 1]);
+                    const float u = fmaf(-z[m][rr], fsx, fmaf(f, v, a0));
+                    acc[t][m][rr] = fmaf(s[m][rr], u, acc[t][m][rr]);
                 }
-#pragma unroll
-            for (int t = 0; t < NTILE; ++t) {
-                if (t < gr.nt) {
-                    const int j = 4 * t + tq;
-                    const float f = pow2i(sexp[j * L.ngp + g] - 14);
-                    const float sx = has_start ? static_cast<float>(ssum[j * L.ngp + g]) : 0.f;
-                    const float ck = 0.5f * static_cast<float>((1 << (B - gr.tk[t])) - 1);
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                        for (int rr = 0; rr < 2; ++rr) {
-                            float v = static_cast<float>(C[t][m][2 * rr] + 256 * C[t][m][2 * rr + 1]);
-                            v = fmaf(ck - z[m][rr], sx, v);
-                            acc[t][m][rr] = fmaf(s[m][rr] * f, v, acc[t][m][rr]);
-                            C[t][m][2 * rr] = C[t][m][2 * rr + 1] = 0;
-                        }
-                }
-            }
-            has_start = false;
         }
+        sp.j = 0;
+        ++sp.g;
     }
 }
 
 // ---------------------------------------------------------------------------------------
-// consumer: one column slice of one chunk, binary-coded planes
+// consumer: one column slice of one chunk, binary-coded planes (KM planes, NT tiles):
+//   acc += alpha_p (2 f S_p - f SX)   per plane p < k of the tile and group portion
 // ---------------------------------------------------------------------------------------
-template <int B, int NRT, int NTILE, int NMAT>
+template <int B, int KM, int NT, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_bcq(const VpArgs& a, const VLayout& L, const unsigned char* st,
                                           const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0, int b1,
                                           int rt, float (&acc)[NTILE][NMAT][2]) {
     using Gm = Geo<NRT>;
     const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
-    const int G = a.G, K = a.K, ng = K / G, nbc = L.CK / 64;
-    const uint32_t* planes = reinterpret_cast<const uint32_t*>(st);
+    const int ng = a.K / a.G, bpg = a.G / 64, nbc = L.CK / 64;
+    const int pstride = NRT * nbc * 32;
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(st) + rt * nbc * 32 + lane;
     const __half* meta = reinterpret_cast<const __half*>(st + L.st_meta);
-    const int* sexp = reinterpret_cast<const int*>(gs + L.sl_exp);
-    const int* ssum = reinterpret_cast<const int*>(gs + L.sl_sum);
-    // the slice's blocks in group portions [p0, p1)
-    int p0 = b0;
-    while (p0 < b1) {
-        const int colb0 = col0 + p0 * 64;
-        int p1 = p0 + 1;
-        while (p1 < b1 && (col0 + p1 * 64) % G != 0) ++p1;
-        const int g = colb0 / G;
-        const bool has_start = colb0 % G == 0;
-#pragma unroll
-        for (int p = 0; p < B; ++p) {
-            if (p < gr.kmax) {
-                int C[NTILE][NMAT][4];
-#pragma unroll
-                for (int t = 0; t < NTILE; ++t)
-#pragma unroll
-                    for (int m = 0; m < NMAT; ++m) C[t][m][0] = C[t][m][1] = C[t][m][2] = C[t][m][3] = 0;
+    const float* fscl = reinterpret_cast<const float*>(gs + L.sl_exp) + tq * L.ngp;
+    const float* ffsx = reinterpret_cast<const float*>(gs + L.sl_sum) + tq * L.ngp;
+    const unsigned char* bsrc = gs + static_cast<size_t>((gid >> 1) * 2 + (gid & 1)) * L.dig_stride + 16 * tq + col0;
+    SlicePos sp = slice_pos(col0, b0, bpg);
+    int cb0 = b0;
 #pragma unroll 1
-                for (int cb = p0; cb < p1; ++cb) {
-                    const int colb = col0 + cb * 64;
-                    uint4 bt[NTILE];
+    while (cb0 < b1) {
+        const int n = min(bpg - sp.j, b1 - cb0);
+        const bool has_start = sp.j == 0;
+        const int g = sp.g;
+#pragma unroll 1
+        for (int p = 0; p < KM; ++p) {
+            int C[NT][NMAT][4];
 #pragma unroll
-                    for (int t = 0; t < NTILE; ++t)
-                        if (t < gr.nt && gr.tk[t] > p)
-                            bt[t] = lds128(gs + static_cast<size_t>((4 * t + (gid >> 1)) * 2 + (gid & 1)) * L.dig_stride +
-                                           colb + 16 * tq);
+            for (int t = 0; t < NT; ++t)
 #pragma unroll
-                    for (int m = 0; m < NMAT; ++m) {
-                        const uint32_t w = planes[(((m * kMaxB + p) * NRT + rt) * nbc + cb) * 32 + lane];
-                        uint32_t lo[4], hi[4];
+                for (int m = 0; m < NMAT; ++m) C[t][m][0] = C[t][m][1] = C[t][m][2] = C[t][m][3] = 0;
+#pragma unroll 1
+            for (int i = 0; i < n; ++i) {
+                const int cb = cb0 + i;
+                uint4 bt[NT];
 #pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            lo[r] = (w >> r) & 0x01010101u;
-                            hi[r] = (w >> (r + 4)) & 0x01010101u;
-                        }
+                for (int t = 0; t < NT; ++t)
+                    if (gr.tk[t] > p) bt[t] = lds128(bsrc + static_cast<size_t>(8 * t) * L.dig_stride + cb * 64);
 #pragma unroll
-                        for (int t = 0; t < NTILE; ++t) {
-                            if (t < gr.nt && gr.tk[t] > p) {
-                                mma_u8s8(C[t][m], lo[0], lo[1], lo[2], lo[3], bt[t].x, bt[t].y);
-                                mma_u8s8(C[t][m], hi[0], hi[1], hi[2], hi[3], bt[t].z, bt[t].w);
-                            }
-                        }
+                for (int m = 0; m < NMAT; ++m) {
+                    const uint32_t w = pw[(m * kMaxB + p) * pstride + cb * 32];
+                    uint32_t lo[4], hi[4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        lo[r] = (w >> r) & 0x01010101u;
+                        hi[r] = (w >> (r + 4)) & 0x01010101u;
                     }
-                }
-                float al[NMAT][2];
 #pragma unroll
-                for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr)
-                        al[m][rr] = __half2float(meta[((m * gr.kmax + p) * Gm::RB + rt * 16 + gid + 8 * rr) * ng + g]);
-#pragma unroll
-                for (int t = 0; t < NTILE; ++t) {
-                    if (t < gr.nt && gr.tk[t] > p) {
-                        const int j = 4 * t + tq;
-                        const float f = pow2i(sexp[j * L.ngp + g] - 14);
-                        const float sx = has_start ? static_cast<float>(ssum[j * L.ngp + g]) : 0.f;
-#pragma unroll
-                        for (int m = 0; m < NMAT; ++m)
-#pragma unroll
-                            for (int rr = 0; rr < 2; ++rr) {
-                                const float v = static_cast<float>(C[t][m][2 * rr] + 256 * C[t][m][2 * rr + 1]);
-                                acc[t][m][rr] = fmaf(al[m][rr] * f, fmaf(2.f, v, -sx), acc[t][m][rr]);
-                            }
+                    for (int t = 0; t < NT; ++t) {
+                        if (gr.tk[t] > p) {
+                            mma_u8s8(C[t][m], lo[0], lo[1], lo[2], lo[3], bt[t].x, bt[t].y);
+                            mma_u8s8(C[t][m], hi[0], hi[1], hi[2], hi[3], bt[t].z, bt[t].w);
+                        }
                     }
                 }
             }
+            float al[NMAT][2];
+#pragma unroll
+            for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr)
+                    al[m][rr] = __half2float(meta[((m * KM + p) * Gm::RB + rt * 16 + gid + 8 * rr) * ng + g]);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                if (gr.tk[t] > p) {
+                    const float f2 = 2.f * fscl[4 * t * L.ngp + g];
+                    const float fsx = has_start ? ffsx[4 * t * L.ngp + g] : 0.f;
+#pragma unroll
+                    for (int m = 0; m < NMAT; ++m)
+#pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            const float v = static_cast<float>(C[t][m][2 * rr] + 256 * C[t][m][2 * rr + 1]);
+                            acc[t][m][rr] = fmaf(al[m][rr], fmaf(f2, v, -fsx), acc[t][m][rr]);
+                        }
+                }
+            }
         }
-        p0 = p1;
+        cb0 += n;
+        sp.j = 0;
+        ++sp.g;
     }
+}
+
+// one slice with the group's plane count and tile count as compile-time constants
+template <int FMT, int B, int NRT, int NTILE, int NMAT>
+__device__ __forceinline__ void slice_b(const VpArgs& a, const VLayout& L, const unsigned char* st,
+                                        const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0, int b1,
+                                        int rt, float (&acc)[NTILE][NMAT][2]) {
+#define DPA_SLICE(KM, NT)                                                                                 \
+    do {                                                                                                  \
+        if constexpr (FMT == DPA_FMT_UNIFORM)                                                             \
+            slice_uniform<B, KM, NT, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc);           \
+        else                                                                                              \
+            slice_bcq<B, KM, NT, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc);               \
+    } while (0)
+    const int km = gr.kmax;
+    if (NTILE == 1 || gr.nt == 1) {
+        if (km == 1) DPA_SLICE(1, 1);
+        else if (km == 2 && B >= 2) DPA_SLICE(2 <= B ? 2 : B, 1);
+        else if (km == 3 && B >= 3) DPA_SLICE(3 <= B ? 3 : B, 1);
+        else DPA_SLICE(B, 1);
+    } else {
+        constexpr int NT2 = NTILE >= 2 ? 2 : 1;
+        if (km == 1) DPA_SLICE(1, NT2);
+        else if (km == 2 && B >= 2) DPA_SLICE(2 <= B ? 2 : B, NT2);
+        else if (km == 3 && B >= 3) DPA_SLICE(3 <= B ? 3 : B, NT2);
+        else DPA_SLICE(B, NT2);
+    }
+#undef DPA_SLICE
 }
 
 template <int FMT, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_dispatch(const VpArgs& a, const VLayout& L, const unsigned char* st,
                                                const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0,
                                                int b1, int rt, float (&acc)[NTILE][NMAT][2]) {
-    if constexpr (FMT == DPA_FMT_UNIFORM) {
-        switch (a.B) {
-            case 1: slice_uniform<1, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-            case 2: slice_uniform<2, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-            case 3: slice_uniform<3, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-            default: slice_uniform<4, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-        }
-    } else {
-        switch (a.B) {
-            case 1: slice_bcq<1, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-            case 2: slice_bcq<2, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-            case 3: slice_bcq<3, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-            default: slice_bcq<4, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
-        }
+    switch (a.B) {
+        case 1: slice_b<FMT, 1, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+        case 2: slice_b<FMT, 2, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+        case 3: slice_b<FMT, 3, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
+        default: slice_b<FMT, 4, NRT, NTILE, NMAT>(a, L, st, gs, gr, col0, b0, b1, rt, acc); break;
     }
 }
 
@@ -432,9 +469,9 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                         bulk_g2s(gs + static_cast<size_t>(lane * 2 + d) * L.dig_stride,
                                  a.dig + (static_cast<size_t>(drow) * 2 + d) * K, static_cast<uint32_t>(K), &s_gfull[slot]);
                     bulk_g2s(gs + L.sl_exp + static_cast<size_t>(lane) * L.ngp * 4,
-                             a.dexp + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u, &s_gfull[slot]);
+                             a.dscl + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u, &s_gfull[slot]);
                     bulk_g2s(gs + L.sl_sum + static_cast<size_t>(lane) * L.ngp * 4,
-                             a.dsum + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u, &s_gfull[slot]);
+                             a.dfsx + static_cast<size_t>(drow) * L.ngp, static_cast<uint32_t>(L.ngp) * 4u, &s_gfull[slot]);
                 }
                 cur_g = gi;
                 ++gcount;
@@ -527,6 +564,9 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
             for (int t = 0; t < NTILE; ++t) {
                 gr.tk[t] = rec[4 + t];
                 gr.tn[t] = rec[6 + t];
+                const int k = gr.tk[t] > 0 ? gr.tk[t] : 1;
+                gr.mk[t] = level_mask(a.B, k);
+                gr.ck[t] = 0.5f * static_cast<float>((1 << (a.B - k)) - 1);
             }
             cur_g = gi;
             ++gcount;
@@ -644,9 +684,10 @@ __global__ void __launch_bounds__(256) digits_kernel(DigitArgs d) {
         d1row[off] = static_cast<int8_t>(hi);
     }
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    if (lane == 0) {
-        d.dexp[static_cast<size_t>(r) * ngp + g] = E;
-        d.dsum[static_cast<size_t>(r) * ngp + g] = sum;
+    if (lane == 0) {   // |sum| <= G 2^14 <= 2^23: the scaled sum is exact in fp32
+        const float scl = ldexpf(1.f, E - 14);
+        d.dscl[static_cast<size_t>(r) * ngp + g] = scl;
+        d.dfsx[static_cast<size_t>(r) * ngp + g] = scl * static_cast<float>(sum);
     }
 }
 
@@ -665,34 +706,43 @@ cudaError_t launch_variant(const VpArgs& a, cudaStream_t stream, int sms) {
 
 }  // namespace
 
-// Variants: gate/up (two matrices) on 16-row items, down (one matrix) on 32-row items; token
-// groups of two tiles (8 tokens), or one tile (4 tokens) where the group slot would not fit.
+// Variants: gate/up (two matrices) and down (one matrix); items of the larger row block where
+// shared memory allows; token groups of two tiles (8 tokens), or one tile (4 tokens) where no
+// row block fits with two.
+template <int NMAT>
+static size_t vp_bytes(bool big, int tpg, int K, int G, int fmt, int B) {
+    constexpr int NB = NMAT == 2 ? kGuNRT : kDnNRT, NS = NMAT == 2 ? kGuNRTSmall : kDnNRTSmall;
+    if (big) return tpg == 2 ? vlayout<NB, 2, NMAT>(K, G, fmt, B).total : vlayout<NB, 1, NMAT>(K, G, fmt, B).total;
+    return tpg == 2 ? vlayout<NS, 2, NMAT>(K, G, fmt, B).total : vlayout<NS, 1, NMAT>(K, G, fmt, B).total;
+}
+
 int vp_tiles_per_group(int K_gateup, int K_down, int G, int fmt, int B) {
-    const bool two = vlayout<1, 2, 2>(K_gateup, G, fmt, B).total <= kVpMaxSmem &&
-                     vlayout<2, 2, 1>(K_down, G, fmt, B).total <= kVpMaxSmem;
+    const bool two = vp_bytes<2>(false, 2, K_gateup, G, fmt, B) <= kVpMaxSmem &&
+                     vp_bytes<1>(false, 2, K_down, G, fmt, B) <= kVpMaxSmem;
     return two ? 2 : 1;
 }
 
+// the smallest configuration of a variant (the shape is supported when it fits)
 size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, int tiles_per_group) {
-    if (nmat == 2)
-        return tiles_per_group == 2 ? vlayout<1, 2, 2>(K, G, fmt, B).total : vlayout<1, 1, 2>(K, G, fmt, B).total;
-    return tiles_per_group == 2 ? vlayout<2, 2, 1>(K, G, fmt, B).total : vlayout<2, 1, 1>(K, G, fmt, B).total;
+    return nmat == 2 ? vp_bytes<2>(false, tiles_per_group, K, G, fmt, B)
+                     : vp_bytes<1>(false, tiles_per_group, K, G, fmt, B);
+}
+
+template <int FMT, int NMAT>
+static cudaError_t launch_kind(const VpArgs& a, cudaStream_t stream, int sms) {
+    constexpr int NB = NMAT == 2 ? kGuNRT : kDnNRT, NS = NMAT == 2 ? kGuNRTSmall : kDnNRTSmall;
+    const bool two = a.tiles_per_group == 2;
+    const bool big = a.R % (16 * NB) == 0 && vp_bytes<NMAT>(true, two ? 2 : 1, a.K, a.G, FMT, a.B) <= kVpMaxSmem;
+    if (big) return two ? launch_variant<FMT, NB, 2, NMAT>(a, stream, sms) : launch_variant<FMT, NB, 1, NMAT>(a, stream, sms);
+    return two ? launch_variant<FMT, NS, 2, NMAT>(a, stream, sms) : launch_variant<FMT, NS, 1, NMAT>(a, stream, sms);
 }
 
 cudaError_t launch_vp_gemv(const VpArgs& a, cudaStream_t stream, int sms) {
-    const bool two = a.tiles_per_group == 2;
-    if (a.nmat == 2) {
-        if (a.fmt == DPA_FMT_UNIFORM)
-            return two ? launch_variant<DPA_FMT_UNIFORM, 1, 2, 2>(a, stream, sms)
-                       : launch_variant<DPA_FMT_UNIFORM, 1, 1, 2>(a, stream, sms);
-        return two ? launch_variant<DPA_FMT_BCQ, 1, 2, 2>(a, stream, sms)
-                   : launch_variant<DPA_FMT_BCQ, 1, 1, 2>(a, stream, sms);
-    }
-    if (a.fmt == DPA_FMT_UNIFORM)
-        return two ? launch_variant<DPA_FMT_UNIFORM, 2, 2, 1>(a, stream, sms)
-                   : launch_variant<DPA_FMT_UNIFORM, 2, 1, 1>(a, stream, sms);
-    return two ? launch_variant<DPA_FMT_BCQ, 2, 2, 1>(a, stream, sms)
-               : launch_variant<DPA_FMT_BCQ, 2, 1, 1>(a, stream, sms);
+    if (a.nmat == 2)
+        return a.fmt == DPA_FMT_UNIFORM ? launch_kind<DPA_FMT_UNIFORM, 2>(a, stream, sms)
+                                        : launch_kind<DPA_FMT_BCQ, 2>(a, stream, sms);
+    return a.fmt == DPA_FMT_UNIFORM ? launch_kind<DPA_FMT_UNIFORM, 1>(a, stream, sms)
+                                    : launch_kind<DPA_FMT_BCQ, 1>(a, stream, sms);
 }
 
 cudaError_t launch_digits(const DigitArgs& d, cudaStream_t stream) {

@@ -17,8 +17,8 @@ struct RouteArgs {
     double* gate;             // [T][K]
     unsigned* counters;       // [T] zero between calls
     int8_t* xdig;             // [T][2][H] activation digits for the expert GEMV, or nullptr
-    int32_t* xexp;            // [T][ngp] group exponents (ngp = H/G rounded up to 4)
-    int32_t* xsum;            // [T][ngp] group sums
+    float* xscl;              // [T][ngp] group scales 2^(E-14) (ngp = H/G rounded up to 4)
+    float* xfsx;              // [T][ngp] group sums of the fixed-point values times the scale
     WsHeader* hdr;
     int wpe;                  // warps per expert (set by the launcher)
     // large-batch path (nullptr: always the per-logit kernel): per-row exactness statistics
@@ -26,8 +26,20 @@ struct RouteArgs {
     double* n2_x;             // [T] sum of squares
     int16_t* lsb_w;           // [E][H/64]
     double* n2_w;             // [E]
+    double* part;             // [ks][T][E] slice sums of the tiled logits
+    int ks;                   // input slices (set by the launcher)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms = 148);
+
+// Tiling of the large-batch logits: token x expert CTA tiles, input slices to fill the SMs.
+struct RouteTiling {
+    int TT, TE, gx, gy, ks, kslice;
+};
+constexpr int kRouteMaxSms = 256;   // the partial-sum buffer is sized for up to this many SMs
+RouteTiling route_tiling(int T, int E, int H, int sms);
+bool route_tiled_path(int T, int H);
+// doubles of the slice-sum buffer the tiled path needs for T tokens (0: the per-logit path)
+size_t route_partial_doubles(int T, int E, int H);
 
 // A token group of the expert GEMV: [0] expert, [1] kmax over the group, [2] tiles (<= 2),
 // [4 + t] plane count of tile t, [6 + t] pairs in tile t (<= 4), [8 + 4t + q] grouped position
@@ -143,8 +155,8 @@ struct VpArgs {
     int tiles_per_group;      // 1 or 2 (the allocation's grouping)
     const int32_t* vrec;      // token group records [n_vgroups][kVRecInts], count in hdr->n_vgroups
     const int8_t* dig;        // activation digit rows [rows][2][K] (permuted 64-column blocks)
-    const int32_t* dexp;      // [rows][ngp] group exponents
-    const int32_t* dsum;      // [rows][ngp] group sums of the fixed-point values
+    const float* dscl;        // [rows][ngp] group scales 2^(E-14)
+    const float* dfsx;        // [rows][ngp] group sums of the fixed-point values times the scale
     int dig_by_token;         // 1: the digit row of a pair is its token (x); 0: its position (h)
     float* out;               // [P][R] by grouped position
     WsHeader* hdr;
@@ -159,15 +171,15 @@ constexpr size_t kVpMaxSmem = 227 * 1024;
 
 // Fixed-point digits of activation rows (x as bf16, or h as fp32), per group of G columns:
 // X = rint(v * 2^(14 - E)) with |v| < 2^E, as digits d0 + 256 d1 in rows [rows][2][K] with each
-// 64-column block permuted for the B operand; exponents and sums [rows][ngp], ngp = K/G rounded
-// up to a multiple of 4.
+// 64-column block permuted for the B operand; per group the scale 2^(E-14) and the scaled sum
+// 2^(E-14) sum_j X_j (both exact in fp32), [rows][ngp], ngp = K/G rounded up to a multiple of 4.
 struct DigitArgs {
     const uint16_t* x16;      // bf16 rows or nullptr
     const float* x32;         // fp32 rows (when x16 is nullptr)
     int rows, K, G;
     int8_t* dig;
-    int32_t* dexp;
-    int32_t* dsum;
+    float* dscl;
+    float* dfsx;
 };
 cudaError_t launch_digits(const DigitArgs& d, cudaStream_t stream);
 

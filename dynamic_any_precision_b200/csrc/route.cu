@@ -26,7 +26,7 @@ constexpr int kRouteWarps = 8;
 // the number a lane needs in total when that is at most 8, so that no unrolled slot idles.
 constexpr int16_t kNoBit = 0x3FFF;   // lowest-set-bit marker of a zero element
 #ifndef DPA_ROUTE_TILED_MIN_TOKENS
-#define DPA_ROUTE_TILED_MIN_TOKENS 128
+#define DPA_ROUTE_TILED_MIN_TOKENS 2
 #endif
 constexpr int kRouteTiledMinTokens = DPA_ROUTE_TILED_MIN_TOKENS;   // from here on the logits run as a tiled GEMM
 constexpr int kMaxLsbBlocks = 256;          // H <= 16384 on the tiled path
@@ -172,17 +172,38 @@ __device__ __forceinline__ int warp_sum_i(int v) {
 
 // Exact dot product of one (token, router row) pair by a warp: fp64 sum with the per-product
 // lowest-bit proof (every product a multiple of 2^lmin, sum |p| < 2^(lmin+53)), else the
-// fixed-point accumulator. Both operands are bf16 rows in global or shared memory.
+// fixed-point accumulator. Both operands are bf16 rows (global or shared memory, 16-byte
+// aligned, H a multiple of 8); a lane takes 8 consecutive inputs per 16-byte load and issues
+// up to 8 such loads per operand before using them.
 __device__ double exact_dot_warp(const uint16_t* x, const uint16_t* w, int H, int lane) {
     double acc = 0.0, absacc = 0.0;
     int lmin = 1 << 20;
-    for (int j = lane; j < H; j += 32) {
-        const uint32_t xu = x[j], wu = w[j];
-        const double p = __dmul_rn(static_cast<double>(__uint_as_float(xu << 16)),
-                                   static_cast<double>(__uint_as_float(wu << 16)));
-        acc = __dadd_rn(acc, p);
-        absacc = __dadd_rn(absacc, fabs(p));
-        if ((xu & 0x7FFF) && (wu & 0x7FFF)) lmin = min(lmin, bf16_lsb(xu) + bf16_lsb(wu));
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const uint4* wv = reinterpret_cast<const uint4*>(w);
+    const int nq = H >> 3;
+    for (int q0 = 0; q0 < nq; q0 += 32 * 8) {
+        uint4 xa[8], wa[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int q = q0 + 32 * u + lane;
+            xa[u] = q < nq ? xv[q] : make_uint4(0, 0, 0, 0);
+            wa[u] = q < nq ? wv[q] : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const uint32_t xw[4] = {xa[u].x, xa[u].y, xa[u].z, xa[u].w};
+            const uint32_t ww[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
+#pragma unroll
+            for (int h = 0; h < 8; ++h) {
+                const uint32_t xu = (xw[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                const uint32_t wu = (ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                const double p = __dmul_rn(static_cast<double>(__uint_as_float(xu << 16)),
+                                           static_cast<double>(__uint_as_float(wu << 16)));
+                acc = __dadd_rn(acc, p);
+                absacc = __dadd_rn(absacc, fabs(p));
+                if ((xu & 0x7FFF) && (wu & 0x7FFF)) lmin = min(lmin, bf16_lsb(xu) + bf16_lsb(wu));
+            }
+        }
     }
     acc = warp_sum_f64(acc);
     absacc = warp_sum_f64(absacc);
@@ -198,8 +219,8 @@ __device__ double exact_dot_warp(const uint16_t* x, const uint16_t* w, int H, in
 // this warp; xs is the token's bf16 row (shared or global memory). Per group of G inputs,
 // X = rint(x * 2^(14 - E)) with |x| < 2^E, stored as digits d0 + 256 d1 in rows [T][2][H] whose
 // 64-column blocks are permuted (column c at byte 16*((c%16)/4) + 4*(c/16) + c%4) so that one
-// 16-byte load gives an MMA lane its B-operand words; exponents and sums [T][ngp], ngp = H/G
-// rounded up to a multiple of 4.
+// 16-byte load gives an MMA lane its B-operand words; the group scales 2^(E-14) and scaled sums
+// [T][ngp], ngp = H/G rounded up to a multiple of 4.
 __device__ void token_digits(const RouteArgs& a, int t, const uint16_t* xs, int g0, int gstep) {
     const int H = a.H, G = a.G, ng = H / G, ngp = (ng + 3) & ~3, lane = threadIdx.x & 31;
     for (int g = g0; g < ng; g += gstep) {
@@ -220,9 +241,10 @@ __device__ void token_digits(const RouteArgs& a, int t, const uint16_t* xs, int 
             a.xdig[off + H] = static_cast<int8_t>(hi);
         }
         sum = warp_sum_i(sum);
-        if (lane == 0) {
-            a.xexp[t * ngp + g] = Eg;
-            a.xsum[t * ngp + g] = sum;
+        if (lane == 0) {   // |sum| <= G 2^14 <= 2^23: the scaled sum is exact in fp32
+            const float scl = ldexpf(1.f, Eg - 14);
+            a.xscl[t * ngp + g] = scl;
+            a.xfsx[t * ngp + g] = scl * static_cast<float>(sum);
         }
     }
 }
@@ -540,59 +562,75 @@ __global__ void __launch_bounds__(128) route_stats_kernel(RouteArgs a) {
     }
 }
 
-constexpr int kGT = 64, kGE = 128, kGK = 32;   // CTA tile: tokens x experts, k per stage
-constexpr int kGThreads = 256;                  // 8 warps of 16 tokens x 64 experts
+constexpr int kGK = 32;            // inputs per k stage of the tiled logits
+constexpr int kGThreads = 256;     // 8 warps: 4 token quarters x 2 expert halves of the CTA tile
 
 __device__ __forceinline__ double bf16_to_f64(uint32_t u) { return static_cast<double>(__uint_as_float(u << 16)); }
 
-// grid (ceil(T/64), ceil(E/128), k slices). Shared: x [2][kGK][kGT], w [2][kGK][kGE] in fp64.
+// Tiled logits: CTA tile TT tokens x TE experts over one slice of the inputs, fp64 FMAs (every
+// product of two bf16 values is exact in fp64; the sums are exact whenever the bound above
+// holds, which the selection kernel checks). Each thread owns TT/16 tokens x TE/16 experts.
+// Grid (ceil(T/TT), ceil(E/TE), ks); the slice sums go to part[ks][T][E] (no atomics; the
+// selection kernel adds the ks slices of a logit).
+template <int TT, int TE>
 __global__ void __launch_bounds__(kGThreads) route_gemm_kernel(RouteArgs a, int kslice) {
+    constexpr int MT = TT / 16, ME = TE / 16;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    double* sx = reinterpret_cast<double*>(smem_raw);          // [2][kGK][kGT]
-    double* sw = sx + 2 * kGK * kGT;                            // [2][kGK][kGE]
+    double* sx = reinterpret_cast<double*>(smem_raw);          // [2][kGK][TT]
+    double* sw = sx + 2 * kGK * TT;                             // [2][kGK][TE]
     const int H = a.H, T = a.T, E = a.E;
-    const int t0 = blockIdx.x * kGT, e0 = blockIdx.y * kGE;
+    const int t0 = blockIdx.x * TT, e0 = blockIdx.y * TE;
     const int k0 = blockIdx.z * kslice, k1 = min(H, k0 + kslice);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wt = warp & 3, we = warp >> 2, tg = lane & 3, eg = lane >> 2;
-    const int tb = 16 * wt + 4 * tg, eb = 64 * we + 8 * eg;   // this thread's 4 tokens, 8 experts
+    const int tb = (TT / 4) * wt + MT * tg, eb = (TE / 2) * we + ME * eg;   // this thread's tokens, experts
     pdl_wait();
 
-    // staging: x tile 64 x 32 (one uint4 per thread), w tile 128 x 32 (two per thread)
-    const int xt = tid & 63, xk = (tid >> 6) * 8;
-    const int wi = tid & 127, wk = (tid >> 7) * 8;
-    uint4 rx, rw0, rw1;
+    // staging: the x tile (TT rows x 32 inputs) and the w tile (TE rows x 32), 8 inputs per uint4
+    constexpr int NXL = (TT * 4 + kGThreads - 1) / kGThreads, NWL = (TE * 4 + kGThreads - 1) / kGThreads;
+    uint4 rx[NXL], rw[NWL];
     auto load = [&](int kc) {
-        rx = make_uint4(0, 0, 0, 0);
-        rw0 = rx;
-        rw1 = rx;
-        if (t0 + xt < T) rx = *reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + xt) * H + kc + xk);
-        if (e0 + wi < E) {
-            const uint16_t* wrow = a.wr + static_cast<size_t>(e0 + wi) * H + kc;
-            rw0 = *reinterpret_cast<const uint4*>(wrow + wk);
-            rw1 = *reinterpret_cast<const uint4*>(wrow + wk + 16);
+#pragma unroll
+        for (int u = 0; u < NXL; ++u) {
+            const int i = tid + u * kGThreads, xt = i % TT, xk = (i / TT) * 8;
+            rx[u] = make_uint4(0, 0, 0, 0);
+            if (i < TT * 4 && t0 + xt < T) rx[u] = *reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + xt) * H + kc + xk);
+        }
+#pragma unroll
+        for (int u = 0; u < NWL; ++u) {
+            const int i = tid + u * kGThreads, wi = i % TE, wk = (i / TE) * 8;
+            rw[u] = make_uint4(0, 0, 0, 0);
+            if (i < TE * 4 && e0 + wi < E) rw[u] = *reinterpret_cast<const uint4*>(a.wr + static_cast<size_t>(e0 + wi) * H + kc + wk);
         }
     };
     auto store = [&](int buf) {
-        double* bx = sx + buf * kGK * kGT;
-        double* bw = sw + buf * kGK * kGE;
-        const uint32_t xv[4] = {rx.x, rx.y, rx.z, rx.w};
-        const uint32_t w0[4] = {rw0.x, rw0.y, rw0.z, rw0.w};
-        const uint32_t w1[4] = {rw1.x, rw1.y, rw1.z, rw1.w};
+        double* bx = sx + buf * kGK * TT;
+        double* bw = sw + buf * kGK * TE;
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            const int sh = 16 * (h & 1);
-            bx[(xk + h) * kGT + xt] = bf16_to_f64((xv[h >> 1] >> sh) & 0xFFFFu);
-            bw[(wk + h) * kGE + wi] = bf16_to_f64((w0[h >> 1] >> sh) & 0xFFFFu);
-            bw[(wk + 16 + h) * kGE + wi] = bf16_to_f64((w1[h >> 1] >> sh) & 0xFFFFu);
+        for (int u = 0; u < NXL; ++u) {
+            const int i = tid + u * kGThreads, xt = i % TT, xk = (i / TT) * 8;
+            if (i < TT * 4) {
+                const uint32_t v[4] = {rx[u].x, rx[u].y, rx[u].z, rx[u].w};
+#pragma unroll
+                for (int h = 0; h < 8; ++h) bx[(xk + h) * TT + xt] = bf16_to_f64((v[h >> 1] >> (16 * (h & 1))) & 0xFFFFu);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < NWL; ++u) {
+            const int i = tid + u * kGThreads, wi = i % TE, wk = (i / TE) * 8;
+            if (i < TE * 4) {
+                const uint32_t v[4] = {rw[u].x, rw[u].y, rw[u].z, rw[u].w};
+#pragma unroll
+                for (int h = 0; h < 8; ++h) bw[(wk + h) * TE + wi] = bf16_to_f64((v[h >> 1] >> (16 * (h & 1))) & 0xFFFFu);
+            }
         }
     };
 
-    double acc[4][8];
+    double acc[MT][ME];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < MT; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+        for (int j = 0; j < ME; ++j) acc[i][j] = 0.0;
 
     int buf = 0;
     load(k0);
@@ -601,36 +639,45 @@ __global__ void __launch_bounds__(kGThreads) route_gemm_kernel(RouteArgs a, int 
     for (int kc = k0; kc < k1; kc += kGK) {
         const bool more = kc + kGK < k1;
         if (more) load(kc + kGK);
-        const double* bx = sx + buf * kGK * kGT;
-        const double* bw = sw + buf * kGK * kGE;
+        const double* bx = sx + buf * kGK * TT;
+        const double* bw = sw + buf * kGK * TE;
 #pragma unroll 4
         for (int k = 0; k < kGK; ++k) {
-            const double2 x01 = *reinterpret_cast<const double2*>(bx + k * kGT + tb);
-            const double2 x23 = *reinterpret_cast<const double2*>(bx + k * kGT + tb + 2);
-            const double2 w01 = *reinterpret_cast<const double2*>(bw + k * kGE + eb);
-            const double2 w23 = *reinterpret_cast<const double2*>(bw + k * kGE + eb + 2);
-            const double2 w45 = *reinterpret_cast<const double2*>(bw + k * kGE + eb + 4);
-            const double2 w67 = *reinterpret_cast<const double2*>(bw + k * kGE + eb + 6);
-            const double xv[4] = {x01.x, x01.y, x23.x, x23.y};
-            const double wv[8] = {w01.x, w01.y, w23.x, w23.y, w45.x, w45.y, w67.x, w67.y};
+            double xv[MT], wv[ME];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < MT; i += 2) {
+                if (i + 1 < MT) {
+                    const double2 v = *reinterpret_cast<const double2*>(bx + k * TT + tb + i);
+                    xv[i] = v.x;
+                    xv[i + 1] = v.y;
+                } else {
+                    xv[i] = bx[k * TT + tb + i];
+                }
+            }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = __fma_rn(xv[i], wv[j], acc[i][j]);
+            for (int j = 0; j < ME; j += 2) {
+                const double2 v = *reinterpret_cast<const double2*>(bw + k * TE + eb + j);
+                wv[j] = v.x;
+                wv[j + 1] = v.y;
+            }
+#pragma unroll
+            for (int i = 0; i < MT; ++i)
+#pragma unroll
+                for (int j = 0; j < ME; ++j) acc[i][j] = __fma_rn(xv[i], wv[j], acc[i][j]);
         }
         if (more) store(buf ^ 1);
         __syncthreads();
         buf ^= 1;
     }
-    double* dst = a.logits_user ? a.logits_user : a.logits_ws;
+    double* dst = a.part + static_cast<size_t>(blockIdx.z) * T * E;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < MT; ++i) {
         const int t = t0 + tb + i;
         if (t >= T) continue;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < ME; ++j) {
             const int e = e0 + eb + j;
-            if (e < E) atomicAdd(dst + static_cast<size_t>(t) * E + e, acc[i][j]);
+            if (e < E) dst[static_cast<size_t>(t) * E + e] = acc[i][j];
         }
     }
 }
@@ -651,8 +698,22 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
     __syncthreads();
     const double nx = a.n2_x[t];
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        // the logit: the tiled kernel's slice sums (exact, in any order, when the bound holds);
+        // eight independent loads in flight per step
+        const double* pe = a.part + static_cast<size_t>(t) * E + e;
+        const size_t qs = static_cast<size_t>(a.T) * E;
+        double v = 0.0;
+        for (int q0 = 0; q0 < a.ks; q0 += 8) {
+            double u[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) u[j] = q0 + j < a.ks ? __ldcg(pe + (q0 + j) * qs) : 0.0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v = __dadd_rn(v, u[j]);
+        }
+        dst[e] = v;
         const int16_t* lw = a.lsb_w + static_cast<size_t>(e) * nb;
         int L = 2 * kNoLsb;
+#pragma unroll 4
         for (int b0 = 0; b0 < nb; b0 += 8) {   // nb is a multiple of 8 (H % 512 == 0 on this path)
             const uint4 v = *reinterpret_cast<const uint4*>(lw + b0);
             const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
@@ -693,30 +754,56 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
 
 }  // namespace
 
+RouteTiling route_tiling(int T, int E, int H, int sms) {
+    RouteTiling r;
+    r.TT = T <= 16 ? 16 : 64;
+    r.TE = T <= 64 ? 32 : 128;
+    r.gx = (T + r.TT - 1) / r.TT;
+    r.gy = (E + r.TE - 1) / r.TE;
+    const int nchunks = H / kGK;
+    int ks = 1;   // input slices: enough CTAs for every SM, each slice a whole number of k stages
+    while (r.gx * r.gy * ks * 2 <= sms && ks * 2 <= nchunks && nchunks % (ks * 2) == 0) ks *= 2;
+    r.ks = ks;
+    r.kslice = (nchunks / ks) * kGK;
+    return r;
+}
+
+bool route_tiled_path(int T, int H) {
+    return T >= kRouteTiledMinTokens && H % kGK == 0 && H % (8 * kLsbBlock) == 0 && H / kLsbBlock <= kMaxLsbBlocks;
+}
+
+size_t route_partial_doubles(int T, int E, int H) {
+    if (!route_tiled_path(T, H)) return 0;
+    const RouteTiling r = route_tiling(T, E, H, kRouteMaxSms);
+    return static_cast<size_t>(r.ks) * T * E;
+}
+
+template <int TT, int TE>
+static cudaError_t launch_route_gemm(RouteArgs& b, const RouteTiling& r, cudaStream_t stream) {
+    const size_t smem = sizeof(double) * 2 * kGK * (TT + TE);
+    const void* fn = reinterpret_cast<const void*>(route_gemm_kernel<TT, TE>);
+    if (smem > 48 * 1024) {
+        cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+    }
+    int kslice = r.kslice;
+    void* gargs[] = {&b, &kslice};
+    return launch_pdl_raw(fn, dim3(r.gx, r.gy, r.ks), dim3(kGThreads), smem, stream, gargs);
+}
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms) {
-    if (a.T >= kRouteTiledMinTokens && a.H % kGK == 0 && a.H % (8 * kLsbBlock) == 0 &&
-        a.H / kLsbBlock <= kMaxLsbBlocks && a.lsb_x != nullptr) {
-        // large batch: stats, tiled fp64 GEMM with split-K atomics, per-token selection
-        double* dst = a.logits_user ? a.logits_user : a.logits_ws;
-        cudaError_t err = cudaMemsetAsync(dst, 0, sizeof(double) * static_cast<size_t>(a.T) * a.E, stream);
-        if (err != cudaSuccess) return err;
+    if (route_tiled_path(a.T, a.H) && a.lsb_x != nullptr && a.part != nullptr) {
+        // stats, tiled fp64 logits by input slice, per-token selection
+        const RouteTiling r = route_tiling(a.T, a.E, a.H, sms < kRouteMaxSms ? sms : kRouteMaxSms);
         RouteArgs b = a;
+        b.ks = r.ks;
         void* args[] = {&b};
-        err = launch_pdl_raw(reinterpret_cast<const void*>(route_stats_kernel), dim3(a.T + a.E), dim3(128), 0,
-                             stream, args);
+        cudaError_t err = launch_pdl_raw(reinterpret_cast<const void*>(route_stats_kernel), dim3(a.T + a.E), dim3(128),
+                                         0, stream, args);
         if (err != cudaSuccess) return err;
-        const int gx = (a.T + kGT - 1) / kGT, gy = (a.E + kGE - 1) / kGE;
-        const int nchunks = a.H / kGK;
-        int ks = 1;   // k slices: enough CTAs for every SM, each slice a whole number of chunks
-        while (gx * gy * ks < sms && ks * 2 <= nchunks && nchunks % (ks * 2) == 0) ks *= 2;
-        int kslice = (nchunks / ks) * kGK;
-        const size_t smem = sizeof(double) * 2 * kGK * (kGT + kGE);
-        err = cudaFuncSetAttribute(route_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem));
-        if (err != cudaSuccess) return err;
-        void* gargs[] = {&b, &kslice};
-        err = launch_pdl_raw(reinterpret_cast<const void*>(route_gemm_kernel), dim3(gx, gy, ks), dim3(kGThreads), smem,
-                             stream, gargs);
+        if (r.TT == 16) err = launch_route_gemm<16, 32>(b, r, stream);
+        else if (r.TE == 32) err = launch_route_gemm<64, 32>(b, r, stream);
+        else err = launch_route_gemm<64, 128>(b, r, stream);
         if (err != cudaSuccess) return err;
         size_t ssm = (static_cast<size_t>(a.E) * 24 + 15) & ~static_cast<size_t>(15);
         if (ssm > 48 * 1024) {

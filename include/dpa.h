@@ -81,9 +81,12 @@ typedef struct dpa_layer_desc {
  *          gate, up, down; experts follow in order.
  *          Inside a plane the bits are in the decode kernel's fragment order: 16-row tiles,
  *          then 64-column blocks, then 32 lanes of one 32-bit word. Lane l = 4*g + c holds
- *          rows {g, g+8} and, for rho in 0..3 and m in 0..7, bit 4*m + rho is the weight at
+ *          rows {g, g+8}; for rho in 0..3 and m in 0..7 the weight at
  *            row    = tile*16 + g + 8*(rho & 1)
- *            column = block*64 + 32*(m & 1) + 16*(rho >> 1) + 4*c + (m >> 1).
+ *            column = block*64 + 32*(m & 1) + 16*(rho >> 1) + 4*c + (m >> 1)
+ *          sits at bit 4*m + rho of the word (DPA_FMT_BCQ), or at bit
+ *          (4*m + (B-1-p) - rho) mod 32 in plane p (DPA_FMT_UNIFORM: rotated per plane, so
+ *          that a decoder merges the planes under fixed masks and rotates once per rho).
  *          Use dpa_export_codes to read codes back in natural order.
  *  meta:   DPA_FMT_UNIFORM: per (e, m, row, group) an fp16 pair {s, z}, row-major,
  *          [E][3][R][C/G] with the three matrices in order.
