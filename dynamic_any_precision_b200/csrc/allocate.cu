@@ -67,6 +67,7 @@ __device__ __forceinline__ int choose_k(const double* c, int nk, int kmin, const
 
 __device__ __forceinline__ double midpoint(double lo, double hi) { return __dmul_rn(0.5, __dadd_rn(lo, hi)); }
 
+
 // the same decision with the pair's costs in registers
 __device__ __forceinline__ int choose_k_reg(const double (&c)[4], int nk, int kmin, const KVals& kv, double lam) {
     double best = __dadd_rn(c[0], __dmul_rn(lam, kv.v[0]));
@@ -109,13 +110,46 @@ __device__ __forceinline__ int block_incl_scan(int v, int* s_tmp) {
     return r;
 }
 
+// inclusive block scan of NV ints per thread at once (one exchange through shared memory)
+template <int NV>
+__device__ __forceinline__ void block_incl_scan_n(int (&v)[NV], int (*s_tmp)[32]) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int u = __shfl_up_sync(0xffffffffu, v[j], o);
+            if (lane >= o) v[j] += u;
+        }
+    }
+    if (lane == 31)
+#pragma unroll
+        for (int j = 0; j < NV; ++j) s_tmp[j][warp] = v[j];
+    __syncthreads();
+    if (warp < NV) {   // warp j scans the warp totals of value j
+        int w = lane < nw ? s_tmp[warp][lane] : 0;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += u;
+        }
+        s_tmp[warp][lane] = w;
+    }
+    __syncthreads();
+    if (warp > 0)
+#pragma unroll
+        for (int j = 0; j < NV; ++j) v[j] += s_tmp[j][warp - 1];
+    __syncthreads();
+}
+
 // Shared-memory carve-up: [costs (if they fit)] [counts E*nk] [seg E*nk+1] [sorted P] [k P]
 struct AllocSmem {
-    size_t costs, counts, seg, sorted, kk, bp, bj, total;
+    size_t costs, counts, seg, sorted, kk, bp, bj, ptok, rexp, rfirst, total;
     bool costs_in_smem;
 };
 
-__host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk) {
+// recs: the GEMV records are written (token of each grouped position, each record's owner
+// expert and each expert's first record are kept in shared memory for them)
+__host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk, bool recs) {
     AllocSmem L;
     L.costs_in_smem = static_cast<size_t>(P) * nk <= static_cast<size_t>(kSmemCostDoubles);
     L.costs = 0;
@@ -135,6 +169,14 @@ __host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk) {
     off += nbp * 8;
     L.bj = off;
     off += nbp * 4;
+    off = (off + 15) & ~static_cast<size_t>(15);
+    const size_t nrec = static_cast<size_t>(P) / 4 + static_cast<size_t>(E) * nk + 1;
+    L.ptok = off;
+    off += recs ? static_cast<size_t>(P) * 4 : 0;
+    L.rexp = off;
+    off += recs ? nrec * 4 : 0;
+    L.rfirst = off;
+    off += recs ? static_cast<size_t>(E) * 4 : 0;
     L.total = (off + 15) & ~static_cast<size_t>(15);
     return L;
 }
@@ -142,6 +184,7 @@ __host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk) {
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ int s_tmp[32];
+    __shared__ int s_scan5[5][32];
     __shared__ double s_max[32];
     __shared__ unsigned char s_pred[2][kAllocThreads];
     // speculative replay of the bisection (small batches)
@@ -156,10 +199,13 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     const int nk = a.kmax - a.kmin + 1;
     const KVals kv = make_kvals(a.kmin);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const AllocSmem Ls = alloc_smem_layout(P, a.E, nk);
+    const AllocSmem Ls = alloc_smem_layout(P, a.E, nk, a.vrec != nullptr);
     double* c_base = Ls.costs_in_smem ? reinterpret_cast<double*>(smem + Ls.costs) : a.cbuf;
     uint8_t* s_k = smem + Ls.kk;
 
+    // the residual table is static: bring its lines towards this SM while the router finishes
+    for (int i = tid * 16; i < a.E * a.B; i += blockDim.x * 16)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(a.rtable + i));
     pdl_wait();   // the routed pairs come from the previous kernel
     pdl_trigger();   // the successor may become resident now (it waits for this kernel)
     // the budget, the pairs' experts and gates are loaded together (one round trip)
@@ -628,69 +674,43 @@ grouping:
         if (tid == 0) s_seg[nkeys] = P;
     }
     __syncthreads();
+    int* s_ptok = reinterpret_cast<int*>(smem + Ls.ptok);   // token of each grouped position
     for (int p = tid; p < P; p += blockDim.x) {
         const int key = a.idx[p] * nk + (s_k[p] - a.kmin);
         const int pos = atomicAdd(&s_counts[key], 1);
+        const int tok = p / a.K;
         s_sorted[pos] = p;
+        if (a.vrec) s_ptok[pos] = tok;
         a.pair_pos[p] = pos;
-        if (a.pos_tok) a.pos_tok[pos] = p / a.K;
+        if (a.pos_tok) a.pos_tok[pos] = tok;
     }
     __syncthreads();
-    // per-expert descriptors and two-token tiles (tiles never straddle k classes); experts in
-    // rounds of blockDim so that the active list stays in ascending expert order
-    int rank_base = 0, tile_base = 0, gt_base = 0, vt_base = 0, vg_base = 0;
+    // Per expert: the prefill GEMM's token tiles (one (expert, k) class each) and the start of its
+    // GEMV records (groups of up to vtpg tiles of up to 4 pairs of one class, classes ascending in
+    // k); experts in rounds of blockDim so that both lists stay in ascending expert order. Each
+    // record's owner expert goes to s_rexp; the records themselves are written below, one warp
+    // per record.
+    int rank_base = 0, gt_base = 0, vg_base = 0;
     const int vtpg = a.vtiles_per_group > 0 ? a.vtiles_per_group : 1;
+    int* s_rexp = reinterpret_cast<int*>(smem + Ls.rexp);   // [records] owner expert
+    int* s_rfirst = reinterpret_cast<int*>(smem + Ls.rfirst);   // [E] first record of each expert
     for (int e0 = 0; e0 < a.E; e0 += blockDim.x) {
         const int e = e0 + tid;
-        int km = 0, ntiles = 0, ngt = 0, nvt = 0;
+        int km = 0, ngt = 0, nvt = 0;
         if (e < a.E) {
             for (int i = 0; i < nk; ++i) {
                 const int n = s_seg[e * nk + i + 1] - s_seg[e * nk + i];
                 if (n > 0) km = a.kmin + i;
-                ntiles += (n + 1) >> 1;
                 ngt += (n + kGemmTileTokens - 1) / kGemmTileTokens;
                 nvt += (n + 3) >> 2;
             }
         }
-        const int nvg = (nvt + vtpg - 1) / vtpg;
+        const int nvg = a.vrec ? (nvt + vtpg - 1) / vtpg : 0;
         const int flag = km > 0 ? 1 : 0;
-        const int rank_incl = block_incl_scan(flag, s_tmp);
-        const int tiles_incl = block_incl_scan(ntiles, s_tmp);
-        const int gt_incl = a.gtiles ? block_incl_scan(ngt, s_tmp) : 0;
-        const int vt_incl = a.vrec ? block_incl_scan(nvt, s_tmp) : 0;
-        const int vg_incl = a.vrec ? block_incl_scan(nvg, s_tmp) : 0;
-        const int rank = rank_base + rank_incl - flag;
-        const int tile_off = tile_base + tiles_incl - ntiles;
-        if (a.vrec && nvt > 0) {   // 4-pair tiles of one (expert, k) class, in groups of vtpg tiles
-            int gi = vg_base + vg_incl - nvg, in_group = 0;
-            int32_t* rec = a.vrec + static_cast<size_t>(gi) * kVRecInts;
-            for (int i = 0; i < nk; ++i) {
-                const int s0 = s_seg[e * nk + i];
-                const int n = s_seg[e * nk + i + 1] - s0;
-                for (int j = 0; j < n; j += 4) {
-                    if (in_group == 0) {   // a new record: expert, and every slot unused
-                        rec[0] = e;
-                        for (int q = 3; q < kVRecInts; ++q) rec[q] = q >= 8 && q < 24 ? -1 : 0;
-                    }
-                    const int cnt = min(4, n - j);
-                    rec[1] = a.kmin + i;            // tiles ascend in k: the last is the group's kmax
-                    rec[4 + in_group] = a.kmin + i;
-                    rec[6 + in_group] = cnt;
-                    for (int q = 0; q < cnt; ++q) {
-                        const int pos = s0 + j + q;
-                        rec[8 + 4 * in_group + q] = pos;                    // output row
-                        rec[16 + 4 * in_group + q] = s_sorted[pos] / a.K;   // token
-                    }
-                    rec[2] = ++in_group;
-                    if (in_group == vtpg) {
-                        in_group = 0;
-                        rec += kVRecInts;
-                    }
-                }
-            }
-        }
+        int sc[3] = {flag, a.gtiles ? ngt : 0, nvg};   // one block scan of the three counts
+        block_incl_scan_n<3>(sc, s_scan5);
         if (a.gtiles && ngt > 0) {   // token tiles of the prefill GEMMs: one (expert, k) class each
-            int t = gt_base + gt_incl - ngt;
+            int t = gt_base + sc[1] - ngt;
             for (int i = 0; i < nk; ++i) {
                 const int s0 = s_seg[e * nk + i];
                 const int n = s_seg[e * nk + i + 1] - s0;
@@ -698,37 +718,56 @@ grouping:
                     a.gtiles[t++] = make_int4(e, a.kmin + i, s0 + j, min(kGemmTileTokens, n - j));
             }
         }
-        if (flag) {
-            a.exp_desc[2 * rank] = make_int4(e, km, ntiles, tile_off);
-            int t = tile_off;
-            for (int i = 0; i < nk; ++i) {
-                const int s0 = s_seg[e * nk + i];
-                const int n = s_seg[e * nk + i + 1] - s0;
-                for (int j = 0; j < n; j += 2) {
-                    const int posA = s0 + j, posB = j + 1 < n ? s0 + j + 1 : -1;
-                    const int tokA = s_sorted[posA] / a.K;
-                    const int tokB = posB >= 0 ? s_sorted[posB] / a.K : -1;
-                    const int4 tile = make_int4(a.kmin + i, posA, posB, (tokA & 0xFFFF) | ((tokB & 0xFFFF) << 16));
-                    if (t == tile_off) a.exp_desc[2 * rank + 1] = tile;   // first tile rides with the descriptor
-                    a.tiles[t++] = tile;
+        if (a.vrec && e < a.E) {
+            const int r0 = vg_base + sc[2] - nvg;
+            s_rfirst[e] = r0;
+            for (int j = 0; j < nvg; ++j) s_rexp[r0 + j] = e;
+        }
+        // totals of this round: the scan's last warp totals, still in shared memory; every thread
+        // reads them before the barrier below, ahead of the next round's scan
+        rank_base += s_scan5[0][nw - 1];
+        gt_base += s_scan5[1][nw - 1];
+        vg_base += s_scan5[2][nw - 1];
+        __syncthreads();
+    }
+    if (a.vrec) {
+        // record r of expert e holds the expert's tiles [j vtpg, (j+1) vtpg), j = r - first(e);
+        // lane q computes field q (layout of kVRecInts) and the warp stores the record at once
+        for (int r = warp; r < vg_base; r += nw) {
+            const int e = s_rexp[r];
+            const int j = r - s_rfirst[e];
+            int tk[2] = {0, 0}, tn[2] = {0, 0}, tpos[2] = {0, 0}, nt = 0;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                int g = j * vtpg + t;   // the expert's tile index
+                if (t >= vtpg) break;
+                for (int i = 0; i < nk; ++i) {
+                    const int s0 = s_seg[e * nk + i];
+                    const int n = s_seg[e * nk + i + 1] - s0;
+                    const int ntc = (n + 3) >> 2;
+                    if (g < ntc) {
+                        tk[t] = a.kmin + i;
+                        tn[t] = min(4, n - 4 * g);
+                        tpos[t] = s0 + 4 * g;
+                        nt = t + 1;
+                        break;
+                    }
+                    g -= ntc;
                 }
             }
+            int v = 0;
+            if (lane == 0) v = e;
+            else if (lane == 1) v = tk[nt - 1];            // tiles ascend in k: the last is the group's kmax
+            else if (lane == 2) v = nt;
+            else if (lane == 4 || lane == 5) v = tk[lane - 4];
+            else if (lane == 6 || lane == 7) v = tn[lane - 6];
+            else if (lane >= 8 && lane < 24) {
+                const int f = lane & 7, t = f >> 2, u = f & 3;
+                const bool used = t < nt && u < tn[t];
+                v = !used ? -1 : (lane < 16 ? tpos[t] + u : s_ptok[tpos[t] + u]);
+            }
+            a.vrec[static_cast<size_t>(r) * kVRecInts + lane] = v;
         }
-        // totals of this round (the last thread's inclusive sums), broadcast
-        if (tid == blockDim.x - 1) {
-            s_tmp[0] = rank_incl;
-            s_tmp[1] = tiles_incl;
-            s_tmp[2] = gt_incl;
-            s_tmp[3] = vt_incl;
-            s_tmp[4] = vg_incl;
-        }
-        __syncthreads();
-        rank_base += s_tmp[0];
-        tile_base += s_tmp[1];
-        gt_base += s_tmp[2];
-        vt_base += s_tmp[3];
-        vg_base += s_tmp[4];
-        __syncthreads();
     }
     if (tid == 0) {
         a.hdr->n_active = static_cast<uint32_t>(rank_base);
@@ -889,7 +928,7 @@ cudaError_t launch_calibrate(const CalibArgs& a, cudaStream_t stream) {
                           args);
 }
 
-size_t allocate_smem_bytes(int P, int E, int nk) { return alloc_smem_layout(P, E, nk).total; }
+size_t allocate_smem_bytes(int P, int E, int nk, bool recs) { return alloc_smem_layout(P, E, nk, recs).total; }
 
 int allocate_threads(int P) { return P <= kSmallP ? 256 : kAllocThreads; }   // small: 8 warps x 8 nodes
 
@@ -925,7 +964,7 @@ cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* c
         if (err != cudaSuccess) return err;
         b.k_given = 1;
     }
-    const size_t smem = allocate_smem_bytes(P, a.E, nk);
+    const size_t smem = allocate_smem_bytes(P, a.E, nk, a.vrec != nullptr);
     if (smem > 48 * 1024) {
         cudaError_t err = cudaFuncSetAttribute(allocate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));

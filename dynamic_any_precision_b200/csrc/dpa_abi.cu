@@ -35,7 +35,7 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xscl, xfsx, h, out_pair, sh_h, sh_out,
-        desc, tiles, gtiles, postok, coop, rstats, rpart, xperm, hdig, hscl, hfsx, vrec, total;
+        gtiles, postok, coop, rstats, rpart, xperm, hdig, hscl, hfsx, vrec, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -69,8 +69,6 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.out_pair = take(4 * P * H);
     L.sh_h = take(4 * static_cast<size_t>(T) * d->n_shared * I);
     L.sh_out = take(4 * static_cast<size_t>(T) * H);
-    L.desc = take(32 * E);
-    L.tiles = take(16 * (P + E * nk));
     L.gtiles = take(16 * (P / dpa::kGemmTileTokens + E * nk + 1));
     L.postok = take(4 * P);
     L.coop = take(sizeof(dpa::CoopSync));
@@ -261,8 +259,6 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.cbuf = at<double>(ws, L.cbuf);
     a.do_permute = permute ? 1 : 0;
     a.pair_pos = at<int32_t>(ws, L.pairpos);
-    a.exp_desc = at<int4>(ws, L.desc);
-    a.tiles = at<int4>(ws, L.tiles);
     a.gtiles = gemm_tiles ? at<int4>(ws, L.gtiles) : nullptr;
     a.pos_tok = gemm_tiles ? at<int32_t>(ws, L.postok) : nullptr;
     a.vrec = permute && !gemm_tiles ? at<int32_t>(ws, L.vrec) : nullptr;

@@ -43,11 +43,20 @@ constexpr int kCW = 8;                        // consumer warps
 constexpr int kVThreads = (kCW + 1) * 32;     // + the producer warp
 constexpr int kMaxStages = 8;                 // ring depth: as many stages as shared memory holds
 constexpr int kMaxB = 4;
-constexpr int kMaxChunk = 1024;               // columns per chunk
+#ifndef DPA_VP_CHUNK
+#define DPA_VP_CHUNK 2048
+#endif
+constexpr int kMaxChunk = DPA_VP_CHUNK;       // columns per chunk
 // Row tiles (16 rows each) per item: the larger where the ring and group slots fit in shared
 // memory, else the smaller (wide matrices, whose scale data and digit rows take more room).
-constexpr int kGuNRT = 2, kGuNRTSmall = 1;    // gate/up: 32 (16) rows, 4 (8) column slices
-constexpr int kDnNRT = 4, kDnNRTSmall = 2;    // down: 64 (32) rows, 2 (4) column slices
+#ifndef DPA_VP_GU_NRT
+#define DPA_VP_GU_NRT 2
+#endif
+#ifndef DPA_VP_DN_NRT
+#define DPA_VP_DN_NRT 4
+#endif
+constexpr int kGuNRT = DPA_VP_GU_NRT, kGuNRTSmall = 1;   // gate/up: 32 (16) rows, 4 (8) column slices
+constexpr int kDnNRT = DPA_VP_DN_NRT, kDnNRTSmall = 2;   // down: 64 (32) rows, 2 (4) column slices
 constexpr int kDigPad = 64;                   // bytes of padding per staged digit row (banks)
 
 template <int NRT>
@@ -76,11 +85,8 @@ __host__ __device__ inline VLayout vlayout(int K, int G, int fmt, int B) {
     VLayout L;
     const size_t ng = K / G;
     L.ngp = static_cast<int>((ng + 3) & ~static_cast<size_t>(3));
-    const size_t CK = K < kMaxChunk ? K : kMaxChunk;
-    const size_t planes = static_cast<size_t>(NMAT) * kMaxB * NRT * (CK / 64) * 128;
     const size_t meta = fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(NMAT) * Gm::RB * ng * 4
                                                : static_cast<size_t>(NMAT) * B * Gm::RB * ng * 2;
-    const size_t stage = al128(planes + al16(meta));
     const size_t dig_stride = static_cast<size_t>(K) + kDigPad;
     const size_t digs = static_cast<size_t>(4 * NTILE) * 2 * dig_stride;
     const size_t sl_exp = al16(digs);
@@ -90,6 +96,15 @@ __host__ __device__ inline VLayout vlayout(int K, int G, int fmt, int B) {
     const size_t red_per = static_cast<size_t>(32) * NTILE * NMAT * 2 * 4;
     const size_t red = static_cast<size_t>(NRT) * Gm::CS * red_per;   // one partial per warp
     const size_t fixed = 2 * slot + red;
+    // columns per chunk: every column (one copy per matrix and plane takes all the item's row
+    // tiles) where two stages fit beside the fixed parts, else halved down to 512
+    size_t CK = K < kMaxChunk ? K : kMaxChunk, planes = 0, stage = 0;
+    for (;;) {
+        planes = static_cast<size_t>(NMAT) * kMaxB * NRT * (CK / 64) * 128;
+        stage = al128(planes + al16(meta));
+        if (fixed + 2 * stage <= kVpMaxSmem || CK <= 512 || (CK / 2) % 64 != 0) break;
+        CK /= 2;
+    }
     int nst = 2;   // at least double buffering; more while the ring fits beside the fixed parts
     while (nst < kMaxStages && fixed + (nst + 1) * stage <= kVpMaxSmem) ++nst;
     size_t total = nst * stage + fixed;
@@ -495,7 +510,17 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                 }
                 __syncwarp();
                 fence_proxy_async();
-                // plane words: (m, p, rt) copies of the chunk's columns (2 bytes per column)
+                // plane words: (m, p, rt) copies of the chunk's columns (2 bytes per column); a chunk
+                // of every column takes the item's NRT consecutive row tiles in one copy per (m, p)
+                if (static_cast<int>(L.CK) == K) {
+                    for (int i = lane; i < NMAT * kmax; i += 32) {
+                        const int p = i % kmax, m = i / kmax;
+                        const uint8_t* src = pbase + a.planes_mat_off[a.mat0 + m] + p * plane_bytes +
+                                             static_cast<uint64_t>(rb * NRT) * (K / 64) * 128;
+                        bulk_g2s(st + (static_cast<size_t>(m * kMaxB + p) * NRT * (K / 64)) * 128, src,
+                                 static_cast<uint32_t>(NRT * (K / 64)) * 128u, &s_full[s]);
+                    }
+                } else
                 for (int i = lane; i < n_pc; i += 32) {
                     const int rt = i % NRT, mp = i / NRT, p = mp % kmax, m = mp / kmax;
                     const uint8_t* src = pbase + a.planes_mat_off[a.mat0 + m] + p * plane_bytes +

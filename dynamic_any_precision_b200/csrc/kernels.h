@@ -58,8 +58,6 @@ struct AllocArgs {
     // grouping outputs (do_permute)
     int do_permute;
     int32_t* pair_pos;        // [P] position of each pair in the (expert, k)-grouped order
-    int4* exp_desc;           // [E][2] per active expert: {expert, kmax, n_tiles, first tile}, first tile
-    int4* tiles;              // [P + E*nk] two-token tiles: {k, posA, posB, tokA | tokB << 16}
     int k_given;              // 1: k_out already holds the plane counts (grid-wide bisection ran)
     int4* gtiles;             // nullptr, or [P/kGemmTileTokens + E*nk] GEMM token tiles {e, k, pos0, n}
     int32_t* pos_tok;         // nullptr, or [P] token of each grouped position
@@ -83,7 +81,7 @@ struct CoopSync {
 };
 // coop: workspace counters for the grid-wide bisection of large batches (nullptr: single CTA).
 cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* coop = nullptr, int sms = 0);
-size_t allocate_smem_bytes(int P, int E, int nk);
+size_t allocate_smem_bytes(int P, int E, int nk, bool recs);
 int allocate_threads(int P);
 
 // Threshold calibration of the score-threshold policy: 64 bisection steps over n scores.

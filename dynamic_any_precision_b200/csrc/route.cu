@@ -519,12 +519,11 @@ constexpr int kNoLsb = 0x3FFF;      // block (or row) without a nonzero element
 constexpr int kLsbBlock = 64;       // inputs per lowest-bit block
 
 // One CTA per row (tokens 0..T-1, then router rows): per-block lowest set bit, sum of squares,
-// NaN/Inf flag.
-__global__ void __launch_bounds__(128) route_stats_kernel(RouteArgs a) {
-    __shared__ double s_n[4];
-    __shared__ int s_b[4];
-    pdl_wait();
-    const int r = blockIdx.x, H = a.H, nb = H / kLsbBlock;
+// NaN/Inf flag. Any block of up to 8 warps.
+__device__ void route_stats_row(const RouteArgs& a, int r) {
+    __shared__ double s_n[8];
+    __shared__ int s_b[8];
+    const int H = a.H, nb = H / kLsbBlock;
     const bool is_tok = r < a.T;
     const uint16_t* row = is_tok ? a.x + static_cast<size_t>(r) * H : a.wr + static_cast<size_t>(r - a.T) * H;
     int16_t* lrow = is_tok ? a.lsb_x + static_cast<size_t>(r) * nb : a.lsb_w + static_cast<size_t>(r - a.T) * nb;
@@ -549,13 +548,13 @@ __global__ void __launch_bounds__(128) route_stats_kernel(RouteArgs a) {
         for (int o = 1; o < 8; o <<= 1) l = min(l, __shfl_xor_sync(0xffffffffu, l, o));
         if (c < H / 8 && (c & 7) == 0) lrow[c >> 3] = static_cast<int16_t>(l);
     }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     n2 = warp_sum_f64(n2);
     bad = __any_sync(0xffffffffu, bad);
     if (lane == 0) { s_n[warp] = n2; s_b[warp] = bad; }
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < 4; ++w) { n2 = __dadd_rn(n2, s_n[w]); bad |= s_b[w]; }
+        for (int w = 1; w < nw; ++w) { n2 = __dadd_rn(n2, s_n[w]); bad |= s_b[w]; }
         if (is_tok) a.n2_x[r] = n2;
         else a.n2_w[r - a.T] = n2;
         if (bad) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, is_tok ? 1 : 2);
@@ -573,18 +572,17 @@ __device__ __forceinline__ double bf16_to_f64(uint32_t u) { return static_cast<d
 // Grid (ceil(T/TT), ceil(E/TE), ks); the slice sums go to part[ks][T][E] (no atomics; the
 // selection kernel adds the ks slices of a logit).
 template <int TT, int TE>
-__global__ void __launch_bounds__(kGThreads) route_gemm_kernel(RouteArgs a, int kslice) {
+__device__ __forceinline__ void route_gemm_tile(const RouteArgs& a, int kslice, int bx, int by, int bz,
+                                                unsigned char* smem_raw) {
     constexpr int MT = TT / 16, ME = TE / 16;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
     double* sx = reinterpret_cast<double*>(smem_raw);          // [2][kGK][TT]
     double* sw = sx + 2 * kGK * TT;                             // [2][kGK][TE]
     const int H = a.H, T = a.T, E = a.E;
-    const int t0 = blockIdx.x * TT, e0 = blockIdx.y * TE;
-    const int k0 = blockIdx.z * kslice, k1 = min(H, k0 + kslice);
+    const int t0 = bx * TT, e0 = by * TE;
+    const int k0 = bz * kslice, k1 = min(H, k0 + kslice);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int wt = warp & 3, we = warp >> 2, tg = lane & 3, eg = lane >> 2;
     const int tb = (TT / 4) * wt + MT * tg, eb = (TE / 2) * we + ME * eg;   // this thread's tokens, experts
-    pdl_wait();
 
     // staging: the x tile (TT rows x 32 inputs) and the w tile (TE rows x 32), 8 inputs per uint4
     constexpr int NXL = (TT * 4 + kGThreads - 1) / kGThreads, NWL = (TE * 4 + kGThreads - 1) / kGThreads;
@@ -669,7 +667,7 @@ __global__ void __launch_bounds__(kGThreads) route_gemm_kernel(RouteArgs a, int 
         __syncthreads();
         buf ^= 1;
     }
-    double* dst = a.part + static_cast<size_t>(blockIdx.z) * T * E;
+    double* dst = a.part + static_cast<size_t>(bz) * T * E;
 #pragma unroll
     for (int i = 0; i < MT; ++i) {
         const int t = t0 + tb + i;
@@ -682,8 +680,27 @@ __global__ void __launch_bounds__(kGThreads) route_gemm_kernel(RouteArgs a, int 
     }
 }
 
+// The router's first launch: three independent jobs side by side, by block index: the tiled
+// logits (gx * gy * ks tiles), the exactness statistics of every token and router row (T + E
+// rows), and the tokens' fixed-point digits for the expert GEMV (T tokens, when requested).
+template <int TT, int TE>
+__global__ void __launch_bounds__(kGThreads) route_prep_kernel(RouteArgs a, int kslice, int gx, int gy, int ks) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    pdl_wait();
+    const int n_gemm = gx * gy * ks;
+    const int b = blockIdx.x;
+    if (b < n_gemm) {
+        route_gemm_tile<TT, TE>(a, kslice, b % gx, (b / gx) % gy, b / (gx * gy), smem_raw);
+    } else if (b < n_gemm + a.T + a.E) {
+        route_stats_row(a, b - n_gemm);
+    } else {
+        const int t = b - n_gemm - a.T - a.E;
+        token_digits(a, t, a.x + static_cast<size_t>(t) * a.H, threadIdx.x >> 5, kGThreads / 32);
+    }
+}
+
 // One CTA (4 warps) per token: check each logit's exactness bound, recompute the failures with
-// the fixed-point dot product, then top-k and gates (and the GEMV digits when requested).
+// the exact dot product, then top-k and gates.
 __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int s_fail[256];
@@ -749,7 +766,6 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
         __syncthreads();
     }
     select_topk_gates(a, t, smem_raw);
-    if (a.xdig != nullptr) token_digits(a, t, xrow, warp, 4);
 }
 
 }  // namespace
@@ -779,31 +795,29 @@ size_t route_partial_doubles(int T, int E, int H) {
 }
 
 template <int TT, int TE>
-static cudaError_t launch_route_gemm(RouteArgs& b, const RouteTiling& r, cudaStream_t stream) {
+static cudaError_t launch_route_prep(RouteArgs& b, const RouteTiling& r, cudaStream_t stream) {
     const size_t smem = sizeof(double) * 2 * kGK * (TT + TE);
-    const void* fn = reinterpret_cast<const void*>(route_gemm_kernel<TT, TE>);
-    if (smem > 48 * 1024) {
-        cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (err != cudaSuccess) return err;
-    }
-    int kslice = r.kslice;
-    void* gargs[] = {&b, &kslice};
-    return launch_pdl_raw(fn, dim3(r.gx, r.gy, r.ks), dim3(kGThreads), smem, stream, gargs);
+    const void* fn = reinterpret_cast<const void*>(route_prep_kernel<TT, TE>);
+    // always raised: with the statistics role's static shared memory, 48 KB of dynamic does not fit
+    // under the default limit
+    cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    int kslice = r.kslice, gx = r.gx, gy = r.gy, ks = r.ks;
+    const int blocks = gx * gy * ks + b.T + b.E + (b.xdig != nullptr ? b.T : 0);
+    void* gargs[] = {&b, &kslice, &gx, &gy, &ks};
+    return launch_pdl_raw(fn, dim3(blocks), dim3(kGThreads), smem, stream, gargs);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms) {
     if (route_tiled_path(a.T, a.H) && a.lsb_x != nullptr && a.part != nullptr) {
-        // stats, tiled fp64 logits by input slice, per-token selection
+        // logits by input slice + row statistics + token digits in one launch; per-token selection
         const RouteTiling r = route_tiling(a.T, a.E, a.H, sms < kRouteMaxSms ? sms : kRouteMaxSms);
         RouteArgs b = a;
         b.ks = r.ks;
-        void* args[] = {&b};
-        cudaError_t err = launch_pdl_raw(reinterpret_cast<const void*>(route_stats_kernel), dim3(a.T + a.E), dim3(128),
-                                         0, stream, args);
-        if (err != cudaSuccess) return err;
-        if (r.TT == 16) err = launch_route_gemm<16, 32>(b, r, stream);
-        else if (r.TE == 32) err = launch_route_gemm<64, 32>(b, r, stream);
-        else err = launch_route_gemm<64, 128>(b, r, stream);
+        cudaError_t err;
+        if (r.TT == 16) err = launch_route_prep<16, 32>(b, r, stream);
+        else if (r.TE == 32) err = launch_route_prep<64, 32>(b, r, stream);
+        else err = launch_route_prep<64, 128>(b, r, stream);
         if (err != cudaSuccess) return err;
         size_t ssm = (static_cast<size_t>(a.E) * 24 + 15) & ~static_cast<size_t>(15);
         if (ssm > 48 * 1024) {
@@ -811,6 +825,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms) {
                                        static_cast<int>(ssm));
             if (err != cudaSuccess) return err;
         }
+        void* args[] = {&b};
         return launch_pdl_raw(reinterpret_cast<const void*>(route_select_kernel), dim3(a.T), dim3(128), ssm, stream,
                               args);
     }
