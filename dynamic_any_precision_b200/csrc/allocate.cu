@@ -23,6 +23,8 @@
 // expert GEMV consumes.
 #include <cstdint>
 
+#include <math_constants.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -80,6 +82,11 @@ __device__ __forceinline__ int choose_k_reg(const double (&c)[4], int nk, int km
         }
     }
     return kb;
+}
+
+// Stored planes of expert e (per-expert stored widths; else every expert holds kmax).
+__device__ __forceinline__ int stored_width(const AllocArgs& a, int e) {
+    return a.expert_width ? static_cast<int>(a.expert_width[e]) : a.kmax;
 }
 
 constexpr int kRegPairs = 4;   // pairs per lane held in registers by the small-batch bisection
@@ -218,14 +225,21 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
                   : (!budget_policy || (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)))
                         ? 0 : 1;
     if (bad && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, a.policy == DPA_ALLOC_THRESHOLD ? 12 : 10);
-    int bad_e = 0;
+    int bad_e = 0, bad_w = 0;
     for (int p = tid; p < P; p += blockDim.x) {
         const int e = a.idx[p];
-        bad_e |= (e < 0 || e >= a.E) ? 1 : 0;
+        const bool ok = e >= 0 && e < a.E;
+        bad_e |= ok ? 0 : 1;
+        if (ok && a.expert_width) {
+            const int w = a.expert_width[e];
+            bad_w |= (w < a.kmin || w > a.kmax) ? 1 : 0;
+        }
     }
     const int any_bad_e = __syncthreads_or(bad_e);
+    const int any_bad_w = __syncthreads_or(bad_w);
     if (any_bad_e && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 11);
-    if (bad || any_bad_e) {
+    if (!any_bad_e && any_bad_w && tid == 0) set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, 15);
+    if (bad || any_bad_e || any_bad_w) {
         if (a.do_permute && tid == 0) {   // nothing downstream may read a previous call's work lists
             a.hdr->n_active = 0;
             a.hdr->n_gtiles = 0;
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
         const int nb = static_cast<int>(floor(__dmul_rn(target, static_cast<double>(P))));
         const int base = nb / P, rem = nb - base * P;
         for (int p = tid; p < P; p += blockDim.x) {
-            const int k = base + (p < rem ? 1 : 0);
+            const int k = min(base + (p < rem ? 1 : 0), stored_width(a, a.idx[p]));
             a.k_out[p] = static_cast<uint8_t>(k);
             s_k[p] = static_cast<uint8_t>(k);
         }
@@ -267,7 +281,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             return;
         }
         for (int p = tid; p < P; p += blockDim.x) {
-            const int k = a.expert_k[a.idx[p]];
+            const int k = min(static_cast<int>(a.expert_k[a.idx[p]]), stored_width(a, a.idx[p]));
             a.k_out[p] = static_cast<uint8_t>(k);
             s_k[p] = static_cast<uint8_t>(k);
         }
@@ -278,7 +292,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     if (a.policy == DPA_ALLOC_THRESHOLD) {
         // high precision above the calibrated score threshold, low precision otherwise
         for (int p = tid; p < P; p += blockDim.x) {
-            const int k = a.gate[p] > tau ? a.kmax : a.kmin;
+            const int k = min(a.gate[p] > tau ? a.kmax : a.kmin, stored_width(a, a.idx[p]));
             a.k_out[p] = static_cast<uint8_t>(k);
             s_k[p] = static_cast<uint8_t>(k);
         }
@@ -292,6 +306,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     for (int p = tid; p < P; p += blockDim.x) {
         const int e = a.idx[p];
         const double g = a.gate[p];
+        const int wmax = stored_width(a, e);   // counts above the expert's stored planes cost +inf
         double r[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -299,7 +314,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             if (i < nk) {
-                const double c = __dmul_rn(g, r[i]);
+                const double c = a.kmin + i > wmax ? CUDART_INF : __dmul_rn(g, r[i]);
                 c_base[static_cast<size_t>(p) * nk + i] = c;
                 if (i == 0) mx = fmax(mx, c);
             }
@@ -767,6 +782,54 @@ grouping:
                 v = !used ? -1 : (lane < 16 ? tpos[t] + u : s_ptok[tpos[t] + u]);
             }
             a.vrec[static_cast<size_t>(r) * kVRecInts + lane] = v;
+            // the record's work weight per row block (planes read, token tiles), in the owner slot
+            __syncwarp();
+            if (lane == 0) s_rexp[r] = 5 + 2 * tk[nt - 1] + 3 * nt;
+        }
+        const bool tab0 = a.vstart[0] && vg_base * a.vnrb[0] > a.vgrid[0];
+        const bool tab1 = a.vstart[1] && vg_base * a.vnrb[1] > a.vgrid[1];
+        if (tab0 || tab1) {   // (with no more items than CTAs the GEMV splits items evenly)
+            __syncthreads();
+            // exclusive prefix of the weights over the records: s_rexp[0..vg_base]
+            const int nrec = vg_base;
+            const int per = (nrec + blockDim.x - 1) / blockDim.x;
+            const int r0 = tid * per, r1 = min(nrec, r0 + per);
+            int run = 0;
+            for (int r = r0; r < r1; ++r) run += s_rexp[r];
+            int base = block_incl_scan(run, s_tmp) - run;
+            for (int r = r0; r < r1; ++r) {
+                const int w = s_rexp[r];
+                s_rexp[r] = base;
+                base += w;
+            }
+            if (tid == blockDim.x - 1) s_rexp[nrec] = base;   // the total (the last thread's running sum)
+            __syncthreads();
+            const long long wtot = s_rexp[nrec];
+            for (int j = 0; j < 2; ++j) {
+                if (!(j == 0 ? tab0 : tab1)) continue;
+                const int grid = a.vgrid[j], nrb = a.vnrb[j];
+                for (int b = tid; b <= grid; b += blockDim.x) {
+                    // first item i whose preceding work reaches b/grid of the total
+                    const long long tb = wtot * nrb * b / grid;
+                    int lo = 0, hi = nrec;   // largest g with prefix(g) * nrb <= tb
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (static_cast<long long>(s_rexp[mid]) * nrb <= tb) lo = mid;
+                        else hi = mid - 1;
+                    }
+                    long long start;
+                    if (lo >= nrec) {
+                        start = static_cast<long long>(nrec) * nrb;
+                    } else {
+                        const long long pg = static_cast<long long>(s_rexp[lo]) * nrb;
+                        const long long wg = s_rexp[lo + 1] - s_rexp[lo];
+                        long long rb = (tb - pg + wg - 1) / wg;
+                        if (rb > nrb) rb = nrb;
+                        start = static_cast<long long>(lo) * nrb + rb;
+                    }
+                    a.vstart[j][b] = static_cast<int32_t>(start);
+                }
+            }
         }
     }
     if (tid == 0) {
@@ -808,13 +871,16 @@ __global__ void __launch_bounds__(kCoopThreads) allocate_coop_kernel(AllocArgs a
         const int p = p0 + j;
         const int e = a.idx[p];
         double c[4] = {0.0, 0.0, 0.0, 0.0};
-        if (e < 0 || e >= a.E) {
+        if (e < 0 || e >= a.E || (a.expert_width && (a.expert_width[e] < a.kmin || a.expert_width[e] > a.kmax))) {
             bad_e = 1;
         } else {
             const double g = a.gate[p];
+            const int wmax = stored_width(a, e);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                if (i < nk) c[i] = __dmul_rn(g, a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)]);
+                if (i < nk)
+                    c[i] = a.kmin + i > wmax ? CUDART_INF
+                                             : __dmul_rn(g, a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)]);
             mx = fmax(mx, c[0]);
         }
 #pragma unroll

@@ -35,10 +35,12 @@ dpa_status check_desc(const dpa_layer_desc* d) {
 // ---- workspace layout ----
 struct WsLayout {
     size_t hdr, counters, logits, idx, gate, k, lambda, cbuf, pairpos, xdig, xscl, xfsx, h, out_pair, sh_h, sh_out,
-        gtiles, postok, coop, rstats, rpart, xperm, hdig, hscl, hfsx, vrec, total;
+        gtiles, postok, coop, rstats, rpart, vstart, xperm, hdig, hscl, hfsx, vrec, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+constexpr int kVpMaxGrid = 512;   // CTAs of an expert GEMV launch the balanced start tables cover
 
 WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     WsLayout L;
@@ -74,6 +76,7 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.coop = take(sizeof(dpa::CoopSync));
     L.rstats = take((8 + 2 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 16);
     L.rpart = take(8 * dpa::route_partial_doubles(T, static_cast<int>(E), static_cast<int>(H)));
+    L.vstart = take(4 * 2 * (kVpMaxGrid + 1));
     L.xperm = take(2 * P * H);
     L.hdig = take(2 * P * I);
     L.hscl = take(4 * P * ngp_i);
@@ -137,6 +140,55 @@ static dpa_status combine_stage(const dpa_layer_desc* d, const dpa_layer_weights
     if (dpa::launch_combine(ca, s) != cudaSuccess) return DPA_ERR_CUDA;
     mark(6);
     return DPA_OK;
+}
+
+// Arguments of one expert GEMV launch of the forward: gate/up (down = false: x digits by token
+// -> h [P][I]) or down (h digits by grouped position -> per-pair outputs [P][H]).
+static dpa::VpArgs vp_launch_args(const dpa_layer_desc* d, const dpa_layer_weights* w, const dpa_sizes& sz, void* ws,
+                                  const WsLayout& L, int T, int tpg, bool down) {
+    dpa::VpArgs va{};
+    const int P = T * d->top_k;
+    const int nk = d->kmax - d->kmin + 1;
+    va.planes = static_cast<const uint8_t*>(w->planes);
+    va.meta = static_cast<const uint8_t*>(w->meta);
+    va.planes_per_expert = sz.planes_per_expert;
+    va.meta_per_expert = sz.meta_per_expert;
+    for (int m = 0; m < 3; ++m) {
+        va.planes_mat_off[m] = sz.planes_matrix_offset[m];
+        va.meta_mat_off[m] = sz.meta_matrix_offset[m];
+    }
+    va.fmt = d->format;
+    va.B = d->bits;
+    va.G = d->group;
+    va.tiles_per_group = tpg;
+    va.vrec = at<int32_t>(ws, L.vrec);
+    va.hdr = at<dpa::WsHeader>(ws, L.hdr);
+    va.expert_off = w->expert_offsets;
+    va.expert_width = w->expert_width;
+    const int tiles_bound = P / 4 + d->n_experts * nk;
+    va.max_groups = P < tiles_bound ? P : tiles_bound;
+    if (!down) {
+        va.R = d->inter;
+        va.K = d->hidden;
+        va.mat0 = 0;
+        va.nmat = 2;
+        va.dig = at<int8_t>(ws, L.xdig);
+        va.dscl = at<float>(ws, L.xscl);
+        va.dfsx = at<float>(ws, L.xfsx);
+        va.dig_by_token = 1;
+        va.out = at<float>(ws, L.h);
+    } else {
+        va.R = d->hidden;
+        va.K = d->inter;
+        va.mat0 = 2;
+        va.nmat = 1;
+        va.dig = at<int8_t>(ws, L.hdig);
+        va.dscl = at<float>(ws, L.hscl);
+        va.dfsx = at<float>(ws, L.hfsx);
+        va.dig_by_token = 0;
+        va.out = at<float>(ws, L.out_pair);
+    }
+    return va;
 }
 
 // Per-row exactness statistics of the large-batch router, carved from the workspace.
@@ -239,11 +291,13 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
                                 double* lambda_out, void* ws, const WsLayout& L, bool permute, cudaStream_t s,
                                 bool gemm_tiles = false, int policy = DPA_ALLOC_LAGRANGE,
                                 const double* threshold = nullptr, int vtiles_per_group = 1,
-                                const uint8_t* expert_k = nullptr) {
+                                const uint8_t* expert_k = nullptr, const int* vgrid = nullptr,
+                                const int* vnrb = nullptr, const uint8_t* expert_width = nullptr) {
     dpa::AllocArgs a{};
     a.policy = policy;
     a.threshold = threshold;
     a.expert_k = expert_k;
+    a.expert_width = expert_width;
     a.rtable = rtable;
     a.idx = idx;
     a.gate = gate;
@@ -263,6 +317,12 @@ static dpa_status allocate_impl(const dpa_layer_desc* d, const double* rtable, c
     a.pos_tok = gemm_tiles ? at<int32_t>(ws, L.postok) : nullptr;
     a.vrec = permute && !gemm_tiles ? at<int32_t>(ws, L.vrec) : nullptr;
     a.vtiles_per_group = vtiles_per_group;
+    for (int j = 0; j < 2; ++j) {   // balanced CTA ranges of the two GEMV launches
+        const bool use = a.vrec && vgrid && vgrid[j] > 0 && vgrid[j] <= kVpMaxGrid;
+        a.vstart[j] = use ? at<int32_t>(ws, L.vstart) + j * (kVpMaxGrid + 1) : nullptr;
+        a.vgrid[j] = use ? vgrid[j] : 0;
+        a.vnrb[j] = use ? vnrb[j] : 0;
+    }
     a.hdr = at<dpa::WsHeader>(ws, L.hdr);
     return dpa::launch_allocate(a, s, at<dpa::CoopSync>(ws, L.coop), num_sms_current()) == cudaSuccess ? DPA_OK
                                                                                                   : DPA_ERR_CUDA;
@@ -403,9 +463,11 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     if (!policy_inputs_ok(policy, target_bpw, threshold, expert_k)) return DPA_ERR_INVALID_ARG;
     const bool tc_shape = d->format == DPA_FMT_UNIFORM && d->hidden % 256 == 0 && d->inter % 256 == 0 &&
                           (d->group & (d->group - 1)) == 0;   // scale groups of 64 * 2^n inputs
-    if (path == DPA_PATH_TC && !tc_shape) return DPA_ERR_UNSUPPORTED;
+    const bool compact = w->expert_width != nullptr || w->expert_offsets != nullptr;
+    if (compact && !(w->expert_width && w->expert_offsets)) return DPA_ERR_INVALID_ARG;
+    if (path == DPA_PATH_TC && (!tc_shape || compact)) return DPA_ERR_UNSUPPORTED;
     const bool use_tc = path == DPA_PATH_TC ||
-                        (path == DPA_PATH_AUTO && tc_shape &&
+                        (path == DPA_PATH_AUTO && tc_shape && !compact &&
                          static_cast<long long>(T) * K >= static_cast<long long>(DPA_TC_MIN_PAIRS_PER_EXPERT) * d->n_experts);
 
     int32_t* idx = (aux && aux->topk_idx) ? aux->topk_idx : at<int32_t>(ws, L.idx);
@@ -446,8 +508,21 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     // otherwise token groups of up to two 4-pair tiles, where their staging fits
     // token groups of the expert GEMV: two 4-pair tiles where the group slots fit, else one
     const int tpg = dpa::vp_tiles_per_group(d->hidden, d->inter, d->group, d->format, d->bits);
+    // the two GEMV launches (decode path): their grids and row blocks per record, for which the
+    // allocation writes work-balanced CTA ranges
+    dpa::VpArgs va_gu{}, va_dn{};
+    int vgrid[2] = {0, 0}, vnrb[2] = {0, 0};
+    if (!use_tc) {
+        const int nsm = num_sms_current();
+        va_gu = vp_launch_args(d, w, sz, ws, L, T, tpg, false);
+        va_dn = vp_launch_args(d, w, sz, ws, L, T, tpg, true);
+        vgrid[0] = dpa::vp_grid(va_gu, nsm);
+        vgrid[1] = dpa::vp_grid(va_dn, nsm);
+        vnrb[0] = va_gu.R / dpa::vp_rows_per_item(va_gu);
+        vnrb[1] = va_dn.R / dpa::vp_rows_per_item(va_dn);
+    }
     dpa_status st2 = allocate_impl(d, w->rtable, idx, gate, T, target_bpw, kk, lam, ws, L, true, s, use_tc, policy,
-                                   threshold, tpg, expert_k);
+                                   threshold, tpg, expert_k, vgrid, vnrb, w->expert_width);
     if (st2 != DPA_OK) return st2;
     mark(2);
 
@@ -502,34 +577,10 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
         return combine_stage(d, w, gate, T, aux, y, ws, L, hdr, s, mark);
     }
     const int P = T * K;
-    const int nk = d->kmax - d->kmin + 1;
-    dpa::VpArgs va{};
-    va.planes = static_cast<const uint8_t*>(w->planes);
-    va.meta = static_cast<const uint8_t*>(w->meta);
-    va.planes_per_expert = sz.planes_per_expert;
-    va.meta_per_expert = sz.meta_per_expert;
-    for (int m = 0; m < 3; ++m) {
-        va.planes_mat_off[m] = sz.planes_matrix_offset[m];
-        va.meta_mat_off[m] = sz.meta_matrix_offset[m];
-    }
-    va.fmt = d->format;
-    va.B = d->bits;
-    va.G = d->group;
-    va.tiles_per_group = tpg;
-    va.vrec = at<int32_t>(ws, L.vrec);
-    va.hdr = hdr;
-    const int tiles_bound = P / 4 + d->n_experts * nk;
-    va.max_groups = P < tiles_bound ? P : tiles_bound;
     // gate and up with SwiGLU: x digits by token -> h [P][I]
-    va.R = d->inter;
-    va.K = d->hidden;
-    va.mat0 = 0;
-    va.nmat = 2;
-    va.dig = at<int8_t>(ws, L.xdig);
-    va.dscl = at<float>(ws, L.xscl);
-    va.dfsx = at<float>(ws, L.xfsx);
-    va.dig_by_token = 1;
-    va.out = at<float>(ws, L.h);
+    dpa::VpArgs va = va_gu;
+    va.vstart = vgrid[0] > 0 && vgrid[0] <= kVpMaxGrid ? at<int32_t>(ws, L.vstart) : nullptr;
+    va.vgrid = vgrid[0];
     if (dpa::launch_vp_gemv(va, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(4);
     // digits of h, then down -> per-pair outputs [P][H]
@@ -543,15 +594,9 @@ dpa_status dpa_moe_forward(const dpa_layer_desc* d, const dpa_layer_weights* w, 
     da.dscl = at<float>(ws, L.hscl);
     da.dfsx = at<float>(ws, L.hfsx);
     if (dpa::launch_digits(da, s) != cudaSuccess) return DPA_ERR_CUDA;
-    va.R = d->hidden;
-    va.K = d->inter;
-    va.mat0 = 2;
-    va.nmat = 1;
-    va.dig = at<int8_t>(ws, L.hdig);
-    va.dscl = at<float>(ws, L.hscl);
-    va.dfsx = at<float>(ws, L.hfsx);
-    va.dig_by_token = 0;
-    va.out = at<float>(ws, L.out_pair);
+    va = va_dn;
+    va.vstart = vgrid[1] > 0 && vgrid[1] <= kVpMaxGrid ? at<int32_t>(ws, L.vstart) + (kVpMaxGrid + 1) : nullptr;
+    va.vgrid = vgrid[1];
     if (dpa::launch_vp_gemv(va, s, sms) != cudaSuccess) return DPA_ERR_CUDA;
     mark(5);
     return combine_stage(d, w, gate, T, aux, y, ws, L, hdr, s, mark);

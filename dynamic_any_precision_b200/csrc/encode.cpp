@@ -16,6 +16,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <limits>
 #include <thread>
 #include <vector>
 
@@ -395,6 +396,128 @@ extern "C" dpa_status dpa_export_meta(const dpa_layer_desc* desc, const void* me
     } else {
         for (uint64_t i = 0; i < static_cast<uint64_t>(desc->bits) * R * ng; ++i)
             s_or_alpha[i] = static_cast<float>(f16_bits_to_f64(mm[i]));
+    }
+    return DPA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Per-expert stored widths (MatMoE, review "Core Contribution": an offline ILP over each
+// expert's maximum bit-width under a memory budget). Exact dynamic programming over the experts
+// from the last; every fp64 operation is a separate rounding (this file is built without
+// contraction), so the result is reproducible by any IEEE implementation of the same steps.
+// ---------------------------------------------------------------------------------------
+extern "C" dpa_status dpa_solve_stored_widths(const dpa_layer_desc* desc, const double* importance,
+                                              const double* rtable, int64_t budget_planes, uint8_t* widths) {
+    dpa_sizes sz;
+    const dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!importance || !rtable || !widths) return DPA_ERR_INVALID_ARG;
+    const int E = desc->n_experts, B = desc->bits, kmin = desc->kmin, kmax = desc->kmax;
+    for (int e = 0; e < E; ++e)
+        if (!(importance[e] >= 0.0 && importance[e] <= 1.0e300)) return DPA_ERR_INVALID_ARG;
+    if (budget_planes < static_cast<int64_t>(E) * kmin) return DPA_ERR_INVALID_ARG;
+    const int64_t cap = static_cast<int64_t>(E) * kmax;
+    const int U = static_cast<int>(budget_planes < cap ? budget_planes : cap);
+    const double inf = std::numeric_limits<double>::infinity();
+    std::vector<double> f(static_cast<size_t>(U) + 1, 0.0), g(static_cast<size_t>(U) + 1);
+    std::vector<uint8_t> choice(static_cast<size_t>(E) * (U + 1), 0);
+    for (int e = E - 1; e >= 0; --e) {
+        const int need_after = kmin * (E - e - 1);
+        for (int u = 0; u <= U; ++u) {
+            double best = inf;
+            int bb = 0;
+            for (int b = kmin; b <= kmax; ++b) {
+                if (u - b < need_after) break;
+                const double t = importance[e] * rtable[static_cast<size_t>(e) * B + (b - 1)];
+                const double v = t + f[u - b];
+                if (v < best) {
+                    best = v;
+                    bb = b;
+                }
+            }
+            g[u] = best;
+            choice[static_cast<size_t>(e) * (U + 1) + u] = static_cast<uint8_t>(bb);
+        }
+        f.swap(g);
+    }
+    int u = U;
+    for (int e = 0; e < E; ++e) {
+        const int b = choice[static_cast<size_t>(e) * (U + 1) + u];
+        widths[e] = static_cast<uint8_t>(b);
+        u -= b;
+    }
+    return DPA_OK;
+}
+
+namespace {
+// bytes of one plane of one matrix, and of one plane's (or, uniform, the matrix's) scale data
+struct CompactGeom {
+    uint64_t plane_bytes;    // R * C / 8 (the same for gate, up and down)
+    uint64_t meta_matrix;    // uniform: a matrix's {s, z}; binary-coded: one plane's alphas
+};
+CompactGeom compact_geom(const dpa_layer_desc* d) {
+    CompactGeom g;
+    g.plane_bytes = static_cast<uint64_t>(d->hidden) * d->inter / 8;
+    const uint64_t groups = static_cast<uint64_t>(d->inter) * (d->hidden / d->group);   // R * C/G per matrix
+    g.meta_matrix = d->format == DPA_FMT_UNIFORM ? groups * 4 : groups * 2;
+    return g;
+}
+bool widths_ok(const dpa_layer_desc* d, const uint8_t* widths) {
+    for (int e = 0; e < d->n_experts; ++e)
+        if (widths[e] < d->kmin || widths[e] > d->kmax) return false;
+    return true;
+}
+uint64_t compact_expert_planes(const CompactGeom& g, int w) { return 3ull * w * g.plane_bytes; }
+uint64_t compact_expert_meta(const dpa_layer_desc* d, const CompactGeom& g, int w) {
+    return d->format == DPA_FMT_UNIFORM ? 3ull * g.meta_matrix : 3ull * w * g.meta_matrix;
+}
+}  // namespace
+
+extern "C" dpa_status dpa_compact_sizes(const dpa_layer_desc* desc, const uint8_t* widths, uint64_t* planes_bytes,
+                                        uint64_t* meta_bytes) {
+    dpa_sizes sz;
+    const dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!widths || !planes_bytes || !meta_bytes || !widths_ok(desc, widths)) return DPA_ERR_INVALID_ARG;
+    const CompactGeom g = compact_geom(desc);
+    uint64_t pb = 0, mb = 0;
+    for (int e = 0; e < desc->n_experts; ++e) {
+        pb += compact_expert_planes(g, widths[e]);
+        mb += compact_expert_meta(desc, g, widths[e]);
+    }
+    *planes_bytes = pb;
+    *meta_bytes = mb;
+    return DPA_OK;
+}
+
+extern "C" dpa_status dpa_compact_layer(const dpa_layer_desc* desc, const void* planes, const void* meta,
+                                        const uint8_t* widths, void* planes_out, void* meta_out, uint64_t* offsets) {
+    dpa_sizes sz;
+    const dpa_status st = dpa_encoded_sizes(desc, &sz);
+    if (st != DPA_OK) return st;
+    if (!planes || !meta || !widths || !planes_out || !meta_out || !offsets || !widths_ok(desc, widths))
+        return DPA_ERR_INVALID_ARG;
+    const CompactGeom g = compact_geom(desc);
+    const uint8_t* pin = static_cast<const uint8_t*>(planes);
+    const uint8_t* min_ = static_cast<const uint8_t*>(meta);
+    uint8_t* pout = static_cast<uint8_t*>(planes_out);
+    uint8_t* mout = static_cast<uint8_t*>(meta_out);
+    uint64_t po = 0, mo = 0;
+    for (int e = 0; e < desc->n_experts; ++e) {
+        const int w = widths[e];
+        offsets[2 * e] = po;
+        offsets[2 * e + 1] = mo;
+        for (int m = 0; m < 3; ++m) {   // the first w planes of each matrix: a prefix of its bytes
+            const uint8_t* src = pin + static_cast<uint64_t>(e) * sz.planes_per_expert + sz.planes_matrix_offset[m];
+            std::memcpy(pout + po, src, w * g.plane_bytes);
+            po += w * g.plane_bytes;
+        }
+        for (int m = 0; m < 3; ++m) {
+            const uint8_t* src = min_ + static_cast<uint64_t>(e) * sz.meta_per_expert + sz.meta_matrix_offset[m];
+            const uint64_t n = desc->format == DPA_FMT_UNIFORM ? g.meta_matrix : w * g.meta_matrix;
+            std::memcpy(mout + mo, src, n);
+            mo += n;
+        }
     }
     return DPA_OK;
 }

@@ -448,8 +448,14 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
     const int n_chunks = (K + static_cast<int>(L.CK) - 1) / static_cast<int>(L.CK);
     const int n_items = static_cast<int>(__ldcg(&a.hdr->n_vgroups)) * n_rb;
     // this CTA's contiguous range of items
-    const int it0 = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
-    const int it1 = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
+    int it0 = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
+    int it1 = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
+    if (a.vstart && a.vgrid == static_cast<int>(gridDim.x) && n_items > static_cast<int>(gridDim.x)) {
+        // ranges balanced by the groups' estimated work (written for batches with more items
+        // than CTAs)
+        it0 = min(__ldcg(a.vstart + blockIdx.x), n_items);
+        it1 = min(__ldcg(a.vstart + blockIdx.x + 1), n_items);
+    }
 
     if (warp == kCW) {
         // ================================ producer ================================
@@ -492,8 +498,30 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                 ++gcount;
                 groups_issued = gcount;
             }
-            const uint8_t* pbase = a.planes + static_cast<uint64_t>(e) * a.planes_per_expert;
-            const uint8_t* mbase = a.meta + static_cast<uint64_t>(e) * a.meta_per_expert;
+            // the expert's planes and scale data: the full layout, or the compact layer of
+            // per-expert stored widths (expert e holds w_e planes per matrix at its own offsets)
+            const uint8_t* pbase;
+            const uint8_t* mbase;
+            uint64_t pmat[NMAT], mplane = static_cast<uint64_t>(a.R) * ng * 2;   // BCQ alphas per plane
+            uint64_t mmat[NMAT];
+            if (a.expert_off) {
+                const uint64_t w = __ldg(a.expert_width + e);
+                pbase = a.planes + __ldg(a.expert_off + 2 * e);
+                mbase = a.meta + __ldg(a.expert_off + 2 * e + 1);
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                    pmat[m] = (a.mat0 + m) * w * plane_bytes;
+                    mmat[m] = FMT == DPA_FMT_UNIFORM ? a.meta_mat_off[a.mat0 + m] : (a.mat0 + m) * w * mplane;
+                }
+            } else {
+                pbase = a.planes + static_cast<uint64_t>(e) * a.planes_per_expert;
+                mbase = a.meta + static_cast<uint64_t>(e) * a.meta_per_expert;
+#pragma unroll
+                for (int m = 0; m < NMAT; ++m) {
+                    pmat[m] = a.planes_mat_off[a.mat0 + m];
+                    mmat[m] = a.meta_mat_off[a.mat0 + m];
+                }
+            }
             const int n_meta = FMT == DPA_FMT_UNIFORM ? NMAT : NMAT * kmax;
             for (int c = 0; c < n_chunks; ++c, ++q) {
                 const int s = q % L.nst;
@@ -515,7 +543,7 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                 if (static_cast<int>(L.CK) == K) {
                     for (int i = lane; i < NMAT * kmax; i += 32) {
                         const int p = i % kmax, m = i / kmax;
-                        const uint8_t* src = pbase + a.planes_mat_off[a.mat0 + m] + p * plane_bytes +
+                        const uint8_t* src = pbase + pmat[m] + p * plane_bytes +
                                              static_cast<uint64_t>(rb * NRT) * (K / 64) * 128;
                         bulk_g2s(st + (static_cast<size_t>(m * kMaxB + p) * NRT * (K / 64)) * 128, src,
                                  static_cast<uint32_t>(NRT * (K / 64)) * 128u, &s_full[s]);
@@ -523,7 +551,7 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                 } else
                 for (int i = lane; i < n_pc; i += 32) {
                     const int rt = i % NRT, mp = i / NRT, p = mp % kmax, m = mp / kmax;
-                    const uint8_t* src = pbase + a.planes_mat_off[a.mat0 + m] + p * plane_bytes +
+                    const uint8_t* src = pbase + pmat[m] + p * plane_bytes +
                                          static_cast<uint64_t>(rb * NRT + rt) * (K / 64) * 128 +
                                          static_cast<uint64_t>(col0 / 64) * 128;
                     bulk_g2s(st + ((static_cast<size_t>(m * kMaxB + p) * NRT + rt) * (L.CK / 64)) * 128, src,
@@ -533,10 +561,10 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
                 for (int i = lane; i < n_meta; i += 32) {
                     const uint8_t* src;
                     if (FMT == DPA_FMT_UNIFORM) {
-                        src = mbase + a.meta_mat_off[a.mat0 + i] + static_cast<uint64_t>(rb) * mrow;
+                        src = mbase + mmat[i] + static_cast<uint64_t>(rb) * mrow;
                     } else {
                         const int m = i / kmax, p = i % kmax;
-                        src = mbase + a.meta_mat_off[a.mat0 + m] + static_cast<uint64_t>(p) * a.R * ng * 2 +
+                        src = mbase + mmat[m] + static_cast<uint64_t>(p) * mplane +
                               static_cast<uint64_t>(rb) * mrow;
                     }
                     bulk_g2s(st + L.st_meta + static_cast<size_t>(i) * mrow, src, mrow, &s_full[s]);
@@ -760,6 +788,24 @@ static cudaError_t launch_kind(const VpArgs& a, cudaStream_t stream, int sms) {
     const bool big = a.R % (16 * NB) == 0 && vp_bytes<NMAT>(true, two ? 2 : 1, a.K, a.G, FMT, a.B) <= kVpMaxSmem;
     if (big) return two ? launch_variant<FMT, NB, 2, NMAT>(a, stream, sms) : launch_variant<FMT, NB, 1, NMAT>(a, stream, sms);
     return two ? launch_variant<FMT, NS, 2, NMAT>(a, stream, sms) : launch_variant<FMT, NS, 1, NMAT>(a, stream, sms);
+}
+
+template <int FMT, int NMAT>
+static bool vp_big(const VpArgs& a) {
+    constexpr int NB = NMAT == 2 ? kGuNRT : kDnNRT;
+    return a.R % (16 * NB) == 0 && vp_bytes<NMAT>(true, a.tiles_per_group == 2 ? 2 : 1, a.K, a.G, FMT, a.B) <= kVpMaxSmem;
+}
+
+int vp_rows_per_item(const VpArgs& a) {
+    bool big;
+    if (a.nmat == 2) big = a.fmt == DPA_FMT_UNIFORM ? vp_big<DPA_FMT_UNIFORM, 2>(a) : vp_big<DPA_FMT_BCQ, 2>(a);
+    else big = a.fmt == DPA_FMT_UNIFORM ? vp_big<DPA_FMT_UNIFORM, 1>(a) : vp_big<DPA_FMT_BCQ, 1>(a);
+    return 16 * (a.nmat == 2 ? (big ? kGuNRT : kGuNRTSmall) : (big ? kDnNRT : kDnNRTSmall));
+}
+
+int vp_grid(const VpArgs& a, int sms) {
+    const int items = a.max_groups * (a.R / vp_rows_per_item(a));
+    return items < sms ? (items > 0 ? items : 1) : sms;
 }
 
 cudaError_t launch_vp_gemv(const VpArgs& a, cudaStream_t stream, int sms) {

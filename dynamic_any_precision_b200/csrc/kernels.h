@@ -69,7 +69,13 @@ struct AllocArgs {
     // kVRecInts ints (see kVRec*); count in hdr->n_vgroups
     int32_t* vrec;            // [P/4 + E*nk][kVRecInts]
     int vtiles_per_group;
+    // per GEMV launch j (0: gate/up, 1: down), unless vstart[j] is nullptr: the first item of each
+    // of its vgrid[j] CTAs over items (record, row block; vnrb[j] row blocks per record), with
+    // equal shares of the estimated work; vstart[j][vgrid[j]] = the item count
+    int32_t* vstart[2];
+    int vgrid[2], vnrb[2];
     const uint8_t* expert_k;  // [E] plane count per expert (DPA_ALLOC_EXPERT_TABLE)
+    const uint8_t* expert_width;   // nullptr, or [E] stored planes per expert: no pair reads more
 };
 // Counters of the grid-wide bisection (zeroed by the launcher before every call).
 constexpr int kCoopRoundsMax = 16;
@@ -159,8 +165,17 @@ struct VpArgs {
     float* out;               // [P][R] by grouped position
     WsHeader* hdr;
     int max_groups;           // host bound of the token groups
+    const uint64_t* expert_off;   // nullptr (full layout), or [E][2] byte offsets of each expert's
+                                  // planes and scale data in the compact layer of stored widths
+    const uint8_t* expert_width;  // [E] stored planes per expert (with expert_off)
+    const int32_t* vstart;    // nullptr (equal item counts per CTA), or [grid + 1] first item of each
+                              // CTA, balanced by estimated work (written by the allocation)
+    int vgrid;                // the grid vstart was written for (used only when the launch matches)
 };
 cudaError_t launch_vp_gemv(const VpArgs& a, cudaStream_t stream, int sms);
+// The launch geometry of a variant, as launch_vp_gemv will use it: CTAs and rows per item.
+int vp_grid(const VpArgs& a, int sms);
+int vp_rows_per_item(const VpArgs& a);
 // tiles per token group the layer's shapes allow (2 where the group slots fit, else 1)
 int vp_tiles_per_group(int K_gateup, int K_down, int G, int fmt, int B);
 // dynamic shared memory of one CTA of a variant

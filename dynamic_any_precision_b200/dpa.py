@@ -45,7 +45,8 @@ class Sizes(ctypes.Structure):
 class LayerWeights(ctypes.Structure):
     _fields_ = [("planes", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("rtable", ctypes.c_void_p),
                 ("w_router", ctypes.c_void_p), ("shared_gate", ctypes.c_void_p),
-                ("shared_up", ctypes.c_void_p), ("shared_down", ctypes.c_void_p)]
+                ("shared_up", ctypes.c_void_p), ("shared_down", ctypes.c_void_p),
+                ("expert_width", ctypes.c_void_p), ("expert_offsets", ctypes.c_void_p)]
 
 
 class Aux(ctypes.Structure):
@@ -62,7 +63,7 @@ EXPORTED = ("dpa_encoded_sizes", "dpa_encode", "dpa_export_codes", "dpa_export_m
             "dpa_allocate", "dpa_allocate_ex", "dpa_calibrate_threshold", "dpa_forward_workspace_size",
             "dpa_moe_forward", "dpa_device_status", "dpa_status_string", "dpa_version", "dpa_residual_rmsnorm",
             "dpa_debug_timeout_probe", "dpa_distortion_tensor", "dpa_profile_prefill", "dpa_solve_expert_rates",
-            "dpa_stream_prefixes")
+            "dpa_stream_prefixes", "dpa_solve_stored_widths", "dpa_compact_sizes", "dpa_compact_layer")
 
 _lib = None
 
@@ -96,6 +97,9 @@ def lib() -> ctypes.CDLL:
     L.dpa_debug_timeout_probe.argtypes = [vp, sz, i32, ctypes.c_uint64, vp]
     L.dpa_stream_prefixes.argtypes = [P(LayerDesc), vp, vp, vp, vp, i32, vp, vp, P(ctypes.c_uint64), vp]
     L.dpa_residual_rmsnorm.argtypes = [vp, vp, i32, i32, vp, vp]
+    L.dpa_solve_stored_widths.argtypes = [P(LayerDesc), vp, vp, ctypes.c_int64, vp]
+    L.dpa_compact_sizes.argtypes = [P(LayerDesc), vp, P(ctypes.c_uint64), P(ctypes.c_uint64)]
+    L.dpa_compact_layer.argtypes = [P(LayerDesc), vp, vp, vp, vp, vp, vp]
     L.dpa_status_string.argtypes = [i32]
     L.dpa_status_string.restype = ctypes.c_char_p
     L.dpa_version.argtypes = []
@@ -279,13 +283,16 @@ def calibrate_threshold(desc: LayerDesc, scores, target, ws, stream=None):
 class DeviceLayer:
     """Encoded layer resident in device memory (torch tensors) plus its C weight struct."""
 
-    def __init__(self, desc: LayerDesc, planes, meta, rtable, w_router, shared=None):
+    def __init__(self, desc: LayerDesc, planes, meta, rtable, w_router, shared=None, widths=None, offsets=None):
+        """widths (uint8 [E]) and offsets (uint64 [E][2] as int64) on the device: a compact layer
+        of per-expert stored widths (dpa_compact_layer); both None: the full layout."""
         self.desc = desc
         self.planes, self.meta, self.rtable, self.w_router = planes, meta, rtable, w_router
         self.shared = shared
+        self.widths, self.offsets = widths, offsets
         sg, su, sd = shared if shared is not None else (None, None, None)
         self.weights = LayerWeights(_dptr(planes), _dptr(meta), _dptr(rtable), _dptr(w_router), _dptr(sg),
-                                    _dptr(su), _dptr(sd))
+                                    _dptr(su), _dptr(sd), _dptr(widths), _dptr(offsets))
 
     @classmethod
     def from_host(cls, desc: LayerDesc, planes: np.ndarray, meta: np.ndarray, rtable: np.ndarray,
@@ -349,6 +356,32 @@ def stream_prefixes(desc: LayerDesc, host_planes, host_meta, experts, kplanes, d
                                      _ptr(kp), int(ex.size), _dptr(dev_planes), _dptr(dev_meta), ctypes.byref(nbytes),
                                      _stream(stream)), "dpa_stream_prefixes")
     return int(nbytes.value)
+
+
+def solve_stored_widths(desc: LayerDesc, importance: np.ndarray, rtable: np.ndarray, budget_planes: int) -> np.ndarray:
+    """Per-expert stored planes (uint8 [E]) minimising sum_e importance[e] * rtable[e][b_e - 1]
+    within a budget of stored planes over all experts (host)."""
+    imp = np.ascontiguousarray(importance, dtype=np.float64)
+    r = np.ascontiguousarray(rtable, dtype=np.float64)
+    w = np.zeros(desc.n_experts, dtype=np.uint8)
+    _check(lib().dpa_solve_stored_widths(ctypes.byref(desc), _ptr(imp), _ptr(r), int(budget_planes), _ptr(w)),
+           "dpa_solve_stored_widths")
+    return w
+
+
+def compact_layer(desc: LayerDesc, planes: np.ndarray, meta: np.ndarray, widths: np.ndarray):
+    """Host compact layer for per-expert stored widths: (planes, meta, offsets uint64 [E][2])."""
+    w = np.ascontiguousarray(widths, dtype=np.uint8)
+    pb, mb = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check(lib().dpa_compact_sizes(ctypes.byref(desc), _ptr(w), ctypes.byref(pb), ctypes.byref(mb)),
+           "dpa_compact_sizes")
+    po = np.zeros(pb.value, dtype=np.uint8)
+    mo = np.zeros(mb.value, dtype=np.uint8)
+    off = np.zeros((desc.n_experts, 2), dtype=np.uint64)
+    _check(lib().dpa_compact_layer(ctypes.byref(desc), _ptr(np.ascontiguousarray(planes)),
+                                   _ptr(np.ascontiguousarray(meta)), _ptr(w), _ptr(po), _ptr(mo), _ptr(off)),
+           "dpa_compact_layer")
+    return po, mo, off
 
 
 def device_error_detail(ws) -> Tuple[int, int]:

@@ -113,6 +113,17 @@ typedef struct dpa_layer_weights {
     const void* shared_gate;
     const void* shared_up;
     const void* shared_down;
+    /* Per-expert stored widths (MatMoE, review "Core Contribution": each expert's maximum
+     * bit-width, chosen offline under a memory budget). Both NULL: every expert holds all B
+     * planes in the layout of dpa_encode. Both set: the layer is the compact blob of
+     * dpa_compact_layer, expert_width uint8 [E] (device) holds each expert's stored planes
+     * (kmin..kmax) and expert_offsets uint64 [E][2] (device) the byte offsets of each expert's
+     * planes and scale data in `planes` and `meta`; every allocation policy then reads at most
+     * expert_width[e] planes of expert e (the Lagrangian optimises within the widths; the other
+     * policies' counts are clipped to them). The compact layout runs the decode GEMV kernels
+     * only (DPA_PATH_TC returns DPA_ERR_UNSUPPORTED). */
+    const uint8_t* expert_width;
+    const uint64_t* expert_offsets;
 } dpa_layer_weights;
 
 /* Optional device outputs of dpa_moe_forward's decision path (any field may be NULL).
@@ -373,6 +384,38 @@ dpa_status dpa_residual_rmsnorm(const void* y, float* h, int n_tokens, int hidde
 dpa_status dpa_stream_prefixes(const dpa_layer_desc* desc, const void* host_planes, const void* host_meta,
                                const int32_t* experts, const uint8_t* kplanes, int n, void* dev_planes,
                                void* dev_meta, uint64_t* bytes_out, void* stream);
+
+/* ---- Per-expert stored widths ----
+ * MatMoE, review "Core Contribution": offline, an ILP picks each expert's maximum bit-width
+ * (2/3/4) under a memory budget, with the metric routing score x Fisher-approximated Hessian
+ * x quantization error. Here the ILP is
+ *     minimise sum_e fl(importance[e] * rtable[e][b_e - 1])
+ *     subject to sum_e b_e <= budget_planes,  kmin <= b_e <= kmax,
+ * solved exactly by dynamic programming over the experts from the last
+ * (f(e, u) = min_b fl(fl(importance[e] rtable[e][b-1]) + f(e+1, u-b)), ties to the smaller b;
+ * the widths are read off from u = min(budget, E kmax) forwards). Every plane of every expert
+ * has the same size, so the memory budget is a count of stored planes over all experts.
+ * importance: fp64 [E] (host), e.g. each expert's routing mass over a calibration batch (the sum
+ * of its routed pairs' gates); no Fisher information is used (factor 1). rtable: fp64 [E][B]
+ * (host, from dpa_encode). widths: uint8 [E] (host, written). Host, synchronous.
+ * Errors: DPA_ERR_INVALID_ARG for NULL pointers, non-finite or negative importance, or a budget
+ * below E * kmin. */
+dpa_status dpa_solve_stored_widths(const dpa_layer_desc* desc, const double* importance, const double* rtable,
+                                   int64_t budget_planes, uint8_t* widths);
+
+/* Bytes of the compact layer for per-expert widths (host): expert e holds, per matrix (gate,
+ * up, down in order), its first widths[e] planes (the prefix of dpa_encode's planes), then its
+ * scale data (uniform: as in dpa_encode; binary-coded: the first widths[e] planes' alphas per
+ * matrix). Errors: DPA_ERR_INVALID_ARG for NULL pointers or a width outside [kmin, kmax]. */
+dpa_status dpa_compact_sizes(const dpa_layer_desc* desc, const uint8_t* widths, uint64_t* planes_bytes,
+                             uint64_t* meta_bytes);
+
+/* Builds the compact layer from dpa_encode's planes and meta (host buffers; planes_out and
+ * meta_out of dpa_compact_sizes' sizes, caller-owned) and the per-expert byte offsets
+ * offsets[e][0] (planes) and offsets[e][1] (meta), uint64 [E][2]. Experts follow in order.
+ * Host, synchronous. Errors: as dpa_compact_sizes. */
+dpa_status dpa_compact_layer(const dpa_layer_desc* desc, const void* planes, const void* meta, const uint8_t* widths,
+                             void* planes_out, void* meta_out, uint64_t* offsets);
 
 /* Test support for the device-side failure handling (the pages have no counterpart).
  * Runs one of the library's bounded device waits against a barrier that nothing completes,

@@ -16,7 +16,8 @@ Pages (cited by title and section):
   [MAT]  MatMoE: Matryoshka Mixture-of-Experts with Dynamic Mixed-Precision Quantization,
          Abstract and review section "Core Contribution"
          (floor-and-compensation, bitplane storage, routing-score driven bit-widths
-          found by a binary search to a target average bit-width)
+          found by a binary search to a target average bit-width, an offline ILP over each
+          expert's maximum bit-width under a memory budget)
 
 Where the pages leave a step open, the reading taken is stated at the function.
 
@@ -46,6 +47,12 @@ Parity status of each function (what pins it; see tests/test_oracle_pins.py):
   solve_expert_rates  pinned: brute-force count-weighted optimum (Everett) on tiny inputs;
                       frequency cancels (scaling counts leaves every k(lambda) unchanged);
                       endpoint targets; monotone plane count along the bisection
+  routing_mass        pinned: equals an independent scatter-add of the gates
+  solve_stored_widths pinned: lexicographically smallest optimum by exhaustive enumeration
+                      (exact integer data, non-convex residuals so greedy upgrades fail);
+                      endpoint budgets (all kmin, all kmax); cost non-increasing in the budget
+  allocate (cap)      pinned: k never above the width; width kmax for all = no cap; width kmin
+                      for all = every pair at kmin; budget criterion kept
   expert_ffn / moe    pinned: hand-worked tiny layer; top-1 identity; linearity of the
                       gate-weighted combine; prefix property (low bits ignored); at
                       target = kmax = B the layer equals a torch fp32 computation (topk,
@@ -328,12 +335,18 @@ def route(x_bits: np.ndarray, wr_bits: np.ndarray, K: int, norm_topk: int,
 # ---------------------------------------------------------------------------
 
 
-def pair_costs(idx: np.ndarray, gates: np.ndarray, r: np.ndarray, kmin: int, kmax: int) -> np.ndarray:
-    """c[p][k - kmin] = fl(g_p * r_{e_p}(k)) for the pairs in token-major, slot order."""
+def pair_costs(idx: np.ndarray, gates: np.ndarray, r: np.ndarray, kmin: int, kmax: int,
+               cap: Optional[np.ndarray] = None) -> np.ndarray:
+    """c[p][k - kmin] = fl(g_p * r_{e_p}(k)) for the pairs in token-major, slot order; with
+    per-expert stored widths `cap`, plane counts above the expert's width cost +inf (never
+    chosen: an expert stored at b planes can be read at no more than b)."""
     e = idx.reshape(-1)
     g = gates.reshape(-1)
     ks = np.arange(kmin, kmax + 1)
-    return g[:, None] * r[e][:, ks - 1]
+    c = g[:, None] * r[e][:, ks - 1]
+    if cap is not None:
+        c = np.where(ks[None, :] > np.asarray(cap)[e][:, None], np.inf, c)
+    return c
 
 
 def choose_k(c: np.ndarray, lam: float, kmin: int, kmax: int) -> np.ndarray:
@@ -343,11 +356,11 @@ def choose_k(c: np.ndarray, lam: float, kmin: int, kmax: int) -> np.ndarray:
 
 
 def allocate(idx: np.ndarray, gates: np.ndarray, r: np.ndarray, kmin: int, kmax: int,
-             target: float, iters: int = 64, trace: Optional[list] = None):
-    """Returns (k int [T][K], lambda)."""
+             target: float, iters: int = 64, trace: Optional[list] = None, cap: Optional[np.ndarray] = None):
+    """Returns (k int [T][K], lambda). `cap`: per-expert stored widths (k <= cap[e])."""
     if not (kmin <= target <= kmax):
         raise ValueError("target outside [kmin, kmax]")
-    c = pair_costs(idx, gates, r, kmin, kmax)
+    c = pair_costs(idx, gates, r, kmin, kmax, cap)
     P = c.shape[0]
     budget = float(target) * float(P)
     lo = 0.0
@@ -567,30 +580,92 @@ def shared_outputs(x_row: np.ndarray, shared) -> List[np.ndarray]:
             for s in range(sg.shape[0])]
 
 
+# ---------------------------------------------------------------------------
+# Per-expert stored width ([MAT] Core Contribution: offline, an ILP picks each expert's maximum
+# bit-width, 2/3/4, under a memory budget; the metric is routing score x Fisher-approximated
+# Hessian x quantization error).
+#   Readings: the routing score of expert e is its routing mass, the sum of the gates of its
+#   routed pairs over a calibration batch (in token-major slot order); no Fisher information is
+#   available, so the Hessian factor is 1; the quantization error at b stored planes is the
+#   residual r_e(b). Every plane of every expert has the same size, so the memory budget is a
+#   number of stored planes. The ILP
+#       minimise sum_e fl(imp_e * r_e(b_e))  s.t.  sum_e b_e <= budget,  kmin <= b_e <= kmax
+#   is solved exactly by dynamic programming over the experts from the last:
+#       f(E, u) = 0;  f(e, u) = min_b fl(fl(imp_e * r_e(b)) + f(e+1, u - b)),
+#   b over [kmin, kmax] with u - b >= kmin * (E - e - 1), ties to the smaller b; the widths
+#   are read off from u = budget (clipped to E * kmax) forwards.
+# ---------------------------------------------------------------------------
+
+
+def routing_mass(idx: np.ndarray, gates: np.ndarray, n_experts: int) -> np.ndarray:
+    """Sum of each expert's gates over the routed pairs, in token-major slot order."""
+    m = np.zeros(n_experts, dtype=np.float64)
+    for e, g in zip(idx.reshape(-1).tolist(), gates.reshape(-1).tolist()):
+        m[e] = m[e] + g
+    return m
+
+
+def solve_stored_widths(importance: np.ndarray, r: np.ndarray, kmin: int, kmax: int, budget: int) -> np.ndarray:
+    """Stored planes per expert (int [E]) minimising the importance-weighted residual."""
+    E = len(importance)
+    if budget < E * kmin:
+        raise ValueError("budget below every expert at kmin")
+    budget = min(int(budget), E * kmax)
+    inf = float("inf")
+    f = [0.0] * (budget + 1)                      # f(E, u)
+    choice = [[0] * (budget + 1) for _ in range(E)]
+    for e in range(E - 1, -1, -1):
+        need_after = kmin * (E - e - 1)
+        g = [inf] * (budget + 1)
+        for u in range(budget + 1):
+            best, bb = inf, 0
+            for b in range(kmin, kmax + 1):
+                if u - b < need_after:
+                    break
+                v = float(np.float64(importance[e]) * np.float64(r[e][b - 1])) + f[u - b]
+                if v < best:
+                    best, bb = v, b
+            g[u], choice[e][u] = best, bb
+        f = g
+    widths, u = [], budget
+    for e in range(E):
+        b = choice[e][u]
+        widths.append(b)
+        u -= b
+    return np.array(widths, dtype=np.int64)
+
+
 ALLOC_LAGRANGE, ALLOC_UNIFORM, ALLOC_THRESHOLD, ALLOC_EXPERT_TABLE = 0, 1, 2, 3
 
 
 def allocate_policy(policy: int, idx: np.ndarray, gates: np.ndarray, r_table: Optional[np.ndarray], kmin: int,
                     kmax: int, target: float, threshold: Optional[float] = None,
-                    expert_k: Optional[np.ndarray] = None):
+                    expert_k: Optional[np.ndarray] = None, cap: Optional[np.ndarray] = None):
     """Plane counts [T][K] and the policy's multiplier (lambda; the threshold; 0 for uniform and
-    for the expert-rate table)."""
-    if policy == ALLOC_EXPERT_TABLE:
-        return allocate_expert_table(idx, expert_k), 0.0
+    for the expert-rate table). With per-expert stored widths `cap`, the Lagrangian optimises
+    within them (costs above a width are +inf) and the other policies' counts are clipped to
+    them."""
     if policy == ALLOC_LAGRANGE:
-        return allocate(idx, gates, r_table, kmin, kmax, target)
-    if policy == ALLOC_UNIFORM:
-        return allocate_uniform(idx.size, kmin, kmax, target).reshape(idx.shape), 0.0
-    if policy == ALLOC_THRESHOLD:
-        return allocate_threshold(gates, threshold, kmin, kmax).reshape(idx.shape), float(threshold)
-    raise ValueError("unknown allocation policy")
+        return allocate(idx, gates, r_table, kmin, kmax, target, cap=cap)
+    if policy == ALLOC_EXPERT_TABLE:
+        k, lam = allocate_expert_table(idx, expert_k), 0.0
+    elif policy == ALLOC_UNIFORM:
+        k, lam = allocate_uniform(idx.size, kmin, kmax, target).reshape(idx.shape), 0.0
+    elif policy == ALLOC_THRESHOLD:
+        k, lam = allocate_threshold(gates, threshold, kmin, kmax).reshape(idx.shape), float(threshold)
+    else:
+        raise ValueError("unknown allocation policy")
+    if cap is not None:
+        k = np.minimum(k, np.asarray(cap, dtype=np.int64)[idx])
+    return k, lam
 
 
 def moe_forward(x_bits: np.ndarray, wr_bits: np.ndarray, experts: Dict[int, Dict], shape,
                 target: float, shared: Optional[Tuple[np.ndarray, np.ndarray, np.ndarray]] = None,
                 r_table: Optional[np.ndarray] = None, logits: Optional[np.ndarray] = None,
                 token_subset: Optional[Sequence[int]] = None, policy: int = ALLOC_LAGRANGE,
-                threshold: Optional[float] = None, expert_k: Optional[np.ndarray] = None):
+                threshold: Optional[float] = None, expert_k: Optional[np.ndarray] = None,
+                widths: Optional[np.ndarray] = None):
     """One MoE layer. `experts` maps expert id -> encode_expert() output (only the experts that
     are routed to are needed); `r_table` is [E][B] (all experts' residuals; defaults to the
     encoded ones, which then must cover every expert). Returns y fp64 [T][H] (rows outside
@@ -599,7 +674,8 @@ def moe_forward(x_bits: np.ndarray, wr_bits: np.ndarray, experts: Dict[int, Dict
     idx, g, logits = route(x_bits, wr_bits, shape.top_k, shape.norm_topk, logits)
     if r_table is None and policy == ALLOC_LAGRANGE:
         r_table = np.stack([experts[e]["r"] for e in range(shape.n_experts)])
-    k, lam = allocate_policy(policy, idx, g, r_table, shape.kmin, shape.kmax, target, threshold, expert_k)
+    k, lam = allocate_policy(policy, idx, g, r_table, shape.kmin, shape.kmax, target, threshold, expert_k,
+                             cap=widths)
     x = bf16_bits_to_f64(x_bits)
     T = x.shape[0]
     toks = range(T) if token_subset is None else token_subset

@@ -772,3 +772,82 @@ def test_rmsnorm_closed_form_and_bf16_rounding():
     for v_, b in zip(vals, bits):
         got = Fraction(float(np.array([int(b) << 16], dtype=np.uint32).view(np.float32)[0]))
         assert got == rne_to_format(Fraction(v_), 7, -126), v_
+
+
+# ---- per-expert stored widths (MatMoE, "Core Contribution": offline ILP over 2/3/4-bit
+# maximum widths under a memory budget) ----
+
+def _brute_widths(imp, r, kmin, kmax, budget):
+    """Lexicographically smallest optimal widths by enumeration (exact: integer data)."""
+    import itertools
+    best, arg = None, None
+    for ws in itertools.product(range(kmin, kmax + 1), repeat=len(imp)):
+        if sum(ws) > budget:
+            continue
+        cost = sum(int(imp[e]) * int(r[e][b - 1]) for e, b in enumerate(ws))
+        if best is None or cost < best:
+            best, arg = cost, ws
+    return np.array(arg, dtype=np.int64)
+
+
+def test_stored_widths_dp_matches_brute_force():
+    rng = np.random.default_rng(11)
+    for trial in range(60):
+        E = int(rng.integers(1, 5))
+        kmin, kmax = (2, 4) if trial % 2 else (1, 3)
+        imp = rng.integers(1, 10, size=E).astype(np.float64)
+        # residuals: integers, non-increasing in the width but not convex (plane steps of uneven
+        # worth), so that a greedy per-step upgrade would not be optimal
+        steps = rng.integers(0, 50, size=(E, 4))
+        r = np.cumsum(steps[:, ::-1], axis=1)[:, ::-1].astype(np.float64)
+        for budget in range(E * kmin, E * kmax + 2):
+            got = O.solve_stored_widths(imp, r, kmin, kmax, budget)
+            want = _brute_widths(imp, r, kmin, kmax, budget)
+            assert np.array_equal(got, want), (trial, budget, got, want)
+
+
+def test_stored_widths_endpoints_and_budget():
+    rng = np.random.default_rng(12)
+    imp = rng.random(16) + 0.1
+    r = np.sort(rng.random((16, 4)) * 100, axis=1)[:, ::-1].copy()
+    assert np.all(O.solve_stored_widths(imp, r, 2, 4, 32) == 2)          # budget = E * kmin
+    assert np.all(O.solve_stored_widths(imp, r, 2, 4, 64) == 4)          # budget = E * kmax
+    assert np.all(O.solve_stored_widths(imp, r, 2, 4, 1000) == 4)        # more than enough
+    prev = None
+    for budget in range(32, 65):
+        w = O.solve_stored_widths(imp, r, 2, 4, budget)
+        assert w.sum() <= budget and np.all((w >= 2) & (w <= 4))
+        cost = float(np.sum(imp * r[np.arange(16), w - 1]))
+        assert prev is None or cost <= prev + 1e-12                       # more memory never hurts
+        prev = cost
+    with pytest.raises(ValueError):
+        O.solve_stored_widths(imp, r, 2, 4, 31)
+
+
+def test_routing_mass_is_the_gate_sum_per_expert():
+    rng = np.random.default_rng(13)
+    idx = np.stack([rng.choice(8, 3, replace=False) for _ in range(20)])
+    g = rng.random((20, 3))
+    want = np.zeros(8)
+    np.add.at(want, idx.reshape(-1), g.reshape(-1))
+    assert np.allclose(O.routing_mass(idx, g, 8), want, rtol=0, atol=1e-12)
+
+
+def test_allocation_respects_stored_widths():
+    rng = np.random.default_rng(14)
+    E, T, K = 12, 40, 3
+    idx = np.stack([rng.choice(E, K, replace=False) for _ in range(T)])
+    g = -np.sort(-rng.dirichlet(np.ones(K), size=T), axis=1)
+    r = np.sort(rng.random((E, 4)) * 10, axis=1)[:, ::-1].copy()
+    cap = rng.integers(2, 5, size=E)
+    for target in (2.0, 2.7, 3.4, 4.0):
+        k, _ = O.allocate(idx, g, r, 2, 4, target, cap=cap)
+        assert np.all(k <= cap[idx]) and np.all(k >= 2)
+        assert k.sum() <= target * k.size
+        k_full, _ = O.allocate(idx, g, r, 2, 4, target, cap=np.full(E, 4))
+        assert np.array_equal(k_full, O.allocate(idx, g, r, 2, 4, target)[0])   # width kmax: no cap
+    k_min, _ = O.allocate(idx, g, r, 2, 4, 4.0, cap=np.full(E, 2))
+    assert np.all(k_min == 2)
+    for pol in (O.ALLOC_UNIFORM, O.ALLOC_THRESHOLD):
+        k, _ = O.allocate_policy(pol, idx, g, r, 2, 4, 3.0, threshold=0.3, cap=cap)
+        assert np.all(k <= cap[idx])
