@@ -18,9 +18,14 @@
 // taking at every level exactly the branch the sequential bisection takes. The resulting lo,
 // hi and lambda are bit-identical to the step-by-step loop.
 //
-// Then pairs are grouped by key (expert, k) with a counting sort, and for every expert with
-// pairs the kernel writes a work descriptor and a table of two-token tiles (same k) that the
-// expert GEMV consumes.
+// Where the steps run: up to 64 pairs one CTA, speculating (a replay against the summed hull
+// breakpoints, checked exactly, trees from the first disagreement); 65 to 2048 pairs a cluster of
+// 8 CTAs exchanging each tree's counts through distributed shared memory; beyond, every SM
+// (cooperative launch, grid barrier per tree).
+//
+// Then pairs are grouped by key (expert, k) with a counting sort; per expert the prefill GEMM's
+// token tiles and the expert GEMV's token-group records, and for the two GEMV launches the
+// work-balanced ranges of their CTAs.
 #include <cstdint>
 
 #include <math_constants.h>
@@ -34,7 +39,7 @@ namespace {
 constexpr int kAllocThreads = 1024;       // maximum block size
 constexpr int kSmemCostDoubles = 8192;    // costs kept in shared memory up to this many
 constexpr int kSmallP = 64;               // up to this many pairs one warp runs the bisection
-constexpr int kSpecMaxP = 2048;           // up to this many pairs the whole block speculates and verifies
+constexpr int kSpecMaxP = 2048;           // up to this many pairs (Lagrangian): the cluster bisection
 constexpr int kCoopThreads = 512;         // grid-wide bisection: threads per CTA
 constexpr int kCoopMaxPairsPerBlock = 6144;   // shared-memory costs: 6144 pairs x 32 B = 192 KB per CTA
 constexpr int kCoopDepth = 6;             // bisection steps per grid round (63 midpoints)
@@ -150,7 +155,7 @@ __device__ __forceinline__ void block_incl_scan_n(int (&v)[NV], int (*s_tmp)[32]
 
 // Shared-memory carve-up: [costs (if they fit)] [counts E*nk] [seg E*nk+1] [sorted P] [k P]
 struct AllocSmem {
-    size_t costs, counts, seg, sorted, kk, bp, bj, ptok, rexp, rfirst, total;
+    size_t costs, counts, seg, sorted, kk, ptok, rexp, rfirst, total;
     bool costs_in_smem;
 };
 
@@ -169,13 +174,6 @@ __host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk, boo
     off += static_cast<size_t>(P) * 4;
     L.kk = off;
     off += static_cast<size_t>(P);
-    // breakpoints of the speculative bisection (mid-size batches): P*(nk-1) doubles and ints
-    const size_t nbp = (P > kSmallP && P <= kSpecMaxP && L.costs_in_smem) ? static_cast<size_t>(P) * (nk - 1) : 0;
-    off = (off + 7) & ~static_cast<size_t>(7);
-    L.bp = off;
-    off += nbp * 8;
-    L.bj = off;
-    off += nbp * 4;
     off = (off + 15) & ~static_cast<size_t>(15);
     const size_t nrec = static_cast<size_t>(P) / 4 + static_cast<size_t>(E) * nk + 1;
     L.ptok = off;
@@ -186,6 +184,182 @@ __host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk, boo
     off += recs ? static_cast<size_t>(E) * 4 : 0;
     L.total = (off + 15) & ~static_cast<size_t>(15);
     return L;
+}
+
+// Grouping of the pairs by (expert, k) once every pair's plane count is in s_k (this CTA's
+// shared memory, P entries): positions, the prefill GEMM's token tiles, the GEMV records and
+// the GEMV launches' work-balanced CTA ranges. Whole block.
+__device__ void group_pairs(const AllocArgs& a, unsigned char* smem, const AllocSmem& Ls, int P, int nk,
+                            const uint8_t* s_k, int* s_tmp, int (*s_scan5)[32]) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+
+    // ---------------- grouping by (expert, k), all in shared memory ----------------
+    int* s_counts = reinterpret_cast<int*>(smem + Ls.counts);
+    int* s_seg = reinterpret_cast<int*>(smem + Ls.seg);
+    int* s_sorted = reinterpret_cast<int*>(smem + Ls.sorted);
+    const int nkeys = a.E * nk;
+    for (int i = tid; i < nkeys; i += blockDim.x) s_counts[i] = 0;
+    __syncthreads();
+    for (int p = tid; p < P; p += blockDim.x) atomicAdd(&s_counts[a.idx[p] * nk + (s_k[p] - a.kmin)], 1);
+    __syncthreads();
+    {   // exclusive scan of the counts into s_seg; counts become placement cursors
+        const int per = (nkeys + blockDim.x - 1) / blockDim.x;
+        const int k0 = tid * per, k1 = min(nkeys, k0 + per);
+        int run = 0;
+        for (int i = k0; i < k1; ++i) run += s_counts[i];
+        int base = block_incl_scan(run, s_tmp) - run;
+        for (int i = k0; i < k1; ++i) {
+            const int c = s_counts[i];
+            s_seg[i] = base;
+            s_counts[i] = base;
+            base += c;
+        }
+        if (tid == 0) s_seg[nkeys] = P;
+    }
+    __syncthreads();
+    int* s_ptok = reinterpret_cast<int*>(smem + Ls.ptok);   // token of each grouped position
+    for (int p = tid; p < P; p += blockDim.x) {
+        const int key = a.idx[p] * nk + (s_k[p] - a.kmin);
+        const int pos = atomicAdd(&s_counts[key], 1);
+        const int tok = p / a.K;
+        s_sorted[pos] = p;
+        if (a.vrec) s_ptok[pos] = tok;
+        a.pair_pos[p] = pos;
+        if (a.pos_tok) a.pos_tok[pos] = tok;
+    }
+    __syncthreads();
+    // Per expert: the prefill GEMM's token tiles (one (expert, k) class each) and its GEMV records
+    // (groups of up to vtpg tiles of up to 4 pairs of one class, classes ascending in k); experts
+    // in rounds of blockDim so that both lists stay in ascending expert order. Each record's work
+    // weight goes to s_rexp for the balanced ranges below.
+    int rank_base = 0, gt_base = 0, vg_base = 0;
+    const int vtpg = a.vtiles_per_group > 0 ? a.vtiles_per_group : 1;
+    int* s_rexp = reinterpret_cast<int*>(smem + Ls.rexp);   // [records] work weight, then its prefix
+    for (int e0 = 0; e0 < a.E; e0 += blockDim.x) {
+        const int e = e0 + tid;
+        int km = 0, ngt = 0, nvt = 0;
+        if (e < a.E) {
+            for (int i = 0; i < nk; ++i) {
+                const int n = s_seg[e * nk + i + 1] - s_seg[e * nk + i];
+                if (n > 0) km = a.kmin + i;
+                ngt += (n + kGemmTileTokens - 1) / kGemmTileTokens;
+                nvt += (n + 3) >> 2;
+            }
+        }
+        const int nvg = a.vrec ? (nvt + vtpg - 1) / vtpg : 0;
+        const int flag = km > 0 ? 1 : 0;
+        int sc[3] = {flag, a.gtiles ? ngt : 0, nvg};   // one block scan of the three counts
+        block_incl_scan_n<3>(sc, s_scan5);
+        if (a.gtiles && ngt > 0) {   // token tiles of the prefill GEMMs: one (expert, k) class each
+            int t = gt_base + sc[1] - ngt;
+            for (int i = 0; i < nk; ++i) {
+                const int s0 = s_seg[e * nk + i];
+                const int n = s_seg[e * nk + i + 1] - s0;
+                for (int j = 0; j < n; j += kGemmTileTokens)
+                    a.gtiles[t++] = make_int4(e, a.kmin + i, s0 + j, min(kGemmTileTokens, n - j));
+            }
+        }
+        if (a.vrec && nvg > 0) {
+            // this expert's records: its tiles in class order, vtpg per record, each record of
+            // kVRecInts ints written as eight 16-byte stores; its work weight to s_rexp[r]
+            int r = vg_base + sc[2] - nvg;
+            int t = 0, kk0 = 0, nn0 = 0, qq0 = 0, kk1 = 0, nn1 = 0, qq1 = 0;
+            for (int i = 0; i < nk; ++i) {
+                const int s0 = s_seg[e * nk + i];
+                const int n = s_seg[e * nk + i + 1] - s0;
+                for (int j = 0; j < n; j += 4) {
+                    if (t == 0) { kk0 = a.kmin + i; nn0 = min(4, n - j); qq0 = s0 + j; }
+                    else { kk1 = a.kmin + i; nn1 = min(4, n - j); qq1 = s0 + j; }
+                    ++t;
+                    const bool last = j + 4 >= n && i == nk - 1;
+                    bool more = false;   // any tile of a later class?
+                    if (j + 4 >= n)
+                        for (int i2 = i + 1; i2 < nk; ++i2) more |= s_seg[e * nk + i2 + 1] > s_seg[e * nk + i2];
+                    if (t == vtpg || (j + 4 >= n && !more) || last) {
+                        const int nt = t, klast = nt == 2 ? kk1 : kk0;
+                        int4* dst = reinterpret_cast<int4*>(a.vrec + static_cast<size_t>(r) * kVRecInts);
+                        auto pos = [&](int tt, int u) {
+                            const int nn = tt == 0 ? nn0 : (nt == 2 ? nn1 : 0);
+                            return u < nn ? (tt == 0 ? qq0 : qq1) + u : -1;
+                        };
+                        auto tok = [&](int tt, int u) {
+                            const int p = pos(tt, u);
+                            return p < 0 ? -1 : s_ptok[p];
+                        };
+                        dst[0] = make_int4(e, klast, nt, 0);
+                        dst[1] = make_int4(kk0, nt == 2 ? kk1 : 0, nn0, nt == 2 ? nn1 : 0);
+                        dst[2] = make_int4(pos(0, 0), pos(0, 1), pos(0, 2), pos(0, 3));
+                        dst[3] = make_int4(pos(1, 0), pos(1, 1), pos(1, 2), pos(1, 3));
+                        dst[4] = make_int4(tok(0, 0), tok(0, 1), tok(0, 2), tok(0, 3));
+                        dst[5] = make_int4(tok(1, 0), tok(1, 1), tok(1, 2), tok(1, 3));
+                        dst[6] = make_int4(0, 0, 0, 0);
+                        dst[7] = make_int4(0, 0, 0, 0);
+                        s_rexp[r] = 5 + 2 * klast + 3 * nt;   // work weight per row block
+                        ++r;
+                        t = 0;
+                    }
+                }
+            }
+        }
+        // totals of this round: the scan's last warp totals, still in shared memory; every thread
+        // reads them before the barrier below, ahead of the next round's scan
+        rank_base += s_scan5[0][nw - 1];
+        gt_base += s_scan5[1][nw - 1];
+        vg_base += s_scan5[2][nw - 1];
+        __syncthreads();
+    }
+    if (a.vrec) {
+        const bool tab0 = a.vstart[0] && vg_base * a.vnrb[0] > 2 * a.vgrid[0];
+        const bool tab1 = a.vstart[1] && vg_base * a.vnrb[1] > 2 * a.vgrid[1];
+        if (tab0 || tab1) {   // (with at most two items per CTA the GEMV splits items evenly)
+            __syncthreads();
+            // exclusive prefix of the weights over the records: s_rexp[0..vg_base]
+            const int nrec = vg_base;
+            const int per = (nrec + blockDim.x - 1) / blockDim.x;
+            const int r0 = tid * per, r1 = min(nrec, r0 + per);
+            int run = 0;
+            for (int r = r0; r < r1; ++r) run += s_rexp[r];
+            int base = block_incl_scan(run, s_tmp) - run;
+            for (int r = r0; r < r1; ++r) {
+                const int w = s_rexp[r];
+                s_rexp[r] = base;
+                base += w;
+            }
+            if (tid == blockDim.x - 1) s_rexp[nrec] = base;   // the total (the last thread's running sum)
+            __syncthreads();
+            const long long wtot = s_rexp[nrec];
+            for (int j = 0; j < 2; ++j) {
+                if (!(j == 0 ? tab0 : tab1)) continue;
+                const int grid = a.vgrid[j], nrb = a.vnrb[j];
+                for (int b = tid; b <= grid; b += blockDim.x) {
+                    // first item i whose preceding work reaches b/grid of the total
+                    const long long tb = wtot * nrb * b / grid;
+                    int lo = 0, hi = nrec;   // largest g with prefix(g) * nrb <= tb
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (static_cast<long long>(s_rexp[mid]) * nrb <= tb) lo = mid;
+                        else hi = mid - 1;
+                    }
+                    long long start;
+                    if (lo >= nrec) {
+                        start = static_cast<long long>(nrec) * nrb;
+                    } else {
+                        const long long pg = static_cast<long long>(s_rexp[lo]) * nrb;
+                        const long long wg = s_rexp[lo + 1] - s_rexp[lo];
+                        long long rb = (tb - pg + wg - 1) / wg;
+                        if (rb > nrb) rb = nrb;
+                        start = static_cast<long long>(lo) * nrb + rb;
+                    }
+                    a.vstart[j][b] = static_cast<int32_t>(start);
+                }
+            }
+        }
+    }
+    if (tid == 0) {
+        a.hdr->n_active = static_cast<uint32_t>(rank_base);
+        a.hdr->n_gtiles = static_cast<uint32_t>(gt_base);
+        a.hdr->n_vgroups = static_cast<uint32_t>(vg_base);
+    }
 }
 
 __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
@@ -473,147 +647,7 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
             it += D;
         }
     } else {
-        int it_start = 0;
-        if (P <= kSpecMaxP && Ls.costs_in_smem) {
-            // ---- speculation for mid-size batches (the same idea as above, at block scale).
-            // Breakpoints of every pair's lower convex hull, at fixed slots p*(nk-1)+i (unused: -1).
-            const double* s_costs = reinterpret_cast<const double*>(smem + Ls.costs);
-            double* s_bpv = reinterpret_cast<double*>(smem + Ls.bp);
-            int* s_bjv = reinterpret_cast<int*>(smem + Ls.bj);
-            const int nslot = nk - 1;
-            for (int p = tid; p < P; p += blockDim.x) {
-                const double* c = s_costs + p * nk;
-                int cur = 0;
-                for (int i = 1; i < nk; ++i) if (c[i] < c[cur]) cur = i;
-                int slotb = 0;
-                while (cur > 0) {
-                    int jn = -1;
-                    double tn = 0.0;
-                    for (int j = 0; j < cur; ++j) {
-                        const double t = __dmul_rn(__dsub_rn(c[j], c[cur]), inv_gap(cur - j));
-                        if (jn < 0 || t < tn) { jn = j; tn = t; }
-                    }
-                    s_bpv[p * nslot + slotb] = tn;
-                    s_bjv[p * nslot + slotb] = cur - jn;
-                    ++slotb;
-                    cur = jn;
-                }
-                for (; slotb < nslot; ++slotb) {
-                    s_bpv[p * nslot + slotb] = -1.0;
-                    s_bjv[p * nslot + slotb] = 0;
-                }
-            }
-            // lam_c = the largest breakpoint v with W(>= v) > budget - P*kmin (W: summed jumps):
-            // weighted radix select, 8 bits per pass, on the (non-negative) fp64 bit patterns
-            __shared__ int s_hist[256];
-            __shared__ unsigned long long s_prefix;
-            __shared__ double s_rem;
-            __shared__ int s_found;
-            const int nall = P * nslot;
-            if (tid == 0) {
-                s_prefix = 0ull;
-                s_rem = __dsub_rn(budget, static_cast<double>(P * a.kmin));
-                s_found = 1;
-            }
-            for (int pass = 0; pass < 8; ++pass) {
-                const int shift = 56 - 8 * pass;
-                for (int b = tid; b < 256; b += blockDim.x) s_hist[b] = 0;
-                __syncthreads();
-                const unsigned long long pre = s_prefix;
-                const unsigned long long hmask = pass == 0 ? 0ull : (~0ull << (shift + 8));
-                if (s_found) {
-                    // the leading digits repeat across most keys: aggregate equal buckets per warp
-                    // before the shared-memory atomic
-                    for (int q0 = warp * 32; q0 < nall; q0 += blockDim.x) {
-                        const int q = q0 + lane;
-                        int bucket = -1, wgt = 0;
-                        if (q < nall) {
-                            const double v = s_bpv[q];
-                            if (v >= 0.0) {
-                                const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(v));
-                                if ((key & hmask) == pre) {
-                                    bucket = static_cast<int>((key >> shift) & 255u);
-                                    wgt = s_bjv[q];
-                                }
-                            }
-                        }
-                        const unsigned grp = __match_any_sync(0xffffffffu, bucket);
-                        const int tot = static_cast<int>(__reduce_add_sync(grp, static_cast<unsigned>(wgt)));
-                        if (bucket >= 0 && lane == __ffs(static_cast<int>(grp)) - 1) atomicAdd(&s_hist[bucket], tot);
-                    }
-                }
-                __syncthreads();
-                if (warp == 0 && s_found) {
-                    // lane l holds buckets 255-8l .. 248-8l; the first bucket from the top whose
-                    // cumulative weight exceeds the remainder is picked
-                    const double rem = s_rem;
-                    int part = 0;
-                    for (int u = 0; u < 8; ++u) part += s_hist[255 - 8 * lane - u];
-                    int incl = part;
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += t;
-                    }
-                    const int excl = incl - part;
-                    const bool crosses = static_cast<double>(incl) > rem && !(static_cast<double>(excl) > rem);
-                    const unsigned who = __ballot_sync(0xffffffffu, crosses);
-                    if (who == 0u) {
-                        if (lane == 0) s_found = 0;   // the jumps never exceed the budget: lam_c = 0
-                    } else if (lane == __ffs(static_cast<int>(who)) - 1) {
-                        int acc = excl, pick = -1;
-                        for (int u = 0; u < 8; ++u) {
-                            const int b = 255 - 8 * lane - u;
-                            const int h = s_hist[b];
-                            if (static_cast<double>(acc + h) > rem) { pick = b; break; }
-                            acc += h;
-                        }
-                        s_prefix = pre | (static_cast<unsigned long long>(pick) << shift);
-                        s_rem = __dsub_rn(rem, static_cast<double>(acc));
-                    }
-                }
-                __syncthreads();
-            }
-            if (tid == 0) {
-                const double lam_c = s_found ? __longlong_as_double(static_cast<long long>(s_prefix)) : 0.0;
-                double l = lo, h = hi;
-                for (int i = 0; i < 64; ++i) {   // replay with the real-arithmetic predicate
-                    s_lo[i] = l;
-                    s_hi[i] = h;
-                    const double m = midpoint(l, h);
-                    const int pr = m < lam_c ? 1 : 0;
-                    s_mid[i] = m;
-                    s_spred[i] = static_cast<unsigned char>(pr);
-                    if (pr) l = m; else h = m;
-                }
-                s_lo[64] = l;
-                s_hi[64] = h;
-            }
-            __syncthreads();
-            // exact check of the 64 recorded steps: warp w checks steps 2w and 2w+1 (32 warps)
-            for (int st0 = 2 * warp; st0 < 64; st0 += 2 * nw) {
-                const double m0 = s_mid[st0], m1 = s_mid[st0 + 1];
-                int n0 = 0, n1 = 0;
-                for (int p = lane; p < P; p += 32) {
-                    const double* c = s_costs + p * nk;
-                    n0 += choose_k(c, nk, a.kmin, kv, m0);
-                    n1 += choose_k(c, nk, a.kmin, kv, m1);
-                }
-                n0 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n0)));
-                n1 = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(n1)));
-                if (lane == 0) {
-                    s_pred[0][st0] = (n0 > nb ? 1 : 0) != s_spred[st0] ? 1 : 0;
-                    s_pred[0][st0 + 1] = (n1 > nb ? 1 : 0) != s_spred[st0 + 1] ? 1 : 0;
-                }
-            }
-            __syncthreads();
-            int it0 = 64;
-            for (int i = 0; i < 64; ++i)
-                if (s_pred[0][i]) { it0 = i; break; }
-            lo = s_lo[it0];
-            hi = s_hi[it0];
-            it_start = it0;
-            __syncthreads();   // s_pred is reused by the tree below
-        }
+        const int it_start = 0;   // (65 to 2048 pairs run on the cluster kernel; this is the general tree)
         // whole block: a group of gs threads per node, trees of depth D per round
         int gs_log = 0;
         while ((1 << gs_log) < 32 && (P >> (gs_log + 3)) > 0) ++gs_log;   // ~8 pairs per thread
@@ -664,179 +698,203 @@ __global__ void __launch_bounds__(kAllocThreads) allocate_kernel(AllocArgs a) {
     }
 grouping:
     if (!a.do_permute) return;
+    group_pairs(a, smem, Ls, P, nk, s_k, s_tmp, s_scan5);
 
-    // ---------------- grouping by (expert, k), all in shared memory ----------------
-    int* s_counts = reinterpret_cast<int*>(smem + Ls.counts);
-    int* s_seg = reinterpret_cast<int*>(smem + Ls.seg);
-    int* s_sorted = reinterpret_cast<int*>(smem + Ls.sorted);
-    const int nkeys = a.E * nk;
-    for (int i = tid; i < nkeys; i += blockDim.x) s_counts[i] = 0;
+}
+
+// ---------------- cluster bisection for mid-size batches ----------------
+// The same 64 exact steps as the single-CTA kernel, run by a cluster of kClCtas CTAs (one per
+// SM). CTA r keeps the costs of pairs [P r / n, P (r+1) / n) in shared memory. Each round
+// evaluates the 63 midpoints the next 6 steps can visit (a tree, as in allocate_kernel): every
+// CTA counts planes over its pairs per midpoint, the counts are exchanged through distributed
+// shared memory (each CTA reads every CTA's 63 counts), and every thread walks the tree with
+// the exact predicates, so all CTAs take the same steps. Rounds are separated by a cluster
+// barrier built from mbarriers (every CTA arrives remotely on every CTA's barrier; waits are
+// bounded). Afterwards CTA 0 reads back all plane counts and groups the pairs.
+#ifndef DPA_ALLOC_CLUSTER
+#define DPA_ALLOC_CLUSTER 8
+#endif
+constexpr int kClCtas = DPA_ALLOC_CLUSTER;   // 8 (portable) or 16 (non-portable cluster size)
+constexpr int kClThreads = 512;   // 64 node slots x 8 threads
+constexpr int kClDepth = 6;       // bisection steps per round (63 midpoints)
+constexpr int kClNodes = 1 << kClDepth;
+constexpr int kClMinPairs = 65;   // below: the single-CTA kernel's small-batch path
+
+struct ClShared {
+    uint64_t bar[2];                   // the cluster barrier, alternating by barrier index
+    int part[2][kClCtas][kClNodes];    // every CTA's plane counts per node (pushed here by their
+                                       // owners), by round parity
+    int flags[kClCtas];                // every CTA's invalid-input bits
+    double mx[kClCtas];                // every CTA's max cost at kmin
+};
+
+// barrier i of the cluster: every CTA's thread 0 arrives on every CTA's bar[i & 1] (release),
+// then waits on its own (acquire, bounded); the block barriers order the other threads
+__device__ __forceinline__ bool cluster_sync(ClShared& cs, int i, uint32_t n, WsHeader* hdr, uint32_t where) {
     __syncthreads();
-    for (int p = tid; p < P; p += blockDim.x) atomicAdd(&s_counts[a.idx[p] * nk + (s_k[p] - a.kmin)], 1);
-    __syncthreads();
-    {   // exclusive scan of the counts into s_seg; counts become placement cursors
-        const int per = (nkeys + blockDim.x - 1) / blockDim.x;
-        const int k0 = tid * per, k1 = min(nkeys, k0 + per);
-        int run = 0;
-        for (int i = k0; i < k1; ++i) run += s_counts[i];
-        int base = block_incl_scan(run, s_tmp) - run;
-        for (int i = k0; i < k1; ++i) {
-            const int c = s_counts[i];
-            s_seg[i] = base;
-            s_counts[i] = base;
-            base += c;
-        }
-        if (tid == 0) s_seg[nkeys] = P;
-    }
-    __syncthreads();
-    int* s_ptok = reinterpret_cast<int*>(smem + Ls.ptok);   // token of each grouped position
-    for (int p = tid; p < P; p += blockDim.x) {
-        const int key = a.idx[p] * nk + (s_k[p] - a.kmin);
-        const int pos = atomicAdd(&s_counts[key], 1);
-        const int tok = p / a.K;
-        s_sorted[pos] = p;
-        if (a.vrec) s_ptok[pos] = tok;
-        a.pair_pos[p] = pos;
-        if (a.pos_tok) a.pos_tok[pos] = tok;
-    }
-    __syncthreads();
-    // Per expert: the prefill GEMM's token tiles (one (expert, k) class each) and the start of its
-    // GEMV records (groups of up to vtpg tiles of up to 4 pairs of one class, classes ascending in
-    // k); experts in rounds of blockDim so that both lists stay in ascending expert order. Each
-    // record's owner expert goes to s_rexp; the records themselves are written below, one warp
-    // per record.
-    int rank_base = 0, gt_base = 0, vg_base = 0;
-    const int vtpg = a.vtiles_per_group > 0 ? a.vtiles_per_group : 1;
-    int* s_rexp = reinterpret_cast<int*>(smem + Ls.rexp);   // [records] owner expert
-    int* s_rfirst = reinterpret_cast<int*>(smem + Ls.rfirst);   // [E] first record of each expert
-    for (int e0 = 0; e0 < a.E; e0 += blockDim.x) {
-        const int e = e0 + tid;
-        int km = 0, ngt = 0, nvt = 0;
-        if (e < a.E) {
-            for (int i = 0; i < nk; ++i) {
-                const int n = s_seg[e * nk + i + 1] - s_seg[e * nk + i];
-                if (n > 0) km = a.kmin + i;
-                ngt += (n + kGemmTileTokens - 1) / kGemmTileTokens;
-                nvt += (n + 3) >> 2;
-            }
-        }
-        const int nvg = a.vrec ? (nvt + vtpg - 1) / vtpg : 0;
-        const int flag = km > 0 ? 1 : 0;
-        int sc[3] = {flag, a.gtiles ? ngt : 0, nvg};   // one block scan of the three counts
-        block_incl_scan_n<3>(sc, s_scan5);
-        if (a.gtiles && ngt > 0) {   // token tiles of the prefill GEMMs: one (expert, k) class each
-            int t = gt_base + sc[1] - ngt;
-            for (int i = 0; i < nk; ++i) {
-                const int s0 = s_seg[e * nk + i];
-                const int n = s_seg[e * nk + i + 1] - s0;
-                for (int j = 0; j < n; j += kGemmTileTokens)
-                    a.gtiles[t++] = make_int4(e, a.kmin + i, s0 + j, min(kGemmTileTokens, n - j));
-            }
-        }
-        if (a.vrec && e < a.E) {
-            const int r0 = vg_base + sc[2] - nvg;
-            s_rfirst[e] = r0;
-            for (int j = 0; j < nvg; ++j) s_rexp[r0 + j] = e;
-        }
-        // totals of this round: the scan's last warp totals, still in shared memory; every thread
-        // reads them before the barrier below, ahead of the next round's scan
-        rank_base += s_scan5[0][nw - 1];
-        gt_base += s_scan5[1][nw - 1];
-        vg_base += s_scan5[2][nw - 1];
-        __syncthreads();
-    }
-    if (a.vrec) {
-        // record r of expert e holds the expert's tiles [j vtpg, (j+1) vtpg), j = r - first(e);
-        // lane q computes field q (layout of kVRecInts) and the warp stores the record at once
-        for (int r = warp; r < vg_base; r += nw) {
-            const int e = s_rexp[r];
-            const int j = r - s_rfirst[e];
-            int tk[2] = {0, 0}, tn[2] = {0, 0}, tpos[2] = {0, 0}, nt = 0;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                int g = j * vtpg + t;   // the expert's tile index
-                if (t >= vtpg) break;
-                for (int i = 0; i < nk; ++i) {
-                    const int s0 = s_seg[e * nk + i];
-                    const int n = s_seg[e * nk + i + 1] - s0;
-                    const int ntc = (n + 3) >> 2;
-                    if (g < ntc) {
-                        tk[t] = a.kmin + i;
-                        tn[t] = min(4, n - 4 * g);
-                        tpos[t] = s0 + 4 * g;
-                        nt = t + 1;
-                        break;
-                    }
-                    g -= ntc;
-                }
-            }
-            int v = 0;
-            if (lane == 0) v = e;
-            else if (lane == 1) v = tk[nt - 1];            // tiles ascend in k: the last is the group's kmax
-            else if (lane == 2) v = nt;
-            else if (lane == 4 || lane == 5) v = tk[lane - 4];
-            else if (lane == 6 || lane == 7) v = tn[lane - 6];
-            else if (lane >= 8 && lane < 24) {
-                const int f = lane & 7, t = f >> 2, u = f & 3;
-                const bool used = t < nt && u < tn[t];
-                v = !used ? -1 : (lane < 16 ? tpos[t] + u : s_ptok[tpos[t] + u]);
-            }
-            a.vrec[static_cast<size_t>(r) * kVRecInts + lane] = v;
-            // the record's work weight per row block (planes read, token tiles), in the owner slot
-            __syncwarp();
-            if (lane == 0) s_rexp[r] = 5 + 2 * tk[nt - 1] + 3 * nt;
-        }
-        const bool tab0 = a.vstart[0] && vg_base * a.vnrb[0] > a.vgrid[0];
-        const bool tab1 = a.vstart[1] && vg_base * a.vnrb[1] > a.vgrid[1];
-        if (tab0 || tab1) {   // (with no more items than CTAs the GEMV splits items evenly)
-            __syncthreads();
-            // exclusive prefix of the weights over the records: s_rexp[0..vg_base]
-            const int nrec = vg_base;
-            const int per = (nrec + blockDim.x - 1) / blockDim.x;
-            const int r0 = tid * per, r1 = min(nrec, r0 + per);
-            int run = 0;
-            for (int r = r0; r < r1; ++r) run += s_rexp[r];
-            int base = block_incl_scan(run, s_tmp) - run;
-            for (int r = r0; r < r1; ++r) {
-                const int w = s_rexp[r];
-                s_rexp[r] = base;
-                base += w;
-            }
-            if (tid == blockDim.x - 1) s_rexp[nrec] = base;   // the total (the last thread's running sum)
-            __syncthreads();
-            const long long wtot = s_rexp[nrec];
-            for (int j = 0; j < 2; ++j) {
-                if (!(j == 0 ? tab0 : tab1)) continue;
-                const int grid = a.vgrid[j], nrb = a.vnrb[j];
-                for (int b = tid; b <= grid; b += blockDim.x) {
-                    // first item i whose preceding work reaches b/grid of the total
-                    const long long tb = wtot * nrb * b / grid;
-                    int lo = 0, hi = nrec;   // largest g with prefix(g) * nrb <= tb
-                    while (lo < hi) {
-                        const int mid = (lo + hi + 1) >> 1;
-                        if (static_cast<long long>(s_rexp[mid]) * nrb <= tb) lo = mid;
-                        else hi = mid - 1;
-                    }
-                    long long start;
-                    if (lo >= nrec) {
-                        start = static_cast<long long>(nrec) * nrb;
-                    } else {
-                        const long long pg = static_cast<long long>(s_rexp[lo]) * nrb;
-                        const long long wg = s_rexp[lo + 1] - s_rexp[lo];
-                        long long rb = (tb - pg + wg - 1) / wg;
-                        if (rb > nrb) rb = nrb;
-                        start = static_cast<long long>(lo) * nrb + rb;
-                    }
-                    a.vstart[j][b] = static_cast<int32_t>(start);
+    bool ok = true;
+    if (threadIdx.x < n)   // one thread per destination CTA, after the block barrier (cumulative release)
+        mbar_arrive_cluster(mapa_shared(smem_u32(&cs.bar[i & 1]), threadIdx.x));
+    if (threadIdx.x == 0) {
+        const uint32_t parity = (i >> 1) & 1;
+        if (!mbar_try_wait_acq_cluster(&cs.bar[i & 1], parity)) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait_acq_cluster(&cs.bar[i & 1], parity)) {
+                if (globaltimer() - t0 > kWaitNs) {
+                    set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
+                    ok = false;
+                    break;
                 }
             }
         }
     }
+    return __syncthreads_and(ok ? 1 : 0) != 0;
+}
+
+__global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ ClShared cs;
+    __shared__ int s_tmp[32];
+    __shared__ int s_scan5[5][32];
+    __shared__ int s_tot[kClNodes];
+    __shared__ double s_wmx[kClThreads / 32];
+    const int P = a.T * a.K;
+    const int nk = a.kmax - a.kmin + 1;
+    const KVals kv = make_kvals(a.kmin);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
+    const int p0 = static_cast<int>((static_cast<long long>(P) * rank) / ncta);
+    const int p1 = static_cast<int>((static_cast<long long>(P) * (rank + 1)) / ncta);
+    const int np = p1 - p0;
+    const AllocSmem Ls = alloc_smem_layout(P, a.E, nk, a.vrec != nullptr);
+    double* s_c = reinterpret_cast<double*>(smem + Ls.total);   // this CTA's costs [np][nk]
+    uint8_t* s_k = smem + Ls.kk;
+    __shared__ int s_myflags;
     if (tid == 0) {
-        a.hdr->n_active = static_cast<uint32_t>(rank_base);
-        a.hdr->n_gtiles = static_cast<uint32_t>(gt_base);
-        a.hdr->n_vgroups = static_cast<uint32_t>(vg_base);
+        mbar_init(&cs.bar[0], ncta);
+        mbar_init(&cs.bar[1], ncta);
+        s_myflags = 0;
+        fence_mbarrier_init_cluster();
     }
+    for (int i = tid * 16; i < a.E * a.B; i += blockDim.x * 16)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(a.rtable + i));
+    cluster_barrier_once();   // the barriers exist before anyone arrives on them
+    pdl_wait();
+    pdl_trigger();
+    // ---- inputs: budget, this CTA's pairs (expert ids, widths) and their costs
+    const double target = *a.target;
+    int flags = (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1;
+    double mx = 0.0;
+    for (int j = tid; j < np; j += blockDim.x) {
+        const int p = p0 + j;
+        const int e = a.idx[p];
+        if (e < 0 || e >= a.E) {
+            flags |= 2;
+            continue;
+        }
+        const int wmax = stored_width(a, e);
+        if (wmax < a.kmin || wmax > a.kmax) {
+            flags |= 4;
+            continue;
+        }
+        const double g = a.gate[p];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (i < nk) {
+                const double c = a.kmin + i > wmax ? CUDART_INF
+                                                   : __dmul_rn(g, a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)]);
+                s_c[j * nk + i] = c;
+                if (i == 0) mx = fmax(mx, c);
+            }
+        }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        flags |= __shfl_xor_sync(0xffffffffu, flags, o);
+    }
+    if (lane == 0) s_wmx[warp] = mx;
+    if (lane == 0 && flags) atomicOr(&s_myflags, flags);
+    __syncthreads();
+    // ---- exchange: this CTA's flags and max pushed into every CTA's slot `rank`
+    if (tid < static_cast<int>(ncta)) {
+        double m = s_wmx[0];
+        for (int w = 1; w < nw; ++w) m = fmax(m, s_wmx[w]);
+        st_cluster_s32(mapa_shared(smem_u32(&cs.flags[rank]), tid), s_myflags);
+        st_cluster_f64(mapa_shared(smem_u32(&cs.mx[rank]), tid), m);
+    }
+    if (!cluster_sync(cs, 0, ncta, a.hdr, 0x250)) return;
+    int all_flags = 0;
+    mx = 0.0;
+    for (uint32_t r = 0; r < ncta; ++r) {
+        all_flags |= cs.flags[r];
+        mx = fmax(mx, cs.mx[r]);
+    }
+    if (all_flags) {
+        if (rank == 0 && tid == 0) {
+            set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, (all_flags & 2) ? 11 : ((all_flags & 1) ? 10 : 15));
+            if (a.do_permute) {
+                a.hdr->n_active = 0;
+                a.hdr->n_gtiles = 0;
+                a.hdr->n_vgroups = 0;
+            }
+        }
+        cluster_sync(cs, 1, ncta, a.hdr, 0x251);   // nobody reads another CTA's shared memory after this
+        return;
+    }
+    const double budget = __dmul_rn(target, static_cast<double>(P));
+    const int nb = static_cast<int>(floor(budget));
+    double lo = 0.0;
+    double hi = __dadd_rn(__dmul_rn(2.0, mx), 1.0);
+    // ---- 64 steps, kClDepth per round
+    constexpr int TPN = kClThreads / kClNodes;   // threads per node
+    const int node_slot = tid / TPN, gsub = tid % TPN;
+    int round = 0;
+    for (int it = 0; it < 64; ++round) {
+        const int D = min(kClDepth, 64 - it);
+        const int node = node_slot + 1;
+        const bool active = node < (1 << D);
+        int n = 0;
+        if (active) {
+            const int depth = 31 - __clz(node);
+            double l = lo, h = hi;
+            for (int lev = depth - 1; lev >= 0; --lev) {
+                const double m = midpoint(l, h);
+                if ((node >> lev) & 1) l = m; else h = m;
+            }
+            const double mid = midpoint(l, h);
+            for (int j = gsub; j < np; j += TPN) n += choose_k(s_c + j * nk, nk, a.kmin, kv, mid);
+        }
+#pragma unroll
+        for (int o = 1; o < TPN; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        // push this node's count into every CTA's slot `rank` (the node's threads share the stores)
+        for (int r = gsub; r < static_cast<int>(ncta); r += TPN)
+            st_cluster_s32(mapa_shared(smem_u32(&cs.part[round & 1][rank][node_slot]), r), n);
+        if (!cluster_sync(cs, 1 + round, ncta, a.hdr, 0x252)) return;
+        if (tid < kClNodes) {   // the cluster's count at node tid + 1, from the local slots
+            int t = 0;
+            for (uint32_t r = 0; r < ncta; ++r) t += cs.part[round & 1][r][tid];
+            s_tot[tid] = t;
+        }
+        __syncthreads();
+        int nd = 1;
+        for (int lev = 0; lev < D; ++lev) {
+            const int pr = s_tot[nd - 1] > nb ? 1 : 0;
+            const double m = midpoint(lo, hi);
+            if (pr) lo = m; else hi = m;
+            nd = 2 * nd + pr;
+        }
+        it += D;
+    }
+    // ---- plane counts of this CTA's pairs
+    for (int j = tid; j < np; j += blockDim.x)
+        a.k_out[p0 + j] = static_cast<uint8_t>(choose_k(s_c + j * nk, nk, a.kmin, kv, hi));
+    if (rank == 0 && tid == 0 && a.lambda_out) *a.lambda_out = hi;
+    // every CTA's counts are written and no CTA reads another's shared memory any more
+    if (!cluster_sync(cs, 1 + round, ncta, a.hdr, 0x253)) return;
+    if (rank != 0 || !a.do_permute) return;
+    for (int p = tid; p < P; p += blockDim.x) s_k[p] = __ldcg(a.k_out + p);
+    __syncthreads();
+    group_pairs(a, smem, Ls, P, nk, s_k, s_tmp, s_scan5);
 }
 
 // ---------------- grid-wide bisection for large batches ----------------
@@ -1002,6 +1060,7 @@ cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* c
     const int nk = a.kmax - a.kmin + 1;
     const int P = a.T * a.K;
     AllocArgs b = a;
+    bool coop_ran = false;
     const int coop_blocks = sms > 0 ? (P / 64 < sms ? (P + 63) / 64 : sms) : 1;
     int per_block = (P + coop_blocks - 1) / coop_blocks;
     if (coop && a.policy == DPA_ALLOC_LAGRANGE && P > kCoopMinPairs && per_block <= kCoopMaxPairsPerBlock) {
@@ -1029,6 +1088,35 @@ cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* c
         err = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(allocate_coop_kernel), cargs);
         if (err != cudaSuccess) return err;
         b.k_given = 1;
+        coop_ran = true;
+    }
+    if (!coop_ran && a.policy == DPA_ALLOC_LAGRANGE && P >= kClMinPairs && P <= kSpecMaxP) {
+        // mid-size batches: the bisection over a cluster of SMs, then CTA 0 groups the pairs
+        const size_t smem = allocate_smem_bytes(P, a.E, nk, a.vrec != nullptr) +
+                            static_cast<size_t>(P / kClCtas + 1) * nk * 8;
+        cudaError_t err = cudaFuncSetAttribute(allocate_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        if (kClCtas > 8) {
+            err = cudaFuncSetAttribute(allocate_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (err != cudaSuccess) return err;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kClCtas);
+        cfg.blockDim = dim3(kClThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kClCtas;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        void* cargs[] = {&b};
+        return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(allocate_cluster_kernel), cargs);
     }
     const size_t smem = allocate_smem_bytes(P, a.E, nk, a.vrec != nullptr);
     if (smem > 48 * 1024) {

@@ -450,9 +450,9 @@ __global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
     // this CTA's contiguous range of items
     int it0 = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
     int it1 = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
-    if (a.vstart && a.vgrid == static_cast<int>(gridDim.x) && n_items > static_cast<int>(gridDim.x)) {
-        // ranges balanced by the groups' estimated work (written for batches with more items
-        // than CTAs)
+    if (a.vstart && a.vgrid == static_cast<int>(gridDim.x) && n_items > 2 * static_cast<int>(gridDim.x)) {
+        // ranges balanced by the groups' estimated work (written for batches with more than two
+        // items per CTA)
         it0 = min(__ldcg(a.vstart + blockIdx.x), n_items);
         it1 = min(__ldcg(a.vstart + blockIdx.x + 1), n_items);
     }
