@@ -706,15 +706,16 @@ grouping:
 // The same 64 exact steps as the single-CTA kernel, run by a cluster of kClCtas CTAs (one per
 // SM). CTA r keeps the costs of pairs [P r / n, P (r+1) / n) in shared memory. Each round
 // evaluates the 63 midpoints the next 6 steps can visit (a tree, as in allocate_kernel): every
-// CTA counts planes over its pairs per midpoint, the counts are exchanged through distributed
-// shared memory (each CTA reads every CTA's 63 counts), and every thread walks the tree with
-// the exact predicates, so all CTAs take the same steps. Rounds are separated by a cluster
-// barrier built from mbarriers (every CTA arrives remotely on every CTA's barrier; waits are
-// bounded). Afterwards CTA 0 reads back all plane counts and groups the pairs.
+// CTA counts planes over its pairs per midpoint and stores its counts into every CTA's shared
+// memory with st.async, which completes the bytes on that CTA's round barrier (armed with the
+// round's expected bytes; waits bounded); then every thread sums the slots and walks the tree
+// with the exact predicates, so all CTAs take the same steps. Two cluster barriers made of
+// remote mbarrier arrivals (at the start, and before CTA 0 reads back every pair's count)
+// order the rest. Afterwards CTA 0 groups the pairs.
 #ifndef DPA_ALLOC_CLUSTER
-#define DPA_ALLOC_CLUSTER 8
+#define DPA_ALLOC_CLUSTER 16
 #endif
-constexpr int kClCtas = DPA_ALLOC_CLUSTER;   // 8 (portable) or 16 (non-portable cluster size)
+constexpr int kClCtas = DPA_ALLOC_CLUSTER;   // CTAs of the cluster (16: a non-portable cluster size)
 constexpr int kClThreads = 512;   // 64 node slots x 8 threads
 constexpr int kClDepth = 6;       // bisection steps per round (63 midpoints)
 constexpr int kClNodes = 1 << kClDepth;
@@ -722,6 +723,7 @@ constexpr int kClMinPairs = 65;   // below: the single-CTA kernel's small-batch 
 
 struct ClShared {
     uint64_t bar[2];                   // the cluster barrier, alternating by barrier index
+    uint64_t rbar[2];                  // a round's counts have arrived (by round parity)
     int part[2][kClCtas][kClNodes];    // every CTA's plane counts per node (pushed here by their
                                        // owners), by round parity
     int flags[kClCtas];                // every CTA's invalid-input bits
@@ -773,6 +775,8 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
     if (tid == 0) {
         mbar_init(&cs.bar[0], ncta);
         mbar_init(&cs.bar[1], ncta);
+        mbar_init(&cs.rbar[0], 1);
+        mbar_init(&cs.rbar[1], 1);
         s_myflags = 0;
         fence_mbarrier_init_cluster();
     }
@@ -851,6 +855,9 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
     int round = 0;
     for (int it = 0; it < 64; ++round) {
         const int D = min(kClDepth, 64 - it);
+        // this round's counts from every CTA: ncta x kClNodes ints, stored into this CTA by
+        // st.async, each completing its bytes on rbar[round & 1]
+        if (tid == 0) mbar_arrive_expect_tx(&cs.rbar[round & 1], ncta * kClNodes * 4u);
         const int node = node_slot + 1;
         const bool active = node < (1 << D);
         int n = 0;
@@ -868,8 +875,25 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
         for (int o = 1; o < TPN; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
         // push this node's count into every CTA's slot `rank` (the node's threads share the stores)
         for (int r = gsub; r < static_cast<int>(ncta); r += TPN)
-            st_cluster_s32(mapa_shared(smem_u32(&cs.part[round & 1][rank][node_slot]), r), n);
-        if (!cluster_sync(cs, 1 + round, ncta, a.hdr, 0x252)) return;
+            st_async_s32(mapa_shared(smem_u32(&cs.part[round & 1][rank][node_slot]), r), n,
+                         mapa_shared(smem_u32(&cs.rbar[round & 1]), r));
+        {   // wait until every CTA's counts of this round are here (bounded)
+            bool ok = true;
+            if (tid == 0) {
+                const uint32_t parity = (round >> 1) & 1;
+                if (!mbar_try_wait_acq_cluster(&cs.rbar[round & 1], parity)) {
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try_wait_acq_cluster(&cs.rbar[round & 1], parity)) {
+                        if (globaltimer() - t0 > kWaitNs) {
+                            set_error(a.hdr, DPA_ERR_DEVICE_TIMEOUT, 0x252);
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+            }
+            if (!__syncthreads_and(ok ? 1 : 0)) return;
+        }
         if (tid < kClNodes) {   // the cluster's count at node tid + 1, from the local slots
             int t = 0;
             for (uint32_t r = 0; r < ncta; ++r) t += cs.part[round & 1][r][tid];
@@ -889,8 +913,8 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
     for (int j = tid; j < np; j += blockDim.x)
         a.k_out[p0 + j] = static_cast<uint8_t>(choose_k(s_c + j * nk, nk, a.kmin, kv, hi));
     if (rank == 0 && tid == 0 && a.lambda_out) *a.lambda_out = hi;
-    // every CTA's counts are written and no CTA reads another's shared memory any more
-    if (!cluster_sync(cs, 1 + round, ncta, a.hdr, 0x253)) return;
+    // every CTA's plane counts are written, and no CTA stores into another's shared memory any more
+    if (!cluster_sync(cs, 1, ncta, a.hdr, 0x253)) return;
     if (rank != 0 || !a.do_permute) return;
     for (int p = tid; p < P; p += blockDim.x) s_k[p] = __ldcg(a.k_out + p);
     __syncthreads();

@@ -207,6 +207,13 @@ __device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int v) {
 __device__ __forceinline__ void st_cluster_f64(uint32_t cluster_addr, double v) {
     asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(cluster_addr), "d"(v) : "memory");
 }
+// asynchronous remote store of 4 bytes into CTA shared memory of the cluster that completes 4
+// bytes of transaction count on that CTA's mbarrier (both shared::cluster addresses)
+__device__ __forceinline__ void st_async_s32(uint32_t cluster_addr, int v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "r"(v), "r"(cluster_bar)
+                 : "memory");
+}
 // arrive (release at cluster scope) on an mbarrier of any CTA of the cluster
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
