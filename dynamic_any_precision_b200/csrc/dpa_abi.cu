@@ -74,7 +74,7 @@ WsLayout ws_layout(const dpa_layer_desc* d, int T) {
     L.gtiles = take(16 * (P / dpa::kGemmTileTokens + E * nk + 1));
     L.postok = take(4 * P);
     L.coop = take(sizeof(dpa::CoopSync));
-    L.rstats = take((8 + 2 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 16);
+    L.rstats = take((8 + 4 * (H / 64 + 1)) * (static_cast<size_t>(T) + E) + 32);
     L.rpart = take(8 * dpa::route_partial_doubles(T, static_cast<int>(E), static_cast<int>(H)));
     L.vstart = take(4 * 2 * (kVpMaxGrid + 1));
     L.xperm = take(2 * P * H);
@@ -197,8 +197,11 @@ static void set_route_stats(dpa::RouteArgs& r, void* ws, const WsLayout& L, int 
     r.n2_x = reinterpret_cast<double*>(base);
     r.n2_w = r.n2_x + T;
     const size_t lsb_off = (8 * (static_cast<size_t>(T) + E) + 15) & ~static_cast<size_t>(15);
-    r.lsb_x = reinterpret_cast<int16_t*>(base + lsb_off);   // 16-byte aligned rows of H/64 entries
-    r.lsb_w = r.lsb_x + static_cast<size_t>(T) * (r.H / 64);
+    const size_t nrow = static_cast<size_t>(r.H / 64);   // H % 512 == 0 on the tiled path: 16-byte rows
+    r.lsb_x = reinterpret_cast<int16_t*>(base + lsb_off);
+    r.lsb_w = r.lsb_x + static_cast<size_t>(T) * nrow;
+    r.hb_x = r.lsb_w + static_cast<size_t>(E) * nrow;
+    r.hb_w = r.hb_x + static_cast<size_t>(T) * nrow;
     r.part = at<double>(ws, L.rpart);
 }
 

@@ -20,11 +20,13 @@
 // four pairs of one expert, each tile of one plane count k, tiles ascending in k. Items are
 // (token group, block of RB = 16 NRT rows); every CTA (one per SM, persistent) takes a contiguous
 // range of items, so consecutive items mostly share their group. Roles:
-//   - warp 8 (producer): per group, bulk copies (no multicast) of the tokens' digit rows, group
+//   - warp CW (producer; CW = 12 consumer warps for uniform codes, 8 for binary-coded planes):
+//     per group, bulk copies (no multicast) of the tokens' digit rows, group
 //     exponents and sums into one of two group slots; per item and chunk of up to 2048 columns,
 //     bulk copies of the chunk's plane words (one copy per matrix, plane p < kmax and row tile:
 //     2 bytes per column) and, with the first chunk, the item's scale data into a ring stage;
-//   - warps 0-7 (consumers): row tile rt and column slice cs of every chunk; wait for the stage,
+//   - warps 0..CW-1 (consumers): row tile rt and column slice cs of every chunk (CW / NRT
+//     slices per row tile); wait for the stage,
 //     compute, release it; after the item's last chunk the slices of a row tile are summed in a
 //     fixed order by one of them (rotating with the item) and the epilogue (SwiGLU for gate/up,
 //     the per-pair output for down) is written.
@@ -39,8 +41,17 @@
 namespace dpa {
 namespace {
 
-constexpr int kCW = 8;                        // consumer warps
-constexpr int kVThreads = (kCW + 1) * 32;     // + the producer warp
+// Consumer warps per CTA, by weight format. Uniform codes run 12: with the producer that is 13
+// warps, so at most 4 share a scheduler and each thread keeps up to 128 registers, and the
+// extra warps hide more of the decode's dependent latency (8 warps: 2 per scheduler). The
+// binary-coded variants keep 8: their two-tile kernels need more than 128 registers.
+#ifndef DPA_VP_CW_UNIFORM
+#define DPA_VP_CW_UNIFORM 12
+#endif
+#ifndef DPA_VP_CW_BCQ
+#define DPA_VP_CW_BCQ 8
+#endif
+__host__ __device__ constexpr int vp_cw(int fmt) { return fmt == DPA_FMT_UNIFORM ? DPA_VP_CW_UNIFORM : DPA_VP_CW_BCQ; }
 constexpr int kMaxStages = 8;                 // ring depth: as many stages as shared memory holds
 constexpr int kMaxB = 4;
 #ifndef DPA_VP_CHUNK
@@ -59,9 +70,10 @@ constexpr int kGuNRT = DPA_VP_GU_NRT, kGuNRTSmall = 1;   // gate/up: 32 (16) row
 constexpr int kDnNRT = DPA_VP_DN_NRT, kDnNRTSmall = 2;   // down: 64 (32) rows, 2 (4) column slices
 constexpr int kDigPad = 64;                   // bytes of padding per staged digit row (banks)
 
-template <int NRT>
+template <int CW, int NRT>
 struct Geo {
-    static constexpr int CS = kCW / NRT;      // column slices per chunk
+    static_assert(CW % NRT == 0, "the consumer warps split into row tiles x column slices");
+    static constexpr int CS = CW / NRT;       // column slices per chunk
     static constexpr int RB = 16 * NRT;       // rows per item
 };
 
@@ -81,12 +93,13 @@ struct VLayout {                              // byte offsets in dynamic shared 
 
 template <int NRT, int NTILE, int NMAT>
 __host__ __device__ inline VLayout vlayout(int K, int G, int fmt, int B) {
-    using Gm = Geo<NRT>;
+    constexpr int RB = 16 * NRT;
+    const int CS = vp_cw(fmt) / NRT;
     VLayout L;
     const size_t ng = K / G;
     L.ngp = static_cast<int>((ng + 3) & ~static_cast<size_t>(3));
-    const size_t meta = fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(NMAT) * Gm::RB * ng * 4
-                                               : static_cast<size_t>(NMAT) * B * Gm::RB * ng * 2;
+    const size_t meta = fmt == DPA_FMT_UNIFORM ? static_cast<size_t>(NMAT) * RB * ng * 4
+                                               : static_cast<size_t>(NMAT) * B * RB * ng * 2;
     const size_t dig_stride = static_cast<size_t>(K) + kDigPad;
     const size_t digs = static_cast<size_t>(4 * NTILE) * 2 * dig_stride;
     const size_t sl_exp = al16(digs);
@@ -94,7 +107,7 @@ __host__ __device__ inline VLayout vlayout(int K, int G, int fmt, int B) {
     const size_t sl_rec = sl_sum + static_cast<size_t>(4 * NTILE) * L.ngp * 4;
     const size_t slot = al128(sl_rec + kVRecInts * 4);
     const size_t red_per = static_cast<size_t>(32) * NTILE * NMAT * 2 * 4;
-    const size_t red = static_cast<size_t>(NRT) * Gm::CS * red_per;   // one partial per warp
+    const size_t red = static_cast<size_t>(NRT) * CS * red_per;   // one partial per warp
     const size_t fixed = 2 * slot + red;
     // columns per chunk: every column (one copy per matrix and plane takes all the item's row
     // tiles) where two stages fit beside the fixed parts, else halved down to 512
@@ -207,7 +220,6 @@ template <int B, int KM, int NT, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L, const unsigned char* st,
                                               const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0,
                                               int b1, int rt, float (&acc)[NTILE][NMAT][2]) {
-    using Gm = Geo<NRT>;
     const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
     const int ng = a.K / a.G, bpg = a.G / 64, nbc = L.CK / 64;
     const int pstride = NRT * nbc * 32;                                   // words per (matrix, plane) slab
@@ -261,7 +273,7 @@ __device__ __forceinline__ void slice_uniform(const VpArgs& a, const VLayout& L,
         for (int m = 0; m < NMAT; ++m)
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
-                const uint32_t sz = mrow[(m * Gm::RB + 8 * rr) * ng + g];
+                const uint32_t sz = mrow[(m * 16 * NRT + 8 * rr) * ng + g];
                 s[m][rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(sz & 0xFFFFu)));
                 z[m][rr] = __half2float(__ushort_as_half(static_cast<unsigned short>(sz >> 16)));
             }
@@ -292,7 +304,6 @@ template <int B, int KM, int NT, int NRT, int NTILE, int NMAT>
 __device__ __forceinline__ void slice_bcq(const VpArgs& a, const VLayout& L, const unsigned char* st,
                                           const unsigned char* gs, const Group<NTILE>& gr, int col0, int b0, int b1,
                                           int rt, float (&acc)[NTILE][NMAT][2]) {
-    using Gm = Geo<NRT>;
     const int lane = threadIdx.x & 31, gid = lane >> 2, tq = lane & 3;
     const int ng = a.K / a.G, bpg = a.G / 64, nbc = L.CK / 64;
     const int pstride = NRT * nbc * 32;
@@ -345,7 +356,7 @@ __device__ __forceinline__ void slice_bcq(const VpArgs& a, const VLayout& L, con
             for (int m = 0; m < NMAT; ++m)
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr)
-                    al[m][rr] = __half2float(meta[((m * KM + p) * Gm::RB + rt * 16 + gid + 8 * rr) * ng + g]);
+                    al[m][rr] = __half2float(meta[((m * KM + p) * 16 * NRT + rt * 16 + gid + 8 * rr) * ng + g]);
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 if (gr.tk[t] > p) {
@@ -411,8 +422,9 @@ __device__ __forceinline__ void slice_dispatch(const VpArgs& a, const VLayout& L
 // the kernel
 // ---------------------------------------------------------------------------------------
 template <int FMT, int NRT, int NTILE, int NMAT>
-__global__ void __launch_bounds__(kVThreads, 1) vp_gemv_kernel(VpArgs a) {
-    using Gm = Geo<NRT>;
+__global__ void __launch_bounds__((vp_cw(FMT) + 1) * 32, 1) vp_gemv_kernel(VpArgs a) {
+    constexpr int kCW = vp_cw(FMT);   // consumer warps; warp kCW is the producer
+    using Gm = Geo<kCW, NRT>;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ uint64_t s_full[kMaxStages], s_empty[kMaxStages], s_gfull[2], s_gempty[2];
     // the reduction's "partials written" barrier alternates with the item's parity: warps run up
@@ -750,11 +762,11 @@ cudaError_t launch_variant(const VpArgs& a, cudaStream_t stream, int sms) {
     const void* fn = reinterpret_cast<const void*>(vp_gemv_kernel<FMT, NRT, NTILE, NMAT>);
     cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
     if (err != cudaSuccess) return err;
-    const int items = a.max_groups * (a.R / Geo<NRT>::RB);
+    const int items = a.max_groups * (a.R / (16 * NRT));
     const int grid = items < sms ? (items > 0 ? items : 1) : sms;
     VpArgs copy = a;
     void* args[] = {&copy};
-    return launch_pdl_raw(fn, dim3(grid), dim3(kVThreads), L.total, stream, args);
+    return launch_pdl_raw(fn, dim3(grid), dim3((vp_cw(FMT) + 1) * 32), L.total, stream, args);
 }
 
 }  // namespace

@@ -23,8 +23,10 @@ struct RouteArgs {
     int wpe;                  // warps per expert (set by the launcher)
     // large-batch path (nullptr: always the per-logit kernel): per-row exactness statistics
     int16_t* lsb_x;           // [T][H/64] lowest set bit over each 64-input block's nonzero elements
+    int16_t* hb_x;            // [T][H/64] h with |x_b| < 2^h (Euclidean norm of the block)
     double* n2_x;             // [T] sum of squares
     int16_t* lsb_w;           // [E][H/64]
+    int16_t* hb_w;            // [E][H/64]
     double* n2_w;             // [E]
     double* part;             // [ks][T][E] slice sums of the tiled logits
     int ks;                   // input slices (set by the launcher)

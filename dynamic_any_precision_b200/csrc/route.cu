@@ -79,6 +79,15 @@ __device__ __forceinline__ int bf16_lsb(uint32_t u) {
     return p.exp + (__ffs(p.mant) - 1);
 }
 
+// exponent of the lowest set bit of a finite double (a large value for zero)
+__device__ __forceinline__ int f64_lsb(double v) {
+    const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(v));
+    const int ef = static_cast<int>((b >> 52) & 0x7FF);
+    unsigned long long m = b & 0xFFFFFFFFFFFFFull;
+    if (ef) m |= 1ull << 52;
+    return m ? (ef ? ef : 1) - 1075 + (__ffsll(static_cast<long long>(m)) - 1) : (1 << 20);
+}
+
 // 2^k as a double, k in [-1022, 1023]
 __device__ __forceinline__ double pow2(int k) {
     return __longlong_as_double(static_cast<long long>(k + 1023) << 52);
@@ -507,32 +516,45 @@ __global__ void __launch_bounds__(kRouteWarps * 32) route_kernel(RouteArgs a) {
 // ---------------- large batches: logits as a tiled fp64 GEMM ----------------
 // Exactness without per-product bookkeeping. Split the H inputs into blocks b of 64. Every
 // product x_j * w_j of block b is a multiple of 2^(Lx_b + Lw_b) (lowest set bit over the block's
-// nonzero elements of the token / the router row), so every product is a multiple of 2^L with
-// L = min_b (Lx_b + Lw_b); by Cauchy-Schwarz, sum_j |x_j w_j| <= |x| |w|. If
-// |x|^2 |w|^2 < 2^(2 (L + 53)), every partial sum in any order is a multiple of 2^L below
-// 2^(L+53): exact in fp64. Then the logit may be accumulated in any blocking and summed across
-// CTAs with fp64 atomics. Logits whose bound fails are recomputed with the fixed-point dot
-// product by the selection kernel, so the result is always the exact dot product rounded once,
-// as in the per-logit kernel.
+// nonzero elements of the token / the router row). Two tests, either of which proves that the
+// logit the selection kernel sums is the exact dot product:
+//  - whole row: every product is a multiple of 2^L with L = min_b (Lx_b + Lw_b), and by
+//    Cauchy-Schwarz every partial sum, in any order, is at most |x| |w|. If
+//    |x|^2 |w|^2 < 2^(2 (L + 53)), every partial sum is a multiple of 2^L below 2^(L+53): exact.
+//  - per slice, then across slices: a slice of the tiled GEMM touches blocks b0..b1; its
+//    products are multiples of 2^Ls, Ls = min (Lx_b + Lw_b) over those blocks, and each of its
+//    partial sums is at most sum_b |x_b| |w_b| < (b1 - b0 + 1) 2^Hs with |x_b| < 2^hx_b,
+//    |w_b| < 2^hw_b, Hs = max (hx_b + hw_b). If that bound is at most 2^(Ls+53), the slice sum
+//    is exact. The exact slice sums v_s are then multiples of 2^m (m: the lowest set bit over
+//    the nonzero v_s, read from their bits) and their partial sums are at most sum_s |v_s|; if
+//    that is below 2^(m+53), the sum over the slices is exact too. This test only fails where
+//    one slice really spans more than 53 bits, where the whole-row test fails for any token
+//    with one tiny element.
+// Logits for which both tests fail are recomputed by the selection kernel with the per-product
+// proof and, failing that, the fixed-point dot product, so the result is always the exact dot
+// product rounded once, as in the per-logit kernel.
 
 constexpr int kNoLsb = 0x3FFF;      // block (or row) without a nonzero element
 constexpr int kLsbBlock = 64;       // inputs per lowest-bit block
 
-// One CTA per row (tokens 0..T-1, then router rows): per-block lowest set bit, sum of squares,
-// NaN/Inf flag. Any block of up to 8 warps.
+// One CTA per row (tokens 0..T-1, then router rows): per-block lowest set bit and norm
+// exponent, sum of squares, NaN/Inf flag. Any block of up to 8 warps.
 __device__ void route_stats_row(const RouteArgs& a, int r) {
     __shared__ double s_n[8];
     __shared__ int s_b[8];
     const int H = a.H, nb = H / kLsbBlock;
     const bool is_tok = r < a.T;
+    const size_t ro = static_cast<size_t>(is_tok ? r : r - a.T) * nb;
     const uint16_t* row = is_tok ? a.x + static_cast<size_t>(r) * H : a.wr + static_cast<size_t>(r - a.T) * H;
-    int16_t* lrow = is_tok ? a.lsb_x + static_cast<size_t>(r) * nb : a.lsb_w + static_cast<size_t>(r - a.T) * nb;
+    int16_t* lrow = (is_tok ? a.lsb_x : a.lsb_w) + ro;
+    int16_t* hrow = (is_tok ? a.hb_x : a.hb_w) + ro;
     int bad = 0;
     double n2 = 0.0;
     // thread c covers elements 8c .. 8c+7; 8 consecutive lanes make one block of 64
     for (int c0 = 0; c0 < H / 8; c0 += blockDim.x) {
         const int c = c0 + threadIdx.x;
         int l = kNoLsb;
+        double q = 0.0;   // this thread's part of the block's sum of squares
         if (c < H / 8) {
             const uint4 v = reinterpret_cast<const uint4*>(row)[c];
             const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
@@ -542,11 +564,27 @@ __device__ void route_stats_row(const RouteArgs& a, int r) {
                 if (u & 0x7FFF) l = min(l, bf16_lsb(u));
                 bad |= ((u >> 7) & 0xFF) == 0xFF;
                 const double d = static_cast<double>(__uint_as_float(u << 16));
-                n2 = __dadd_rn(n2, __dmul_rn(d, d));
+                q = __dadd_rn(q, __dmul_rn(d, d));
             }
         }
-        for (int o = 1; o < 8; o <<= 1) l = min(l, __shfl_xor_sync(0xffffffffu, l, o));
-        if (c < H / 8 && (c & 7) == 0) lrow[c >> 3] = static_cast<int16_t>(l);
+        n2 = __dadd_rn(n2, q);
+        for (int o = 1; o < 8; o <<= 1) {
+            l = min(l, __shfl_xor_sync(0xffffffffu, l, o));
+            q = __dadd_rn(q, __shfl_xor_sync(0xffffffffu, q, o));
+        }
+        if (c < H / 8 && (c & 7) == 0) {
+            // squares of bf16 values are exact; 63 roundings of the sum stay below 2^-46
+            // relative, so q (1 + 2^-40) bounds the block's sum of squares from above; with
+            // q (1 + 2^-40) < 2^ex, the block's norm is below 2^ceil(ex / 2)
+            int hb = -kNoLsb;
+            if (q > 0.0) {
+                int ex;
+                frexp(__dmul_rn(q, 1.0 + 0x1p-40), &ex);
+                hb = (ex + 1) >> 1;
+            }
+            lrow[c >> 3] = static_cast<int16_t>(l);
+            hrow[c >> 3] = static_cast<int16_t>(hb);
+        }
     }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     n2 = warp_sum_f64(n2);
@@ -705,30 +743,41 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int s_fail[256];
     __shared__ int s_nfail;
-    __shared__ int16_t s_lx[kMaxLsbBlocks];
+    __shared__ int16_t s_lx[kMaxLsbBlocks], s_hx[kMaxLsbBlocks];
     pdl_wait();
     const int t = blockIdx.x, E = a.E, H = a.H, nb = H / kLsbBlock;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     double* dst = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
     if (threadIdx.x == 0) s_nfail = 0;
-    for (int b = threadIdx.x; b < nb; b += blockDim.x) s_lx[b] = a.lsb_x[static_cast<size_t>(t) * nb + b];
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+        s_lx[b] = a.lsb_x[static_cast<size_t>(t) * nb + b];
+        s_hx[b] = a.hb_x[static_cast<size_t>(t) * nb + b];
+    }
     __syncthreads();
     const double nx = a.n2_x[t];
+    const int kslice = H / a.ks;   // inputs per slice of the tiled logits
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        // the logit: the tiled kernel's slice sums (exact, in any order, when the bound holds);
-        // eight independent loads in flight per step
+        // the logit: the tiled kernel's slice sums, added in slice order (eight independent loads
+        // in flight per step), with their lowest set bit and the sum of their magnitudes
         const double* pe = a.part + static_cast<size_t>(t) * E + e;
         const size_t qs = static_cast<size_t>(a.T) * E;
-        double v = 0.0;
+        double v = 0.0, av = 0.0;
+        int mv = 1 << 20;
         for (int q0 = 0; q0 < a.ks; q0 += 8) {
             double u[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) u[j] = q0 + j < a.ks ? __ldcg(pe + (q0 + j) * qs) : 0.0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) v = __dadd_rn(v, u[j]);
+            for (int j = 0; j < 8; ++j) {
+                v = __dadd_rn(v, u[j]);
+                av = __dadd_rn(av, fabs(u[j]));
+                mv = min(mv, f64_lsb(u[j]));
+            }
         }
         dst[e] = v;
         const int16_t* lw = a.lsb_w + static_cast<size_t>(e) * nb;
+        const int16_t* hw = a.hb_w + static_cast<size_t>(e) * nb;
+        // whole-row test: L over all blocks with nonzero products
         int L = 2 * kNoLsb;
 #pragma unroll 4
         for (int b0 = 0; b0 < nb; b0 += 8) {   // nb is a multiple of 8 (H % 512 == 0 on this path)
@@ -746,6 +795,32 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
             // margin 2^-20 covers the rounding of the two fp64 sums of squares
             const double lhs = __dmul_rn(__dmul_rn(nx, a.n2_w[e]), 1.0 + 0x1p-20);
             ok = L2 >= 1024 || (L2 > -1022 && lhs < pow2(L2));
+        }
+        if (!ok) {
+            // per-slice test, then the sum over the slices
+            bool oks = true;
+            for (int sl = 0; sl < a.ks && oks; ++sl) {
+                const int b0 = (sl * kslice) / kLsbBlock, b1 = ((sl + 1) * kslice - 1) / kLsbBlock;
+                int Ls = kNoLsb, Hs = -kNoLsb;
+                for (int b = b0; b <= b1; ++b) {
+                    const int lx = s_lx[b], lwb = lw[b];
+                    if (lx < kNoLsb && lwb < kNoLsb) {   // both blocks hold nonzero elements
+                        Ls = min(Ls, lx + lwb);
+                        Hs = max(Hs, static_cast<int>(s_hx[b]) + static_cast<int>(hw[b]));
+                    }
+                }
+                const int nbt = b1 - b0 + 1;
+                const int cl = nbt > 1 ? 32 - __clz(nbt - 1) : 0;   // ceil(log2 nbt)
+                oks = Ls >= kNoLsb || Hs + cl <= Ls + 53;
+            }
+            if (oks && av > 0.0) {
+                // partial sums of the slice sums: multiples of 2^mv, at most av (summed with at
+                // most 255 roundings; 2^-40 bounds them)
+                int ea;
+                frexp(__dmul_rn(av, 1.0 + 0x1p-40), &ea);
+                oks = ea <= mv + 53;
+            }
+            ok = oks;
         }
         if (!ok) {
             const int slot = atomicAdd(&s_nfail, 1);

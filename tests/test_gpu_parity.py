@@ -103,7 +103,7 @@ def check_forward(shape, x_bits, target, sample_pairs=None, token_subset=None, p
 
 @pytest.mark.parametrize("shape,T", [(W.TINY, 4), (W.QWEN3_B1, 1), (W.QWEN3_B64, 64), (W.DEEPSEEK_B16, 16),
                                      (W.QWEN3_B1, 37), (W.TINY, 3),
-                                     # from 128 tokens on: tiled fp64 GEMM (ragged token tiles)
+                                     # from 2 tokens on: tiled fp64 GEMM (ragged token tiles)
                                      (W.TINY, 200), (W.DEEPSEEK_B16, 130), (W.QWEN3_B64, 300)])
 def test_route_bit_exact(shape, T):
     d = dpa.make_desc(shape)
@@ -136,6 +136,35 @@ def test_route_exact_path_for_wide_exponent_spread(T):
     w = (rng.standard_normal((E, H)) * 0.02).astype(np.float32)
     w[:, 1] = w[:, 0]
     w[:, 10:20] *= np.float32(2.0 ** -60)
+    xb, wb = W.f32_to_bf16_bits(x), W.f32_to_bf16_bits(w)
+    ws = dpa.new_workspace(d, T)
+    logits = torch.empty((T, E), dtype=torch.float64, device="cuda")
+    idx, gate = dpa.route(d, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(wb.view(np.int16)).cuda(),
+                          ws, logits=logits)
+    assert dpa.device_status(ws) == 0
+    ridx, rg, rl = O.route(xb, wb, shape.top_k, shape.norm_topk)
+    assert np.array_equal(logits.cpu().numpy(), rl)
+    assert np.array_equal(idx.cpu().numpy(), ridx) and np.array_equal(gate.cpu().numpy(), rg)
+
+
+@pytest.mark.parametrize("case", ["tiny_elements", "block_scales"])
+def test_route_tiled_slice_bounds(case):
+    # The tiled router proves a logit exact by a whole-row bound or, failing that, by per-slice
+    # bounds and a bound on the sum of the slice sums. tiny_elements: one element of 2^-30 per
+    # token, so that the whole-row bound fails for ~1/6 of the logits, the per-slice bounds rescue
+    # more than half of those and the rest is recomputed; block_scales: blocks of 64 inputs at
+    # 2^-40, 1 and 2^40, so every slice is exact on its own and their sum never is.
+    shape = W.with_sizes(W.TINY, name="tiny_slices")
+    d = dpa.make_desc(shape)
+    T, H, E = 64, shape.hidden, shape.n_experts
+    rng = np.random.default_rng(17)
+    x = rng.standard_normal((T, H)).astype(np.float32)
+    w = (rng.standard_normal((E, H)) * 0.02).astype(np.float32)
+    if case == "tiny_elements":
+        x[np.arange(T), rng.integers(0, H, T)] = np.float32(2.0 ** -30)
+    else:
+        for b in range(H // 64):
+            x[:, 64 * b:64 * (b + 1)] *= np.float32(2.0 ** (40 * (b % 3 - 1)))
     xb, wb = W.f32_to_bf16_bits(x), W.f32_to_bf16_bits(w)
     ws = dpa.new_workspace(d, T)
     logits = torch.empty((T, E), dtype=torch.float64, device="cuda")
