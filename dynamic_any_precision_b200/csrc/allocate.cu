@@ -191,7 +191,7 @@ __host__ __device__ inline AllocSmem alloc_smem_layout(int P, int E, int nk, boo
 // the GEMV launches' work-balanced CTA ranges. Whole block.
 __device__ void group_pairs(const AllocArgs& a, unsigned char* smem, const AllocSmem& Ls, int P, int nk,
                             const uint8_t* s_k, int* s_tmp, int (*s_scan5)[32]) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int tid = threadIdx.x, nw = blockDim.x >> 5;
 
     // ---------------- grouping by (expert, k), all in shared memory ----------------
     int* s_counts = reinterpret_cast<int*>(smem + Ls.counts);
@@ -703,94 +703,87 @@ grouping:
 }
 
 // ---------------- cluster bisection for mid-size batches ----------------
-// The same 64 exact steps as the single-CTA kernel, run by a cluster of kClCtas CTAs (one per
-// SM). CTA r keeps the costs of pairs [P r / n, P (r+1) / n) in shared memory. Each round
-// evaluates the 63 midpoints the next 6 steps can visit (a tree, as in allocate_kernel): every
-// CTA counts planes over its pairs per midpoint and stores its counts into every CTA's shared
-// memory with st.async, which completes the bytes on that CTA's round barrier (armed with the
-// round's expected bytes; waits bounded); then every thread sums the slots and walks the tree
-// with the exact predicates, so all CTAs take the same steps. Two cluster barriers made of
-// remote mbarrier arrivals (at the start, and before CTA 0 reads back every pair's count)
-// order the rest. Afterwards CTA 0 groups the pairs.
+// The same 64 exact steps, run by a cluster of kClCtas CTAs (one per SM), every CTA holding all
+// P pairs' costs in shared memory. A round takes D steps: the 2^D - 1 midpoints those steps can
+// visit form a tree (heap order). Node n belongs to CTA (n - 1) mod kClCtas; each of a CTA's
+// nodes is one warp, which computes the node's midpoint, counts planes over the listed pairs,
+// and stores the node's predicate into every CTA's shared memory with st.async, completing on
+// that CTA's round barrier (armed with the bytes it expects; waits bounded). Then every thread
+// walks the D steps with the predicates, recomputing the path's midpoints. One block barrier
+// per round.
+// Pruning, once, at the start of round kClPruneRound. A pair's cost of a count,
+// v_k(lam) = fl(c_k + fl(lam k)), never decreases as lam grows (both roundings are monotone).
+// So if, a being the pair's choice at hi, v_a(hi) < v_b(lo) for every count b below a and
+// v_a(hi) <= v_b(lo) for every count above a (the first minimum wins ties), the pair chooses a
+// everywhere in [lo, hi] and so at every later midpoint (they all lie in [lo, hi]): its count
+// joins a fixed sum and it leaves the list the nodes evaluate. After the first rounds only pairs
+// with a breakpoint near the final lambda stay listed.
 #ifndef DPA_ALLOC_CLUSTER
 #define DPA_ALLOC_CLUSTER 16
 #endif
-constexpr int kClCtas = DPA_ALLOC_CLUSTER;   // CTAs of the cluster (16: a non-portable cluster size)
-constexpr int kClThreads = 512;   // 64 node slots x 8 threads
-constexpr int kClDepth = 6;       // bisection steps per round (63 midpoints)
+constexpr int kClCtas = DPA_ALLOC_CLUSTER;      // CTAs of the cluster (16: a non-portable cluster size)
+constexpr int kClThreads = 512;
+constexpr int kClWarps = kClThreads / 32;
+constexpr int kClDepthEarly = 6;                // steps of the rounds before the pruning (every pair listed)
+constexpr int kClDepth = 8;                     // steps of the later rounds
+constexpr int kClPruneRound = 2;
 constexpr int kClNodes = 1 << kClDepth;
-constexpr int kClMinPairs = 65;   // below: the single-CTA kernel's small-batch path
+constexpr int kClNodesPerCta = (kClNodes - 1 + kClCtas - 1) / kClCtas;
+constexpr int kClMinPairs = 65;                 // below: the single-CTA kernel's small-batch path
+static_assert((kClCtas & (kClCtas - 1)) == 0, "cluster size a power of two");
+static_assert(kClNodesPerCta <= kClWarps, "at least one warp per node");
+static_assert(kClCtas <= 32, "one lane per destination CTA");
 
+// Predicates are kept for three rounds: a warp that owns no node may still be walking round r
+// when the other CTAs send round r + 2 (their round r + 1 needs only this CTA's node warps), but
+// round r + 3 needs this CTA past its round r + 1 barrier, which every warp reaches after its
+// round r walk. The barriers alternate by parity: a round's stores into a barrier can start only
+// after this CTA has waited on the round two before.
 struct ClShared {
-    uint64_t bar[2];                   // the cluster barrier, alternating by barrier index
-    uint64_t rbar[2];                  // a round's counts have arrived (by round parity)
-    int part[2][kClCtas][kClNodes];    // every CTA's plane counts per node (pushed here by their
-                                       // owners), by round parity
-    int flags[kClCtas];                // every CTA's invalid-input bits
-    double mx[kClCtas];                // every CTA's max cost at kmin
+    uint64_t rbar[2];                          // a round's predicates have arrived (by round parity)
+    int pw[3][kClNodes];                       // node predicates [round mod 3][heap index]
 };
-
-// barrier i of the cluster: every CTA's thread 0 arrives on every CTA's bar[i & 1] (release),
-// then waits on its own (acquire, bounded); the block barriers order the other threads
-__device__ __forceinline__ bool cluster_sync(ClShared& cs, int i, uint32_t n, WsHeader* hdr, uint32_t where) {
-    __syncthreads();
-    bool ok = true;
-    if (threadIdx.x < n)   // one thread per destination CTA, after the block barrier (cumulative release)
-        mbar_arrive_cluster(mapa_shared(smem_u32(&cs.bar[i & 1]), threadIdx.x));
-    if (threadIdx.x == 0) {
-        const uint32_t parity = (i >> 1) & 1;
-        if (!mbar_try_wait_acq_cluster(&cs.bar[i & 1], parity)) {
-            const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait_acq_cluster(&cs.bar[i & 1], parity)) {
-                if (globaltimer() - t0 > kWaitNs) {
-                    set_error(hdr, DPA_ERR_DEVICE_TIMEOUT, where);
-                    ok = false;
-                    break;
-                }
-            }
-        }
-    }
-    return __syncthreads_and(ok ? 1 : 0) != 0;
-}
 
 __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ ClShared cs;
     __shared__ int s_tmp[32];
     __shared__ int s_scan5[5][32];
-    __shared__ int s_tot[kClNodes];
-    __shared__ double s_wmx[kClThreads / 32];
+    __shared__ double s_wmx[kClWarps];
+    __shared__ int s_part[kClNodesPerCta];   // plane counts of nodes shared by several warps
+    __shared__ int s_nl;       // listed pairs
+    __shared__ int s_fixed;    // planes of the pairs that left the list
+    __shared__ int s_bad;
     const int P = a.T * a.K;
     const int nk = a.kmax - a.kmin + 1;
     const KVals kv = make_kvals(a.kmin);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
-    const int p0 = static_cast<int>((static_cast<long long>(P) * rank) / ncta);
-    const int p1 = static_cast<int>((static_cast<long long>(P) * (rank + 1)) / ncta);
-    const int np = p1 - p0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int rank = static_cast<int>(cluster_ctarank());
     const AllocSmem Ls = alloc_smem_layout(P, a.E, nk, a.vrec != nullptr);
-    double* s_c = reinterpret_cast<double*>(smem + Ls.total);   // this CTA's costs [np][nk]
+    double* s_c = reinterpret_cast<double*>(smem + Ls.total);                    // [P][nk] costs
+    int* s_list = reinterpret_cast<int*>(s_c + static_cast<size_t>(P) * nk);    // [P] listed pairs
+    uint8_t* s_kf = reinterpret_cast<uint8_t*>(s_list + P);                     // [P] final counts
     uint8_t* s_k = smem + Ls.kk;
-    __shared__ int s_myflags;
     if (tid == 0) {
-        mbar_init(&cs.bar[0], ncta);
-        mbar_init(&cs.bar[1], ncta);
         mbar_init(&cs.rbar[0], 1);
         mbar_init(&cs.rbar[1], 1);
-        s_myflags = 0;
+        s_nl = P;
+        s_fixed = 0;
+        s_bad = 0;
         fence_mbarrier_init_cluster();
     }
     for (int i = tid * 16; i < a.E * a.B; i += blockDim.x * 16)
         asm volatile("prefetch.global.L1 [%0];" ::"l"(a.rtable + i));
-    cluster_barrier_once();   // the barriers exist before anyone arrives on them
+    cluster_barrier_once();   // every CTA's barriers exist before anyone stores into it
     pdl_wait();
     pdl_trigger();
-    // ---- inputs: budget, this CTA's pairs (expert ids, widths) and their costs
+    // ---- inputs, checked by every CTA alike (so all take the same exit): budget, expert ids,
+    // stored widths; every pair's costs
     const double target = *a.target;
     int flags = (target >= static_cast<double>(a.kmin) && target <= static_cast<double>(a.kmax)) ? 0 : 1;
     double mx = 0.0;
-    for (int j = tid; j < np; j += blockDim.x) {
-        const int p = p0 + j;
+    for (int p = tid; p < P; p += blockDim.x) {
+        s_list[p] = p;
         const int e = a.idx[p];
         if (e < 0 || e >= a.E) {
             flags |= 2;
@@ -807,7 +800,7 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
             if (i < nk) {
                 const double c = a.kmin + i > wmax ? CUDART_INF
                                                    : __dmul_rn(g, a.rtable[static_cast<size_t>(e) * a.B + (a.kmin + i - 1)]);
-                s_c[j * nk + i] = c;
+                s_c[p * nk + i] = c;
                 if (i == 0) mx = fmax(mx, c);
             }
         }
@@ -817,51 +810,90 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
         flags |= __shfl_xor_sync(0xffffffffu, flags, o);
     }
     if (lane == 0) s_wmx[warp] = mx;
-    if (lane == 0 && flags) atomicOr(&s_myflags, flags);
+    if (lane == 0 && flags) atomicOr(&s_bad, flags);
     __syncthreads();
-    // ---- exchange: this CTA's flags and max pushed into every CTA's slot `rank`
-    if (tid < static_cast<int>(ncta)) {
-        double m = s_wmx[0];
-        for (int w = 1; w < nw; ++w) m = fmax(m, s_wmx[w]);
-        st_cluster_s32(mapa_shared(smem_u32(&cs.flags[rank]), tid), s_myflags);
-        st_cluster_f64(mapa_shared(smem_u32(&cs.mx[rank]), tid), m);
-    }
-    if (!cluster_sync(cs, 0, ncta, a.hdr, 0x250)) return;
-    int all_flags = 0;
-    mx = 0.0;
-    for (uint32_t r = 0; r < ncta; ++r) {
-        all_flags |= cs.flags[r];
-        mx = fmax(mx, cs.mx[r]);
-    }
-    if (all_flags) {
+    if (s_bad) {   // nothing has been stored into another CTA yet
         if (rank == 0 && tid == 0) {
-            set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, (all_flags & 2) ? 11 : ((all_flags & 1) ? 10 : 15));
+            const int f = s_bad;
+            set_error(a.hdr, DPA_ERR_DEVICE_INVALID_INPUT, (f & 2) ? 11 : ((f & 1) ? 10 : 15));
             if (a.do_permute) {
                 a.hdr->n_active = 0;
                 a.hdr->n_gtiles = 0;
                 a.hdr->n_vgroups = 0;
             }
         }
-        cluster_sync(cs, 1, ncta, a.hdr, 0x251);   // nobody reads another CTA's shared memory after this
         return;
     }
+    mx = s_wmx[0];
+    for (int w = 1; w < kClWarps; ++w) mx = fmax(mx, s_wmx[w]);
     const double budget = __dmul_rn(target, static_cast<double>(P));
     const int nb = static_cast<int>(floor(budget));
     double lo = 0.0;
     double hi = __dadd_rn(__dmul_rn(2.0, mx), 1.0);
-    // ---- 64 steps, kClDepth per round
-    constexpr int TPN = kClThreads / kClNodes;   // threads per node
-    const int node_slot = tid / TPN, gsub = tid % TPN;
+
     int round = 0;
     for (int it = 0; it < 64; ++round) {
-        const int D = min(kClDepth, 64 - it);
-        // this round's counts from every CTA: ncta x kClNodes ints, stored into this CTA by
-        // st.async, each completing its bytes on rbar[round & 1]
-        if (tid == 0) mbar_arrive_expect_tx(&cs.rbar[round & 1], ncta * kClNodes * 4u);
-        const int node = node_slot + 1;
-        const bool active = node < (1 << D);
+        const int D = min(round < kClPruneRound ? kClDepthEarly : kClDepth, 64 - it);
+        const int nn = (1 << D) - 1;
+        const int par = round & 1, buf = round % 3;
+        if (round == kClPruneRound) {   // the pairs whose choice no longer changes leave the list
+            double klo[4], khi[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                klo[i] = __dmul_rn(lo, kv.v[i]);
+                khi[i] = __dmul_rn(hi, kv.v[i]);
+            }
+            if (tid == 0) s_nl = 0;
+            __syncthreads();
+            int fixed = 0;
+            for (int b = warp * 32; b < P; b += blockDim.x) {
+                const int p = b + lane;
+                bool keep = false;
+                if (p < P) {
+                    const double* c = s_c + p * nk;
+                    double vlo[4], vhi[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        vlo[i] = i < nk ? __dadd_rn(c[i], klo[i]) : 0.0;
+                        vhi[i] = i < nk ? __dadd_rn(c[i], khi[i]) : 0.0;
+                    }
+                    int ia = 0;
+                    double va = vhi[0];
+#pragma unroll
+                    for (int i = 1; i < 4; ++i)
+                        if (i < nk && vhi[i] < va) { va = vhi[i]; ia = i; }
+                    bool same = true;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (i < nk && i != ia) same = same && (i < ia ? va < vlo[i] : va <= vlo[i]);
+                    if (same) {
+                        fixed += a.kmin + ia;
+                        s_kf[p] = static_cast<uint8_t>(a.kmin + ia);
+                    } else {
+                        keep = true;
+                    }
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, keep);
+                int base = 0;
+                if (lane == 0 && m) base = atomicAdd(&s_nl, __popc(m));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (keep) s_list[base + __popc(m & ((1u << lane) - 1u))] = p;
+            }
+            for (int o = 16; o > 0; o >>= 1) fixed += __shfl_xor_sync(0xffffffffu, fixed, o);
+            if (lane == 0 && fixed) atomicAdd(&s_fixed, fixed);
+            __syncthreads();
+        }
+        if (tid == 0) mbar_arrive_expect_tx(&cs.rbar[par], static_cast<uint32_t>(nn) * 4u);
+        // this CTA's nodes (0-based ids rank, rank + kClCtas, ...), wpn warps each (a power of
+        // two: all warps share the nodes of a small tree); each warp computes its node's midpoint
+        // and counts planes over its share of the listed pairs
+        const int nloc = nn > rank ? (nn - rank + kClCtas - 1) / kClCtas : 0;
+        int wpn = kClWarps;
+        while (wpn > 1 && wpn * nloc > kClWarps) wpn >>= 1;
+        const int j = warp / wpn, sw = warp - j * wpn;
+        const int node = rank + kClCtas * j + 1;   // heap index
         int n = 0;
-        if (active) {
+        if (j < nloc) {
             const int depth = 31 - __clz(node);
             double l = lo, h = hi;
             for (int lev = depth - 1; lev >= 0; --lev) {
@@ -869,21 +901,33 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
                 if ((node >> lev) & 1) l = m; else h = m;
             }
             const double mid = midpoint(l, h);
-            for (int j = gsub; j < np; j += TPN) n += choose_k(s_c + j * nk, nk, a.kmin, kv, mid);
+            const int nl = s_nl, step = 32 * wpn;
+            int n0 = 0, n1 = 0;
+            int q = 32 * sw + lane;
+            for (; q + step < nl; q += 2 * step) {   // two independent pairs per iteration
+                n0 += choose_k(s_c + s_list[q] * nk, nk, a.kmin, kv, mid);
+                n1 += choose_k(s_c + s_list[q + step] * nk, nk, a.kmin, kv, mid);
+            }
+            if (q < nl) n0 += choose_k(s_c + s_list[q] * nk, nk, a.kmin, kv, mid);
+            n = __reduce_add_sync(0xffffffffu, n0 + n1);
         }
-#pragma unroll
-        for (int o = 1; o < TPN; o <<= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-        // push this node's count into every CTA's slot `rank` (the node's threads share the stores)
-        for (int r = gsub; r < static_cast<int>(ncta); r += TPN)
-            st_async_s32(mapa_shared(smem_u32(&cs.part[round & 1][rank][node_slot]), r), n,
-                         mapa_shared(smem_u32(&cs.rbar[round & 1]), r));
-        {   // wait until every CTA's counts of this round are here (bounded)
+        if (wpn > 1) {   // the warps of a node meet in shared memory
+            if (tid < kClNodesPerCta) s_part[tid] = 0;
+            __syncthreads();
+            if (j < nloc && lane == 0) atomicAdd(&s_part[j], n);
+            __syncthreads();
+            n = s_part[j < nloc ? j : 0];
+        }
+        if (j < nloc && sw == 0 && lane < kClCtas)   // the node's predicate, to every CTA
+            st_async_s32(mapa_shared(smem_u32(&cs.pw[buf][node]), static_cast<uint32_t>(lane)), s_fixed + n > nb ? 1 : 0,
+                         mapa_shared(smem_u32(&cs.rbar[par]), static_cast<uint32_t>(lane)));
+        {   // every node's predicate of this round is here (bounded)
             bool ok = true;
             if (tid == 0) {
                 const uint32_t parity = (round >> 1) & 1;
-                if (!mbar_try_wait_acq_cluster(&cs.rbar[round & 1], parity)) {
+                if (!mbar_try_wait_acq_cluster(&cs.rbar[par], parity)) {
                     const uint64_t t0 = globaltimer();
-                    while (!mbar_try_wait_acq_cluster(&cs.rbar[round & 1], parity)) {
+                    while (!mbar_try_wait_acq_cluster(&cs.rbar[par], parity)) {
                         if (globaltimer() - t0 > kWaitNs) {
                             set_error(a.hdr, DPA_ERR_DEVICE_TIMEOUT, 0x252);
                             ok = false;
@@ -894,29 +938,34 @@ __global__ void __launch_bounds__(kClThreads, 1) allocate_cluster_kernel(AllocAr
             }
             if (!__syncthreads_and(ok ? 1 : 0)) return;
         }
-        if (tid < kClNodes) {   // the cluster's count at node tid + 1, from the local slots
-            int t = 0;
-            for (uint32_t r = 0; r < ncta; ++r) t += cs.part[round & 1][r][tid];
-            s_tot[tid] = t;
-        }
-        __syncthreads();
-        int nd = 1;
+        int nd = 1;   // the D steps
         for (int lev = 0; lev < D; ++lev) {
-            const int pr = s_tot[nd - 1] > nb ? 1 : 0;
+            const int pr = cs.pw[buf][nd];
             const double m = midpoint(lo, hi);
-            if (pr) lo = m; else hi = m;
+            lo = pr ? m : lo;
+            hi = pr ? hi : m;
             nd = 2 * nd + pr;
         }
         it += D;
     }
-    // ---- plane counts of this CTA's pairs
-    for (int j = tid; j < np; j += blockDim.x)
-        a.k_out[p0 + j] = static_cast<uint8_t>(choose_k(s_c + j * nk, nk, a.kmin, kv, hi));
-    if (rank == 0 && tid == 0 && a.lambda_out) *a.lambda_out = hi;
-    // every CTA's plane counts are written, and no CTA stores into another's shared memory any more
-    if (!cluster_sync(cs, 1, ncta, a.hdr, 0x253)) return;
-    if (rank != 0 || !a.do_permute) return;
-    for (int p = tid; p < P; p += blockDim.x) s_k[p] = __ldcg(a.k_out + p);
+    // Every CTA has received all the predicates stored into it, and stores nothing more: the
+    // others may exit. CTA 0 writes the plane counts (listed pairs choose at the final hi) and
+    // groups the pairs.
+    if (rank != 0) return;
+    {
+        const int nl = s_nl;
+        for (int q = tid; q < nl; q += blockDim.x) {
+            const int p = s_list[q];
+            s_kf[p] = static_cast<uint8_t>(choose_k(s_c + p * nk, nk, a.kmin, kv, hi));
+        }
+    }
+    __syncthreads();
+    for (int p = tid; p < P; p += blockDim.x) {
+        a.k_out[p] = s_kf[p];
+        s_k[p] = s_kf[p];
+    }
+    if (tid == 0 && a.lambda_out) *a.lambda_out = hi;
+    if (!a.do_permute) return;
     __syncthreads();
     group_pairs(a, smem, Ls, P, nk, s_k, s_tmp, s_scan5);
 }
@@ -1116,8 +1165,9 @@ cudaError_t launch_allocate(const AllocArgs& a, cudaStream_t stream, CoopSync* c
     }
     if (!coop_ran && a.policy == DPA_ALLOC_LAGRANGE && P >= kClMinPairs && P <= kSpecMaxP) {
         // mid-size batches: the bisection over a cluster of SMs, then CTA 0 groups the pairs
-        const size_t smem = allocate_smem_bytes(P, a.E, nk, a.vrec != nullptr) +
-                            static_cast<size_t>(P / kClCtas + 1) * nk * 8;
+        // the grouping's layout, then every pair's costs, the pair list and the final counts
+        const size_t smem = allocate_smem_bytes(P, a.E, nk, a.vrec != nullptr) + static_cast<size_t>(P) * nk * 8 +
+                            static_cast<size_t>(P) * 5;
         cudaError_t err = cudaFuncSetAttribute(allocate_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(smem));
         if (err != cudaSuccess) return err;
