@@ -258,6 +258,110 @@ __device__ void token_digits(const RouteArgs& a, int t, const uint16_t* xs, int 
     }
 }
 
+// ---- top-k by warp extraction (E <= 32 w experts on the first w warps, w K <= 32) ----
+// A logit as an order-preserving 64-bit key: larger logit, larger key; -0 ties with +0; NaN is
+// below every number.
+__device__ __forceinline__ unsigned long long logit_key(double v) {
+    if (v != v) return 0ull;
+    const unsigned long long b = v == 0.0 ? 0ull : static_cast<unsigned long long>(__double_as_longlong(v));
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+// The K largest keys among the lanes with `avail`, largest first, equal keys by lowest lane:
+// lane r < K receives the r-th key and the lane that held it (ok false: none was left).
+__device__ __forceinline__ void warp_extract(unsigned long long key, bool avail, int K, int lane,
+                                             unsigned long long& out_key, int& out_lane, bool& out_ok) {
+    out_key = 0ull;
+    out_lane = 0;
+    out_ok = false;
+    for (int r = 0; r < K; ++r) {
+        const uint32_t hi = avail ? static_cast<uint32_t>(key >> 32) : 0u;
+        const uint32_t mh = __reduce_max_sync(0xffffffffu, hi);
+        const bool c1 = avail && hi == mh;
+        const uint32_t lo = c1 ? static_cast<uint32_t>(key) : 0u;
+        const uint32_t ml = __reduce_max_sync(0xffffffffu, lo);
+        const unsigned c2 = __ballot_sync(0xffffffffu, c1 && static_cast<uint32_t>(key) == ml);
+        const int win = __ffs(static_cast<int>(c2)) - 1;
+        if (lane == r) {
+            out_ok = win >= 0;
+            out_lane = win >= 0 ? win : 0;
+            out_key = (static_cast<unsigned long long>(mh) << 32) | ml;
+        }
+        if (lane == win) avail = false;
+    }
+}
+// Each of the first w warps extracts the K largest of its 32 experts; warp 0 extracts the K
+// largest of those w K candidates (laid out by warp, then in extraction order, so equal keys
+// stay in ascending expert id), then computes the gates with shuffles. The same order and the
+// same arithmetic as the rank-based path below. Returns false (before any work) where the
+// shape does not fit; the decision is uniform over the block.
+__device__ bool select_topk_gates_warp(const RouteArgs& a, int t, const double* lrow, unsigned char* smem_raw) {
+    __shared__ unsigned long long s_ck[32];
+    __shared__ double s_cv[32];
+    __shared__ int s_ce[32], s_cok[32];
+    __shared__ double s_lmax, s_den;
+    const int E = a.E, K = a.K;
+    const int nwu = (E + 31) >> 5;
+    if (K > 32 || nwu * K > 32 || nwu * 32 > static_cast<int>(blockDim.x)) return false;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    double v = 0.0;
+    if (warp < nwu) {
+        const int e = warp * 32 + lane;
+        const bool valid = e < E;
+        v = valid ? __ldcg(lrow + e) : 0.0;
+        unsigned long long ck;
+        int cl;
+        bool ok;
+        warp_extract(valid ? logit_key(v) : 0ull, valid, K, lane, ck, cl, ok);
+        const double cv = __shfl_sync(0xffffffffu, v, cl);
+        if (lane < K) {
+            s_ck[warp * K + lane] = ck;
+            s_cv[warp * K + lane] = cv;
+            s_ce[warp * K + lane] = warp * 32 + cl;
+            s_cok[warp * K + lane] = ok ? 1 : 0;
+        }
+    }
+    __syncthreads();
+    double num = 0.0, vs = 0.0;
+    int es = 0;
+    if (warp == 0) {
+        const bool have = lane < nwu * K && s_cok[lane] != 0;
+        unsigned long long fk;
+        int fl;
+        bool ok;
+        warp_extract(have ? s_ck[lane] : 0ull, have, K, lane, fk, fl, ok);
+        es = s_ce[fl];
+        vs = s_cv[fl];
+        const double lmax = __shfl_sync(0xffffffffu, vs, 0);
+        if (lane < K) num = dexp_fixed(__dsub_rn(vs, lmax));
+        if (lane == 0) s_lmax = lmax;
+    }
+    if (!a.norm_topk) {   // the denominator sums every expert's exp, in expert order
+        double* ex = reinterpret_cast<double*>(smem_raw);   // [E]
+        __syncthreads();
+        if (warp < nwu && warp * 32 + lane < E) ex[warp * 32 + lane] = dexp_fixed(__dsub_rn(v, s_lmax));
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double den = 0.0;
+            for (int i = 0; i < E; ++i) den = __dadd_rn(den, ex[i]);
+            s_den = den;
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+        double den = 0.0;
+        if (a.norm_topk) {
+            for (int j = 0; j < K; ++j) den = __dadd_rn(den, __shfl_sync(0xffffffffu, num, j));
+        } else {
+            den = s_den;
+        }
+        if (lane < K) {
+            a.idx[t * K + lane] = es;
+            a.gate[t * K + lane] = __ddiv_rn(num, den);
+        }
+    }
+    return true;
+}
+
 // Top-k by exact fp64 logit (descending, ties to the lower expert id, NaN last) and the gates
 // (fixed fp64 exp; softmax over the top-k or over all experts). Whole block; smem_raw holds at
 // least 24 * E bytes.
@@ -268,6 +372,7 @@ __device__ void select_topk_gates(const RouteArgs& a, int t, unsigned char* smem
     const int E = a.E;
     // the logits were written by other blocks or kernels (fenced / completed); read them from L2
     const double* lrow = (a.logits_user ? a.logits_user : a.logits_ws) + static_cast<size_t>(t) * E;
+    if (select_topk_gates_warp(a, t, lrow, smem_raw)) return;
     double* vals = reinterpret_cast<double*>(smem_raw);             // [E] logits (token no longer needed)
     float* fk = reinterpret_cast<float*>(vals + E);                 // [E] fp32 roundings of the logits
     for (int i = threadIdx.x; i < E; i += blockDim.x) {
@@ -757,18 +862,18 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
     const double nx = a.n2_x[t];
     const int kslice = H / a.ks;   // inputs per slice of the tiled logits
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        // the logit: the tiled kernel's slice sums, added in slice order (eight independent loads
-        // in flight per step), with their lowest set bit and the sum of their magnitudes
+        // the logit: the tiled kernel's slice sums, added in slice order (up to 32 independent
+        // loads in flight), with their lowest set bit and the sum of their magnitudes
         const double* pe = a.part + static_cast<size_t>(t) * E + e;
         const size_t qs = static_cast<size_t>(a.T) * E;
         double v = 0.0, av = 0.0;
         int mv = 1 << 20;
-        for (int q0 = 0; q0 < a.ks; q0 += 8) {
-            double u[8];
+        for (int q0 = 0; q0 < a.ks; q0 += 32) {
+            double u[32];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) u[j] = q0 + j < a.ks ? __ldcg(pe + (q0 + j) * qs) : 0.0;
+            for (int j = 0; j < 32; ++j) u[j] = q0 + j < a.ks ? __ldcg(pe + (q0 + j) * qs) : 0.0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 v = __dadd_rn(v, u[j]);
                 av = __dadd_rn(av, fabs(u[j]));
                 mv = min(mv, f64_lsb(u[j]));
