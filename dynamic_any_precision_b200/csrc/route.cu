@@ -842,9 +842,13 @@ __global__ void __launch_bounds__(kGThreads) route_prep_kernel(RouteArgs a, int 
     }
 }
 
-// One CTA (4 warps) per token: check each logit's exactness bound, recompute the failures with
+// One CTA per token (16 warps for small batches, so that a token's recomputed logits run at
+// once; 4 for large ones, so that several tokens share an SM): check each logit's exactness
+// bound, recompute the failures with
 // the exact dot product, then top-k and gates.
-__global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
+constexpr int kSelWarpsMax = 16;
+constexpr int kSelSmallBatch = 256;   // up to this many tokens: kSelWarpsMax warps per token
+__global__ void __launch_bounds__(kSelWarpsMax * 32) route_select_kernel(RouteArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ int s_fail[256];
     __shared__ int s_nfail;
@@ -938,7 +942,7 @@ __global__ void __launch_bounds__(128) route_select_kernel(RouteArgs a) {
     if (nfail > 0) {
         // more failures than the list holds: recompute every logit of the token
         const int n = nfail <= 256 ? nfail : E;
-        for (int i = warp; i < n; i += 4) {
+        for (int i = warp; i < n; i += static_cast<int>(blockDim.x >> 5)) {
             const int e = nfail <= 256 ? s_fail[i] : i;
             const double v = exact_dot_warp(xrow, a.wr + static_cast<size_t>(e) * H, H, lane);
             if (lane == 0) dst[e] = v;
@@ -1006,7 +1010,7 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t stream, int sms) {
             if (err != cudaSuccess) return err;
         }
         void* args[] = {&b};
-        return launch_pdl_raw(reinterpret_cast<const void*>(route_select_kernel), dim3(a.T), dim3(128), ssm, stream,
+        return launch_pdl_raw(reinterpret_cast<const void*>(route_select_kernel), dim3(a.T), dim3(a.T <= kSelSmallBatch ? kSelWarpsMax * 32 : 128), ssm, stream,
                               args);
     }
     // few tokens: split each expert's dot product over 4 warps to shorten the serial chain
