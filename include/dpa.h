@@ -385,7 +385,7 @@ dpa_status dpa_stream_prefixes(const dpa_layer_desc* desc, const void* host_plan
                                const int32_t* experts, const uint8_t* kplanes, int n, void* dev_planes,
                                void* dev_meta, uint64_t* bytes_out, void* stream);
 
-/* ---- Per-expert stored widths (SURVEY row f2) ----
+/* ---- Per-expert stored widths ----
  * MatMoE, review "Core Contribution": offline, an ILP picks each expert's maximum bit-width
  * (2/3/4) under a memory budget, with the metric routing score x Fisher-approximated Hessian
  * x quantization error. Here the ILP is
