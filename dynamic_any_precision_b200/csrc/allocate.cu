@@ -724,7 +724,10 @@ grouping:
 constexpr int kClCtas = DPA_ALLOC_CLUSTER;      // CTAs of the cluster (16: a non-portable cluster size)
 constexpr int kClThreads = 512;
 constexpr int kClWarps = kClThreads / 32;
-constexpr int kClDepthEarly = 6;                // steps of the rounds before the pruning (every pair listed)
+#ifndef DPA_ALLOC_CL_DEPTH_EARLY
+#define DPA_ALLOC_CL_DEPTH_EARLY 6
+#endif
+constexpr int kClDepthEarly = DPA_ALLOC_CL_DEPTH_EARLY;   // steps of the rounds before the pruning (every pair listed)
 constexpr int kClDepth = 8;                     // steps of the later rounds
 constexpr int kClPruneRound = 2;
 constexpr int kClNodes = 1 << kClDepth;

@@ -60,13 +60,18 @@ constexpr int kMaxB = 4;
 constexpr int kMaxChunk = DPA_VP_CHUNK;       // columns per chunk
 // Row tiles (16 rows each) per item: the larger where the ring and group slots fit in shared
 // memory, else the smaller (wide matrices, whose scale data and digit rows take more room).
-#ifndef DPA_VP_GU_NRT
-#define DPA_VP_GU_NRT 2
+#ifndef DPA_VP_GU_NRT_UNIFORM
+#define DPA_VP_GU_NRT_UNIFORM 4
+#endif
+#ifndef DPA_VP_GU_NRT_BCQ
+#define DPA_VP_GU_NRT_BCQ 2
 #endif
 #ifndef DPA_VP_DN_NRT
 #define DPA_VP_DN_NRT 4
 #endif
-constexpr int kGuNRT = DPA_VP_GU_NRT, kGuNRTSmall = 1;   // gate/up: 32 (16) rows, 4 (8) column slices
+// gate/up: 64 rows (uniform codes, 3 column slices of the 12 consumer warps) or 32 rows
+// (binary-coded planes, 4 slices of 8), else 16 rows
+constexpr int kGuNRTUniform = DPA_VP_GU_NRT_UNIFORM, kGuNRTBcq = DPA_VP_GU_NRT_BCQ, kGuNRTSmall = 1;
 constexpr int kDnNRT = DPA_VP_DN_NRT, kDnNRTSmall = 2;   // down: 64 (32) rows, 2 (4) column slices
 constexpr int kDigPad = 64;                   // bytes of padding per staged digit row (banks)
 
@@ -774,11 +779,23 @@ cudaError_t launch_variant(const VpArgs& a, cudaStream_t stream, int sms) {
 // Variants: gate/up (two matrices) and down (one matrix); items of the larger row block where
 // shared memory allows; token groups of two tiles (8 tokens), or one tile (4 tokens) where no
 // row block fits with two.
+// row tiles per item: the larger (big) where shared memory allows, else the smaller
+template <int FMT, int NMAT>
+struct VpNrt {
+    static constexpr int big = NMAT == 2 ? (FMT == DPA_FMT_UNIFORM ? kGuNRTUniform : kGuNRTBcq) : kDnNRT;
+    static constexpr int small = NMAT == 2 ? kGuNRTSmall : kDnNRTSmall;
+};
+
+template <int FMT, int NMAT>
+static size_t vp_bytes_f(bool big, int tpg, int K, int G, int B) {
+    constexpr int NB = VpNrt<FMT, NMAT>::big, NS = VpNrt<FMT, NMAT>::small;
+    if (big) return tpg == 2 ? vlayout<NB, 2, NMAT>(K, G, FMT, B).total : vlayout<NB, 1, NMAT>(K, G, FMT, B).total;
+    return tpg == 2 ? vlayout<NS, 2, NMAT>(K, G, FMT, B).total : vlayout<NS, 1, NMAT>(K, G, FMT, B).total;
+}
 template <int NMAT>
 static size_t vp_bytes(bool big, int tpg, int K, int G, int fmt, int B) {
-    constexpr int NB = NMAT == 2 ? kGuNRT : kDnNRT, NS = NMAT == 2 ? kGuNRTSmall : kDnNRTSmall;
-    if (big) return tpg == 2 ? vlayout<NB, 2, NMAT>(K, G, fmt, B).total : vlayout<NB, 1, NMAT>(K, G, fmt, B).total;
-    return tpg == 2 ? vlayout<NS, 2, NMAT>(K, G, fmt, B).total : vlayout<NS, 1, NMAT>(K, G, fmt, B).total;
+    return fmt == DPA_FMT_UNIFORM ? vp_bytes_f<DPA_FMT_UNIFORM, NMAT>(big, tpg, K, G, B)
+                                  : vp_bytes_f<DPA_FMT_BCQ, NMAT>(big, tpg, K, G, B);
 }
 
 int vp_tiles_per_group(int K_gateup, int K_down, int G, int fmt, int B) {
@@ -795,7 +812,7 @@ size_t vp_smem_bytes(int K, int G, int fmt, int B, int nmat, int tiles_per_group
 
 template <int FMT, int NMAT>
 static cudaError_t launch_kind(const VpArgs& a, cudaStream_t stream, int sms) {
-    constexpr int NB = NMAT == 2 ? kGuNRT : kDnNRT, NS = NMAT == 2 ? kGuNRTSmall : kDnNRTSmall;
+    constexpr int NB = VpNrt<FMT, NMAT>::big, NS = VpNrt<FMT, NMAT>::small;
     const bool two = a.tiles_per_group == 2;
     const bool big = a.R % (16 * NB) == 0 && vp_bytes<NMAT>(true, two ? 2 : 1, a.K, a.G, FMT, a.B) <= kVpMaxSmem;
     if (big) return two ? launch_variant<FMT, NB, 2, NMAT>(a, stream, sms) : launch_variant<FMT, NB, 1, NMAT>(a, stream, sms);
@@ -804,15 +821,18 @@ static cudaError_t launch_kind(const VpArgs& a, cudaStream_t stream, int sms) {
 
 template <int FMT, int NMAT>
 static bool vp_big(const VpArgs& a) {
-    constexpr int NB = NMAT == 2 ? kGuNRT : kDnNRT;
+    constexpr int NB = VpNrt<FMT, NMAT>::big;
     return a.R % (16 * NB) == 0 && vp_bytes<NMAT>(true, a.tiles_per_group == 2 ? 2 : 1, a.K, a.G, FMT, a.B) <= kVpMaxSmem;
 }
 
 int vp_rows_per_item(const VpArgs& a) {
-    bool big;
-    if (a.nmat == 2) big = a.fmt == DPA_FMT_UNIFORM ? vp_big<DPA_FMT_UNIFORM, 2>(a) : vp_big<DPA_FMT_BCQ, 2>(a);
-    else big = a.fmt == DPA_FMT_UNIFORM ? vp_big<DPA_FMT_UNIFORM, 1>(a) : vp_big<DPA_FMT_BCQ, 1>(a);
-    return 16 * (a.nmat == 2 ? (big ? kGuNRT : kGuNRTSmall) : (big ? kDnNRT : kDnNRTSmall));
+    const bool uni = a.fmt == DPA_FMT_UNIFORM;
+    if (a.nmat == 2) {
+        const bool big = uni ? vp_big<DPA_FMT_UNIFORM, 2>(a) : vp_big<DPA_FMT_BCQ, 2>(a);
+        return 16 * (big ? (uni ? kGuNRTUniform : kGuNRTBcq) : kGuNRTSmall);
+    }
+    const bool big = uni ? vp_big<DPA_FMT_UNIFORM, 1>(a) : vp_big<DPA_FMT_BCQ, 1>(a);
+    return 16 * (big ? kDnNRT : kDnNRTSmall);
 }
 
 int vp_grid(const VpArgs& a, int sms) {
