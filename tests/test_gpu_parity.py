@@ -176,6 +176,31 @@ def test_route_tiled_slice_bounds(case):
     assert np.array_equal(idx.cpu().numpy(), ridx) and np.array_equal(gate.cpu().numpy(), rg)
 
 
+@pytest.mark.parametrize("E,K,T", [(64, 6, 1), (64, 6, 64), (256, 8, 1), (256, 8, 64)])
+def test_route_ties_and_expert_counts(E, K, T):
+    # Routers with repeated rows (equal logits: ties go to the lower expert id) at 64 experts,
+    # where the top-k runs as warp extraction, and at 256 experts, where it runs as ranks (the
+    # extraction covers at most 32 candidates); one token (per-logit kernel) and 64 (tiled).
+    shape = W.with_sizes(W.QWEN3_B1, n_experts=E, top_k=K, name=f"route_e{E}")
+    d = dpa.make_desc(shape)
+    rng = np.random.default_rng(E * 100 + T)
+    w = (rng.standard_normal((E, shape.hidden)) * 0.02).astype(np.float32)
+    for dst in range(1, E, 3):   # every third row repeats an earlier one
+        w[dst] = w[int(rng.integers(0, dst))]
+    wb = W.f32_to_bf16_bits(w)
+    xb = W.tokens(shape, T, step=21)
+    ws = dpa.new_workspace(d, T)
+    logits = torch.empty((T, E), dtype=torch.float64, device="cuda")
+    idx, gate = dpa.route(d, torch.from_numpy(xb.view(np.int16)).cuda(), torch.from_numpy(wb.view(np.int16)).cuda(),
+                          ws, logits=logits)
+    assert dpa.device_status(ws) == 0
+    ridx, rg, rl = O.route(xb, wb, K, shape.norm_topk)
+    assert np.array_equal(logits.cpu().numpy(), rl)
+    assert np.array_equal(idx.cpu().numpy(), ridx) and np.array_equal(gate.cpu().numpy(), rg)
+    # the repeated rows do produce equal logits among the selected experts' rivals
+    assert any(len(np.unique(rl[t])) < E for t in range(T))
+
+
 # ----------------------------------------------------------------------------- allocation
 
 def _alloc_inputs(seed, T, K, E, B, ties=False):
