@@ -169,7 +169,7 @@ def build_layer(shape, seed=None):
 # kernel, from one ncu capture of the current kernel code (the capture commands and figures are
 # kept with the profile summaries). Workloads without such a capture report null.
 NCU_TRAFFIC_BYTES = {
-    ("qwen3_30b_a3b_moe_decode_b64", 3.0): 173_064_192,         # vp_gemv_kernel<0,2,2,2> (gate/up)
+    ("qwen3_30b_a3b_moe_decode_b64", 3.0): 172_652_288,         # vp_gemv_kernel<0,4,2,2> (gate/up)
     ("qwen3_30b_a3b_moe_prefill_t2048", 4.0): 301_577_728,      # gemm_tc_kernel<0,4> (gate/up)
 }
 

@@ -325,7 +325,7 @@ dpa_status dpa_calibrate_threshold(const dpa_layer_desc* desc, const double* sco
  * which every GPU that loads the library holds until the process exits.
  * Limits: n_tokens <= 1024 and n_tokens * n_experts <= 65536, else DPA_ERR_UNSUPPORTED
  * (nothing launched). Every batch runs the router's per-logit kernel (dpa_route switches to
- * its tiled kernels from 128 tokens; the decisions are the same). The first call on a device
+ * its tiled kernels from 2 tokens; the decisions are the same). The first call on a device
  * looks up the array's device address, so make it before any stream capture; the address is
  * kept for the life of the process, so resetting the device (cudaDeviceReset) after that first
  * call is not supported. Every call shares the array: calls whose executions
