@@ -609,7 +609,7 @@ def main(argv=None):
         secs = res["ms"] * 1e-3
         tokens = world * shape.tokens * args.steps
         config.update({"layers": res["n_layers"], "prefill_tokens": W.STACK_PREFILL_TOKENS,
-                       "targets_cycled": list(shape.targets),
+                       "target_bpw": "cycled", "targets_cycled": list(shape.targets),
                        "l2": "48 resident layers (~15 GB) per step, far larger than L2"})
         line = {"metric": metric, "value": tokens / secs, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps,
