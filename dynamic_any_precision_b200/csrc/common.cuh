@@ -180,32 +180,11 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
     return r;
 }
-__device__ __forceinline__ uint32_t cluster_nctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-    return r;
-}
 // address of the same shared-memory object in CTA `rank` of the cluster
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
     return r;
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
-    int v;
-    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ double ld_cluster_f64(uint32_t cluster_addr) {
-    double v;
-    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(cluster_addr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int v) {
-    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster_f64(uint32_t cluster_addr, double v) {
-    asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(cluster_addr), "d"(v) : "memory");
 }
 // asynchronous remote store of 4 bytes into CTA shared memory of the cluster that completes 4
 // bytes of transaction count on that CTA's mbarrier (both shared::cluster addresses)
@@ -213,10 +192,6 @@ __device__ __forceinline__ void st_async_s32(uint32_t cluster_addr, int v, uint3
     asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
                  "r"(v), "r"(cluster_bar)
                  : "memory");
-}
-// arrive (release at cluster scope) on an mbarrier of any CTA of the cluster
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
