@@ -20,8 +20,9 @@
 //
 // Where the steps run: up to 64 pairs one CTA, speculating (a replay against the summed hull
 // breakpoints, checked exactly, trees from the first disagreement); 65 to 2048 pairs a cluster of
-// 8 CTAs exchanging each tree's counts through distributed shared memory; beyond, every SM
-// (cooperative launch, grid barrier per tree).
+// 16 CTAs that split each tree's nodes and exchange the nodes' predicates through distributed
+// shared memory, evaluating after one pruning pass only the pairs whose choice can still change;
+// beyond, every SM (cooperative launch, grid barrier per tree).
 //
 // Then pairs are grouped by key (expert, k) with a counting sort; per expert the prefill GEMM's
 // token tiles and the expert GEMV's token-group records, and for the two GEMV launches the
