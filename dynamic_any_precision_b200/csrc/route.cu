@@ -865,50 +865,72 @@ __global__ void __launch_bounds__(kSelWarpsMax * 32) route_select_kernel(RouteAr
     __syncthreads();
     const double nx = a.n2_x[t];
     const int kslice = H / a.ks;   // inputs per slice of the tiled logits
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        // the logit: the tiled kernel's slice sums, added in slice order (up to 32 independent
-        // loads in flight), with their lowest set bit and the sum of their magnitudes
-        const double* pe = a.part + static_cast<size_t>(t) * E + e;
-        const size_t qs = static_cast<size_t>(a.T) * E;
-        double v = 0.0, av = 0.0;
-        int mv = 1 << 20;
-        for (int q0 = 0; q0 < a.ks; q0 += 32) {
-            double u[32];
+    // tpe threads per expert (a power of two up to 4, neighbours in one warp): each takes the
+    // slices sl = sub, sub + tpe, ... with the blocks they cover. Both exactness tests hold for
+    // any order of the additions, so the partial sums may be combined in any order; a logit that
+    // passes neither test is recomputed below.
+    int tpe = 1;
+    while (tpe < 4 && tpe * 2 * E <= static_cast<int>(blockDim.x)) tpe *= 2;
+    const int sub = threadIdx.x & (tpe - 1);
+    const size_t qs = static_cast<size_t>(a.T) * E;
+    for (int g0 = 0; g0 < E * tpe; g0 += blockDim.x) {   // warp-uniform trip count
+        const int e = (g0 + static_cast<int>(threadIdx.x)) / tpe;
+        const bool act = e < E;
+        const int16_t* lw = a.lsb_w + static_cast<size_t>(act ? e : 0) * nb;
+        const int16_t* hw = a.hb_w + static_cast<size_t>(act ? e : 0) * nb;
+        double v = 0.0, av = 0.0;   // this thread's slices: sum, sum of magnitudes
+        int mv = 1 << 20;           //   lowest set bit over the nonzero slice sums
+        int L = 2 * kNoLsb;         //   lowest product bit over their blocks (whole-row test)
+        if (act) {
+            const double* pe = a.part + static_cast<size_t>(t) * E + e;
+            for (int q0 = sub; q0 < a.ks; q0 += 32 * tpe) {
+                double u[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = q0 + j < a.ks ? __ldcg(pe + (q0 + j) * qs) : 0.0;
+                for (int j = 0; j < 32; ++j) u[j] = q0 + j * tpe < a.ks ? __ldcg(pe + (q0 + j * tpe) * qs) : 0.0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                v = __dadd_rn(v, u[j]);
-                av = __dadd_rn(av, fabs(u[j]));
-                mv = min(mv, f64_lsb(u[j]));
+                for (int j = 0; j < 32; ++j) {
+                    v = __dadd_rn(v, u[j]);
+                    av = __dadd_rn(av, fabs(u[j]));
+                    mv = min(mv, f64_lsb(u[j]));
+                }
             }
-        }
-        dst[e] = v;
-        const int16_t* lw = a.lsb_w + static_cast<size_t>(e) * nb;
-        const int16_t* hw = a.hb_w + static_cast<size_t>(e) * nb;
-        // whole-row test: L over all blocks with nonzero products
-        int L = 2 * kNoLsb;
+            if (tpe == 1) {   // every block, eight at a time (nb is a multiple of 8: H % 512 == 0)
 #pragma unroll 4
-        for (int b0 = 0; b0 < nb; b0 += 8) {   // nb is a multiple of 8 (H % 512 == 0 on this path)
-            const uint4 v = *reinterpret_cast<const uint4*>(lw + b0);
-            const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+                for (int b0 = 0; b0 < nb; b0 += 8) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(lw + b0);
+                    const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-            for (int h = 0; h < 8; ++h) {
-                const int lv = static_cast<int16_t>((ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu);
-                L = min(L, static_cast<int>(s_lx[b0 + h]) + lv);
+                    for (int h = 0; h < 8; ++h) {
+                        const int lv = static_cast<int16_t>((ww[h >> 1] >> (16 * (h & 1))) & 0xFFFFu);
+                        L = min(L, static_cast<int>(s_lx[b0 + h]) + lv);
+                    }
+                }
+            } else {          // the blocks of this thread's slices
+                for (int sl = sub; sl < a.ks; sl += tpe) {
+                    const int b0 = (sl * kslice) / kLsbBlock, b1 = ((sl + 1) * kslice - 1) / kLsbBlock;
+                    for (int b = b0; b <= b1; ++b) L = min(L, static_cast<int>(s_lx[b]) + static_cast<int>(lw[b]));
+                }
             }
         }
+        for (int o = 1; o < tpe; o <<= 1) {   // the expert's threads meet (every lane takes part)
+            v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+            av = __dadd_rn(av, __shfl_xor_sync(0xffffffffu, av, o));
+            mv = min(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+            L = min(L, __shfl_xor_sync(0xffffffffu, L, o));
+        }
+        // whole-row test (the same verdict in every thread of the expert): every product a
+        // multiple of 2^L, every partial sum below |x| |w|
         bool ok = true;
-        if (L < kNoLsb) {   // some block has nonzero products (else the logit is exactly 0)
+        if (act && L < kNoLsb) {   // some block has nonzero products (else the logit is exactly 0)
             const int L2 = 2 * (L + 53);
             // margin 2^-20 covers the rounding of the two fp64 sums of squares
             const double lhs = __dmul_rn(__dmul_rn(nx, a.n2_w[e]), 1.0 + 0x1p-20);
             ok = L2 >= 1024 || (L2 > -1022 && lhs < pow2(L2));
         }
-        if (!ok) {
-            // per-slice test, then the sum over the slices
-            bool oks = true;
-            for (int sl = 0; sl < a.ks && oks; ++sl) {
+        // else each slice exact on its own (this thread's slices), then the sum over the slices
+        bool oks = true;
+        if (act && !ok) {
+            for (int sl = sub; sl < a.ks && oks; sl += tpe) {
                 const int b0 = (sl * kslice) / kLsbBlock, b1 = ((sl + 1) * kslice - 1) / kLsbBlock;
                 int Ls = kNoLsb, Hs = -kNoLsb;
                 for (int b = b0; b <= b1; ++b) {
@@ -922,18 +944,25 @@ __global__ void __launch_bounds__(kSelWarpsMax * 32) route_select_kernel(RouteAr
                 const int cl = nbt > 1 ? 32 - __clz(nbt - 1) : 0;   // ceil(log2 nbt)
                 oks = Ls >= kNoLsb || Hs + cl <= Ls + 53;
             }
-            if (oks && av > 0.0) {
-                // partial sums of the slice sums: multiples of 2^mv, at most av (summed with at
-                // most 255 roundings; 2^-40 bounds them)
-                int ea;
-                frexp(__dmul_rn(av, 1.0 + 0x1p-40), &ea);
-                oks = ea <= mv + 53;
-            }
-            ok = oks;
         }
-        if (!ok) {
-            const int slot = atomicAdd(&s_nfail, 1);
-            if (slot < 256) s_fail[slot] = e;
+        for (int o = 1; o < tpe; o <<= 1) oks = (__shfl_xor_sync(0xffffffffu, oks ? 1 : 0, o) != 0) && oks;
+        if (act && sub == 0) {
+            dst[e] = v;
+            if (!ok && oks) {
+                if (av > 0.0) {
+                    // the partial sums of the slice sums are multiples of 2^mv and at most av
+                    // (summed with at most 255 roundings; 2^-40 bounds them)
+                    int ea;
+                    frexp(__dmul_rn(av, 1.0 + 0x1p-40), &ea);
+                    ok = ea <= mv + 53;
+                } else {
+                    ok = true;   // every slice sum is zero: the logit is exactly 0
+                }
+            }
+            if (!ok) {
+                const int slot = atomicAdd(&s_nfail, 1);
+                if (slot < 256) s_fail[slot] = e;
+            }
         }
     }
     __syncthreads();
